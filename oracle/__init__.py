@@ -1,0 +1,117 @@
+"""fp64 CPU oracle for paged decode attention and the paged KV-cache write.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package.  It shares no code with
+the CUDA library (``paged_kv_cache_459_b200``) and never imports it; the only
+common module is the seeded input generator, which holds no attention
+arithmetic.
+
+* ``paged_decode``          -- softmax(scale * q K^T) V per (sequence, query head),
+                               K and V gathered through the block table (C, fp64).
+* ``paged_decode_partitioned`` -- the same in independent token partitions
+                               combined by log-sum-exp (C, fp64).
+* ``kv_write``              -- the new token's K/V copied into its slot (C).
+* ``alloc_model.BlockManager`` -- the block allocator's reference model (Python).
+
+Pins (all CPU tests): the pages' worked block-table, waste and sharing
+examples; closed forms (len 1, equal keys, two keys, one dominant key); brute
+force against torch's fp64 scaled_dot_product_attention on un-paged K/V;
+invariance under physical-block relabelling; the partition identity.
+No function here is left unpinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        l = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        l.oracle_kv_write.argtypes = [P, P, P, P, P, i64, i32, i32, i64]
+        l.oracle_kv_write.restype = i32
+        l.oracle_paged_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i64, f64, i32]
+        l.oracle_paged_decode.restype = i32
+        l.oracle_paged_decode_partitioned.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32,
+                                                      i64, f64, i32]
+        l.oracle_paged_decode_partitioned.restype = i32
+        l.oracle_block_tokens.restype = i32
+        _lib = l
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, "bf16 inputs are passed as uint16 bit patterns"
+    return a
+
+
+def block_tokens() -> int:
+    return int(lib().oracle_block_tokens())
+
+
+def kv_write(k_cache, v_cache, k, v, slot_mapping):
+    """Return copies of the caches after writing k/v [T, Hkv, d] at the slots."""
+    kc, vc = np.array(_u16(k_cache), copy=True), np.array(_u16(v_cache), copy=True)
+    k, v = _u16(k), _u16(v)
+    slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    nb, hkv, bt, d = kc.shape
+    assert bt == block_tokens() and k.shape == (len(slots), hkv, d) and v.shape == k.shape
+    valid = slots[slots >= 0]
+    if len(np.unique(valid)) != len(valid):
+        raise ValueError("duplicate slots in one write")
+    rc = lib().oracle_kv_write(_ptr(kc), _ptr(vc), _ptr(k), _ptr(v), _ptr(slots), len(slots),
+                               hkv, d, nb)
+    if rc:
+        raise ValueError("slot outside the pool")
+    return kc, vc
+
+
+def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, nthreads: int = 0):
+    """fp64 attention output [B, Hq, d]."""
+    q, kc, vc = _u16(q), _u16(k_cache), _u16(v_cache)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    b, hq, d = q.shape
+    nb, hkv = kc.shape[0], kc.shape[1]
+    out = np.zeros((b, hq, d), dtype=np.float64)
+    rc = lib().oracle_paged_decode(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(tables),
+                                   tables.shape[1], _ptr(lens), b, hq, hkv, d, nb, float(scale),
+                                   int(nthreads))
+    if rc:
+        raise ValueError(f"oracle_paged_decode failed ({rc})")
+    return out
+
+
+def paged_decode_partitioned(q, k_cache, v_cache, block_tables, seq_lens, scale, partition_tokens):
+    q, kc, vc = _u16(q), _u16(k_cache), _u16(v_cache)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    b, hq, d = q.shape
+    nb, hkv = kc.shape[0], kc.shape[1]
+    out = np.zeros((b, hq, d), dtype=np.float64)
+    rc = lib().oracle_paged_decode_partitioned(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc),
+                                               _ptr(tables), tables.shape[1], _ptr(lens), b, hq,
+                                               hkv, d, nb, float(scale), int(partition_tokens))
+    if rc:
+        raise ValueError(f"oracle_paged_decode_partitioned failed ({rc})")
+    return out
+
+
+def threads_available() -> int:
+    return len(os.sched_getaffinity(0))

@@ -1,0 +1,140 @@
+"""Reference model of the paged KV block manager -- TEST INFRASTRUCTURE.
+
+A plain dictionary model of the lifecycle on "vLLM 與 PagedAttention：高吞吐推理
+的關鍵", section 三 (運作流程): a new request gets an empty block table and no
+blocks up front (step 一); prefill writes its tokens block by block and takes
+a new block each time one fills (step 二); each decoded token goes into the
+current block, or into a new block when the current one is full (step 三);
+when the request ends all of its blocks go back to the pool for any other
+request (step 四).  Section 二 fixes the block size (16 tokens) and the table
+(logical block i -> physical block); sharing (section 二, "無法共享"): several
+tables may point at the same physical blocks.  Reference counts are how
+"shared" and "freed on completion" fit together: a block returns to the pool
+when the last table that holds it lets go.
+
+Readings where the pages are silent:
+  * the initial free list is a caller-given permutation of [0, NB); blocks are
+    taken from its front and freed blocks are appended to its back;
+  * ``fork(parent, child, n)`` gives the child the parent's first n tokens by
+    sharing the blocks that hold them (refcount + 1 each); n defaults to the
+    parent's length;
+  * appending into a partly filled block that another table also holds needs a
+    copy-on-write this model does not do: it is refused ("unsupported");
+  * every failing call leaves the state exactly as it was.
+"""
+from __future__ import annotations
+
+from collections import deque
+
+BLOCK_TOKENS = 16
+
+
+class AllocError(Exception):
+    def __init__(self, kind: str, msg: str = ""):
+        super().__init__(f"{kind}: {msg}")
+        self.kind = kind  # "invalid" | "oom" | "unsupported"
+
+
+def blocks_for(n_tokens: int) -> int:
+    return -(-n_tokens // BLOCK_TOKENS)
+
+
+class BlockManager:
+    def __init__(self, num_blocks: int, free_order=None):
+        self.num_blocks = int(num_blocks)
+        order = list(range(self.num_blocks)) if free_order is None else [int(b) for b in free_order]
+        if sorted(order) != list(range(self.num_blocks)):
+            raise AllocError("invalid", "free order must be a permutation of the pool")
+        self.free = deque(order)
+        self.ref = [0] * self.num_blocks
+        self.tables: dict[int, list[int]] = {}
+        self.lens: dict[int, int] = {}
+
+    # -- lifecycle ---------------------------------------------------------
+    def add_seq(self, seq_id: int, num_tokens: int) -> None:
+        if seq_id in self.tables or num_tokens < 0:
+            raise AllocError("invalid", "sequence exists or negative length")
+        need = blocks_for(num_tokens)
+        if need > len(self.free):
+            raise AllocError("oom")
+        blocks = [self.free.popleft() for _ in range(need)]
+        for b in blocks:
+            self.ref[b] = 1
+        self.tables[seq_id] = blocks
+        self.lens[seq_id] = num_tokens
+
+    def append_token(self, seq_id: int) -> int:
+        if seq_id not in self.tables:
+            raise AllocError("invalid", "unknown sequence")
+        blocks, pos = self.tables[seq_id], self.lens[seq_id]
+        if pos % BLOCK_TOKENS == 0:
+            if not self.free:
+                raise AllocError("oom")
+            b = self.free.popleft()
+            self.ref[b] = 1
+            blocks.append(b)
+        elif self.ref[blocks[-1]] > 1:
+            raise AllocError("unsupported", "append into a shared, partly filled block")
+        self.lens[seq_id] = pos + 1
+        return blocks[pos // BLOCK_TOKENS] * BLOCK_TOKENS + pos % BLOCK_TOKENS
+
+    def fork(self, parent: int, child: int, num_tokens: int | None = None) -> None:
+        if parent not in self.tables or child in self.tables:
+            raise AllocError("invalid", "unknown parent or existing child")
+        n = self.lens[parent] if num_tokens is None or num_tokens < 0 else num_tokens
+        if n > self.lens[parent]:
+            raise AllocError("invalid", "fork longer than the parent")
+        self.tables[child] = list(self.tables[parent][: blocks_for(n)])
+        self.lens[child] = n
+        for b in self.tables[child]:
+            self.ref[b] += 1
+
+    def free_seq(self, seq_id: int) -> None:
+        if seq_id not in self.tables:
+            raise AllocError("invalid", "unknown sequence")
+        for b in self.tables.pop(seq_id):
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+        del self.lens[seq_id]
+
+    # -- views -------------------------------------------------------------
+    def export(self, seq_ids, width: int):
+        import numpy as np
+
+        tables = np.full((len(seq_ids), width), -1, dtype=np.int32)
+        lens = np.zeros(len(seq_ids), dtype=np.int32)
+        for i, s in enumerate(seq_ids):
+            if s not in self.tables:
+                raise AllocError("invalid", "unknown sequence")
+            blocks = self.tables[s]
+            if len(blocks) > width:
+                raise AllocError("invalid", "table wider than the export width")
+            tables[i, : len(blocks)] = blocks
+            lens[i] = self.lens[s]
+        return tables, lens
+
+    def free_blocks(self) -> list[int]:
+        return list(self.free)
+
+    def slot_of(self, seq_id: int, pos: int) -> int:
+        if not 0 <= pos < self.lens[seq_id]:
+            raise AllocError("invalid", "position outside the sequence")
+        return self.tables[seq_id][pos // BLOCK_TOKENS] * BLOCK_TOKENS + pos % BLOCK_TOKENS
+
+    def refcount(self, block: int) -> int:
+        return self.ref[block]
+
+    def stats(self):
+        """(free, used, shared, utilisation); utilisation = filled slots of the
+        used blocks / (16 * used blocks)."""
+        free = len(self.free)
+        used = self.num_blocks - free
+        shared = sum(1 for r in self.ref if r > 1)
+        fill = {}
+        for s, blocks in self.tables.items():
+            n = self.lens[s]
+            for j, b in enumerate(blocks):
+                fill[b] = max(fill.get(b, 0), min(BLOCK_TOKENS, n - j * BLOCK_TOKENS))
+        util = (sum(fill.values()) / (BLOCK_TOKENS * used)) if used else 0.0
+        return free, used, shared, util
