@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the paged KV-cache decode step on B200.
+
+One step = the whole hot path over one batch: the cache write of every
+sequence's new token (pkv_paged_kv_write) and single-query decode attention
+over the paged cache (pkv_paged_attention_decode).  Block tables and slots
+come from the library's C++ block allocator; values are seeded synthetic bf16
+N(0,1) draws.  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config llama]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch
+(seed + rank) -- independent problems, no collective on the data path -- and
+the job time is the max over ranks of the device-timed K steps.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: KV HBM GB/s (% of B200 peak) and sequences·steps/sec"
+UNIT = "seq*steps/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+WORKLOAD_NAMES = {
+    "tiny": "tiny paged decode: 4 seqs, lens {1,17,33,100}, 4/4 heads, d 64",
+    "llama": "Llama-2-7B-shaped MHA decode: batch 64, 32/32 heads, d 128, len U[128,2048]",
+    "qwen": "Qwen2.5-7B-shaped GQA decode: batch 256, 28/4 heads, d 128, len U[512,4096]",
+    "prefix": "prefix-shared decode: batch 128, 2000-token shared prefix + U[16,512], 32/32, d 128",
+    "long": "long-context GQA decode: batch 8 x 32768, 32/8 heads, d 128, 512-token split-K",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
+    ap.add_argument("--config", choices=sorted(WORKLOAD_NAMES), default="llama")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--variant", choices=["auto", "single", "split"], default="auto")
+    ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU time budget of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def measured_peak_hbm():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(w) -> dict:
+    """Bytes the decode step must move at minimum: every sequence's K and V
+    rows once (len x Hkv x d x 2 B, twice) plus Q; the write moves the new
+    K/V rows in and out."""
+    cfg = w.cfg
+    d, hq, hkv = cfg["head_dim"], cfg["num_heads"], cfg["num_kv_heads"]
+    toks = int(np.asarray(w.lens, dtype=np.int64).sum())
+    kv = toks * hkv * d * 2 * 2
+    q = cfg["batch"] * hq * d * 2
+    out = cfg["batch"] * hq * d * 2
+    write = cfg["batch"] * hkv * d * 2 * 2 * 2
+    return dict(kv=kv, q=q, out=out, write=write, tokens=toks)
+
+
+def source_sha(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the current kernel source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[workload][kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    src = os.path.join(ROOT, "paged_kv_cache_459_b200", "csrc", "decode.cu")
+    if rec.get("decode_cu_sha") != source_sha(src):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is loaded."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str | None):
+        self.proc = None
+        self.lines: list[str] = []
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "50"]
+        if device_id:
+            cmd += ["--id", device_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v
+                          and "Not" not in v})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def device_pci_id(dev) -> str | None:
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- CPU oracle
+class OracleStep:
+    """The fp64 oracle as it stands (C, OpenMP over sequence x KV head) run as
+    one decode step -- write + decode, in place -- over the first `nseq`
+    sequences of a workload, on the host cores."""
+
+    def __init__(self, w):
+        import oracle
+        self.lib = oracle.lib()
+        self.cores = oracle.threads_available()
+        self.w = w
+        self.kc, self.vc = w.k_cache.copy(), w.v_cache.copy()
+        c = w.cfg
+        self.out = np.zeros((c["batch"], c["num_heads"], c["head_dim"]), np.float64)
+        self.tables = np.ascontiguousarray(w.block_tables, np.int32)
+        self.lens = np.ascontiguousarray(w.lens, np.int32)
+
+    def __call__(self, nseq: int) -> None:
+        w, c = self.w, self.w.cfg
+        self.lib.oracle_kv_write(self.kc.ctypes.data, self.vc.ctypes.data, w.k_new.ctypes.data,
+                                 w.v_new.ctypes.data, w.slot_mapping.ctypes.data, nseq,
+                                 c["num_kv_heads"], c["head_dim"], w.num_blocks)
+        rc = self.lib.oracle_paged_decode(
+            self.out.ctypes.data, w.q.ctypes.data, self.kc.ctypes.data, self.vc.ctypes.data,
+            self.tables.ctypes.data, self.tables.shape[1], self.lens.ctypes.data, nseq,
+            c["num_heads"], c["num_kv_heads"], c["head_dim"], w.num_blocks, float(c["scale"]),
+            self.cores)
+        if rc != 0:
+            raise RuntimeError(f"oracle failed ({rc})")
+
+    def seconds_per_seq(self) -> float:
+        n = min(4, self.w.cfg["batch"])
+        t0 = time.perf_counter()
+        self(n)
+        return max(time.perf_counter() - t0, 1e-5) / n
+
+    def timed(self, nseq: int, reps: int) -> float:
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            self(nseq)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s: float) -> dict:
+    """Bounded sample of the oracle on this host: about `budget_s` seconds."""
+    st = OracleStep(w)
+    per_seq = st.seconds_per_seq()
+    b = w.cfg["batch"]
+    nseq = int(min(b, max(1, budget_s / 3 / per_seq)))
+    reps = max(1, int(budget_s / (nseq * per_seq)))
+    el = st.timed(nseq, reps)
+    return {"value": nseq * reps / el, "unit": UNIT, "cores": st.cores, "kind": "oracle",
+            "sample": f"{reps} oracle steps (KV write + decode, fp64) over the first {nseq} of "
+                      f"{b} sequences, {el:.1f} s on {st.cores} threads"}
+
+
+def run_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    from oracle.alloc_model import BlockManager
+    from paged_kv_cache_459_b200 import workloads as wl
+    w = wl.build(args.config, args.seed, BlockManager)
+    st = OracleStep(w)
+    per_seq = st.seconds_per_seq()
+    b = w.cfg["batch"]
+    per_step = 120.0 / max(1, args.steps + args.warmup)  # the whole run within ~2 minutes
+    nseq = int(min(b, max(1, per_step / per_seq)))
+    st.timed(nseq, args.warmup)
+    el = st.timed(nseq, args.steps)
+    val = nseq * args.steps / el
+    line = {
+        "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * el / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[args.config], "name": args.config,
+                   "sample_seqs_per_step": nseq},
+        "impl": "reference",
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": st.cores, "kind": "oracle",
+                         "sample": f"each step: oracle KV write + decode (fp64) over the first "
+                                   f"{nseq} of {b} sequences"},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- GPU path
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from paged_kv_cache_459_b200 import pkv
+    from paged_kv_cache_459_b200 import workloads as wl
+
+    w = wl.build(args.config, args.seed + rank, pkv.BlockAllocator)
+    cfg = w.cfg
+    B, hq, hkv, d = cfg["batch"], cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"]
+
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    q_h, k_h, v_h = (up(x).pin_memory() for x in (w.q, w.k_new, w.v_new))
+    tables_h = torch.from_numpy(w.block_tables).pin_memory()
+    lens_h = torch.from_numpy(w.lens.astype(np.int32)).pin_memory()
+    slots_h = torch.from_numpy(w.slot_mapping).pin_memory()
+    kc = up(w.k_cache).to(dev)
+    vc = up(w.v_cache).to(dev)
+    q, k_new, v_new = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    tables, lens, slots = tables_h.to(dev), lens_h.to(dev), slots_h.to(dev)
+    out = torch.empty_like(q)
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    variant = {"auto": pkv.DECODE_AUTO, "single": pkv.DECODE_SINGLE,
+               "split": pkv.DECODE_SPLIT}[args.variant]
+    W = w.block_tables.shape[1]
+    ws_bytes = pkv.decode_workspace_bytes(B, hq, d, W, args.partition)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    split = variant == pkv.DECODE_SPLIT or (variant == pkv.DECODE_AUTO and W > args.partition // 16)
+    scale = cfg["scale"]
+
+    def write():
+        pkv.paged_kv_write(k_new, v_new, kc, vc, slots, err=err)
+
+    def decode():
+        pkv.paged_attention_decode(out, q, kc, vc, tables, lens, scale, hkv, variant=variant,
+                                   partition_tokens=args.partition, workspace=ws, err=err)
+
+    stream = torch.cuda.current_stream(dev)
+    K, Wm = args.steps, args.warmup
+    for _ in range(Wm):
+        write()
+        decode()
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error word {int(err.item())} after warm-up")
+
+    sampler = ClockSampler(device_pci_id(dev)) if rank == 0 else None
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        write()
+        ev[i][1].record(stream)
+        decode()
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    write_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
+    decode_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev)
+    # keep the GPU loaded long enough for the clock sampler to see it
+    if sampler is not None:
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 1.0:
+            for _ in range(50):
+                write()
+                decode()
+            torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler is not None else None
+
+    # end to end through the public API: pinned host inputs in, output back
+    e2e_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, tables_h, lens_h, slots_h))
+    d2h = out_h.numel() * out_h.element_size()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e2e_ev[0].record(stream)
+    for _ in range(K):
+        for dst, src in ((q, q_h), (k_new, k_h), (v_new, v_h), (tables, tables_h),
+                         (lens, lens_h), (slots, slots_h)):
+            dst.copy_(src, non_blocking=True)
+        write()
+        decode()
+        out_h.copy_(out, non_blocking=True)
+    e2e_ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1])
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error word {int(err.item())} after the timed steps")
+
+    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(times[0]), float(times[1])
+
+    ab = algorithmic_bytes(w)
+    peak, peak_kind = measured_peak_hbm()
+    dec_bytes = ab["kv"] + ab["q"]
+    achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
+    value = B * K * world / (total_ms * 1e-3)
+    e2e_value = B * K * world / (e2e_ms * 1e-3)
+    launches_per_step = 1 + 1 + (1 if split else 0)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD_NAMES[args.config], "name": args.config, "batch": B,
+            "num_heads": hq, "num_kv_heads": hkv, "head_dim": d, "block_tokens": 16,
+            "tokens": ab["tokens"], "num_blocks": w.num_blocks, "table_width": W,
+            "variant": ("split-K %d-token partitions + merge" % args.partition) if split
+            else "single pass (one CTA per sequence x KV head)",
+            "l2": f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), "
+                  "no flush" if ab["kv"] > L2_BYTES else "inputs fit in L2",
+            "parallelism": f"{world} independent replicas (batch per GPU fixed)",
+            "seed": args.seed,
+        },
+        "kv_hbm_gbs": achieved,
+        "kv_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+        "kv_frac_of_measured_copy": achieved / peak,
+        "write_us": write_ms * 1e3, "decode_us": decode_ms * 1e3,
+        "roofline": {
+            "bound": "hbm", "kernel": "paged_attention_decode (decode kernel + split-K merge)",
+            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_kind": peak_kind,
+            "traffic": committed_traffic("paged_decode_kernel", args.config),
+            "algorithmic_bytes_per_launch": dec_bytes,
+        },
+        "gpu_launches": K * launches_per_step,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K},
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

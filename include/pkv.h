@@ -1,0 +1,209 @@
+/*
+ * pkv -- paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libpkv.so.  Plain pointers and sizes only; every device buffer is
+ * owned by the caller (the library never allocates or frees device memory),
+ * and every call is asynchronous on the caller's CUDA stream (`stream` is a
+ * cudaStream_t passed as void*; NULL = the legacy default stream).
+ *
+ * The method (page titles and sections of the pages this library follows):
+ *  - "vLLM 與 PagedAttention：高吞吐推理的關鍵", section 二: the KV cache is cut
+ *    into fixed blocks of 16 tokens; a per-sequence block table maps logical
+ *    block i to a physical block, so a logically contiguous cache can sit
+ *    anywhere in memory; tables of different sequences may point at the same
+ *    physical blocks (shared prefixes).
+ *  - same page, section 三 (運作流程): blocks are taken on demand (step 一/二);
+ *    each decoded token's K/V is written into the current block or into a new
+ *    one when it is full, then attention over all earlier K/V is computed by
+ *    looking them up through the block table (step 三); a finished request
+ *    returns all of its blocks (step 四).
+ *  - "vllm" (xiexianbin.cn), "PagedAttention 的核心原理": on-demand physical
+ *    blocks, logical-to-physical block table, sharing between sequences.
+ *
+ * Layouts (bf16 = IEEE bfloat16, row-major, contiguous):
+ *   k_cache, v_cache   [num_blocks][num_kv_heads][16][head_dim]
+ *   q, out             [num_seqs][num_heads][head_dim]
+ *   k, v (new tokens)  [num_tokens][num_kv_heads][head_dim]
+ *   block_tables       int32 [num_seqs][max_blocks_per_seq]
+ *   seq_lens           int32 [num_seqs]   tokens of each sequence, including
+ *                                         the one decoded this step
+ *   slot_mapping       int64 [num_tokens] slot = physical_block * 16 + offset;
+ *                                         a negative slot means "skip"
+ *
+ * Errors: host-side argument checks return a status before anything is
+ * launched.  Bad data found on the device (a table entry outside
+ * [0, num_blocks), a slot past the pool, a length past the table) never
+ * traps: the offending block, slot or excess length is skipped and a
+ * PKV_DEV_ERR_* bit is OR-ed into *err_word when err_word (a device pointer
+ * to one unsigned int) is non-NULL.  Pipeline waits inside the kernels are
+ * bounded; one that gives up sets PKV_DEV_ERR_TIMEOUT instead of hanging.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#define PKV_BLOCK_TOKENS 16
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned buffer, bad id */
+    PKV_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, pool size, CoW) */
+    PKV_ERR_WORKSPACE = 3,   /* split-K requested without a large enough workspace */
+    PKV_ERR_OOM = 4,         /* block pool exhausted (allocator state unchanged) */
+    PKV_ERR_CUDA = 5         /* a CUDA runtime/driver call failed */
+} pkv_status;
+
+/* Bits OR-ed into *err_word by the kernels. */
+#define PKV_DEV_ERR_BAD_SLOT 1u  /* write: slot >= num_blocks * 16, token skipped */
+#define PKV_DEV_ERR_BAD_BLOCK 2u /* decode: table entry outside [0, num_blocks), block skipped */
+#define PKV_DEV_ERR_BAD_LEN 4u   /* decode: seq_len < 0 or > max_blocks_per_seq * 16, clamped */
+#define PKV_DEV_ERR_TIMEOUT 8u   /* a bounded pipeline wait gave up */
+
+typedef enum {
+    PKV_DECODE_AUTO = 0,   /* choose from the shapes (see pkv_paged_attention_decode) */
+    PKV_DECODE_SINGLE = 1, /* one CTA per (sequence, KV head [, group of 8 query heads]) */
+    PKV_DECODE_SPLIT = 2   /* split-K token partitions + log-sum-exp merge kernel */
+} pkv_decode_variant;
+
+/* Human-readable name of a pkv_status value (static storage). */
+PKV_API const char *pkv_status_string(int status);
+
+/* Tokens per physical block (16). */
+PKV_API int pkv_block_tokens(void);
+
+/* Library version string (static storage). */
+PKV_API const char *pkv_version(void);
+
+/*
+ * Cache write ("vLLM 與 PagedAttention：高吞吐推理的關鍵", section 三, step 三:
+ * the new token's K/V goes into the slot the block manager handed out).
+ * For every token t with slot_mapping[t] >= 0 and every KV head h:
+ *   k_cache[slot / 16][h][slot % 16][:] = k[t][h][:]   (and the same for v)
+ * Bit-exact copy.  head_dim must be a multiple of 8 (16-byte rows); all
+ * device pointers 16-byte aligned.  Duplicate non-negative slots within one
+ * call are a caller error (the surviving value is unspecified).
+ * Slots >= num_blocks * 16 are skipped and flagged PKV_DEV_ERR_BAD_SLOT.
+ */
+PKV_API pkv_status pkv_paged_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
+                              const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                              int head_dim, int64_t num_blocks, unsigned int *err_word,
+                              void *stream);
+
+/*
+ * Workspace (device bytes) that the split-K variant needs for these sizes;
+ * 0 if a size is invalid.  The single-pass variant needs none.
+ */
+PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                  int max_blocks_per_seq, int partition_tokens);
+
+/*
+ * Single-query decode attention over the paged cache (section 三, step 三:
+ * attention over all earlier K/V looked up through the block table), read as
+ *   out[b][h][:] = softmax_p( scale * q[b][h] . K_b[p] ) V_b[p],  p in [0, seq_lens[b])
+ * where K_b[p] = k_cache[block_tables[b][p / 16]][h / (num_heads/num_kv_heads)][p % 16]
+ * (query heads grouped contiguously over KV heads) and the same for V.
+ * bf16 inputs, fp32 accumulation and softmax, bf16 output (round to nearest
+ * even).  seq_lens[b] == 0 gives a zero row.  Table entries at or past
+ * ceil(seq_lens[b] / 16) are never read.
+ *
+ * head_dim: 64 or 128.  num_heads % num_kv_heads == 0.  Pointers 16-byte
+ * aligned.  num_blocks * num_kv_heads * 16 must be < 2^31.
+ * This entry point takes PKV_DECODE_AUTO with 512-token partitions: split-K
+ * when a sequence may span more than one partition and `workspace` holds
+ * pkv_decode_workspace_bytes(...) bytes, the single-pass variant otherwise.
+ * The workspace is scratch owned by the caller; calls that share one
+ * workspace must be ordered on the GPU (the same stream, or events).
+ */
+PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_tables,
+                                      int max_blocks_per_seq, const int32_t *seq_lens,
+                                      int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_dim, int64_t num_blocks, float scale,
+                                      void *workspace, size_t workspace_bytes,
+                                      unsigned int *err_word, void *stream);
+
+/*
+ * As pkv_paged_attention_decode, with the variant and the split-K partition
+ * length chosen by the caller.  partition_tokens: a multiple of 16 in
+ * [16, 65536] (ignored by PKV_DECODE_SINGLE).  PKV_DECODE_SPLIT without enough
+ * workspace returns PKV_ERR_WORKSPACE.
+ */
+PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
+                                         const void *v_cache, const int32_t *block_tables,
+                                         int max_blocks_per_seq, const int32_t *seq_lens,
+                                         int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int64_t num_blocks, float scale,
+                                         int variant, int partition_tokens, void *workspace,
+                                         size_t workspace_bytes, unsigned int *err_word,
+                                         void *stream);
+
+/* ------------------------------------------------------------------------
+ * Host block allocator (section 二 and section 三 of the first page): a pool
+ * of num_blocks physical blocks with reference counts, per-sequence block
+ * tables, on-demand allocation, prefix sharing by fork, and release.
+ * Not thread-safe: one allocator per thread, or external locking.
+ * Every failing call leaves the allocator exactly as it was.
+ * ------------------------------------------------------------------------ */
+typedef struct pkv_alloc pkv_alloc;
+
+/* free_order: a permutation of [0, num_blocks) giving the initial free list
+ * (blocks are taken from its front, freed blocks go to its back); NULL means
+ * ascending order. */
+PKV_API pkv_status pkv_alloc_create(int64_t num_blocks, const int64_t *free_order, pkv_alloc **out);
+PKV_API void pkv_alloc_destroy(pkv_alloc *a);
+
+/* New sequence holding num_tokens prefilled tokens: ceil(num_tokens/16) blocks. */
+PKV_API pkv_status pkv_alloc_add_seq(pkv_alloc *a, int64_t seq_id, int64_t num_tokens);
+
+/* child gets the parent's first num_tokens tokens (num_tokens < 0: all of
+ * them) by sharing the blocks that hold them; each shared block's reference
+ * count goes up by one. */
+PKV_API pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, int64_t num_tokens);
+
+/* One more token for seq_id; *slot_out receives its slot.  A new block is
+ * taken when the last one is full (or there is none).  Appending into a
+ * partly filled block that another sequence also holds would need a
+ * copy-on-write: PKV_ERR_UNSUPPORTED. */
+PKV_API pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_out);
+
+/* One token for each of n distinct sequences (a decode step); all or none. */
+PKV_API pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n,
+                                   int64_t *slots_out);
+
+/* Release a sequence: every block whose count drops to zero returns to the pool. */
+PKV_API pkv_status pkv_alloc_free_seq(pkv_alloc *a, int64_t seq_id);
+
+/* tables_out [n][width] (entries past a sequence's blocks set to -1) and
+ * lens_out [n] for the listed sequences (host memory). */
+PKV_API pkv_status pkv_alloc_export(const pkv_alloc *a, const int64_t *seq_ids, int n, int width,
+                            int32_t *tables_out, int32_t *lens_out);
+
+/* free and used blocks, blocks with count > 1, and utilisation = filled
+ * slots of the used blocks / (16 * used blocks) (0 when nothing is used). */
+PKV_API pkv_status pkv_alloc_stats(const pkv_alloc *a, int64_t *free_blocks, int64_t *used_blocks,
+                           int64_t *shared_blocks, double *utilisation);
+
+/* The free list, front first: up to cap ids into out, the count into *n_out. */
+PKV_API pkv_status pkv_alloc_free_list(const pkv_alloc *a, int64_t *out, int64_t cap, int64_t *n_out);
+
+PKV_API pkv_status pkv_alloc_refcount(const pkv_alloc *a, int64_t block, int32_t *out);
+PKV_API pkv_status pkv_alloc_seq_len(const pkv_alloc *a, int64_t seq_id, int64_t *len_out);
+PKV_API pkv_status pkv_alloc_slot_of(const pkv_alloc *a, int64_t seq_id, int64_t pos, int64_t *slot_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -78,6 +78,23 @@ class BlockManager:
         self.lens[seq_id] = pos + 1
         return blocks[pos // BLOCK_TOKENS] * BLOCK_TOKENS + pos % BLOCK_TOKENS
 
+    def append_tokens(self, seq_ids) -> list[int]:
+        """One token for each listed sequence (one decode step), all or none:
+        an unknown or repeated id, then a shared partly filled last block, then
+        a shortage of free blocks is reported before anything changes."""
+        ids = list(seq_ids)
+        if len(set(ids)) != len(ids) or any(s not in self.tables for s in ids):
+            raise AllocError("invalid", "unknown or repeated sequence")
+        need = 0
+        for s in ids:
+            if self.lens[s] % BLOCK_TOKENS == 0:
+                need += 1
+            elif self.ref[self.tables[s][-1]] > 1:
+                raise AllocError("unsupported", "append into a shared, partly filled block")
+        if need > len(self.free):
+            raise AllocError("oom")
+        return [self.append_token(s) for s in ids]
+
     def fork(self, parent: int, child: int, num_tokens: int | None = None) -> None:
         if parent not in self.tables or child in self.tables:
             raise AllocError("invalid", "unknown parent or existing child")

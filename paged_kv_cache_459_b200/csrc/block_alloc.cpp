@@ -1,0 +1,272 @@
+// Host block allocator: reference-counted physical blocks, per-sequence block
+// tables, on-demand allocation, prefix sharing and release.
+//
+// Follows "vLLM 與 PagedAttention：高吞吐推理的關鍵": section 二 (fixed 16-token
+// blocks; a table maps logical block i to a physical block; several tables may
+// point at the same blocks) and section 三 (an empty table at admission, a new
+// block whenever the current one fills during prefill and decode, every block
+// returned when the request finishes).  Reference counts reconcile sharing
+// with release: a block goes back to the pool when its last holder lets go.
+//
+// The free list is a deque: blocks are taken from the front and returned to
+// the back, starting from a caller-given permutation, so tables are
+// reproducible for a seed.  Every call validates first and mutates only once
+// it cannot fail, so an error leaves the state unchanged.
+#include <algorithm>
+#include <deque>
+#include <new>
+#include <unordered_map>
+#include <unordered_set>
+#include <vector>
+
+#include "../../include/pkv.h"
+
+namespace {
+
+constexpr int64_t kBlockTokens = PKV_BLOCK_TOKENS;
+
+int64_t blocks_for(int64_t tokens) { return (tokens + kBlockTokens - 1) / kBlockTokens; }
+
+struct Sequence {
+    std::vector<int32_t> blocks;
+    int64_t len = 0;
+};
+
+}  // namespace
+
+struct pkv_alloc {
+    int64_t num_blocks = 0;
+    std::deque<int32_t> free_list;
+    std::vector<int32_t> refcount;
+    std::unordered_map<int64_t, Sequence> seqs;
+};
+
+extern "C" {
+
+pkv_status pkv_alloc_create(int64_t num_blocks, const int64_t *free_order, pkv_alloc **out) {
+    if (!out || num_blocks <= 0 || num_blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    pkv_alloc *a = new (std::nothrow) pkv_alloc;
+    if (!a) return PKV_ERR_OOM;
+    try {
+        a->num_blocks = num_blocks;
+        a->refcount.assign(static_cast<size_t>(num_blocks), 0);
+        if (free_order) {
+            std::vector<char> seen(static_cast<size_t>(num_blocks), 0);
+            for (int64_t i = 0; i < num_blocks; ++i) {
+                int64_t b = free_order[i];
+                if (b < 0 || b >= num_blocks || seen[b]) {
+                    delete a;
+                    return PKV_ERR_INVALID_ARG;
+                }
+                seen[b] = 1;
+                a->free_list.push_back(static_cast<int32_t>(b));
+            }
+        } else {
+            for (int64_t i = 0; i < num_blocks; ++i) a->free_list.push_back(static_cast<int32_t>(i));
+        }
+    } catch (const std::bad_alloc &) {
+        delete a;
+        return PKV_ERR_OOM;
+    }
+    *out = a;
+    return PKV_OK;
+}
+
+void pkv_alloc_destroy(pkv_alloc *a) { delete a; }
+
+pkv_status pkv_alloc_add_seq(pkv_alloc *a, int64_t seq_id, int64_t num_tokens) {
+    if (!a || num_tokens < 0 || a->seqs.count(seq_id)) return PKV_ERR_INVALID_ARG;
+    int64_t need = blocks_for(num_tokens);
+    if (need > static_cast<int64_t>(a->free_list.size())) return PKV_ERR_OOM;
+    try {
+        Sequence s;
+        s.blocks.reserve(static_cast<size_t>(need));
+        s.len = num_tokens;
+        for (int64_t i = 0; i < need; ++i) s.blocks.push_back(a->free_list[static_cast<size_t>(i)]);
+        a->seqs.emplace(seq_id, std::move(s));
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    for (int64_t i = 0; i < need; ++i) {
+        a->refcount[a->free_list.front()] = 1;
+        a->free_list.pop_front();
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, int64_t num_tokens) {
+    if (!a) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(parent);
+    if (it == a->seqs.end() || a->seqs.count(child)) return PKV_ERR_INVALID_ARG;
+    int64_t n = num_tokens < 0 ? it->second.len : num_tokens;
+    if (n > it->second.len) return PKV_ERR_INVALID_ARG;
+    try {
+        Sequence s;
+        s.len = n;
+        s.blocks.assign(it->second.blocks.begin(), it->second.blocks.begin() + blocks_for(n));
+        for (int32_t b : s.blocks) a->refcount[b] += 1;
+        a->seqs.emplace(child, std::move(s));
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    return PKV_OK;
+}
+
+// Checks one append; returns whether it needs a new block.
+static pkv_status check_append(const pkv_alloc *a, const Sequence &s, bool *needs_block) {
+    *needs_block = (s.len % kBlockTokens) == 0;
+    if (!*needs_block && a->refcount[s.blocks.back()] > 1) return PKV_ERR_UNSUPPORTED;
+    return PKV_OK;
+}
+
+static int64_t do_append(pkv_alloc *a, Sequence &s, bool needs_block) {
+    if (needs_block) {
+        int32_t b = a->free_list.front();
+        a->free_list.pop_front();
+        a->refcount[b] = 1;
+        s.blocks.push_back(b);
+    }
+    int64_t pos = s.len++;
+    return static_cast<int64_t>(s.blocks[pos / kBlockTokens]) * kBlockTokens + pos % kBlockTokens;
+}
+
+pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_out) {
+    if (!a || !slot_out) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+    bool needs_block;
+    pkv_status st = check_append(a, it->second, &needs_block);
+    if (st != PKV_OK) return st;
+    if (needs_block && a->free_list.empty()) return PKV_ERR_OOM;
+    try {
+        if (needs_block) it->second.blocks.reserve(it->second.blocks.size() + 1);
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    *slot_out = do_append(a, it->second, needs_block);
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *slots_out) {
+    if (!a || n < 0 || (n > 0 && (!seq_ids || !slots_out))) return PKV_ERR_INVALID_ARG;
+    std::vector<Sequence *> seqs;
+    std::vector<char> needs;
+    try {
+        std::unordered_set<int64_t> seen;
+        seqs.reserve(static_cast<size_t>(n));
+        needs.reserve(static_cast<size_t>(n));
+        int64_t new_blocks = 0;
+        for (int i = 0; i < n; ++i) {
+            if (!seen.insert(seq_ids[i]).second) return PKV_ERR_INVALID_ARG;
+            auto it = a->seqs.find(seq_ids[i]);
+            if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+            bool nb;
+            pkv_status st = check_append(a, it->second, &nb);
+            if (st != PKV_OK) return st;
+            if (nb) it->second.blocks.reserve(it->second.blocks.size() + 1);
+            new_blocks += nb;
+            seqs.push_back(&it->second);
+            needs.push_back(nb);
+        }
+        if (new_blocks > static_cast<int64_t>(a->free_list.size())) return PKV_ERR_OOM;
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    for (int i = 0; i < n; ++i) slots_out[i] = do_append(a, *seqs[i], needs[i] != 0);
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_free_seq(pkv_alloc *a, int64_t seq_id) {
+    if (!a) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+    for (int32_t b : it->second.blocks) {
+        if (--a->refcount[b] == 0) a->free_list.push_back(b);
+    }
+    a->seqs.erase(it);
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_export(const pkv_alloc *a, const int64_t *seq_ids, int n, int width,
+                            int32_t *tables_out, int32_t *lens_out) {
+    if (!a || n < 0 || width <= 0 || (n > 0 && (!seq_ids || !tables_out || !lens_out)))
+        return PKV_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        auto it = a->seqs.find(seq_ids[i]);
+        if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+        if (static_cast<int64_t>(it->second.blocks.size()) > width || it->second.len > INT32_MAX)
+            return PKV_ERR_INVALID_ARG;
+    }
+    for (int i = 0; i < n; ++i) {
+        const Sequence &s = a->seqs.find(seq_ids[i])->second;
+        int32_t *row = tables_out + static_cast<size_t>(i) * width;
+        std::fill(row, row + width, -1);
+        std::copy(s.blocks.begin(), s.blocks.end(), row);
+        lens_out[i] = static_cast<int32_t>(s.len);
+    }
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_stats(const pkv_alloc *a, int64_t *free_blocks, int64_t *used_blocks,
+                           int64_t *shared_blocks, double *utilisation) {
+    if (!a) return PKV_ERR_INVALID_ARG;
+    int64_t free_n = static_cast<int64_t>(a->free_list.size());
+    int64_t used = a->num_blocks - free_n;
+    int64_t shared = 0;
+    for (int32_t r : a->refcount) shared += r > 1;
+    double util = 0.0;
+    if (used > 0) {
+        std::vector<int16_t> fill(static_cast<size_t>(a->num_blocks), 0);
+        for (const auto &kv : a->seqs) {
+            const Sequence &s = kv.second;
+            for (size_t j = 0; j < s.blocks.size(); ++j) {
+                int64_t f = std::min<int64_t>(kBlockTokens, s.len - static_cast<int64_t>(j) * kBlockTokens);
+                int16_t &slot = fill[s.blocks[j]];
+                slot = std::max<int16_t>(slot, static_cast<int16_t>(f));
+            }
+        }
+        int64_t filled = 0;
+        for (int16_t f : fill) filled += f;
+        util = static_cast<double>(filled) / static_cast<double>(kBlockTokens * used);
+    }
+    if (free_blocks) *free_blocks = free_n;
+    if (used_blocks) *used_blocks = used;
+    if (shared_blocks) *shared_blocks = shared;
+    if (utilisation) *utilisation = util;
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_free_list(const pkv_alloc *a, int64_t *out, int64_t cap, int64_t *n_out) {
+    if (!a || !n_out || cap < 0 || (cap > 0 && !out)) return PKV_ERR_INVALID_ARG;
+    int64_t n = static_cast<int64_t>(a->free_list.size());
+    int64_t m = std::min(n, cap);
+    for (int64_t i = 0; i < m; ++i) out[i] = a->free_list[static_cast<size_t>(i)];
+    *n_out = n;
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_refcount(const pkv_alloc *a, int64_t block, int32_t *out) {
+    if (!a || !out || block < 0 || block >= a->num_blocks) return PKV_ERR_INVALID_ARG;
+    *out = a->refcount[static_cast<size_t>(block)];
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_seq_len(const pkv_alloc *a, int64_t seq_id, int64_t *len_out) {
+    if (!a || !len_out) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+    *len_out = it->second.len;
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_slot_of(const pkv_alloc *a, int64_t seq_id, int64_t pos, int64_t *slot_out) {
+    if (!a || !slot_out) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || pos < 0 || pos >= it->second.len) return PKV_ERR_INVALID_ARG;
+    *slot_out = static_cast<int64_t>(it->second.blocks[pos / kBlockTokens]) * kBlockTokens +
+                pos % kBlockTokens;
+    return PKV_OK;
+}
+
+}  // extern "C"

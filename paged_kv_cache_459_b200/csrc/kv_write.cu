@@ -1,0 +1,58 @@
+// Paged KV-cache write: scatter each new token's K and V rows into the slot
+// the block manager handed out ("vLLM 與 PagedAttention：高吞吐推理的關鍵",
+// section 三, step 三: write into the current block, or a new one when full).
+//
+// One thread per 16-byte vector of a (token, KV head) row; K and V move in
+// the same thread.  A few MB per decode step at most, so the kernel is
+// launch- and latency-bound; coalesced 16-byte loads and stores are all it
+// needs.  Bit-exact: plain copies, no arithmetic on the values.
+#include "../../include/pkv.h"
+#include "internal.h"
+
+namespace pkv {
+
+__global__ void __launch_bounds__(256) kv_write_kernel(const uint4 *__restrict__ k,
+                                                       const uint4 *__restrict__ v,
+                                                       uint4 *__restrict__ k_cache,
+                                                       uint4 *__restrict__ v_cache,
+                                                       const int64_t *__restrict__ slots,
+                                                       long long total, int vec_per_row, int Hkv,
+                                                       long long num_blocks, unsigned int *err) {
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const int vec = static_cast<int>(idx % vec_per_row);
+    const long long row = idx / vec_per_row;
+    const int h = static_cast<int>(row % Hkv);
+    const long long t = row / Hkv;
+    const long long slot = slots[t];
+    if (slot < 0) return;
+    if (slot >= num_blocks * kBlockTokens) {
+        if (err != nullptr && vec == 0 && h == 0) atomicOr(err, PKV_DEV_ERR_BAD_SLOT);
+        return;
+    }
+    const long long blk = slot / kBlockTokens;
+    const int off = static_cast<int>(slot % kBlockTokens);
+    const long long dst = ((blk * Hkv + h) * kBlockTokens + off) * vec_per_row + vec;
+    const uint4 kv = __ldg(k + idx);
+    const uint4 vv = __ldg(v + idx);
+    k_cache[dst] = kv;
+    v_cache[dst] = vv;
+}
+
+cudaError_t launch_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
+                            const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                            int head_dim, long long num_blocks, unsigned int *err,
+                            cudaStream_t stream) {
+    const int vec_per_row = head_dim / 8;
+    const long long total = static_cast<long long>(num_tokens) * num_kv_heads * vec_per_row;
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    const long long blocks = (total + threads - 1) / threads;
+    kv_write_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(k_cache),
+        static_cast<uint4 *>(v_cache), slot_mapping, total, vec_per_row, num_kv_heads, num_blocks,
+        err);
+    return cudaGetLastError();
+}
+
+}  // namespace pkv

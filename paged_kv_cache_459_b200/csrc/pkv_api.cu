@@ -1,0 +1,196 @@
+// C ABI of libpkv.so: argument checks, TMA descriptor set-up and dispatch.
+// Nothing here allocates device memory; every launch goes on the caller's
+// stream.  See include/pkv.h for the contract of each entry point.
+#include <cmath>
+#include <cstdlib>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/pkv.h"
+#include "internal.h"
+
+namespace {
+
+constexpr int kDefaultPartitionTokens = 512;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// One cache array seen by TMA as a 2-D bf16 tensor: rows = (block, kv head,
+// token) flattened, columns = head_dim.  Boxes are [16 rows][64 columns] --
+// 128-byte rows, the 128-byte swizzle -- so a (block, head) tile of K or V is
+// head_dim/64 boxes.
+bool encode_cache_map(CUtensorMap *m, const void *cache, int64_t rows, int head_dim) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(cache), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int env_int(const char *name, int fallback) {
+    const char *s = std::getenv(name);
+    return (s && *s) ? std::atoi(s) : fallback;
+}
+
+int num_parts_for(int max_blocks_per_seq, int partition_tokens) {
+    const int pb = partition_tokens / PKV_BLOCK_TOKENS;
+    return (max_blocks_per_seq + pb - 1) / pb;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pkv_status_string(int status) {
+    switch (status) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_INVALID_ARG: return "invalid argument";
+        case PKV_ERR_UNSUPPORTED: return "unsupported";
+        case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+        case PKV_ERR_OOM: return "out of blocks";
+        case PKV_ERR_CUDA: return "CUDA error";
+        default: return "unknown status";
+    }
+}
+
+int pkv_block_tokens(void) { return PKV_BLOCK_TOKENS; }
+
+const char *pkv_version(void) { return "pkv 0.1 sm_100a"; }
+
+pkv_status pkv_paged_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
+                              const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                              int head_dim, int64_t num_blocks, unsigned int *err_word,
+                              void *stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 || num_blocks <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_INVALID_ARG;
+    if (num_blocks > (INT64_MAX / PKV_BLOCK_TOKENS) / num_kv_heads / head_dim)
+        return PKV_ERR_INVALID_ARG;
+    cudaError_t e = pkv::launch_kv_write(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                         num_kv_heads, head_dim, num_blocks, err_word,
+                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                  int max_blocks_per_seq, int partition_tokens) {
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0) return 0;
+    if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
+    if (partition_tokens % PKV_BLOCK_TOKENS) return 0;
+    const size_t parts = static_cast<size_t>(num_parts_for(max_blocks_per_seq, partition_tokens));
+    const size_t rows = static_cast<size_t>(num_seqs) * num_heads * parts;
+    return rows * (static_cast<size_t>(head_dim) + 2) * sizeof(float);
+}
+
+pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
+                                         const void *v_cache, const int32_t *block_tables,
+                                         int max_blocks_per_seq, const int32_t *seq_lens,
+                                         int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int64_t num_blocks, float scale,
+                                         int variant, int partition_tokens, void *workspace,
+                                         size_t workspace_bytes, unsigned int *err_word,
+                                         void *stream) {
+    if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_heads % num_kv_heads || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        !std::isfinite(scale))
+        return PKV_ERR_INVALID_ARG;
+    if (variant < PKV_DECODE_AUTO || variant > PKV_DECODE_SPLIT) return PKV_ERR_INVALID_ARG;
+    if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
+    if (partition_tokens % PKV_BLOCK_TOKENS || partition_tokens > 65536) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_INVALID_ARG;
+    const int64_t rows = num_blocks * num_kv_heads * PKV_BLOCK_TOKENS;
+    if (num_blocks > INT32_MAX / PKV_BLOCK_TOKENS / num_kv_heads) return PKV_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(max_blocks_per_seq) * PKV_BLOCK_TOKENS > INT32_MAX)
+        return PKV_ERR_INVALID_ARG;
+
+    const int part_blocks = partition_tokens / PKV_BLOCK_TOKENS;
+    const size_t need = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                   max_blocks_per_seq, partition_tokens);
+    const bool ws_ok = workspace != nullptr && workspace_bytes >= need && aligned16(workspace);
+    bool split;
+    if (variant == PKV_DECODE_SPLIT) {
+        if (!ws_ok) return PKV_ERR_WORKSPACE;
+        split = true;
+    } else if (variant == PKV_DECODE_SINGLE) {
+        split = false;
+    } else {
+        split = max_blocks_per_seq > part_blocks && ws_ok;
+    }
+
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, k_cache, rows, head_dim) ||
+        !encode_cache_map(&tmv, v_cache, rows, head_dim))
+        return PKV_ERR_CUDA;
+
+    pkv::DecodeParams p{};
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err = err_word;
+    p.num_blocks = num_blocks;
+    p.W = max_blocks_per_seq;
+    p.B = num_seqs;
+    p.Hq = num_heads;
+    p.Hkv = num_kv_heads;
+    p.group = num_heads / num_kv_heads;
+    p.chunks = (p.group + 7) / 8;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    if (split) {
+        p.part_blocks = part_blocks;
+        p.num_parts = num_parts_for(max_blocks_per_seq, partition_tokens);
+        const size_t rows_ws = static_cast<size_t>(num_seqs) * num_heads * p.num_parts;
+        p.ws_o = static_cast<float *>(workspace);
+        p.ws_ml = p.ws_o + rows_ws * head_dim;
+    } else {
+        p.part_blocks = max_blocks_per_seq;
+        p.num_parts = 1;
+    }
+    pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 3)};
+    cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, split, t,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_tables,
+                                      int max_blocks_per_seq, const int32_t *seq_lens,
+                                      int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_dim, int64_t num_blocks, float scale,
+                                      void *workspace, size_t workspace_bytes,
+                                      unsigned int *err_word, void *stream) {
+    return pkv_paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables,
+                                         max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                                         num_kv_heads, head_dim, num_blocks, scale,
+                                         PKV_DECODE_AUTO, kDefaultPartitionTokens, workspace,
+                                         workspace_bytes, err_word, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,273 @@
+"""Python binding of libpkv.so (ctypes): argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels; PyTorch supplies
+device memory and the current stream.  If the library has not been built the
+import fails loudly -- there is no fallback implementation.
+
+    paged_kv_write(k, v, k_cache, v_cache, slot_mapping)
+    paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, num_kv_heads)
+    BlockAllocator(num_blocks, free_order=None)   # host allocator (C++)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "pkv.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_459_b200.build` "
+        "(nvcc, sm_100a). There is no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_OOM, ERR_CUDA = range(6)
+DEV_ERR_BAD_SLOT, DEV_ERR_BAD_BLOCK, DEV_ERR_BAD_LEN, DEV_ERR_TIMEOUT = 1, 2, 4, 8
+DECODE_AUTO, DECODE_SINGLE, DECODE_SPLIT = 0, 1, 2
+BLOCK_TOKENS = 16
+DEFAULT_PARTITION_TOKENS = 512
+
+_P, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_sigs = {
+    "pkv_status_string": ([_i32], ctypes.c_char_p),
+    "pkv_block_tokens": ([], _i32),
+    "pkv_version": ([], ctypes.c_char_p),
+    "pkv_paged_kv_write": ([_P, _P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P], _i32),
+    "pkv_decode_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
+    "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
+                                    _f32, _P, _sz, _P, _P], _i32),
+    "pkv_paged_attention_decode_ex": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
+                                       _f32, _i32, _i32, _P, _sz, _P, _P], _i32),
+    "pkv_alloc_create": ([_i64, _P, _P], _i32),
+    "pkv_alloc_destroy": ([_P], None),
+    "pkv_alloc_add_seq": ([_P, _i64, _i64], _i32),
+    "pkv_alloc_fork": ([_P, _i64, _i64, _i64], _i32),
+    "pkv_alloc_append_token": ([_P, _i64, _P], _i32),
+    "pkv_alloc_append_tokens": ([_P, _P, _i32, _P], _i32),
+    "pkv_alloc_free_seq": ([_P, _i64], _i32),
+    "pkv_alloc_export": ([_P, _P, _i32, _i32, _P, _P], _i32),
+    "pkv_alloc_stats": ([_P, _P, _P, _P, _P], _i32),
+    "pkv_alloc_free_list": ([_P, _P, _i64, _P], _i32),
+    "pkv_alloc_refcount": ([_P, _i64, _P], _i32),
+    "pkv_alloc_seq_len": ([_P, _i64, _P], _i32),
+    "pkv_alloc_slot_of": ([_P, _i64, _i64, _P], _i32),
+}
+for _name, (_args, _res) in _sigs.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def declared_symbols(header: str = HEADER) -> list[str]:
+    """Names of the functions include/pkv.h declares."""
+    text = open(header).read()
+    return sorted(set(re.findall(r"^PKV_API[^(;]*?\b(pkv_\w+)\s*\(", text, flags=re.M)))
+
+
+def status_string(code: int) -> str:
+    return _lib.pkv_status_string(code).decode()
+
+
+class PkvError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+def _check(code: int, what: str) -> None:
+    if code != OK:
+        raise PkvError(code, what)
+
+
+# ------------------------------------------------------------------ kernels
+def _dev_tensor(t, dtype, name):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_ptr(device) -> int:
+    import torch
+
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def paged_kv_write(k, v, k_cache, v_cache, slot_mapping, err=None) -> None:
+    """k, v [T, Hkv, d] bf16; caches [NB, Hkv, 16, d] bf16; slot_mapping [T] int64."""
+    import torch
+
+    bf = torch.bfloat16
+    T, hkv, d = k.shape
+    if v.shape != k.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (hkv, BLOCK_TOKENS, d) or slot_mapping.shape != (T,):
+        raise ValueError("shape mismatch")
+    ptrs = [_dev_tensor(x, bf, n) for x, n in ((k, "k"), (v, "v"), (k_cache, "k_cache"),
+                                                 (v_cache, "v_cache"))]
+    sp = _dev_tensor(slot_mapping, torch.int64, "slot_mapping")
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    _check(_lib.pkv_paged_kv_write(*ptrs, sp, T, hkv, d, k_cache.shape[0], ep,
+                                   _stream_ptr(k.device)), "pkv_paged_kv_write")
+
+
+_workspaces: dict = {}
+
+
+def _workspace(device, nbytes: int):
+    import torch
+
+    key = (device.type, device.index)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def decode_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_seq,
+                           partition_tokens=DEFAULT_PARTITION_TOKENS) -> int:
+    return int(_lib.pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_seq,
+                                               partition_tokens))
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, num_kv_heads,
+                           *, variant: int = DECODE_AUTO,
+                           partition_tokens: int = DEFAULT_PARTITION_TOKENS,
+                           workspace=None, err=None) -> None:
+    """out, q [B, Hq, d] bf16; caches [NB, Hkv, 16, d] bf16; block_tables [B, W]
+    int32; seq_lens [B] int32.  The split-K workspace is allocated once per
+    device and reused unless one is passed in (a uint8 CUDA tensor)."""
+    import torch
+
+    bf = torch.bfloat16
+    B, hq, d = q.shape
+    W = block_tables.shape[1] if block_tables.dim() == 2 else -1
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
+            or block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("shape mismatch")
+    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"),
+                                                 (v_cache, "v_cache"))]
+    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
+    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    need = decode_workspace_bytes(B, hq, d, W, partition_tokens) if W > 0 else 0
+    if workspace is None and variant != DECODE_SINGLE and need > 0:
+        workspace = _workspace(q.device, need)
+    wp = _dev_tensor(workspace, torch.uint8, "workspace") if workspace is not None else None
+    wbytes = workspace.numel() if workspace is not None else 0
+    _check(_lib.pkv_paged_attention_decode_ex(ptrs[0], ptrs[1], ptrs[2], ptrs[3], tp, W, lp, B, hq,
+                                              num_kv_heads, d, k_cache.shape[0], float(scale),
+                                              variant, partition_tokens, wp, wbytes, ep,
+                                              _stream_ptr(q.device)),
+           "pkv_paged_attention_decode")
+
+
+# ---------------------------------------------------------------- allocator
+class AllocError(PkvError):
+    @property
+    def kind(self) -> str:
+        return {ERR_OOM: "oom", ERR_UNSUPPORTED: "unsupported"}.get(self.code, "invalid")
+
+
+def _acheck(code: int, what: str) -> None:
+    if code != OK:
+        raise AllocError(code, what)
+
+
+class BlockAllocator:
+    """The C++ block allocator: reference-counted blocks, per-sequence tables."""
+
+    def __init__(self, num_blocks: int, free_order=None):
+        h = ctypes.c_void_p()
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int64)
+            if order.shape != (num_blocks,):
+                raise AllocError(ERR_INVALID_ARG, "free order length")
+        _acheck(_lib.pkv_alloc_create(int(num_blocks), order.ctypes.data if order is not None
+                                      else None, ctypes.byref(h)), "pkv_alloc_create")
+        self._h = h
+        self.num_blocks = int(num_blocks)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib.pkv_alloc_destroy(h)
+            self._h = None
+
+    def add_seq(self, seq_id: int, num_tokens: int) -> None:
+        _acheck(_lib.pkv_alloc_add_seq(self._h, int(seq_id), int(num_tokens)), "add_seq")
+
+    def fork(self, parent: int, child: int, num_tokens: int | None = None) -> None:
+        _acheck(_lib.pkv_alloc_fork(self._h, int(parent), int(child),
+                                    -1 if num_tokens is None else int(num_tokens)), "fork")
+
+    def append_token(self, seq_id: int) -> int:
+        out = ctypes.c_int64()
+        _acheck(_lib.pkv_alloc_append_token(self._h, int(seq_id), ctypes.byref(out)), "append_token")
+        return out.value
+
+    def append_tokens(self, seq_ids) -> np.ndarray:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        out = np.empty(len(ids), dtype=np.int64)
+        _acheck(_lib.pkv_alloc_append_tokens(self._h, ids.ctypes.data, len(ids), out.ctypes.data),
+                "append_tokens")
+        return out
+
+    def free_seq(self, seq_id: int) -> None:
+        _acheck(_lib.pkv_alloc_free_seq(self._h, int(seq_id)), "free_seq")
+
+    def export(self, seq_ids, width: int):
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        tables = np.empty((len(ids), width), dtype=np.int32)
+        lens = np.empty(len(ids), dtype=np.int32)
+        _acheck(_lib.pkv_alloc_export(self._h, ids.ctypes.data, len(ids), int(width),
+                                      tables.ctypes.data, lens.ctypes.data), "export")
+        return tables, lens
+
+    def stats(self):
+        f, u, s, x = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64(), ctypes.c_double()
+        _acheck(_lib.pkv_alloc_stats(self._h, ctypes.byref(f), ctypes.byref(u), ctypes.byref(s),
+                                     ctypes.byref(x)), "stats")
+        return f.value, u.value, s.value, x.value
+
+    def free_blocks(self) -> list[int]:
+        n = ctypes.c_int64()
+        _acheck(_lib.pkv_alloc_free_list(self._h, None, 0, ctypes.byref(n)), "free_list")
+        out = np.empty(n.value, dtype=np.int64)
+        _acheck(_lib.pkv_alloc_free_list(self._h, out.ctypes.data if n.value else None, n.value,
+                                         ctypes.byref(n)), "free_list")
+        return out.tolist()
+
+    def refcount(self, block: int) -> int:
+        out = ctypes.c_int32()
+        _acheck(_lib.pkv_alloc_refcount(self._h, int(block), ctypes.byref(out)), "refcount")
+        return out.value
+
+    def seq_len(self, seq_id: int) -> int:
+        out = ctypes.c_int64()
+        _acheck(_lib.pkv_alloc_seq_len(self._h, int(seq_id), ctypes.byref(out)), "seq_len")
+        return out.value
+
+    def slot_of(self, seq_id: int, pos: int) -> int:
+        out = ctypes.c_int64()
+        _acheck(_lib.pkv_alloc_slot_of(self._h, int(seq_id), int(pos), ctypes.byref(out)), "slot_of")
+        return out.value

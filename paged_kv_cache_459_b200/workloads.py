@@ -20,14 +20,16 @@ prefix     128    32/32   128  2000-token shared prefix + U[16, 512] suffix
 long       8      32/8    128  32768 each; 20000-block pool
 =========  =====  ======  ===  ===========================================
 
-Values are bf16 = round-to-nearest-even of N(0, 1) float32 draws from a PCG64
-generator.  Every block starts with random values; blocks that no table uses,
-the unused tail slots of each sequence's last block and the slot of the new
-token are then set to bf16 NaN so that a stray read shows up in the output.
+Values are bf16 = round-to-nearest-even of N(0, 1) float32 draws from PCG64
+generators (one per 4M-element chunk, keyed by seed, stream and chunk).
+Every block starts with random values; blocks that no table uses, the unused
+tail slots of each sequence's last block and the slot of the new token are
+then set to bf16 NaN so that a stray read shows up in the output.
 """
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -62,17 +64,35 @@ def rng(seed: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(seed))
 
 
-def bf16_normal(shape, gen: np.random.Generator, chunk: int = 1 << 24) -> np.ndarray:
-    """bf16 bit patterns (uint16) of round-to-nearest-even N(0,1) float32 draws."""
+_CHUNK = 1 << 22
+
+
+def _normal_chunk(args):
+    seed, stream, c, n = args
+    gen = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, stream, c])))
+    f = gen.standard_normal(n, dtype=np.float32)
+    u = f.view(np.uint32)
+    # round to nearest even on the upper 16 bits; the draws are finite
+    u += np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_normal(shape, seed: int, stream: int) -> np.ndarray:
+    """bf16 bit patterns (uint16) of round-to-nearest-even N(0,1) float32 draws.
+
+    Element i of stream ``stream`` comes from chunk i // 2^22, drawn by its own
+    PCG64 seeded with SeedSequence([seed, stream, chunk]); chunks are drawn in
+    parallel threads, so the values do not depend on the thread count."""
     n = int(np.prod(shape))
-    out = np.empty(n, dtype=np.uint16)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
-        f = gen.standard_normal(e - s, dtype=np.float32)
-        u = f.view(np.uint32)
-        # RNE to the upper 16 bits; the draws are finite, so no NaN handling.
-        u = u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
-        out[s:e] = (u >> np.uint32(16)).astype(np.uint16)
+    jobs = [(int(seed), int(stream), c, min(_CHUNK, n - c * _CHUNK))
+            for c in range(-(-n // _CHUNK))]
+    if len(jobs) <= 1:
+        parts = [_normal_chunk(j) for j in jobs]
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+            parts = list(ex.map(_normal_chunk, jobs))
+    out = np.concatenate(parts) if parts else np.empty(0, np.uint16)
     return out.reshape(shape)
 
 
@@ -169,14 +189,14 @@ def build(name: str, seed: int, alloc_factory, *, batch: int | None = None,
     tables, out_lens = alloc.export(seq_ids, w)
     assert np.array_equal(out_lens.astype(np.int64), lens)
     hq, hkv, d = cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"]
-    q = bf16_normal((b, hq, d), gen)
-    k_new = bf16_normal((b, hkv, d), gen)
-    v_new = bf16_normal((b, hkv, d), gen)
+    q = bf16_normal((b, hq, d), seed, 1)
+    k_new = bf16_normal((b, hkv, d), seed, 2)
+    v_new = bf16_normal((b, hkv, d), seed, 3)
     free = np.asarray(alloc.free_blocks(), dtype=np.int64)
     kc = vc = None
     if with_cache:
-        kc = bf16_normal((nblocks, hkv, BLOCK_TOKENS, d), gen)
-        vc = bf16_normal((nblocks, hkv, BLOCK_TOKENS, d), gen)
+        kc = bf16_normal((nblocks, hkv, BLOCK_TOKENS, d), seed, 4)
+        vc = bf16_normal((nblocks, hkv, BLOCK_TOKENS, d), seed, 5)
         if poison:
             poison_cache(kc, vc, free, tables, out_lens, slots)
     return Workload(cfg=cfg, seed=seed, lens=out_lens.astype(np.int32), block_tables=tables,

@@ -1,0 +1,94 @@
+"""The C-ABI library builds, loads and exports what include/pkv.h declares;
+host-side argument checks answer with a status before any launch (no GPU is
+touched: every call here fails validation first)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from paged_kv_cache_459_b200 import build as pkv_build
+
+pkv_build.build()
+from paged_kv_cache_459_b200 import pkv  # noqa: E402
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation rejects first
+
+
+def test_header_symbols_are_exported():
+    names = pkv.declared_symbols()
+    assert len(names) >= 20 and "pkv_paged_kv_write" in names and "pkv_paged_attention_decode" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", pkv.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(pkv.lib(), n)
+    # nothing else of ours leaks out of the library
+    assert all(not s.startswith("_ZN3pkv") for s in exported)
+
+
+def test_status_strings_and_constants():
+    assert pkv.lib().pkv_block_tokens() == 16
+    assert pkv.status_string(0) == "ok"
+    assert pkv.status_string(pkv.ERR_WORKSPACE).startswith("workspace")
+    assert pkv.status_string(99) == "unknown status"
+    assert b"sm_100a" in pkv.lib().pkv_version()
+
+
+def decode(**kw):
+    args = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, tables=FAKE, W=8, lens=FAKE, B=2, Hq=4, Hkv=2,
+                D=128, NB=64, scale=0.1, variant=0, part=512, ws=None, wsb=0)
+    args.update(kw)
+    return pkv.lib().pkv_paged_attention_decode_ex(
+        args["out"], args["q"], args["kc"], args["vc"], args["tables"], args["W"], args["lens"],
+        args["B"], args["Hq"], args["Hkv"], args["D"], args["NB"], args["scale"], args["variant"],
+        args["part"], args["ws"], args["wsb"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), pkv.ERR_UNSUPPORTED),
+    (dict(D=256), pkv.ERR_UNSUPPORTED),
+    (dict(Hq=5, Hkv=2), pkv.ERR_INVALID_ARG),
+    (dict(Hkv=0), pkv.ERR_INVALID_ARG),
+    (dict(q=None), pkv.ERR_INVALID_ARG),
+    (dict(tables=None), pkv.ERR_INVALID_ARG),
+    (dict(out=FAKE + 2), pkv.ERR_INVALID_ARG),
+    (dict(kc=FAKE + 8), pkv.ERR_INVALID_ARG),
+    (dict(W=0), pkv.ERR_INVALID_ARG),
+    (dict(NB=0), pkv.ERR_INVALID_ARG),
+    (dict(B=-1), pkv.ERR_INVALID_ARG),
+    (dict(B=70000), pkv.ERR_INVALID_ARG),
+    (dict(scale=float("nan")), pkv.ERR_INVALID_ARG),
+    (dict(variant=7), pkv.ERR_INVALID_ARG),
+    (dict(part=40), pkv.ERR_INVALID_ARG),
+    (dict(NB=1 << 26, Hkv=2), pkv.ERR_UNSUPPORTED),
+    (dict(variant=2), pkv.ERR_WORKSPACE),
+    (dict(variant=2, ws=FAKE, wsb=16), pkv.ERR_WORKSPACE),
+])
+def test_decode_argument_checks(kw, code):
+    assert decode(**kw) == code
+
+
+def test_empty_batch_is_a_no_op():
+    assert decode(B=0, out=None, q=None) == pkv.OK
+
+
+def test_workspace_size():
+    # (B * Hq * parts) rows of (d + 2) floats, parts = ceil(W / (partition / 16))
+    assert pkv.decode_workspace_bytes(8, 32, 128, 2048, 512) == 8 * 32 * 64 * 130 * 4
+    assert pkv.decode_workspace_bytes(3, 4, 64, 33, 512) == 3 * 4 * 2 * 66 * 4
+    assert pkv.decode_workspace_bytes(3, 4, 64, 33, 24) == 0  # not a multiple of 16
+    assert pkv.decode_workspace_bytes(3, 0, 64, 33, 512) == 0
+
+
+@pytest.mark.parametrize("args,code", [
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 100, 64), pkv.ERR_INVALID_ARG),   # head_dim % 8
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 128, 64), pkv.ERR_INVALID_ARG),
+    ((None, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 64), pkv.ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE + 4, FAKE, FAKE, 4, 2, 128, 64), pkv.ERR_INVALID_ARG),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 0), pkv.ERR_INVALID_ARG),
+    ((None, None, None, None, None, 0, 2, 128, 64), pkv.OK),                # nothing to write
+])
+def test_write_argument_checks(args, code):
+    assert pkv.lib().pkv_paged_kv_write(*args, None, None) == code

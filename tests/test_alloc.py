@@ -1,0 +1,147 @@
+"""The C++ block allocator against the reference model (oracle/alloc_model.py):
+the pages' worked examples, random operation sequences compared step by step,
+all-or-nothing failures, and the tables of every decode workload."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle.alloc_model import AllocError as ModelError, BlockManager
+from paged_kv_cache_459_b200 import build as pkv_build
+from paged_kv_cache_459_b200 import workloads as wl
+
+pkv_build.build()
+from paged_kv_cache_459_b200.pkv import AllocError, BlockAllocator  # noqa: E402
+
+BT = 16
+
+
+def same_state(a: BlockAllocator, m: BlockManager, seq_ids):
+    assert a.free_blocks() == m.free_blocks()
+    assert [a.refcount(b) for b in range(m.num_blocks)] == m.ref
+    ids = sorted(seq_ids)
+    if ids:
+        w = max(1, max(len(m.tables[s]) for s in ids))
+        ta, la = a.export(ids, w)
+        tm, lm = m.export(ids, w)
+        assert np.array_equal(ta, tm) and np.array_equal(la, lm)
+    fa, ua, sa, xa = a.stats()
+    fm, um, sm, xm = m.stats()
+    assert (fa, ua, sa) == (fm, um, sm) and xa == pytest.approx(xm, abs=1e-12)
+
+
+def test_sharing_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "sharing_example.json")))
+    a = BlockAllocator(16, list(range(1, 16)) + [0])
+    a.add_seq(0, 64)
+    a.fork(0, 1, 48)
+    for _ in range(16):
+        a.append_token(1)
+    a.fork(0, 2, 32)
+    for _ in range(32):
+        a.append_token(2)
+    tables, _ = a.export([0, 1, 2], 4)
+    assert tables.tolist() == [g["printed"]["tables"][k] for k in "ABC"]
+    for blk, rc in g["expected_refcounts"].items():
+        assert a.refcount(int(blk)) == rc
+    a.free_seq(0)
+    for blk, rc in g["expected_after_freeing_A"]["refcounts"].items():
+        assert a.refcount(int(blk)) == rc
+    assert a.free_blocks()[-1] == 4
+
+
+def test_block_table_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "block_table_example.json")))
+    t = g["printed"]["request_A_block_table"]
+    order = [t["0"], t["1"], t["2"]] + [b for b in range(64) if b not in (t["0"], t["1"], t["2"])]
+    a = BlockAllocator(64, order)
+    a.add_seq(7, 0)
+    slots = [a.append_token(7) for _ in range(48)]
+    for tok, slot in g["expected_slot_by_token"].items():
+        assert slots[int(tok) - 1] == slot == a.slot_of(7, int(tok) - 1)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_operations_match_model(seed):
+    gen = np.random.default_rng(seed)
+    nb = int(gen.integers(8, 64))
+    order = gen.permutation(nb)
+    a, m = BlockAllocator(nb, order), BlockManager(nb, order)
+    live, next_id = [], 0
+    for step in range(400):
+        op = gen.choice(["add", "append", "appends", "fork", "free"], p=[.2, .35, .15, .15, .15])
+        args = ()
+        if op == "add":
+            args = (next_id, int(gen.integers(0, 70)))
+            next_id += 1
+        elif op in ("append", "free") and live:
+            args = (int(gen.choice(live)),)
+        elif op == "appends" and live:
+            k = int(gen.integers(1, len(live) + 1))
+            args = (list(gen.choice(live, size=k, replace=False)),)
+        elif op == "fork" and live:
+            p = int(gen.choice(live))
+            args = (p, next_id, int(gen.integers(-1, m.lens[p] + 2)))
+            next_id += 1
+        else:
+            continue
+        ra = rm = None
+        ea = em = None
+        try:
+            ra = {"add": a.add_seq, "append": a.append_token, "appends": a.append_tokens,
+                  "fork": a.fork, "free": a.free_seq}[op](*args)
+        except AllocError as e:
+            ea = e.kind
+        try:
+            rm = {"add": m.add_seq, "append": m.append_token, "appends": m.append_tokens,
+                  "fork": m.fork, "free": m.free_seq}[op](*args)
+        except ModelError as e:
+            em = e.kind
+        assert ea == em, (step, op, args, ea, em)
+        if ea is None:
+            if op in ("append", "appends"):
+                assert list(np.atleast_1d(ra)) == list(np.atleast_1d(rm))
+            if op in ("add", "fork"):
+                live.append(args[1] if op == "fork" else args[0])
+            if op == "free":
+                live.remove(args[0])
+        same_state(a, m, live)
+
+
+def test_failures_change_nothing():
+    a = BlockAllocator(4)
+    a.add_seq(0, 40)
+    before = (a.free_blocks(), [a.refcount(b) for b in range(4)], a.export([0], 3))
+    for call in (lambda: a.add_seq(1, 33), lambda: a.add_seq(0, 1), lambda: a.fork(0, 0),
+                 lambda: a.fork(5, 1), lambda: a.free_seq(9), lambda: a.fork(0, 1, 41),
+                 lambda: a.append_tokens([0, 0]), lambda: a.append_tokens([0, 3])):
+        with pytest.raises(AllocError):
+            call()
+        after = (a.free_blocks(), [a.refcount(b) for b in range(4)], a.export([0], 3))
+        assert after[0] == before[0] and after[1] == before[1]
+        assert np.array_equal(after[2][0], before[2][0])
+    a.fork(0, 1)
+    with pytest.raises(AllocError) as e:
+        a.append_token(1)
+    assert e.value.kind == "unsupported"
+    a.add_seq(2, 16)
+    with pytest.raises(AllocError) as e:
+        a.append_tokens([2])  # its block is full and the pool is empty
+    assert e.value.kind == "oom"
+    with pytest.raises(AllocError):
+        BlockAllocator(3, [0, 1, 1])
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("llama", {}), ("qwen", {}), ("prefix", {}),
+                                     ("long", {})])
+def test_workload_tables_match_model(name, kw):
+    w1 = wl.build(name, 0, BlockAllocator, with_cache=False, **kw)
+    w2 = wl.build(name, 0, BlockManager, with_cache=False, **kw)
+    assert np.array_equal(w1.block_tables, w2.block_tables)
+    assert np.array_equal(w1.slot_mapping, w2.slot_mapping)
+    assert np.array_equal(w1.lens, w2.lens)
+    assert w1.free_blocks.tolist() == w2.free_blocks.tolist()
+    if name == "prefix":
+        assert all(w1.alloc.refcount(int(b)) == w1.cfg["batch"] for b in w1.block_tables[0, :125])
+        assert w1.alloc.stats()[2] == 125

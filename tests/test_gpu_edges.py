@@ -1,0 +1,96 @@
+"""GPU edge cases: empty sequences, bad data caught on the device (flagged in
+the error word, skipped, never trapping), skipped and out-of-range slots."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import DeviceStep, bits_to_f64, build, check_close, host_bits
+
+pytestmark = pytest.mark.gpu
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from paged_kv_cache_459_b200 import pkv  # noqa: E402
+
+VARIANTS = [(pkv.DECODE_SINGLE, 512), (pkv.DECODE_SPLIT, 32)]
+
+
+@pytest.mark.parametrize("name", ["llama", "qwen"])
+def test_zero_length_sequence_gives_zero_row(name):
+    w = build(name, 5, batch=4, len_lo=1, len_hi=120, head_dim=64)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    lens = w.lens.copy()
+    lens[2] = 0
+    ref = oracle.paged_decode(w.q, kc, vc, w.block_tables, lens, w.cfg["scale"])
+    for v, part in VARIANTS:
+        out = d.decode(v, part, lens=torch.from_numpy(lens).cuda())
+        assert (out[2] == 0).all()
+        check_close(out, ref, f"zero-length, variant {v}")
+    assert d.err_word() == 0
+
+
+@pytest.mark.parametrize("name", ["llama", "qwen"])
+def test_bad_table_entry_is_flagged_and_skipped(name):
+    w = build(name, 6, batch=4, len_lo=40, len_hi=200)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    ref = oracle.paged_decode(w.q, kc, vc, w.block_tables, w.lens, w.cfg["scale"])
+    for bad in (w.num_blocks, w.num_blocks + 1000, -5, 2**31 - 1):
+        t = w.block_tables.copy()
+        t[1, 1] = bad
+        d.err.zero_()
+        for v, part in VARIANTS:
+            out = d.decode(v, part, tables=torch.from_numpy(t).cuda())
+            assert np.isfinite(bits_to_f64(out)).all()
+            keep = [0, 2, 3]
+            check_close(out[keep], ref[keep], f"rows beside a bad table entry, variant {v}")
+        assert d.err_word() & pkv.DEV_ERR_BAD_BLOCK
+
+
+def test_length_past_the_table_is_clamped_and_flagged():
+    w = build("llama", 7, batch=3, len_lo=20, len_hi=60, head_dim=64)
+    d = DeviceStep(w)
+    d.write()
+    lens = w.lens.copy()
+    lens[0] = w.block_tables.shape[1] * 16 + 5
+    lens[1] = -3
+    for v, part in VARIANTS:
+        d.err.zero_()
+        out = d.decode(v, part, lens=torch.from_numpy(lens).cuda())
+        assert d.err_word() & pkv.DEV_ERR_BAD_LEN
+        assert (out[1] == 0).all()
+
+
+def test_write_skips_negative_and_flags_out_of_range_slots():
+    w = build("qwen", 8, batch=5, len_lo=1, len_hi=50)
+    d = DeviceStep(w)
+    slots = w.slot_mapping.copy()
+    slots[1] = -1
+    slots[3] = w.num_blocks * 16 + 7
+    d.slots = torch.from_numpy(slots).cuda()
+    d.write()
+    assert d.err_word() & pkv.DEV_ERR_BAD_SLOT
+    s2 = slots.copy()
+    s2[3] = -1
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, s2)
+    assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
+
+
+def test_python_binding_rejects_bad_tensors():
+    w = build("tiny", 0)
+    d = DeviceStep(w)
+    with pytest.raises(TypeError):
+        pkv.paged_kv_write(d.k_new.float(), d.v_new, d.kc, d.vc, d.slots)
+    with pytest.raises(ValueError):
+        pkv.paged_kv_write(d.k_new.cpu(), d.v_new, d.kc, d.vc, d.slots)
+    with pytest.raises(ValueError):
+        pkv.paged_attention_decode(d.out, d.q, d.kc, d.vc, d.tables[:2], d.lens, 0.1, 4)
+    with pytest.raises(pkv.PkvError) as e:
+        pkv.paged_attention_decode(d.out[:, :, :48].contiguous(), d.q[:, :, :48].contiguous(),
+                                   d.kc[..., :48].contiguous(), d.vc[..., :48].contiguous(),
+                                   d.tables, d.lens, 0.1, 4)
+    assert e.value.code == pkv.ERR_UNSUPPORTED

@@ -1,0 +1,140 @@
+"""GPU parity: the CUDA write and decode kernels, called through the C ABI,
+against the fp64 oracle on the same seeded inputs.
+
+* write: the whole cache pool bit-exact against the oracle's write;
+* decode: every output element within |err| <= 1e-2 + 1e-2 |ref|, for the
+  single-pass and split-K variants, at sizes the oracle finishes in seconds
+  (several blocks per partition, ragged tails) and at the full workload sizes
+  on sampled sequences.
+Free blocks, slots past each sequence's end and the new token's slot hold bf16
+NaN before the write, so a stray read or a missed write shows up as NaN.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import DeviceStep, build, check_close, host_bits, oracle_after_write
+
+pytestmark = pytest.mark.gpu
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from paged_kv_cache_459_b200 import pkv  # noqa: E402
+from paged_kv_cache_459_b200 import workloads as wl  # noqa: E402
+
+SINGLE, SPLIT = pkv.DECODE_SINGLE, pkv.DECODE_SPLIT
+
+
+def test_tiny_end_to_end():
+    w = build("tiny", 0)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc, ref = oracle_after_write(w)
+    assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
+    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 16), (SPLIT, 32)):
+        out = d.decode(variant, part)
+        check_close(out, ref, f"tiny variant {variant} partition {part}")
+    assert d.err_word() == 0
+
+
+SMALL = [
+    ("tiny", {}),
+    ("llama", dict(batch=6, len_lo=1, len_hi=700)),
+    ("qwen", dict(batch=5, len_lo=1, len_hi=1300)),
+    ("prefix", dict(batch=4, prefix_len=512, suffix_lo=1, suffix_hi=90)),
+    ("long", dict(batch=2, len_fixed=2600, num_blocks=400)),
+    ("llama", dict(batch=5, head_dim=64, len_lo=1, len_hi=300)),
+    ("qwen", dict(batch=4, head_dim=64, len_lo=1, len_hi=500)),
+    ("qwen", dict(batch=3, num_heads=8, num_kv_heads=4, len_lo=1, len_hi=400)),   # group 2
+    ("qwen", dict(batch=3, num_heads=32, num_kv_heads=4, len_lo=1, len_hi=400)),  # group 8
+    ("qwen", dict(batch=3, num_heads=24, num_kv_heads=2, len_lo=1, len_hi=400)),  # group 12
+    ("qwen", dict(batch=2, num_heads=16, num_kv_heads=1, len_lo=1, len_hi=300, head_dim=64)),
+]
+
+
+@pytest.mark.parametrize("name,kw", SMALL, ids=[f"{n}-{i}" for i, (n, _) in enumerate(SMALL)])
+def test_parity_small(name, kw):
+    w = build(name, 1, **kw)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc, ref = oracle_after_write(w)
+    assert np.array_equal(host_bits(d.kc), kc), "write not bit-exact (K)"
+    assert np.array_equal(host_bits(d.vc), vc), "write not bit-exact (V)"
+    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 64), (pkv.DECODE_AUTO, 512)):
+        check_close(d.decode(variant, part), ref, f"{name} {kw} variant {variant}/{part}")
+    assert d.err_word() == 0
+
+
+FULL = ["llama", "qwen", "prefix", "long"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_parity_full_size_sampled(name):
+    w = build(name, 0)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
+    B = w.cfg["batch"]
+    sel = np.unique(np.concatenate([[0, B - 1], wl.rng(9).choice(B, size=min(B, 6), replace=False)]))
+    ref = oracle.paged_decode(w.q[sel], kc, vc, w.block_tables[sel], w.lens[sel], w.cfg["scale"])
+    for variant in (pkv.DECODE_AUTO, SINGLE, SPLIT):
+        out = d.decode(variant, 512)
+        check_close(out[sel], ref, f"{name} full, variant {variant}")
+        assert np.isfinite(wl.bf16_to_f32(out)).all()
+    assert d.err_word() == 0
+
+
+def test_len_one_is_v_exactly():
+    w = build("qwen", 2, batch=4, len_lo=1, len_hi=1)
+    d = DeviceStep(w)
+    d.write()
+    g = w.cfg["num_heads"] // w.cfg["num_kv_heads"]
+    for variant in (SINGLE, SPLIT):
+        out = d.decode(variant, 512)
+        assert np.array_equal(out, np.repeat(w.v_new, g, axis=1))
+    w = build("llama", 2, batch=3, len_lo=1, len_hi=1)
+    d = DeviceStep(w)
+    d.write()
+    assert np.array_equal(d.decode(SINGLE), w.v_new)
+
+
+def test_block_relabelling_is_bit_exact_on_gpu():
+    for name, kw in (("qwen", dict(batch=4, len_lo=20, len_hi=900)),
+                     ("llama", dict(batch=4, len_lo=20, len_hi=900))):
+        w = build(name, 3, **kw)
+        d = DeviceStep(w)
+        d.write()
+        outs = {v: d.decode(v, 128) for v in (SINGLE, SPLIT)}
+        perm = wl.rng(4).permutation(w.num_blocks)
+        t2, s2, kc2, vc2 = wl.permute_pool(perm, w.block_tables, w.slot_mapping,
+                                           host_bits(d.kc), host_bits(d.vc))
+        d2 = DeviceStep(w)
+        d2.kc.copy_(torch.from_numpy(kc2.view(np.int16)).view(torch.bfloat16))
+        d2.vc.copy_(torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16))
+        d2.tables = torch.from_numpy(t2).cuda()
+        for v in (SINGLE, SPLIT):
+            assert np.array_equal(d2.decode(v, 128), outs[v])
+
+
+def test_shared_prefix_matches_private_copy_on_gpu():
+    w = build("prefix", 4, batch=6, prefix_len=320, suffix_lo=1, suffix_hi=60)
+    d = DeviceStep(w)
+    d.write()
+    base = d.decode(SPLIT, 128)
+    nb, npre = w.num_blocks, 20
+    shared = w.block_tables[0, :npre]
+    assert (w.block_tables[:, :npre] == shared).all()
+    kc = host_bits(d.kc)
+    vc = host_bits(d.vc)
+    kc2 = np.concatenate([kc] + [kc[shared]] * 6)
+    vc2 = np.concatenate([vc] + [vc[shared]] * 6)
+    t2 = w.block_tables.copy()
+    for b in range(6):
+        t2[b, :npre] = nb + npre * b + np.arange(npre)
+    d2 = DeviceStep(w)
+    d2.kc = torch.from_numpy(kc2.view(np.int16)).view(torch.bfloat16).cuda()
+    d2.vc = torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16).cuda()
+    d2.tables = torch.from_numpy(t2).cuda()
+    assert np.array_equal(d2.decode(SPLIT, 128), base)

@@ -22,6 +22,11 @@ from paged_kv_cache_459_b200 import workloads as wl
 BT = 16
 
 
+def rb(shape, gen):
+    """Seeded bf16 N(0,1) bits, the seed drawn from `gen`."""
+    return wl.bf16_normal(shape, int(gen.integers(1 << 31)), 0)
+
+
 def f32(bits):
     return wl.bf16_to_f32(np.asarray(bits, dtype=np.uint16)).astype(np.float64)
 
@@ -33,8 +38,8 @@ def page_sequences(ks, vs, num_blocks, seed, lib=None):
     gen = wl.rng(seed)
     hkv, d = ks[0].shape[1], ks[0].shape[2]
     bm = BlockManager(num_blocks, gen.permutation(num_blocks))
-    kc = wl.bf16_normal((num_blocks, hkv, BT, d), gen)
-    vc = wl.bf16_normal((num_blocks, hkv, BT, d), gen)
+    kc = rb((num_blocks, hkv, BT, d), gen)
+    vc = rb((num_blocks, hkv, BT, d), gen)
     slots, krows, vrows = [], [], []
     for s, (k, v) in enumerate(zip(ks, vs)):
         bm.add_seq(s, 0)
@@ -63,9 +68,9 @@ def sdpa_reference(q_bits, ks, vs, scale):
 
 def random_case(seed, lens, hq, hkv, d):
     gen = wl.rng(seed)
-    ks = [wl.bf16_normal((n, hkv, d), gen) for n in lens]
-    vs = [wl.bf16_normal((n, hkv, d), gen) for n in lens]
-    q = wl.bf16_normal((len(lens), hq, d), gen)
+    ks = [rb((n, hkv, d), gen) for n in lens]
+    vs = [rb((n, hkv, d), gen) for n in lens]
+    q = rb((len(lens), hq, d), gen)
     return q, ks, vs
 
 
@@ -242,9 +247,9 @@ def test_two_keys_logistic_weights():
 def test_dominant_key_is_one_hot():
     d = 64
     gen = wl.rng(10)
-    q = wl.bf16_normal((1, 1, d), gen)
-    k = wl.bf16_normal((40, 1, d), gen)
-    v = wl.bf16_normal((40, 1, d), gen)
+    q = rb((1, 1, d), gen)
+    k = rb((40, 1, d), gen)
+    v = rb((40, 1, d), gen)
     # key 23 = 64 * q (exact in bf16: power-of-two multiple), so its score dominates by ~1e3
     k[23, 0] = (wl.bf16_to_f32(q[0, 0]) * 64).astype(np.float32).view(np.uint32) >> 16
     kc, vc, tables, lens = page_sequences([k], [v], 8, seed=6)
@@ -313,8 +318,8 @@ def test_partitioned_merge_equals_single_pass():
 
 def test_write_skips_negative_slots_and_rejects_bad_ones():
     gen = wl.rng(4)
-    kc = wl.bf16_normal((4, 2, BT, 8), gen)
-    k = wl.bf16_normal((3, 2, 8), gen)
+    kc = rb((4, 2, BT, 8), gen)
+    k = rb((3, 2, 8), gen)
     k2, _ = oracle.kv_write(kc, kc, k, k, np.array([-1, 5, -7]))
     diff = np.argwhere((k2 != kc).any(axis=-1))
     assert set(map(tuple, diff[:, [0, 2]])) <= {(0, 5)}
