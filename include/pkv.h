@@ -149,6 +149,39 @@ PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const
                                          size_t workspace_bytes, unsigned int *err_word,
                                          void *stream);
 
+/*
+ * Scratch-free split-K decode.  The pages have no counterpart to this call:
+ * it exists for callers that must not allocate device memory when they run
+ * decode -- e.g. an engine plugin whose execution path may not allocate, a
+ * server that reserves all of its memory at start-up, or code that must avoid
+ * cudaMalloc/cudaFree because those can synchronise the device.
+ *
+ * Same arguments and result as pkv_paged_attention_decode_ex with
+ * PKV_DECODE_SPLIT, minus the workspace: the split-K partials go to a
+ * PKV_STATIC_SCRATCH_BYTES (32 MiB) array inside the library, which every
+ * GPU that loads the library holds until the process exits.  The call itself
+ * allocates nothing.
+ *  - Sizes whose partials need more than PKV_STATIC_SCRATCH_BYTES (see
+ *    pkv_decode_workspace_bytes) are rejected with PKV_ERR_WORKSPACE.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, once per device, with that device current).
+ *    Make that first call before any stream capture begins.
+ *  - All calls share the one array and it keeps the last call's contents
+ *    (nothing in it needs clearing).  Calls that overlap on the GPU -- on
+ *    unordered streams, or from several host threads -- race on it and give
+ *    wrong results: order them.
+ */
+#define PKV_STATIC_SCRATCH_BYTES (32u << 20)
+PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, const void *k_cache,
+                                                     const void *v_cache,
+                                                     const int32_t *block_tables,
+                                                     int max_blocks_per_seq,
+                                                     const int32_t *seq_lens, int num_seqs,
+                                                     int num_heads, int num_kv_heads,
+                                                     int head_dim, int64_t num_blocks,
+                                                     float scale, int partition_tokens,
+                                                     unsigned int *err_word, void *stream);
+
 /* ------------------------------------------------------------------------
  * Host block allocator (section 二 and section 三 of the first page): a pool
  * of num_blocks physical blocks with reference counts, per-sequence block

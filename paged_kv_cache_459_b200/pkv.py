@@ -44,6 +44,8 @@ _sigs = {
                                     _f32, _P, _sz, _P, _P], _i32),
     "pkv_paged_attention_decode_ex": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
                                        _f32, _i32, _i32, _P, _sz, _P, _P], _i32),
+    "pkv_paged_attention_decode_static": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
+                                           _i64, _f32, _i32, _P, _P], _i32),
     "pkv_alloc_create": ([_i64, _P, _P], _i32),
     "pkv_alloc_destroy": ([_P], None),
     "pkv_alloc_add_seq": ([_P, _i64, _i64], _i32),
