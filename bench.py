@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
     ap.add_argument("--config", choices=sorted(WORKLOAD_NAMES), default="llama")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for ncu captures)")
     ap.add_argument("--variant", choices=["auto", "single", "split"], default="auto")
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -258,7 +260,7 @@ def run_gpu(args):
     from paged_kv_cache_459_b200 import pkv
     from paged_kv_cache_459_b200 import workloads as wl
 
-    w = wl.build(args.config, args.seed + rank, pkv.BlockAllocator)
+    w = wl.build(args.config, args.seed + rank, pkv.BlockAllocator, batch=args.batch)
     cfg = w.cfg
     B, hq, hkv, d = cfg["batch"], cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"]
 
@@ -281,7 +283,9 @@ def run_gpu(args):
     W = w.block_tables.shape[1]
     ws_bytes = pkv.decode_workspace_bytes(B, hq, d, W, args.partition)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    split = variant == pkv.DECODE_SPLIT or (variant == pkv.DECODE_AUTO and W > args.partition // 16)
+    split = variant == pkv.DECODE_SPLIT or (
+        variant == pkv.DECODE_AUTO and W > args.partition // 16
+        and B * hkv * ((hq // hkv + 7) // 8) < 4 * 3 * torch.cuda.get_device_properties(dev).multi_processor_count)
     scale = cfg["scale"]
 
     def write():

@@ -52,6 +52,15 @@ int env_int(const char *name, int fallback) {
     return (s && *s) ? std::atoi(s) : fallback;
 }
 
+// Streaming multiprocessors of the current device (148 on B200).
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
 int num_parts_for(int max_blocks_per_seq, int partition_tokens) {
     const int pb = partition_tokens / PKV_BLOCK_TOKENS;
     return (max_blocks_per_seq + pb - 1) / pb;
@@ -141,7 +150,11 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
     } else if (variant == PKV_DECODE_SINGLE) {
         split = false;
     } else {
-        split = max_blocks_per_seq > part_blocks && ws_ok;
+        // Split only when one pass would leave the GPU short of CTAs: fewer
+        // than ~4 waves of (sequence, KV head) units, with 3 CTAs per SM.
+        const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads *
+                              ((num_heads / num_kv_heads + 7) / 8);
+        split = max_blocks_per_seq > part_blocks && ws_ok && units < 4 * 3 * sm_count();
     }
 
     CUtensorMap tmk, tmv;
@@ -173,7 +186,7 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
         p.part_blocks = max_blocks_per_seq;
         p.num_parts = 1;
     }
-    pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 3)};
+    pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
     cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, split, t,
                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
