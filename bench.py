@@ -55,7 +55,7 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for ncu captures)")
-    ap.add_argument("--variant", choices=["auto", "single", "split"], default="auto")
+    ap.add_argument("--variant", choices=["auto", "single", "split", "stream"], default="auto")
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -278,14 +278,13 @@ def run_gpu(args):
     out = torch.empty_like(q)
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    variant = {"auto": pkv.DECODE_AUTO, "single": pkv.DECODE_SINGLE,
-               "split": pkv.DECODE_SPLIT}[args.variant]
+    variant = {"auto": pkv.DECODE_AUTO, "single": pkv.DECODE_SINGLE, "split": pkv.DECODE_SPLIT,
+               "stream": pkv.DECODE_STREAM}[args.variant]
     W = w.block_tables.shape[1]
-    ws_bytes = pkv.decode_workspace_bytes(B, hq, d, W, args.partition)
+    ws_bytes = pkv.decode_workspace_bytes_for(variant, B, hq, hkv, d, W, args.partition)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    split = variant == pkv.DECODE_SPLIT or (
-        variant == pkv.DECODE_AUTO and W > args.partition // 16
-        and B * hkv * ((hq // hkv + 7) // 8) < 4 * 3 * torch.cuda.get_device_properties(dev).multi_processor_count)
+    chosen = variant if variant != pkv.DECODE_AUTO else pkv.decode_variant_for(
+        B, hq, hkv, d, W, args.partition, ws.numel())
     scale = cfg["scale"]
 
     def write():
@@ -366,7 +365,7 @@ def run_gpu(args):
     achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
     value = B * K * world / (total_ms * 1e-3)
     e2e_value = B * K * world / (e2e_ms * 1e-3)
-    launches_per_step = 1 + 1 + (1 if split else 0)
+    launches_per_step = 2 + (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -375,8 +374,10 @@ def run_gpu(args):
             "workload": WORKLOAD_NAMES[args.config], "name": args.config, "batch": B,
             "num_heads": hq, "num_kv_heads": hkv, "head_dim": d, "block_tokens": 16,
             "tokens": ab["tokens"], "num_blocks": w.num_blocks, "table_width": W,
-            "variant": ("split-K %d-token partitions + merge" % args.partition) if split
-            else "single pass (one CTA per sequence x KV head)",
+            "variant": {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head)",
+                        pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % args.partition,
+                        pkv.DECODE_STREAM: "balanced stream-K (equal tile ranges per warp) + merge",
+                        }[chosen],
             "l2": f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), "
                   "no flush" if ab["kv"] > L2_BYTES else "inputs fit in L2",
             "parallelism": f"{world} independent replicas (batch per GPU fixed)",
@@ -387,7 +388,7 @@ def run_gpu(args):
         "kv_frac_of_measured_copy": achieved / peak,
         "write_us": write_ms * 1e3, "decode_us": decode_ms * 1e3,
         "roofline": {
-            "bound": "hbm", "kernel": "paged_attention_decode (decode kernel + split-K merge)",
+            "bound": "hbm", "kernel": "paged_attention_decode (decode kernel + merge kernel)",
             "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "peak_kind": peak_kind,
             "traffic": committed_traffic("paged_decode_kernel", args.config),

@@ -74,7 +74,9 @@ typedef enum {
 typedef enum {
     PKV_DECODE_AUTO = 0,   /* choose from the shapes (see pkv_paged_attention_decode) */
     PKV_DECODE_SINGLE = 1, /* one CTA per (sequence, KV head [, group of 8 query heads]) */
-    PKV_DECODE_SPLIT = 2   /* split-K token partitions + log-sum-exp merge kernel */
+    PKV_DECODE_SPLIT = 2,  /* split-K token partitions + log-sum-exp merge kernel */
+    PKV_DECODE_STREAM = 3  /* balanced: every warp of a persistent grid takes an equal share of
+                              all (sequence, head, block) tiles; cut segments merged by LSE */
 } pkv_decode_variant;
 
 /* Human-readable name of a pkv_status value (static storage). */
@@ -109,6 +111,25 @@ PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_
                                   int max_blocks_per_seq, int partition_tokens);
 
 /*
+ * Workspace (device bytes) that `variant` needs for these sizes on the
+ * current device (PKV_DECODE_AUTO: enough for any variant it may pick;
+ * PKV_DECODE_SINGLE: 0); 0 if a size is invalid.  partition_tokens <= 0
+ * means 512.
+ */
+PKV_API size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads,
+                                              int num_kv_heads, int head_dim,
+                                              int max_blocks_per_seq, int partition_tokens);
+
+/*
+ * The variant PKV_DECODE_AUTO picks for these sizes given `workspace_bytes`
+ * of workspace (PKV_DECODE_SINGLE, _SPLIT or _STREAM); -1 if a size is
+ * invalid.
+ */
+PKV_API int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                   int max_blocks_per_seq, int partition_tokens,
+                                   size_t workspace_bytes);
+
+/*
  * Single-query decode attention over the paged cache (section 三, step 三:
  * attention over all earlier K/V looked up through the block table), read as
  *   out[b][h][:] = softmax_p( scale * q[b][h] . K_b[p] ) V_b[p],  p in [0, seq_lens[b])
@@ -120,9 +141,12 @@ PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_
  *
  * head_dim: 64 or 128.  num_heads % num_kv_heads == 0.  Pointers 16-byte
  * aligned.  num_blocks * num_kv_heads * 16 must be < 2^31.
- * This entry point takes PKV_DECODE_AUTO with 512-token partitions: split-K
- * when a sequence may span more than one partition and `workspace` holds
- * pkv_decode_workspace_bytes(...) bytes, the single-pass variant otherwise.
+ * This entry point takes PKV_DECODE_AUTO with 512-token partitions: the
+ * balanced variant when `workspace` holds pkv_decode_workspace_bytes_for(
+ * PKV_DECODE_STREAM, ...) bytes and num_seqs <= 8192; else split-K when a
+ * sequence may span more than one partition, the GPU would otherwise be short
+ * of CTAs and `workspace` holds pkv_decode_workspace_bytes(...) bytes; else
+ * the single-pass variant.
  * The workspace is scratch owned by the caller; calls that share one
  * workspace must be ordered on the GPU (the same stream, or events).
  */
@@ -137,8 +161,8 @@ PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *q, const vo
 /*
  * As pkv_paged_attention_decode, with the variant and the split-K partition
  * length chosen by the caller.  partition_tokens: a multiple of 16 in
- * [16, 65536] (ignored by PKV_DECODE_SINGLE).  PKV_DECODE_SPLIT without enough
- * workspace returns PKV_ERR_WORKSPACE.
+ * [16, 65536] (used by PKV_DECODE_SPLIT only).  PKV_DECODE_SPLIT or
+ * PKV_DECODE_STREAM without enough workspace returns PKV_ERR_WORKSPACE.
  */
 PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,

@@ -34,6 +34,32 @@ struct DecodeTuning {
     int stages;  // TMA stages per warp (one K tile + one V tile each)
 };
 
+// Balanced (stream-K) decode: a persistent grid whose warps each take an
+// equal contiguous range of the flattened (sequence, head segment, block)
+// tile order; segments cut between warps are merged by a second kernel.
+constexpr int kStreamMaxCtasPerSm = 8;
+constexpr int kStreamWarps = 4;
+
+struct StreamParams {
+    __nv_bfloat16 *out;
+    const __nv_bfloat16 *q;
+    const int32_t *block_tables;
+    const int32_t *seq_lens;
+    int2 *ws_dir;     // [B * Y] (first worker, last worker) of each segment
+    float *ws_piece;  // [max_workers + B * Y][HP][D + 2]: o, then m[HP], then l[HP]
+    unsigned int *err;
+    long long num_blocks;
+    long long max_workers;  // piece slots reserved for workers
+    int W, B, Hq, Hkv;
+    int group, chunks;
+    int Y;   // head segments per sequence: Hkv (one query row per KV head) or Hkv * chunks
+    int HP;  // query heads per segment slot: 1, or min(8, group)
+    float scale_log2;
+};
+
+cudaError_t launch_decode_stream(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                 const StreamParams &p, int head_dim, cudaStream_t stream);
+
 // Launches the decode kernel (and the merge kernel when split) on `stream`.
 cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                           int head_dim, bool split, DecodeTuning tuning, cudaStream_t stream);

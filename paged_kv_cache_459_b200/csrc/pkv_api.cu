@@ -114,6 +114,72 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
     return rows * (static_cast<size_t>(head_dim) + 2) * sizeof(float);
 }
 
+namespace {
+
+struct StreamLayout {
+    int Y, HP;
+    long long max_workers;
+    size_t dir_bytes, piece_bytes;
+};
+
+StreamLayout stream_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim) {
+    StreamLayout l{};
+    const int group = num_heads / num_kv_heads;
+    const int chunks = (group + 7) / 8;
+    l.Y = group > 1 ? num_kv_heads * chunks : num_kv_heads;
+    l.HP = group > 1 ? (group < 8 ? group : 8) : 1;
+    l.max_workers = static_cast<long long>(sm_count()) * pkv::kStreamMaxCtasPerSm * pkv::kStreamWarps;
+    const size_t segs = static_cast<size_t>(num_seqs) * l.Y;
+    l.dir_bytes = (segs * 8 + 255) / 256 * 256;
+    l.piece_bytes = (static_cast<size_t>(l.max_workers) + segs) * l.HP *
+                    (static_cast<size_t>(head_dim) + 2) * sizeof(float);
+    return l;
+}
+
+}  // namespace
+
+size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_dim, int max_blocks_per_seq, int partition_tokens) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
+        head_dim <= 0 || max_blocks_per_seq <= 0)
+        return 0;
+    const size_t split = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                    max_blocks_per_seq, partition_tokens);
+    const StreamLayout l = stream_layout(num_seqs, num_heads, num_kv_heads, head_dim);
+    const size_t stream = l.dir_bytes + l.piece_bytes;
+    switch (variant) {
+        case PKV_DECODE_SINGLE: return 0;
+        case PKV_DECODE_SPLIT: return split;
+        case PKV_DECODE_STREAM: return stream;
+        case PKV_DECODE_AUTO: return split > stream ? split : stream;
+        default: return 0;
+    }
+}
+
+int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                           int max_blocks_per_seq, int partition_tokens, size_t workspace_bytes) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
+        head_dim <= 0 || max_blocks_per_seq <= 0)
+        return -1;
+    if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
+    if (partition_tokens % PKV_BLOCK_TOKENS) return -1;
+    const auto need = [&](int v) {
+        return pkv_decode_workspace_bytes_for(v, num_seqs, num_heads, num_kv_heads, head_dim,
+                                              max_blocks_per_seq, partition_tokens);
+    };
+    // The balanced variant keeps every SM's TMA rings full whatever the length
+    // mix; its length scan runs once per CTA, so very large batches skip it.
+    if (num_seqs <= 8192 && workspace_bytes >= need(PKV_DECODE_STREAM)) return PKV_DECODE_STREAM;
+    // Otherwise split only when one pass would leave the GPU short of CTAs:
+    // fewer than ~4 waves of (sequence, KV head) units at 3 CTAs per SM.
+    const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads *
+                          ((num_heads / num_kv_heads + 7) / 8);
+    if (max_blocks_per_seq > partition_tokens / PKV_BLOCK_TOKENS &&
+        workspace_bytes >= need(PKV_DECODE_SPLIT) && units < 4 * 3 * sm_count())
+        return PKV_DECODE_SPLIT;
+    return PKV_DECODE_SINGLE;
+}
+
 pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,
                                          int max_blocks_per_seq, const int32_t *seq_lens,
@@ -126,7 +192,7 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
         num_heads % num_kv_heads || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
         !std::isfinite(scale))
         return PKV_ERR_INVALID_ARG;
-    if (variant < PKV_DECODE_AUTO || variant > PKV_DECODE_SPLIT) return PKV_ERR_INVALID_ARG;
+    if (variant < PKV_DECODE_AUTO || variant > PKV_DECODE_STREAM) return PKV_ERR_INVALID_ARG;
     if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
     if (partition_tokens % PKV_BLOCK_TOKENS || partition_tokens > 65536) return PKV_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
@@ -140,27 +206,48 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
         return PKV_ERR_INVALID_ARG;
 
     const int part_blocks = partition_tokens / PKV_BLOCK_TOKENS;
-    const size_t need = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
-                                                   max_blocks_per_seq, partition_tokens);
-    const bool ws_ok = workspace != nullptr && workspace_bytes >= need && aligned16(workspace);
-    bool split;
-    if (variant == PKV_DECODE_SPLIT) {
-        if (!ws_ok) return PKV_ERR_WORKSPACE;
-        split = true;
-    } else if (variant == PKV_DECODE_SINGLE) {
-        split = false;
-    } else {
-        // Split only when one pass would leave the GPU short of CTAs: fewer
-        // than ~4 waves of (sequence, KV head) units, with 3 CTAs per SM.
-        const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads *
-                              ((num_heads / num_kv_heads + 7) / 8);
-        split = max_blocks_per_seq > part_blocks && ws_ok && units < 4 * 3 * sm_count();
-    }
+    const bool ws_aligned = workspace != nullptr && aligned16(workspace);
+    const size_t have = ws_aligned ? workspace_bytes : 0;
+    if (variant == PKV_DECODE_AUTO)
+        variant = pkv_decode_variant_for(num_seqs, num_heads, num_kv_heads, head_dim,
+                                         max_blocks_per_seq, partition_tokens, have);
+    if (variant != PKV_DECODE_SINGLE &&
+        have < pkv_decode_workspace_bytes_for(variant, num_seqs, num_heads, num_kv_heads, head_dim,
+                                              max_blocks_per_seq, partition_tokens))
+        return PKV_ERR_WORKSPACE;
+    const bool stream_k = variant == PKV_DECODE_STREAM;
+    const bool split = variant == PKV_DECODE_SPLIT;
+    const StreamLayout sl = stream_layout(num_seqs, num_heads, num_kv_heads, head_dim);
 
     CUtensorMap tmk, tmv;
     if (!encode_cache_map(&tmk, k_cache, rows, head_dim) ||
         !encode_cache_map(&tmv, v_cache, rows, head_dim))
         return PKV_ERR_CUDA;
+
+    if (stream_k) {
+        pkv::StreamParams sp{};
+        sp.out = static_cast<__nv_bfloat16 *>(out);
+        sp.q = static_cast<const __nv_bfloat16 *>(q);
+        sp.block_tables = block_tables;
+        sp.seq_lens = seq_lens;
+        sp.ws_dir = static_cast<int2 *>(workspace);
+        sp.ws_piece = reinterpret_cast<float *>(static_cast<char *>(workspace) + sl.dir_bytes);
+        sp.err = err_word;
+        sp.num_blocks = num_blocks;
+        sp.max_workers = sl.max_workers;
+        sp.W = max_blocks_per_seq;
+        sp.B = num_seqs;
+        sp.Hq = num_heads;
+        sp.Hkv = num_kv_heads;
+        sp.group = num_heads / num_kv_heads;
+        sp.chunks = (sp.group + 7) / 8;
+        sp.Y = sl.Y;
+        sp.HP = sl.HP;
+        sp.scale_log2 = scale * 1.4426950408889634f;
+        cudaError_t e = pkv::launch_decode_stream(tmk, tmv, sp, head_dim,
+                                                  static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    }
 
     pkv::DecodeParams p{};
     p.out = static_cast<__nv_bfloat16 *>(out);

@@ -29,7 +29,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_OOM, ERR_CUDA = range(6)
 DEV_ERR_BAD_SLOT, DEV_ERR_BAD_BLOCK, DEV_ERR_BAD_LEN, DEV_ERR_TIMEOUT = 1, 2, 4, 8
-DECODE_AUTO, DECODE_SINGLE, DECODE_SPLIT = 0, 1, 2
+DECODE_AUTO, DECODE_SINGLE, DECODE_SPLIT, DECODE_STREAM = 0, 1, 2, 3
 BLOCK_TOKENS = 16
 DEFAULT_PARTITION_TOKENS = 512
 
@@ -40,6 +40,8 @@ _sigs = {
     "pkv_version": ([], ctypes.c_char_p),
     "pkv_paged_kv_write": ([_P, _P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P], _i32),
     "pkv_decode_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
+    "pkv_decode_workspace_bytes_for": ([_i32, _i32, _i32, _i32, _i32, _i32, _i32], _sz),
+    "pkv_decode_variant_for": ([_i32, _i32, _i32, _i32, _i32, _i32, _sz], _i32),
     "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
                                     _f32, _P, _sz, _P, _P], _i32),
     "pkv_paged_attention_decode_ex": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
@@ -149,6 +151,20 @@ def decode_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_seq,
                                                partition_tokens))
 
 
+def decode_workspace_bytes_for(variant, num_seqs, num_heads, num_kv_heads, head_dim,
+                               max_blocks_per_seq,
+                               partition_tokens=DEFAULT_PARTITION_TOKENS) -> int:
+    return int(_lib.pkv_decode_workspace_bytes_for(variant, num_seqs, num_heads, num_kv_heads,
+                                                   head_dim, max_blocks_per_seq, partition_tokens))
+
+
+def decode_variant_for(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                       partition_tokens=DEFAULT_PARTITION_TOKENS, workspace_bytes=0) -> int:
+    """The variant the automatic choice takes for these sizes and workspace."""
+    return int(_lib.pkv_decode_variant_for(num_seqs, num_heads, num_kv_heads, head_dim,
+                                           max_blocks_per_seq, partition_tokens, workspace_bytes))
+
+
 def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, num_kv_heads,
                            *, variant: int = DECODE_AUTO,
                            partition_tokens: int = DEFAULT_PARTITION_TOKENS,
@@ -170,8 +186,9 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
     tp = _dev_tensor(block_tables, torch.int32, "block_tables")
     lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
     ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
-    need = decode_workspace_bytes(B, hq, d, W, partition_tokens) if W > 0 else 0
-    if workspace is None and variant != DECODE_SINGLE and need > 0:
+    need = decode_workspace_bytes_for(variant, B, hq, num_kv_heads, d, W, partition_tokens) \
+        if W > 0 and num_kv_heads > 0 and hq % num_kv_heads == 0 else 0
+    if workspace is None and need > 0:
         workspace = _workspace(q.device, need)
     wp = _dev_tensor(workspace, torch.uint8, "workspace") if workspace is not None else None
     wbytes = workspace.numel() if workspace is not None else 0

@@ -92,3 +92,23 @@ def test_workspace_size():
 ])
 def test_write_argument_checks(args, code):
     assert pkv.lib().pkv_paged_kv_write(*args, None, None) == code
+
+
+def test_variant_choice_and_workspace_sizes():
+    B, hq, hkv, d, W = 64, 32, 32, 128, 128
+    stream = pkv.decode_workspace_bytes_for(pkv.DECODE_STREAM, B, hq, hkv, d, W)
+    split = pkv.decode_workspace_bytes_for(pkv.DECODE_SPLIT, B, hq, hkv, d, W)
+    assert split == pkv.decode_workspace_bytes(B, hq, d, W)
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_AUTO, B, hq, hkv, d, W) == max(split, stream)
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_SINGLE, B, hq, hkv, d, W) == 0
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_STREAM, B, 28, 5, d, W) == 0  # 28 % 5
+    # no workspace: single pass; enough for the balanced variant: balanced
+    assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, 0) == pkv.DECODE_SINGLE
+    assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, stream) == pkv.DECODE_STREAM
+    # only split-K workspace: split when short of CTAs (8 x 8 units), single pass otherwise
+    long_split = pkv.decode_workspace_bytes(8, 32, d, 2048)
+    assert pkv.decode_variant_for(8, 32, 8, d, 2048, 512, long_split) in (pkv.DECODE_SPLIT,
+                                                                          pkv.DECODE_STREAM)
+    assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, min(split, stream - 1)) == pkv.DECODE_SINGLE
+    assert pkv.decode_variant_for(B, 5, 2, d, W, 512, 0) == -1
+    assert decode(variant=3) == pkv.ERR_WORKSPACE

@@ -23,7 +23,7 @@ if not torch.cuda.is_available():
 from paged_kv_cache_459_b200 import pkv  # noqa: E402
 from paged_kv_cache_459_b200 import workloads as wl  # noqa: E402
 
-SINGLE, SPLIT = pkv.DECODE_SINGLE, pkv.DECODE_SPLIT
+SINGLE, SPLIT, STREAM = pkv.DECODE_SINGLE, pkv.DECODE_SPLIT, pkv.DECODE_STREAM
 
 
 def test_tiny_end_to_end():
@@ -32,7 +32,7 @@ def test_tiny_end_to_end():
     d.write()
     kc, vc, ref = oracle_after_write(w)
     assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
-    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 16), (SPLIT, 32)):
+    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 16), (SPLIT, 32), (STREAM, 512)):
         out = d.decode(variant, part)
         check_close(out, ref, f"tiny variant {variant} partition {part}")
     assert d.err_word() == 0
@@ -61,7 +61,8 @@ def test_parity_small(name, kw):
     kc, vc, ref = oracle_after_write(w)
     assert np.array_equal(host_bits(d.kc), kc), "write not bit-exact (K)"
     assert np.array_equal(host_bits(d.vc), vc), "write not bit-exact (V)"
-    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 64), (pkv.DECODE_AUTO, 512)):
+    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 64), (STREAM, 512),
+                          (pkv.DECODE_AUTO, 512)):
         check_close(d.decode(variant, part), ref, f"{name} {kw} variant {variant}/{part}")
     assert d.err_word() == 0
 
@@ -79,7 +80,7 @@ def test_parity_full_size_sampled(name):
     B = w.cfg["batch"]
     sel = np.unique(np.concatenate([[0, B - 1], wl.rng(9).choice(B, size=min(B, 6), replace=False)]))
     ref = oracle.paged_decode(w.q[sel], kc, vc, w.block_tables[sel], w.lens[sel], w.cfg["scale"])
-    for variant in (pkv.DECODE_AUTO, SINGLE, SPLIT):
+    for variant in (pkv.DECODE_AUTO, SINGLE, SPLIT, STREAM):
         out = d.decode(variant, 512)
         check_close(out[sel], ref, f"{name} full, variant {variant}")
         assert np.isfinite(wl.bf16_to_f32(out)).all()
@@ -91,13 +92,14 @@ def test_len_one_is_v_exactly():
     d = DeviceStep(w)
     d.write()
     g = w.cfg["num_heads"] // w.cfg["num_kv_heads"]
-    for variant in (SINGLE, SPLIT):
+    for variant in (SINGLE, SPLIT, STREAM):
         out = d.decode(variant, 512)
         assert np.array_equal(out, np.repeat(w.v_new, g, axis=1))
     w = build("llama", 2, batch=3, len_lo=1, len_hi=1)
     d = DeviceStep(w)
     d.write()
     assert np.array_equal(d.decode(SINGLE), w.v_new)
+    assert np.array_equal(d.decode(STREAM), w.v_new)
 
 
 def test_block_relabelling_is_bit_exact_on_gpu():
@@ -106,7 +108,7 @@ def test_block_relabelling_is_bit_exact_on_gpu():
         w = build(name, 3, **kw)
         d = DeviceStep(w)
         d.write()
-        outs = {v: d.decode(v, 128) for v in (SINGLE, SPLIT)}
+        outs = {v: d.decode(v, 128) for v in (SINGLE, SPLIT, STREAM)}
         perm = wl.rng(4).permutation(w.num_blocks)
         t2, s2, kc2, vc2 = wl.permute_pool(perm, w.block_tables, w.slot_mapping,
                                            host_bits(d.kc), host_bits(d.vc))
@@ -114,7 +116,7 @@ def test_block_relabelling_is_bit_exact_on_gpu():
         d2.kc.copy_(torch.from_numpy(kc2.view(np.int16)).view(torch.bfloat16))
         d2.vc.copy_(torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16))
         d2.tables = torch.from_numpy(t2).cuda()
-        for v in (SINGLE, SPLIT):
+        for v in (SINGLE, SPLIT, STREAM):
             assert np.array_equal(d2.decode(v, 128), outs[v])
 
 
@@ -138,3 +140,23 @@ def test_shared_prefix_matches_private_copy_on_gpu():
     d2.vc = torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16).cuda()
     d2.tables = torch.from_numpy(t2).cuda()
     assert np.array_equal(d2.decode(SPLIT, 128), base)
+    assert np.array_equal(d2.decode(STREAM), d.decode(STREAM))
+
+
+STREAM_SHAPES = [
+    ("llama", dict(batch=200, len_lo=1, len_hi=40, head_dim=64)),   # many short segments per worker
+    ("long", dict(batch=1, len_fixed=32768)),                       # segments cut across ~200 workers
+    ("qwen", dict(batch=1, len_lo=1, len_hi=1)),                    # fewer tiles than workers
+    ("qwen", dict(batch=300, len_lo=1, len_hi=300, num_heads=24, num_kv_heads=2)),  # 12-head groups
+]
+
+
+@pytest.mark.parametrize("name,kw", STREAM_SHAPES, ids=[f"{n}-{i}" for i, (n, _) in enumerate(STREAM_SHAPES)])
+def test_stream_variant_shapes(name, kw):
+    w = build(name, 11, **kw)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc, ref = oracle_after_write(w)
+    out = d.decode(STREAM)
+    check_close(out, ref, f"stream {name} {kw}")
+    assert d.err_word() == 0
