@@ -141,12 +141,10 @@ PKV_API int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads
  *
  * head_dim: 64 or 128.  num_heads % num_kv_heads == 0.  Pointers 16-byte
  * aligned.  num_blocks * num_kv_heads * 16 must be < 2^31.
- * This entry point takes PKV_DECODE_AUTO with 512-token partitions: the
- * balanced variant when `workspace` holds pkv_decode_workspace_bytes_for(
- * PKV_DECODE_STREAM, ...) bytes and num_seqs <= 8192; else split-K when a
- * sequence may span more than one partition, the GPU would otherwise be short
- * of CTAs and `workspace` holds pkv_decode_workspace_bytes(...) bytes; else
- * the single-pass variant.
+ * This entry point takes PKV_DECODE_AUTO with 512-token partitions: split-K
+ * when a sequence may span more than one partition, the single-pass grid
+ * would be short of CTAs (fewer than ~4 waves) and `workspace` holds
+ * pkv_decode_workspace_bytes(...) bytes; the single-pass variant otherwise.
  * The workspace is scratch owned by the caller; calls that share one
  * workspace must be ordered on the GPU (the same stream, or events).
  */

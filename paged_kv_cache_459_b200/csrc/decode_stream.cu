@@ -70,10 +70,13 @@ struct RowWindow {
     __device__ __forceinline__ int32_t get(int j) const { return __shfl_sync(0xffffffffu, cur, j & 31); }
 };
 
-// Position of the producer in the flattened tile order.
+// Position of the producer in the flattened tile order, with the constants
+// of the segment it is in (computed once per segment).
 struct Cursor {
     int b, y, j, nblk, len;
     long long seq_f;  // flattened index of tile (b, 0, 0)
+    int seg_flags;    // kFlagWhole / kFlagDir for this worker's piece of the segment
+    int w_hi;         // worker holding the segment's last tile
 };
 
 template <int D, int NW, int S, bool MMA>
@@ -132,6 +135,7 @@ __global__ void __launch_bounds__(NW * 32)
         __syncthreads();
     }
     const long long T = s_pref[NW * 32];
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.ws_total = T;
     const long long f0 = w * T / G, f1 = (w + 1) * T / G;
     if (f0 >= f1) return;
     const int ntiles = static_cast<int>(f1 - f0);
@@ -166,6 +170,13 @@ __global__ void __launch_bounds__(NW * 32)
         cu.y = static_cast<int>(off / cu.nblk);
         cu.j = static_cast<int>(off % cu.nblk);
     }
+    auto enter_segment = [&]() {
+        const long long F0 = cu.seq_f + static_cast<long long>(cu.y) * cu.nblk;
+        const long long F1 = F0 + cu.nblk;
+        cu.seg_flags = (F0 >= f0 && F1 <= f1 ? kFlagWhole : 0) | (F0 >= f0 ? kFlagDir : 0);
+        cu.w_hi = static_cast<int>((G * F1 - 1) / T);  // owner of tile F1 - 1
+    };
+    enter_segment();
     RowWindow win;
     win.reset(p.block_tables + static_cast<size_t>(cu.b) * p.W, cu.nblk, cu.j, lane);
     const uint64_t policy = l2_policy_evict_first();
@@ -173,16 +184,11 @@ __global__ void __launch_bounds__(NW * 32)
     // Issues tile k (the cursor's position) into stage k % S and steps the cursor.
     auto issue = [&](int k) {
         const int32_t phys = win.get(cu.j);
-        const long long f = f0 + k;
-        const long long F0 = cu.seq_f + static_cast<long long>(cu.y) * cu.nblk;
-        const long long F1 = F0 + cu.nblk;
         const int seg = cu.b * Y + cu.y;
-        int flags = min(kBlockTokens, cu.len - cu.j * kBlockTokens);
+        int flags = min(kBlockTokens, cu.len - cu.j * kBlockTokens) | cu.seg_flags;
         if (k == 0 || cu.j == 0) flags |= kFlagFirst;
-        if (f == f1 - 1 || cu.j == cu.nblk - 1) flags |= kFlagLast;
-        if (F0 >= f0 && F1 <= f1) flags |= kFlagWhole;
-        if (F0 >= f0) flags |= kFlagDir;
-        const int w_hi = static_cast<int>((G * F1 - 1) / T);  // worker of tile F1 - 1
+        if (k == ntiles - 1 || cu.j == cu.nblk - 1) flags |= kFlagLast;
+        const int w_hi = cu.w_hi;
         const bool ok = phys >= 0 && phys < p.num_blocks;
         const int s = k % S;
         if (lane == 0) {
@@ -218,6 +224,7 @@ __global__ void __launch_bounds__(NW * 32)
                 cu.nblk = (cu.len + kBlockTokens - 1) / kBlockTokens;
             } while (cu.nblk == 0);
         }
+        enter_segment();
         win.reset(p.block_tables + static_cast<size_t>(cu.b) * p.W, cu.nblk, 0, lane);
     };
 
@@ -333,15 +340,20 @@ __global__ void __launch_bounds__(D) stream_merge_kernel(const StreamParams p) {
     }
     const int2 dir = p.ws_dir[seg];
     if (dir.x == dir.y) return;  // finished by its only worker
+    // With fewer tiles than workers some workers own no tile; they left no piece.
+    const long long T = *p.ws_total, G = p.num_workers;
+    const auto has_tiles = [&](int w) { return (w + 1) * T / G > w * T / G; };
     for (int n = 0; n < heads; ++n) {
         float M = -INFINITY;
         for (int w = dir.x; w <= dir.y; ++w) {
+            if (!has_tiles(w)) continue;
             const float *pc = p.ws_piece + static_cast<size_t>(w + seg) * p.HP * (D + 2);
             M = fmaxf(M, pc[p.HP * D + n]);
         }
         float L = 0.f, O = 0.f;
         if (M != -INFINITY) {
             for (int w = dir.x; w <= dir.y; ++w) {
+                if (!has_tiles(w)) continue;
                 const float *pc = p.ws_piece + static_cast<size_t>(w + seg) * p.HP * (D + 2);
                 const float c = exp2f(pc[p.HP * D + n] - M);
                 L = fmaf(pc[p.HP * D + p.HP + n], c, L);
@@ -368,6 +380,7 @@ cudaError_t launch_stream_one(const CUtensorMap &tmk, const CUtensorMap &tmv, St
     per_sm = max(1, min(per_sm, kStreamMaxCtasPerSm));
     const int grid = sms * per_sm;
     if (static_cast<long long>(grid) * NW > p.max_workers) return cudaErrorInvalidValue;
+    p.num_workers = static_cast<long long>(grid) * NW;
     kern<<<grid, NW * 32, kSmem, stream>>>(tmk, tmv, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     stream_merge_kernel<D><<<p.B * p.Y, D, 0, stream>>>(p);

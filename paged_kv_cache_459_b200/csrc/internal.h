@@ -45,11 +45,13 @@ struct StreamParams {
     const __nv_bfloat16 *q;
     const int32_t *block_tables;
     const int32_t *seq_lens;
+    long long *ws_total;  // total tiles of the launch (read by the merge kernel)
     int2 *ws_dir;     // [B * Y] (first worker, last worker) of each segment
     float *ws_piece;  // [max_workers + B * Y][HP][D + 2]: o, then m[HP], then l[HP]
     unsigned int *err;
     long long num_blocks;
     long long max_workers;  // piece slots reserved for workers
+    long long num_workers;  // warps of the launched grid
     int W, B, Hq, Hkv;
     int group, chunks;
     int Y;   // head segments per sequence: Hkv (one query row per KV head) or Hkv * chunks

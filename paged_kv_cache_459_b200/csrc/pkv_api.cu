@@ -130,7 +130,7 @@ StreamLayout stream_layout(int num_seqs, int num_heads, int num_kv_heads, int he
     l.HP = group > 1 ? (group < 8 ? group : 8) : 1;
     l.max_workers = static_cast<long long>(sm_count()) * pkv::kStreamMaxCtasPerSm * pkv::kStreamWarps;
     const size_t segs = static_cast<size_t>(num_seqs) * l.Y;
-    l.dir_bytes = (segs * 8 + 255) / 256 * 256;
+    l.dir_bytes = (256 + segs * 8 + 255) / 256 * 256;  // total-tile word, then the directory
     l.piece_bytes = (static_cast<size_t>(l.max_workers) + segs) * l.HP *
                     (static_cast<size_t>(head_dim) + 2) * sizeof(float);
     return l;
@@ -167,11 +167,10 @@ int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads, int he
         return pkv_decode_workspace_bytes_for(v, num_seqs, num_heads, num_kv_heads, head_dim,
                                               max_blocks_per_seq, partition_tokens);
     };
-    // The balanced variant keeps every SM's TMA rings full whatever the length
-    // mix; its length scan runs once per CTA, so very large batches skip it.
-    if (num_seqs <= 8192 && workspace_bytes >= need(PKV_DECODE_STREAM)) return PKV_DECODE_STREAM;
-    // Otherwise split only when one pass would leave the GPU short of CTAs:
-    // fewer than ~4 waves of (sequence, KV head) units at 3 CTAs per SM.
+    // Split only when one pass would leave the GPU short of CTAs: fewer than
+    // ~4 waves of (sequence, KV head) units at 3 CTAs per SM.  (The balanced
+    // variant measured slower than both on every workload tried, so it is
+    // only used when asked for.)
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads *
                           ((num_heads / num_kv_heads + 7) / 8);
     if (max_blocks_per_seq > partition_tokens / PKV_BLOCK_TOKENS &&
@@ -230,7 +229,8 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
         sp.q = static_cast<const __nv_bfloat16 *>(q);
         sp.block_tables = block_tables;
         sp.seq_lens = seq_lens;
-        sp.ws_dir = static_cast<int2 *>(workspace);
+        sp.ws_total = static_cast<long long *>(workspace);
+        sp.ws_dir = reinterpret_cast<int2 *>(static_cast<char *>(workspace) + 256);
         sp.ws_piece = reinterpret_cast<float *>(static_cast<char *>(workspace) + sl.dir_bytes);
         sp.err = err_word;
         sp.num_blocks = num_blocks;

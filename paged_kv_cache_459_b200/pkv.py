@@ -224,12 +224,13 @@ class BlockAllocator:
         _acheck(_lib.pkv_alloc_create(int(num_blocks), order.ctypes.data if order is not None
                                       else None, ctypes.byref(h)), "pkv_alloc_create")
         self._h = h
+        self._destroy = _lib.pkv_alloc_destroy  # kept: module globals may be gone at exit
         self.num_blocks = int(num_blocks)
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            _lib.pkv_alloc_destroy(h)
+            self._destroy(h)
             self._h = None
 
     def add_seq(self, seq_id: int, num_tokens: int) -> None:
