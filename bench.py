@@ -57,6 +57,8 @@ def parse_args():
                     help="override the workload's batch (smaller cases for ncu captures)")
     ap.add_argument("--variant", choices=["auto", "single", "split", "stream"], default="auto")
     ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--cascade", action="store_true",
+                    help="shared-prefix decode: prefix blocks read once per group and KV head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU time budget of the oracle baseline sample")
@@ -285,14 +287,24 @@ def run_gpu(args):
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     chosen = variant if variant != pkv.DECODE_AUTO else pkv.decode_variant_for(
         B, hq, hkv, d, W, args.partition, ws.numel())
+    if args.cascade:
+        pb_h, offs_h, mem_h = w.alloc.prefix_groups(list(range(B)))
+        pb, offs, mem = (torch.from_numpy(x).to(dev) for x in (pb_h, offs_h, mem_h))
+        ws = torch.empty(pkv.decode_prefix_workspace_bytes(B, hq, d, W, args.partition),
+                         dtype=torch.uint8, device=dev)
     scale = cfg["scale"]
 
     def write():
         pkv.paged_kv_write(k_new, v_new, kc, vc, slots, err=err)
 
     def decode():
-        pkv.paged_attention_decode(out, q, kc, vc, tables, lens, scale, hkv, variant=variant,
-                                   partition_tokens=args.partition, workspace=ws, err=err)
+        if args.cascade:
+            pkv.paged_attention_decode_prefix(out, q, kc, vc, tables, lens, scale, hkv, pb, offs, mem,
+                                              partition_tokens=args.partition, workspace=ws,
+                                              err=err)
+        else:
+            pkv.paged_attention_decode(out, q, kc, vc, tables, lens, scale, hkv, variant=variant,
+                                       partition_tokens=args.partition, workspace=ws, err=err)
 
     stream = torch.cuda.current_stream(dev)
     K, Wm = args.steps, args.warmup
@@ -362,10 +374,17 @@ def run_gpu(args):
     ab = algorithmic_bytes(w)
     peak, peak_kind = measured_peak_hbm()
     dec_bytes = ab["kv"] + ab["q"]
+    if args.cascade:
+        # what the cascade must read: each group's prefix once, every suffix once
+        unique_tokens = int((np.asarray(w.lens, np.int64) - 16 * pb_h.astype(np.int64)).sum())
+        unique_tokens += sum(16 * int(pb_h[mem_h[offs_h[g]]]) for g in range(len(offs_h) - 1))
+        dec_bytes = unique_tokens * hkv * d * 2 * 2 + ab["q"]
     achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
     value = B * K * world / (total_ms * 1e-3)
     e2e_value = B * K * world / (e2e_ms * 1e-3)
     launches_per_step = 2 + (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) else 0)
+    if args.cascade:
+        launches_per_step = 1 + 3  # write; prefix chunks, suffix split-K, merge
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -377,7 +396,9 @@ def run_gpu(args):
             "variant": {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head)",
                         pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % args.partition,
                         pkv.DECODE_STREAM: "balanced stream-K (equal tile ranges per warp) + merge",
-                        }[chosen],
+                        }[chosen] if not args.cascade else
+            "shared-prefix cascade (prefix once per group x KV head, split-K suffixes, merge)",
+            "logical_kv_bytes": ab["kv"],
             "l2": f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), "
                   "no flush" if ab["kv"] > L2_BYTES else "inputs fit in L2",
             "parallelism": f"{world} independent replicas (batch per GPU fixed)",

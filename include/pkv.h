@@ -204,6 +204,36 @@ PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, c
                                                      float scale, int partition_tokens,
                                                      unsigned int *err_word, void *stream);
 
+/*
+ * Shared-prefix ("cascade") decode -- the sharing of "vLLM 與 PagedAttention：
+ * 高吞吐推理的關鍵", section 二 (無法共享: the tables of requests with a common
+ * prefix point at the same physical blocks) used to cut reads: the shared
+ * blocks are read once per (group, KV head) instead of once per sequence.
+ * Same result as pkv_paged_attention_decode (up to fp32 rounding order).
+ *
+ * Groups are given in CSR form: the members of group g are the sequence
+ * indices group_seqs[group_offsets[g] .. group_offsets[g+1]).  Every member b
+ * of a group has prefix_blocks[b] = the number of leading blocks all members'
+ * tables share (full blocks, identical entries); sequences in no group have
+ * prefix_blocks[b] = 0.  The group's shared block ids are read from its first
+ * member's table row.  pkv_alloc_prefix_groups builds all three arrays from
+ * the allocator's state.  All five arrays are device int32.
+ * Work: a tensor-core kernel computes each group's prefix attention in
+ * chunks of 8 blocks (queries of all members x heads as MMA rows); the
+ * split-K kernel (partition_tokens, <= 0: 512) covers each sequence past its
+ * prefix; a merge kernel combines the partials.  Workspace:
+ * pkv_decode_prefix_workspace_bytes(...), else PKV_ERR_WORKSPACE.
+ */
+PKV_API size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                                 int max_blocks_per_seq, int partition_tokens);
+PKV_API pkv_status pkv_paged_attention_decode_prefix(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+    int num_heads, int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
+    const int32_t *prefix_blocks, const int32_t *group_offsets, const int32_t *group_seqs,
+    int num_groups, int partition_tokens, void *workspace, size_t workspace_bytes,
+    unsigned int *err_word, void *stream);
+
 /* ------------------------------------------------------------------------
  * Host block allocator (section 二 and section 三 of the first page): a pool
  * of num_blocks physical blocks with reference counts, per-sequence block
@@ -253,6 +283,16 @@ PKV_API pkv_status pkv_alloc_stats(const pkv_alloc *a, int64_t *free_blocks, int
 /* The free list, front first: up to cap ids into out, the count into *n_out. */
 PKV_API pkv_status pkv_alloc_free_list(const pkv_alloc *a, int64_t *out, int64_t cap, int64_t *n_out);
 
+/* Shared-prefix groups among the listed sequences (for
+ * pkv_paged_attention_decode_prefix): sequences whose first block is full and
+ * held by several tables are grouped by that block (groups in order of first
+ * appearance, members in list order); a group's prefix is the longest run of
+ * leading blocks identical in, and full for, every member.  Outputs (host):
+ * prefix_blocks_out [n] (0 outside groups), group_offsets_out [n + 1] (CSR,
+ * first *num_groups_out + 1 used), group_seqs_out [n] (indices into seq_ids). */
+PKV_API pkv_status pkv_alloc_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, int n,
+                                           int32_t *prefix_blocks_out, int32_t *group_offsets_out,
+                                           int32_t *group_seqs_out, int32_t *num_groups_out);
 PKV_API pkv_status pkv_alloc_refcount(const pkv_alloc *a, int64_t block, int32_t *out);
 PKV_API pkv_status pkv_alloc_seq_len(const pkv_alloc *a, int64_t seq_id, int64_t *len_out);
 PKV_API pkv_status pkv_alloc_slot_of(const pkv_alloc *a, int64_t seq_id, int64_t pos, int64_t *slot_out);

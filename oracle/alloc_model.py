@@ -139,6 +139,37 @@ class BlockManager:
             raise AllocError("invalid", "position outside the sequence")
         return self.tables[seq_id][pos // BLOCK_TOKENS] * BLOCK_TOKENS + pos % BLOCK_TOKENS
 
+    def prefix_groups(self, seq_ids):
+        """Sequences sharing leading blocks: those whose first block is full and
+        held by several tables, grouped by it (first-appearance order); the
+        group's prefix is the longest run of leading blocks identical in, and
+        full for, every member.  Returns (prefix_blocks, offsets, members) with
+        members given as indices into seq_ids."""
+        import numpy as np
+
+        ids = list(seq_ids)
+        by_first: dict[int, list[int]] = {}
+        for i, s in enumerate(ids):
+            if self.lens[s] >= BLOCK_TOKENS and self.ref[self.tables[s][0]] >= 2:
+                by_first.setdefault(self.tables[s][0], []).append(i)
+        pb = np.zeros(len(ids), np.int32)
+        offs, members = [0], []
+        for grp in by_first.values():
+            if len(grp) < 2:
+                continue
+            common = min(self.lens[ids[i]] // BLOCK_TOKENS for i in grp)
+            t0 = self.tables[ids[grp[0]]]
+            k = 0
+            while k < common and all(self.tables[ids[i]][k] == t0[k] for i in grp):
+                k += 1
+            if k == 0:
+                continue
+            for i in grp:
+                pb[i] = k
+                members.append(i)
+            offs.append(len(members))
+        return pb, np.array(offs, np.int32), np.array(members, np.int32)
+
     def refcount(self, block: int) -> int:
         return self.ref[block]
 

@@ -246,6 +246,57 @@ pkv_status pkv_alloc_free_list(const pkv_alloc *a, int64_t *out, int64_t cap, in
     return PKV_OK;
 }
 
+pkv_status pkv_alloc_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, int n,
+                                   int32_t *prefix_blocks_out, int32_t *group_offsets_out,
+                                   int32_t *group_seqs_out, int32_t *num_groups_out) {
+    if (!a || n < 0 || !num_groups_out ||
+        (n > 0 && (!seq_ids || !prefix_blocks_out || !group_offsets_out || !group_seqs_out)))
+        return PKV_ERR_INVALID_ARG;
+    std::vector<const Sequence *> seqs(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i) {
+        auto it = a->seqs.find(seq_ids[i]);
+        if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+        seqs[i] = &it->second;
+    }
+    // Candidates: sequences whose first block is full and held by several tables,
+    // grouped by that block in order of first appearance.
+    std::vector<int> order;  // distinct first blocks, first appearance order
+    std::unordered_map<int32_t, std::vector<int>> by_first;
+    for (int i = 0; i < n; ++i) {
+        const Sequence &s = *seqs[i];
+        if (s.len < kBlockTokens || a->refcount[s.blocks[0]] < 2) continue;
+        auto &v = by_first[s.blocks[0]];
+        if (v.empty()) order.push_back(s.blocks[0]);
+        v.push_back(i);
+    }
+    std::fill(prefix_blocks_out, prefix_blocks_out + n, 0);
+    int32_t groups = 0, pos = 0;
+    group_offsets_out[0] = 0;
+    for (int32_t blk : order) {
+        const std::vector<int> &members = by_first[blk];
+        if (members.size() < 2) continue;
+        // longest run of identical leading blocks that is full in every member
+        int64_t common = INT64_MAX;
+        for (int i : members) common = std::min<int64_t>(common, seqs[i]->len / kBlockTokens);
+        const Sequence &s0 = *seqs[members[0]];
+        int64_t k = 0;
+        while (k < common) {
+            bool same = true;
+            for (int i : members) same = same && seqs[i]->blocks[k] == s0.blocks[k];
+            if (!same) break;
+            ++k;
+        }
+        if (k == 0) continue;
+        for (int i : members) {
+            prefix_blocks_out[i] = static_cast<int32_t>(k);
+            group_seqs_out[pos++] = i;
+        }
+        group_offsets_out[++groups] = pos;
+    }
+    *num_groups_out = groups;
+    return PKV_OK;
+}
+
 pkv_status pkv_alloc_refcount(const pkv_alloc *a, int64_t block, int32_t *out) {
     if (!a || !out || block < 0 || block >= a->num_blocks) return PKV_ERR_INVALID_ARG;
     *out = a->refcount[static_cast<size_t>(block)];

@@ -61,8 +61,10 @@ __global__ void __launch_bounds__(NW * 32)
         len = len < 0 ? 0 : p.W * kBlockTokens;
     }
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
-    const int blk_begin = part * p.part_blocks;
-    const int blk_end = min(nblk, blk_begin + p.part_blocks);
+    int start = 0;
+    if (p.start_blocks != nullptr) start = min(max(__ldg(p.start_blocks + b), 0), len / kBlockTokens);
+    const int blk_begin = max(part * p.part_blocks, start);
+    const int blk_end = min(nblk, (part + 1) * p.part_blocks);
     if (blk_begin >= blk_end) {
         // Nothing to read.  Single pass: the (empty) sequence's rows are zero.
         // Split-K: the merge kernel only reads partitions that hold tokens.
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(NW * 32)
         }
         const size_t row = static_cast<size_t>(b) * p.Hq + h0 + n;
         if constexpr (SPLIT) {
-            const size_t pr = row * p.num_parts + part;
+            const size_t pr = row * p.ws_parts + p.ws_part0 + part;
             p.ws_o[pr * D + e] = O;
             if (e == 0) {
                 p.ws_ml[2 * pr] = M;
@@ -206,8 +208,8 @@ __global__ void __launch_bounds__(D) splitk_merge_kernel(const DecodeParams p) {
     const int part_tokens = p.part_blocks * kBlockTokens;
     const int np = (len + part_tokens - 1) / part_tokens;
     const size_t row = static_cast<size_t>(b) * p.Hq + h;
-    const float *ml = p.ws_ml + 2 * row * p.num_parts;
-    const float *o = p.ws_o + row * p.num_parts * D;
+    const float *ml = p.ws_ml + 2 * (row * p.ws_parts + p.ws_part0);
+    const float *o = p.ws_o + (row * p.ws_parts + p.ws_part0) * D;
     float M = -INFINITY;
     for (int q = 0; q < np; ++q) M = fmaxf(M, ml[2 * q]);
     float L = 0.f, O = 0.f;
@@ -234,7 +236,7 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
                     static_cast<unsigned>(p.B));
     kern<<<grid, NW * 32, G::kSmemBytes, stream>>>(tmk, tmv, p);
     e = cudaGetLastError();
-    if (e != cudaSuccess || !SPLIT) return e;
+    if (e != cudaSuccess || !SPLIT || p.skip_merge) return e;
     splitk_merge_kernel<D><<<dim3(static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B)), D, 0,
                              stream>>>(p);
     return cudaGetLastError();

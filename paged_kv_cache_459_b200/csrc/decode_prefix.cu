@@ -1,0 +1,293 @@
+// Shared-prefix ("cascade") decode attention.
+//
+// Several sequences whose block tables start with the same physical blocks
+// ("vLLM 與 PagedAttention：高吞吐推理的關鍵", section 二, 無法共享: the tables of
+// requests with a common prefix point at one set of blocks) need the same
+// prefix K/V.  Plain decode streams those shared blocks once per sequence;
+// here they are read once per (group, KV head) and the attention of every
+// member's query against them is computed as one dense product:
+//   rows = (member, query head of this KV head) pairs, 16 per warp tile,
+//   S[16 rows x 16 tokens] = Q . K_blk^T  and  O[16 x d] += P . V_blk
+// on mma.m16n8k16 (bf16 in, fp32 accumulate) -- with 128 members this is a
+// 128-row tile per KV head, a real dense contraction.  Each CTA takes a chunk
+// of CB prefix blocks, loads its K and V tiles once with TMA, and leaves one
+// partial (m, l, o) per row.  The private suffixes go through the split-K
+// kernel starting past the prefix, and the merge below combines prefix and
+// suffix partials of each (sequence, query head) by log-sum-exp.  The result
+// equals plain decode over the whole sequence.
+#include "decode_common.cuh"
+
+namespace pkv {
+
+namespace {
+
+using namespace dev;
+
+constexpr int kPrefixWarps = 4;
+
+template <int D, int CB>
+__global__ void __launch_bounds__(kPrefixWarps * 32)
+    prefix_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
+                        const __grid_constant__ CUtensorMap tmv, const PrefixParams p) {
+    constexpr int KS = D / 16;                     // k-steps of S = Q K^T over d
+    constexpr int NT = D / 8;                      // 8-column tiles of O
+    constexpr int kTile = (D / 64) * kBoxBytes;    // one K or V tile of a block
+    const int c = blockIdx.x, kvh = blockIdx.y, g = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tig = lane & 3, gid = lane >> 2;
+
+    const int off = __ldg(p.group_offsets + g);
+    const int members = __ldg(p.group_offsets + g + 1) - off;
+    if (members <= 0) return;
+    const int b0 = __ldg(p.group_seqs + off);
+    if (b0 < 0 || b0 >= p.B) {
+        if (threadIdx.x == 0) flag(p.err, PKV_DEV_ERR_BAD_LEN);
+        return;
+    }
+    int len0 = __ldg(p.seq_lens + b0);
+    len0 = len0 < 0 ? 0 : min(len0, p.W * kBlockTokens);
+    const int nb = min(max(__ldg(p.prefix_blocks + b0), 0), len0 / kBlockTokens);  // full blocks
+    const int j0 = c * CB, j1 = min(nb, j0 + CB);
+    if (j0 >= j1) return;
+    const int nt = j1 - j0;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *ktiles = smem;                    // [CB][kTile]
+    uint8_t *vtiles = smem + CB * kTile;       // [CB][kTile]
+    const uint32_t bar = smem_u32(smem + 2 * CB * kTile);
+    int *valid = reinterpret_cast<int *>(smem + 2 * CB * kTile + 8);  // [CB]
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int32_t *row = p.block_tables + static_cast<size_t>(b0) * p.W;
+        uint32_t bytes = 0;
+        for (int t = 0; t < nt; ++t) {
+            const int32_t phys = __ldg(row + j0 + t);
+            valid[t] = phys >= 0 && phys < p.num_blocks ? phys : -1;
+            if (valid[t] >= 0) bytes += 2 * kTile;
+        }
+        mbar_arrive_expect_tx(bar, bytes);
+        const uint64_t policy = l2_policy_evict_first();
+        for (int t = 0; t < nt; ++t) {
+            if (valid[t] < 0) {
+                flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
+                continue;
+            }
+            const int y = valid[t] * (p.Hkv * kBlockTokens) + kvh * kBlockTokens;
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh) {
+                tma_load_2d(smem_u32(ktiles + t * kTile) + hh * kBoxBytes, &tmk, hh * 64, y, bar, policy);
+                tma_load_2d(smem_u32(vtiles + t * kTile) + hh * kBoxBytes, &tmv, hh * 64, y, bar, policy);
+            }
+        }
+    }
+    __syncthreads();  // valid[] written
+    if (!mbar_wait(bar, 0, kWaitLimitNs)) {
+        if (threadIdx.x == 0) flag(p.err, PKV_DEV_ERR_TIMEOUT);
+        mbar_wait(bar, 0, kWaitLimitNs);  // let copies in flight land before exiting
+        return;
+    }
+
+    const int G = p.group;        // query heads per KV head
+    const int R = members * G;    // query rows of this group and KV head
+    for (int rt = warp; rt * 16 < R; rt += kPrefixWarps) {
+        // Q rows (member, head) as mma A fragments: rows gid and gid + 8.
+        int rb[2], rh[2];
+        const uint32_t *qr[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = rt * 16 + gid + 8 * i;
+            rb[i] = -1;
+            rh[i] = 0;
+            qr[i] = nullptr;
+            if (r < R) {
+                const int b = __ldg(p.group_seqs + off + r / G);
+                if (b >= 0 && b < p.B) {
+                    rb[i] = b;
+                    rh[i] = kvh * G + r % G;
+                    qr[i] = reinterpret_cast<const uint32_t *>(p.q + (static_cast<size_t>(b) * p.Hq + rh[i]) * D);
+                }
+            }
+        }
+        uint32_t qa[KS][4];
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qa[ks][0] = qr[0] ? __ldg(qr[0] + (16 * ks + 2 * tig) / 2) : 0u;
+            qa[ks][1] = qr[1] ? __ldg(qr[1] + (16 * ks + 2 * tig) / 2) : 0u;
+            qa[ks][2] = qr[0] ? __ldg(qr[0] + (16 * ks + 8 + 2 * tig) / 2) : 0u;
+            qa[ks][3] = qr[1] ? __ldg(qr[1] + (16 * ks + 8 + 2 * tig) / 2) : 0u;
+        }
+        float o[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[n][i] = 0.f;
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+
+        for (int t = 0; t < nt; ++t) {
+            if (valid[t] < 0) continue;
+            const uint32_t kt = smem_u32(ktiles + t * kTile), vt = smem_u32(vtiles + t * kTile);
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};  // tokens 0-7, 8-15
+            {
+                const int tok = (lane & 7) + (lane >> 4) * 8;
+                const int cb = (lane >> 3) & 1;
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    uint32_t b00, b01, b10, b11;
+                    ldmatrix_x4(kt + tile_off(tok, 2 * ks + cb), b00, b01, b10, b11);
+                    mma_bf16_16816(s0, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
+                    mma_bf16_16816(s1, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s0[i] *= p.scale_log2;
+                s1[i] *= p.scale_log2;
+            }
+            // row gid: s0[0], s0[1], s1[0], s1[1]; row gid + 8: s0[2], s0[3], s1[2], s1[3]
+            float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
+            float mx1 = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
+#pragma unroll
+            for (int m = 1; m < 4; m <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, m));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, m));
+            }
+            const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+            const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
+            m_run[0] = mn0;
+            m_run[1] = mn1;
+            float pr0[4], pr1[4];
+            pr0[0] = exp2f(s0[0] - mn0);
+            pr0[1] = exp2f(s0[1] - mn0);
+            pr1[0] = exp2f(s1[0] - mn0);
+            pr1[1] = exp2f(s1[1] - mn0);
+            pr0[2] = exp2f(s0[2] - mn1);
+            pr0[3] = exp2f(s0[3] - mn1);
+            pr1[2] = exp2f(s1[2] - mn1);
+            pr1[3] = exp2f(s1[3] - mn1);
+            l_run[0] = l_run[0] * al0 + pr0[0] + pr0[1] + pr1[0] + pr1[1];
+            l_run[1] = l_run[1] * al1 + pr0[2] + pr0[3] + pr1[2] + pr1[3];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                o[n][0] *= al0;
+                o[n][1] *= al0;
+                o[n][2] *= al1;
+                o[n][3] *= al1;
+            }
+            const uint32_t pa0 = pack_bf16x2(pr0[0], pr0[1]), pa1 = pack_bf16x2(pr0[2], pr0[3]);
+            const uint32_t pa2 = pack_bf16x2(pr1[0], pr1[1]), pa3 = pack_bf16x2(pr1[2], pr1[3]);
+            const int tok = (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int cb = lane >> 4;
+#pragma unroll
+            for (int i = 0; i < NT / 2; ++i) {
+                uint32_t v0, v1, v2, v3;
+                ldmatrix_x4_trans(vt + tile_off(tok, 2 * i + cb), v0, v1, v2, v3);
+                mma_bf16_16816(o[2 * i], pa0, pa1, pa2, pa3, v0, v1);
+                mma_bf16_16816(o[2 * i + 1], pa0, pa1, pa2, pa3, v2, v3);
+            }
+        }
+#pragma unroll
+        for (int m = 1; m < 4; m <<= 1) {
+            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], m);
+            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], m);
+        }
+        // partial of (sequence, head) for prefix chunk c
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if (rb[i] < 0) continue;
+            const size_t slot = (static_cast<size_t>(rb[i]) * p.Hq + rh[i]) * p.ws_parts + c;
+            float *dst = p.ws_o + slot * D;
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+                *reinterpret_cast<float2 *>(dst + 8 * n + 2 * tig) = make_float2(o[n][2 * i], o[n][2 * i + 1]);
+            if (tig == 0) {
+                p.ws_ml[2 * slot] = m_run[i];
+                p.ws_ml[2 * slot + 1] = l_run[i];
+            }
+        }
+    }
+}
+
+// Merge of one (sequence, query head): prefix chunks [0, ceil(pb / CB)) and
+// the suffix split-K partitions that hold tokens past the prefix, in index
+// order, by log-sum-exp.
+template <int D, int CB>
+__global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) {
+    const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
+    int len = __ldg(p.seq_lens + b);
+    len = len < 0 ? 0 : min(len, p.W * kBlockTokens);
+    const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
+    const int pb = min(max(__ldg(p.prefix_blocks + b), 0), len / kBlockTokens);
+    const int nchunks = (pb + CB - 1) / CB;
+    const size_t row = static_cast<size_t>(b) * p.Hq + h;
+    const float *ml = p.ws_ml + 2 * row * p.ws_parts;
+    const float *o = p.ws_o + row * p.ws_parts * D;
+    const auto used = [&](int part) {  // slot `part` holds a partial for this row
+        if (part < p.prefix_parts) return part < nchunks;
+        const int q = part - p.prefix_parts;
+        return max(q * p.part_blocks, pb) < min((q + 1) * p.part_blocks, nblk);
+    };
+    float M = -INFINITY;
+    for (int q = 0; q < p.ws_parts; ++q)
+        if (used(q)) M = fmaxf(M, ml[2 * q]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+        for (int q = 0; q < p.ws_parts; ++q) {
+            if (!used(q)) continue;
+            const float c = exp2f(ml[2 * q] - M);
+            L = fmaf(ml[2 * q + 1], c, L);
+            O = fmaf(o[static_cast<size_t>(q) * D + e], c, O);
+        }
+    }
+    p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
+}
+
+template <int D>
+cudaError_t launch_prefix_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &p,
+                            int num_groups, cudaStream_t stream) {
+    constexpr int CB = kPrefixChunkBlocks;
+    constexpr int kTile = (D / 64) * kBoxBytes;
+    constexpr int kSmem = 2 * CB * kTile + 8 + CB * 4 + 1024;
+    auto kern = prefix_chunk_kernel<D, CB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    if (num_groups > 0) {
+        const dim3 grid(static_cast<unsigned>(p.prefix_parts), static_cast<unsigned>(p.Hkv),
+                        static_cast<unsigned>(num_groups));
+        kern<<<grid, kPrefixWarps * 32, kSmem, stream>>>(tmk, tmv, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_cascade_merge_d(const PrefixParams &p, cudaStream_t stream) {
+    cascade_merge_kernel<D, kPrefixChunkBlocks>
+        <<<dim3(static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B)), D, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefix_chunks(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                 const PrefixParams &p, int head_dim, int num_groups,
+                                 cudaStream_t stream) {
+    if (head_dim == 128) return launch_prefix_d<128>(tmk, tmv, p, num_groups, stream);
+    if (head_dim == 64) return launch_prefix_d<64>(tmk, tmv, p, num_groups, stream);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_cascade_merge(const PrefixParams &p, int head_dim, cudaStream_t stream) {
+    if (head_dim == 128) return launch_cascade_merge_d<128>(p, stream);
+    if (head_dim == 64) return launch_cascade_merge_d<64>(p, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pkv

@@ -27,6 +27,15 @@ struct DecodeParams {
     int part_blocks;  // blocks per CTA work unit (partition, or W for single pass)
     int num_parts;    // partitions per sequence (grid.x)
     float scale_log2; // scale * log2(e)
+    // Split-K workspace addressing: partition p of a row is partial slot
+    // (row * ws_parts + ws_part0 + p).  Plain split-K: ws_parts = num_parts,
+    // ws_part0 = 0.
+    int ws_parts, ws_part0;
+    // Optional [B]: sequence b's first start_blocks[b] blocks are left out
+    // (their part of the attention is computed elsewhere and merged later);
+    // clamped to the sequence's full blocks.
+    const int32_t *start_blocks;
+    bool skip_merge;  // split-K without its merge kernel (the caller merges)
 };
 
 struct DecodeTuning {
@@ -65,6 +74,34 @@ cudaError_t launch_decode_stream(const CUtensorMap &tmk, const CUtensorMap &tmv,
 // Launches the decode kernel (and the merge kernel when split) on `stream`.
 cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                           int head_dim, bool split, DecodeTuning tuning, cudaStream_t stream);
+
+// Shared-prefix (cascade) decode: prefix blocks read once per (group, KV
+// head) by a dense tensor-core kernel; suffixes by split-K; LSE merge.
+constexpr int kPrefixChunkBlocks = 8;  // prefix blocks per CTA
+
+struct PrefixParams {
+    __nv_bfloat16 *out;
+    const __nv_bfloat16 *q;
+    const int32_t *block_tables;
+    const int32_t *seq_lens;
+    const int32_t *prefix_blocks;   // [B] shared leading blocks of each sequence (0: none)
+    const int32_t *group_offsets;   // [G + 1] CSR offsets into group_seqs
+    const int32_t *group_seqs;      // members of each group (sequence indices)
+    float *ws_o;                    // [B][Hq][ws_parts][D]
+    float *ws_ml;                   // [B][Hq][ws_parts][2]
+    unsigned int *err;
+    long long num_blocks;
+    int W, B, Hq, Hkv, group;
+    int ws_parts;      // prefix_parts + suffix partitions
+    int prefix_parts;  // ceil(W / kPrefixChunkBlocks): slots 0.. hold prefix chunks
+    int part_blocks;   // suffix split-K partition (blocks)
+    float scale_log2;
+};
+
+cudaError_t launch_prefix_chunks(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                 const PrefixParams &p, int head_dim, int num_groups,
+                                 cudaStream_t stream);
+cudaError_t launch_cascade_merge(const PrefixParams &p, int head_dim, cudaStream_t stream);
 
 cudaError_t launch_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
                             const int64_t *slot_mapping, int num_tokens, int num_kv_heads,

@@ -269,6 +269,7 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
         const size_t rows_ws = static_cast<size_t>(num_seqs) * num_heads * p.num_parts;
         p.ws_o = static_cast<float *>(workspace);
         p.ws_ml = p.ws_o + rows_ws * head_dim;
+        p.ws_parts = p.num_parts;
     } else {
         p.part_blocks = max_blocks_per_seq;
         p.num_parts = 1;
@@ -276,6 +277,116 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
     pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
     cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, split, t,
                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                         int max_blocks_per_seq, int partition_tokens) {
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0) return 0;
+    if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
+    if (partition_tokens % PKV_BLOCK_TOKENS) return 0;
+    const size_t parts =
+        static_cast<size_t>(num_parts_for(max_blocks_per_seq, partition_tokens)) +
+        (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+    return static_cast<size_t>(num_seqs) * num_heads * parts * (static_cast<size_t>(head_dim) + 2) *
+           sizeof(float);
+}
+
+pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const void *k_cache,
+                                             const void *v_cache, const int32_t *block_tables,
+                                             int max_blocks_per_seq, const int32_t *seq_lens,
+                                             int num_seqs, int num_heads, int num_kv_heads,
+                                             int head_dim, int64_t num_blocks, float scale,
+                                             const int32_t *prefix_blocks,
+                                             const int32_t *group_offsets,
+                                             const int32_t *group_seqs, int num_groups,
+                                             int partition_tokens, void *workspace,
+                                             size_t workspace_bytes, unsigned int *err_word,
+                                             void *stream) {
+    if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_heads % num_kv_heads || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+        !std::isfinite(scale) || num_groups < 0 || num_groups > 65535)
+        return PKV_ERR_INVALID_ARG;
+    if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
+    if (partition_tokens % PKV_BLOCK_TOKENS || partition_tokens > 65536) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !prefix_blocks ||
+        (num_groups > 0 && (!group_offsets || !group_seqs)))
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_INVALID_ARG;
+    if (num_blocks > INT32_MAX / PKV_BLOCK_TOKENS / num_kv_heads) return PKV_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(max_blocks_per_seq) * PKV_BLOCK_TOKENS > INT32_MAX)
+        return PKV_ERR_INVALID_ARG;
+    const size_t need = pkv_decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                          max_blocks_per_seq, partition_tokens);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return PKV_ERR_WORKSPACE;
+
+    const int64_t rows = num_blocks * num_kv_heads * PKV_BLOCK_TOKENS;
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, k_cache, rows, head_dim) ||
+        !encode_cache_map(&tmv, v_cache, rows, head_dim))
+        return PKV_ERR_CUDA;
+
+    const int suffix_parts = num_parts_for(max_blocks_per_seq, partition_tokens);
+    const int prefix_parts = (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+    const size_t ws_rows = static_cast<size_t>(num_seqs) * num_heads * (prefix_parts + suffix_parts);
+    float *ws_o = static_cast<float *>(workspace);
+    float *ws_ml = ws_o + ws_rows * head_dim;
+
+    pkv::PrefixParams pp{};
+    pp.out = static_cast<__nv_bfloat16 *>(out);
+    pp.q = static_cast<const __nv_bfloat16 *>(q);
+    pp.block_tables = block_tables;
+    pp.seq_lens = seq_lens;
+    pp.prefix_blocks = prefix_blocks;
+    pp.group_offsets = group_offsets;
+    pp.group_seqs = group_seqs;
+    pp.ws_o = ws_o;
+    pp.ws_ml = ws_ml;
+    pp.err = err_word;
+    pp.num_blocks = num_blocks;
+    pp.W = max_blocks_per_seq;
+    pp.B = num_seqs;
+    pp.Hq = num_heads;
+    pp.Hkv = num_kv_heads;
+    pp.group = num_heads / num_kv_heads;
+    pp.ws_parts = prefix_parts + suffix_parts;
+    pp.prefix_parts = prefix_parts;
+    pp.part_blocks = partition_tokens / PKV_BLOCK_TOKENS;
+    pp.scale_log2 = scale * 1.4426950408889634f;
+
+    pkv::DecodeParams dp{};
+    dp.out = pp.out;
+    dp.q = pp.q;
+    dp.block_tables = block_tables;
+    dp.seq_lens = seq_lens;
+    dp.err = err_word;
+    dp.num_blocks = num_blocks;
+    dp.W = max_blocks_per_seq;
+    dp.B = num_seqs;
+    dp.Hq = num_heads;
+    dp.Hkv = num_kv_heads;
+    dp.group = pp.group;
+    dp.chunks = (pp.group + 7) / 8;
+    dp.scale_log2 = pp.scale_log2;
+    dp.part_blocks = pp.part_blocks;
+    dp.num_parts = suffix_parts;
+    dp.ws_o = ws_o;
+    dp.ws_ml = ws_ml;
+    dp.ws_parts = pp.ws_parts;
+    dp.ws_part0 = prefix_parts;
+    dp.start_blocks = prefix_blocks;
+    dp.skip_merge = true;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = pkv::launch_prefix_chunks(tmk, tmv, pp, head_dim, num_groups, st);
+    if (e == cudaSuccess) {
+        pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
+        e = pkv::launch_decode(tmk, tmv, dp, head_dim, true, t, st);
+    }
+    if (e == cudaSuccess) e = pkv::launch_cascade_merge(pp, head_dim, st);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

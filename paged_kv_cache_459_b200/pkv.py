@@ -59,6 +59,11 @@ _sigs = {
     "pkv_alloc_stats": ([_P, _P, _P, _P, _P], _i32),
     "pkv_alloc_free_list": ([_P, _P, _i64, _P], _i32),
     "pkv_alloc_refcount": ([_P, _i64, _P], _i32),
+    "pkv_alloc_prefix_groups": ([_P, _P, _i32, _P, _P, _P, _P], _i32),
+    "pkv_decode_prefix_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
+    "pkv_paged_attention_decode_prefix": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
+                                           _i64, _f32, _P, _P, _P, _i32, _i32, _P, _sz, _P, _P],
+                                          _i32),
     "pkv_alloc_seq_len": ([_P, _i64, _P], _i32),
     "pkv_alloc_slot_of": ([_P, _i64, _i64, _P], _i32),
 }
@@ -199,6 +204,46 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
            "pkv_paged_attention_decode")
 
 
+def decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_seq,
+                                  partition_tokens=DEFAULT_PARTITION_TOKENS) -> int:
+    return int(_lib.pkv_decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                      max_blocks_per_seq, partition_tokens))
+
+
+def paged_attention_decode_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
+                                  num_kv_heads, prefix_blocks, group_offsets, group_seqs, *,
+                                  partition_tokens: int = DEFAULT_PARTITION_TOKENS,
+                                  workspace=None, err=None) -> None:
+    """Decode with shared prefixes read once per group (see include/pkv.h).
+    prefix_blocks [B], group_offsets [G + 1], group_seqs [members]: int32 CUDA."""
+    import torch
+
+    bf = torch.bfloat16
+    B, hq, d = q.shape
+    W = block_tables.shape[1]
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
+            or block_tables.shape[0] != B or seq_lens.shape != (B,) or prefix_blocks.shape != (B,):
+        raise ValueError("shape mismatch")
+    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"),
+                                                 (v_cache, "v_cache"))]
+    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
+    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
+    pp = _dev_tensor(prefix_blocks, torch.int32, "prefix_blocks")
+    G = group_offsets.numel() - 1
+    op = _dev_tensor(group_offsets, torch.int32, "group_offsets")
+    gp = _dev_tensor(group_seqs, torch.int32, "group_seqs") if group_seqs.numel() else None
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    if workspace is None:
+        workspace = _workspace(q.device, decode_prefix_workspace_bytes(B, hq, d, W,
+                                                                       partition_tokens))
+    wp = _dev_tensor(workspace, torch.uint8, "workspace")
+    _check(_lib.pkv_paged_attention_decode_prefix(
+        ptrs[0], ptrs[1], ptrs[2], ptrs[3], tp, W, lp, B, hq, num_kv_heads, d, k_cache.shape[0],
+        float(scale), pp, op, gp, G, partition_tokens, wp, workspace.numel(), ep,
+        _stream_ptr(q.device)), "pkv_paged_attention_decode_prefix")
+
+
 # ---------------------------------------------------------------- allocator
 class AllocError(PkvError):
     @property
@@ -276,6 +321,20 @@ class BlockAllocator:
         _acheck(_lib.pkv_alloc_free_list(self._h, out.ctypes.data if n.value else None, n.value,
                                          ctypes.byref(n)), "free_list")
         return out.tolist()
+
+    def prefix_groups(self, seq_ids):
+        """(prefix_blocks [n], group_offsets [G + 1], group_seqs [members]) as int32
+        arrays for paged_attention_decode_prefix; group_seqs index into seq_ids."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = len(ids)
+        pb = np.zeros(n, np.int32)
+        offs = np.zeros(n + 1, np.int32)
+        members = np.zeros(max(n, 1), np.int32)
+        g = ctypes.c_int32()
+        _acheck(_lib.pkv_alloc_prefix_groups(self._h, ids.ctypes.data, n, pb.ctypes.data,
+                                             offs.ctypes.data, members.ctypes.data,
+                                             ctypes.byref(g)), "prefix_groups")
+        return pb, offs[: g.value + 1].copy(), members[: offs[g.value]].copy()
 
     def refcount(self, block: int) -> int:
         out = ctypes.c_int32()

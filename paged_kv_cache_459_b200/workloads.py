@@ -115,12 +115,19 @@ def draw_lens(cfg: dict, gen: np.random.Generator) -> np.ndarray:
     return gen.integers(cfg["len_lo"], cfg["len_hi"], size=b, endpoint=True).astype(np.int64)
 
 
+def _shares_prefix(cfg: dict, s: int) -> bool:
+    every = cfg.get("unshared_every", 0)
+    return "prefix_len" in cfg and not (every and s % every == every - 1)
+
+
 def pool_blocks(cfg: dict, lens: np.ndarray) -> int:
     if "num_blocks" in cfg:
         return int(cfg["num_blocks"])
     nb = lambda n: -(-int(n) // BLOCK_TOKENS)  # noqa: E731  (blocks to hold n tokens)
     if "prefix_len" in cfg:
-        need = nb(cfg["prefix_len"]) + sum(nb(int(l) - cfg["prefix_len"]) for l in lens)
+        pl = cfg["prefix_len"]
+        need = nb(pl) * cfg.get("prefix_groups", 1) + sum(
+            nb(int(l) - pl) if _shares_prefix(cfg, s) else nb(int(l)) for s, l in enumerate(lens))
     else:
         need = sum(nb(int(l)) for l in lens)
     return int(math.ceil(cfg["pool_factor"] * need))
@@ -158,7 +165,9 @@ def build(name: str, seed: int, alloc_factory, *, batch: int | None = None,
     tokens, then one token is appended, whose slot is the step's
     ``slot_mapping`` entry.  In the ``prefix`` workload a 2000-token prefix is
     prefilled once, forked into every sequence and then released by its owner,
-    so its blocks are shared by all ``batch`` tables.
+    so its blocks are shared by all ``batch`` tables (``prefix_groups`` > 1:
+    that many prefixes, sequence s joining group s % prefix_groups;
+    ``unshared_every`` = n: every n-th sequence holds no shared prefix).
     """
     cfg = config(name, **overrides)
     if batch is not None:
@@ -173,14 +182,19 @@ def build(name: str, seed: int, alloc_factory, *, batch: int | None = None,
     b = cfg["batch"]
     seq_ids = list(range(b))
     if "prefix_len" in cfg:
-        owner = b  # an id outside the batch
-        alloc.add_seq(owner, cfg["prefix_len"])
+        # owners of the shared prefixes get ids outside the batch
+        owners = [b + g for g in range(cfg.get("prefix_groups", 1))]
+        for o in owners:
+            alloc.add_seq(o, cfg["prefix_len"])
         for s in seq_ids:
-            alloc.fork(owner, s)
-        for s in seq_ids:
-            for _ in range(int(lens[s]) - 1 - cfg["prefix_len"]):
-                alloc.append_token(s)
-        alloc.free_seq(owner)
+            if _shares_prefix(cfg, s):
+                alloc.fork(owners[s % len(owners)], s)
+                for _ in range(int(lens[s]) - 1 - cfg["prefix_len"]):
+                    alloc.append_token(s)
+            else:
+                alloc.add_seq(s, int(lens[s]) - 1)
+        for o in owners:
+            alloc.free_seq(o)
     else:
         for s in seq_ids:
             alloc.add_seq(s, int(lens[s]) - 1)

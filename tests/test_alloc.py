@@ -145,3 +145,69 @@ def test_workload_tables_match_model(name, kw):
     if name == "prefix":
         assert all(w1.alloc.refcount(int(b)) == w1.cfg["batch"] for b in w1.block_tables[0, :125])
         assert w1.alloc.stats()[2] == 125
+
+
+def test_prefix_groups_sharing_example(golden_dir):
+    """The pages' example: blocks 1 and 2 are shared by all three tables."""
+    g = json.load(open(os.path.join(golden_dir, "sharing_example.json")))
+    for alloc_cls in (BlockAllocator, BlockManager):
+        a = alloc_cls(16, list(range(1, 16)) + [0])
+        a.add_seq(0, 64)
+        a.fork(0, 1, 48)
+        for _ in range(16):
+            a.append_token(1)
+        a.fork(0, 2, 32)
+        for _ in range(32):
+            a.append_token(2)
+        pb, offs, members = a.prefix_groups([0, 1, 2])
+        assert pb.tolist() == [len(g["printed"]["shared_by_three"])] * 3
+        assert offs.tolist() == [0, 3] and members.tolist() == [0, 1, 2]
+
+
+@pytest.mark.parametrize("kw", [dict(batch=12), dict(batch=20, prefix_groups=3, unshared_every=4),
+                                dict(batch=9, prefix_len=48, suffix_lo=1, suffix_hi=30)])
+def test_prefix_groups_match_model(kw):
+    w1 = wl.build("prefix", 3, BlockAllocator, with_cache=False, **kw)
+    w2 = wl.build("prefix", 3, BlockManager, with_cache=False, **kw)
+    ids = list(range(w1.cfg["batch"]))
+    r1, r2 = w1.alloc.prefix_groups(ids), w2.alloc.prefix_groups(ids)
+    for x, y in zip(r1, r2):
+        assert np.array_equal(x, y)
+    pb, offs, members = r1
+    groups = kw.get("prefix_groups", 1)
+    assert len(offs) - 1 == groups
+    # a member's prefix is the shared full blocks; 2000 tokens = 125 blocks
+    for gi in range(groups):
+        mem = members[offs[gi]:offs[gi + 1]]
+        assert (pb[mem] == min(w1.cfg["prefix_len"], int(w1.lens[mem].min())) // 16).all()
+        rows = w1.block_tables[mem, :pb[mem[0]]]
+        assert (rows == rows[0]).all()
+
+
+def test_prefix_groups_random_forks_match_model():
+    gen = np.random.default_rng(5)
+    for trial in range(20):
+        nb = 200
+        order = gen.permutation(nb)
+        a, m = BlockAllocator(nb, order), BlockManager(nb, order)
+        n0 = int(gen.integers(0, 90)) if trial % 2 else 64
+        for x in (a, m):
+            x.add_seq(0, n0)
+        live = [0]
+        r = np.random.default_rng(trial)
+        for s in range(1, 12):
+            parent = int(r.choice(live))
+            n = int(r.integers(0, m.lens[parent] + 1))
+            ext = int(r.integers(0, 40))
+            for x in (a, m):
+                x.fork(parent, s, n)
+            try:
+                for _ in range(ext):
+                    for x in (a, m):
+                        x.append_token(s)
+            except Exception:
+                pass
+            live.append(s)
+        ids = list(range(12))
+        for x, y in zip(a.prefix_groups(ids), m.prefix_groups(ids)):
+            assert np.array_equal(x, y)

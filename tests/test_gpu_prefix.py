@@ -1,0 +1,82 @@
+"""GPU parity of the shared-prefix (cascade) decode: the prefix blocks that a
+group of block tables share are read once per (group, KV head); the result
+must match the fp64 oracle, which reads every sequence's blocks on its own."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import DeviceStep, build, check_close, host_bits, oracle_after_write
+
+pytestmark = pytest.mark.gpu
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from paged_kv_cache_459_b200 import pkv  # noqa: E402
+from paged_kv_cache_459_b200 import workloads as wl  # noqa: E402
+
+
+def cascade(d: DeviceStep, part=512, tables=None):
+    w = d.w
+    pb, offs, members = w.alloc.prefix_groups(list(range(w.cfg["batch"])))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).cuda()  # noqa: E731
+    pkv.paged_attention_decode_prefix(d.out, d.q, d.kc, d.vc, d.tables if tables is None else tables,
+                                      d.lens, w.cfg["scale"], w.cfg["num_kv_heads"], dev(pb),
+                                      dev(offs), dev(members), partition_tokens=part, err=d.err)
+    torch.cuda.synchronize()
+    return host_bits(d.out), pb, offs
+
+
+CASES = [
+    ("prefix", dict(batch=6, prefix_len=320, suffix_lo=1, suffix_hi=60)),
+    ("prefix", dict(batch=20, prefix_len=160, suffix_lo=1, suffix_hi=200, prefix_groups=3,
+                    unshared_every=4)),
+    ("prefix", dict(batch=9, prefix_len=208, suffix_lo=1, suffix_hi=100, num_heads=28,
+                    num_kv_heads=4)),
+    ("prefix", dict(batch=7, prefix_len=144, suffix_lo=1, suffix_hi=90, head_dim=64,
+                    num_heads=16, num_kv_heads=2)),
+    ("prefix", dict(batch=40, prefix_len=16, suffix_lo=1, suffix_hi=20)),   # one shared block
+    ("prefix", dict(batch=5, prefix_len=48, suffix_lo=1, suffix_hi=1)),     # suffix = new token
+]
+
+
+@pytest.mark.parametrize("name,kw", CASES, ids=[str(i) for i in range(len(CASES))])
+def test_cascade_matches_oracle(name, kw):
+    w = build(name, 13, **kw)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc, ref = oracle_after_write(w)
+    for part in (512, 64):
+        out, pb, offs = cascade(d, part)
+        assert len(offs) - 1 == kw.get("prefix_groups", 1) and pb.max() > 0
+        check_close(out, ref, f"cascade {kw} partition {part}")
+    assert d.err_word() == 0
+
+
+def test_cascade_full_size_sampled():
+    w = build("prefix", 0)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    out, pb, offs = cascade(d)
+    assert (pb == 125).all() and len(offs) == 2
+    sel = np.array([0, 5, 64, 127])
+    ref = oracle.paged_decode(w.q[sel], kc, vc, w.block_tables[sel], w.lens[sel], w.cfg["scale"])
+    check_close(out[sel], ref, "cascade full size")
+    plain = d.decode(pkv.DECODE_SINGLE)
+    check_close(out, wl.bf16_to_f32(plain).astype(np.float64), "cascade vs single pass")
+    assert d.err_word() == 0
+
+
+def test_cascade_block_relabelling_is_bit_exact():
+    w = build("prefix", 14, batch=10, prefix_len=256, suffix_lo=1, suffix_hi=80, prefix_groups=2)
+    d = DeviceStep(w)
+    d.write()
+    base, _, _ = cascade(d)
+    perm = wl.rng(3).permutation(w.num_blocks)
+    t2, _, kc2, vc2 = wl.permute_pool(perm, w.block_tables, w.slot_mapping, host_bits(d.kc),
+                                      host_bits(d.vc))
+    d.kc.copy_(torch.from_numpy(kc2.view(np.int16)).view(torch.bfloat16))
+    d.vc.copy_(torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16))
+    out, _, _ = cascade(d, tables=torch.from_numpy(t2).cuda())
+    assert np.array_equal(out, base)
