@@ -59,7 +59,7 @@ extern "C" {
 typedef enum {
     PKV_OK = 0,
     PKV_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned buffer, bad id */
-    PKV_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, pool size, CoW) */
+    PKV_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, pool size) */
     PKV_ERR_WORKSPACE = 3,   /* split-K requested without a large enough workspace */
     PKV_ERR_OOM = 4,         /* block pool exhausted (allocator state unchanged) */
     PKV_ERR_CUDA = 5         /* a CUDA runtime/driver call failed */
@@ -234,6 +234,19 @@ PKV_API pkv_status pkv_paged_attention_decode_prefix(
     int num_groups, int partition_tokens, void *workspace, size_t workspace_bytes,
     unsigned int *err_word, void *stream);
 
+/*
+ * Block copy for copy-on-write (a sequence that shares a partly filled block,
+ * e.g. a beam forked mid-block -- "vllm" (xiexianbin.cn), "PagedAttention 的核
+ * 心原理": beam candidates share prefix blocks -- takes a private copy before
+ * its next token is written).  For every i: all num_kv_heads x 16 slots of
+ * block src[i] are copied to block dst[i], in both caches (bit copy).
+ * src, dst: device int64 [n]; a dst must not be the src of another pair.
+ * Ids outside [0, num_blocks) are skipped and flagged PKV_DEV_ERR_BAD_BLOCK.
+ */
+PKV_API pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, const int64_t *src,
+                                   const int64_t *dst, int n, int num_kv_heads, int head_dim,
+                                   int64_t num_blocks, unsigned int *err_word, void *stream);
+
 /* ------------------------------------------------------------------------
  * Host block allocator (section 二 and section 三 of the first page): a pool
  * of num_blocks physical blocks with reference counts, per-sequence block
@@ -258,14 +271,22 @@ PKV_API pkv_status pkv_alloc_add_seq(pkv_alloc *a, int64_t seq_id, int64_t num_t
 PKV_API pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, int64_t num_tokens);
 
 /* One more token for seq_id; *slot_out receives its slot.  A new block is
- * taken when the last one is full (or there is none).  Appending into a
- * partly filled block that another sequence also holds would need a
- * copy-on-write: PKV_ERR_UNSUPPORTED. */
+ * taken when the last one is full (or there is none).  Appending into a partly
+ * filled last block that other tables also hold is a copy-on-write: the
+ * sequence gets a fresh block in its place, and the pair (shared block, fresh
+ * block) is queued for pkv_alloc_take_copies; the caller must copy those
+ * blocks on the device (pkv_copy_blocks) before writing the new token. */
 PKV_API pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_out);
 
 /* One token for each of n distinct sequences (a decode step); all or none. */
 PKV_API pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n,
                                    int64_t *slots_out);
+
+/* Takes the queued copy-on-write pairs: *n_out = their number; if cap >= it,
+ * src_out[i] -> dst_out[i] are filled (host arrays) and the queue is emptied;
+ * otherwise nothing is taken (call again with room for *n_out). */
+PKV_API pkv_status pkv_alloc_take_copies(pkv_alloc *a, int64_t *src_out, int64_t *dst_out,
+                                         int64_t cap, int64_t *n_out);
 
 /* Release a sequence: every block whose count drops to zero returns to the pool. */
 PKV_API pkv_status pkv_alloc_free_seq(pkv_alloc *a, int64_t seq_id);

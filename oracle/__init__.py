@@ -11,6 +11,7 @@ arithmetic.
 * ``paged_decode_partitioned`` -- the same in independent token partitions
                                combined by log-sum-exp (C, fp64).
 * ``kv_write``              -- the new token's K/V copied into its slot (C).
+* ``copy_blocks``           -- copy-on-write copies of whole blocks (C).
 * ``alloc_model.BlockManager`` -- the block allocator's reference model (Python).
 
 Pins (all CPU tests): the pages' worked block-table, waste and sharing
@@ -46,6 +47,8 @@ def lib() -> ctypes.CDLL:
                                                       i64, f64, i32]
         l.oracle_paged_decode_partitioned.restype = i32
         l.oracle_block_tokens.restype = i32
+        l.oracle_copy_blocks.argtypes = [P, P, P, P, i64, i32, i32, i64]
+        l.oracle_copy_blocks.restype = i32
         _lib = l
     return _lib
 
@@ -79,6 +82,17 @@ def kv_write(k_cache, v_cache, k, v, slot_mapping):
                                hkv, d, nb)
     if rc:
         raise ValueError("slot outside the pool")
+    return kc, vc
+
+
+def copy_blocks(k_cache, v_cache, src, dst):
+    """Copies of the caches after copying block src[i] to dst[i] for every i."""
+    kc, vc = np.array(_u16(k_cache), copy=True), np.array(_u16(v_cache), copy=True)
+    s = np.ascontiguousarray(src, dtype=np.int64)
+    d = np.ascontiguousarray(dst, dtype=np.int64)
+    nb, hkv, bt, hd = kc.shape
+    if lib().oracle_copy_blocks(_ptr(kc), _ptr(vc), _ptr(s), _ptr(d), len(s), hkv, hd, nb):
+        raise ValueError("block id outside the pool")
     return kc, vc
 
 

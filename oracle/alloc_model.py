@@ -18,8 +18,10 @@ Readings where the pages are silent:
   * ``fork(parent, child, n)`` gives the child the parent's first n tokens by
     sharing the blocks that hold them (refcount + 1 each); n defaults to the
     parent's length;
-  * appending into a partly filled block that another table also holds needs a
-    copy-on-write this model does not do: it is refused ("unsupported");
+  * appending into a partly filled last block that other tables also hold is a
+    copy-on-write: the sequence takes a fresh block in its place and the pair
+    (shared block, fresh block) is queued for the caller to copy on the device
+    (beam candidates share prefix blocks -- "vllm", PagedAttention 的核心原理);
   * every failing call leaves the state exactly as it was.
 """
 from __future__ import annotations
@@ -49,6 +51,7 @@ class BlockManager:
         self.ref = [0] * self.num_blocks
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        self.copies: list[tuple[int, int]] = []
 
     # -- lifecycle ---------------------------------------------------------
     def add_seq(self, seq_id: int, num_tokens: int) -> None:
@@ -73,27 +76,44 @@ class BlockManager:
             b = self.free.popleft()
             self.ref[b] = 1
             blocks.append(b)
-        elif self.ref[blocks[-1]] > 1:
-            raise AllocError("unsupported", "append into a shared, partly filled block")
+        elif self.ref[blocks[-1]] > 1:  # copy-on-write of the shared last block
+            if not self.free:
+                raise AllocError("oom")
+            b = self.free.popleft()
+            self.ref[b] = 1
+            self.ref[blocks[-1]] -= 1
+            self.copies.append((blocks[-1], b))
+            blocks[-1] = b
         self.lens[seq_id] = pos + 1
         return blocks[pos // BLOCK_TOKENS] * BLOCK_TOKENS + pos % BLOCK_TOKENS
 
     def append_tokens(self, seq_ids) -> list[int]:
         """One token for each listed sequence (one decode step), all or none:
-        an unknown or repeated id, then a shared partly filled last block, then
-        a shortage of free blocks is reported before anything changes."""
+        an unknown or repeated id, then a shortage of free blocks (fresh and
+        copy-on-write blocks together) is reported before anything changes."""
         ids = list(seq_ids)
         if len(set(ids)) != len(ids) or any(s not in self.tables for s in ids):
             raise AllocError("invalid", "unknown or repeated sequence")
-        need = 0
+        need, released = 0, {}
         for s in ids:
             if self.lens[s] % BLOCK_TOKENS == 0:
                 need += 1
-            elif self.ref[self.tables[s][-1]] > 1:
-                raise AllocError("unsupported", "append into a shared, partly filled block")
+            else:
+                last = self.tables[s][-1]
+                if self.ref[last] - released.get(last, 0) > 1:
+                    released[last] = released.get(last, 0) + 1
+                    need += 1
         if need > len(self.free):
             raise AllocError("oom")
         return [self.append_token(s) for s in ids]
+
+    def take_copies(self):
+        import numpy as np
+
+        src = np.array([c[0] for c in self.copies], np.int64)
+        dst = np.array([c[1] for c in self.copies], np.int64)
+        self.copies = []
+        return src, dst
 
     def fork(self, parent: int, child: int, num_tokens: int | None = None) -> None:
         if parent not in self.tables or child in self.tables:

@@ -79,6 +79,30 @@ int oracle_kv_write(uint16_t *k_cache, uint16_t *v_cache,
 }
 
 /*
+ * Copy-on-write block copy: a sequence that shares a partly filled block
+ * (beam candidates share prefix blocks -- "vllm", PagedAttention 的核心原理)
+ * gets a private copy before its next token is written.  Every slot of every
+ * KV head of block src[i] is copied to block dst[i], pairs in order.
+ * Returns 0, or -1 if an id is outside the pool (nothing copied then).
+ */
+int oracle_copy_blocks(uint16_t *k_cache, uint16_t *v_cache, const int64_t *src,
+                       const int64_t *dst, int64_t n, int num_kv_heads, int head_dim,
+                       int64_t num_blocks) {
+    for (int64_t i = 0; i < n; ++i)
+        if (src[i] < 0 || src[i] >= num_blocks || dst[i] < 0 || dst[i] >= num_blocks) return -1;
+    for (int64_t i = 0; i < n; ++i)
+        for (int h = 0; h < num_kv_heads; ++h)
+            for (int off = 0; off < ORACLE_BLOCK_TOKENS; ++off)
+                for (int e = 0; e < head_dim; ++e) {
+                    size_t from = cache_index(src[i], h, off, e, num_kv_heads, head_dim);
+                    size_t to = cache_index(dst[i], h, off, e, num_kv_heads, head_dim);
+                    k_cache[to] = k_cache[from];
+                    v_cache[to] = v_cache[from];
+                }
+    return 0;
+}
+
+/*
  * Copy the logical K and V rows of one sequence and KV head, in token order,
  * through the block table (section 二: logical block p/16 -> physical block).
  * Returns -1 if a table entry on the path is outside [0, num_blocks).

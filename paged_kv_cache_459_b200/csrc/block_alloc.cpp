@@ -39,6 +39,8 @@ struct pkv_alloc {
     std::deque<int32_t> free_list;
     std::vector<int32_t> refcount;
     std::unordered_map<int64_t, Sequence> seqs;
+    // Copy-on-write block copies (src, dst) not yet taken by the caller.
+    std::vector<std::pair<int32_t, int32_t>> pending_copies;
 };
 
 extern "C" {
@@ -113,19 +115,29 @@ pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, int64_t n
     return PKV_OK;
 }
 
-// Checks one append; returns whether it needs a new block.
-static pkv_status check_append(const pkv_alloc *a, const Sequence &s, bool *needs_block) {
-    *needs_block = (s.len % kBlockTokens) == 0;
-    if (!*needs_block && a->refcount[s.blocks.back()] > 1) return PKV_ERR_UNSUPPORTED;
-    return PKV_OK;
+// What appending one token to a sequence takes: room in its last block, a
+// fresh block (none yet, or the last one is full), or a copy-on-write of a
+// partly filled last block that other tables also hold.
+enum class AppendKind { kInPlace, kNewBlock, kCopyOnWrite };
+
+static AppendKind append_kind(const Sequence &s, int32_t last_refcount) {
+    if (s.len % kBlockTokens == 0) return AppendKind::kNewBlock;
+    return last_refcount > 1 ? AppendKind::kCopyOnWrite : AppendKind::kInPlace;
 }
 
-static int64_t do_append(pkv_alloc *a, Sequence &s, bool needs_block) {
-    if (needs_block) {
+static int64_t do_append(pkv_alloc *a, Sequence &s, AppendKind kind) {
+    if (kind != AppendKind::kInPlace) {
         int32_t b = a->free_list.front();
         a->free_list.pop_front();
         a->refcount[b] = 1;
-        s.blocks.push_back(b);
+        if (kind == AppendKind::kNewBlock) {
+            s.blocks.push_back(b);
+        } else {  // the sequence gets a private copy of its shared last block
+            const int32_t old = s.blocks.back();
+            a->refcount[old] -= 1;  // still >= 1: other tables hold it
+            a->pending_copies.emplace_back(old, b);
+            s.blocks.back() = b;
+        }
     }
     int64_t pos = s.len++;
     return static_cast<int64_t>(s.blocks[pos / kBlockTokens]) * kBlockTokens + pos % kBlockTokens;
@@ -135,45 +147,69 @@ pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_ou
     if (!a || !slot_out) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(seq_id);
     if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
-    bool needs_block;
-    pkv_status st = check_append(a, it->second, &needs_block);
-    if (st != PKV_OK) return st;
-    if (needs_block && a->free_list.empty()) return PKV_ERR_OOM;
+    Sequence &s = it->second;
+    const AppendKind kind = append_kind(s, s.blocks.empty() ? 0 : a->refcount[s.blocks.back()]);
+    if (kind != AppendKind::kInPlace && a->free_list.empty()) return PKV_ERR_OOM;
     try {
-        if (needs_block) it->second.blocks.reserve(it->second.blocks.size() + 1);
+        if (kind == AppendKind::kNewBlock) s.blocks.reserve(s.blocks.size() + 1);
+        if (kind == AppendKind::kCopyOnWrite) a->pending_copies.reserve(a->pending_copies.size() + 1);
     } catch (const std::bad_alloc &) {
         return PKV_ERR_OOM;
     }
-    *slot_out = do_append(a, it->second, needs_block);
+    *slot_out = do_append(a, s, kind);
     return PKV_OK;
 }
 
 pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *slots_out) {
     if (!a || n < 0 || (n > 0 && (!seq_ids || !slots_out))) return PKV_ERR_INVALID_ARG;
     std::vector<Sequence *> seqs;
-    std::vector<char> needs;
+    std::vector<AppendKind> kinds;
     try {
         std::unordered_set<int64_t> seen;
+        std::unordered_map<int32_t, int32_t> released;  // copy-on-writes earlier in this batch
         seqs.reserve(static_cast<size_t>(n));
-        needs.reserve(static_cast<size_t>(n));
-        int64_t new_blocks = 0;
+        kinds.reserve(static_cast<size_t>(n));
+        int64_t new_blocks = 0, cows = 0;
         for (int i = 0; i < n; ++i) {
             if (!seen.insert(seq_ids[i]).second) return PKV_ERR_INVALID_ARG;
             auto it = a->seqs.find(seq_ids[i]);
             if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
-            bool nb;
-            pkv_status st = check_append(a, it->second, &nb);
-            if (st != PKV_OK) return st;
-            if (nb) it->second.blocks.reserve(it->second.blocks.size() + 1);
-            new_blocks += nb;
-            seqs.push_back(&it->second);
-            needs.push_back(nb);
+            Sequence &s = it->second;
+            int32_t rc = 0;
+            if (!s.blocks.empty()) {
+                auto r = released.find(s.blocks.back());
+                rc = a->refcount[s.blocks.back()] - (r == released.end() ? 0 : r->second);
+            }
+            const AppendKind kind = append_kind(s, rc);
+            if (kind == AppendKind::kNewBlock) s.blocks.reserve(s.blocks.size() + 1);
+            if (kind == AppendKind::kCopyOnWrite) {
+                released[s.blocks.back()] += 1;
+                ++cows;
+            }
+            new_blocks += kind != AppendKind::kInPlace;
+            seqs.push_back(&s);
+            kinds.push_back(kind);
         }
         if (new_blocks > static_cast<int64_t>(a->free_list.size())) return PKV_ERR_OOM;
+        a->pending_copies.reserve(a->pending_copies.size() + static_cast<size_t>(cows));
     } catch (const std::bad_alloc &) {
         return PKV_ERR_OOM;
     }
-    for (int i = 0; i < n; ++i) slots_out[i] = do_append(a, *seqs[i], needs[i] != 0);
+    for (int i = 0; i < n; ++i) slots_out[i] = do_append(a, *seqs[i], kinds[i]);
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_take_copies(pkv_alloc *a, int64_t *src_out, int64_t *dst_out, int64_t cap,
+                                 int64_t *n_out) {
+    if (!a || !n_out || cap < 0 || (cap > 0 && (!src_out || !dst_out))) return PKV_ERR_INVALID_ARG;
+    const int64_t n = static_cast<int64_t>(a->pending_copies.size());
+    *n_out = n;
+    if (cap < n) return PKV_OK;  // nothing taken: ask again with room for all
+    for (int64_t i = 0; i < n; ++i) {
+        src_out[i] = a->pending_copies[static_cast<size_t>(i)].first;
+        dst_out[i] = a->pending_copies[static_cast<size_t>(i)].second;
+    }
+    a->pending_copies.clear();
     return PKV_OK;
 }
 

@@ -15,7 +15,7 @@
 // kernel starting past the prefix, and the merge below combines prefix and
 // suffix partials of each (sequence, query head) by log-sum-exp.  The result
 // equals plain decode over the whole sequence.
-#include "decode_common.cuh"
+#include "decode_unit.cuh"
 
 namespace pkv {
 
@@ -26,13 +26,19 @@ using namespace dev;
 constexpr int kPrefixWarps = 4;
 
 template <int D, int CB>
-__global__ void __launch_bounds__(kPrefixWarps * 32)
-    prefix_chunk_kernel(const __grid_constant__ CUtensorMap tmk,
-                        const __grid_constant__ CUtensorMap tmv, const PrefixParams p) {
+struct PrefixGeometry {
+    static constexpr int kTile = (D / 64) * kBoxBytes;  // one K or V tile of a block
+    static constexpr int kSmemBytes = 2 * CB * kTile + 8 + CB * 4 + 1024;
+};
+
+// Prefix chunk c (blocks [c*CB, (c+1)*CB) of group g's shared prefix) for KV
+// head kvh: all member rows against the chunk's K/V, one partial per row.
+template <int D, int CB>
+__device__ __forceinline__ void prefix_unit(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                            const PrefixParams &p, int c, int kvh, int g) {
     constexpr int KS = D / 16;                     // k-steps of S = Q K^T over d
     constexpr int NT = D / 8;                      // 8-column tiles of O
-    constexpr int kTile = (D / 64) * kBoxBytes;    // one K or V tile of a block
-    const int c = blockIdx.x, kvh = blockIdx.y, g = blockIdx.z;
+    constexpr int kTile = PrefixGeometry<D, CB>::kTile;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tig = lane & 3, gid = lane >> 2;
 
@@ -216,8 +222,8 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
 }
 
 // Merge of one (sequence, query head): prefix chunks [0, ceil(pb / CB)) and
-// the suffix split-K partitions that hold tokens past the prefix, in index
-// order, by log-sum-exp.
+// the suffix split-K partitions that hold tokens past the prefix (counted
+// from the prefix end), in slot order, by log-sum-exp with a running maximum.
 template <int D, int CB>
 __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) {
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
@@ -226,67 +232,83 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
     const int pb = min(max(__ldg(p.prefix_blocks + b), 0), len / kBlockTokens);
     const int nchunks = (pb + CB - 1) / CB;
+    const int nsuffix = (nblk - pb + p.part_blocks - 1) / p.part_blocks;
     const size_t row = static_cast<size_t>(b) * p.Hq + h;
     const float *ml = p.ws_ml + 2 * row * p.ws_parts;
     const float *o = p.ws_o + row * p.ws_parts * D;
-    const auto used = [&](int part) {  // slot `part` holds a partial for this row
-        if (part < p.prefix_parts) return part < nchunks;
-        const int q = part - p.prefix_parts;
-        return max(q * p.part_blocks, pb) < min((q + 1) * p.part_blocks, nblk);
+    float M = -INFINITY, L = 0.f, O = 0.f;
+    const auto add = [&](int slot) {
+        const float2 v = *reinterpret_cast<const float2 *>(ml + 2 * slot);  // (m, l)
+        const float x = o[static_cast<size_t>(slot) * D + e];
+        if (v.x == -INFINITY) return;
+        const float Mn = fmaxf(M, v.x);
+        const float a = exp2f(M - Mn), c = exp2f(v.x - Mn);
+        L = L * a + v.y * c;
+        O = O * a + x * c;
+        M = Mn;
     };
-    float M = -INFINITY;
-    for (int q = 0; q < p.ws_parts; ++q)
-        if (used(q)) M = fmaxf(M, ml[2 * q]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-        for (int q = 0; q < p.ws_parts; ++q) {
-            if (!used(q)) continue;
-            const float c = exp2f(ml[2 * q] - M);
-            L = fmaf(ml[2 * q + 1], c, L);
-            O = fmaf(o[static_cast<size_t>(q) * D + e], c, O);
-        }
-    }
+    for (int q = 0; q < nchunks; ++q) add(q);
+    for (int q = 0; q < nsuffix; ++q) add(p.prefix_parts + q);
     p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
 }
 
-template <int D>
-cudaError_t launch_prefix_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &p,
-                            int num_groups, cudaStream_t stream) {
-    constexpr int CB = kPrefixChunkBlocks;
-    constexpr int kTile = (D / 64) * kBoxBytes;
-    constexpr int kSmem = 2 * CB * kTile + 8 + CB * 4 + 1024;
-    auto kern = prefix_chunk_kernel<D, CB>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    if (num_groups > 0) {
-        const dim3 grid(static_cast<unsigned>(p.prefix_parts), static_cast<unsigned>(p.Hkv),
-                        static_cast<unsigned>(num_groups));
-        kern<<<grid, kPrefixWarps * 32, kSmem, stream>>>(tmk, tmv, p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+// One launch for the prefix chunks and the suffix split-K units: CTAs
+// [0, n_pre) take prefix chunks (chunk fastest, then KV head, then group), the
+// rest take suffix units (partition fastest, then head segment, then
+// sequence).  The prefix work is short and latency-bound; running it beside
+// the bandwidth-bound suffix stream hides it.
+template <int D, bool MMA>
+__global__ void __launch_bounds__(kPrefixWarps * 32)
+    cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                   const PrefixParams pp, const DecodeParams dp, int n_pre) {
+    int id = blockIdx.x;
+    if (id < n_pre) {
+        const int c = id % pp.prefix_parts;
+        id /= pp.prefix_parts;
+        prefix_unit<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
+        return;
     }
-    return cudaSuccess;
+    id -= n_pre;
+    const int ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
+    const int part = id % dp.num_parts;
+    id /= dp.num_parts;
+    decode_unit<D, kPrefixWarps, 2, MMA, true>(tmk, tmv, dp, part, id % ny, id / ny);
 }
 
-template <int D>
-cudaError_t launch_cascade_merge_d(const PrefixParams &p, cudaStream_t stream) {
+template <int D, bool MMA>
+cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
+                             const DecodeParams &dp, int num_groups, cudaStream_t stream) {
+    constexpr int kSmem = PrefixGeometry<D, kPrefixChunkBlocks>::kSmemBytes >
+                                  Geometry<D, kPrefixWarps, 2>::kSmemBytes
+                              ? PrefixGeometry<D, kPrefixChunkBlocks>::kSmemBytes
+                              : Geometry<D, kPrefixWarps, 2>::kSmemBytes;
+    auto kern = cascade_kernel<D, MMA>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    const long long n_pre = static_cast<long long>(pp.prefix_parts) * pp.Hkv * num_groups;
+    const long long ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
+    const long long n_suf = static_cast<long long>(dp.num_parts) * ny * dp.B;
+    if (n_pre + n_suf >= (1ll << 31)) return cudaErrorInvalidValue;
+    kern<<<static_cast<unsigned>(n_pre + n_suf), kPrefixWarps * 32, kSmem, stream>>>(
+        tmk, tmv, pp, dp, static_cast<int>(n_pre));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cascade_merge_kernel<D, kPrefixChunkBlocks>
-        <<<dim3(static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B)), D, 0, stream>>>(p);
+        <<<dim3(static_cast<unsigned>(pp.Hq), static_cast<unsigned>(pp.B)), D, 0, stream>>>(pp);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefix_chunks(const CUtensorMap &tmk, const CUtensorMap &tmv,
-                                 const PrefixParams &p, int head_dim, int num_groups,
-                                 cudaStream_t stream) {
-    if (head_dim == 128) return launch_prefix_d<128>(tmk, tmv, p, num_groups, stream);
-    if (head_dim == 64) return launch_prefix_d<64>(tmk, tmv, p, num_groups, stream);
-    return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_cascade_merge(const PrefixParams &p, int head_dim, cudaStream_t stream) {
-    if (head_dim == 128) return launch_cascade_merge_d<128>(p, stream);
-    if (head_dim == 64) return launch_cascade_merge_d<64>(p, stream);
+cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
+                           const DecodeParams &dp, int head_dim, int num_groups,
+                           cudaStream_t stream) {
+    const bool mma = dp.group > 1;
+    if (head_dim == 128)
+        return mma ? launch_cascade_d<128, true>(tmk, tmv, pp, dp, num_groups, stream)
+                   : launch_cascade_d<128, false>(tmk, tmv, pp, dp, num_groups, stream);
+    if (head_dim == 64)
+        return mma ? launch_cascade_d<64, true>(tmk, tmv, pp, dp, num_groups, stream)
+                   : launch_cascade_d<64, false>(tmk, tmv, pp, dp, num_groups, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -1,0 +1,166 @@
+// The per-unit decode kernel body (single pass and split-K), shared by the
+// plain decode launch and the shared-prefix launch that runs it beside the
+// prefix kernel.  Method, layouts and tiling: see decode.cu.
+#pragma once
+
+#include "decode_common.cuh"
+
+namespace pkv {
+namespace dev {
+
+// One work unit (partition `part` of sequence b, KV head / head chunk `by`)
+// of the per-unit decode kernel, run by a CTA of NW warps.
+template <int D, int NW, int S, bool MMA, bool SPLIT>
+__device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                            const DecodeParams &p, int part, int by, int b) {
+    using G = Geometry<D, NW, S>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kvh = MMA ? by / p.chunks : by;
+    const int chunk = MMA ? by % p.chunks : 0;
+    const int h0 = MMA ? kvh * p.group + chunk * 8 : kvh;  // first query head of this CTA
+    const int heads = MMA ? min(8, p.group - chunk * 8) : 1;
+
+    int len = __ldg(p.seq_lens + b);
+    if (len < 0 || len > p.W * kBlockTokens) {
+        if (threadIdx.x == 0 && part == 0 && by == 0) flag(p.err, PKV_DEV_ERR_BAD_LEN);
+        len = len < 0 ? 0 : p.W * kBlockTokens;
+    }
+    const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
+    int start = 0;
+    if (p.start_blocks != nullptr) start = min(max(__ldg(p.start_blocks + b), 0), len / kBlockTokens);
+    // Partitions are counted from the start block.
+    const int blk_begin = start + part * p.part_blocks;
+    const int blk_end = min(nblk, start + (part + 1) * p.part_blocks);
+    if (blk_begin >= blk_end) {
+        // Nothing to read.  Single pass: the (empty) sequence's rows are zero.
+        // Split-K: the merge kernel only reads partitions that hold tokens.
+        if (!SPLIT)
+            for (int i = threadIdx.x; i < heads * D; i += NW * 32)
+                p.out[(static_cast<size_t>(b) * p.Hq + h0 + i / D) * D + i % D] = __float2bfloat16(0.f);
+        return;
+    }
+
+    extern __shared__ uint8_t smem_raw[];
+    // Stage buffers must sit on 1024-byte boundaries for the 128-byte swizzle.
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *ring = smem + warp * S * G::kStageBytes;
+    const uint32_t bars = smem_u32(smem + G::kRingBytes) + warp * S * 8;
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(bars + 8 * s, 1);
+        fence_mbar_init();
+    }
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+    }
+    __syncthreads();
+
+    const int n_mine = blk_end - blk_begin > warp ? (blk_end - blk_begin - warp + NW - 1) / NW : 0;
+    TableWindow tw;
+    tw.row = p.block_tables + static_cast<size_t>(b) * p.W;
+    tw.first = blk_begin + warp;
+    tw.stride = NW;
+    tw.count = n_mine;
+    tw.init(lane);
+    const uint64_t policy = l2_policy_evict_first();
+    const int y_head = kvh * kBlockTokens;
+
+    auto issue = [&](int i) {  // warp-uniform
+        const int32_t phys = tw.get(i);
+        if (lane == 0) {
+            const uint32_t bar = bars + 8 * (i % S);
+            if (phys >= 0 && phys < p.num_blocks) {
+                const uint32_t dst = smem_u32(ring + (i % S) * G::kStageBytes);
+                const int y = phys * (p.Hkv * kBlockTokens) + y_head;
+                mbar_arrive_expect_tx(bar, G::kStageBytes);
+#pragma unroll
+                for (int hh = 0; hh < G::kHalves; ++hh) {
+                    tma_load_2d(dst + hh * kBoxBytes, &tmk, hh * 64, y, bar, policy);
+                    tma_load_2d(dst + G::kTileBytes + hh * kBoxBytes, &tmv, hh * 64, y, bar, policy);
+                }
+            } else {
+                flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
+                mbar_arrive(bar);  // an empty phase: the consumer skips the block
+            }
+        }
+    };
+
+    using Head = typename std::conditional<MMA, GroupHeads<D>, ScalarHead<D>>::type;
+    Head st;
+    if constexpr (MMA)
+        st.init(p.q + (static_cast<size_t>(b) * p.Hq + h0) * D, heads, p.scale_log2, lane);
+    else
+        st.init(p.q + (static_cast<size_t>(b) * p.Hq + h0) * D, p.scale_log2, lane);
+
+    for (int i = 0; i < S && i < n_mine; ++i) issue(i);
+
+    int i = 0;
+    for (; i < n_mine; ++i) {
+        tw.advance_to(i, lane);
+        const int s = i % S;
+        if (!mbar_wait(bars + 8 * s, static_cast<uint32_t>((i / S) & 1), kWaitLimitNs)) {
+            if (lane == 0) flag(p.err, PKV_DEV_ERR_TIMEOUT);
+            break;
+        }
+        const int32_t phys = tw.get(i);
+        if (phys >= 0 && phys < p.num_blocks) {
+            const int lb = blk_begin + warp + NW * i;
+            const int nvalid = min(kBlockTokens, len - lb * kBlockTokens);
+            const uint8_t *kt = ring + s * G::kStageBytes;
+            if constexpr (MMA)
+                st.tile(smem_u32(kt), smem_u32(kt + G::kTileBytes), nvalid, lane);
+            else
+                st.tile(kt, kt + G::kTileBytes, nvalid, lane);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (i + S < n_mine) issue(i + S);
+    }
+    if (i < n_mine) {
+        // A wait gave up: let the copies still in flight land before the
+        // shared memory is reused or released (again bounded).
+        for (int j = i; j < n_mine && j < i + S; ++j)
+            mbar_wait(bars + 8 * (j % S), static_cast<uint32_t>((j / S) & 1), kWaitLimitNs);
+    }
+
+    // ---- combine the warps of this CTA (all rings are drained) ----
+    __syncthreads();
+    constexpr int kRed = MMA ? 16 + 8 * D : D + 2;
+    float *red = reinterpret_cast<float *>(smem);
+    st.finish(red + warp * kRed, lane);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < heads * D; idx += NW * 32) {
+        const int n = idx / D, e = idx % D;
+        float mw[NW];
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            mw[w] = MMA ? red[w * kRed + n] : red[w * kRed + D];
+            M = fmaxf(M, mw[w]);
+        }
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float c = exp2f(mw[w] - M);
+                L = fmaf(MMA ? red[w * kRed + 8 + n] : red[w * kRed + D + 1], c, L);
+                O = fmaf(MMA ? red[w * kRed + 16 + n * D + e] : red[w * kRed + e], c, O);
+            }
+        }
+        const size_t row = static_cast<size_t>(b) * p.Hq + h0 + n;
+        if constexpr (SPLIT) {
+            const size_t pr = row * p.ws_parts + p.ws_part0 + part;
+            p.ws_o[pr * D + e] = O;
+            if (e == 0) {
+                p.ws_ml[2 * pr] = M;
+                p.ws_ml[2 * pr + 1] = L;
+            }
+        } else {
+            p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
+        }
+    }
+}
+
+}  // namespace dev
+}  // namespace pkv

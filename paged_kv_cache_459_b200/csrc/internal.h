@@ -98,10 +98,15 @@ struct PrefixParams {
     float scale_log2;
 };
 
-cudaError_t launch_prefix_chunks(const CUtensorMap &tmk, const CUtensorMap &tmv,
-                                 const PrefixParams &p, int head_dim, int num_groups,
-                                 cudaStream_t stream);
-cudaError_t launch_cascade_merge(const PrefixParams &p, int head_dim, cudaStream_t stream);
+// One launch running prefix chunks and suffix split-K units side by side,
+// then the merge.  dp must describe split-K with start_blocks = prefix_blocks.
+cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
+                           const DecodeParams &dp, int head_dim, int num_groups,
+                           cudaStream_t stream);
+
+cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, const int64_t *dst,
+                               int n, int num_kv_heads, int head_dim, long long num_blocks,
+                               unsigned int *err, cudaStream_t stream);
 
 cudaError_t launch_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
                             const int64_t *slot_mapping, int num_tokens, int num_kv_heads,

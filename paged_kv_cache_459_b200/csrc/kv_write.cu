@@ -6,6 +6,8 @@
 // the same thread.  A few MB per decode step at most, so the kernel is
 // launch- and latency-bound; coalesced 16-byte loads and stores are all it
 // needs.  Bit-exact: plain copies, no arithmetic on the values.
+#include <algorithm>
+
 #include "../../include/pkv.h"
 #include "internal.h"
 
@@ -52,6 +54,38 @@ cudaError_t launch_kv_write(const void *k, const void *v, void *k_cache, void *v
         static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(k_cache),
         static_cast<uint4 *>(v_cache), slot_mapping, total, vec_per_row, num_kv_heads, num_blocks,
         err);
+    return cudaGetLastError();
+}
+
+// Whole-block copies (copy-on-write): pair blockIdx.y, 16-byte vectors over
+// the block's Hkv x 16 x d elements of both caches.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ k_cache,
+                                                          uint4 *__restrict__ v_cache,
+                                                          const int64_t *__restrict__ src,
+                                                          const int64_t *__restrict__ dst,
+                                                          long long vec_per_block,
+                                                          long long num_blocks, unsigned int *err) {
+    const long long s = src[blockIdx.y], d = dst[blockIdx.y];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+        if (err != nullptr && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(err, PKV_DEV_ERR_BAD_BLOCK);
+        return;
+    }
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < vec_per_block;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        k_cache[d * vec_per_block + i] = k_cache[s * vec_per_block + i];
+        v_cache[d * vec_per_block + i] = v_cache[s * vec_per_block + i];
+    }
+}
+
+cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, const int64_t *dst,
+                               int n, int num_kv_heads, int head_dim, long long num_blocks,
+                               unsigned int *err, cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    const long long vec = static_cast<long long>(num_kv_heads) * kBlockTokens * head_dim / 8;
+    const long long per_cta = 256 * 4;
+    const unsigned gx = static_cast<unsigned>(std::min<long long>((vec + per_cta - 1) / per_cta, 1024));
+    copy_blocks_kernel<<<dim3(gx, static_cast<unsigned>(n)), 256, 0, stream>>>(
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), src, dst, vec, num_blocks, err);
     return cudaGetLastError();
 }
 

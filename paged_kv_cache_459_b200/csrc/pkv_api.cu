@@ -104,6 +104,19 @@ pkv_status pkv_paged_kv_write(const void *k, const void *v, void *k_cache, void 
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, const int64_t *dst,
+                           int n, int num_kv_heads, int head_dim, int64_t num_blocks,
+                           unsigned int *err_word, void *stream) {
+    if (n < 0 || n > 65535 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 || num_blocks <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (n == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !src || !dst || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_INVALID_ARG;
+    cudaError_t e = pkv::launch_copy_blocks(k_cache, v_cache, src, dst, n, num_kv_heads, head_dim,
+                                            num_blocks, err_word, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                   int max_blocks_per_seq, int partition_tokens) {
     if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0) return 0;
@@ -380,13 +393,8 @@ pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const voi
     dp.start_blocks = prefix_blocks;
     dp.skip_merge = true;
 
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = pkv::launch_prefix_chunks(tmk, tmv, pp, head_dim, num_groups, st);
-    if (e == cudaSuccess) {
-        pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
-        e = pkv::launch_decode(tmk, tmv, dp, head_dim, true, t, st);
-    }
-    if (e == cudaSuccess) e = pkv::launch_cascade_merge(pp, head_dim, st);
+    cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
+                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -59,6 +59,8 @@ _sigs = {
     "pkv_alloc_stats": ([_P, _P, _P, _P, _P], _i32),
     "pkv_alloc_free_list": ([_P, _P, _i64, _P], _i32),
     "pkv_alloc_refcount": ([_P, _i64, _P], _i32),
+    "pkv_alloc_take_copies": ([_P, _P, _P, _i64, _P], _i32),
+    "pkv_copy_blocks": ([_P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P], _i32),
     "pkv_alloc_prefix_groups": ([_P, _P, _i32, _P, _P, _P, _P], _i32),
     "pkv_decode_prefix_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
     "pkv_paged_attention_decode_prefix": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
@@ -134,6 +136,21 @@ def paged_kv_write(k, v, k_cache, v_cache, slot_mapping, err=None) -> None:
     ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
     _check(_lib.pkv_paged_kv_write(*ptrs, sp, T, hkv, d, k_cache.shape[0], ep,
                                    _stream_ptr(k.device)), "pkv_paged_kv_write")
+
+
+def copy_blocks(k_cache, v_cache, src, dst, err=None) -> None:
+    """Copy whole blocks src[i] -> dst[i] (device int64) in both caches."""
+    import torch
+
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4 or src.shape != dst.shape:
+        raise ValueError("shape mismatch")
+    nb, hkv, bt, d = k_cache.shape
+    ptrs = [_dev_tensor(x, torch.bfloat16, n) for x, n in ((k_cache, "k_cache"), (v_cache, "v_cache"))]
+    sp = _dev_tensor(src, torch.int64, "src")
+    dp = _dev_tensor(dst, torch.int64, "dst")
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    _check(_lib.pkv_copy_blocks(*ptrs, sp, dp, src.numel(), hkv, d, nb, ep,
+                                _stream_ptr(k_cache.device)), "pkv_copy_blocks")
 
 
 _workspaces: dict = {}
@@ -321,6 +338,17 @@ class BlockAllocator:
         _acheck(_lib.pkv_alloc_free_list(self._h, out.ctypes.data if n.value else None, n.value,
                                          ctypes.byref(n)), "free_list")
         return out.tolist()
+
+    def take_copies(self):
+        """Queued copy-on-write pairs (src, dst) as int64 arrays; clears the queue."""
+        n = ctypes.c_int64()
+        _acheck(_lib.pkv_alloc_take_copies(self._h, None, None, 0, ctypes.byref(n)), "take_copies")
+        src = np.empty(n.value, np.int64)
+        dst = np.empty(n.value, np.int64)
+        _acheck(_lib.pkv_alloc_take_copies(self._h, src.ctypes.data if n.value else None,
+                                           dst.ctypes.data if n.value else None, n.value,
+                                           ctypes.byref(n)), "take_copies")
+        return src, dst
 
     def prefix_groups(self, seq_ids):
         """(prefix_blocks [n], group_offsets [G + 1], group_seqs [members]) as int32

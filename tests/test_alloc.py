@@ -96,6 +96,9 @@ def test_random_operations_match_model(seed):
         try:
             rm = {"add": m.add_seq, "append": m.append_token, "appends": m.append_tokens,
                   "fork": m.fork, "free": m.free_seq}[op](*args)
+            if op in ("append", "appends"):
+                ca, cm = a.take_copies(), m.take_copies()
+                assert all(np.array_equal(x, y) for x, y in zip(ca, cm)), (step, op)
         except ModelError as e:
             em = e.kind
         assert ea == em, (step, op, args, ea, em)
@@ -121,14 +124,20 @@ def test_failures_change_nothing():
         after = (a.free_blocks(), [a.refcount(b) for b in range(4)], a.export([0], 3))
         assert after[0] == before[0] and after[1] == before[1]
         assert np.array_equal(after[2][0], before[2][0])
-    a.fork(0, 1)
-    with pytest.raises(AllocError) as e:
-        a.append_token(1)
-    assert e.value.kind == "unsupported"
-    a.add_seq(2, 16)
-    with pytest.raises(AllocError) as e:
-        a.append_tokens([2])  # its block is full and the pool is empty
-    assert e.value.kind == "oom"
+    a.fork(0, 1)  # shares the partly filled third block
+    a.add_seq(2, 16)  # takes the last free block
+    before = (a.free_blocks(), [a.refcount(b) for b in range(4)])
+    for call in (lambda: a.append_token(1), lambda: a.append_tokens([2]),
+                 lambda: a.append_tokens([0, 1])):  # copy-on-write / new block: pool empty
+        with pytest.raises(AllocError) as e:
+            call()
+        assert e.value.kind == "oom"
+        assert (a.free_blocks(), [a.refcount(b) for b in range(4)]) == before
+    a.free_seq(2)
+    # sequence 0 comes first: it takes the copy; sequence 1 then holds the old block alone
+    assert a.append_tokens([0, 1]).tolist()[0] == a.slot_of(0, 40)
+    src, dst = a.take_copies()
+    assert src.tolist() == [a.export([1], 3)[0][0, 2]] and dst.tolist() == [a.export([0], 3)[0][0, 2]]
     with pytest.raises(AllocError):
         BlockAllocator(3, [0, 1, 1])
 

@@ -176,10 +176,12 @@ def test_allocator_errors_leave_state_unchanged():
         assert (list(bm.free), list(bm.ref), {k: list(v) for k, v in bm.tables.items()},
                 dict(bm.lens)) == before
     bm.fork(0, 1)  # shares the partly filled third block
-    with pytest.raises(Exception) as e:
-        bm.append_token(1)
-    assert e.value.kind == "unsupported"
-    bm.add_seq(2, 16)
+    shared = bm.tables[0][2]
+    slot = bm.append_token(1)  # copy-on-write: a private copy of the shared block
+    assert bm.tables[1][:2] == bm.tables[0][:2] and bm.tables[1][2] != shared
+    assert slot == bm.tables[1][2] * 16 + 8 and bm.refcount(shared) == 1
+    assert [tuple(x) for x in zip(*bm.take_copies())] == [(shared, bm.tables[1][2])]
+    assert bm.take_copies()[0].size == 0
     with pytest.raises(Exception) as e:
         bm.add_seq(3, 1)
     assert e.value.kind == "oom"
@@ -382,3 +384,36 @@ def test_planted_mistakes_are_caught(name, tmp_path):
         assert failures >= 1, f"mutation '{name}' passed every pin"
     finally:
         oracle._lib = saved
+
+
+def test_copy_on_write_beams_attend_to_their_own_tokens():
+    """Beams forked mid-block (the parent's last block is partly filled) share
+    the prefix blocks; each beam's next token triggers a private copy of the
+    shared block.  Every beam must then attend to the shared prefix plus its
+    own token only -- checked against torch fp64 attention on un-paged K/V."""
+    d, hkv, hq = 64, 2, 4
+    gen = wl.rng(31)
+    prefix_k, prefix_v = rb((40, hkv, d), gen), rb((40, hkv, d), gen)
+    nb = 32
+    bm = BlockManager(nb, gen.permutation(nb))
+    kc, vc = rb((nb, hkv, BT, d), gen), rb((nb, hkv, BT, d), gen)
+    bm.add_seq(0, 0)
+    slots = [bm.append_token(0) for _ in range(40)]
+    kc, vc = oracle.kv_write(kc, vc, prefix_k, prefix_v, np.array(slots))
+    for beam in (1, 2, 3):
+        bm.fork(0, beam)
+    beams = [0, 1, 2, 3]
+    new_k, new_v = rb((4, hkv, d), gen), rb((4, hkv, d), gen)
+    step_slots = np.array(bm.append_tokens(beams))
+    src, dst = bm.take_copies()
+    assert len(src) == 3 and len(set(dst.tolist())) == 3   # three beams copy, the last keeps it
+    kc, vc = oracle.copy_blocks(kc, vc, src, dst)
+    kc, vc = oracle.kv_write(kc, vc, new_k, new_v, step_slots)
+    tables, lens = bm.export(beams, 3)
+    q = rb((4, hq, d), gen)
+    got = oracle.paged_decode(q, kc, vc, tables, lens, 0.125)
+    ks = [np.concatenate([prefix_k, new_k[i:i + 1]]) for i in range(4)]
+    vs = [np.concatenate([prefix_v, new_v[i:i + 1]]) for i in range(4)]
+    np.testing.assert_allclose(got, sdpa_reference(q, ks, vs, 0.125), rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.copy_blocks(kc, vc, np.array([0]), np.array([nb]))
