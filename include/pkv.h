@@ -71,6 +71,10 @@ typedef enum {
 #define PKV_DEV_ERR_BAD_LEN 4u   /* decode: seq_len < 0 or > max_blocks_per_seq * 16, clamped */
 #define PKV_DEV_ERR_TIMEOUT 8u   /* a bounded pipeline wait gave up */
 
+/* Directions of a block swap between the GPU cache and host swap space. */
+#define PKV_SWAP_OUT 0 /* GPU block -> host slot */
+#define PKV_SWAP_IN 1  /* host slot -> GPU block */
+
 typedef enum {
     PKV_DECODE_AUTO = 0,   /* choose from the shapes (see pkv_paged_attention_decode) */
     PKV_DECODE_SINGLE = 1, /* one CTA per (sequence, KV head [, group of 8 query heads]) */
@@ -247,6 +251,25 @@ PKV_API pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, const int64_t *
                                    const int64_t *dst, int n, int num_kv_heads, int head_dim,
                                    int64_t num_blocks, unsigned int *err_word, void *stream);
 
+/*
+ * Block swap between the GPU cache and host swap space (the "--swap-space"
+ * of "vLLM 与 PagedAttention：大模型高性能推理服务实战", section 二 2.2: CPU
+ * memory that holds the KV of preempted requests).  host_k, host_v: pinned
+ * host buffers laid out like the caches, [num_host_blocks][Hkv][16][d] bf16,
+ * that the device can reach (page-locked, e.g. cudaHostAlloc or torch
+ * pin_memory; anything else is PKV_ERR_INVALID_ARG, checked with
+ * cudaPointerGetAttributes).  For every i: direction PKV_SWAP_OUT copies GPU
+ * block gpu_blocks[i] to host slot host_blocks[i]; PKV_SWAP_IN the reverse.
+ * gpu_blocks, host_blocks: device-readable int64 [n] (device memory).  The
+ * kernel moves the bytes itself over the host link (no staging buffer).
+ * Ids out of range are skipped and flagged PKV_DEV_ERR_BAD_BLOCK.
+ */
+PKV_API pkv_status pkv_swap_blocks(void *k_cache, void *v_cache, void *host_k, void *host_v,
+                                   const int64_t *gpu_blocks, const int64_t *host_blocks, int n,
+                                   int direction, int num_kv_heads, int head_dim,
+                                   int64_t num_blocks, int64_t num_host_blocks,
+                                   unsigned int *err_word, void *stream);
+
 /* ------------------------------------------------------------------------
  * Host block allocator (section 二 and section 三 of the first page): a pool
  * of num_blocks physical blocks with reference counts, per-sequence block
@@ -287,6 +310,28 @@ PKV_API pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids,
  * otherwise nothing is taken (call again with room for *n_out). */
 PKV_API pkv_status pkv_alloc_take_copies(pkv_alloc *a, int64_t *src_out, int64_t *dst_out,
                                          int64_t cap, int64_t *n_out);
+
+/* Host swap space of num_host_blocks slots (none by default); refused while a
+ * sequence is swapped out. */
+PKV_API pkv_status pkv_alloc_set_host_pool(pkv_alloc *a, int64_t num_host_blocks);
+
+/* Preemption: move every block of seq_id to host slots (its GPU blocks return
+ * to the pool; queued as PKV_SWAP_OUT pairs).  Refused with
+ * PKV_ERR_UNSUPPORTED if any of its blocks is shared, PKV_ERR_OOM if the host
+ * space is short.  A swapped-out sequence can only be swapped in or freed. */
+PKV_API pkv_status pkv_alloc_swap_out(pkv_alloc *a, int64_t seq_id);
+
+/* Resume: give seq_id fresh GPU blocks for its host slots (queued as
+ * PKV_SWAP_IN pairs; its table then lists the new blocks).  PKV_ERR_OOM if
+ * the GPU pool is short. */
+PKV_API pkv_status pkv_alloc_swap_in(pkv_alloc *a, int64_t seq_id);
+
+/* Takes the queued swap pairs of one direction: as pkv_alloc_take_copies,
+ * with gpu_out[i] / host_out[i] the GPU block and host slot of pair i.  Run
+ * them with pkv_swap_blocks: swap-outs before the freed GPU blocks are written
+ * again, swap-ins before the sequence is decoded. */
+PKV_API pkv_status pkv_alloc_take_swaps(pkv_alloc *a, int direction, int64_t *gpu_out,
+                                        int64_t *host_out, int64_t cap, int64_t *n_out);
 
 /* Release a sequence: every block whose count drops to zero returns to the pool. */
 PKV_API pkv_status pkv_alloc_free_seq(pkv_alloc *a, int64_t seq_id);

@@ -12,6 +12,7 @@ arithmetic.
                                combined by log-sum-exp (C, fp64).
 * ``kv_write``              -- the new token's K/V copied into its slot (C).
 * ``copy_blocks``           -- copy-on-write copies of whole blocks (C).
+* ``swap_blocks``           -- blocks moved to / from host swap space (C).
 * ``alloc_model.BlockManager`` -- the block allocator's reference model (Python).
 
 Pins (all CPU tests): the pages' worked block-table, waste and sharing
@@ -49,6 +50,8 @@ def lib() -> ctypes.CDLL:
         l.oracle_block_tokens.restype = i32
         l.oracle_copy_blocks.argtypes = [P, P, P, P, i64, i32, i32, i64]
         l.oracle_copy_blocks.restype = i32
+        l.oracle_swap_blocks.argtypes = [P, P, P, P, P, P, i64, i32, i32, i32, i64, i64]
+        l.oracle_swap_blocks.restype = i32
         _lib = l
     return _lib
 
@@ -94,6 +97,20 @@ def copy_blocks(k_cache, v_cache, src, dst):
     if lib().oracle_copy_blocks(_ptr(kc), _ptr(vc), _ptr(s), _ptr(d), len(s), hkv, hd, nb):
         raise ValueError("block id outside the pool")
     return kc, vc
+
+
+def swap_blocks(k_cache, v_cache, host_k, host_v, gpu, host, direction):
+    """(k_cache, v_cache, host_k, host_v) after moving blocks between the cache
+    and the host swap space (direction 0: out, 1: in); all copies."""
+    kc, vc = np.array(_u16(k_cache), copy=True), np.array(_u16(v_cache), copy=True)
+    hk, hv = np.array(_u16(host_k), copy=True), np.array(_u16(host_v), copy=True)
+    g = np.ascontiguousarray(gpu, dtype=np.int64)
+    h = np.ascontiguousarray(host, dtype=np.int64)
+    nb, hkv, bt, d = kc.shape
+    if lib().oracle_swap_blocks(_ptr(kc), _ptr(vc), _ptr(hk), _ptr(hv), _ptr(g), _ptr(h), len(g),
+                                int(direction), hkv, d, nb, hk.shape[0]):
+        raise ValueError("block id outside the pool or the swap space")
+    return kc, vc, hk, hv
 
 
 def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, nthreads: int = 0):

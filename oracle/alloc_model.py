@@ -22,6 +22,10 @@ Readings where the pages are silent:
     copy-on-write: the sequence takes a fresh block in its place and the pair
     (shared block, fresh block) is queued for the caller to copy on the device
     (beam candidates share prefix blocks -- "vllm", PagedAttention 的核心原理);
+  * swap space (P3 section 二 2.2, --swap-space): a sequence whose blocks are
+    all unshared can be moved to host slots (its GPU blocks return to the
+    pool) and later back into fresh GPU blocks; the moves are queued as
+    (GPU block, host slot) pairs; while out it can only come back or be freed;
   * every failing call leaves the state exactly as it was.
 """
 from __future__ import annotations
@@ -52,6 +56,9 @@ class BlockManager:
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
         self.copies: list[tuple[int, int]] = []
+        self.host_free: deque = deque()
+        self.swapped: set = set()
+        self.moves = {0: [], 1: []}  # 0: out (gpu -> host), 1: in (host -> gpu)
 
     # -- lifecycle ---------------------------------------------------------
     def add_seq(self, seq_id: int, num_tokens: int) -> None:
@@ -67,8 +74,8 @@ class BlockManager:
         self.lens[seq_id] = num_tokens
 
     def append_token(self, seq_id: int) -> int:
-        if seq_id not in self.tables:
-            raise AllocError("invalid", "unknown sequence")
+        if seq_id not in self.tables or seq_id in self.swapped:
+            raise AllocError("invalid", "unknown or swapped-out sequence")
         blocks, pos = self.tables[seq_id], self.lens[seq_id]
         if pos % BLOCK_TOKENS == 0:
             if not self.free:
@@ -92,7 +99,7 @@ class BlockManager:
         an unknown or repeated id, then a shortage of free blocks (fresh and
         copy-on-write blocks together) is reported before anything changes."""
         ids = list(seq_ids)
-        if len(set(ids)) != len(ids) or any(s not in self.tables for s in ids):
+        if len(set(ids)) != len(ids) or any(s not in self.tables or s in self.swapped for s in ids):
             raise AllocError("invalid", "unknown or repeated sequence")
         need, released = 0, {}
         for s in ids:
@@ -116,7 +123,7 @@ class BlockManager:
         return src, dst
 
     def fork(self, parent: int, child: int, num_tokens: int | None = None) -> None:
-        if parent not in self.tables or child in self.tables:
+        if parent not in self.tables or parent in self.swapped or child in self.tables:
             raise AllocError("invalid", "unknown parent or existing child")
         n = self.lens[parent] if num_tokens is None or num_tokens < 0 else num_tokens
         if n > self.lens[parent]:
@@ -129,11 +136,60 @@ class BlockManager:
     def free_seq(self, seq_id: int) -> None:
         if seq_id not in self.tables:
             raise AllocError("invalid", "unknown sequence")
-        for b in self.tables.pop(seq_id):
-            self.ref[b] -= 1
-            if self.ref[b] == 0:
-                self.free.append(b)
+        if seq_id in self.swapped:
+            self.host_free.extend(self.tables.pop(seq_id))
+            self.swapped.discard(seq_id)
+        else:
+            for b in self.tables.pop(seq_id):
+                self.ref[b] -= 1
+                if self.ref[b] == 0:
+                    self.free.append(b)
         del self.lens[seq_id]
+
+    def set_host_pool(self, n: int) -> None:
+        if n < 0 or self.swapped:
+            raise AllocError("invalid", "bad size or host slots in use")
+        self.host_free = deque(range(n))
+
+    def swap_out(self, seq_id: int) -> None:
+        if seq_id not in self.tables or seq_id in self.swapped:
+            raise AllocError("invalid", "unknown or swapped sequence")
+        blocks = self.tables[seq_id]
+        if any(self.ref[b] != 1 for b in blocks):
+            raise AllocError("unsupported", "shared blocks stay on the GPU")
+        if len(blocks) > len(self.host_free):
+            raise AllocError("oom")
+        slots = []
+        for b in blocks:
+            h = self.host_free.popleft()
+            self.moves[0].append((b, h))
+            self.ref[b] = 0
+            self.free.append(b)
+            slots.append(h)
+        self.tables[seq_id] = slots
+        self.swapped.add(seq_id)
+
+    def swap_in(self, seq_id: int) -> None:
+        if seq_id not in self.swapped:
+            raise AllocError("invalid", "not swapped out")
+        slots = self.tables[seq_id]
+        if len(slots) > len(self.free):
+            raise AllocError("oom")
+        blocks = []
+        for h in slots:
+            b = self.free.popleft()
+            self.ref[b] = 1
+            self.moves[1].append((b, h))
+            self.host_free.append(h)
+            blocks.append(b)
+        self.tables[seq_id] = blocks
+        self.swapped.discard(seq_id)
+
+    def take_swaps(self, direction: int):
+        import numpy as np
+
+        pairs, self.moves[direction] = self.moves[direction], []
+        return (np.array([p[0] for p in pairs], np.int64), np.array([p[1] for p in pairs], np.int64))
 
     # -- views -------------------------------------------------------------
     def export(self, seq_ids, width: int):
@@ -142,8 +198,8 @@ class BlockManager:
         tables = np.full((len(seq_ids), width), -1, dtype=np.int32)
         lens = np.zeros(len(seq_ids), dtype=np.int32)
         for i, s in enumerate(seq_ids):
-            if s not in self.tables:
-                raise AllocError("invalid", "unknown sequence")
+            if s not in self.tables or s in self.swapped:
+                raise AllocError("invalid", "unknown or swapped-out sequence")
             blocks = self.tables[s]
             if len(blocks) > width:
                 raise AllocError("invalid", "table wider than the export width")
@@ -155,7 +211,7 @@ class BlockManager:
         return list(self.free)
 
     def slot_of(self, seq_id: int, pos: int) -> int:
-        if not 0 <= pos < self.lens[seq_id]:
+        if seq_id in self.swapped or not 0 <= pos < self.lens[seq_id]:
             raise AllocError("invalid", "position outside the sequence")
         return self.tables[seq_id][pos // BLOCK_TOKENS] * BLOCK_TOKENS + pos % BLOCK_TOKENS
 
@@ -168,6 +224,8 @@ class BlockManager:
         import numpy as np
 
         ids = list(seq_ids)
+        if any(s not in self.tables or s in self.swapped for s in ids):
+            raise AllocError("invalid", "unknown or swapped-out sequence")
         by_first: dict[int, list[int]] = {}
         for i, s in enumerate(ids):
             if self.lens[s] >= BLOCK_TOKENS and self.ref[self.tables[s][0]] >= 2:
@@ -201,6 +259,8 @@ class BlockManager:
         shared = sum(1 for r in self.ref if r > 1)
         fill = {}
         for s, blocks in self.tables.items():
+            if s in self.swapped:
+                continue
             n = self.lens[s]
             for j, b in enumerate(blocks):
                 fill[b] = max(fill.get(b, 0), min(BLOCK_TOKENS, n - j * BLOCK_TOKENS))

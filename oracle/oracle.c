@@ -103,6 +103,36 @@ int oracle_copy_blocks(uint16_t *k_cache, uint16_t *v_cache, const int64_t *src,
 }
 
 /*
+ * Swap space ("vLLM 与 PagedAttention：大模型高性能推理服务实战", section 二
+ * 2.2, --swap-space: host memory for the KV of preempted requests).  Host
+ * slots are laid out like cache blocks.  direction 0: GPU block gpu[i] ->
+ * host slot host[i]; direction 1: the reverse.  Returns 0, or -1 on an id out
+ * of range (nothing moved then).
+ */
+int oracle_swap_blocks(uint16_t *k_cache, uint16_t *v_cache, uint16_t *host_k, uint16_t *host_v,
+                       const int64_t *gpu, const int64_t *host, int64_t n, int direction,
+                       int num_kv_heads, int head_dim, int64_t num_blocks, int64_t num_host_blocks) {
+    for (int64_t i = 0; i < n; ++i)
+        if (gpu[i] < 0 || gpu[i] >= num_blocks || host[i] < 0 || host[i] >= num_host_blocks)
+            return -1;
+    for (int64_t i = 0; i < n; ++i)
+        for (int h = 0; h < num_kv_heads; ++h)
+            for (int off = 0; off < ORACLE_BLOCK_TOKENS; ++off)
+                for (int e = 0; e < head_dim; ++e) {
+                    size_t g = cache_index(gpu[i], h, off, e, num_kv_heads, head_dim);
+                    size_t c = cache_index(host[i], h, off, e, num_kv_heads, head_dim);
+                    if (direction == 0) {
+                        host_k[c] = k_cache[g];
+                        host_v[c] = v_cache[g];
+                    } else {
+                        k_cache[g] = host_k[c];
+                        v_cache[g] = host_v[c];
+                    }
+                }
+    return 0;
+}
+
+/*
  * Copy the logical K and V rows of one sequence and KV head, in token order,
  * through the block table (section 二: logical block p/16 -> physical block).
  * Returns -1 if a table entry on the path is outside [0, num_blocks).

@@ -28,8 +28,9 @@ constexpr int64_t kBlockTokens = PKV_BLOCK_TOKENS;
 int64_t blocks_for(int64_t tokens) { return (tokens + kBlockTokens - 1) / kBlockTokens; }
 
 struct Sequence {
-    std::vector<int32_t> blocks;
+    std::vector<int32_t> blocks;  // GPU blocks, or host slots while swapped out
     int64_t len = 0;
+    bool swapped = false;
 };
 
 }  // namespace
@@ -41,6 +42,11 @@ struct pkv_alloc {
     std::unordered_map<int64_t, Sequence> seqs;
     // Copy-on-write block copies (src, dst) not yet taken by the caller.
     std::vector<std::pair<int32_t, int32_t>> pending_copies;
+    // Host swap space: free host block slots, and queued moves (GPU block,
+    // host slot) out of and into the GPU pool.
+    std::deque<int32_t> host_free;
+    int64_t num_host_blocks = 0;
+    std::vector<std::pair<int32_t, int32_t>> pending_out, pending_in;
 };
 
 extern "C" {
@@ -100,7 +106,7 @@ pkv_status pkv_alloc_add_seq(pkv_alloc *a, int64_t seq_id, int64_t num_tokens) {
 pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, int64_t num_tokens) {
     if (!a) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(parent);
-    if (it == a->seqs.end() || a->seqs.count(child)) return PKV_ERR_INVALID_ARG;
+    if (it == a->seqs.end() || it->second.swapped || a->seqs.count(child)) return PKV_ERR_INVALID_ARG;
     int64_t n = num_tokens < 0 ? it->second.len : num_tokens;
     if (n > it->second.len) return PKV_ERR_INVALID_ARG;
     try {
@@ -146,7 +152,7 @@ static int64_t do_append(pkv_alloc *a, Sequence &s, AppendKind kind) {
 pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_out) {
     if (!a || !slot_out) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(seq_id);
-    if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+    if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
     Sequence &s = it->second;
     const AppendKind kind = append_kind(s, s.blocks.empty() ? 0 : a->refcount[s.blocks.back()]);
     if (kind != AppendKind::kInPlace && a->free_list.empty()) return PKV_ERR_OOM;
@@ -173,7 +179,7 @@ pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, 
         for (int i = 0; i < n; ++i) {
             if (!seen.insert(seq_ids[i]).second) return PKV_ERR_INVALID_ARG;
             auto it = a->seqs.find(seq_ids[i]);
-            if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+            if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
             Sequence &s = it->second;
             int32_t rc = 0;
             if (!s.blocks.empty()) {
@@ -217,11 +223,99 @@ pkv_status pkv_alloc_free_seq(pkv_alloc *a, int64_t seq_id) {
     if (!a) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(seq_id);
     if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
-    for (int32_t b : it->second.blocks) {
-        if (--a->refcount[b] == 0) a->free_list.push_back(b);
+    if (it->second.swapped) {
+        for (int32_t h : it->second.blocks) a->host_free.push_back(h);
+    } else {
+        for (int32_t b : it->second.blocks) {
+            if (--a->refcount[b] == 0) a->free_list.push_back(b);
+        }
     }
     a->seqs.erase(it);
     return PKV_OK;
+}
+
+pkv_status pkv_alloc_set_host_pool(pkv_alloc *a, int64_t num_host_blocks) {
+    if (!a || num_host_blocks < 0 || num_host_blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
+    for (const auto &kv : a->seqs)
+        if (kv.second.swapped) return PKV_ERR_INVALID_ARG;  // host slots in use
+    try {
+        std::deque<int32_t> fresh;
+        for (int64_t i = 0; i < num_host_blocks; ++i) fresh.push_back(static_cast<int32_t>(i));
+        a->host_free.swap(fresh);
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    a->num_host_blocks = num_host_blocks;
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_swap_out(pkv_alloc *a, int64_t seq_id) {
+    if (!a) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
+    Sequence &s = it->second;
+    for (int32_t b : s.blocks)
+        if (a->refcount[b] != 1) return PKV_ERR_UNSUPPORTED;  // shared blocks stay on the GPU
+    if (s.blocks.size() > a->host_free.size()) return PKV_ERR_OOM;
+    try {
+        a->pending_out.reserve(a->pending_out.size() + s.blocks.size());
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    for (int32_t &b : s.blocks) {
+        const int32_t h = a->host_free.front();
+        a->host_free.pop_front();
+        a->pending_out.emplace_back(b, h);
+        a->refcount[b] = 0;
+        a->free_list.push_back(b);
+        b = h;
+    }
+    s.swapped = true;
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_swap_in(pkv_alloc *a, int64_t seq_id) {
+    if (!a) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || !it->second.swapped) return PKV_ERR_INVALID_ARG;
+    Sequence &s = it->second;
+    if (s.blocks.size() > a->free_list.size()) return PKV_ERR_OOM;
+    try {
+        a->pending_in.reserve(a->pending_in.size() + s.blocks.size());
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    for (int32_t &h : s.blocks) {
+        const int32_t b = a->free_list.front();
+        a->free_list.pop_front();
+        a->refcount[b] = 1;
+        a->pending_in.emplace_back(b, h);
+        a->host_free.push_back(h);
+        h = b;
+    }
+    s.swapped = false;
+    return PKV_OK;
+}
+
+static pkv_status take_pairs(std::vector<std::pair<int32_t, int32_t>> &q, int64_t *gpu_out,
+                             int64_t *host_out, int64_t cap, int64_t *n_out) {
+    if (!n_out || cap < 0 || (cap > 0 && (!gpu_out || !host_out))) return PKV_ERR_INVALID_ARG;
+    const int64_t n = static_cast<int64_t>(q.size());
+    *n_out = n;
+    if (cap < n) return PKV_OK;
+    for (int64_t i = 0; i < n; ++i) {
+        gpu_out[i] = q[static_cast<size_t>(i)].first;
+        host_out[i] = q[static_cast<size_t>(i)].second;
+    }
+    q.clear();
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_take_swaps(pkv_alloc *a, int direction, int64_t *gpu_out, int64_t *host_out,
+                                int64_t cap, int64_t *n_out) {
+    if (!a || (direction != PKV_SWAP_OUT && direction != PKV_SWAP_IN)) return PKV_ERR_INVALID_ARG;
+    return take_pairs(direction == PKV_SWAP_OUT ? a->pending_out : a->pending_in, gpu_out, host_out,
+                      cap, n_out);
 }
 
 pkv_status pkv_alloc_export(const pkv_alloc *a, const int64_t *seq_ids, int n, int width,
@@ -230,7 +324,7 @@ pkv_status pkv_alloc_export(const pkv_alloc *a, const int64_t *seq_ids, int n, i
         return PKV_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) {
         auto it = a->seqs.find(seq_ids[i]);
-        if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+        if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
         if (static_cast<int64_t>(it->second.blocks.size()) > width || it->second.len > INT32_MAX)
             return PKV_ERR_INVALID_ARG;
     }
@@ -256,6 +350,7 @@ pkv_status pkv_alloc_stats(const pkv_alloc *a, int64_t *free_blocks, int64_t *us
         std::vector<int16_t> fill(static_cast<size_t>(a->num_blocks), 0);
         for (const auto &kv : a->seqs) {
             const Sequence &s = kv.second;
+            if (s.swapped) continue;
             for (size_t j = 0; j < s.blocks.size(); ++j) {
                 int64_t f = std::min<int64_t>(kBlockTokens, s.len - static_cast<int64_t>(j) * kBlockTokens);
                 int16_t &slot = fill[s.blocks[j]];
@@ -291,7 +386,7 @@ pkv_status pkv_alloc_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, i
     std::vector<const Sequence *> seqs(static_cast<size_t>(n));
     for (int i = 0; i < n; ++i) {
         auto it = a->seqs.find(seq_ids[i]);
-        if (it == a->seqs.end()) return PKV_ERR_INVALID_ARG;
+        if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
         seqs[i] = &it->second;
     }
     // Candidates: sequences whose first block is full and held by several tables,
@@ -350,7 +445,8 @@ pkv_status pkv_alloc_seq_len(const pkv_alloc *a, int64_t seq_id, int64_t *len_ou
 pkv_status pkv_alloc_slot_of(const pkv_alloc *a, int64_t seq_id, int64_t pos, int64_t *slot_out) {
     if (!a || !slot_out) return PKV_ERR_INVALID_ARG;
     auto it = a->seqs.find(seq_id);
-    if (it == a->seqs.end() || pos < 0 || pos >= it->second.len) return PKV_ERR_INVALID_ARG;
+    if (it == a->seqs.end() || it->second.swapped || pos < 0 || pos >= it->second.len)
+        return PKV_ERR_INVALID_ARG;
     *slot_out = static_cast<int64_t>(it->second.blocks[pos / kBlockTokens]) * kBlockTokens +
                 pos % kBlockTokens;
     return PKV_OK;

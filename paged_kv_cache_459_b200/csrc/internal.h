@@ -108,6 +108,11 @@ cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *src,
                                int n, int num_kv_heads, int head_dim, long long num_blocks,
                                unsigned int *err, cudaStream_t stream);
 
+cudaError_t launch_swap_blocks(void *k_cache, void *v_cache, void *host_k, void *host_v,
+                               const int64_t *gpu_blocks, const int64_t *host_blocks, int n,
+                               int direction, int num_kv_heads, int head_dim, long long num_blocks,
+                               long long num_host_blocks, unsigned int *err, cudaStream_t stream);
+
 cudaError_t launch_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
                             const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
                             int head_dim, long long num_blocks, unsigned int *err,

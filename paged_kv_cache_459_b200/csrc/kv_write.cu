@@ -89,4 +89,44 @@ cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *src,
     return cudaGetLastError();
 }
 
+// Block swap over the host link: pair blockIdx.y; the host side is pinned,
+// device-mapped memory reached directly by the loads or stores.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(uint4 *k_cache, uint4 *v_cache,
+                                                          uint4 *host_k, uint4 *host_v,
+                                                          const int64_t *__restrict__ gpu_blocks,
+                                                          const int64_t *__restrict__ host_blocks,
+                                                          int direction, long long vec_per_block,
+                                                          long long num_blocks,
+                                                          long long num_host_blocks,
+                                                          unsigned int *err) {
+    const long long g = gpu_blocks[blockIdx.y], h = host_blocks[blockIdx.y];
+    if (g < 0 || g >= num_blocks || h < 0 || h >= num_host_blocks) {
+        if (err != nullptr && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(err, PKV_DEV_ERR_BAD_BLOCK);
+        return;
+    }
+    uint4 *dk = direction == PKV_SWAP_OUT ? host_k + h * vec_per_block : k_cache + g * vec_per_block;
+    uint4 *dv = direction == PKV_SWAP_OUT ? host_v + h * vec_per_block : v_cache + g * vec_per_block;
+    const uint4 *sk = direction == PKV_SWAP_OUT ? k_cache + g * vec_per_block : host_k + h * vec_per_block;
+    const uint4 *sv = direction == PKV_SWAP_OUT ? v_cache + g * vec_per_block : host_v + h * vec_per_block;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < vec_per_block;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        dk[i] = sk[i];
+        dv[i] = sv[i];
+    }
+}
+
+cudaError_t launch_swap_blocks(void *k_cache, void *v_cache, void *host_k, void *host_v,
+                               const int64_t *gpu_blocks, const int64_t *host_blocks, int n,
+                               int direction, int num_kv_heads, int head_dim, long long num_blocks,
+                               long long num_host_blocks, unsigned int *err, cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    const long long vec = static_cast<long long>(num_kv_heads) * kBlockTokens * head_dim / 8;
+    const unsigned gx = static_cast<unsigned>(std::min<long long>((vec + 1023) / 1024, 256));
+    swap_blocks_kernel<<<dim3(gx, static_cast<unsigned>(n)), 256, 0, stream>>>(
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), static_cast<uint4 *>(host_k),
+        static_cast<uint4 *>(host_v), gpu_blocks, host_blocks, direction, vec, num_blocks,
+        num_host_blocks, err);
+    return cudaGetLastError();
+}
+
 }  // namespace pkv

@@ -117,6 +117,39 @@ pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, con
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+// Device address of pinned, device-mapped host memory, or nullptr.
+static void *mapped_host_pointer(void *p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the error the query left behind
+        return nullptr;
+    }
+    if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr) return nullptr;
+    return attr.devicePointer;
+}
+
+pkv_status pkv_swap_blocks(void *k_cache, void *v_cache, void *host_k, void *host_v,
+                           const int64_t *gpu_blocks, const int64_t *host_blocks, int n,
+                           int direction, int num_kv_heads, int head_dim, int64_t num_blocks,
+                           int64_t num_host_blocks, unsigned int *err_word, void *stream) {
+    if (n < 0 || n > 65535 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 ||
+        num_blocks <= 0 || num_host_blocks <= 0 ||
+        (direction != PKV_SWAP_OUT && direction != PKV_SWAP_IN))
+        return PKV_ERR_INVALID_ARG;
+    if (n == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !host_k || !host_v || !gpu_blocks || !host_blocks ||
+        !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(host_k) || !aligned16(host_v))
+        return PKV_ERR_INVALID_ARG;
+    void *dk = mapped_host_pointer(host_k);
+    void *dv = mapped_host_pointer(host_v);
+    if (!dk || !dv || !aligned16(dk) || !aligned16(dv)) return PKV_ERR_INVALID_ARG;
+    cudaError_t e = pkv::launch_swap_blocks(k_cache, v_cache, dk, dv, gpu_blocks, host_blocks, n,
+                                            direction, num_kv_heads, head_dim, num_blocks,
+                                            num_host_blocks, err_word,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                   int max_blocks_per_seq, int partition_tokens) {
     if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0) return 0;

@@ -30,6 +30,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_OOM, ERR_CUDA = range(6)
 DEV_ERR_BAD_SLOT, DEV_ERR_BAD_BLOCK, DEV_ERR_BAD_LEN, DEV_ERR_TIMEOUT = 1, 2, 4, 8
 DECODE_AUTO, DECODE_SINGLE, DECODE_SPLIT, DECODE_STREAM = 0, 1, 2, 3
+SWAP_OUT, SWAP_IN = 0, 1
 BLOCK_TOKENS = 16
 DEFAULT_PARTITION_TOKENS = 512
 
@@ -61,6 +62,11 @@ _sigs = {
     "pkv_alloc_refcount": ([_P, _i64, _P], _i32),
     "pkv_alloc_take_copies": ([_P, _P, _P, _i64, _P], _i32),
     "pkv_copy_blocks": ([_P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P], _i32),
+    "pkv_swap_blocks": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i64, _i64, _P, _P], _i32),
+    "pkv_alloc_set_host_pool": ([_P, _i64], _i32),
+    "pkv_alloc_swap_out": ([_P, _i64], _i32),
+    "pkv_alloc_swap_in": ([_P, _i64], _i32),
+    "pkv_alloc_take_swaps": ([_P, _i32, _P, _P, _i64, _P], _i32),
     "pkv_alloc_prefix_groups": ([_P, _P, _i32, _P, _P, _P, _P], _i32),
     "pkv_decode_prefix_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
     "pkv_paged_attention_decode_prefix": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
@@ -151,6 +157,30 @@ def copy_blocks(k_cache, v_cache, src, dst, err=None) -> None:
     ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
     _check(_lib.pkv_copy_blocks(*ptrs, sp, dp, src.numel(), hkv, d, nb, ep,
                                 _stream_ptr(k_cache.device)), "pkv_copy_blocks")
+
+
+def swap_blocks(k_cache, v_cache, host_k, host_v, gpu_blocks, host_blocks, direction,
+                err=None) -> None:
+    """Move whole blocks between the GPU caches and pinned host swap space
+    (host_k/host_v: pinned CPU bf16 tensors [num_host_blocks, Hkv, 16, d])."""
+    import torch
+
+    if k_cache.shape != v_cache.shape or host_k.shape != host_v.shape \
+            or tuple(host_k.shape[1:]) != tuple(k_cache.shape[1:]) \
+            or gpu_blocks.shape != host_blocks.shape:
+        raise ValueError("shape mismatch")
+    for t, n in ((host_k, "host_k"), (host_v, "host_v")):
+        if t.device.type != "cpu" or not t.is_pinned() or t.dtype != torch.bfloat16 \
+                or not t.is_contiguous():
+            raise ValueError(f"{n} must be a pinned, contiguous bf16 CPU tensor")
+    nb, hkv, bt, d = k_cache.shape
+    ptrs = [_dev_tensor(x, torch.bfloat16, n) for x, n in ((k_cache, "k_cache"), (v_cache, "v_cache"))]
+    gp = _dev_tensor(gpu_blocks, torch.int64, "gpu_blocks")
+    hp = _dev_tensor(host_blocks, torch.int64, "host_blocks")
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    _check(_lib.pkv_swap_blocks(*ptrs, host_k.data_ptr(), host_v.data_ptr(), gp, hp,
+                                gpu_blocks.numel(), int(direction), hkv, d, nb, host_k.shape[0], ep,
+                                _stream_ptr(k_cache.device)), "pkv_swap_blocks")
 
 
 _workspaces: dict = {}
@@ -338,6 +368,27 @@ class BlockAllocator:
         _acheck(_lib.pkv_alloc_free_list(self._h, out.ctypes.data if n.value else None, n.value,
                                          ctypes.byref(n)), "free_list")
         return out.tolist()
+
+    def set_host_pool(self, num_host_blocks: int) -> None:
+        _acheck(_lib.pkv_alloc_set_host_pool(self._h, int(num_host_blocks)), "set_host_pool")
+
+    def swap_out(self, seq_id: int) -> None:
+        _acheck(_lib.pkv_alloc_swap_out(self._h, int(seq_id)), "swap_out")
+
+    def swap_in(self, seq_id: int) -> None:
+        _acheck(_lib.pkv_alloc_swap_in(self._h, int(seq_id)), "swap_in")
+
+    def take_swaps(self, direction: int):
+        """Queued (gpu_block, host_slot) pairs of one direction; clears them."""
+        n = ctypes.c_int64()
+        _acheck(_lib.pkv_alloc_take_swaps(self._h, direction, None, None, 0, ctypes.byref(n)),
+                "take_swaps")
+        g = np.empty(n.value, np.int64)
+        h = np.empty(n.value, np.int64)
+        _acheck(_lib.pkv_alloc_take_swaps(self._h, direction, g.ctypes.data if n.value else None,
+                                          h.ctypes.data if n.value else None, n.value,
+                                          ctypes.byref(n)), "take_swaps")
+        return g, h
 
     def take_copies(self):
         """Queued copy-on-write pairs (src, dst) as int64 arrays; clears the queue."""

@@ -20,7 +20,7 @@ BT = 16
 def same_state(a: BlockAllocator, m: BlockManager, seq_ids):
     assert a.free_blocks() == m.free_blocks()
     assert [a.refcount(b) for b in range(m.num_blocks)] == m.ref
-    ids = sorted(seq_ids)
+    ids = sorted(s for s in seq_ids if s not in m.swapped)
     if ids:
         w = max(1, max(len(m.tables[s]) for s in ids))
         ta, la = a.export(ids, w)
@@ -68,14 +68,17 @@ def test_random_operations_match_model(seed):
     nb = int(gen.integers(8, 64))
     order = gen.permutation(nb)
     a, m = BlockAllocator(nb, order), BlockManager(nb, order)
+    a.set_host_pool(24)
+    m.set_host_pool(24)
     live, next_id = [], 0
     for step in range(400):
-        op = gen.choice(["add", "append", "appends", "fork", "free"], p=[.2, .35, .15, .15, .15])
+        op = gen.choice(["add", "append", "appends", "fork", "free", "out", "in"],
+                        p=[.18, .3, .14, .14, .12, .06, .06])
         args = ()
         if op == "add":
             args = (next_id, int(gen.integers(0, 70)))
             next_id += 1
-        elif op in ("append", "free") and live:
+        elif op in ("append", "free", "out", "in") and live:
             args = (int(gen.choice(live)),)
         elif op == "appends" and live:
             k = int(gen.integers(1, len(live) + 1))
@@ -90,15 +93,19 @@ def test_random_operations_match_model(seed):
         ea = em = None
         try:
             ra = {"add": a.add_seq, "append": a.append_token, "appends": a.append_tokens,
-                  "fork": a.fork, "free": a.free_seq}[op](*args)
+                  "fork": a.fork, "free": a.free_seq, "out": a.swap_out, "in": a.swap_in}[op](*args)
         except AllocError as e:
             ea = e.kind
         try:
             rm = {"add": m.add_seq, "append": m.append_token, "appends": m.append_tokens,
-                  "fork": m.fork, "free": m.free_seq}[op](*args)
+                  "fork": m.fork, "free": m.free_seq, "out": m.swap_out, "in": m.swap_in}[op](*args)
             if op in ("append", "appends"):
                 ca, cm = a.take_copies(), m.take_copies()
                 assert all(np.array_equal(x, y) for x, y in zip(ca, cm)), (step, op)
+            if op in ("out", "in"):
+                d = 0 if op == "out" else 1
+                sa, sm = a.take_swaps(d), m.take_swaps(d)
+                assert all(np.array_equal(x, y) for x, y in zip(sa, sm)), (step, op)
         except ModelError as e:
             em = e.kind
         assert ea == em, (step, op, args, ea, em)

@@ -417,3 +417,34 @@ def test_copy_on_write_beams_attend_to_their_own_tokens():
     np.testing.assert_allclose(got, sdpa_reference(q, ks, vs, 0.125), rtol=0, atol=1e-12)
     with pytest.raises(ValueError):
         oracle.copy_blocks(kc, vc, np.array([0]), np.array([nb]))
+
+
+def test_swap_out_and_in_leaves_attention_unchanged():
+    """Swap space: moving a sequence's blocks to host slots and back into
+    other GPU blocks (with the freed blocks overwritten meanwhile) gives the
+    same attention output, bit for bit."""
+    w = wl.build("llama", 6, BlockManager, batch=5, len_lo=20, len_hi=90, head_dim=64,
+                 poison=False, pool_factor=2.0)
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    base = oracle.paged_decode(w.q, kc, vc, w.block_tables, w.lens, w.cfg["scale"])
+    bm = w.alloc
+    bm.set_host_pool(32)
+    hk = np.zeros((32,) + kc.shape[1:], np.uint16)
+    hv = np.zeros_like(hk)
+    for s in (1, 3):
+        bm.swap_out(s)
+    g, h = bm.take_swaps(0)
+    kc, vc, hk, hv = oracle.swap_blocks(kc, vc, hk, hv, g, h, 0)
+    kc[g] = wl.BF16_NAN  # the freed blocks are reused meanwhile
+    vc[g] = wl.BF16_NAN
+    with pytest.raises(Exception):
+        bm.append_token(1)  # a swapped-out sequence only comes back or is freed
+    for s in (3, 1):
+        bm.swap_in(s)
+    g2, h2 = bm.take_swaps(1)
+    assert sorted(h2.tolist()) == sorted(h.tolist())
+    kc, vc, hk, hv = oracle.swap_blocks(kc, vc, hk, hv, g2, h2, 1)
+    tables, lens = bm.export(list(range(5)), w.block_tables.shape[1])
+    assert not np.array_equal(tables, w.block_tables)  # sequences 1 and 3 moved
+    out = oracle.paged_decode(w.q, kc, vc, tables, lens, w.cfg["scale"])
+    assert np.array_equal(out, base)
