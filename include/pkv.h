@@ -270,6 +270,30 @@ PKV_API pkv_status pkv_swap_blocks(void *k_cache, void *v_cache, void *host_k, v
                                    int64_t num_blocks, int64_t num_host_blocks,
                                    unsigned int *err_word, void *stream);
 
+/*
+ * Paged prefill attention ("vLLM 與 PagedAttention：高吞吐推理的關鍵", section 三
+ * step 二: the prompt's K/V are written into blocks, a new block taken as each
+ * fills -- pkv_alloc_extend + pkv_paged_kv_write -- and the prompt attends over
+ * them): causal attention of each sequence's new tokens over its paged K/V.
+ * Sequence b has query rows query_start[b] .. query_start[b+1] of q / out
+ * ([T][num_heads][head_dim] bf16, T = query_start[num_seqs]) and context
+ * length seq_lens[b] >= its row count, including them: its new tokens sit at
+ * positions seq_lens[b] - rows .. seq_lens[b] - 1 (earlier positions -- a
+ * cached prefix, earlier chunks -- are read from the cache), and the token at
+ * position p attends to positions [0, p].  The K/V of the new tokens must be
+ * in the cache already.  max_query_len >= every sequence's row count.
+ * Tensor cores (mma.m16n8k16, bf16 -> fp32); TMA-fed shared K/V ring.
+ * A sequence with seq_lens[b] < its rows or past its table is skipped
+ * (rows not written) and flagged PKV_DEV_ERR_BAD_LEN.
+ */
+PKV_API pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_cache,
+                                               const void *v_cache, const int32_t *block_tables,
+                                               int max_blocks_per_seq, const int32_t *seq_lens,
+                                               const int32_t *query_start, int num_seqs,
+                                               int max_query_len, int num_heads, int num_kv_heads,
+                                               int head_dim, int64_t num_blocks, float scale,
+                                               unsigned int *err_word, void *stream);
+
 /* ------------------------------------------------------------------------
  * Host block allocator (section 二 and section 三 of the first page): a pool
  * of num_blocks physical blocks with reference counts, per-sequence block
@@ -300,6 +324,11 @@ PKV_API pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, i
  * block) is queued for pkv_alloc_take_copies; the caller must copy those
  * blocks on the device (pkv_copy_blocks) before writing the new token. */
 PKV_API pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_out);
+
+/* n more tokens for seq_id (a prompt or a prefill chunk), their slots into
+ * slots_out [n] (host): blocks are taken as each one fills (copy-on-write
+ * first if the last block is shared and partly filled); all or none. */
+PKV_API pkv_status pkv_alloc_extend(pkv_alloc *a, int64_t seq_id, int64_t n, int64_t *slots_out);
 
 /* One token for each of n distinct sequences (a decode step); all or none. */
 PKV_API pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n,

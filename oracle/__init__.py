@@ -10,6 +10,8 @@ arithmetic.
                                K and V gathered through the block table (C, fp64).
 * ``paged_decode_partitioned`` -- the same in independent token partitions
                                combined by log-sum-exp (C, fp64).
+* ``paged_prefill``         -- causal attention of new (prompt) tokens: each row
+                               is the decode definition at its own position.
 * ``kv_write``              -- the new token's K/V copied into its slot (C).
 * ``copy_blocks``           -- copy-on-write copies of whole blocks (C).
 * ``swap_blocks``           -- blocks moved to / from host swap space (C).
@@ -127,6 +129,19 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, nthreads: i
     if rc:
         raise ValueError(f"oracle_paged_decode failed ({rc})")
     return out
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, seq_lens, query_start, scale):
+    """Causal prefill: row r of sequence b (query_start[b] <= r < query_start[b+1])
+    is the token at position p = seq_lens[b] - n_b + (r - query_start[b]) and
+    attends to positions [0, p] -- the decode definition with length p + 1."""
+    qs = np.asarray(query_start, dtype=np.int64)
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    tables = np.asarray(block_tables, dtype=np.int32)
+    rows_seq = np.repeat(np.arange(len(lens)), np.diff(qs))
+    first = lens[rows_seq] - np.diff(qs)[rows_seq]
+    pos = first + (np.arange(qs[-1]) - qs[rows_seq])
+    return paged_decode(q, k_cache, v_cache, tables[rows_seq], (pos + 1).astype(np.int32), scale)
 
 
 def paged_decode_partitioned(q, k_cache, v_cache, block_tables, seq_lens, scale, partition_tokens):

@@ -122,6 +122,20 @@ class BlockManager:
         self.copies = []
         return src, dst
 
+    def extend(self, seq_id: int, n: int):
+        """n more tokens (a prompt or a prefill chunk), all or none: step 二
+        of the lifecycle -- a new block each time one fills."""
+        import numpy as np
+
+        if seq_id not in self.tables or seq_id in self.swapped or n < 0:
+            raise AllocError("invalid", "unknown or swapped-out sequence")
+        blocks, ln = self.tables[seq_id], self.lens[seq_id]
+        cow = ln % BLOCK_TOKENS != 0 and self.ref[blocks[-1]] > 1 and n > 0
+        need = int(cow) + blocks_for(ln + n) - len(blocks)
+        if need > len(self.free):
+            raise AllocError("oom")
+        return np.array([self.append_token(seq_id) for _ in range(n)], np.int64)
+
     def fork(self, parent: int, child: int, num_tokens: int | None = None) -> None:
         if parent not in self.tables or parent in self.swapped or child in self.tables:
             raise AllocError("invalid", "unknown parent or existing child")

@@ -205,6 +205,28 @@ pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, 
     return PKV_OK;
 }
 
+pkv_status pkv_alloc_extend(pkv_alloc *a, int64_t seq_id, int64_t n, int64_t *slots_out) {
+    if (!a || n < 0 || (n > 0 && !slots_out)) return PKV_ERR_INVALID_ARG;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
+    Sequence &s = it->second;
+    if (n == 0) return PKV_OK;
+    // blocks needed: a private copy of a shared partly filled last block, then
+    // one per 16 positions past the current blocks
+    const bool cow = s.len % kBlockTokens != 0 && a->refcount[s.blocks.back()] > 1;
+    const int64_t need = (cow ? 1 : 0) + blocks_for(s.len + n) - static_cast<int64_t>(s.blocks.size());
+    if (need > static_cast<int64_t>(a->free_list.size())) return PKV_ERR_OOM;
+    try {
+        s.blocks.reserve(static_cast<size_t>(blocks_for(s.len + n)));
+        if (cow) a->pending_copies.reserve(a->pending_copies.size() + 1);
+    } catch (const std::bad_alloc &) {
+        return PKV_ERR_OOM;
+    }
+    for (int64_t i = 0; i < n; ++i)
+        slots_out[i] = do_append(a, s, append_kind(s, s.blocks.empty() ? 0 : a->refcount[s.blocks.back()]));
+    return PKV_OK;
+}
+
 pkv_status pkv_alloc_take_copies(pkv_alloc *a, int64_t *src_out, int64_t *dst_out, int64_t cap,
                                  int64_t *n_out) {
     if (!a || !n_out || cap < 0 || (cap > 0 && (!src_out || !dst_out))) return PKV_ERR_INVALID_ARG;

@@ -104,6 +104,22 @@ cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const
                            const DecodeParams &dp, int head_dim, int num_groups,
                            cudaStream_t stream);
 
+// Causal prefill attention of each sequence's new tokens over its paged K/V.
+struct PrefillParams {
+    __nv_bfloat16 *out;           // [T][Hq][D]
+    const __nv_bfloat16 *q;       // [T][Hq][D]
+    const int32_t *block_tables;  // [B][W]
+    const int32_t *seq_lens;      // [B] context length including the new tokens
+    const int32_t *query_start;   // [B + 1] rows of sequence b: [query_start[b], query_start[b+1])
+    unsigned int *err;
+    long long num_blocks;
+    int W, B, Hq, Hkv, group;
+    float scale_log2;
+};
+
+cudaError_t launch_prefill(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
+                           int head_dim, int max_query_len, cudaStream_t stream);
+
 cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, const int64_t *dst,
                                int n, int num_kv_heads, int head_dim, long long num_blocks,
                                unsigned int *err, cudaStream_t stream);

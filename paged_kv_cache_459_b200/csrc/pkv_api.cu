@@ -431,6 +431,50 @@ pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const voi
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       int max_blocks_per_seq, const int32_t *seq_lens,
+                                       const int32_t *query_start, int num_seqs, int max_query_len,
+                                       int num_heads, int num_kv_heads, int head_dim,
+                                       int64_t num_blocks, float scale, unsigned int *err_word,
+                                       void *stream) {
+    if (num_seqs < 0 || num_seqs > 65535 || max_query_len < 0 || num_heads <= 0 ||
+        num_kv_heads <= 0 || num_kv_heads > 65535 || num_heads % num_kv_heads ||
+        max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale))
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || max_query_len == 0) return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_INVALID_ARG;
+    if (num_blocks > INT32_MAX / PKV_BLOCK_TOKENS / num_kv_heads) return PKV_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(max_blocks_per_seq) * PKV_BLOCK_TOKENS > INT32_MAX)
+        return PKV_ERR_INVALID_ARG;
+    const int64_t rows = num_blocks * num_kv_heads * PKV_BLOCK_TOKENS;
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, k_cache, rows, head_dim) ||
+        !encode_cache_map(&tmv, v_cache, rows, head_dim))
+        return PKV_ERR_CUDA;
+    pkv::PrefillParams p{};
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.query_start = query_start;
+    p.err = err_word;
+    p.num_blocks = num_blocks;
+    p.W = max_blocks_per_seq;
+    p.B = num_seqs;
+    p.Hq = num_heads;
+    p.Hkv = num_kv_heads;
+    p.group = num_heads / num_kv_heads;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    cudaError_t e = pkv::launch_prefill(tmk, tmv, p, head_dim, max_query_len,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
                                       const void *v_cache, const int32_t *block_tables,
                                       int max_blocks_per_seq, const int32_t *seq_lens,

@@ -64,6 +64,9 @@ _sigs = {
     "pkv_copy_blocks": ([_P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P], _i32),
     "pkv_swap_blocks": ([_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, _i64, _i64, _P, _P], _i32),
     "pkv_alloc_set_host_pool": ([_P, _i64], _i32),
+    "pkv_alloc_extend": ([_P, _i64, _i64, _P], _i32),
+    "pkv_paged_attention_prefill": ([_P, _P, _P, _P, _P, _i32, _P, _P, _i32, _i32, _i32, _i32, _i32,
+                                     _i64, _f32, _P, _P], _i32),
     "pkv_alloc_swap_out": ([_P, _i64], _i32),
     "pkv_alloc_swap_in": ([_P, _i64], _i32),
     "pkv_alloc_take_swaps": ([_P, _i32, _P, _P, _i64, _P], _i32),
@@ -181,6 +184,32 @@ def swap_blocks(k_cache, v_cache, host_k, host_v, gpu_blocks, host_blocks, direc
     _check(_lib.pkv_swap_blocks(*ptrs, host_k.data_ptr(), host_v.data_ptr(), gp, hp,
                                 gpu_blocks.numel(), int(direction), hkv, d, nb, host_k.shape[0], ep,
                                 _stream_ptr(k_cache.device)), "pkv_swap_blocks")
+
+
+def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, query_start, scale,
+                            num_kv_heads, max_query_len: int, err=None) -> None:
+    """Causal attention of each sequence's new tokens over its paged K/V.
+    q, out [T, Hq, d] bf16; query_start [B + 1] int32 (rows of each sequence);
+    seq_lens [B] int32 context lengths including the new tokens."""
+    import torch
+
+    T, hq, d = q.shape
+    B = seq_lens.shape[0]
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
+            or block_tables.shape[0] != B or query_start.shape != (B + 1,):
+        raise ValueError("shape mismatch")
+    ptrs = [_dev_tensor(x, torch.bfloat16, n) for x, n in ((out, "out"), (q, "q"),
+                                                            (k_cache, "k_cache"),
+                                                            (v_cache, "v_cache"))]
+    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
+    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
+    sp = _dev_tensor(query_start, torch.int32, "query_start")
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    _check(_lib.pkv_paged_attention_prefill(*ptrs, tp, block_tables.shape[1], lp, sp, B,
+                                            int(max_query_len), hq, num_kv_heads, d,
+                                            k_cache.shape[0], float(scale), ep,
+                                            _stream_ptr(q.device)), "pkv_paged_attention_prefill")
 
 
 _workspaces: dict = {}
@@ -336,6 +365,13 @@ class BlockAllocator:
         out = ctypes.c_int64()
         _acheck(_lib.pkv_alloc_append_token(self._h, int(seq_id), ctypes.byref(out)), "append_token")
         return out.value
+
+    def extend(self, seq_id: int, n: int) -> np.ndarray:
+        """Slots of n more tokens (blocks taken as each fills)."""
+        out = np.empty(int(n), dtype=np.int64)
+        _acheck(_lib.pkv_alloc_extend(self._h, int(seq_id), int(n),
+                                      out.ctypes.data if n else None), "extend")
+        return out
 
     def append_tokens(self, seq_ids) -> np.ndarray:
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)

@@ -227,3 +227,18 @@ def test_prefix_groups_random_forks_match_model():
         ids = list(range(12))
         for x, y in zip(a.prefix_groups(ids), m.prefix_groups(ids)):
             assert np.array_equal(x, y)
+
+
+def test_extend_matches_model_and_takes_blocks_as_they_fill():
+    for alloc_cls in (BlockAllocator, BlockManager):
+        a = alloc_cls(16, list(range(16)))
+        a.add_seq(0, 0)
+        slots = a.extend(0, 40)  # a 40-token prompt: blocks 0, 1, 2
+        assert slots.tolist() == list(range(40))
+        a.fork(0, 1)  # shares the partly filled third block
+        s2 = a.extend(1, 30)  # copy-on-write first, then blocks as they fill
+        assert s2[0] == 3 * 16 + 8 and a.take_copies()[0].tolist() == [2]
+        with pytest.raises(Exception):
+            a.extend(1, 16 * 20)  # not enough blocks: nothing changes
+        n = a.seq_len(1) if hasattr(a, "seq_len") else a.lens[1]
+        assert n == 70

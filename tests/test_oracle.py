@@ -448,3 +448,40 @@ def test_swap_out_and_in_leaves_attention_unchanged():
     assert not np.array_equal(tables, w.block_tables)  # sequences 1 and 3 moved
     out = oracle.paged_decode(w.q, kc, vc, tables, lens, w.cfg["scale"])
     assert np.array_equal(out, base)
+
+
+@pytest.mark.parametrize("hq,hkv,d,lens", [(4, 4, 64, [1, 37, 90]), (8, 2, 128, [20, 65])])
+def test_prefill_matches_causal_library_attention(hq, hkv, d, lens):
+    """Fresh prompts: the paged causal prefill equals torch's fp64 causal
+    scaled_dot_product_attention on the un-paged K/V."""
+    q, ks, vs = random_case(40 + d, lens, hq, hkv, d)
+    gen = wl.rng(41)
+    qrows = rb((sum(lens), hq, d), gen)
+    kc, vc, tables, lens_ = page_sequences(ks, vs, 64, seed=42)
+    qs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    got = oracle.paged_prefill(qrows, kc, vc, tables, lens_, qs, 0.125)
+    for b, n in enumerate(lens):
+        qt = torch.from_numpy(f32(qrows[qs[b]:qs[b + 1]])).permute(1, 0, 2)[None]   # [1, Hq, n, d]
+        kt = torch.from_numpy(f32(ks[b])).permute(1, 0, 2)[None]
+        vt = torch.from_numpy(f32(vs[b])).permute(1, 0, 2)[None]
+        want = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=0.125,
+                                              enable_gqa=True)[0].permute(1, 0, 2).numpy()
+        np.testing.assert_allclose(got[qs[b]:qs[b + 1]], want, rtol=0, atol=1e-12)
+
+
+def test_prefill_after_cached_prefix_uses_an_offset_causal_mask():
+    """A chunk of new tokens after cached ones: row i (position c + i) sees
+    keys [0, c + i] -- torch attention with that explicit mask."""
+    hq = hkv = 2
+    d, ctx, new = 64, 75, 11
+    q, ks, vs = random_case(43, [ctx], hq, hkv, d)
+    qrows = rb((new, hq, d), wl.rng(44))
+    kc, vc, tables, lens_ = page_sequences(ks, vs, 16, seed=45)
+    got = oracle.paged_prefill(qrows, kc, vc, tables, lens_, np.array([0, new]), 0.3)
+    pos = ctx - new + np.arange(new)
+    mask = torch.from_numpy(np.arange(ctx)[None, :] <= pos[:, None])
+    qt = torch.from_numpy(f32(qrows)).permute(1, 0, 2)[None]
+    kt = torch.from_numpy(f32(ks[0])).permute(1, 0, 2)[None]
+    vt = torch.from_numpy(f32(vs[0])).permute(1, 0, 2)[None]
+    want = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.3)[0].permute(1, 0, 2)
+    np.testing.assert_allclose(got, want.numpy(), rtol=0, atol=1e-12)
