@@ -57,6 +57,8 @@ def parse_args():
                     help="override the workload's batch (smaller cases for ncu captures)")
     ap.add_argument("--variant", choices=["auto", "single", "split", "stream"], default="auto")
     ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--row", choices=["decode", "prefill", "cow", "swap"], default="decode",
+                    help="which part of the path to measure (decode: the default step)")
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix decode: prefix blocks read once per group and KV head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -85,6 +87,23 @@ def algorithmic_bytes(w) -> dict:
     out = cfg["batch"] * hq * d * 2
     write = cfg["batch"] * hkv * d * 2 * 2 * 2
     return dict(kv=kv, q=q, out=out, write=write, tokens=toks)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity when not
+    distributed): the job time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(units_per_rank: int, steps: int, world: int, job_ms: float) -> float:
+    """Units all ranks processed per second of the slowest rank's time."""
+    return units_per_rank * steps * world / (job_ms * 1e-3)
 
 
 def source_sha(path: str) -> str:
@@ -366,10 +385,7 @@ def run_gpu(args):
     if int(err.item()) != 0:
         raise SystemExit(f"device error word {int(err.item())} after the timed steps")
 
-    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(times[0]), float(times[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
 
     ab = algorithmic_bytes(w)
     peak, peak_kind = measured_peak_hbm()
@@ -380,8 +396,8 @@ def run_gpu(args):
         unique_tokens += sum(16 * int(pb_h[mem_h[offs_h[g]]]) for g in range(len(offs_h) - 1))
         dec_bytes = unique_tokens * hkv * d * 2 * 2 + ab["q"]
     achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
-    value = B * K * world / (total_ms * 1e-3)
-    e2e_value = B * K * world / (e2e_ms * 1e-3)
+    value = job_throughput(B, K, world, total_ms)
+    e2e_value = job_throughput(B, K, world, e2e_ms)
     launches_per_step = 2 + (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) else 0)
     if args.cascade:
         launches_per_step = 1 + 3  # write; prefix chunks, suffix split-K, merge
@@ -429,10 +445,116 @@ def run_gpu(args):
     return 0
 
 
+def measured_peak_tensor():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def _events_time(fn, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps  # ms
+
+
+def run_row(args):
+    """Measurements of the rows next to the decode step: prefill attention,
+    copy-on-write block copies, and block swap over the host link."""
+    import torch
+    from paged_kv_cache_459_b200 import pkv
+    from paged_kv_cache_459_b200 import workloads as wl
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    steps, warm = args.steps, max(3, args.warmup)
+    up = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    line = {"row": args.row, "n_gpus": 1, "steps": steps, "warmup": warm, "data": "synthetic"}
+    if args.row == "prefill":
+        # Llama-2-7B-shaped heads (or Qwen2.5-7B-shaped with --config qwen), 4 prompts x 2048
+        cfg = wl.config("qwen" if args.config == "qwen" else "llama")
+        hq, hkv, d, B, n = cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"], 4, 2048
+        alloc = pkv.BlockAllocator(B * n // 16 + 8, wl.rng(args.seed).permutation(B * n // 16 + 8))
+        slots = []
+        for b in range(B):
+            alloc.add_seq(b, 0)
+            slots.append(alloc.extend(b, n))
+        tables, lens = alloc.export(list(range(B)), n // 16)
+        nb = alloc.num_blocks
+        kc, vc = up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 1)), up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 2))
+        T = B * n
+        q = up(wl.bf16_normal((T, hq, d), args.seed, 3))
+        k_new, v_new = up(wl.bf16_normal((T, hkv, d), args.seed, 4)), up(wl.bf16_normal((T, hkv, d), args.seed, 5))
+        out = torch.empty_like(q)
+        t_d, l_d = torch.from_numpy(tables).to(dev), torch.from_numpy(lens).to(dev)
+        qs = torch.tensor([b * n for b in range(B + 1)], dtype=torch.int32, device=dev)
+        sl = torch.from_numpy(np.concatenate(slots)).to(dev)
+        wr_ms = _events_time(lambda: pkv.paged_kv_write(k_new, v_new, kc, vc, sl), steps, warm)
+        ms = _events_time(lambda: pkv.paged_attention_prefill(out, q, kc, vc, t_d, l_d, qs, cfg["scale"], hkv, n),
+                          steps, warm)
+        flops = B * 4.0 * d * hq * n * (n + 1) / 2  # causal: row i sees i + 1 keys
+        peak, kind = measured_peak_tensor()
+        ach = flops / (ms * 1e-3) / 1e12
+        line.update(metric="paged prefill attention TFLOP/s (causal, bf16 in / fp32 accumulate)",
+                    value=ach, unit="TFLOP/s", ms_per_step=ms, higher_is_better=True,
+                    config={"workload": f"{B} prompts x {n} tokens, {hq}/{hkv} heads, d {d}"},
+                    prompt_write_gbs=T * hkv * d * 2 * 2 * 2 / (wr_ms * 1e-3) / 1e9,
+                    roofline={"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                              "frac": ach / peak, "peak_kind": kind,
+                              "note": "warp-level mma.sync m16n8k16 (not tcgen05)"})
+    elif args.row == "cow":
+        cfg = wl.config("llama")
+        hkv, d, nb, n = cfg["num_kv_heads"], cfg["head_dim"], 8192, 2048
+        kc = up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 1))
+        vc = up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 2))
+        perm = wl.rng(args.seed).permutation(nb)
+        src = torch.from_numpy(perm[:n].copy()).to(dev)
+        dst = torch.from_numpy(perm[n:2 * n].copy()).to(dev)
+        ms = _events_time(lambda: pkv.copy_blocks(kc, vc, src, dst), steps, warm)
+        nbytes = n * hkv * 16 * d * 2 * 2 * 2  # read + write, K and V
+        peak, kind = measured_peak_hbm()
+        ach = nbytes / (ms * 1e-3) / 1e9
+        line.update(metric="copy-on-write block copy GB/s (read + write)", value=ach, unit="GB/s",
+                    ms_per_step=ms, higher_is_better=True,
+                    config={"workload": f"{n} random block pairs, {hkv} KV heads x 16 x {d} bf16"},
+                    roofline={"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                              "frac": ach / peak, "peak_kind": kind})
+    else:  # swap
+        cfg = wl.config("llama")
+        hkv, d, nb, n = cfg["num_kv_heads"], cfg["head_dim"], 4096, 1024
+        kc = up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 1))
+        vc = up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 2))
+        hk = torch.empty((n, hkv, 16, d), dtype=torch.bfloat16).pin_memory()
+        hv = torch.empty_like(hk).pin_memory()
+        g = torch.from_numpy(wl.rng(args.seed).permutation(nb)[:n].copy()).to(dev)
+        h = torch.arange(n, dtype=torch.int64, device=dev)
+        ms_out = _events_time(lambda: pkv.swap_blocks(kc, vc, hk, hv, g, h, pkv.SWAP_OUT), steps, warm)
+        ms_in = _events_time(lambda: pkv.swap_blocks(kc, vc, hk, hv, g, h, pkv.SWAP_IN), steps, warm)
+        nbytes = n * hkv * 16 * d * 2 * 2
+        line.update(metric="block swap GB/s over the host link (out, in)",
+                    value=nbytes / (ms_out * 1e-3) / 1e9, unit="GB/s", ms_per_step=ms_out,
+                    higher_is_better=True, swap_in_gbs=nbytes / (ms_in * 1e-3) / 1e9,
+                    config={"workload": f"{n} blocks of {hkv} KV heads x 16 x {d} bf16, K and V "
+                                        f"({nbytes / 1e6:.0f} MB each way), pinned host memory"})
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.row != "decode":
+        return run_row(args)
     return run_gpu(args)
 
 
