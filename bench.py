@@ -398,7 +398,9 @@ def run_gpu(args):
     achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
     value = job_throughput(B, K, world, total_ms)
     e2e_value = job_throughput(B, K, world, e2e_ms)
-    launches_per_step = 2 + (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) else 0)
+    # write + decode, + the merge (split-K, balanced) or the longest-first order (single pass)
+    ordered = chosen == pkv.DECODE_SINGLE and ws.numel() >= 4 * B
+    launches_per_step = 2 + (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) or ordered else 0)
     if args.cascade:
         launches_per_step = 1 + 3  # write; prefix chunks, suffix split-K, merge
     line = {
@@ -409,7 +411,9 @@ def run_gpu(args):
             "workload": WORKLOAD_NAMES[args.config], "name": args.config, "batch": B,
             "num_heads": hq, "num_kv_heads": hkv, "head_dim": d, "block_tokens": 16,
             "tokens": ab["tokens"], "num_blocks": w.num_blocks, "table_width": W,
-            "variant": {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head)",
+            "variant": {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head, longest "
+                                            "first)" if ordered else
+                        "single pass (one CTA per sequence x KV head)",
                         pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % args.partition,
                         pkv.DECODE_STREAM: "balanced stream-K (equal tile ranges per warp) + merge",
                         }[chosen] if not args.cascade else

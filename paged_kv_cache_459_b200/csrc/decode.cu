@@ -45,32 +45,123 @@ template <int D, int NW, int S, bool MMA, bool SPLIT>
 __global__ void __launch_bounds__(NW * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-    decode_unit<D, NW, S, MMA, SPLIT>(tmk, tmv, p, blockIdx.x, blockIdx.y, blockIdx.z);
+    int b = blockIdx.z;
+    if (p.order != nullptr) {
+        pdl_wait_primary();  // the order kernel's output
+        b = __ldg(p.order + b);
+    }
+    decode_unit<D, NW, S, MMA, SPLIT>(tmk, tmv, p, blockIdx.x, blockIdx.y, b);
+}
+
+// Longest-first order of the sequences by block count (counting sort; ties in
+// any order -- the order only steers scheduling, never the arithmetic).
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderBuckets = 4096;
+
+__global__ void __launch_bounds__(kOrderThreads)
+    order_kernel(const int32_t *__restrict__ seq_lens, int B, int W, int shift, int32_t *order) {
+    pdl_launch_dependents();
+    __shared__ int count[kOrderBuckets];
+    __shared__ int warp_tot[kOrderThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < kOrderBuckets; i += kOrderThreads) count[i] = 0;
+    __syncthreads();
+    const auto bucket = [&](int b) {  // descending: the longest sequences get bucket 0
+        int len = __ldg(seq_lens + b);
+        len = len < 0 ? 0 : min(len, W * kBlockTokens);
+        const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
+        return (kOrderBuckets - 1) - min(nblk >> shift, kOrderBuckets - 1);
+    };
+    for (int b = tid; b < B; b += kOrderThreads) atomicAdd(&count[bucket(b)], 1);
+    __syncthreads();
+    // exclusive scan of the bucket counts: each thread owns 4 consecutive buckets
+    constexpr int kPer = kOrderBuckets / kOrderThreads;
+    int local[kPer], sum = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        local[i] = count[tid * kPer + i];
+        sum += local[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    int run = before + incl - sum;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        count[tid * kPer + i] = run;  // now the next free position of the bucket
+        run += local[i];
+    }
+    __syncthreads();
+    for (int b = tid; b < B; b += kOrderThreads) order[atomicAdd(&count[bucket(b)], 1)] = b;
 }
 
 // Log-sum-exp merge of the split-K partitions of one (sequence, query head):
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
-// Partitions are visited in index order, so the result does not depend on
-// which CTA finished first.
+// The (m, l) pairs of all partitions are read at once into shared memory and
+// their weights computed once; each thread then sums its output column over
+// the partitions with the loads batched.  Partitions are combined in index
+// order, so the result does not depend on which CTA finished first.
 template <int D>
 __global__ void __launch_bounds__(D) splitk_merge_kernel(const DecodeParams p) {
+    constexpr int kMaxParts = 256;  // per pass; longer rows loop
+    __shared__ float s_w[kMaxParts];
+    __shared__ float s_red[D / 32][2];
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
+    pdl_wait_primary();  // the decode grid's partials
     int len = __ldg(p.seq_lens + b);
     len = len < 0 ? 0 : min(len, p.W * kBlockTokens);
-    const int part_tokens = p.part_blocks * kBlockTokens;
-    const int np = (len + part_tokens - 1) / part_tokens;
+    int start = 0;
+    if (p.start_blocks != nullptr) start = min(max(__ldg(p.start_blocks + b), 0), len / kBlockTokens);
+    const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
+    const int np = (nblk - start + p.part_blocks - 1) / p.part_blocks;
     const size_t row = static_cast<size_t>(b) * p.Hq + h;
     const float *ml = p.ws_ml + 2 * (row * p.ws_parts + p.ws_part0);
     const float *o = p.ws_o + (row * p.ws_parts + p.ws_part0) * D;
+    // M over all partitions
+    float mx = -INFINITY;
+    for (int q = e; q < np; q += D) mx = fmaxf(mx, ml[2 * q]);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    if ((e & 31) == 0) s_red[e >> 5][0] = mx;
+    __syncthreads();
     float M = -INFINITY;
-    for (int q = 0; q < np; ++q) M = fmaxf(M, ml[2 * q]);
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, s_red[w][0]);
     float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-        for (int q = 0; q < np; ++q) {
-            const float c = exp2f(ml[2 * q] - M);
-            L = fmaf(ml[2 * q + 1], c, L);
-            O = fmaf(o[static_cast<size_t>(q) * D + e], c, O);
+    for (int base = 0; base < np; base += kMaxParts) {
+        const int n = min(kMaxParts, np - base);
+        __syncthreads();  // s_w and s_red reuse
+        float lsum = 0.f;
+        for (int q = e; q < n; q += D) {
+            const float2 v = *reinterpret_cast<const float2 *>(ml + 2 * (base + q));
+            const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+            s_w[q] = w;
+            lsum = fmaf(v.y, w, lsum);
         }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
+        if ((e & 31) == 0) s_red[e >> 5][1] = lsum;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) L += s_red[w][1];
+        const float *ob = o + static_cast<size_t>(base) * D + e;
+        int q = 0;
+        for (; q + 8 <= n; q += 8) {
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = ob[static_cast<size_t>(q + i) * D];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) O = fmaf(x[i], s_w[q + i], O);
+        }
+        for (; q < n; ++q) O = fmaf(ob[static_cast<size_t>(q) * D], s_w[q], O);
     }
     p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
 }
@@ -86,12 +177,25 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
     const dim3 grid(static_cast<unsigned>(p.num_parts),
                     static_cast<unsigned>(MMA ? p.Hkv * p.chunks : p.Hq),
                     static_cast<unsigned>(p.B));
-    kern<<<grid, NW * 32, G::kSmemBytes, stream>>>(tmk, tmv, p);
-    e = cudaGetLastError();
+    if (p.order != nullptr) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(NW * 32);
+        cfg.dynamicSmemBytes = G::kSmemBytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p);
+    } else {
+        kern<<<grid, NW * 32, G::kSmemBytes, stream>>>(tmk, tmv, p);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess || !SPLIT || p.skip_merge) return e;
-    splitk_merge_kernel<D><<<dim3(static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B)), D, 0,
-                             stream>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(splitk_merge_kernel<D>, dim3(static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B)),
+                            dim3(D), stream, p);
 }
 
 template <int D, bool MMA, bool SPLIT>
@@ -117,6 +221,13 @@ cudaError_t launch_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const Decod
 }
 
 }  // namespace
+
+cudaError_t launch_order(const int32_t *seq_lens, int B, int W, int32_t *order, cudaStream_t stream) {
+    int shift = 0;
+    while ((W >> shift) >= kOrderBuckets) ++shift;
+    order_kernel<<<1, kOrderThreads, 0, stream>>>(seq_lens, B, W, shift, order);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                           int head_dim, bool split, DecodeTuning tuning, cudaStream_t stream) {

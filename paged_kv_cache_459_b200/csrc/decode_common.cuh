@@ -12,6 +12,26 @@
 #include "ptx.cuh"
 
 namespace pkv {
+
+// Launches `kern` so that it may be scheduled before the preceding kernel in
+// the stream finishes (programmatic dependent launch); the kernel must call
+// pdl_wait_primary() before it reads that kernel's output.
+template <typename... Args>
+cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, cudaStream_t stream,
+                             Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 namespace dev {
 
 constexpr uint64_t kWaitLimitNs = 250ull * 1000ull * 1000ull;  // 0.25 s per wait

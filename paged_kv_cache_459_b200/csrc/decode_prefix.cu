@@ -223,32 +223,61 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap &tmk, const CUtens
 
 // Merge of one (sequence, query head): prefix chunks [0, ceil(pb / CB)) and
 // the suffix split-K partitions that hold tokens past the prefix (counted
-// from the prefix end), in slot order, by log-sum-exp with a running maximum.
+// from the prefix end), in slot order, by log-sum-exp.  As in the split-K
+// merge: all (m, l) read at once, weights computed once, output loads batched.
 template <int D, int CB>
 __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) {
+    constexpr int kMaxSlots = 256;
+    __shared__ float s_w[kMaxSlots];
+    __shared__ float s_red[D / 32][2];
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
+    pdl_wait_primary();  // the cascade grid's partials
     int len = __ldg(p.seq_lens + b);
     len = len < 0 ? 0 : min(len, p.W * kBlockTokens);
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
     const int pb = min(max(__ldg(p.prefix_blocks + b), 0), len / kBlockTokens);
     const int nchunks = (pb + CB - 1) / CB;
-    const int nsuffix = (nblk - pb + p.part_blocks - 1) / p.part_blocks;
+    const int ntot = nchunks + (nblk - pb + p.part_blocks - 1) / p.part_blocks;
+    const auto slot = [&](int q) { return q < nchunks ? q : p.prefix_parts + (q - nchunks); };
     const size_t row = static_cast<size_t>(b) * p.Hq + h;
     const float *ml = p.ws_ml + 2 * row * p.ws_parts;
     const float *o = p.ws_o + row * p.ws_parts * D;
-    float M = -INFINITY, L = 0.f, O = 0.f;
-    const auto add = [&](int slot) {
-        const float2 v = *reinterpret_cast<const float2 *>(ml + 2 * slot);  // (m, l)
-        const float x = o[static_cast<size_t>(slot) * D + e];
-        if (v.x == -INFINITY) return;
-        const float Mn = fmaxf(M, v.x);
-        const float a = exp2f(M - Mn), c = exp2f(v.x - Mn);
-        L = L * a + v.y * c;
-        O = O * a + x * c;
-        M = Mn;
-    };
-    for (int q = 0; q < nchunks; ++q) add(q);
-    for (int q = 0; q < nsuffix; ++q) add(p.prefix_parts + q);
+    float mx = -INFINITY;
+    for (int q = e; q < ntot; q += D) mx = fmaxf(mx, ml[2 * slot(q)]);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+    if ((e & 31) == 0) s_red[e >> 5][0] = mx;
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, s_red[w][0]);
+    float L = 0.f, O = 0.f;
+    for (int base = 0; base < ntot; base += kMaxSlots) {
+        const int n = min(kMaxSlots, ntot - base);
+        __syncthreads();  // s_w and s_red reuse
+        float lsum = 0.f;
+        for (int q = e; q < n; q += D) {
+            const float2 v = *reinterpret_cast<const float2 *>(ml + 2 * slot(base + q));
+            const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+            s_w[q] = w;
+            lsum = fmaf(v.y, w, lsum);
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
+        if ((e & 31) == 0) s_red[e >> 5][1] = lsum;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) L += s_red[w][1];
+        int q = 0;
+        for (; q + 8 <= n; q += 8) {
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = o[static_cast<size_t>(slot(base + q + i)) * D + e];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) O = fmaf(x[i], s_w[q + i], O);
+        }
+        for (; q < n; ++q) O = fmaf(o[static_cast<size_t>(slot(base + q)) * D + e], s_w[q], O);
+    }
     p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
 }
 
@@ -261,6 +290,7 @@ template <int D, bool MMA>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const PrefixParams pp, const DecodeParams dp, int n_pre) {
+    pdl_launch_dependents();
     int id = blockIdx.x;
     if (id < n_pre) {
         const int c = id % pp.prefix_parts;
@@ -292,9 +322,9 @@ cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, con
     kern<<<static_cast<unsigned>(n_pre + n_suf), kPrefixWarps * 32, kSmem, stream>>>(
         tmk, tmv, pp, dp, static_cast<int>(n_pre));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    cascade_merge_kernel<D, kPrefixChunkBlocks>
-        <<<dim3(static_cast<unsigned>(pp.Hq), static_cast<unsigned>(pp.B)), D, 0, stream>>>(pp);
-    return cudaGetLastError();
+    return launch_dependent(cascade_merge_kernel<D, kPrefixChunkBlocks>,
+                            dim3(static_cast<unsigned>(pp.Hq), static_cast<unsigned>(pp.B)), dim3(D),
+                            stream, pp);
 }
 
 }  // namespace

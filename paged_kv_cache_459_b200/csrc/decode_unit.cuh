@@ -14,6 +14,9 @@ template <int D, int NW, int S, bool MMA, bool SPLIT>
 __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtensorMap &tmv,
                                             const DecodeParams &p, int part, int by, int b) {
     using G = Geometry<D, NW, S>;
+    // The merge kernel may be scheduled as soon as every unit has started; it
+    // waits for this grid to finish before reading the partials.
+    if constexpr (SPLIT) pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kvh = MMA ? by / p.chunks : by;
     const int chunk = MMA ? by % p.chunks : 0;

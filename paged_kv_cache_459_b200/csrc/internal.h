@@ -36,7 +36,14 @@ struct DecodeParams {
     // clamped to the sequence's full blocks.
     const int32_t *start_blocks;
     bool skip_merge;  // split-K without its merge kernel (the caller merges)
+    // Optional [B]: unit z of the grid decodes sequence order[z] (longest
+    // first); written by the order kernel launched just before.
+    const int32_t *order;
 };
+
+// Longest-first order of the sequences (by block count) into order[B], for
+// the single-pass decode grid; one CTA, counting sort.
+cudaError_t launch_order(const int32_t *seq_lens, int B, int W, int32_t *order, cudaStream_t stream);
 
 struct DecodeTuning {
     int warps;   // consumer warps per CTA
@@ -71,7 +78,9 @@ struct StreamParams {
 cudaError_t launch_decode_stream(const CUtensorMap &tmk, const CUtensorMap &tmv,
                                  const StreamParams &p, int head_dim, cudaStream_t stream);
 
-// Launches the decode kernel (and the merge kernel when split) on `stream`.
+// Launches the decode kernel (and the merge kernel when split) on `stream`;
+// when p.order is set the decode grid is launched as a programmatic dependent
+// of the order kernel and waits for it.
 cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                           int head_dim, bool split, DecodeTuning tuning, cudaStream_t stream);
 

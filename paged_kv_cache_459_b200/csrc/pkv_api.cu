@@ -1,6 +1,7 @@
 // C ABI of libpkv.so: argument checks, TMA descriptor set-up and dispatch.
 // Nothing here allocates device memory; every launch goes on the caller's
 // stream.  See include/pkv.h for the contract of each entry point.
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <mutex>
@@ -193,11 +194,12 @@ size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads, 
                                                     max_blocks_per_seq, partition_tokens);
     const StreamLayout l = stream_layout(num_seqs, num_heads, num_kv_heads, head_dim);
     const size_t stream = l.dir_bytes + l.piece_bytes;
+    const size_t order = (static_cast<size_t>(num_seqs) * sizeof(int32_t) + 255) / 256 * 256;
     switch (variant) {
-        case PKV_DECODE_SINGLE: return 0;
+        case PKV_DECODE_SINGLE: return order;  // optional: longest-first scheduling
         case PKV_DECODE_SPLIT: return split;
         case PKV_DECODE_STREAM: return stream;
-        case PKV_DECODE_AUTO: return split > stream ? split : stream;
+        case PKV_DECODE_AUTO: return std::max(std::max(split, stream), order);
         default: return 0;
     }
 }
@@ -213,14 +215,18 @@ int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads, int he
         return pkv_decode_workspace_bytes_for(v, num_seqs, num_heads, num_kv_heads, head_dim,
                                               max_blocks_per_seq, partition_tokens);
     };
-    // Split only when one pass would leave the GPU short of CTAs: fewer than
-    // ~4 waves of (sequence, KV head) units at 3 CTAs per SM.  (The balanced
-    // variant measured slower than both on every workload tried, so it is
-    // only used when asked for.)
+    // Single pass, its units run longest first when the workspace holds the
+    // order (measured best on the Llama and Qwen shapes); split-K only when
+    // one pass would leave the GPU short of CTAs -- fewer than ~1.5 waves of
+    // (sequence, KV head) units at 3 CTAs per SM (without the order: 4 waves,
+    // since the tail of an unordered grid is longer).  The balanced variant
+    // measured slower than both everywhere, so it is only used when asked for.
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads *
                           ((num_heads / num_kv_heads + 7) / 8);
+    const bool ordered = workspace_bytes >= need(PKV_DECODE_SINGLE);
+    const int64_t min_units = ordered ? 3 * 3 * sm_count() / 2 : 4 * 3 * sm_count();
     if (max_blocks_per_seq > partition_tokens / PKV_BLOCK_TOKENS &&
-        workspace_bytes >= need(PKV_DECODE_SPLIT) && units < 4 * 3 * sm_count())
+        workspace_bytes >= need(PKV_DECODE_SPLIT) && units < min_units)
         return PKV_DECODE_SPLIT;
     return PKV_DECODE_SINGLE;
 }
@@ -319,6 +325,15 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
     } else {
         p.part_blocks = max_blocks_per_seq;
         p.num_parts = 1;
+        // longest sequences first, when the workspace has room for the order
+        if (workspace != nullptr && aligned16(workspace) &&
+            workspace_bytes >= static_cast<size_t>(num_seqs) * sizeof(int32_t)) {
+            int32_t *order = static_cast<int32_t *>(workspace);
+            cudaError_t e = pkv::launch_order(seq_lens, num_seqs, max_blocks_per_seq, order,
+                                              static_cast<cudaStream_t>(stream));
+            if (e != cudaSuccess) return PKV_ERR_CUDA;
+            p.order = order;
+        }
     }
     pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
     cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, split, t,

@@ -99,8 +99,8 @@ def test_variant_choice_and_workspace_sizes():
     stream = pkv.decode_workspace_bytes_for(pkv.DECODE_STREAM, B, hq, hkv, d, W)
     split = pkv.decode_workspace_bytes_for(pkv.DECODE_SPLIT, B, hq, hkv, d, W)
     assert split == pkv.decode_workspace_bytes(B, hq, d, W)
-    assert pkv.decode_workspace_bytes_for(pkv.DECODE_AUTO, B, hq, hkv, d, W) == max(split, stream)
-    assert pkv.decode_workspace_bytes_for(pkv.DECODE_SINGLE, B, hq, hkv, d, W) == 0
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_AUTO, B, hq, hkv, d, W) == max(split, stream, 256)
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_SINGLE, B, hq, hkv, d, W) == 256  # the order
     assert pkv.decode_workspace_bytes_for(pkv.DECODE_STREAM, B, 28, 5, d, W) == 0  # 28 % 5
     # no workspace: single pass; enough for the balanced variant: balanced
     assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, 0) == pkv.DECODE_SINGLE

@@ -160,3 +160,21 @@ def test_stream_variant_shapes(name, kw):
     out = d.decode(STREAM)
     check_close(out, ref, f"stream {name} {kw}")
     assert d.err_word() == 0
+
+
+def test_longest_first_order_changes_nothing_but_scheduling():
+    """The single-pass grid runs its units longest-first when the workspace can
+    hold the order; the outputs are bit-identical to the unordered grid."""
+    w = build("qwen", 15, batch=40, len_lo=1, len_hi=900)
+    d = DeviceStep(w)
+    d.write()
+    ordered = d.decode(SINGLE)  # the binding supplies the workspace
+    c = w.cfg
+    rc = pkv.lib().pkv_paged_attention_decode_ex(
+        d.out.data_ptr(), d.q.data_ptr(), d.kc.data_ptr(), d.vc.data_ptr(), d.tables.data_ptr(),
+        d.tables.shape[1], d.lens.data_ptr(), c["batch"], c["num_heads"], c["num_kv_heads"],
+        c["head_dim"], w.num_blocks, c["scale"], SINGLE, 512, None, 0, None,
+        torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == pkv.OK
+    assert np.array_equal(host_bits(d.out), ordered)
