@@ -503,8 +503,11 @@ def run_row(args):
         qs = torch.tensor([b * n for b in range(B + 1)], dtype=torch.int32, device=dev)
         sl = torch.from_numpy(np.concatenate(slots)).to(dev)
         wr_ms = _events_time(lambda: pkv.paged_kv_write(k_new, v_new, kc, vc, sl), steps, warm)
-        ms = _events_time(lambda: pkv.paged_attention_prefill(out, q, kc, vc, t_d, l_d, qs, cfg["scale"], hkv, n),
-                          steps, warm)
+        run = lambda: pkv.paged_attention_prefill(out, q, kc, vc, t_d, l_d, qs, cfg["scale"], hkv, n)  # noqa: E731
+        os.environ["PKV_PREFILL_WARP_MMA"] = "1"
+        ms_warp = _events_time(run, steps, warm)
+        os.environ.pop("PKV_PREFILL_WARP_MMA")
+        ms = _events_time(run, steps, warm)
         flops = B * 4.0 * d * hq * n * (n + 1) / 2  # causal: row i sees i + 1 keys
         peak, kind = measured_peak_tensor()
         ach = flops / (ms * 1e-3) / 1e12
@@ -512,9 +515,10 @@ def run_row(args):
                     value=ach, unit="TFLOP/s", ms_per_step=ms, higher_is_better=True,
                     config={"workload": f"{B} prompts x {n} tokens, {hq}/{hkv} heads, d {d}"},
                     prompt_write_gbs=T * hkv * d * 2 * 2 * 2 / (wr_ms * 1e-3) / 1e9,
+                    warp_mma_tflops=flops / (ms_warp * 1e-3) / 1e12,
                     roofline={"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                               "frac": ach / peak, "peak_kind": kind,
-                              "note": "warp-level mma.sync m16n8k16 (not tcgen05)"})
+                              "kernel": "paged_prefill_tc_kernel (tcgen05, TMEM accumulators)"})
     elif args.row == "cow":
         cfg = wl.config("llama")
         hkv, d, nb, n = cfg["num_kv_heads"], cfg["head_dim"], 8192, 2048

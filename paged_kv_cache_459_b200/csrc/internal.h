@@ -128,6 +128,9 @@ struct PrefillParams {
 
 cudaError_t launch_prefill(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
                            int head_dim, int max_query_len, cudaStream_t stream);
+// The same on tcgen05 / TMEM (128 query rows per CTA).
+cudaError_t launch_prefill_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
+                              int head_dim, int max_query_len, cudaStream_t stream);
 
 cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, const int64_t *dst,
                                int n, int num_kv_heads, int head_dim, long long num_blocks,

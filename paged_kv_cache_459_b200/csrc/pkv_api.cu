@@ -485,8 +485,13 @@ pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_c
     p.Hkv = num_kv_heads;
     p.group = num_heads / num_kv_heads;
     p.scale_log2 = scale * 1.4426950408889634f;
-    cudaError_t e = pkv::launch_prefill(tmk, tmv, p, head_dim, max_query_len,
-                                        static_cast<cudaStream_t>(stream));
+    // tcgen05 kernel by default; PKV_PREFILL_WARP_MMA=1 selects the warp-level
+    // mma.sync kernel (kept for comparison).
+    cudaError_t e = env_int("PKV_PREFILL_WARP_MMA", 0)
+                        ? pkv::launch_prefill(tmk, tmv, p, head_dim, max_query_len,
+                                              static_cast<cudaStream_t>(stream))
+                        : pkv::launch_prefill_tc(tmk, tmv, p, head_dim, max_query_len,
+                                                 static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -55,19 +55,31 @@ def run_prefill(hq, hkv, d, cached, new, seed):
     return host_bits(out), ref
 
 
+@pytest.fixture(params=["tcgen05", "warp_mma"])
+def prefill_impl(request, monkeypatch):
+    """The tcgen05/TMEM kernel (default) and the warp-level mma.sync kernel."""
+    if request.param == "warp_mma":
+        monkeypatch.setenv("PKV_PREFILL_WARP_MMA", "1")
+    else:
+        monkeypatch.delenv("PKV_PREFILL_WARP_MMA", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("hq,hkv,d,cached,new", [
     (4, 4, 64, [0, 0, 0], [1, 37, 100]),
     (32, 32, 128, [0, 0], [300, 129]),
     (28, 4, 128, [0, 0, 0], [5, 64, 250]),
     (8, 2, 64, [200, 16, 0], [70, 1, 33]),       # chunks after cached tokens
     (16, 1, 128, [40], [90]),                      # one KV head, 16-query groups
+    (8, 8, 128, [0, 1000], [700, 300]),            # several 64-key tiles, lazy rescaling
+    (28, 4, 64, [0], [200]),                       # 1400 rows: several 128-row CTAs
 ])
-def test_prefill_matches_oracle(hq, hkv, d, cached, new):
+def test_prefill_matches_oracle(hq, hkv, d, cached, new, prefill_impl):
     out, ref = run_prefill(hq, hkv, d, cached, new, seed=hq + d + len(new))
     check_close(out, ref, f"prefill {hq}/{hkv} d{d} cached {cached} new {new}")
 
 
-def test_prefill_last_row_equals_decode():
+def test_prefill_last_row_equals_decode(prefill_impl):
     """The prompt's last token attends exactly as a decode step at that length."""
     out, ref = run_prefill(8, 8, 128, [0], [77], seed=9)
     check_close(out[-1:], ref[-1:], "last row")
