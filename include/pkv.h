@@ -86,6 +86,12 @@ typedef enum {
 /* Human-readable name of a pkv_status value (static storage). */
 PKV_API const char *pkv_status_string(int status);
 
+/* The CUDA runtime error (cudaError_t value) behind the last PKV_ERR_CUDA
+ * returned on the calling thread, 0 if none yet, and its text.  Added for
+ * diagnostics; the pages have no counterpart. */
+PKV_API int pkv_last_cuda_error(void);
+PKV_API const char *pkv_last_cuda_error_string(void);
+
 /* Tokens per physical block (16). */
 PKV_API int pkv_block_tokens(void);
 

@@ -124,13 +124,15 @@ struct PrefillParams {
     long long num_blocks;
     int W, B, Hq, Hkv, group;
     float scale_log2;
+    int items;  // work items of the persistent tcgen05 kernel (set by its launcher)
 };
 
 cudaError_t launch_prefill(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
                            int head_dim, int max_query_len, cudaStream_t stream);
-// The same on tcgen05 / TMEM (128 query rows per CTA).
+// The same on tcgen05 / TMEM: a persistent kernel, one CTA per SM, work
+// items of two 128-row Q tiles.
 cudaError_t launch_prefill_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
-                              int head_dim, int max_query_len, cudaStream_t stream);
+                              int head_dim, int max_query_len, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, const int64_t *dst,
                                int n, int num_kv_heads, int head_dim, long long num_blocks,

@@ -53,6 +53,15 @@ int env_int(const char *name, int fallback) {
     return (s && *s) ? std::atoi(s) : fallback;
 }
 
+// The CUDA error behind the last PKV_ERR_CUDA returned on this thread.
+thread_local int g_last_cuda_error = 0;
+
+pkv_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return PKV_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return PKV_ERR_CUDA;
+}
+
 // Streaming multiprocessors of the current device (148 on B200).
 int sm_count() {
     int dev = 0, n = 0;
@@ -70,6 +79,12 @@ int num_parts_for(int max_blocks_per_seq, int partition_tokens) {
 }  // namespace
 
 extern "C" {
+
+int pkv_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *pkv_last_cuda_error_string(void) {
+    return cudaGetErrorString(static_cast<cudaError_t>(g_last_cuda_error));
+}
 
 const char *pkv_status_string(int status) {
     switch (status) {
@@ -102,7 +117,7 @@ pkv_status pkv_paged_kv_write(const void *k, const void *v, void *k_cache, void 
     cudaError_t e = pkv::launch_kv_write(k, v, k_cache, v_cache, slot_mapping, num_tokens,
                                          num_kv_heads, head_dim, num_blocks, err_word,
                                          static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cuda_status(e);
 }
 
 pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, const int64_t *dst,
@@ -115,7 +130,7 @@ pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, const int64_t *src, con
         return PKV_ERR_INVALID_ARG;
     cudaError_t e = pkv::launch_copy_blocks(k_cache, v_cache, src, dst, n, num_kv_heads, head_dim,
                                             num_blocks, err_word, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cuda_status(e);
 }
 
 // Device address of pinned, device-mapped host memory, or nullptr.
@@ -148,7 +163,7 @@ pkv_status pkv_swap_blocks(void *k_cache, void *v_cache, void *host_k, void *hos
                                             direction, num_kv_heads, head_dim, num_blocks,
                                             num_host_blocks, err_word,
                                             static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cuda_status(e);
 }
 
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
@@ -298,7 +313,7 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
         sp.scale_log2 = scale * 1.4426950408889634f;
         cudaError_t e = pkv::launch_decode_stream(tmk, tmv, sp, head_dim,
                                                   static_cast<cudaStream_t>(stream));
-        return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+        return cuda_status(e);
     }
 
     pkv::DecodeParams p{};
@@ -331,14 +346,14 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
             int32_t *order = static_cast<int32_t *>(workspace);
             cudaError_t e = pkv::launch_order(seq_lens, num_seqs, max_blocks_per_seq, order,
                                               static_cast<cudaStream_t>(stream));
-            if (e != cudaSuccess) return PKV_ERR_CUDA;
+            if (e != cudaSuccess) return cuda_status(e);
             p.order = order;
         }
     }
     pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
     cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, split, t,
                                        static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cuda_status(e);
 }
 
 size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
@@ -443,7 +458,7 @@ pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const voi
 
     cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
                                         static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cuda_status(e);
 }
 
 pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_cache,
@@ -490,9 +505,9 @@ pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_c
     cudaError_t e = env_int("PKV_PREFILL_WARP_MMA", 0)
                         ? pkv::launch_prefill(tmk, tmv, p, head_dim, max_query_len,
                                               static_cast<cudaStream_t>(stream))
-                        : pkv::launch_prefill_tc(tmk, tmv, p, head_dim, max_query_len,
+                        : pkv::launch_prefill_tc(tmk, tmv, p, head_dim, max_query_len, sm_count(),
                                                  static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return cuda_status(e);
 }
 
 pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,

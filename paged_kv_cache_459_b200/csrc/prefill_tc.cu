@@ -2,22 +2,27 @@
 //
 // Same result as paged_prefill_kernel (prefill.cu): causal attention of each
 // sequence's new tokens over its paged K/V ("vLLM 與 PagedAttention：高吞吐推理
-// 的關鍵", section 三 step 二).  A CTA owns 128 query rows -- (token, query
-// head of one KV head) pairs -- and walks the keys its rows can see in tiles
-// of 64 (four 16-token blocks):
-//   S[128 x 64]  = Q[128 x d] K_tile^T      tcgen05.mma, accumulator in TMEM
-//   P = exp2(S - m)  (bf16, 128-byte-swizzled shared memory)
-//   O[128 x d]  += P[128 x 64] V_tile       tcgen05.mma, accumulator in TMEM
-// Roles: a producer warp streams K and V tiles (TMA, 128-byte swizzle, 3
-// stages; blocks past the table or the pool load as zeros from out-of-range
-// coordinates); one thread of the MMA warp issues the products and commits
-// them to mbarriers; four softmax warps own one row each per thread (TMEM
-// lane = row), read S with tcgen05.ld, mask (causal, sequence end), keep the
-// running max and sum, write P, and rescale O in TMEM only when a row's max
-// grows by more than 2^8 (otherwise the old max is kept: P stays <= 2^8).
-// S is double-buffered in TMEM so that the next S product overlaps softmax.
+// 的關鍵", section 三 step 二).  A CTA owns two Q tiles of 128 query rows each
+// -- (token, query head of one KV head) pairs -- and walks the keys its rows
+// can see in tiles of 128 (eight 16-token blocks); both Q tiles share each
+// K/V tile.  Per Q tile x:
+//   S_x[128 x 128] = Q_x[128 x d] K_tile^T   tcgen05.mma (A, B in shared memory)
+//   P_x = exp2(S_x - m), bf16, written back into TMEM over S_x
+//   O_x[128 x d]  += P_x V_tile              tcgen05.mma (A in TMEM, B in shared memory)
+// with S, P and O accumulated in TMEM (512 columns).
+// Roles: a producer warp streams K and V tiles (TMA, 128-byte swizzle, K and
+// V in separate rings; blocks past the table or the pool load as zeros from
+// out-of-range coordinates); one thread of the MMA warp issues the products
+// and commits them to mbarriers; one softmax warpgroup per Q tile owns one
+// row per thread (TMEM lane = row), reads S with tcgen05.ld, masks (causal,
+// sequence end), keeps the running max and sum, stores P with tcgen05.st, and
+// rescales O in TMEM only when a row's max grows by more than 2^8 (otherwise
+// the old max is kept: P stays <= 2^8).  The two Q tiles ping-pong: the tensor
+// core computes one tile's products while the other tile's softmax runs.
 // Every wait is bounded; on a timeout the kernel flags PKV_DEV_ERR_TIMEOUT,
 // stops issuing, and still frees its TMEM.
+#include <algorithm>
+
 #include "decode_common.cuh"
 
 namespace pkv {
@@ -26,13 +31,14 @@ namespace {
 
 using namespace dev;
 
-constexpr int kRows = 128;                 // query rows per CTA (MMA M)
-constexpr int kKeys = 64;                  // keys per tile (MMA N of S, K of P.V)
-constexpr int kStages = 3;
-constexpr int kSoftmaxWarps = 4;
-constexpr int kProducerWarp = 4, kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
-constexpr int kTmemCols = 256;             // S0 [0,64) S1 [64,128) O [128, 128 + d)
+constexpr int kRows = 128;                 // query rows per Q tile (MMA M)
+constexpr int kTiles = 2;                  // Q tiles per CTA, ping-ponged on the tensor core
+constexpr int kCtaRows = kTiles * kRows;
+constexpr int kKeys = 128;                 // keys per tile (MMA N of S, K of P.V)
+constexpr int kWarpsPerTile = 4;           // one softmax warpgroup per Q tile
+constexpr int kSoftmaxWarps = kTiles * kWarpsPerTile;
+constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -56,6 +62,17 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, ui
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(static_cast<int>(accumulate))
+        : "memory");
+}
+
+// The same with A read from tensor memory (K-major: row = lane, two 16-bit
+// elements per 32-bit column).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                        bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(static_cast<int>(accumulate))
         : "memory");
 }
 
@@ -86,7 +103,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+// The same without the wait: several loads may be in flight before one
+// tcgen05.wait::ld.
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
         "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
@@ -102,68 +135,125 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 template <int D>
 struct TcGeometry {
     static constexpr int kHalves = D / 64;
-    static constexpr int kQBytes = kHalves * kRows * 128;      // Q [half][row][128 B]
+    static constexpr int kKStages = D == 128 ? 3 : 4;           // K ring depth
+    static constexpr int kVStages = D == 128 ? 2 : 4;           // V ring depth
+    static constexpr int kQBytes = kHalves * kRows * 128;      // one Q tile [half][row][128 B]
     static constexpr int kKVBytes = kHalves * kKeys * 128;     // K or V tile [half][key][128 B]
-    static constexpr int kPBytes = kRows * 128;                // P [row][64 keys = 128 B]
-    static constexpr int kQ = 0;
-    static constexpr int kK = kQ + kQBytes;                    // + stage * kKVBytes
-    static constexpr int kV = kK + kStages * kKVBytes;
-    static constexpr int kP = kV + kStages * kKVBytes;
-    static constexpr int kBars = kP + kPBytes;                 // 16 mbarriers
-    static constexpr int kTmemSlot = kBars + 16 * 8;
+    static constexpr int kQ = 0;                               // + tile * kQBytes
+    static constexpr int kK = kQ + kTiles * kQBytes;           // + stage * kKVBytes
+    static constexpr int kV = kK + kKStages * kKVBytes;
+    static constexpr int kBars = kV + kVStages * kKVBytes;     // up to 32 mbarriers
+    static constexpr int kTmemSlot = kBars + 32 * 8;
     static constexpr int kSmemBytes = kTmemSlot + 16 + 1024;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static_assert(2 * (kKStages + kVStages) + 10 <= 32, "barrier slots");
+    // TMEM columns: S of tile x at kKeys x (P, bf16, over its first half),
+    // O of tile x at kO + D x.
+    static constexpr int kO = kTiles * kKeys;
+    static constexpr int kTmemCols = 512;
+    static_assert(kO + kTiles * D <= kTmemCols, "tensor memory columns");
 };
 
+// One work item: 256 query rows (two Q tiles) of one (sequence, KV head).
+struct TcItem {
+    int b, kvh, q0, ctx, rows, r_begin, first_pos, nblk_seq;
+    int nk0, nk1;  // key tiles Q tile 0 / 1 can see (tile 1 may be empty: 0)
+};
+
+// Items are numbered z-major -- z counts 256-row tiles from the END of each
+// sequence, so low numbers see the most keys -- then sequence, then KV head.
+// Returns false for items past a sequence's rows or of a sequence whose
+// lengths are inconsistent (*bad set for the latter).
+__device__ __forceinline__ bool tc_item(const PrefillParams &p, int i, TcItem &it, bool *bad) {
+    const int per_z = p.Hkv * p.B;
+    const int z = i / per_z, rem = i - z * per_z;
+    it.b = rem / p.Hkv;
+    it.kvh = rem - it.b * p.Hkv;
+    it.q0 = __ldg(p.query_start + it.b);
+    const int nq = __ldg(p.query_start + it.b + 1) - it.q0;
+    it.ctx = __ldg(p.seq_lens + it.b);
+    *bad = nq > 0 && (it.ctx < nq || it.ctx > p.W * kBlockTokens);
+    if (nq <= 0 || *bad) return false;
+    it.rows = nq * p.group;
+    const int ntile = (it.rows + kCtaRows - 1) / kCtaRows;
+    if (z >= ntile) return false;
+    it.r_begin = (ntile - 1 - z) * kCtaRows;
+    it.first_pos = it.ctx - nq;
+    it.nblk_seq = (it.ctx + kBlockTokens - 1) / kBlockTokens;
+    const int last0 = min(it.rows, it.r_begin + kRows) - 1;
+    it.nk0 = (it.first_pos + last0 / p.group + kKeys) / kKeys;
+    const int lo1 = it.r_begin + kRows;
+    it.nk1 = lo1 < it.rows ? (it.first_pos + (min(it.rows, lo1 + kRows) - 1) / p.group + kKeys) / kKeys : 0;
+    return true;
+}
+
+// The k-th item of CTA c in a grid of n CTAs: rounds of n items, alternately
+// forwards and backwards ("snake"), so heavy and light items even out.
+__device__ __forceinline__ int tc_item_index(int k, int c, int n) {
+    return k * n + ((k & 1) ? n - 1 - c : c);
+}
+
+// Next valid item of this CTA at or after round k; returns its round or -1.
+__device__ __forceinline__ int tc_next_item(const PrefillParams &p, int k, TcItem &it) {
+    for (;; ++k) {
+        const int i = tc_item_index(k, blockIdx.x, gridDim.x);
+        if (i >= p.items) return -1;
+        bool bad;
+        if (tc_item(p, i, it, &bad)) return k;
+    }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// Persistent: one CTA per SM walks its items; TMEM is allocated once, every
+// barrier's phase runs on across items, and the next item's Q rows are
+// fetched (cp.async) as soon as the current item's last S product is done.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv, const PrefillParams p) {
     using Geo = TcGeometry<D>;
-    const int b = blockIdx.z, kvh = blockIdx.y;
+    constexpr int KS = Geo::kKStages, VS = Geo::kVStages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group;
-
-    const int q0 = __ldg(p.query_start + b), q1 = __ldg(p.query_start + b + 1);
-    const int ctx = __ldg(p.seq_lens + b);
-    const int nq = q1 - q0;
-    if (nq <= 0 || ctx < nq || ctx > p.W * kBlockTokens) {
-        if (nq > 0 && blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0) flag(p.err, PKV_DEV_ERR_BAD_LEN);
-        return;
-    }
-    const int rows = nq * G;
-    const int ntiles_q = (rows + kRows - 1) / kRows;
-    if (static_cast<int>(blockIdx.x) >= ntiles_q) return;
-    const int r_begin = (ntiles_q - 1 - static_cast<int>(blockIdx.x)) * kRows;  // heaviest first
-    const int first_pos = ctx - nq;
-    const int last_row = min(rows, r_begin + kRows) - 1;
-    const int kv_end = first_pos + last_row / G + 1;        // keys this CTA can see
-    const int nk = (kv_end + kKeys - 1) / kKeys;            // key tiles
-    const int nblk_seq = (ctx + kBlockTokens - 1) / kBlockTokens;
-    const long long oob_row = p.num_blocks * p.Hkv * kBlockTokens;  // past the tensor: zero fill
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t bar0 = smem_u32(smem + Geo::kBars);
-    // barriers: kv_full[3] kv_empty[3] s_full[2] s_free[2] p_full o_done
-    const auto kv_full = [&](int s) { return bar0 + 8 * s; };
-    const auto kv_empty = [&](int s) { return bar0 + 8 * (3 + s); };
-    const auto s_full = [&](int i) { return bar0 + 8 * (6 + i); };
-    const auto s_free = [&](int i) { return bar0 + 8 * (8 + i); };
-    const uint32_t p_full = bar0 + 8 * 10, o_done = bar0 + 8 * 11;
+    // barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS], then per Q tile
+    // s_full p_full o_done q_full o_free
+    const auto k_full = [&](int s) { return bar0 + 8 * s; };
+    const auto k_empty = [&](int s) { return bar0 + 8 * (KS + s); };
+    const auto v_full = [&](int s) { return bar0 + 8 * (2 * KS + s); };
+    const auto v_empty = [&](int s) { return bar0 + 8 * (2 * KS + VS + s); };
+    const uint32_t tile_bars = bar0 + 8 * (2 * KS + 2 * VS);
+    const auto s_full = [&](int x) { return tile_bars + 8 * x; };
+    const auto p_full = [&](int x) { return tile_bars + 8 * (2 + x); };
+    const auto o_done = [&](int x) { return tile_bars + 8 * (4 + x); };
+    const auto q_full = [&](int x) { return tile_bars + 8 * (6 + x); };
+    const auto o_free = [&](int x) { return tile_bars + 8 * (8 + x); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Geo::kTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Geo::kTmemSlot + 4);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(kv_full(s), 1);
-            mbar_init(kv_empty(s), 1);
+        for (int s = 0; s < KS; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(k_empty(s), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(s_full(i), 1);
-            mbar_init(s_free(i), kSoftmaxWarps);
+        for (int s = 0; s < VS; ++s) {
+            mbar_init(v_full(s), 1);
+            mbar_init(v_empty(s), 1);
         }
-        mbar_init(p_full, kSoftmaxWarps);
-        mbar_init(o_done, 1);
+        for (int x = 0; x < kTiles; ++x) {
+            mbar_init(s_full(x), 1);
+            mbar_init(p_full(x), kWarpsPerTile);
+            mbar_init(o_done(x), 1);
+            mbar_init(q_full(x), kWarpsPerTile);
+            mbar_init(o_free(x), kWarpsPerTile);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmk);
@@ -172,90 +262,121 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
-                     "n"(kTmemCols)
+                     "n"(Geo::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    // Q rows into shared memory (K-major, 128-byte swizzle): softmax thread t owns row t.
-    int row_pos = -1;
-    size_t out_off = 0;
-    if (warp < kSoftmaxWarps) {
-        const int t = threadIdx.x;
-        const int r = r_begin + t;
-        const uint4 *src = nullptr;
-        if (r < rows) {
-            const int tok = r / G, h = kvh * G + r % G;
-            row_pos = first_pos + tok;
-            out_off = (static_cast<size_t>(q0 + tok) * p.Hq + h) * D;
-            src = reinterpret_cast<const uint4 *>(p.q + out_off);
-        }
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            const uint4 v = src ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(smem + Geo::kQ + (c >> 3) * (kRows * 128) + t * 128 +
-                                       (((c & 7) ^ (t & 7)) << 4)) = v;
-        }
-        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_o = tmem + 128;
 
     if (warp == kProducerWarp) {
         if (lane == 0) {
             const uint64_t policy = l2_policy_evict_normal();
-            const int32_t *trow = p.block_tables + static_cast<size_t>(b) * p.W;
-            for (int j = 0; j < nk && !*abort_flag; ++j) {
-                const int s = j % kStages;
-                if (j >= kStages &&
-                    !mbar_wait(kv_empty(s), static_cast<uint32_t>((j / kStages - 1) & 1), kWaitLimitNs)) {
-                    flag(p.err, PKV_DEV_ERR_TIMEOUT);
-                    *abort_flag = 1;
-                    break;
-                }
-                mbar_arrive_expect_tx(kv_full(s), 2 * Geo::kKVBytes);
-                for (int i = 0; i < kKeys / kBlockTokens; ++i) {
-                    const int blk = j * (kKeys / kBlockTokens) + i;
-                    long long y = oob_row;  // blocks past the sequence or bad entries read as zeros
-                    if (blk < nblk_seq) {
-                        const int32_t phys = __ldg(trow + blk);
-                        if (phys >= 0 && phys < p.num_blocks)
-                            y = (static_cast<long long>(phys) * p.Hkv + kvh) * kBlockTokens;
-                        else
-                            flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
-                    }
+            int gk = 0, gv = 0;  // K / V tiles loaded so far (ring position and phase)
+            TcItem it;
+            for (int k = tc_next_item(p, 0, it); k >= 0 && !*abort_flag; k = tc_next_item(p, k + 1, it)) {
+                const int32_t *trow = p.block_tables + static_cast<size_t>(it.b) * p.W;
+                const int nk = max(it.nk0, it.nk1);
+                for (int j = 0; j < nk && !*abort_flag; ++j) {
+                    int y[kKeys / kBlockTokens];  // tensor-map rows of the tile's blocks
 #pragma unroll
-                    for (int hh = 0; hh < Geo::kHalves; ++hh) {
-                        const uint32_t off = hh * (kKeys * 128) + i * (kBlockTokens * 128);
-                        tma_load_2d(smem_u32(smem + Geo::kK + s * Geo::kKVBytes) + off, &tmk, hh * 64,
-                                    static_cast<int>(y), kv_full(s), policy);
-                        tma_load_2d(smem_u32(smem + Geo::kV + s * Geo::kKVBytes) + off, &tmv, hh * 64,
-                                    static_cast<int>(y), kv_full(s), policy);
+                    for (int i = 0; i < kKeys / kBlockTokens; ++i) {
+                        const int blk = j * (kKeys / kBlockTokens) + i;
+                        long long yy = p.num_blocks * p.Hkv * kBlockTokens;  // past the tensor: zeros
+                        if (blk < it.nblk_seq) {
+                            const int32_t phys = __ldg(trow + blk);
+                            if (phys >= 0 && phys < p.num_blocks)
+                                yy = (static_cast<long long>(phys) * p.Hkv + it.kvh) * kBlockTokens;
+                            else
+                                flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
+                        }
+                        y[i] = static_cast<int>(yy);
                     }
+                    const int sk = gk % KS, sv = gv % VS;
+                    if (gk >= KS &&
+                        !mbar_wait(k_empty(sk), static_cast<uint32_t>((gk / KS - 1) & 1), kWaitLimitNs)) {
+                        flag(p.err, PKV_DEV_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(k_full(sk), Geo::kKVBytes);
+#pragma unroll
+                    for (int i = 0; i < kKeys / kBlockTokens; ++i)
+#pragma unroll
+                        for (int hh = 0; hh < Geo::kHalves; ++hh)
+                            tma_load_2d(smem_u32(smem + Geo::kK + sk * Geo::kKVBytes) +
+                                            hh * (kKeys * 128) + i * (kBlockTokens * 128),
+                                        &tmk, hh * 64, y[i], k_full(sk), policy);
+                    ++gk;
+                    if (gv >= VS &&
+                        !mbar_wait(v_empty(sv), static_cast<uint32_t>((gv / VS - 1) & 1), kWaitLimitNs)) {
+                        flag(p.err, PKV_DEV_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(v_full(sv), Geo::kKVBytes);
+#pragma unroll
+                    for (int i = 0; i < kKeys / kBlockTokens; ++i)
+#pragma unroll
+                        for (int hh = 0; hh < Geo::kHalves; ++hh)
+                            tma_load_2d(smem_u32(smem + Geo::kV + sv * Geo::kKVBytes) +
+                                            hh * (kKeys * 128) + i * (kBlockTokens * 128),
+                                        &tmv, hh * 64, y[i], v_full(sv), policy);
+                    ++gv;
+                }
+            }
+            // on an abort, copies may still be landing: wait (bounded) for the last of each stage
+            for (int g = max(gk - KS, 0); g < gk; ++g)
+                mbar_wait(k_full(g % KS), static_cast<uint32_t>((g / KS) & 1), kWaitLimitNs);
+            for (int g = max(gv - VS, 0); g < gv; ++g)
+                mbar_wait(v_full(g % VS), static_cast<uint32_t>((g / VS) & 1), kWaitLimitNs);
+            // sequences whose lengths do not fit: flagged once each (item z = 0, KV head 0)
+            for (int k = 0;; ++k) {
+                const int i = tc_item_index(k, blockIdx.x, gridDim.x);
+                if (i >= p.items) break;
+                if (i < p.Hkv * p.B && i % p.Hkv == 0) {
+                    TcItem bad_it;
+                    bool bad;
+                    tc_item(p, i, bad_it, &bad);
+                    if (bad) flag(p.err, PKV_DEV_ERR_BAD_LEN);
                 }
             }
         }
     } else if (warp == kMmaWarp) {
+        // Per item: S_0(0), S_1(0); then per key tile j: PV_0(j), S_0(j+1),
+        // PV_1(j), S_1(j+1).  The tensor core runs them in that order, so
+        // while tile 0's softmax works on S_0(j+1) the products of tile 1
+        // proceed, and the other way round.  S_x(j+1) is issued only after
+        // P_x(j) is ready, by which time tile x's softmax has read S_x(j) out
+        // of TMEM; it overwrites P_x(j) (which aliases S_x) only after PV_x(j),
+        // issued before it, has read it; and its completion tells the
+        // softmax that PV_x(j) is done.
         constexpr uint32_t kIdS = umma_idesc(kRows, kKeys, 0);
         constexpr uint32_t kIdO = umma_idesc(kRows, D, 1);
-        const auto issue_s = [&](int j) {  // S[j % 2] = Q . K_j^T
-            const int s = j % kStages;
-            const uint32_t kbase = smem_u32(smem + Geo::kK + s * Geo::kKVBytes);
-            const uint32_t qbase = smem_u32(smem + Geo::kQ);
+        const auto issue_s = [&](int x, int stage) {  // S_x = Q_x . K^T
+            const uint32_t kbase = smem_u32(smem + Geo::kK + stage * Geo::kKVBytes);
+            const uint32_t qbase = smem_u32(smem + Geo::kQ + x * Geo::kQBytes);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const int hh = k >> 2, kk = k & 3;
-                umma(tmem + 64 * (j & 1), umma_desc(qbase + hh * (kRows * 128) + kk * 32, 16, 1024),
+                umma(tmem + kKeys * x, umma_desc(qbase + hh * (kRows * 128) + kk * 32, 16, 1024),
                      umma_desc(kbase + hh * (kKeys * 128) + kk * 32, 16, 1024), kIdS, k > 0);
             }
-            umma_commit(s_full(j & 1));
+            umma_commit(s_full(x));
+        };
+        const auto issue_pv = [&](int x, int stage, bool acc) {  // O_x (+)= P_x . V, P_x from TMEM
+            const uint32_t vbase = smem_u32(smem + Geo::kV + stage * Geo::kKVBytes);
+#pragma unroll
+            for (int k = 0; k < kKeys / 16; ++k)
+                umma_ts(tmem + Geo::kO + D * x, tmem + kKeys * x + 8 * k,
+                        umma_desc(vbase + k * (16 * 128), kKeys * 128, 1024), kIdO, acc || k > 0);
         };
         bool ok = true;
         const auto wait = [&](uint32_t bar, uint32_t parity) {
             if (!ok) return;
-            if (!mbar_wait(bar, parity, kWaitLimitNs)) {
+            if (!mbar_wait(bar, parity, kWaitLimitNs) || *abort_flag) {
                 ok = false;
                 if (lane == 0) {
                     flag(p.err, PKV_DEV_ERR_TIMEOUT);
@@ -263,168 +384,294 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        wait(kv_full(0), 0);
-        tc_fence_after();
-        if (ok && lane == 0) issue_s(0);
-        __syncwarp();
-        for (int j = 0; j < nk && ok; ++j) {
-            if (j + 1 < nk) {
-                const int t = j + 1;
-                wait(kv_full(t % kStages), static_cast<uint32_t>((t / kStages) & 1));
-                if (t >= 2) wait(s_free(t & 1), static_cast<uint32_t>(((t - 2) / 2) & 1));
-                tc_fence_after();
-                if (ok && lane == 0) issue_s(t);
-                __syncwarp();
-            }
-            // V rows of slots at or past the sequence end may hold anything: zero them
-            const int s = j % kStages;
-            const int k_lo = j * kKeys;
-            if (ok && k_lo + kKeys > ctx && k_lo < nblk_seq * kBlockTokens) {
-                const int z0 = max(ctx - k_lo, 0), z1 = min(nblk_seq * kBlockTokens - k_lo, kKeys);
-                uint8_t *vbase = smem + Geo::kV + s * Geo::kKVBytes;
-                for (int idx = lane; idx < (z1 - z0) * Geo::kHalves * 8; idx += 32) {
-                    const int rr = z0 + idx / (Geo::kHalves * 8), rest = idx % (Geo::kHalves * 8);
-                    *reinterpret_cast<uint4 *>(vbase + (rest >> 3) * (kKeys * 128) + rr * 128 +
-                                               ((rest & 7) << 4)) = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            wait(p_full, static_cast<uint32_t>(j & 1));
+        int gk = 0, gv = 0;      // K / V tiles consumed
+        int ns[kTiles] = {0, 0};  // S products per Q tile (s_full / p_full phases)
+        int n_it = 0;            // items done (q_full / o_done / o_free phases)
+        TcItem it;
+        for (int k = tc_next_item(p, 0, it); k >= 0 && ok; k = tc_next_item(p, k + 1, it), ++n_it) {
+            const int nk_t[kTiles] = {it.nk0, it.nk1};
+            const int nk = max(it.nk0, it.nk1);
+            wait(q_full(0), static_cast<uint32_t>(n_it & 1));
+            wait(q_full(1), static_cast<uint32_t>(n_it & 1));
+            wait(k_full(gk % KS), static_cast<uint32_t>((gk / KS) & 1));
             tc_fence_after();
             if (ok && lane == 0) {
-                const uint32_t pbase = smem_u32(smem + Geo::kP);
-                const uint32_t vbase = smem_u32(smem + Geo::kV + s * Geo::kKVBytes);
-#pragma unroll
-                for (int k = 0; k < kKeys / 16; ++k)
-                    umma(t_o, umma_desc(pbase + k * 32, 16, 1024),
-                         umma_desc(vbase + k * (16 * 128), kKeys * 128, 1024), kIdO, j > 0 || k > 0);
-                umma_commit(o_done);
-                umma_commit(kv_empty(s));
+                for (int x = 0; x < kTiles; ++x)
+                    if (nk_t[x] > 0) issue_s(x, gk % KS);
+                umma_commit(k_empty(gk % KS));
             }
             __syncwarp();
+            ++gk;
+            for (int j = 0; j < nk && ok; ++j, ++gv) {
+                const int sv = gv % VS;
+                wait(v_full(sv), static_cast<uint32_t>((gv / VS) & 1));
+                // V rows of slots at or past the sequence end may hold anything: zero them
+                const int k_lo = j * kKeys;
+                if (ok && k_lo + kKeys > it.ctx && k_lo < it.nblk_seq * kBlockTokens) {
+                    const int z0 = max(it.ctx - k_lo, 0), z1 = min(it.nblk_seq * kBlockTokens - k_lo, kKeys);
+                    uint8_t *vbase = smem + Geo::kV + sv * Geo::kKVBytes;
+                    for (int idx = lane; idx < (z1 - z0) * Geo::kHalves * 8; idx += 32) {
+                        const int rr = z0 + idx / (Geo::kHalves * 8), rest = idx % (Geo::kHalves * 8);
+                        *reinterpret_cast<uint4 *>(vbase + (rest >> 3) * (kKeys * 128) + rr * 128 +
+                                                   ((rest & 7) << 4)) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                // the last tile that reads V_j (and K_{j+1}) releases its stage
+                const int last_v = j < nk_t[1] ? 1 : 0;
+                const int last_k = j + 1 < nk_t[1] ? 1 : 0;
+                bool next_ready = false;
+#pragma unroll
+                for (int x = 0; x < kTiles; ++x) {
+                    if (j >= nk_t[x]) continue;
+                    wait(p_full(x), static_cast<uint32_t>(ns[x] & 1));
+                    if (j == 0 && n_it > 0) wait(o_free(x), static_cast<uint32_t>((n_it - 1) & 1));
+                    tc_fence_after();
+                    if (ok && lane == 0) {
+                        issue_pv(x, sv, j > 0);
+                        if (x == last_v) umma_commit(v_empty(sv));
+                        if (j + 1 >= nk_t[x]) umma_commit(o_done(x));
+                    }
+                    ++ns[x];
+                    if (j + 1 < nk_t[x]) {
+                        if (!next_ready) {
+                            wait(k_full(gk % KS), static_cast<uint32_t>((gk / KS) & 1));
+                            tc_fence_after();
+                            next_ready = true;
+                        }
+                        if (ok && lane == 0) {
+                            issue_s(x, gk % KS);
+                            if (x == last_k) umma_commit(k_empty(gk % KS));
+                        }
+                    }
+                    __syncwarp();
+                }
+                if (next_ready) ++gk;
+            }
+            // a Q tile without rows in this item still takes its phases
+            for (int x = 0; x < kTiles; ++x) {
+                if (nk_t[x] > 0) continue;
+                if (n_it > 0) wait(o_free(x), static_cast<uint32_t>((n_it - 1) & 1));
+                if (ok && lane == 0) umma_commit(o_done(x));
+                __syncwarp();
+            }
         }
     } else {
-        // ---------------- softmax warps: thread t = TMEM lane t = row r_begin + t
-        const int t = threadIdx.x;
-        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-        float m_run = -INFINITY, l_run = 0.f;
-        bool ok = true;
-        for (int j = 0; j < nk && ok; ++j) {
-            if (!mbar_wait(s_full(j & 1), static_cast<uint32_t>((j >> 1) & 1), kWaitLimitNs) ||
-                *abort_flag) {
-                ok = false;
-                break;
+        // ---------------- softmax warps: thread t of tile x = TMEM lane t = row r_begin + 128 x + t
+        const int tile = warp / kWarpsPerTile;
+        const int t = threadIdx.x & (kRows - 1);
+        const uint32_t lane_addr = static_cast<uint32_t>((warp % kWarpsPerTile) * 32) << 16;
+        const uint32_t t_s = tmem + lane_addr + kKeys * tile;
+        const uint32_t t_o = tmem + lane_addr + Geo::kO + D * tile;
+        uint8_t *qrow = smem + Geo::kQ + tile * Geo::kQBytes + t * 128;
+        // this thread's Q row of an item into shared memory (K-major, 128-byte
+        // swizzle; rows past the item's rows are zero-filled)
+        const auto fetch_q = [&](const TcItem &nx) {
+            const int r = nx.r_begin + tile * kRows + t;
+            const __nv_bfloat16 *src = p.q;
+            uint32_t bytes = 0;
+            if (r < nx.rows) {
+                src = p.q + (static_cast<size_t>(nx.q0 + r / G) * p.Hq + nx.kvh * G + r % G) * D;
+                bytes = 16;
             }
-            tc_fence_after();
-            uint32_t sr[2][32];
-            tmem_ld32(tmem + lane_addr + 64 * (j & 1), sr[0]);
-            tmem_ld32(tmem + lane_addr + 64 * (j & 1) + 32, sr[1]);
-            tc_fence_before();
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c)
+                cp_async16(smem_u32(qrow + (c >> 3) * (kRows * 128) + (((c & 7) ^ (t & 7)) << 4)),
+                           src + (bytes ? c * 8 : 0), bytes);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        const auto publish_q = [&]() {  // the fetched rows, to the tensor core
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(s_free(j & 1));
-            // scores in the exp2 domain, causal mask by position
-            float s[kKeys];
-            float mx = -INFINITY;
-            const int k0 = j * kKeys;
-#pragma unroll
-            for (int c = 0; c < kKeys; ++c) {
-                const float v = __uint_as_float(sr[c >> 5][c & 31]) * p.scale_log2;
-                s[c] = (k0 + c <= row_pos) ? v : -INFINITY;
-                mx = fmaxf(mx, s[c]);
+            if (lane == 0) mbar_arrive(q_full(tile));
+        };
+        bool ok = true;
+        int ns = 0;    // S products seen (s_full / p_full phases)
+        int n_it = 0;  // items done (o_done phases)
+        TcItem it;     // the current item until its last S product, then the next one
+        int k = tc_next_item(p, 0, it);
+        if (k >= 0) {
+            fetch_q(it);
+            publish_q();
+        }
+        while (k >= 0 && ok) {
+            const int r = it.r_begin + tile * kRows + t;
+            const int row_pos = r < it.rows ? it.first_pos + r / G : -1;
+            const int my_nk = tile == 0 ? it.nk0 : it.nk1;
+            __nv_bfloat16 *out_row =
+                p.out + (static_cast<size_t>(it.q0 + r / G) * p.Hq + it.kvh * G + r % G) * D;
+            float m_run = -INFINITY, l_run = 0.f;
+            int kn = -1;
+            if (my_nk == 0) {
+                kn = tc_next_item(p, k + 1, it);
+                if (kn >= 0) fetch_q(it);
             }
-            // keep the running max unless it grows by more than 2^8
-            const bool grow = mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx != -INFINITY);
-            const float m_new = grow ? mx : m_run;
-            const float base = m_new == -INFINITY ? 0.f : m_new;
-            float rowsum = 0.f;
-            uint32_t pk[kKeys / 2];
-#pragma unroll
-            for (int c = 0; c < kKeys; c += 2) {
-                const float a = exp2f(s[c] - base), bb = exp2f(s[c + 1] - base);
-                rowsum += a + bb;
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
-                pk[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
-            }
-            // O and P belong to the previous product until it completes
-            if (j > 0) {
-                if (!mbar_wait(o_done, static_cast<uint32_t>((j - 1) & 1), kWaitLimitNs)) {
+            for (int j = 0; j < my_nk; ++j, ++ns) {
+                // S_x(j) done; it was issued after PV_x(j - 1), so O_x is free too
+                if (!mbar_wait(s_full(tile), static_cast<uint32_t>(ns & 1), kWaitLimitNs) || *abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const float alpha = (grow && m_run != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + lane_addr + 32 * cc, o);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(t_o + lane_addr + 32 * cc, o);
-                    }
-                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                // the last S product of this item has read Q_x: fetch the next item's rows
+                if (j + 1 == my_nk) {
+                    kn = tc_next_item(p, k + 1, it);
+                    if (kn >= 0) fetch_q(it);
                 }
-                l_run *= alpha;
-            }
-            l_run += rowsum;
-            m_run = m_new;
-            // P row: 64 keys = 128 bytes, chunk c at c ^ (t & 7)
+                // Two passes over S in TMEM, 64 columns at a time, so that a row
+                // never sits in registers whole (ten warps leave 168 registers
+                // a thread): the row max first, then exp2 and P.
+                const int k0 = j * kKeys;
+                const bool masked = __any_sync(0xffffffffu, k0 + kKeys - 1 > row_pos);
+                float mx8[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(smem + Geo::kP + t * 128 + ((c ^ (t & 7)) << 4)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            fence_proxy_async_smem();
+                for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll 1  // one half's 64 registers live at a time
+                for (int h = 0; h < kKeys / 64; ++h) {
+                    uint32_t sr[64];
+                    tmem_ld32_nowait(t_s + 64 * h, sr);
+                    tmem_ld32_nowait(t_s + 64 * h + 32, sr + 32);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    // causal mask by position (only tiles that reach past some row need it)
+                    if (masked) {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;  // -inf
+                    }
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+                }
+                // row max of the raw scores (scale > 0)
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                                 p.scale_log2;
+                // keep the running max unless it grows by more than 2^8
+                const bool grow = mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx != -INFINITY);
+                const float m_new = grow ? mx : m_run;
+                const float nbase = m_new == -INFINITY ? 0.f : -m_new;
+                // P_x over the first half of S_x's columns (two keys per column),
+                // 64 keys at a time; P's columns [32 h, 32 h + 32) overwrite S
+                // columns already read
+                float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1  // one half's 64 registers live at a time
+                for (int h = 0; h < kKeys / 64; ++h) {
+                    uint32_t sr[64];
+                    tmem_ld32_nowait(t_s + 64 * h, sr);
+                    tmem_ld32_nowait(t_s + 64 * h + 32, sr + 32);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    if (masked) {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const float a = ex2_approx(fmaf(__uint_as_float(sr[c]), p.scale_log2, nbase));
+                        const float bb = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), p.scale_log2, nbase));
+                        sum4[(c >> 1) & 3] += a + bb;
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
+                        pk[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
+                    }
+                    tmem_st32(t_s + 32 * h, pk);
+                }
+                const float rowsum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+                if (j > 0) {
+                    const float alpha = (grow && m_run != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
+                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t o[32];
+                            tmem_ld32(t_o + 32 * cc, o);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                            tmem_st32(t_o + 32 * cc, o);
+                        }
+                    }
+                    l_run *= alpha;
+                }
+                l_run += rowsum;
+                m_run = m_new;
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full(tile));
+            }
+            if (!ok) break;
+            // O_x of this item complete (a tile without rows gets a bare commit)
+            if (!mbar_wait(o_done(tile), static_cast<uint32_t>(n_it & 1), kWaitLimitNs) || *abort_flag) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (kn >= 0) publish_q();
+            ++n_it;
+            if (my_nk == 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(o_free(tile));
+                k = kn;
+                continue;
+            }
+            // O row, normalised, packed to bf16 and stored 64 columns at a
+            // time; then O_x is handed back
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            uint4 *dst = reinterpret_cast<uint4 *>(out_row);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) {
+                uint32_t o[64];
+                tmem_ld32_nowait(t_o + 64 * h, o);
+                tmem_ld32_nowait(t_o + 64 * h + 32, o + 32);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (row_pos >= 0) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * e]) * inv,
+                                                                      __uint_as_float(o[8 * i + 2 * e + 1]) * inv);
+                            w[e] = *reinterpret_cast<uint32_t *>(&h2);
+                        }
+                        dst[8 * h + i] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(o_free(tile));
+            k = kn;
         }
-        if (ok && nk > 0 && mbar_wait(o_done, static_cast<uint32_t>((nk - 1) & 1), kWaitLimitNs)) {
-            tc_fence_after();
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                tmem_ld32(t_o + lane_addr + 32 * cc, o);
-                if (row_pos >= 0) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
-                                                                  __uint_as_float(o[2 * i + 1]) * inv);
-                        w[i] = *reinterpret_cast<uint32_t *>(&h2);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + out_off + 32 * cc);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-                }
-            }
-        } else if (threadIdx.x == 0) {
+        if (!ok && t == 0) {
             flag(p.err, PKV_DEV_ERR_TIMEOUT);
             *abort_flag = 1;
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     // everyone (the producer's copies included) is done with TMEM and shared memory
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "n"(Geo::kTmemCols)
                      : "memory");
 }
 
 template <int D>
-cudaError_t launch_prefill_tc_d(const CUtensorMap &tmk, const CUtensorMap &tmv,
-                                const PrefillParams &p, int max_query_len, cudaStream_t stream) {
+cudaError_t launch_prefill_tc_d(const CUtensorMap &tmk, const CUtensorMap &tmv, PrefillParams p,
+                                int max_query_len, int num_sms, cudaStream_t stream) {
     constexpr int kSmem = TcGeometry<D>::kSmemBytes;
     auto kern = paged_prefill_tc_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const long long rows = static_cast<long long>(max_query_len) * p.group;
-    const long long tiles = (rows + kRows - 1) / kRows;
-    if (tiles == 0) return cudaSuccess;
-    if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.Hkv), static_cast<unsigned>(p.B));
+    const long long items = (rows + kCtaRows - 1) / kCtaRows * p.Hkv * p.B;
+    if (items == 0) return cudaSuccess;
+    if (items > 0x7FFFFFFFLL - 2LL * num_sms) return cudaErrorInvalidValue;
+    p.items = static_cast<int>(items);
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(items, num_sms));
     kern<<<grid, kThreads, kSmem, stream>>>(tmk, tmv, p);
     return cudaGetLastError();
 }
@@ -432,9 +679,9 @@ cudaError_t launch_prefill_tc_d(const CUtensorMap &tmk, const CUtensorMap &tmv,
 }  // namespace
 
 cudaError_t launch_prefill_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
-                              int head_dim, int max_query_len, cudaStream_t stream) {
-    if (head_dim == 128) return launch_prefill_tc_d<128>(tmk, tmv, p, max_query_len, stream);
-    if (head_dim == 64) return launch_prefill_tc_d<64>(tmk, tmv, p, max_query_len, stream);
+                              int head_dim, int max_query_len, int num_sms, cudaStream_t stream) {
+    if (head_dim == 128) return launch_prefill_tc_d<128>(tmk, tmv, p, max_query_len, num_sms, stream);
+    if (head_dim == 64) return launch_prefill_tc_d<64>(tmk, tmv, p, max_query_len, num_sms, stream);
     return cudaErrorInvalidValue;
 }
 

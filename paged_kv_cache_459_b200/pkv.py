@@ -37,6 +37,8 @@ DEFAULT_PARTITION_TOKENS = 512
 _P, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 _sigs = {
     "pkv_status_string": ([_i32], ctypes.c_char_p),
+    "pkv_last_cuda_error": ([], _i32),
+    "pkv_last_cuda_error_string": ([], ctypes.c_char_p),
     "pkv_block_tokens": ([], _i32),
     "pkv_version": ([], ctypes.c_char_p),
     "pkv_paged_kv_write": ([_P, _P, _P, _P, _P, _i32, _i32, _i32, _i64, _P, _P], _i32),
@@ -100,7 +102,10 @@ def status_string(code: int) -> str:
 
 class PkvError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {status_string(code)} ({code})")
+        msg = f"{what}: {status_string(code)} ({code})"
+        if code == ERR_CUDA and _lib.pkv_last_cuda_error():
+            msg += f": {_lib.pkv_last_cuda_error_string().decode()}"
+        super().__init__(msg)
         self.code = code
 
 

@@ -83,3 +83,47 @@ def test_prefill_last_row_equals_decode(prefill_impl):
     """The prompt's last token attends exactly as a decode step at that length."""
     out, ref = run_prefill(8, 8, 128, [0], [77], seed=9)
     check_close(out[-1:], ref[-1:], "last row")
+
+
+def test_prefill_many_items_ragged(prefill_impl):
+    """More work items than SMs, with sequences whose last tile is partly or
+    wholly empty and items past a short sequence's rows: each persistent CTA
+    walks many items and all phases carry across them."""
+    out, ref = run_prefill(32, 8, 128, [0, 500, 33, 0, 100, 0], [1500, 3, 700, 129, 1024, 257], seed=21)
+    check_close(out, ref, "many items, ragged")
+
+
+def test_prefill_full_size_sampled(prefill_impl):
+    """The benchmark's size and launch (4 prompts x 2048 tokens, 32/32 heads,
+    d 128), checked on a seeded sample of rows computed by the oracle one by one."""
+    hq = hkv = 32
+    d, B, n = 128, 4, 2048
+    seed = 5
+    nb = B * n // 16 + 8
+    bm = BlockManager(nb, wl.rng(seed).permutation(nb))
+    for b in range(B):
+        bm.add_seq(b, 0)
+    slots = np.concatenate([bm.extend(b, n) for b in range(B)])
+    tables, lens = bm.export(list(range(B)), n // 16)
+    kc = wl.bf16_normal((nb, hkv, 16, d), seed, 0)
+    vc = wl.bf16_normal((nb, hkv, 16, d), seed, 1)
+    T = B * n
+    k_new, v_new = wl.bf16_normal((T, hkv, d), seed, 2), wl.bf16_normal((T, hkv, d), seed, 3)
+    q = wl.bf16_normal((T, hq, d), seed, 4)
+    qs = np.arange(0, T + 1, n, dtype=np.int32)
+    scale = 1 / np.sqrt(d)
+    gk, gv = dev_bf16(kc), dev_bf16(vc)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_kv_write(dev_bf16(k_new), dev_bf16(v_new), gk, gv, torch.from_numpy(slots).cuda(), err=err)
+    out = torch.empty((T, hq, d), dtype=torch.bfloat16, device="cuda")
+    pkv.paged_attention_prefill(out, dev_bf16(q), gk, gv, torch.from_numpy(tables).cuda(),
+                                torch.from_numpy(lens).cuda(), torch.from_numpy(qs).cuda(), scale, hkv,
+                                n, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rows = np.sort(wl.rng(seed + 1).choice(T, size=192, replace=False))
+    rows = np.unique(np.concatenate([rows, [0, n - 1, n, T - 1]]))
+    rk, rv = host_bits(gk), host_bits(gv)
+    seq = rows // n
+    ref = oracle.paged_decode(q[rows], rk, rv, tables[seq], (rows % n + 1).astype(np.int32), scale)
+    check_close(host_bits(out)[rows], ref, "full-size sampled rows")
