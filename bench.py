@@ -113,14 +113,15 @@ def source_sha(path: str) -> str:
 
 def committed_traffic(kernel: str, workload: str):
     """dram read+write bytes per launch from the committed ncu summary, if it
-    was taken on the current kernel source."""
+    was taken on the current source of the kernel (the file named in the
+    record, by its sha1 prefix)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)[workload][kernel]
     except (OSError, KeyError, ValueError):
         return None
-    src = os.path.join(ROOT, "paged_kv_cache_459_b200", "csrc", "decode.cu")
-    if rec.get("decode_cu_sha") != source_sha(src):
+    src = os.path.join(ROOT, "paged_kv_cache_459_b200", "csrc", rec.get("source", ""))
+    if not os.path.isfile(src) or rec.get("source_sha") != source_sha(src):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -506,6 +507,15 @@ def run_gpu(args):
     return 0
 
 
+def measured_peak_tensor_sustained() -> float:
+    """The seconds-long cuBLAS figure (power-capped clocks), for context."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except (OSError, KeyError, ValueError):
+        return 1400.0
+
+
 def measured_peak_tensor():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -575,7 +585,11 @@ def run_row(args):
                     warp_mma_tflops=flops / (ms_warp * 1e-3) / 1e12,
                     roofline={"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                               "frac": ach / peak, "peak_kind": kind,
-                              "kernel": "paged_prefill_tc_kernel (tcgen05, TMEM accumulators)"})
+                              "frac_of_sustained": ach / measured_peak_tensor_sustained(),
+                              "kernel": "paged_prefill_tc_kernel (tcgen05, TMEM accumulators)",
+                              "traffic": committed_traffic(
+                                  "paged_prefill_tc_kernel",
+                                  "prefill_qwen_4x2048" if args.config == "qwen" else "prefill_llama_4x2048")})
     elif args.row == "cow":
         cfg = wl.config("llama")
         hkv, d, nb, n = cfg["num_kv_heads"], cfg["head_dim"], 8192, 2048

@@ -132,6 +132,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 
+// ------------------------------------------------ packed f32x2 arithmetic
+// Two floats in one 64-bit register pair for the sm_100 f32x2 instructions.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 template <int D>
 struct TcGeometry {
     static constexpr int kHalves = D / 64;
@@ -275,8 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint64_t policy = l2_policy_evict_normal();
             int gk = 0, gv = 0;  // K / V tiles loaded so far (ring position and phase)
-            TcItem it;
-            for (int k = tc_next_item(p, 0, it); k >= 0 && !*abort_flag; k = tc_next_item(p, k + 1, it)) {
+            TcItem it, nx;
+            for (int k = tc_next_item(p, 0, it); k >= 0 && !*abort_flag; it = nx) {
+                const int kn = tc_next_item(p, k + 1, nx);
                 const int32_t *trow = p.block_tables + static_cast<size_t>(it.b) * p.W;
                 const int nk = max(it.nk0, it.nk1);
                 for (int j = 0; j < nk && !*abort_flag; ++j) {
@@ -326,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &tmv, hh * 64, y[i], v_full(sv), policy);
                     ++gv;
                 }
+                k = kn;
             }
             // on an abort, copies may still be landing: wait (bounded) for the last of each stage
             for (int g = max(gk - KS, 0); g < gk; ++g)
@@ -387,19 +415,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         int gk = 0, gv = 0;      // K / V tiles consumed
         int ns[kTiles] = {0, 0};  // S products per Q tile (s_full / p_full phases)
         int n_it = 0;            // items done (q_full / o_done / o_free phases)
-        TcItem it;
-        for (int k = tc_next_item(p, 0, it); k >= 0 && ok; k = tc_next_item(p, k + 1, it), ++n_it) {
+        TcItem it, nx;
+        int k = tc_next_item(p, 0, it);
+        for (; k >= 0 && ok; it = nx, ++n_it) {
+            // the next item's parameters are read now, off the item boundary
+            const int kn = tc_next_item(p, k + 1, nx);
             const int nk_t[kTiles] = {it.nk0, it.nk1};
             const int nk = max(it.nk0, it.nk1);
-            wait(q_full(0), static_cast<uint32_t>(n_it & 1));
-            wait(q_full(1), static_cast<uint32_t>(n_it & 1));
             wait(k_full(gk % KS), static_cast<uint32_t>((gk / KS) & 1));
-            tc_fence_after();
-            if (ok && lane == 0) {
-                for (int x = 0; x < kTiles; ++x)
-                    if (nk_t[x] > 0) issue_s(x, gk % KS);
-                umma_commit(k_empty(gk % KS));
+#pragma unroll
+            for (int x = 0; x < kTiles; ++x) {
+                if (nk_t[x] == 0) continue;
+                wait(q_full(x), static_cast<uint32_t>(n_it & 1));
+                tc_fence_after();
+                if (ok && lane == 0) issue_s(x, gk % KS);
+                __syncwarp();
             }
+            if (ok && lane == 0) umma_commit(k_empty(gk % KS));
             __syncwarp();
             ++gk;
             for (int j = 0; j < nk && ok; ++j, ++gv) {
@@ -452,10 +484,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // a Q tile without rows in this item still takes its phases
             for (int x = 0; x < kTiles; ++x) {
                 if (nk_t[x] > 0) continue;
+                wait(q_full(x), static_cast<uint32_t>(n_it & 1));
                 if (n_it > 0) wait(o_free(x), static_cast<uint32_t>((n_it - 1) & 1));
                 if (ok && lane == 0) umma_commit(o_done(x));
                 __syncwarp();
             }
+            k = kn;
         }
     } else {
         // ---------------- softmax warps: thread t of tile x = TMEM lane t = row r_begin + 128 x + t
@@ -490,24 +524,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         int ns = 0;    // S products seen (s_full / p_full phases)
         int n_it = 0;  // items done (o_done phases)
-        TcItem it;     // the current item until its last S product, then the next one
+        TcItem it, nx;  // the current and the next item
         int k = tc_next_item(p, 0, it);
         if (k >= 0) {
             fetch_q(it);
             publish_q();
         }
         while (k >= 0 && ok) {
+            const int kn = tc_next_item(p, k + 1, nx);
             const int r = it.r_begin + tile * kRows + t;
             const int row_pos = r < it.rows ? it.first_pos + r / G : -1;
             const int my_nk = tile == 0 ? it.nk0 : it.nk1;
             __nv_bfloat16 *out_row =
                 p.out + (static_cast<size_t>(it.q0 + r / G) * p.Hq + it.kvh * G + r % G) * D;
             float m_run = -INFINITY, l_run = 0.f;
-            int kn = -1;
-            if (my_nk == 0) {
-                kn = tc_next_item(p, k + 1, it);
-                if (kn >= 0) fetch_q(it);
-            }
+            if (my_nk == 0 && kn >= 0) fetch_q(nx);
             for (int j = 0; j < my_nk; ++j, ++ns) {
                 // S_x(j) done; it was issued after PV_x(j - 1), so O_x is free too
                 if (!mbar_wait(s_full(tile), static_cast<uint32_t>(ns & 1), kWaitLimitNs) || *abort_flag) {
@@ -516,18 +547,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 // the last S product of this item has read Q_x: fetch the next item's rows
-                if (j + 1 == my_nk) {
-                    kn = tc_next_item(p, k + 1, it);
-                    if (kn >= 0) fetch_q(it);
-                }
+                if (j + 1 == my_nk && kn >= 0) fetch_q(nx);
                 // Two passes over S in TMEM, 64 columns at a time, so that a row
                 // never sits in registers whole (ten warps leave 168 registers
                 // a thread): the row max first, then exp2 and P.
                 const int k0 = j * kKeys;
                 const bool masked = __any_sync(0xffffffffu, k0 + kKeys - 1 > row_pos);
-                float mx8[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1  // one half's 64 registers live at a time
                 for (int h = 0; h < kKeys / 64; ++h) {
                     uint32_t sr[64];
@@ -541,12 +567,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;  // -inf
                     }
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+                    for (int c = 0; c < 64; c += 2)
+                        mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
                 }
                 // row max of the raw scores (scale > 0)
-                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
-                                 p.scale_log2;
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
                 // keep the running max unless it grows by more than 2^8
                 const bool grow = mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx != -INFINITY);
                 const float m_new = grow ? mx : m_run;
@@ -554,30 +579,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // P_x over the first half of S_x's columns (two keys per column),
                 // 64 keys at a time; P's columns [32 h, 32 h + 32) overwrite S
                 // columns already read
-                float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
+                const uint64_t nbase2 = f2pack(nbase, nbase);
+                uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
 #pragma unroll 1  // one half's 64 registers live at a time
                 for (int h = 0; h < kKeys / 64; ++h) {
                     uint32_t sr[64];
                     tmem_ld32_nowait(t_s + 64 * h, sr);
                     tmem_ld32_nowait(t_s + 64 * h + 32, sr + 32);
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                    if (masked) {
+                    uint32_t pk[32];
+                    if (masked) {  // diagonal tiles: -inf scores (2^-inf = 0)
 #pragma unroll
                         for (int c = 0; c < 64; ++c)
                             if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;
                     }
-                    uint32_t pk[32];
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        const float a = ex2_approx(fmaf(__uint_as_float(sr[c]), p.scale_log2, nbase));
-                        const float bb = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), p.scale_log2, nbase));
-                        sum4[(c >> 1) & 3] += a + bb;
+                    for (int c = 0; c < 64; c += 2) {  // scale and shift two at a time, 2^x on the SFU
+                        float a, bb;
+                        f2unpack(ffma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), scale2, nbase2), a, bb);
+                        a = ex2_approx(a);
+                        bb = ex2_approx(bb);
+                        sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], f2pack(a, bb));
                         __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
                         pk[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
                     }
                     tmem_st32(t_s + 32 * h, pk);
                 }
-                const float rowsum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+                float s_lo, s_hi, s_lo2, s_hi2;
+                f2unpack(sum2[0], s_lo, s_hi);
+                f2unpack(sum2[1], s_lo2, s_hi2);
+                const float rowsum = (s_lo + s_hi) + (s_lo2 + s_hi2);
                 if (j > 0) {
                     const float alpha = (grow && m_run != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
                     if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -598,6 +630,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full(tile));
+                // This tile's S products of the item are all done, so the tensor
+                // core has taken this item's Q phase: the next one may be posted.
+                if (j + 1 == my_nk && kn >= 0) publish_q();
             }
             if (!ok) break;
             // O_x of this item complete (a tile without rows gets a bare commit)
@@ -606,11 +641,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            if (kn >= 0) publish_q();
+            if (my_nk == 0 && kn >= 0) publish_q();  // after o_done: at most one phase ahead
             ++n_it;
             if (my_nk == 0) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(o_free(tile));
+                it = nx;
                 k = kn;
                 continue;
             }
@@ -641,6 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(o_free(tile));
+            it = nx;
             k = kn;
         }
         if (!ok && t == 0) {
