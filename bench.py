@@ -62,6 +62,9 @@ def parse_args():
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix decode: prefix blocks read once per group and KV head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 256 MB buffer between timed steps (automatic when the "
+                         "step's K/V fit in L2) and time the step from per-step events")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU time budget of the oracle baseline sample")
     return ap.parse_args()
@@ -186,6 +189,7 @@ class OracleStep:
         import oracle
         self.lib = oracle.lib()
         self.cores = oracle.threads_available()
+        self.threads = self.cores
         self.w = w
         self.kc, self.vc = w.k_cache.copy(), w.v_cache.copy()
         c = w.cfg
@@ -202,7 +206,7 @@ class OracleStep:
             self.out.ctypes.data, w.q.ctypes.data, self.kc.ctypes.data, self.vc.ctypes.data,
             self.tables.ctypes.data, self.tables.shape[1], self.lens.ctypes.data, nseq,
             c["num_heads"], c["num_kv_heads"], c["head_dim"], w.num_blocks, float(c["scale"]),
-            self.cores)
+            self.threads)
         if rc != 0:
             raise RuntimeError(f"oracle failed ({rc})")
 
@@ -219,17 +223,36 @@ class OracleStep:
         return time.perf_counter() - t0
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w, budget_s: float) -> dict:
-    """Bounded sample of the oracle on this host: about `budget_s` seconds."""
+    """Bounded sample of the oracle on this host: about `budget_s` seconds on
+    all the process's cores, then about a quarter of that on one thread."""
     st = OracleStep(w)
     per_seq = st.seconds_per_seq()
     b = w.cfg["batch"]
     nseq = int(min(b, max(1, budget_s / 3 / per_seq)))
     reps = max(1, int(budget_s / (nseq * per_seq)))
     el = st.timed(nseq, reps)
+    st.threads = 1
+    per_seq1 = st.seconds_per_seq()
+    nseq1 = int(min(b, max(1, budget_s / 4 / per_seq1)))
+    el1 = st.timed(nseq1, 1)
     return {"value": nseq * reps / el, "unit": UNIT, "cores": st.cores, "kind": "oracle",
             "sample": f"{reps} oracle steps (KV write + decode, fp64) over the first {nseq} of "
-                      f"{b} sequences, {el:.1f} s on {st.cores} threads"}
+                      f"{b} sequences, {el:.1f} s on {st.cores} threads",
+            "single_thread": {"value": nseq1 / el1, "unit": UNIT,
+                              "sample": f"1 step over the first {nseq1} sequences, {el1:.1f} s"},
+            "cpu_model": cpu_model()}
 
 
 def run_reference(args):
@@ -336,6 +359,8 @@ def run_gpu(args):
         raise SystemExit(f"device error word {int(err.item())} after warm-up")
 
     sampler = ClockSampler(device_pci_id(dev)) if rank == 0 else None
+    flush = args.flush_l2 or algorithmic_bytes(w)["kv"] <= L2_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -343,6 +368,8 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     t_start.record(stream)
     for i in range(K):
+        if flush:
+            flush_buf.zero_()  # L2 holds none of this step's inputs
         ev[i][0].record(stream)
         write()
         ev[i][1].record(stream)
@@ -353,6 +380,8 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     total_ms = t_start.elapsed_time(t_end)
+    if flush:  # the flushes are not the step's work: sum the steps' own events
+        total_ms = sum(e[0].elapsed_time(e[2]) for e in ev)
     write_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
     decode_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev)
     # keep the GPU loaded long enough for the clock sampler to see it
@@ -475,8 +504,9 @@ def run_gpu(args):
                         }[chosen] if not args.cascade else
             "shared-prefix cascade (prefix once per group x KV head, split-K suffixes, merge)",
             "logical_kv_bytes": ab["kv"],
-            "l2": f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), "
-                  "no flush" if ab["kv"] > L2_BYTES else "inputs fit in L2",
+            "l2": (f"L2 flushed between steps (256 MB write); step time from per-step events "
+                   f"(KV {ab['kv'] / 1e9:.3f} GB per step)") if flush else
+                  f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), no flush",
             "parallelism": f"{world} independent replicas (batch per GPU fixed)",
             "seed": args.seed,
         },
