@@ -127,3 +127,72 @@ def test_prefill_full_size_sampled(prefill_impl):
     seq = rows // n
     ref = oracle.paged_decode(q[rows], rk, rv, tables[seq], (rows % n + 1).astype(np.int32), scale)
     check_close(host_bits(out)[rows], ref, "full-size sampled rows")
+
+
+def test_prefill_many_items_d64(prefill_impl):
+    """d = 64 with more work items than SMs (4-query groups, ragged prompts)."""
+    out, ref = run_prefill(16, 4, 64, [0, 300, 0], [900, 17, 513], seed=31)
+    check_close(out, ref, "many items, d 64")
+
+
+def test_prefill_empty_prompts_in_batch(prefill_impl):
+    """Sequences with no new tokens in the batch produce no rows and disturb
+    nothing around them."""
+    out, ref = run_prefill(8, 2, 128, [5, 0, 0, 20], [0, 37, 0, 130], seed=41)
+    assert out.shape[0] == 167
+    check_close(out, ref, "empty prompts in the batch")
+
+
+def _prefill_case(hq, hkv, d, new, seed):
+    B = len(new)
+    nb = sum(-(-n // 16) for n in new) + 8
+    bm = BlockManager(nb, wl.rng(seed).permutation(nb))
+    for b in range(B):
+        bm.add_seq(b, 0)
+    slots = np.concatenate([bm.extend(b, new[b]) for b in range(B)])
+    tables, lens = bm.export(list(range(B)), max(-(-n // 16) for n in new))
+    kc = wl.bf16_normal((nb, hkv, 16, d), seed, 0)
+    vc = wl.bf16_normal((nb, hkv, 16, d), seed, 1)
+    T = sum(new)
+    k_new, v_new = wl.bf16_normal((T, hkv, d), seed, 2), wl.bf16_normal((T, hkv, d), seed, 3)
+    q = wl.bf16_normal((T, hq, d), seed, 4)
+    qs = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    rk, rv = oracle.kv_write(kc, vc, k_new, v_new, slots)
+    return q, rk, rv, tables, lens, qs
+
+
+def _run_gpu_prefill(q, rk, rv, tables, lens, qs, hkv, max_q):
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros(q.shape, dtype=torch.bfloat16, device="cuda")
+    pkv.paged_attention_prefill(out, dev_bf16(q), dev_bf16(rk), dev_bf16(rv), torch.from_numpy(tables).cuda(),
+                                torch.from_numpy(lens).cuda(), torch.from_numpy(qs).cuda(),
+                                1 / np.sqrt(q.shape[2]), hkv, max_q, err=err)
+    torch.cuda.synchronize()
+    return host_bits(out), int(err.item())
+
+
+def test_prefill_inconsistent_length_is_flagged_and_skipped(prefill_impl):
+    """A sequence whose context is shorter than its new tokens is skipped with
+    the bad-length bit; the other sequences are unaffected."""
+    new = [70, 90, 33]
+    q, rk, rv, tables, lens, qs = _prefill_case(8, 8, 128, new, seed=51)
+    ref = oracle.paged_prefill(q, rk, rv, tables, lens, qs, 1 / np.sqrt(128))
+    bad = lens.copy()
+    bad[1] = new[1] - 1
+    out, err = _run_gpu_prefill(q, rk, rv, tables, bad, qs, 8, max(new))
+    assert err & 4, err  # PKV_DEV_ERR_BAD_LEN
+    keep = np.r_[qs[0]:qs[1], qs[2]:qs[3]]
+    check_close(out[keep], ref[keep], "sequences next to a bad length")
+
+
+def test_prefill_bad_table_entry_is_flagged(prefill_impl):
+    """A table entry outside the pool is flagged (bad-block bit) and read as
+    zeros; sequences that do not use it are unaffected."""
+    new = [40, 100]
+    q, rk, rv, tables, lens, qs = _prefill_case(8, 8, 64, new, seed=61)
+    ref = oracle.paged_prefill(q, rk, rv, tables, lens, qs, 1 / np.sqrt(64))
+    t = tables.copy()
+    t[1, 2] = rk.shape[0] + 5
+    out, err = _run_gpu_prefill(q, rk, rv, t, lens, qs, 8, max(new))
+    assert err & 2, err  # PKV_DEV_ERR_BAD_BLOCK
+    check_close(out[qs[0]:qs[1]], ref[qs[0]:qs[1]], "sequence next to a bad table entry")
