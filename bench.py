@@ -333,6 +333,7 @@ def run_gpu(args):
     if args.cascade:
         pb_h, offs_h, mem_h = w.alloc.prefix_groups(list(range(B)))
         pb, offs_g, mem = (torch.from_numpy(x).to(dev) for x in (pb_h, offs_h, mem_h))
+        suffix_bound = pkv.suffix_blocks_bound(w.lens, pb_h)  # the allocator's host view
         ws = torch.empty(pkv.decode_prefix_workspace_bytes(B, hq, d, W, args.partition),
                          dtype=torch.uint8, device=dev)
     scale = cfg["scale"]
@@ -343,6 +344,7 @@ def run_gpu(args):
     def decode():
         if args.cascade:
             pkv.paged_attention_decode_prefix(out, q, kc, vc, tables, lens, scale, hkv, pb, offs_g, mem,
+                                              max_suffix_blocks=suffix_bound,
                                               partition_tokens=args.partition, workspace=ws,
                                               err=err)
         else:
@@ -431,8 +433,9 @@ def run_gpu(args):
         pkv.paged_kv_write(c["k"], c["v"], kc, vc, c["slots"], err=err)
         if args.cascade:
             pkv.paged_attention_decode_prefix(o, c["q"], kc, vc, c["tables"], c["lens"], scale, hkv,
-                                              pb, offs_g, mem, partition_tokens=args.partition,
-                                              workspace=ws, err=err)
+                                              pb, offs_g, mem, max_suffix_blocks=suffix_bound,
+                                              partition_tokens=args.partition, workspace=ws,
+                                              err=err)
         else:
             pkv.paged_attention_decode(o, c["q"], kc, vc, c["tables"], c["lens"], scale, hkv,
                                        variant=variant, partition_tokens=args.partition,

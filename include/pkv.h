@@ -233,6 +233,12 @@ PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, c
  * split-K kernel (partition_tokens, <= 0: 512) covers each sequence past its
  * prefix; a merge kernel combines the partials.  Workspace:
  * pkv_decode_prefix_workspace_bytes(...), else PKV_ERR_WORKSPACE.
+ * max_suffix_blocks: an upper bound on ceil(len / 16) - prefix_blocks over the
+ * batch (the blocks past each sequence's prefix), or <= 0 for "unknown"
+ * (max_blocks_per_seq is used).  It sizes the suffix grid, so a tight bound
+ * launches no empty partitions; a suffix longer than the bound is left
+ * incomplete and flagged PKV_DEV_ERR_BAD_LEN (the bound is the caller's
+ * promise, as the lengths are).
  */
 PKV_API size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                                  int max_blocks_per_seq, int partition_tokens);
@@ -241,8 +247,8 @@ PKV_API pkv_status pkv_paged_attention_decode_prefix(
     const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
     int num_heads, int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
     const int32_t *prefix_blocks, const int32_t *group_offsets, const int32_t *group_seqs,
-    int num_groups, int partition_tokens, void *workspace, size_t workspace_bytes,
-    unsigned int *err_word, void *stream);
+    int num_groups, int max_suffix_blocks, int partition_tokens, void *workspace,
+    size_t workspace_bytes, unsigned int *err_word, void *stream);
 
 /*
  * Block copy for copy-on-write (a sequence that shares a partly filled block,

@@ -24,6 +24,7 @@ namespace {
 using namespace dev;
 
 constexpr int kPrefixWarps = 4;
+constexpr float kLazyRescale = 8.0f;  // log2 units: the running max moves past this growth only
 
 template <int D, int CB>
 struct PrefixGeometry {
@@ -137,66 +138,97 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap &tmk, const CUtens
             for (int i = 0; i < 4; ++i) o[n][i] = 0.f;
         float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
-        for (int t = 0; t < nt; ++t) {
-            if (valid[t] < 0) continue;
-            const uint32_t kt = smem_u32(ktiles + t * kTile), vt = smem_u32(vtiles + t * kTile);
-            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};  // tokens 0-7, 8-15
+        // Two blocks (32 tokens) per step: S for both, one row-max update,
+        // one (rare) rescale, then P.V for each block.  The running max only
+        // moves when a row's max grows by more than 2^8, so O is rescaled
+        // seldom and P stays <= 2^8; the partial's m is that base.
+        for (int t0 = 0; t0 < nt; t0 += 2) {
+            const bool v0 = valid[t0] >= 0, v1 = t0 + 1 < nt && valid[t0 + 1] >= 0;
+            float s[4][4];  // 8-token column tiles: block t0 tokens 0-7, 8-15, block t0+1 0-7, 8-15
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[n][i] = 0.f;
             {
                 const int tok = (lane & 7) + (lane >> 4) * 8;
                 const int cb = (lane >> 3) & 1;
 #pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    uint32_t b00, b01, b10, b11;
-                    ldmatrix_x4(kt + tile_off(tok, 2 * ks + cb), b00, b01, b10, b11);
-                    mma_bf16_16816(s0, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
-                    mma_bf16_16816(s1, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
+                for (int half = 0; half < 2; ++half) {
+                    if (!(half ? v1 : v0)) continue;
+                    const uint32_t kt = smem_u32(ktiles + (t0 + half) * kTile);
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        uint32_t b00, b01, b10, b11;
+                        ldmatrix_x4(kt + tile_off(tok, 2 * ks + cb), b00, b01, b10, b11);
+                        mma_bf16_16816(s[2 * half], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
+                        mma_bf16_16816(s[2 * half + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
+                    }
                 }
             }
+            // scores in the exp2 domain; a block that is not there scores -inf
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                s0[i] *= p.scale_log2;
-                s1[i] *= p.scale_log2;
+            for (int n = 0; n < 4; ++n) {
+                const bool there = n < 2 ? v0 : v1;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[n][i] = there ? s[n][i] * p.scale_log2 : -INFINITY;
             }
-            // row gid: s0[0], s0[1], s1[0], s1[1]; row gid + 8: s0[2], s0[3], s1[2], s1[3]
-            float mx0 = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
-            float mx1 = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
+            // row gid: s[n][0], s[n][1]; row gid + 8: s[n][2], s[n][3]
+            float mx0 = fmaxf(fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1])),
+                              fmaxf(fmaxf(s[2][0], s[2][1]), fmaxf(s[3][0], s[3][1])));
+            float mx1 = fmaxf(fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3])),
+                              fmaxf(fmaxf(s[2][2], s[2][3]), fmaxf(s[3][2], s[3][3])));
 #pragma unroll
             for (int m = 1; m < 4; m <<= 1) {
                 mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, m));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, m));
             }
-            const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-            const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
-            m_run[0] = mn0;
-            m_run[1] = mn1;
-            float pr0[4], pr1[4];
-            pr0[0] = exp2f(s0[0] - mn0);
-            pr0[1] = exp2f(s0[1] - mn0);
-            pr1[0] = exp2f(s1[0] - mn0);
-            pr1[1] = exp2f(s1[1] - mn0);
-            pr0[2] = exp2f(s0[2] - mn1);
-            pr0[3] = exp2f(s0[3] - mn1);
-            pr1[2] = exp2f(s1[2] - mn1);
-            pr1[3] = exp2f(s1[3] - mn1);
-            l_run[0] = l_run[0] * al0 + pr0[0] + pr0[1] + pr1[0] + pr1[1];
-            l_run[1] = l_run[1] * al1 + pr0[2] + pr0[3] + pr1[2] + pr1[3];
+            const bool g0 = mx0 > m_run[0] + kLazyRescale || (m_run[0] == -INFINITY && mx0 != -INFINITY);
+            const bool g1 = mx1 > m_run[1] + kLazyRescale || (m_run[1] == -INFINITY && mx1 != -INFINITY);
+            const float al0 = g0 && m_run[0] != -INFINITY ? ex2_approx(m_run[0] - mx0) : 1.f;
+            const float al1 = g1 && m_run[1] != -INFINITY ? ex2_approx(m_run[1] - mx1) : 1.f;
+            if (g0) m_run[0] = mx0;
+            if (g1) m_run[1] = mx1;
+            if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                o[n][0] *= al0;
-                o[n][1] *= al0;
-                o[n][2] *= al1;
-                o[n][3] *= al1;
+                for (int n = 0; n < NT; ++n) {
+                    o[n][0] *= al0;
+                    o[n][1] *= al0;
+                    o[n][2] *= al1;
+                    o[n][3] *= al1;
+                }
             }
-            const uint32_t pa0 = pack_bf16x2(pr0[0], pr0[1]), pa1 = pack_bf16x2(pr0[2], pr0[3]);
-            const uint32_t pa2 = pack_bf16x2(pr1[0], pr1[1]), pa3 = pack_bf16x2(pr1[2], pr1[3]);
+            const float nb0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
+            const float nb1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
+            float pr[4][4];
+            float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                pr[n][0] = ex2_approx(s[n][0] - nb0);
+                pr[n][1] = ex2_approx(s[n][1] - nb0);
+                pr[n][2] = ex2_approx(s[n][2] - nb1);
+                pr[n][3] = ex2_approx(s[n][3] - nb1);
+                sum0 += pr[n][0] + pr[n][1];
+                sum1 += pr[n][2] + pr[n][3];
+            }
+            l_run[0] = l_run[0] * al0 + sum0;
+            l_run[1] = l_run[1] * al1 + sum1;
             const int tok = (lane & 7) + ((lane >> 3) & 1) * 8;
             const int cb = lane >> 4;
 #pragma unroll
-            for (int i = 0; i < NT / 2; ++i) {
-                uint32_t v0, v1, v2, v3;
-                ldmatrix_x4_trans(vt + tile_off(tok, 2 * i + cb), v0, v1, v2, v3);
-                mma_bf16_16816(o[2 * i], pa0, pa1, pa2, pa3, v0, v1);
-                mma_bf16_16816(o[2 * i + 1], pa0, pa1, pa2, pa3, v2, v3);
+            for (int half = 0; half < 2; ++half) {
+                if (!(half ? v1 : v0)) continue;
+                const uint32_t vt = smem_u32(vtiles + (t0 + half) * kTile);
+                const uint32_t pa0 = pack_bf16x2(pr[2 * half][0], pr[2 * half][1]);
+                const uint32_t pa1 = pack_bf16x2(pr[2 * half][2], pr[2 * half][3]);
+                const uint32_t pa2 = pack_bf16x2(pr[2 * half + 1][0], pr[2 * half + 1][1]);
+                const uint32_t pa3 = pack_bf16x2(pr[2 * half + 1][2], pr[2 * half + 1][3]);
+#pragma unroll
+                for (int i = 0; i < NT / 2; ++i) {
+                    uint32_t w0, w1, w2, w3;
+                    ldmatrix_x4_trans(vt + tile_off(tok, 2 * i + cb), w0, w1, w2, w3);
+                    mma_bf16_16816(o[2 * i], pa0, pa1, pa2, pa3, w0, w1);
+                    mma_bf16_16816(o[2 * i + 1], pa0, pa1, pa2, pa3, w2, w3);
+                }
             }
         }
 #pragma unroll
@@ -237,7 +269,10 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
     const int pb = min(max(__ldg(p.prefix_blocks + b), 0), len / kBlockTokens);
     const int nchunks = (pb + CB - 1) / CB;
-    const int ntot = nchunks + (nblk - pb + p.part_blocks - 1) / p.part_blocks;
+    // suffix partitions with tokens, at most those the launch computed (a
+    // longer suffix was flagged by the cascade kernel)
+    const int ntot = nchunks + min((nblk - pb + p.part_blocks - 1) / p.part_blocks,
+                                   p.ws_parts - p.prefix_parts);
     const auto slot = [&](int q) { return q < nchunks ? q : p.prefix_parts + (q - nchunks); };
     const size_t row = static_cast<size_t>(b) * p.Hq + h;
     const float *ml = p.ws_ml + 2 * row * p.ws_parts;
@@ -281,28 +316,40 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
     p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
 }
 
-// One launch for the prefix chunks and the suffix split-K units: CTAs
-// [0, n_pre) take prefix chunks (chunk fastest, then KV head, then group), the
-// rest take suffix units (partition fastest, then head segment, then
-// sequence).  The prefix work is short and latency-bound; running it beside
-// the bandwidth-bound suffix stream hides it.
+// One launch for the prefix chunks and the suffix split-K units.  Prefix
+// chunk k (chunk fastest, then KV head, then group) is CTA k * stride, spread
+// evenly through the grid, so that every SM runs the short, latency-bound
+// prefix work beside the bandwidth-bound suffix stream; the other CTAs take
+// suffix units in order (partition fastest, then head segment, then
+// sequence).
 template <int D, bool MMA>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const PrefixParams pp, const DecodeParams dp, int n_pre) {
     pdl_launch_dependents();
     int id = blockIdx.x;
-    if (id < n_pre) {
+    const int stride = n_pre > 0 ? static_cast<int>(gridDim.x) / n_pre : 1;
+    if (n_pre > 0 && id % stride == 0 && id / stride < n_pre) {
+        id /= stride;
         const int c = id % pp.prefix_parts;
         id /= pp.prefix_parts;
         prefix_unit<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
         return;
     }
-    id -= n_pre;
+    if (n_pre > 0) id -= min(id / stride + 1, n_pre);  // prefix CTAs at or before this one
     const int ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
     const int part = id % dp.num_parts;
     id /= dp.num_parts;
-    decode_unit<D, kPrefixWarps, 2, MMA, true>(tmk, tmv, dp, part, id % ny, id / ny);
+    const int b = id / ny;
+    if (part == dp.num_parts - 1 && id % ny == 0 && threadIdx.x == 0 && b < dp.B) {
+        // the caller's bound on suffix blocks must cover every suffix
+        int len = __ldg(dp.seq_lens + b);
+        len = len < 0 ? 0 : min(len, dp.W * kBlockTokens);
+        const int start = min(max(__ldg(dp.start_blocks + b), 0), len / kBlockTokens);
+        if (start + dp.num_parts * dp.part_blocks < (len + kBlockTokens - 1) / kBlockTokens)
+            flag(dp.err, PKV_DEV_ERR_BAD_LEN);
+    }
+    decode_unit<D, kPrefixWarps, 2, MMA, true>(tmk, tmv, dp, part, id % ny, b);
 }
 
 template <int D, bool MMA>

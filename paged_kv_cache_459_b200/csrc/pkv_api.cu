@@ -376,9 +376,9 @@ pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const voi
                                              const int32_t *prefix_blocks,
                                              const int32_t *group_offsets,
                                              const int32_t *group_seqs, int num_groups,
-                                             int partition_tokens, void *workspace,
-                                             size_t workspace_bytes, unsigned int *err_word,
-                                             void *stream) {
+                                             int max_suffix_blocks, int partition_tokens,
+                                             void *workspace, size_t workspace_bytes,
+                                             unsigned int *err_word, void *stream) {
     if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_kv_heads <= 0 ||
         num_heads % num_kv_heads || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
         !std::isfinite(scale) || num_groups < 0 || num_groups > 65535)
@@ -405,7 +405,12 @@ pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const voi
         !encode_cache_map(&tmv, v_cache, rows, head_dim))
         return PKV_ERR_CUDA;
 
-    const int suffix_parts = num_parts_for(max_blocks_per_seq, partition_tokens);
+    // suffix partitions the grid covers: from the caller's bound on the blocks
+    // past each prefix (no empty partitions), else from the table width
+    const int suffix_blocks = max_suffix_blocks > 0 && max_suffix_blocks < max_blocks_per_seq
+                                  ? max_suffix_blocks
+                                  : max_blocks_per_seq;
+    const int suffix_parts = num_parts_for(suffix_blocks, partition_tokens);
     const int prefix_parts = (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
     const size_t ws_rows = static_cast<size_t>(num_seqs) * num_heads * (prefix_parts + suffix_parts);
     float *ws_o = static_cast<float *>(workspace);

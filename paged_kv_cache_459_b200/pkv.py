@@ -75,7 +75,8 @@ _sigs = {
     "pkv_alloc_prefix_groups": ([_P, _P, _i32, _P, _P, _P, _P], _i32),
     "pkv_decode_prefix_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
     "pkv_paged_attention_decode_prefix": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
-                                           _i64, _f32, _P, _P, _P, _i32, _i32, _P, _sz, _P, _P],
+                                           _i64, _f32, _P, _P, _P, _i32, _i32, _i32, _P, _sz, _P,
+                                           _P],
                                           _i32),
     "pkv_alloc_seq_len": ([_P, _i64, _P], _i32),
     "pkv_alloc_slot_of": ([_P, _i64, _i64, _P], _i32),
@@ -293,10 +294,13 @@ def decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_
 
 def paged_attention_decode_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
                                   num_kv_heads, prefix_blocks, group_offsets, group_seqs, *,
+                                  max_suffix_blocks: int = 0,
                                   partition_tokens: int = DEFAULT_PARTITION_TOKENS,
                                   workspace=None, err=None) -> None:
     """Decode with shared prefixes read once per group (see include/pkv.h).
-    prefix_blocks [B], group_offsets [G + 1], group_seqs [members]: int32 CUDA."""
+    prefix_blocks [B], group_offsets [G + 1], group_seqs [members]: int32 CUDA.
+    max_suffix_blocks: bound on the blocks past each prefix (0: unknown);
+    suffix_blocks_bound() computes it from host arrays."""
     import torch
 
     bf = torch.bfloat16
@@ -321,8 +325,19 @@ def paged_attention_decode_prefix(out, q, k_cache, v_cache, block_tables, seq_le
     wp = _dev_tensor(workspace, torch.uint8, "workspace")
     _check(_lib.pkv_paged_attention_decode_prefix(
         ptrs[0], ptrs[1], ptrs[2], ptrs[3], tp, W, lp, B, hq, num_kv_heads, d, k_cache.shape[0],
-        float(scale), pp, op, gp, G, partition_tokens, wp, workspace.numel(), ep,
+        float(scale), pp, op, gp, G, int(max_suffix_blocks), partition_tokens, wp,
+        workspace.numel(), ep,
         _stream_ptr(q.device)), "pkv_paged_attention_decode_prefix")
+
+
+def suffix_blocks_bound(seq_lens, prefix_blocks) -> int:
+    """max over the batch of ceil(len / 16) - prefix_blocks (host arrays): the
+    max_suffix_blocks argument of paged_attention_decode_prefix."""
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    pb = np.asarray(prefix_blocks, dtype=np.int64)
+    if lens.size == 0:
+        return 0
+    return int(max(1, (-(-lens // BLOCK_TOKENS) - pb).max()))
 
 
 # ---------------------------------------------------------------- allocator

@@ -16,13 +16,17 @@ from paged_kv_cache_459_b200 import pkv  # noqa: E402
 from paged_kv_cache_459_b200 import workloads as wl  # noqa: E402
 
 
-def cascade(d: DeviceStep, part=512, tables=None):
+def cascade(d: DeviceStep, part=512, tables=None, bound=0):
+    """bound: max_suffix_blocks (0: unknown, "exact": from the host lengths)."""
     w = d.w
     pb, offs, members = w.alloc.prefix_groups(list(range(w.cfg["batch"])))
+    if bound == "exact":
+        bound = pkv.suffix_blocks_bound(w.lens, pb)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).cuda()  # noqa: E731
     pkv.paged_attention_decode_prefix(d.out, d.q, d.kc, d.vc, d.tables if tables is None else tables,
                                       d.lens, w.cfg["scale"], w.cfg["num_kv_heads"], dev(pb),
-                                      dev(offs), dev(members), partition_tokens=part, err=d.err)
+                                      dev(offs), dev(members), max_suffix_blocks=bound,
+                                      partition_tokens=part, err=d.err)
     torch.cuda.synchronize()
     return host_bits(d.out), pb, offs
 
@@ -47,10 +51,21 @@ def test_cascade_matches_oracle(name, kw):
     d.write()
     kc, vc, ref = oracle_after_write(w)
     for part in (512, 64):
-        out, pb, offs = cascade(d, part)
-        assert len(offs) - 1 == kw.get("prefix_groups", 1) and pb.max() > 0
-        check_close(out, ref, f"cascade {kw} partition {part}")
+        for bound in (0, "exact"):
+            out, pb, offs = cascade(d, part, bound=bound)
+            assert len(offs) - 1 == kw.get("prefix_groups", 1) and pb.max() > 0
+            check_close(out, ref, f"cascade {kw} partition {part} suffix bound {bound}")
     assert d.err_word() == 0
+
+
+def test_cascade_suffix_bound_too_small_is_flagged():
+    """A max_suffix_blocks below a real suffix leaves it incomplete and sets the
+    bad-length bit (no out-of-range workspace use)."""
+    w = build("prefix", 13, **CASES[1][1])
+    d = DeviceStep(w)
+    d.write()
+    cascade(d, 64, bound=1)   # 4-block partitions: one covers 4 of up to 13 suffix blocks
+    assert d.err_word() & 4
 
 
 def test_cascade_full_size_sampled():
@@ -58,7 +73,7 @@ def test_cascade_full_size_sampled():
     d = DeviceStep(w)
     d.write()
     kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
-    out, pb, offs = cascade(d)
+    out, pb, offs = cascade(d, bound="exact")
     assert (pb == 125).all() and len(offs) == 2
     sel = np.array([0, 5, 64, 127])
     ref = oracle.paged_decode(w.q[sel], kc, vc, w.block_tables[sel], w.lens[sel], w.cfg["scale"])
