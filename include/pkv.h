@@ -294,9 +294,13 @@ PKV_API pkv_status pkv_swap_blocks(void *k_cache, void *v_cache, void *host_k, v
  * cached prefix, earlier chunks -- are read from the cache), and the token at
  * position p attends to positions [0, p].  The K/V of the new tokens must be
  * in the cache already.  max_query_len >= every sequence's row count.
- * Tensor cores (mma.m16n8k16, bf16 -> fp32); TMA-fed shared K/V ring.
+ * 5th-generation tensor cores (tcgen05.mma, bf16 -> fp32 in tensor memory),
+ * a persistent grid of one CTA per SM over 256-row work items, TMA-fed K and
+ * V rings.  The environment variable PKV_PREFILL_WARP_MMA=1 selects the
+ * warp-level mma.m16n8k16 kernel instead (same result; kept for comparison).
  * A sequence with seq_lens[b] < its rows or past its table is skipped
- * (rows not written) and flagged PKV_DEV_ERR_BAD_LEN.
+ * (rows not written) and flagged PKV_DEV_ERR_BAD_LEN; a table entry outside
+ * the pool is read as zeros and flagged PKV_DEV_ERR_BAD_BLOCK.
  */
 PKV_API pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_cache,
                                                const void *v_cache, const int32_t *block_tables,

@@ -2,10 +2,10 @@
 //
 // Same result as paged_prefill_kernel (prefill.cu): causal attention of each
 // sequence's new tokens over its paged K/V ("vLLM 與 PagedAttention：高吞吐推理
-// 的關鍵", section 三 step 二).  A CTA owns two Q tiles of 128 query rows each
-// -- (token, query head of one KV head) pairs -- and walks the keys its rows
-// can see in tiles of 128 (eight 16-token blocks); both Q tiles share each
-// K/V tile.  Per Q tile x:
+// 的關鍵", section 三 step 二).  A persistent CTA (one per SM) walks work
+// items; an item is two Q tiles of 128 query rows each -- (token, query head
+// of one KV head) pairs of one sequence -- whose keys are walked in tiles of
+// 128 (eight 16-token blocks); both Q tiles share each K/V tile.  Per Q tile x:
 //   S_x[128 x 128] = Q_x[128 x d] K_tile^T   tcgen05.mma (A, B in shared memory)
 //   P_x = exp2(S_x - m), bf16, written back into TMEM over S_x
 //   O_x[128 x d]  += P_x V_tile              tcgen05.mma (A in TMEM, B in shared memory)
