@@ -472,6 +472,10 @@ def run_gpu(args):
     e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1])
     if int(err.item()) != 0:
         raise SystemExit(f"device error word {int(err.item())} after the timed steps")
+    # the end-to-end steps ran the same inputs through staged copies: the
+    # kernels are deterministic, so the output read back must match bit for bit
+    if K > 0 and not torch.equal(outs_h[(K - 1) % 2].view(torch.int16), out.cpu().view(torch.int16)):
+        raise SystemExit("end-to-end output differs from the device-timed output")
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
 
