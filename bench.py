@@ -62,6 +62,9 @@ def parse_args():
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix decode: prefix blocks read once per group and KV head")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the step as separate write and decode calls (the default step "
+                         "is pkv_paged_decode_step, the write fused into the decode kernel)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 256 MB buffer between timed steps (automatic when the "
                          "step's K/V fit in L2) and time the step from per-step events")
@@ -109,9 +112,12 @@ def job_throughput(units_per_rank: int, steps: int, world: int, job_ms: float) -
     return units_per_rank * steps * world / (job_ms * 1e-3)
 
 
-def source_sha(path: str) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()[:12]
+def source_sha(*paths: str) -> str:
+    h = hashlib.sha1()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
 
 
 def committed_traffic(kernel: str, workload: str):
@@ -123,8 +129,11 @@ def committed_traffic(kernel: str, workload: str):
             rec = json.load(f)[workload][kernel]
     except (OSError, KeyError, ValueError):
         return None
-    src = os.path.join(ROOT, "paged_kv_cache_459_b200", "csrc", rec.get("source", ""))
-    if not os.path.isfile(src) or rec.get("source_sha") != source_sha(src):
+    names = rec.get("source", [])
+    paths = [os.path.join(ROOT, "paged_kv_cache_459_b200", "csrc", n)
+             for n in ([names] if isinstance(names, str) else names)]
+    if not paths or not all(os.path.isfile(x) for x in paths) or \
+            rec.get("source_sha") != source_sha(*paths):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -351,11 +360,30 @@ def run_gpu(args):
             pkv.paged_attention_decode(out, q, kc, vc, tables, lens, scale, hkv, variant=variant,
                                        partition_tokens=args.partition, workspace=ws, err=err)
 
+    # The step: the new token's K/V write fused into the decode kernel
+    # (pkv_paged_decode_step), or the write and the decode as two calls.
+    fused = not args.cascade and not args.unfused and chosen != pkv.DECODE_STREAM
+
+    def fused_step(o=None, c=None):
+        c = c or {"q": q, "k": k_new, "v": v_new, "tables": tables, "lens": lens}
+        pkv.paged_decode_step(out if o is None else o, c["q"], c["k"], c["v"], kc, vc, c["tables"],
+                              c["lens"], scale, hkv, variant=variant,
+                              partition_tokens=args.partition, workspace=ws, err=err)
+
+    def step():
+        if fused:
+            fused_step()
+        else:
+            write()
+            decode()
+
     stream = torch.cuda.current_stream(dev)
     K, Wm = args.steps, args.warmup
     for _ in range(Wm):
-        write()
-        decode()
+        step()
+        if fused:
+            write()
+            decode()
     torch.cuda.synchronize(dev)
     if int(err.item()) != 0:
         raise SystemExit(f"device error word {int(err.item())} after warm-up")
@@ -373,9 +401,12 @@ def run_gpu(args):
         if flush:
             flush_buf.zero_()  # L2 holds none of this step's inputs
         ev[i][0].record(stream)
-        write()
-        ev[i][1].record(stream)
-        decode()
+        if fused:
+            fused_step()
+        else:
+            write()
+            ev[i][1].record(stream)
+            decode()
         ev[i][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -384,15 +415,35 @@ def run_gpu(args):
     total_ms = t_start.elapsed_time(t_end)
     if flush:  # the flushes are not the step's work: sum the steps' own events
         total_ms = sum(e[0].elapsed_time(e[2]) for e in ev)
-    write_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
-    decode_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev)
+    if fused:  # one call: the decode kernel's time includes the write
+        write_ms = None
+        decode_ms = statistics.fmean(e[0].elapsed_time(e[2]) for e in ev)
+    else:
+        write_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
+        decode_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev)
+    unfused = None
+    if fused:  # the same step as two calls, for comparison
+        uev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            if flush:
+                flush_buf.zero_()
+            uev[i][0].record(stream)
+            write()
+            uev[i][1].record(stream)
+            decode()
+            uev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        u_total = sum(e[0].elapsed_time(e[2]) for e in uev)
+        unfused = {"write_us": 1e3 * statistics.fmean(e[0].elapsed_time(e[1]) for e in uev),
+                   "decode_us": 1e3 * statistics.fmean(e[1].elapsed_time(e[2]) for e in uev),
+                   "value": job_throughput(B, K, 1, u_total)}
     # keep the GPU loaded long enough for the clock sampler to see it
     if sampler is not None:
         t0 = time.perf_counter()
         while time.perf_counter() - t0 < 1.0:
             for _ in range(50):
-                write()
-                decode()
+                step()
             torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler is not None else None
 
@@ -400,8 +451,9 @@ def run_gpu(args):
     # slots) go host -> device from one pinned staging buffer, and its output comes back.
     # Two device input/output sets and a copy stream let step i+1's upload and step i's
     # download overlap step i's kernels.
-    parts = [("q", q_h), ("k", k_h), ("v", v_h), ("tables", tables_h), ("lens", lens_h),
-             ("slots", slots_h)]
+    parts = [("q", q_h), ("k", k_h), ("v", v_h), ("tables", tables_h), ("lens", lens_h)]
+    if not fused:  # the fused step takes each token's slot from its table
+        parts.append(("slots", slots_h))
     offs, total = {}, 0
     for name, t in parts:
         offs[name] = total
@@ -430,6 +482,9 @@ def run_gpu(args):
     def step_on(i):
         c = sets[i % 2]
         o = outs[i % 2]
+        if fused:
+            fused_step(o, c)
+            return
         pkv.paged_kv_write(c["k"], c["v"], kc, vc, c["slots"], err=err)
         if args.cascade:
             pkv.paged_attention_decode_prefix(o, c["q"], kc, vc, c["tables"], c["lens"], scale, hkv,
@@ -504,12 +559,15 @@ def run_gpu(args):
         unique_tokens = int((np.asarray(w.lens, np.int64) - 16 * pb_h.astype(np.int64)).sum())
         unique_tokens += sum(16 * int(pb_h[mem_h[offs_h[g]]]) for g in range(len(offs_h) - 1))
         dec_bytes = unique_tokens * hkv * d * 2 * 2 + ab["q"]
+    if fused:  # the new tokens' K/V: read once, written once
+        dec_bytes += 2 * B * hkv * d * 2 * 2
     achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
     value = job_throughput(B, K, world, total_ms)
     e2e_value = job_throughput(B, K, world, e2e_ms)
     # write + decode, + the merge (split-K, balanced) or the longest-first order (single pass)
     ordered = chosen == pkv.DECODE_SINGLE and ws.numel() >= 4 * B
-    launches_per_step = 2 + (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) or ordered else 0)
+    launches_per_step = (1 if fused else 2) + \
+        (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) or ordered else 0)
     if args.cascade:
         launches_per_step = 1 + 3  # write; prefix chunks, suffix split-K, merge
     line = {
@@ -537,9 +595,16 @@ def run_gpu(args):
         "kv_hbm_gbs": achieved,
         "kv_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
         "kv_frac_of_measured_copy": achieved / peak,
-        "write_us": write_ms * 1e3, "decode_us": decode_ms * 1e3,
+        "write_us": write_ms * 1e3 if write_ms is not None else None,
+        "decode_us": decode_ms * 1e3,
+        "step": "pkv_paged_decode_step: the write fused into the decode kernel" if fused else
+                "pkv_paged_kv_write, then the decode call",
+        "unfused": unfused,
         "roofline": {
-            "bound": "hbm", "kernel": "paged_attention_decode (decode kernel + merge kernel)",
+            "bound": "hbm",
+            "kernel": ("paged_decode_kernel with the fused write" if fused else "paged_decode_kernel")
+                      + (" + merge kernel" if chosen == pkv.DECODE_SPLIT else
+                         " + order kernel" if ordered else ""),
             "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "peak_kind": peak_kind,
             "traffic": committed_traffic("paged_decode_kernel", args.config),
@@ -552,7 +617,7 @@ def run_gpu(args):
                        "copy stream so transfers overlap the kernels"},
         "e2e_graph": {"value": job_throughput(B, K, world, e2e_graph_ms), "unit": UNIT,
                       "ms_per_step": e2e_graph_ms / K,
-                      "how": "the same loop, each step's write + decode replayed from a CUDA graph"},
+                      "how": "the same loop, each step replayed from a CUDA graph"},
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -182,6 +182,32 @@ PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const
                                          void *stream);
 
 /*
+ * One decode step with the cache write fused in: the same result as
+ * pkv_paged_kv_write of k_new / v_new at each sequence's new-token slot
+ * followed by pkv_paged_attention_decode_ex ("vLLM 與 PagedAttention：高吞吐推
+ * 理的關鍵", section 三 step 三: write the new token's K/V, then attend over all
+ * of the sequence's blocks), in one launch (two with the longest-first order
+ * or the split-K merge).  k_new, v_new: [num_seqs][num_kv_heads][head_dim]
+ * bf16 device, the step's new token of each sequence, which sits at position
+ * seq_lens[b] - 1: its slot is block_tables[b][(len - 1) / 16] * 16 +
+ * (len - 1) % 16, the slot pkv_alloc_append_token hands out.  The work unit
+ * that reads a sequence's last block stores the token there before reading
+ * it.  Sequences with seq_lens[b] <= 0 write nothing.  A table entry outside
+ * the pool for that block is not written and is flagged
+ * PKV_DEV_ERR_BAD_BLOCK.  Variants: PKV_DECODE_AUTO, _SINGLE, _SPLIT
+ * (PKV_DECODE_STREAM: PKV_ERR_UNSUPPORTED).  Workspace as for
+ * pkv_paged_attention_decode_ex.
+ */
+PKV_API pkv_status pkv_paged_decode_step(void *out, const void *q, const void *k_new,
+                                         const void *v_new, void *k_cache, void *v_cache,
+                                         const int32_t *block_tables, int max_blocks_per_seq,
+                                         const int32_t *seq_lens, int num_seqs, int num_heads,
+                                         int num_kv_heads, int head_dim, int64_t num_blocks,
+                                         float scale, int variant, int partition_tokens,
+                                         void *workspace, size_t workspace_bytes,
+                                         unsigned int *err_word, void *stream);
+
+/*
  * Scratch-free split-K decode.  The pages have no counterpart to this call:
  * it exists for callers that must not allocate device memory when they run
  * decode -- e.g. an engine plugin whose execution path may not allocate, a

@@ -96,7 +96,41 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     else
         st.init(p.q + (static_cast<size_t>(b) * p.Hq + h0) * D, p.scale_log2, lane);
 
-    for (int i = 0; i < S && i < n_mine; ++i) issue(i);
+    // The fused write step: the warp that will read the sequence's last block
+    // stores the step's new K and V (position len - 1) into their slot, just
+    // before it issues that block's load -- the value is fetched into
+    // registers now, the store and the proxy fence (then __syncwarp, so lane
+    // 0's TMA read is ordered after them) wait until then.  Several
+    // head-chunk CTAs of one KV head store the same bytes.
+    const int last_local = nblk - 1 - blk_begin;
+    const bool writer = p.k_new != nullptr && blk_end == nblk && len > 0 && warp == last_local % NW;
+    const int i_write = last_local / NW;
+    uint4 new_val = make_uint4(0, 0, 0, 0);
+    __nv_bfloat16 *new_dst = nullptr;
+    if (writer && lane < 2 * (D / 8)) {
+        const int pos = len - 1;
+        const int32_t phys = __ldg(p.block_tables + static_cast<size_t>(b) * p.W + pos / kBlockTokens);
+        if (phys >= 0 && phys < p.num_blocks) {
+            const bool is_v = lane >= D / 8;
+            const int e = (lane % (D / 8)) * 8;
+            new_val = __ldg(reinterpret_cast<const uint4 *>(
+                (is_v ? p.v_new : p.k_new) + (static_cast<size_t>(b) * p.Hkv + kvh) * D + e));
+            new_dst = (is_v ? p.v_cache : p.k_cache) +
+                      ((static_cast<size_t>(phys) * p.Hkv + kvh) * kBlockTokens + pos % kBlockTokens) * D + e;
+        }
+    }
+    auto store_new = [&]() {  // warp-uniform: all lanes of the writer warp
+        if (new_dst != nullptr) {
+            *reinterpret_cast<uint4 *>(new_dst) = new_val;
+            fence_proxy_async_global();
+        }
+        __syncwarp();
+    };
+
+    for (int i = 0; i < S && i < n_mine; ++i) {
+        if (writer && i == i_write) store_new();
+        issue(i);
+    }
 
     int i = 0;
     for (; i < n_mine; ++i) {
@@ -118,7 +152,10 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (i + S < n_mine) issue(i + S);
+        if (i + S < n_mine) {
+            if (writer && i + S == i_write) store_new();
+            issue(i + S);
+        }
     }
     if (i < n_mine) {
         // A wait gave up: let the copies still in flight land before the

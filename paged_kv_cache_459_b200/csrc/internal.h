@@ -39,6 +39,11 @@ struct DecodeParams {
     // Optional [B]: unit z of the grid decodes sequence order[z] (longest
     // first); written by the order kernel launched just before.
     const int32_t *order;
+    // Optional (the fused write + decode step): this step's new K/V
+    // [B][Hkv][D], stored by the unit that holds each sequence's last block
+    // into the slot of position len - 1 before that unit reads the block.
+    const __nv_bfloat16 *k_new, *v_new;
+    __nv_bfloat16 *k_cache, *v_cache;  // [num_blocks][Hkv][16][D], for those stores
 };
 
 // Longest-first order of the sequences (by block count) into order[B], for

@@ -246,14 +246,13 @@ int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads, int he
     return PKV_DECODE_SINGLE;
 }
 
-pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
-                                         const void *v_cache, const int32_t *block_tables,
-                                         int max_blocks_per_seq, const int32_t *seq_lens,
-                                         int num_seqs, int num_heads, int num_kv_heads,
-                                         int head_dim, int64_t num_blocks, float scale,
-                                         int variant, int partition_tokens, void *workspace,
-                                         size_t workspace_bytes, unsigned int *err_word,
-                                         void *stream) {
+static pkv_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_tables, int max_blocks_per_seq,
+                              const int32_t *seq_lens, int num_seqs, int num_heads,
+                              int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
+                              int variant, int partition_tokens, void *workspace,
+                              size_t workspace_bytes, unsigned int *err_word, void *stream,
+                              const void *k_new, const void *v_new) {
     if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_kv_heads <= 0 ||
         num_heads % num_kv_heads || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
         !std::isfinite(scale))
@@ -283,6 +282,7 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
         return PKV_ERR_WORKSPACE;
     const bool stream_k = variant == PKV_DECODE_STREAM;
     const bool split = variant == PKV_DECODE_SPLIT;
+    if (k_new != nullptr && stream_k) return PKV_ERR_UNSUPPORTED;  // fused write: per-unit kernels only
     const StreamLayout sl = stream_layout(num_seqs, num_heads, num_kv_heads, head_dim);
 
     CUtensorMap tmk, tmv;
@@ -330,6 +330,10 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
     p.group = num_heads / num_kv_heads;
     p.chunks = (p.group + 7) / 8;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    p.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
+    p.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
     if (split) {
         p.part_blocks = part_blocks;
         p.num_parts = num_parts_for(max_blocks_per_seq, partition_tokens);
@@ -354,6 +358,35 @@ pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k
     cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, split, t,
                                        static_cast<cudaStream_t>(stream));
     return cuda_status(e);
+}
+
+pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
+                                         const void *v_cache, const int32_t *block_tables,
+                                         int max_blocks_per_seq, const int32_t *seq_lens,
+                                         int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int64_t num_blocks, float scale,
+                                         int variant, int partition_tokens, void *workspace,
+                                         size_t workspace_bytes, unsigned int *err_word,
+                                         void *stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, num_blocks, scale, variant,
+                       partition_tokens, workspace, workspace_bytes, err_word, stream, nullptr,
+                       nullptr);
+}
+
+pkv_status pkv_paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
+                                 void *k_cache, void *v_cache, const int32_t *block_tables,
+                                 int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+                                 int num_heads, int num_kv_heads, int head_dim,
+                                 int64_t num_blocks, float scale, int variant,
+                                 int partition_tokens, void *workspace, size_t workspace_bytes,
+                                 unsigned int *err_word, void *stream) {
+    if (num_seqs > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
+        return PKV_ERR_INVALID_ARG;
+    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, num_blocks, scale, variant,
+                       partition_tokens, workspace, workspace_bytes, err_word, stream, k_new,
+                       v_new);
 }
 
 size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,

@@ -74,6 +74,8 @@ _sigs = {
     "pkv_alloc_take_swaps": ([_P, _i32, _P, _P, _i64, _P], _i32),
     "pkv_alloc_prefix_groups": ([_P, _P, _i32, _P, _P, _P, _P], _i32),
     "pkv_decode_prefix_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
+    "pkv_paged_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
+                               _f32, _i32, _i32, _P, _sz, _P, _P], _i32),
     "pkv_paged_attention_decode_prefix": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
                                            _i64, _f32, _P, _P, _P, _i32, _i32, _i32, _P, _sz, _P,
                                            _P],
@@ -284,6 +286,41 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
                                               variant, partition_tokens, wp, wbytes, ep,
                                               _stream_ptr(q.device)),
            "pkv_paged_attention_decode")
+
+
+def paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale,
+                      num_kv_heads, *, variant: int = DECODE_AUTO,
+                      partition_tokens: int = DEFAULT_PARTITION_TOKENS,
+                      workspace=None, err=None) -> None:
+    """The write of k_new / v_new [B, Hkv, d] (each sequence's new token, at
+    position seq_lens[b] - 1) fused into paged_attention_decode: one call for
+    the whole step (see include/pkv.h, pkv_paged_decode_step)."""
+    import torch
+
+    bf = torch.bfloat16
+    B, hq, d = q.shape
+    W = block_tables.shape[1] if block_tables.dim() == 2 else -1
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
+            or block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,) \
+            or k_new.shape != (B, num_kv_heads, d) or v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch")
+    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_new, "k_new"),
+                                                 (v_new, "v_new"), (k_cache, "k_cache"),
+                                                 (v_cache, "v_cache"))]
+    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
+    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    need = decode_workspace_bytes_for(variant, B, hq, num_kv_heads, d, W, partition_tokens) \
+        if W > 0 and num_kv_heads > 0 and hq % num_kv_heads == 0 else 0
+    if workspace is None and need > 0:
+        workspace = _workspace(q.device, need)
+    wp = _dev_tensor(workspace, torch.uint8, "workspace") if workspace is not None else None
+    wbytes = workspace.numel() if workspace is not None else 0
+    _check(_lib.pkv_paged_decode_step(*ptrs, tp, W, lp, B, hq, num_kv_heads, d, k_cache.shape[0],
+                                      float(scale), variant, partition_tokens, wp, wbytes, ep,
+                                      _stream_ptr(q.device)),
+           "pkv_paged_decode_step")
 
 
 def decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_seq,

@@ -76,6 +76,35 @@ def test_decode_step_replays_from_a_graph(variant):
     assert d.err_word() == 0
 
 
+@pytest.mark.parametrize("variant", [pkv.DECODE_SINGLE, pkv.DECODE_SPLIT])
+def test_fused_step_replays_from_a_graph(variant):
+    w = build("llama", 8, batch=10, len_lo=30, len_hi=900)
+    d = DeviceStep(w)
+    c = w.cfg
+    B, hq, hkv, dh = c["batch"], c["num_heads"], c["num_kv_heads"], c["head_dim"]
+    W = w.block_tables.shape[1]
+    ws = torch.empty(max(pkv.decode_workspace_bytes_for(variant, B, hq, hkv, dh, W, 512), 256),
+                     dtype=torch.uint8, device="cuda")
+    out_g = torch.zeros_like(d.q)
+
+    def step(out):
+        pkv.paged_decode_step(out, d.q, d.k_new, d.v_new, d.kc, d.vc, d.tables, d.lens, c["scale"],
+                              hkv, variant=variant, partition_tokens=512, workspace=ws, err=d.err)
+
+    g = capture(lambda: step(out_g))
+    out_g.zero_()
+    g.replay()
+    out_d = torch.empty_like(d.q)
+    step(out_d)
+    torch.cuda.synchronize()
+    assert same(out_g, out_d)
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
+    ref = oracle.paged_decode(w.q, kc, vc, w.block_tables, w.lens, c["scale"])
+    check_close(host_bits(out_g), ref, f"fused step graph replay, variant {variant}")
+    assert d.err_word() == 0
+
+
 def test_cascade_replays_from_a_graph():
     w = build("prefix", 5, batch=12, prefix_len=320, suffix_lo=1, suffix_hi=150, prefix_groups=2)
     d = DeviceStep(w)
