@@ -362,13 +362,19 @@ def run_gpu(args):
 
     # The step: the new token's K/V write fused into the decode kernel
     # (pkv_paged_decode_step), or the write and the decode as two calls.
-    fused = not args.cascade and not args.unfused and chosen != pkv.DECODE_STREAM
+    fused = not args.unfused and (args.cascade or chosen != pkv.DECODE_STREAM)
 
     def fused_step(o=None, c=None):
         c = c or {"q": q, "k": k_new, "v": v_new, "tables": tables, "lens": lens}
-        pkv.paged_decode_step(out if o is None else o, c["q"], c["k"], c["v"], kc, vc, c["tables"],
-                              c["lens"], scale, hkv, variant=variant,
-                              partition_tokens=args.partition, workspace=ws, err=err)
+        if args.cascade:
+            pkv.paged_decode_prefix_step(out if o is None else o, c["q"], c["k"], c["v"], kc, vc,
+                                         c["tables"], c["lens"], scale, hkv, pb, offs_g, mem,
+                                         max_suffix_blocks=suffix_bound,
+                                         partition_tokens=args.partition, workspace=ws, err=err)
+        else:
+            pkv.paged_decode_step(out if o is None else o, c["q"], c["k"], c["v"], kc, vc,
+                                  c["tables"], c["lens"], scale, hkv, variant=variant,
+                                  partition_tokens=args.partition, workspace=ws, err=err)
 
     def step():
         if fused:
@@ -568,8 +574,8 @@ def run_gpu(args):
     ordered = chosen == pkv.DECODE_SINGLE and ws.numel() >= 4 * B
     launches_per_step = (1 if fused else 2) + \
         (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) or ordered else 0)
-    if args.cascade:
-        launches_per_step = 1 + 3  # write; prefix chunks, suffix split-K, merge
+    if args.cascade:  # (write;) prefix chunks + suffix split-K in one launch, merge
+        launches_per_step = 2 if fused else 3
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -597,12 +603,16 @@ def run_gpu(args):
         "kv_frac_of_measured_copy": achieved / peak,
         "write_us": write_ms * 1e3 if write_ms is not None else None,
         "decode_us": decode_ms * 1e3,
-        "step": "pkv_paged_decode_step: the write fused into the decode kernel" if fused else
+        "step": ("pkv_paged_decode_prefix_step" if args.cascade else "pkv_paged_decode_step") +
+                ": the write fused into the decode kernel" if fused else
                 "pkv_paged_kv_write, then the decode call",
         "unfused": unfused,
         "roofline": {
             "bound": "hbm",
-            "kernel": ("paged_decode_kernel with the fused write" if fused else "paged_decode_kernel")
+            "kernel": ("cascade_kernel (prefix chunks + suffix units" +
+                       (", fused write" if fused else "") + ") + cascade_merge_kernel")
+                      if args.cascade else
+                      ("paged_decode_kernel with the fused write" if fused else "paged_decode_kernel")
                       + (" + merge kernel" if chosen == pkv.DECODE_SPLIT else
                          " + order kernel" if ordered else ""),
             "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,

@@ -277,6 +277,23 @@ PKV_API pkv_status pkv_paged_attention_decode_prefix(
     size_t workspace_bytes, unsigned int *err_word, void *stream);
 
 /*
+ * The shared-prefix decode with the step's write fused in, as
+ * pkv_paged_decode_step is to pkv_paged_attention_decode_ex: k_new, v_new
+ * [num_seqs][num_kv_heads][head_dim] bf16 are each sequence's new token (at
+ * position seq_lens[b] - 1, always past its shared prefix: the token's block
+ * is private -- pkv_alloc_append_token copies a shared one first), stored by
+ * the suffix unit that reads that block before it reads it.  Same cache and
+ * output as pkv_paged_kv_write followed by pkv_paged_attention_decode_prefix.
+ */
+PKV_API pkv_status pkv_paged_decode_prefix_step(
+    void *out, const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *seq_lens, int num_seqs,
+    int num_heads, int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
+    const int32_t *prefix_blocks, const int32_t *group_offsets, const int32_t *group_seqs,
+    int num_groups, int max_suffix_blocks, int partition_tokens, void *workspace,
+    size_t workspace_bytes, unsigned int *err_word, void *stream);
+
+/*
  * Block copy for copy-on-write (a sequence that shares a partly filled block,
  * e.g. a beam forked mid-block -- "vllm" (xiexianbin.cn), "PagedAttention 的核
  * 心原理": beam candidates share prefix blocks -- takes a private copy before

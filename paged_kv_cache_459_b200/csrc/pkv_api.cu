@@ -401,7 +401,7 @@ size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_d
            sizeof(float);
 }
 
-pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const void *k_cache,
+static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
                                              const void *v_cache, const int32_t *block_tables,
                                              int max_blocks_per_seq, const int32_t *seq_lens,
                                              int num_seqs, int num_heads, int num_kv_heads,
@@ -411,7 +411,8 @@ pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const voi
                                              const int32_t *group_seqs, int num_groups,
                                              int max_suffix_blocks, int partition_tokens,
                                              void *workspace, size_t workspace_bytes,
-                                             unsigned int *err_word, void *stream) {
+                                             unsigned int *err_word, void *stream,
+                              const void *k_new, const void *v_new) {
     if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_kv_heads <= 0 ||
         num_heads % num_kv_heads || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
         !std::isfinite(scale) || num_groups < 0 || num_groups > 65535)
@@ -493,10 +494,52 @@ pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const voi
     dp.ws_part0 = prefix_parts;
     dp.start_blocks = prefix_blocks;
     dp.skip_merge = true;
+    dp.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    dp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    dp.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
+    dp.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
 
     cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
                                         static_cast<cudaStream_t>(stream));
     return cuda_status(e);
+}
+
+pkv_status pkv_paged_attention_decode_prefix(void *out, const void *q, const void *k_cache,
+                                             const void *v_cache, const int32_t *block_tables,
+                                             int max_blocks_per_seq, const int32_t *seq_lens,
+                                             int num_seqs, int num_heads, int num_kv_heads,
+                                             int head_dim, int64_t num_blocks, float scale,
+                                             const int32_t *prefix_blocks,
+                                             const int32_t *group_offsets,
+                                             const int32_t *group_seqs, int num_groups,
+                                             int max_suffix_blocks, int partition_tokens,
+                                             void *workspace, size_t workspace_bytes,
+                                             unsigned int *err_word, void *stream) {
+    return prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, num_blocks, scale,
+                       prefix_blocks, group_offsets, group_seqs, num_groups, max_suffix_blocks,
+                       partition_tokens, workspace, workspace_bytes, err_word, stream, nullptr,
+                       nullptr);
+}
+
+pkv_status pkv_paged_decode_prefix_step(void *out, const void *q, const void *k_new,
+                                        const void *v_new, void *k_cache, void *v_cache,
+                                        const int32_t *block_tables, int max_blocks_per_seq,
+                                        const int32_t *seq_lens, int num_seqs, int num_heads,
+                                        int num_kv_heads, int head_dim, int64_t num_blocks,
+                                        float scale, const int32_t *prefix_blocks,
+                                        const int32_t *group_offsets, const int32_t *group_seqs,
+                                        int num_groups, int max_suffix_blocks,
+                                        int partition_tokens, void *workspace,
+                                        size_t workspace_bytes, unsigned int *err_word,
+                                        void *stream) {
+    if (num_seqs > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
+        return PKV_ERR_INVALID_ARG;
+    return prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, num_blocks, scale,
+                       prefix_blocks, group_offsets, group_seqs, num_groups, max_suffix_blocks,
+                       partition_tokens, workspace, workspace_bytes, err_word, stream, k_new,
+                       v_new);
 }
 
 pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_cache,

@@ -76,6 +76,9 @@ _sigs = {
     "pkv_decode_prefix_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
     "pkv_paged_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
                                _f32, _i32, _i32, _P, _sz, _P, _P], _i32),
+    "pkv_paged_decode_prefix_step": ([_P, _P, _P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
+                                      _i64, _f32, _P, _P, _P, _i32, _i32, _i32, _P, _sz, _P, _P],
+                                     _i32),
     "pkv_paged_attention_decode_prefix": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32,
                                            _i64, _f32, _P, _P, _P, _i32, _i32, _i32, _P, _sz, _P,
                                            _P],
@@ -365,6 +368,43 @@ def paged_attention_decode_prefix(out, q, k_cache, v_cache, block_tables, seq_le
         float(scale), pp, op, gp, G, int(max_suffix_blocks), partition_tokens, wp,
         workspace.numel(), ep,
         _stream_ptr(q.device)), "pkv_paged_attention_decode_prefix")
+
+
+def paged_decode_prefix_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale,
+                             num_kv_heads, prefix_blocks, group_offsets, group_seqs, *,
+                             max_suffix_blocks: int = 0,
+                             partition_tokens: int = DEFAULT_PARTITION_TOKENS,
+                             workspace=None, err=None) -> None:
+    """paged_attention_decode_prefix with the write of k_new / v_new [B, Hkv, d]
+    (each sequence's new token, at position seq_lens[b] - 1) fused in."""
+    import torch
+
+    bf = torch.bfloat16
+    B, hq, d = q.shape
+    W = block_tables.shape[1]
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
+            or block_tables.shape[0] != B or seq_lens.shape != (B,) or prefix_blocks.shape != (B,) \
+            or k_new.shape != (B, num_kv_heads, d) or v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch")
+    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_new, "k_new"),
+                                                 (v_new, "v_new"), (k_cache, "k_cache"),
+                                                 (v_cache, "v_cache"))]
+    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
+    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
+    pp = _dev_tensor(prefix_blocks, torch.int32, "prefix_blocks")
+    G = group_offsets.numel() - 1
+    op = _dev_tensor(group_offsets, torch.int32, "group_offsets")
+    gp = _dev_tensor(group_seqs, torch.int32, "group_seqs") if group_seqs.numel() else None
+    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
+    if workspace is None:
+        workspace = _workspace(q.device, decode_prefix_workspace_bytes(B, hq, d, W,
+                                                                       partition_tokens))
+    wp = _dev_tensor(workspace, torch.uint8, "workspace")
+    _check(_lib.pkv_paged_decode_prefix_step(
+        *ptrs, tp, W, lp, B, hq, num_kv_heads, d, k_cache.shape[0], float(scale), pp, op, gp, G,
+        int(max_suffix_blocks), partition_tokens, wp, workspace.numel(), ep,
+        _stream_ptr(q.device)), "pkv_paged_decode_prefix_step")
 
 
 def suffix_blocks_bound(seq_lens, prefix_blocks) -> int:

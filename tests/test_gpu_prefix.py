@@ -95,3 +95,29 @@ def test_cascade_block_relabelling_is_bit_exact():
     d.vc.copy_(torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16))
     out, _, _ = cascade(d, tables=torch.from_numpy(t2).cuda())
     assert np.array_equal(out, base)
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
+def test_cascade_fused_step(idx):
+    """pkv_paged_decode_prefix_step: the step's write fused into the cascade --
+    caches bit-exact with the oracle's write, output within tolerance, and
+    bit-identical to the separate write + cascade."""
+    name, kw = CASES[idx]
+    w = build(name, 31, **kw)
+    kc, vc, ref = oracle_after_write(w)
+    pb, offs, members = w.alloc.prefix_groups(list(range(w.cfg["batch"])))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).cuda()  # noqa: E731
+    bound = pkv.suffix_blocks_bound(w.lens, pb)
+    d = DeviceStep(w)
+    pkv.paged_decode_prefix_step(d.out, d.q, d.k_new, d.v_new, d.kc, d.vc, d.tables, d.lens,
+                                 w.cfg["scale"], w.cfg["num_kv_heads"], dev(pb), dev(offs),
+                                 dev(members), max_suffix_blocks=bound, err=d.err)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
+    out = host_bits(d.out)
+    check_close(out, ref, f"fused cascade step {kw}")
+    e = DeviceStep(w)
+    e.write()
+    sep, _, _ = cascade(e, bound="exact")
+    assert np.array_equal(out, sep)
+    assert d.err_word() == 0
