@@ -440,10 +440,9 @@ def run_gpu(args):
             decode()
             uev[i][2].record(stream)
         torch.cuda.synchronize(dev)
-        u_total = sum(e[0].elapsed_time(e[2]) for e in uev)
         unfused = {"write_us": 1e3 * statistics.fmean(e[0].elapsed_time(e[1]) for e in uev),
                    "decode_us": 1e3 * statistics.fmean(e[1].elapsed_time(e[2]) for e in uev),
-                   "value": job_throughput(B, K, 1, u_total)}
+                   "total_ms": sum(e[0].elapsed_time(e[2]) for e in uev)}
     # keep the GPU loaded long enough for the clock sampler to see it
     if sampler is not None:
         t0 = time.perf_counter()
@@ -559,7 +558,11 @@ def run_gpu(args):
     e2e_graph_ms = pipelined(lambda i: graphs[i % 2].replay())
     del graphs
 
-    total_ms, e2e_ms, e2e_graph_ms = max_over_ranks([total_ms, e2e_ms, e2e_graph_ms], device=dev)
+    total_ms, e2e_ms, e2e_graph_ms, u_ms = max_over_ranks(
+        [total_ms, e2e_ms, e2e_graph_ms, unfused["total_ms"] if unfused else 0.0], device=dev)
+    if unfused:
+        unfused = {"write_us": unfused["write_us"], "decode_us": unfused["decode_us"],
+                   "value": job_throughput(B, K, world, u_ms)}
 
     ab = algorithmic_bytes(w)
     peak, peak_kind = measured_peak_hbm()
