@@ -57,7 +57,7 @@ def parse_args():
                     help="override the workload's batch (smaller cases for ncu captures)")
     ap.add_argument("--variant", choices=["auto", "single", "split", "stream"], default="auto")
     ap.add_argument("--partition", type=int, default=512)
-    ap.add_argument("--row", choices=["decode", "prefill", "cow", "swap"], default="decode",
+    ap.add_argument("--row", choices=["decode", "prefill", "cow", "swap", "alloc"], default="decode",
                     help="which part of the path to measure (decode: the default step)")
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix decode: prefix blocks read once per group and KV head")
@@ -677,9 +677,47 @@ def _events_time(fn, steps, warmup):
     return a.elapsed_time(b) / steps  # ms
 
 
+def run_alloc_row(args):
+    """Host cost of the block allocator per decode step (one new token for
+    every sequence of the workload, then the tables and lengths exported), on
+    the CPU: what the engine pays before each decode call."""
+    from paged_kv_cache_459_b200 import pkv
+    from paged_kv_cache_459_b200 import workloads as wl
+
+    cfg = wl.config("qwen" if args.config == "qwen" else "llama")
+    B = cfg["batch"]
+    rng = wl.rng(args.seed)
+    lens = rng.integers(cfg["len_lo"], cfg["len_hi"] + 1, size=B)
+    steps, warm = args.steps, max(3, args.warmup)
+    need = int(sum(-(-(int(n) + steps + warm) // 16) for n in lens))
+    alloc = pkv.BlockAllocator(need + 64, rng.permutation(need + 64))
+    for b, n in enumerate(lens):
+        alloc.add_seq(b, int(n))
+    ids = list(range(B))
+    width = -(-int(lens.max() + steps + warm) // 16)
+    for _ in range(warm):
+        alloc.append_tokens(ids)
+        alloc.export(ids, width)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        alloc.append_tokens(ids)
+        alloc.export(ids, width)
+    el = time.perf_counter() - t0
+    print(json.dumps({"row": "alloc", "steps": steps, "warmup": warm, "data": "synthetic",
+                      "metric": "host allocator time per decode step (append one token to every "
+                                "sequence, export tables and lengths)",
+                      "value": 1e6 * el / steps, "unit": "us", "higher_is_better": False,
+                      "config": {"workload": f"{B} sequences, lengths U[{cfg['len_lo']},"
+                                             f"{cfg['len_hi']}], table width {width}",
+                                 "threads": 1}}), flush=True)
+    return 0
+
+
 def run_row(args):
     """Measurements of the rows next to the decode step: prefill attention,
     copy-on-write block copies, and block swap over the host link."""
+    if args.row == "alloc":
+        return run_alloc_row(args)
     import torch
     from paged_kv_cache_459_b200 import pkv
     from paged_kv_cache_459_b200 import workloads as wl

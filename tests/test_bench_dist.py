@@ -59,3 +59,13 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_alloc_row_runs_on_the_host():
+    """bench.py --row alloc (host allocator cost per decode step) needs no GPU."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--row", "alloc",
+                        "--steps", "20", "--warmup", "3"], capture_output=True, text=True,
+                       timeout=120, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["row"] == "alloc" and line["unit"] == "us" and line["value"] > 0
