@@ -284,6 +284,9 @@ PKV_API pkv_status pkv_paged_attention_decode_prefix(
  * is private -- pkv_alloc_append_token copies a shared one first), stored by
  * the suffix unit that reads that block before it reads it.  Same cache and
  * output as pkv_paged_kv_write followed by pkv_paged_attention_decode_prefix.
+ * A sequence whose prefix_blocks[b] covers its last block (the new token
+ * inside the shared prefix: not what pkv_alloc_prefix_groups produces) is
+ * not written and is flagged PKV_DEV_ERR_BAD_LEN.
  */
 PKV_API pkv_status pkv_paged_decode_prefix_step(
     void *out, const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -37,6 +37,11 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     if (blk_begin >= blk_end) {
         // Nothing to read.  Single pass: the (empty) sequence's rows are zero.
         // Split-K: the merge kernel only reads partitions that hold tokens.
+        // A fused write whose token lies before the start block (inside a
+        // shared prefix) cannot be done here: flagged.
+        if (p.k_new != nullptr && part == 0 && len > 0 && start >= nblk && threadIdx.x == 0 &&
+            (!MMA || by % p.chunks == 0))
+            flag(p.err, PKV_DEV_ERR_BAD_LEN);
         if (!SPLIT)
             for (int i = threadIdx.x; i < heads * D; i += NW * 32)
                 p.out[(static_cast<size_t>(b) * p.Hq + h0 + i / D) * D + i % D] = __float2bfloat16(0.f);

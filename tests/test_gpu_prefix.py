@@ -121,3 +121,18 @@ def test_cascade_fused_step(idx):
     sep, _, _ = cascade(e, bound="exact")
     assert np.array_equal(out, sep)
     assert d.err_word() == 0
+
+
+def test_cascade_fused_step_token_inside_prefix_is_flagged():
+    """A prefix_blocks entry that covers a sequence's last block (not what the
+    allocator's grouping produces) leaves the fused write undone, flagged."""
+    w = build("prefix", 32, batch=4, prefix_len=64, suffix_lo=16, suffix_hi=16)  # len 80: 5 full blocks
+    pb, offs, members = w.alloc.prefix_groups(list(range(w.cfg["batch"])))
+    pb = pb.copy()
+    pb[1] = int(w.lens[1]) // 16      # claims the whole sequence, its new token included
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).cuda()  # noqa: E731
+    d = DeviceStep(w)
+    pkv.paged_decode_prefix_step(d.out, d.q, d.k_new, d.v_new, d.kc, d.vc, d.tables, d.lens,
+                                 w.cfg["scale"], w.cfg["num_kv_heads"], dev(pb), dev(offs),
+                                 dev(members), err=d.err)
+    assert d.err_word() & 4
