@@ -257,6 +257,36 @@ def decode_variant_for(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_p
                                            max_blocks_per_seq, partition_tokens, workspace_bytes))
 
 
+def _decode_args(out, q, new_kv, k_cache, v_cache, block_tables, seq_lens, num_kv_heads, variant,
+                 partition_tokens, workspace, err):
+    """Checked pointers and sizes shared by the decode entry points: (out, q,
+    [k_new, v_new,] k_cache, v_cache) then the table / length / size arguments
+    up to num_blocks, and (workspace, bytes, err)."""
+    import torch
+
+    B, hq, d = q.shape
+    W = block_tables.shape[1] if block_tables.dim() == 2 else -1
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
+            or block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,) \
+            or any(x.shape != (B, num_kv_heads, d) for x in new_kv):
+        raise ValueError("shape mismatch")
+    named = [(out, "out"), (q, "q")] + list(zip(new_kv, ("k_new", "v_new"))) + \
+        [(k_cache, "k_cache"), (v_cache, "v_cache")]
+    ptrs = [_dev_tensor(x, torch.bfloat16, n) for x, n in named]
+    sizes = [_dev_tensor(block_tables, torch.int32, "block_tables"), W,
+             _dev_tensor(seq_lens, torch.int32, "seq_lens"), B, hq, num_kv_heads, d,
+             k_cache.shape[0]]
+    need = decode_workspace_bytes_for(variant, B, hq, num_kv_heads, d, W, partition_tokens) \
+        if W > 0 and num_kv_heads > 0 and hq % num_kv_heads == 0 else 0
+    if workspace is None and need > 0:
+        workspace = _workspace(q.device, need)
+    tail = [_dev_tensor(workspace, torch.uint8, "workspace") if workspace is not None else None,
+            workspace.numel() if workspace is not None else 0,
+            _dev_tensor(err, torch.int32, "err") if err is not None else None]
+    return ptrs, sizes, tail
+
+
 def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, num_kv_heads,
                            *, variant: int = DECODE_AUTO,
                            partition_tokens: int = DEFAULT_PARTITION_TOKENS,
@@ -264,30 +294,10 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
     """out, q [B, Hq, d] bf16; caches [NB, Hkv, 16, d] bf16; block_tables [B, W]
     int32; seq_lens [B] int32.  The split-K workspace is allocated once per
     device and reused unless one is passed in (a uint8 CUDA tensor)."""
-    import torch
-
-    bf = torch.bfloat16
-    B, hq, d = q.shape
-    W = block_tables.shape[1] if block_tables.dim() == 2 else -1
-    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
-            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
-            or block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,):
-        raise ValueError("shape mismatch")
-    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"),
-                                                 (v_cache, "v_cache"))]
-    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
-    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
-    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
-    need = decode_workspace_bytes_for(variant, B, hq, num_kv_heads, d, W, partition_tokens) \
-        if W > 0 and num_kv_heads > 0 and hq % num_kv_heads == 0 else 0
-    if workspace is None and need > 0:
-        workspace = _workspace(q.device, need)
-    wp = _dev_tensor(workspace, torch.uint8, "workspace") if workspace is not None else None
-    wbytes = workspace.numel() if workspace is not None else 0
-    _check(_lib.pkv_paged_attention_decode_ex(ptrs[0], ptrs[1], ptrs[2], ptrs[3], tp, W, lp, B, hq,
-                                              num_kv_heads, d, k_cache.shape[0], float(scale),
-                                              variant, partition_tokens, wp, wbytes, ep,
-                                              _stream_ptr(q.device)),
+    ptrs, sizes, tail = _decode_args(out, q, (), k_cache, v_cache, block_tables, seq_lens,
+                                     num_kv_heads, variant, partition_tokens, workspace, err)
+    _check(_lib.pkv_paged_attention_decode_ex(*ptrs, *sizes, float(scale), variant,
+                                              partition_tokens, *tail, _stream_ptr(q.device)),
            "pkv_paged_attention_decode")
 
 
@@ -298,31 +308,11 @@ def paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_
     """The write of k_new / v_new [B, Hkv, d] (each sequence's new token, at
     position seq_lens[b] - 1) fused into paged_attention_decode: one call for
     the whole step (see include/pkv.h, pkv_paged_decode_step)."""
-    import torch
-
-    bf = torch.bfloat16
-    B, hq, d = q.shape
-    W = block_tables.shape[1] if block_tables.dim() == 2 else -1
-    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
-            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
-            or block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,) \
-            or k_new.shape != (B, num_kv_heads, d) or v_new.shape != k_new.shape:
-        raise ValueError("shape mismatch")
-    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_new, "k_new"),
-                                                 (v_new, "v_new"), (k_cache, "k_cache"),
-                                                 (v_cache, "v_cache"))]
-    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
-    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
-    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
-    need = decode_workspace_bytes_for(variant, B, hq, num_kv_heads, d, W, partition_tokens) \
-        if W > 0 and num_kv_heads > 0 and hq % num_kv_heads == 0 else 0
-    if workspace is None and need > 0:
-        workspace = _workspace(q.device, need)
-    wp = _dev_tensor(workspace, torch.uint8, "workspace") if workspace is not None else None
-    wbytes = workspace.numel() if workspace is not None else 0
-    _check(_lib.pkv_paged_decode_step(*ptrs, tp, W, lp, B, hq, num_kv_heads, d, k_cache.shape[0],
-                                      float(scale), variant, partition_tokens, wp, wbytes, ep,
-                                      _stream_ptr(q.device)),
+    ptrs, sizes, tail = _decode_args(out, q, (k_new, v_new), k_cache, v_cache, block_tables,
+                                     seq_lens, num_kv_heads, variant, partition_tokens, workspace,
+                                     err)
+    _check(_lib.pkv_paged_decode_step(*ptrs, *sizes, float(scale), variant, partition_tokens,
+                                      *tail, _stream_ptr(q.device)),
            "pkv_paged_decode_step")
 
 
@@ -330,6 +320,38 @@ def decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_
                                   partition_tokens=DEFAULT_PARTITION_TOKENS) -> int:
     return int(_lib.pkv_decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim,
                                                       max_blocks_per_seq, partition_tokens))
+
+
+def _prefix_args(out, q, new_kv, k_cache, v_cache, block_tables, seq_lens, num_kv_heads,
+                 prefix_blocks, group_offsets, group_seqs, partition_tokens, workspace, err):
+    """Checked pointers and sizes shared by the cascade entry points: (out, q,
+    [k_new, v_new,] k_cache, v_cache), the table / length / size arguments up
+    to num_blocks, the group arrays, and (workspace, bytes, err)."""
+    import torch
+
+    B, hq, d = q.shape
+    W = block_tables.shape[1]
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
+            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
+            or block_tables.shape[0] != B or seq_lens.shape != (B,) or prefix_blocks.shape != (B,) \
+            or any(x.shape != (B, num_kv_heads, d) for x in new_kv):
+        raise ValueError("shape mismatch")
+    named = [(out, "out"), (q, "q")] + list(zip(new_kv, ("k_new", "v_new"))) + \
+        [(k_cache, "k_cache"), (v_cache, "v_cache")]
+    ptrs = [_dev_tensor(x, torch.bfloat16, n) for x, n in named]
+    sizes = [_dev_tensor(block_tables, torch.int32, "block_tables"), W,
+             _dev_tensor(seq_lens, torch.int32, "seq_lens"), B, hq, num_kv_heads, d,
+             k_cache.shape[0]]
+    groups = [_dev_tensor(prefix_blocks, torch.int32, "prefix_blocks"),
+              _dev_tensor(group_offsets, torch.int32, "group_offsets"),
+              _dev_tensor(group_seqs, torch.int32, "group_seqs") if group_seqs.numel() else None,
+              group_offsets.numel() - 1]
+    if workspace is None:
+        workspace = _workspace(q.device, decode_prefix_workspace_bytes(B, hq, d, W,
+                                                                       partition_tokens))
+    tail = [_dev_tensor(workspace, torch.uint8, "workspace"), workspace.numel(),
+            _dev_tensor(err, torch.int32, "err") if err is not None else None]
+    return ptrs, sizes, groups, tail
 
 
 def paged_attention_decode_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
@@ -341,33 +363,13 @@ def paged_attention_decode_prefix(out, q, k_cache, v_cache, block_tables, seq_le
     prefix_blocks [B], group_offsets [G + 1], group_seqs [members]: int32 CUDA.
     max_suffix_blocks: bound on the blocks past each prefix (0: unknown);
     suffix_blocks_bound() computes it from host arrays."""
-    import torch
-
-    bf = torch.bfloat16
-    B, hq, d = q.shape
-    W = block_tables.shape[1]
-    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
-            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
-            or block_tables.shape[0] != B or seq_lens.shape != (B,) or prefix_blocks.shape != (B,):
-        raise ValueError("shape mismatch")
-    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"),
-                                                 (v_cache, "v_cache"))]
-    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
-    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
-    pp = _dev_tensor(prefix_blocks, torch.int32, "prefix_blocks")
-    G = group_offsets.numel() - 1
-    op = _dev_tensor(group_offsets, torch.int32, "group_offsets")
-    gp = _dev_tensor(group_seqs, torch.int32, "group_seqs") if group_seqs.numel() else None
-    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
-    if workspace is None:
-        workspace = _workspace(q.device, decode_prefix_workspace_bytes(B, hq, d, W,
-                                                                       partition_tokens))
-    wp = _dev_tensor(workspace, torch.uint8, "workspace")
-    _check(_lib.pkv_paged_attention_decode_prefix(
-        ptrs[0], ptrs[1], ptrs[2], ptrs[3], tp, W, lp, B, hq, num_kv_heads, d, k_cache.shape[0],
-        float(scale), pp, op, gp, G, int(max_suffix_blocks), partition_tokens, wp,
-        workspace.numel(), ep,
-        _stream_ptr(q.device)), "pkv_paged_attention_decode_prefix")
+    ptrs, sizes, groups, tail = _prefix_args(out, q, (), k_cache, v_cache, block_tables, seq_lens,
+                                             num_kv_heads, prefix_blocks, group_offsets,
+                                             group_seqs, partition_tokens, workspace, err)
+    _check(_lib.pkv_paged_attention_decode_prefix(*ptrs, *sizes, float(scale), *groups,
+                                                  int(max_suffix_blocks), partition_tokens,
+                                                  *tail, _stream_ptr(q.device)),
+           "pkv_paged_attention_decode_prefix")
 
 
 def paged_decode_prefix_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale,
@@ -377,34 +379,14 @@ def paged_decode_prefix_step(out, q, k_new, v_new, k_cache, v_cache, block_table
                              workspace=None, err=None) -> None:
     """paged_attention_decode_prefix with the write of k_new / v_new [B, Hkv, d]
     (each sequence's new token, at position seq_lens[b] - 1) fused in."""
-    import torch
-
-    bf = torch.bfloat16
-    B, hq, d = q.shape
-    W = block_tables.shape[1]
-    if out.shape != q.shape or k_cache.shape != v_cache.shape or k_cache.dim() != 4 \
-            or tuple(k_cache.shape[1:]) != (num_kv_heads, BLOCK_TOKENS, d) \
-            or block_tables.shape[0] != B or seq_lens.shape != (B,) or prefix_blocks.shape != (B,) \
-            or k_new.shape != (B, num_kv_heads, d) or v_new.shape != k_new.shape:
-        raise ValueError("shape mismatch")
-    ptrs = [_dev_tensor(x, bf, n) for x, n in ((out, "out"), (q, "q"), (k_new, "k_new"),
-                                                 (v_new, "v_new"), (k_cache, "k_cache"),
-                                                 (v_cache, "v_cache"))]
-    tp = _dev_tensor(block_tables, torch.int32, "block_tables")
-    lp = _dev_tensor(seq_lens, torch.int32, "seq_lens")
-    pp = _dev_tensor(prefix_blocks, torch.int32, "prefix_blocks")
-    G = group_offsets.numel() - 1
-    op = _dev_tensor(group_offsets, torch.int32, "group_offsets")
-    gp = _dev_tensor(group_seqs, torch.int32, "group_seqs") if group_seqs.numel() else None
-    ep = _dev_tensor(err, torch.int32, "err") if err is not None else None
-    if workspace is None:
-        workspace = _workspace(q.device, decode_prefix_workspace_bytes(B, hq, d, W,
-                                                                       partition_tokens))
-    wp = _dev_tensor(workspace, torch.uint8, "workspace")
-    _check(_lib.pkv_paged_decode_prefix_step(
-        *ptrs, tp, W, lp, B, hq, num_kv_heads, d, k_cache.shape[0], float(scale), pp, op, gp, G,
-        int(max_suffix_blocks), partition_tokens, wp, workspace.numel(), ep,
-        _stream_ptr(q.device)), "pkv_paged_decode_prefix_step")
+    ptrs, sizes, groups, tail = _prefix_args(out, q, (k_new, v_new), k_cache, v_cache,
+                                             block_tables, seq_lens, num_kv_heads, prefix_blocks,
+                                             group_offsets, group_seqs, partition_tokens,
+                                             workspace, err)
+    _check(_lib.pkv_paged_decode_prefix_step(*ptrs, *sizes, float(scale), *groups,
+                                             int(max_suffix_blocks), partition_tokens, *tail,
+                                             _stream_ptr(q.device)),
+           "pkv_paged_decode_prefix_step")
 
 
 def suffix_blocks_bound(seq_lens, prefix_blocks) -> int:
