@@ -70,6 +70,45 @@ def test_decode_argument_checks(kw, code):
     assert decode(**kw) == code
 
 
+def step(**kw):
+    """pkv_paged_decode_step: decode's arguments plus the step's new K and V."""
+    args = dict(out=FAKE, q=FAKE, kn=FAKE, vn=FAKE, kc=FAKE, vc=FAKE, tables=FAKE, W=8, lens=FAKE,
+                B=2, Hq=4, Hkv=2, D=128, NB=64, scale=0.1, variant=0, part=512, ws=None, wsb=0)
+    args.update(kw)
+    return pkv.lib().pkv_paged_decode_step(
+        args["out"], args["q"], args["kn"], args["vn"], args["kc"], args["vc"], args["tables"],
+        args["W"], args["lens"], args["B"], args["Hq"], args["Hkv"], args["D"], args["NB"],
+        args["scale"], args["variant"], args["part"], args["ws"], args["wsb"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kn=None), pkv.ERR_INVALID_ARG),
+    (dict(vn=None), pkv.ERR_INVALID_ARG),
+    (dict(kn=FAKE + 4), pkv.ERR_INVALID_ARG),
+    (dict(D=96), pkv.ERR_UNSUPPORTED),
+    (dict(variant=3, ws=FAKE, wsb=1 << 40), pkv.ERR_UNSUPPORTED),   # stream-K: no fused write
+    (dict(variant=2), pkv.ERR_WORKSPACE),
+])
+def test_fused_step_argument_checks(kw, code):
+    assert step(**kw) == code
+
+
+def test_fused_step_empty_batch_is_a_no_op():
+    assert step(B=0, out=None, q=None, kn=None, vn=None) == pkv.OK
+
+
+def test_cascade_steps_check_their_arguments():
+    L = pkv.lib()
+    common = (FAKE, FAKE, FAKE, FAKE, FAKE, 8, FAKE, 2, 4, 2, 128, 64, 0.1, FAKE, FAKE, FAKE, 1)
+    # fused: a missing new K
+    assert L.pkv_paged_decode_prefix_step(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 8, FAKE, 2, 4, 2,
+                                          128, 64, 0.1, FAKE, FAKE, FAKE, 1, 0, 512, FAKE, 1 << 30,
+                                          None, None) == pkv.ERR_INVALID_ARG
+    # plain: too little workspace
+    assert L.pkv_paged_attention_decode_prefix(*common, 0, 512, FAKE, 16, None, None) == \
+        pkv.ERR_WORKSPACE
+
+
 def test_empty_batch_is_a_no_op():
     assert decode(B=0, out=None, q=None) == pkv.OK
 
