@@ -369,6 +369,7 @@ typedef struct pkv_alloc pkv_alloc;
  * (blocks are taken from its front, freed blocks go to its back); NULL means
  * ascending order. */
 PKV_API pkv_status pkv_alloc_create(int64_t num_blocks, const int64_t *free_order, pkv_alloc **out);
+/* Releases the allocator (NULL is a no-op); the device caches are the caller's. */
 PKV_API void pkv_alloc_destroy(pkv_alloc *a);
 
 /* New sequence holding num_tokens prefilled tokens: ceil(num_tokens/16) blocks. */
@@ -450,6 +451,10 @@ PKV_API pkv_status pkv_alloc_free_list(const pkv_alloc *a, int64_t *out, int64_t
 PKV_API pkv_status pkv_alloc_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, int n,
                                            int32_t *prefix_blocks_out, int32_t *group_offsets_out,
                                            int32_t *group_seqs_out, int32_t *num_groups_out);
+/* Queries (host; PKV_ERR_INVALID_ARG for an unknown id or position):
+ * refcount: the number of tables holding block `block` (0 if free); seq_len:
+ * the tokens of a sequence; slot_of: the cache slot (block * 16 + offset) of
+ * position pos in [0, seq_len) of a sequence resident on the GPU. */
 PKV_API pkv_status pkv_alloc_refcount(const pkv_alloc *a, int64_t block, int32_t *out);
 PKV_API pkv_status pkv_alloc_seq_len(const pkv_alloc *a, int64_t seq_id, int64_t *len_out);
 PKV_API pkv_status pkv_alloc_slot_of(const pkv_alloc *a, int64_t seq_id, int64_t pos, int64_t *slot_out);
