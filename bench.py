@@ -443,6 +443,14 @@ def run_gpu(args):
         unfused = {"write_us": 1e3 * statistics.fmean(e[0].elapsed_time(e[1]) for e in uev),
                    "decode_us": 1e3 * statistics.fmean(e[1].elapsed_time(e[2]) for e in uev),
                    "total_ms": sum(e[0].elapsed_time(e[2]) for e in uev)}
+    prefix_tc = None
+    if args.cascade and fused:  # the same step with the prefix chunks on tcgen05 (opt-in path)
+        os.environ["PKV_CASCADE_TC"] = "1"
+        try:
+            prefix_tc = {"step_us": 1e3 * _events_time(step, K, Wm),
+                         "how": "PKV_CASCADE_TC=1: prefix chunks on tcgen05/TMEM, same step, events"}
+        finally:
+            os.environ.pop("PKV_CASCADE_TC")
     # keep the GPU loaded long enough for the clock sampler to see it
     if sampler is not None:
         t0 = time.perf_counter()
@@ -614,6 +622,7 @@ def run_gpu(args):
                 ": the write fused into the decode kernel" if fused else
                 "pkv_paged_kv_write, then the decode call",
         "unfused": unfused,
+        **({"prefix_tcgen05": prefix_tc} if prefix_tc else {}),
         "roofline": {
             "bound": "hbm",
             "kernel": ("cascade_kernel (prefix chunks + suffix units" +

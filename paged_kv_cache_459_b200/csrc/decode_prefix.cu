@@ -15,7 +15,10 @@
 // kernel starting past the prefix, and the merge below combines prefix and
 // suffix partials of each (sequence, query head) by log-sum-exp.  The result
 // equals plain decode over the whole sequence.
+#include <algorithm>
+
 #include "decode_unit.cuh"
+#include "tcgen05.cuh"
 
 namespace pkv {
 
@@ -27,7 +30,7 @@ constexpr int kPrefixWarps = 4;
 constexpr float kLazyRescale = 8.0f;  // log2 units: the running max moves past this growth only
 
 template <int D, int CB>
-struct PrefixGeometry {
+struct PrefixMmaGeometry {
     static constexpr int kTile = (D / 64) * kBoxBytes;  // one K or V tile of a block
     static constexpr int kSmemBytes = 2 * CB * kTile + 8 + CB * 4 + 1024;
 };
@@ -35,11 +38,11 @@ struct PrefixGeometry {
 // Prefix chunk c (blocks [c*CB, (c+1)*CB) of group g's shared prefix) for KV
 // head kvh: all member rows against the chunk's K/V, one partial per row.
 template <int D, int CB>
-__device__ __forceinline__ void prefix_unit(const CUtensorMap &tmk, const CUtensorMap &tmv,
+__device__ __forceinline__ void prefix_unit_mma(const CUtensorMap &tmk, const CUtensorMap &tmv,
                                             const PrefixParams &p, int c, int kvh, int g) {
     constexpr int KS = D / 16;                     // k-steps of S = Q K^T over d
     constexpr int NT = D / 8;                      // 8-column tiles of O
-    constexpr int kTile = PrefixGeometry<D, CB>::kTile;
+    constexpr int kTile = PrefixMmaGeometry<D, CB>::kTile;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tig = lane & 3, gid = lane >> 2;
 
@@ -253,6 +256,294 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap &tmk, const CUtens
     }
 }
 
+template <int D, int CB>
+struct PrefixTcGeometry {
+    static constexpr int kKeys = CB * kBlockTokens;     // keys of one chunk: MMA N of S, K of P.V
+    static constexpr int kKV = (D / 64) * kKeys * 128;  // one K or V chunk [d half][key][128 B]
+    static constexpr int kMeta = 64;                    // 3 mbarriers, TMEM base, valid[CB]
+    static constexpr int kSmemBytes = 2 * kKV + kMeta + 1024;
+    static constexpr int kTmemCols = 256;               // S (P over its first half) | O (Q before it)
+    static_assert(kKeys == 128 && 32 + 4 * CB <= kMeta, "chunk layout");
+    static_assert(kKeys + D <= kTmemCols, "tensor memory columns");
+};
+
+// Prefix chunk c (blocks [c*CB, (c+1)*CB) of group g's shared prefix) for KV
+// head kvh on the tcgen05 tensor cores.  The chunk's K and V (128 keys) are
+// loaded once by TMA; the rows, (member, query head) pairs, go in tiles of
+// 128, one row per thread (= TMEM lane).  Per row tile:
+//   Q rows (bf16) -> TMEM, in O's columns (O is not written before P.V)
+//   S[128 x 128] = Q K^T    tcgen05.mma, A from TMEM, K from shared memory
+//   m = max S * scale, P = 2^(S * scale - m) as bf16 into TMEM over S,
+//   l = sum P (fp32)
+//   O[128 x d]   = P V      tcgen05.mma, A from TMEM, V from shared memory
+// and the row's partial (m, l, O) goes to its workspace slot.  A chunk is one
+// key tile, so the softmax is a single pass with no running max.  Keys of
+// blocks past the prefix or with a bad table entry are loaded as zeros (a row
+// past the tensor) and masked to -inf.  Every wait is bounded; on a timeout the
+// CTA flags it, waits (bounded) for its copies and MMAs, and frees its TMEM.
+template <int D, int CB>
+__device__ __forceinline__ void prefix_unit_tc(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                            const PrefixParams &p, int c, int kvh, int g) {
+    using Geo = PrefixTcGeometry<D, CB>;
+    constexpr int kKeys = Geo::kKeys;
+    constexpr int kColS = 0, kColO = kKeys;  // TMEM columns
+    constexpr uint32_t kIdS = tc::idesc_bf16(128, kKeys, 0);
+    constexpr uint32_t kIdO = tc::idesc_bf16(128, D, 1);
+    const int t = threadIdx.x, warp = t >> 5;
+
+    const int off = __ldg(p.group_offsets + g);
+    const int members = __ldg(p.group_offsets + g + 1) - off;
+    if (members <= 0) return;
+    const int b0 = __ldg(p.group_seqs + off);
+    if (b0 < 0 || b0 >= p.B) {
+        if (t == 0) flag(p.err, PKV_DEV_ERR_BAD_LEN);
+        return;
+    }
+    int len0 = __ldg(p.seq_lens + b0);
+    len0 = len0 < 0 ? 0 : min(len0, p.W * kBlockTokens);
+    const int nb = min(max(__ldg(p.prefix_blocks + b0), 0), len0 / kBlockTokens);  // full blocks
+    const int j0 = c * CB, j1 = min(nb, j0 + CB);
+    if (j0 >= j1) return;
+    const int nt = j1 - j0;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t k_smem = smem_u32(smem), v_smem = smem_u32(smem + Geo::kKV);
+    const uint32_t k_bar = smem_u32(smem + 2 * Geo::kKV);  // K landed
+    const uint32_t v_bar = k_bar + 8;                       // V landed
+    const uint32_t m_bar = k_bar + 16;                      // the MMAs issued so far are done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 2 * Geo::kKV + 24);
+    int *valid = reinterpret_cast<int *>(smem + 2 * Geo::kKV + 32);  // [CB]
+
+    if (t == 0) {
+        mbar_init(k_bar, 1);
+        mbar_init(v_bar, 1);
+        mbar_init(m_bar, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+        const int32_t *row = p.block_tables + static_cast<size_t>(b0) * p.W;
+        const int y_none = static_cast<int>(p.num_blocks * p.Hkv * kBlockTokens);  // past the tensor: zeros
+        int y[CB];
+#pragma unroll
+        for (int i = 0; i < CB; ++i) {
+            valid[i] = -1;
+            y[i] = y_none;
+            if (i < nt) {
+                const int32_t phys = __ldg(row + j0 + i);
+                if (phys >= 0 && phys < p.num_blocks) {
+                    valid[i] = phys;
+                    y[i] = (phys * p.Hkv + kvh) * kBlockTokens;
+                } else {
+                    flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
+                }
+            }
+        }
+        const uint64_t policy = l2_policy_evict_first();
+        // [d half][key][128 B]: key k of half hh at hh * 128 keys * 128 B + k * 128 B
+        mbar_arrive_expect_tx(k_bar, Geo::kKV);
+#pragma unroll
+        for (int i = 0; i < CB; ++i)
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh)
+                tma_load_2d(k_smem + hh * (kKeys * 128) + i * (kBlockTokens * 128), &tmk, hh * 64, y[i], k_bar,
+                            policy);
+        mbar_arrive_expect_tx(v_bar, Geo::kKV);
+#pragma unroll
+        for (int i = 0; i < CB; ++i)
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh)
+                tma_load_2d(v_smem + hh * (kKeys * 128) + i * (kBlockTokens * 128), &tmv, hh * 64, y[i], v_bar,
+                            policy);
+    }
+    if (warp == 1) tc::alloc<Geo::kTmemCols>(smem_u32(tmem_slot));  // beside thread 0's TMA issue
+    tc::fence_before();
+    __syncthreads();  // barriers, valid[] and the TMEM base
+    tc::fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // this thread's lane
+    uint32_t keep = 0;  // bit i: block i of the chunk is there
+#pragma unroll
+    for (int i = 0; i < CB; ++i) keep |= (valid[i] >= 0 ? 1u : 0u) << i;
+
+    const int G = p.group;      // query heads per KV head
+    const int R = members * G;  // rows of this group and KV head
+    bool ok = true;
+    bool mma_pending = false;   // an MMA batch committed to m_bar and not yet seen done
+    uint32_t phase = 0;         // m_bar phase
+    for (int r0 = 0; r0 < R; r0 += 128) {
+        const int r = r0 + t;
+        int b = -1, h = 0;
+        if (r < R) {
+            const int bb = __ldg(p.group_seqs + off + r / G);
+            if (bb >= 0 && bb < p.B) {
+                b = bb;
+                h = kvh * G + r % G;
+            }
+        }
+        // Q row -> TMEM columns [kColO, kColO + D / 2), zeros for rows without
+        // a sequence; all of the row's loads in flight before the stores
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.q + (static_cast<size_t>(b < 0 ? 0 : b) * p.Hq + h) * D);
+            uint32_t w[D / 2];
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                const uint4 v = b >= 0 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+                w[4 * i] = v.x;
+                w[4 * i + 1] = v.y;
+                w[4 * i + 2] = v.z;
+                w[4 * i + 3] = v.w;
+            }
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) tc::st32(lane_base + kColO + 32 * cc, w + 32 * cc);
+            tc::wait_st();
+        }
+        tc::fence_before();
+        const bool k_ok = r0 > 0 || mbar_wait(k_bar, 0, kWaitLimitNs);
+        if (__syncthreads_or(!k_ok)) {
+            ok = false;
+            break;
+        }
+        tc::fence_after();
+        if (t == 0) {  // S = Q K^T
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+                tc::mma_ts(tmem + kColS, tmem + kColO + 8 * k,
+                           tc::smem_desc(k_smem + (k >> 2) * (kKeys * 128) + (k & 3) * 32, 16, 1024), kIdS, k > 0);
+            tc::commit(m_bar);
+        }
+        mma_pending = true;
+        if (__syncthreads_or(!mbar_wait(m_bar, phase, kWaitLimitNs))) {
+            ok = false;
+            break;
+        }
+        mma_pending = false;
+        phase ^= 1;
+        tc::fence_after();
+
+        // softmax of the row, two passes over S (64 columns at a time): max, then P
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // one chain per block of 16
+#pragma unroll 1
+        for (int hf = 0; hf < kKeys / 64; ++hf) {
+            uint32_t s[64];
+            tc::ld32(lane_base + kColS + 64 * hf, s);
+            tc::ld32(lane_base + kColS + 64 * hf + 32, s + 32);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+                if (keep >> (4 * hf + i / kBlockTokens) & 1u)
+                    mx4[i / kBlockTokens] = fmaxf(mx4[i / kBlockTokens], __uint_as_float(s[i]) * p.scale_log2);
+        }
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float nbase = mx == -INFINITY ? 0.f : mx;
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int hf = 0; hf < kKeys / 64; ++hf) {
+            uint32_t s[64];
+            tc::ld32(lane_base + kColS + 64 * hf, s);
+            tc::ld32(lane_base + kColS + 64 * hf + 32, s + 32);
+            tc::wait_ld();
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+                const bool there = keep >> (4 * hf + i / kBlockTokens) & 1u;  // i, i + 1: one block
+                const float p0 = there ? ex2_approx(fmaf(__uint_as_float(s[i]), p.scale_log2, -nbase)) : 0.f;
+                const float p1 = there ? ex2_approx(fmaf(__uint_as_float(s[i + 1]), p.scale_log2, -nbase)) : 0.f;
+                l4[i / kBlockTokens] += p0 + p1;
+                pk[i / 2] = pack_bf16x2(p0, p1);
+            }
+            tc::st32(lane_base + kColS + 32 * hf, pk);  // P columns over S columns already read
+        }
+        const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        tc::wait_st();
+        tc::fence_before();
+        const bool v_ok = r0 > 0 || mbar_wait(v_bar, 0, kWaitLimitNs);
+        if (__syncthreads_or(!v_ok)) {
+            ok = false;
+            break;
+        }
+        tc::fence_after();
+        if (t == 0) {  // O = P V (V MN-major: d contiguous)
+#pragma unroll
+            for (int k = 0; k < kKeys / 16; ++k)
+                tc::mma_ts(tmem + kColO, tmem + kColS + 8 * k,
+                           tc::smem_desc(v_smem + k * (16 * 128), kKeys * 128, 1024), kIdO, k > 0);
+            tc::commit(m_bar);
+        }
+        mma_pending = true;
+        if (__syncthreads_or(!mbar_wait(m_bar, phase, kWaitLimitNs))) {
+            ok = false;
+            break;
+        }
+        mma_pending = false;
+        phase ^= 1;
+        tc::fence_after();
+
+        // the row's partial for chunk c
+        const size_t slot = (static_cast<size_t>(b < 0 ? 0 : b) * p.Hq + h) * p.ws_parts + c;
+        if (b >= 0) {
+            p.ws_ml[2 * slot] = mx;
+            p.ws_ml[2 * slot + 1] = l;
+        }
+        if (R <= 128) {
+            // The only row tile: K and V are no longer read, so the rows go
+            // through their shared memory ([row][D floats], 16-byte chunk j of
+            // row t at j ^ (t % chunks per row)) and each warp then writes its
+            // lanes' rows whole, one 16-byte chunk per lane.
+            constexpr int kChunks = D / 4;  // 16-byte chunks of a row
+            float4 *stage = reinterpret_cast<float4 *>(smem);
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tc::ld32(lane_base + kColO + 32 * cc, o);
+                tc::wait_ld();
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    stage[t * kChunks + ((8 * cc + i) ^ (t & (kChunks - 1)))] =
+                        make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                    __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            }
+            __syncwarp();  // a warp writes out its own lanes' rows
+            const int lane = t & 31;
+#pragma unroll 1
+            for (int i = 0; i < 32; ++i) {
+                const int rr = 32 * warp + i;
+                const unsigned long long rslot = __shfl_sync(0xffffffffu, static_cast<unsigned long long>(slot), i);
+                if (!__shfl_sync(0xffffffffu, b >= 0, i)) continue;
+                float4 *rdst = reinterpret_cast<float4 *>(p.ws_o + rslot * D);
+                for (int j = lane; j < kChunks; j += 32)
+                    rdst[j] = stage[rr * kChunks + (j ^ (rr & (kChunks - 1)))];
+            }
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(p.ws_o + slot * D);
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tc::ld32(lane_base + kColO + 32 * cc, o);
+                tc::wait_ld();
+                if (b >= 0) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[8 * cc + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                                      __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                }
+            }
+        }
+    }
+    if (!ok && t == 0) {
+        flag(p.err, PKV_DEV_ERR_TIMEOUT);
+        if (mma_pending) mbar_wait(m_bar, phase, kWaitLimitNs);  // the batch still running
+    }
+    if (t == 0) {  // copies still landing (done already unless a wait gave up)
+        mbar_wait(k_bar, 0, kWaitLimitNs);
+        mbar_wait(v_bar, 0, kWaitLimitNs);
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (warp == 1) tc::dealloc<Geo::kTmemCols>(tmem);
+}
+
 // Merge of one (sequence, query head): prefix chunks [0, ceil(pb / CB)) and
 // the suffix split-K partitions that hold tokens past the prefix (counted
 // from the prefix end), in slot order, by log-sum-exp.  As in the split-K
@@ -321,8 +612,8 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
 // evenly through the grid, so that every SM runs the short, latency-bound
 // prefix work beside the bandwidth-bound suffix stream; the other CTAs take
 // suffix units in order (partition fastest, then head segment, then
-// sequence).
-template <int D, bool MMA>
+// sequence).  TC: the prefix chunks on tcgen05 (else mma.sync).
+template <int D, bool MMA, bool TC>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const PrefixParams pp, const DecodeParams dp, int n_pre) {
@@ -333,9 +624,17 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
         id /= stride;
         const int c = id % pp.prefix_parts;
         id /= pp.prefix_parts;
-        prefix_unit<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
+        if constexpr (TC)
+            prefix_unit_tc<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
+        else
+            prefix_unit_mma<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
         return;
     }
+    // Suffix units use no TMEM: they give up the right to allocate at once.
+    // A CTA that keeps it (until it exits) holds up the TMEM allocation of a
+    // prefix CTA that starts after it on the same SM (measured: the step took
+    // twice as long).
+    if (TC && n_pre > 0 && threadIdx.x < 32) tc::relinquish();
     if (n_pre > 0) id -= min(id / stride + 1, n_pre);  // prefix CTAs at or before this one
     const int ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
     const int part = id % dp.num_parts;
@@ -352,14 +651,13 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
     decode_unit<D, kPrefixWarps, 2, MMA, true>(tmk, tmv, dp, part, id % ny, b);
 }
 
-template <int D, bool MMA>
+template <int D, bool MMA, bool TC>
 cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                              const DecodeParams &dp, int num_groups, cudaStream_t stream) {
-    constexpr int kSmem = PrefixGeometry<D, kPrefixChunkBlocks>::kSmemBytes >
-                                  Geometry<D, kPrefixWarps, 2>::kSmemBytes
-                              ? PrefixGeometry<D, kPrefixChunkBlocks>::kSmemBytes
-                              : Geometry<D, kPrefixWarps, 2>::kSmemBytes;
-    auto kern = cascade_kernel<D, MMA>;
+    constexpr int kPre = TC ? PrefixTcGeometry<D, kPrefixChunkBlocks>::kSmemBytes
+                            : PrefixMmaGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
+    constexpr int kSmem = std::max(kPre, Geometry<D, kPrefixWarps, 2>::kSmemBytes);
+    auto kern = cascade_kernel<D, MMA, TC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const long long n_pre = static_cast<long long>(pp.prefix_parts) * pp.Hkv * num_groups;
@@ -374,18 +672,24 @@ cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, con
                             stream, pp);
 }
 
+template <int D>
+cudaError_t launch_cascade_h(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
+                             const DecodeParams &dp, int num_groups, bool prefix_tc, cudaStream_t stream) {
+    const bool mma = dp.group > 1;
+    if (prefix_tc)
+        return mma ? launch_cascade_d<D, true, true>(tmk, tmv, pp, dp, num_groups, stream)
+                   : launch_cascade_d<D, false, true>(tmk, tmv, pp, dp, num_groups, stream);
+    return mma ? launch_cascade_d<D, true, false>(tmk, tmv, pp, dp, num_groups, stream)
+               : launch_cascade_d<D, false, false>(tmk, tmv, pp, dp, num_groups, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
-                           const DecodeParams &dp, int head_dim, int num_groups,
+                           const DecodeParams &dp, int head_dim, int num_groups, bool prefix_tc,
                            cudaStream_t stream) {
-    const bool mma = dp.group > 1;
-    if (head_dim == 128)
-        return mma ? launch_cascade_d<128, true>(tmk, tmv, pp, dp, num_groups, stream)
-                   : launch_cascade_d<128, false>(tmk, tmv, pp, dp, num_groups, stream);
-    if (head_dim == 64)
-        return mma ? launch_cascade_d<64, true>(tmk, tmv, pp, dp, num_groups, stream)
-                   : launch_cascade_d<64, false>(tmk, tmv, pp, dp, num_groups, stream);
+    if (head_dim == 128) return launch_cascade_h<128>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
+    if (head_dim == 64) return launch_cascade_h<64>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -41,11 +41,26 @@ CASES = [
                     num_heads=16, num_kv_heads=2)),
     ("prefix", dict(batch=40, prefix_len=16, suffix_lo=1, suffix_hi=20)),   # one shared block
     ("prefix", dict(batch=5, prefix_len=48, suffix_lo=1, suffix_hi=1)),     # suffix = new token
+    # more than 128 rows per (group, KV head): several row tiles, the last one ragged
+    ("prefix", dict(batch=40, prefix_len=272, suffix_lo=1, suffix_hi=40, num_heads=28,
+                    num_kv_heads=4)),                                        # 280 rows, chunks 8+8+1
+    ("prefix", dict(batch=33, prefix_len=144, suffix_lo=1, suffix_hi=30, head_dim=64,
+                    num_heads=8, num_kv_heads=2)),                           # 132 rows, d 64
 ]
 
 
+@pytest.fixture(params=["mma_sync", "tcgen05"])
+def prefix_impl(request, monkeypatch):
+    """The prefix chunks on warp-level mma.sync (default) or on tcgen05/TMEM."""
+    if request.param == "tcgen05":
+        monkeypatch.setenv("PKV_CASCADE_TC", "1")
+    else:
+        monkeypatch.delenv("PKV_CASCADE_TC", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("name,kw", CASES, ids=[str(i) for i in range(len(CASES))])
-def test_cascade_matches_oracle(name, kw):
+def test_cascade_matches_oracle(name, kw, prefix_impl):
     w = build(name, 13, **kw)
     d = DeviceStep(w)
     d.write()
@@ -68,7 +83,7 @@ def test_cascade_suffix_bound_too_small_is_flagged():
     assert d.err_word() & 4
 
 
-def test_cascade_full_size_sampled():
+def test_cascade_full_size_sampled(prefix_impl):
     w = build("prefix", 0)
     d = DeviceStep(w)
     d.write()
@@ -83,7 +98,7 @@ def test_cascade_full_size_sampled():
     assert d.err_word() == 0
 
 
-def test_cascade_block_relabelling_is_bit_exact():
+def test_cascade_block_relabelling_is_bit_exact(prefix_impl):
     w = build("prefix", 14, batch=10, prefix_len=256, suffix_lo=1, suffix_hi=80, prefix_groups=2)
     d = DeviceStep(w)
     d.write()
@@ -98,7 +113,7 @@ def test_cascade_block_relabelling_is_bit_exact():
 
 
 @pytest.mark.parametrize("idx", [0, 1, 2, 3])
-def test_cascade_fused_step(idx):
+def test_cascade_fused_step(idx, prefix_impl):
     """pkv_paged_decode_prefix_step: the step's write fused into the cascade --
     caches bit-exact with the oracle's write, output within tolerance, and
     bit-identical to the separate write + cascade."""
