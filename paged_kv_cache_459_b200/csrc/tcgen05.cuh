@@ -50,10 +50,11 @@ __device__ __forceinline__ void fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Whole warp: gives up this CTA's right to allocate.  A CTA keeps that right
-// until it gives it up or exits, and while it keeps it another CTA's
-// allocation on the SM waits; a CTA that never allocates gives it up at
-// once.  (No tcgen05.alloc may follow in the same CTA.)
+// Whole warp: gives up this CTA's right to allocate (no tcgen05.alloc may
+// follow in the same CTA).  A CTA keeps that right until it gives it up or
+// exits, and a later CTA's allocation on the same SM can wait for it
+// (measured: the cascade step took twice as long until its CTAs that never
+// allocate gave the right up at entry).
 __device__ __forceinline__ void relinquish() {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
