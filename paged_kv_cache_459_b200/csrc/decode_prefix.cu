@@ -9,9 +9,10 @@
 //   rows = (member, query head of this KV head) pairs, 16 per warp tile,
 //   S[16 rows x 16 tokens] = Q . K_blk^T  and  O[16 x d] += P . V_blk
 // on mma.m16n8k16 (bf16 in, fp32 accumulate) -- with 128 members this is a
-// 128-row tile per KV head, a real dense contraction.  Each CTA takes a chunk
-// of CB prefix blocks, loads its K and V tiles once with TMA, and leaves one
-// partial (m, l, o) per row.  The private suffixes go through the split-K
+// 128-row tile per KV head, a real dense contraction.  (The same chunk runs
+// on tcgen05 with TMEM accumulators when selected: prefix_unit_tc below.)
+// Each CTA takes a chunk of CB prefix blocks, loads its K and V tiles once
+// with TMA, and leaves one partial (m, l, o) per row.  The private suffixes go through the split-K
 // kernel starting past the prefix, and the merge below combines prefix and
 // suffix partials of each (sequence, query head) by log-sum-exp.  The result
 // equals plain decode over the whole sequence.
