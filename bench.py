@@ -444,13 +444,15 @@ def run_gpu(args):
                    "decode_us": 1e3 * statistics.fmean(e[1].elapsed_time(e[2]) for e in uev),
                    "total_ms": sum(e[0].elapsed_time(e[2]) for e in uev)}
     prefix_tc = None
-    if args.cascade and fused:  # the same step with the prefix chunks on tcgen05 (opt-in path)
+    if args.cascade and fused:  # the prefix chunks on mma.sync (default) and on tcgen05, one loop each
+        prefix_tc = {"default_step_us": 1e3 * _events_time(step, K, Wm)}
         os.environ["PKV_CASCADE_TC"] = "1"
         try:
-            prefix_tc = {"step_us": 1e3 * _events_time(step, K, Wm),
-                         "how": "PKV_CASCADE_TC=1: prefix chunks on tcgen05/TMEM, same step, events"}
+            prefix_tc["step_us"] = 1e3 * _events_time(step, K, Wm)
         finally:
             os.environ.pop("PKV_CASCADE_TC")
+        prefix_tc["how"] = ("K steps back to back between two events, mma.sync prefix chunks "
+                            "(default_step_us) then PKV_CASCADE_TC=1 (step_us)")
     # keep the GPU loaded long enough for the clock sampler to see it
     if sampler is not None:
         t0 = time.perf_counter()
