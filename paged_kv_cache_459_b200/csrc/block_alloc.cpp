@@ -16,7 +16,6 @@
 #include <deque>
 #include <new>
 #include <unordered_map>
-#include <unordered_set>
 #include <vector>
 
 #include "../../include/pkv.h"
@@ -31,7 +30,13 @@ struct Sequence {
     std::vector<int32_t> blocks;  // GPU blocks, or host slots while swapped out
     int64_t len = 0;
     bool swapped = false;
+    uint64_t mark = 0;  // the batch call that last named it (duplicate check)
 };
+
+// What appending one token to a sequence takes: room in its last block, a
+// fresh block (none yet, or the last one is full), or a copy-on-write of a
+// partly filled last block that other tables also hold.
+enum class AppendKind : uint8_t { kInPlace, kNewBlock, kCopyOnWrite };
 
 }  // namespace
 
@@ -47,6 +52,10 @@ struct pkv_alloc {
     std::deque<int32_t> host_free;
     int64_t num_host_blocks = 0;
     std::vector<std::pair<int32_t, int32_t>> pending_out, pending_in;
+    // Scratch of the batch append, kept between calls (no allocation per step).
+    uint64_t epoch = 0;
+    std::vector<Sequence *> batch_seqs;
+    std::vector<AppendKind> batch_kinds;
 };
 
 extern "C" {
@@ -121,11 +130,6 @@ pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, int64_t n
     return PKV_OK;
 }
 
-// What appending one token to a sequence takes: room in its last block, a
-// fresh block (none yet, or the last one is full), or a copy-on-write of a
-// partly filled last block that other tables also hold.
-enum class AppendKind { kInPlace, kNewBlock, kCopyOnWrite };
-
 static AppendKind append_kind(const Sequence &s, int32_t last_refcount) {
     if (s.len % kBlockTokens == 0) return AppendKind::kNewBlock;
     return last_refcount > 1 ? AppendKind::kCopyOnWrite : AppendKind::kInPlace;
@@ -168,23 +172,31 @@ pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_ou
 
 pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *slots_out) {
     if (!a || n < 0 || (n > 0 && (!seq_ids || !slots_out))) return PKV_ERR_INVALID_ARG;
-    std::vector<Sequence *> seqs;
-    std::vector<AppendKind> kinds;
+    std::vector<Sequence *> &seqs = a->batch_seqs;
+    std::vector<AppendKind> &kinds = a->batch_kinds;
+    seqs.clear();
+    kinds.clear();
+    // a sequence named twice in one call is an error: each sequence carries
+    // the number of the last call that named it
+    const uint64_t epoch = ++a->epoch;
     try {
-        std::unordered_set<int64_t> seen;
         std::unordered_map<int32_t, int32_t> released;  // copy-on-writes earlier in this batch
         seqs.reserve(static_cast<size_t>(n));
         kinds.reserve(static_cast<size_t>(n));
         int64_t new_blocks = 0, cows = 0;
         for (int i = 0; i < n; ++i) {
-            if (!seen.insert(seq_ids[i]).second) return PKV_ERR_INVALID_ARG;
             auto it = a->seqs.find(seq_ids[i]);
             if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
             Sequence &s = it->second;
+            if (s.mark == epoch) return PKV_ERR_INVALID_ARG;
+            s.mark = epoch;
             int32_t rc = 0;
             if (!s.blocks.empty()) {
-                auto r = released.find(s.blocks.back());
-                rc = a->refcount[s.blocks.back()] - (r == released.end() ? 0 : r->second);
+                rc = a->refcount[s.blocks.back()];
+                if (!released.empty()) {
+                    auto r = released.find(s.blocks.back());
+                    if (r != released.end()) rc -= r->second;
+                }
             }
             const AppendKind kind = append_kind(s, rc);
             if (kind == AppendKind::kNewBlock) s.blocks.reserve(s.blocks.size() + 1);
@@ -344,17 +356,32 @@ pkv_status pkv_alloc_export(const pkv_alloc *a, const int64_t *seq_ids, int n, i
                             int32_t *tables_out, int32_t *lens_out) {
     if (!a || n < 0 || width <= 0 || (n > 0 && (!seq_ids || !tables_out || !lens_out)))
         return PKV_ERR_INVALID_ARG;
+    // every sequence checked before any row is written, each looked up once
+    // (the lookups of up to kStack sequences kept on the stack)
+    constexpr int kStack = 256;
+    const Sequence *stack_buf[kStack];
+    std::vector<const Sequence *> heap_buf;
+    const Sequence **found = stack_buf;
+    if (n > kStack) {
+        try {
+            heap_buf.resize(static_cast<size_t>(n));
+        } catch (const std::bad_alloc &) {
+            return PKV_ERR_OOM;
+        }
+        found = heap_buf.data();
+    }
     for (int i = 0; i < n; ++i) {
         auto it = a->seqs.find(seq_ids[i]);
         if (it == a->seqs.end() || it->second.swapped) return PKV_ERR_INVALID_ARG;
         if (static_cast<int64_t>(it->second.blocks.size()) > width || it->second.len > INT32_MAX)
             return PKV_ERR_INVALID_ARG;
+        found[i] = &it->second;
     }
     for (int i = 0; i < n; ++i) {
-        const Sequence &s = a->seqs.find(seq_ids[i])->second;
+        const Sequence &s = *found[i];
         int32_t *row = tables_out + static_cast<size_t>(i) * width;
-        std::fill(row, row + width, -1);
         std::copy(s.blocks.begin(), s.blocks.end(), row);
+        std::fill(row + s.blocks.size(), row + width, -1);
         lens_out[i] = static_cast<int32_t>(s.len);
     }
     return PKV_OK;
