@@ -714,10 +714,26 @@ def run_alloc_row(args):
         alloc.append_tokens(ids)
         alloc.export(ids, width)
     el = time.perf_counter() - t0
+    # the same steps for an engine that keeps its host tables: append_tokens_into
+    # patches the entries a step changes in the exported tables
+    alloc2 = pkv.BlockAllocator(need + 64, wl.rng(args.seed + 1).permutation(need + 64))
+    for b, n in enumerate(lens):
+        alloc2.add_seq(b, int(n))
+    ids_np = np.arange(B, dtype=np.int64)
+    tables, lens_h = alloc2.export(ids_np, width)
+    for _ in range(warm):
+        alloc2.append_tokens_into(ids_np, tables, lens_h)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        alloc2.append_tokens_into(ids_np, tables, lens_h)
+    el_into = time.perf_counter() - t0
     print(json.dumps({"row": "alloc", "steps": steps, "warmup": warm, "data": "synthetic",
                       "metric": "host allocator time per decode step (append one token to every "
                                 "sequence, export tables and lengths)",
                       "value": 1e6 * el / steps, "unit": "us", "higher_is_better": False,
+                      "append_into_us": 1e6 * el_into / steps,
+                      "append_into": "pkv_alloc_append_tokens_into on kept host tables (only the "
+                                     "changed entries written)",
                       "config": {"workload": f"{B} sequences, lengths U[{cfg['len_lo']},"
                                              f"{cfg['len_hi']}], table width {width}",
                                  "threads": 1}}), flush=True)

@@ -400,6 +400,19 @@ PKV_API pkv_status pkv_alloc_extend(pkv_alloc *a, int64_t seq_id, int64_t n, int
 PKV_API pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n,
                                    int64_t *slots_out);
 
+/* pkv_alloc_append_tokens that also updates the caller's host copy of the
+ * tables in place, for an engine that keeps them between steps: tables_io
+ * [n][width] and lens_io [n] must hold what pkv_alloc_export gave for the same
+ * seq_ids in the same order (and width) before this call, with nothing else
+ * changed since.  Only the entries the step changes are written: each
+ * sequence's last table entry (a new block, or the private copy that replaces
+ * a shared one) and its length; a step costs O(n) instead of O(n * width).
+ * A sequence whose blocks would pass width is rejected (INVALID_ARG); on any
+ * error nothing changes, tables_io and lens_io included. */
+PKV_API pkv_status pkv_alloc_append_tokens_into(pkv_alloc *a, const int64_t *seq_ids, int n,
+                                                int64_t *slots_out, int width, int32_t *tables_io,
+                                                int32_t *lens_io);
+
 /* Takes the queued copy-on-write pairs: *n_out = their number; if cap >= it,
  * src_out[i] -> dst_out[i] are filled (host arrays) and the queue is emptied;
  * otherwise nothing is taken (call again with room for *n_out). */

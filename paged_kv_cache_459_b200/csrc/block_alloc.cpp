@@ -170,8 +170,11 @@ pkv_status pkv_alloc_append_token(pkv_alloc *a, int64_t seq_id, int64_t *slot_ou
     return PKV_OK;
 }
 
-pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *slots_out) {
-    if (!a || n < 0 || (n > 0 && (!seq_ids || !slots_out))) return PKV_ERR_INVALID_ARG;
+// One token for each of n distinct sequences, all or none.  With a table
+// (width > 0), every sequence must keep its blocks within width, and row i of
+// tables_io / lens_io[i] get the entry and length the append changed.
+static pkv_status append_batch(pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *slots_out,
+                               int width, int32_t *tables_io, int32_t *lens_io) {
     std::vector<Sequence *> &seqs = a->batch_seqs;
     std::vector<AppendKind> &kinds = a->batch_kinds;
     seqs.clear();
@@ -199,6 +202,9 @@ pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, 
                 }
             }
             const AppendKind kind = append_kind(s, rc);
+            if (tables_io && (s.len >= INT32_MAX ||
+                              static_cast<int64_t>(s.blocks.size()) + (kind == AppendKind::kNewBlock) > width))
+                return PKV_ERR_INVALID_ARG;
             if (kind == AppendKind::kNewBlock) s.blocks.reserve(s.blocks.size() + 1);
             if (kind == AppendKind::kCopyOnWrite) {
                 released[s.blocks.back()] += 1;
@@ -214,7 +220,28 @@ pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, 
         return PKV_ERR_OOM;
     }
     for (int i = 0; i < n; ++i) slots_out[i] = do_append(a, *seqs[i], kinds[i]);
+    if (tables_io) {
+        for (int i = 0; i < n; ++i) {
+            const Sequence &s = *seqs[i];
+            // the last entry is the only one an append changes (a new block, or
+            // the private copy that replaces a shared one)
+            tables_io[static_cast<size_t>(i) * width + s.blocks.size() - 1] = s.blocks.back();
+            lens_io[i] = static_cast<int32_t>(s.len);
+        }
+    }
     return PKV_OK;
+}
+
+pkv_status pkv_alloc_append_tokens(pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *slots_out) {
+    if (!a || n < 0 || (n > 0 && (!seq_ids || !slots_out))) return PKV_ERR_INVALID_ARG;
+    return append_batch(a, seq_ids, n, slots_out, 0, nullptr, nullptr);
+}
+
+pkv_status pkv_alloc_append_tokens_into(pkv_alloc *a, const int64_t *seq_ids, int n, int64_t *slots_out,
+                                        int width, int32_t *tables_io, int32_t *lens_io) {
+    if (!a || n < 0 || width <= 0 || (n > 0 && (!seq_ids || !slots_out || !tables_io || !lens_io)))
+        return PKV_ERR_INVALID_ARG;
+    return append_batch(a, seq_ids, n, slots_out, width, tables_io, lens_io);
 }
 
 pkv_status pkv_alloc_extend(pkv_alloc *a, int64_t seq_id, int64_t n, int64_t *slots_out) {

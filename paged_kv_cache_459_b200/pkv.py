@@ -57,6 +57,7 @@ _sigs = {
     "pkv_alloc_fork": ([_P, _i64, _i64, _i64], _i32),
     "pkv_alloc_append_token": ([_P, _i64, _P], _i32),
     "pkv_alloc_append_tokens": ([_P, _P, _i32, _P], _i32),
+    "pkv_alloc_append_tokens_into": ([_P, _P, _i32, _P, _i32, _P, _P], _i32),
     "pkv_alloc_free_seq": ([_P, _i64], _i32),
     "pkv_alloc_export": ([_P, _P, _i32, _i32, _P, _P], _i32),
     "pkv_alloc_stats": ([_P, _P, _P, _P, _P], _i32),
@@ -406,6 +407,16 @@ class AllocError(PkvError):
         return {ERR_OOM: "oom", ERR_UNSUPPORTED: "unsupported"}.get(self.code, "invalid")
 
 
+def _addr(a: np.ndarray) -> int:
+    """Address of a C-contiguous array's data: the per-step allocator calls
+    take it this way (about half the cost of a.ctypes.data), falling back to
+    a.ctypes.data for read-only or empty arrays."""
+    try:
+        return ctypes.addressof(ctypes.c_char.from_buffer(a))
+    except (TypeError, ValueError, BufferError):
+        return a.ctypes.data
+
+
 def _acheck(code: int, what: str) -> None:
     if code != OK:
         raise AllocError(code, what)
@@ -455,8 +466,26 @@ class BlockAllocator:
     def append_tokens(self, seq_ids) -> np.ndarray:
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
         out = np.empty(len(ids), dtype=np.int64)
-        _acheck(_lib.pkv_alloc_append_tokens(self._h, ids.ctypes.data, len(ids), out.ctypes.data),
+        _acheck(_lib.pkv_alloc_append_tokens(self._h, _addr(ids), len(ids), _addr(out)),
                 "append_tokens")
+        return out
+
+    def append_tokens_into(self, seq_ids, tables: np.ndarray, lens: np.ndarray) -> np.ndarray:
+        """append_tokens, with the host tables / lengths that export() gave for
+        the same seq_ids updated in place (only the entries the step changes)."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = len(ids)
+        if (not isinstance(tables, np.ndarray) or tables.dtype != np.int32 or tables.ndim != 2
+                or tables.shape[0] != n or tables.shape[1] < 1 or not tables.flags.c_contiguous
+                or not tables.flags.writeable or not isinstance(lens, np.ndarray)
+                or lens.dtype != np.int32 or lens.shape != (n,) or not lens.flags.c_contiguous
+                or not lens.flags.writeable):
+            raise AllocError(ERR_INVALID_ARG, "append_tokens_into: tables int32 [n][width] and "
+                                              "lens int32 [n], C-contiguous and writeable")
+        out = np.empty(n, dtype=np.int64)
+        _acheck(_lib.pkv_alloc_append_tokens_into(self._h, _addr(ids), n, _addr(out),
+                                                  int(tables.shape[1]), _addr(tables), _addr(lens)),
+                "append_tokens_into")
         return out
 
     def free_seq(self, seq_id: int) -> None:
@@ -466,8 +495,8 @@ class BlockAllocator:
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
         tables = np.empty((len(ids), width), dtype=np.int32)
         lens = np.empty(len(ids), dtype=np.int32)
-        _acheck(_lib.pkv_alloc_export(self._h, ids.ctypes.data, len(ids), int(width),
-                                      tables.ctypes.data, lens.ctypes.data), "export")
+        _acheck(_lib.pkv_alloc_export(self._h, _addr(ids), len(ids), int(width), _addr(tables),
+                                      _addr(lens)), "export")
         return tables, lens
 
     def stats(self):

@@ -149,6 +149,68 @@ def test_failures_change_nothing():
         BlockAllocator(3, [0, 1, 1])
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_append_into_keeps_the_host_tables_equal_to_export(seed):
+    """The in-place batch append against a twin allocator driven by the plain
+    batch append: the same slots and copy-on-write pairs, and the caller's
+    tables and lengths equal to a fresh export after every step."""
+    gen = np.random.default_rng(100 + seed)
+    nb, width = 800, 40
+    order = gen.permutation(nb)
+    a, b = BlockAllocator(nb, order), BlockAllocator(nb, order)
+    ids = list(range(6))
+    for s in ids:
+        n = int(gen.integers(0, 60))
+        a.add_seq(s, n)
+        b.add_seq(s, n)
+    tables, lens = a.export(ids, width)
+    next_id, cows = len(ids), 0
+    for step in range(200):
+        if gen.random() < 0.06:  # a fork, often mid-block: the child's next append copies
+            p = int(gen.choice(ids))
+            n = int(gen.integers(0, a.seq_len(p) + 1))
+            a.fork(p, next_id, n)
+            b.fork(p, next_id, n)
+            ids.append(next_id)
+            next_id += 1
+            tables, lens = a.export(ids, width)  # a new set of sequences: export again
+        sa = a.append_tokens_into(ids, tables, lens)
+        sb = b.append_tokens(ids)
+        assert sa.tolist() == sb.tolist(), step
+        ca, cb = a.take_copies(), b.take_copies()
+        assert all(np.array_equal(x, y) for x, y in zip(ca, cb)), step
+        cows += len(ca[0])
+        t2, l2 = a.export(ids, width)
+        assert np.array_equal(tables, t2) and np.array_equal(lens, l2), step
+    assert cows > 0 and len(ids) > 6
+
+
+def test_append_into_errors_change_nothing():
+    a = BlockAllocator(8)
+    a.add_seq(0, 32)  # two full blocks: its next token needs a third
+    a.add_seq(1, 5)
+    tables, lens = a.export([0, 1], 2)
+    keep = (tables.copy(), lens.copy(), a.free_blocks())
+    for call in (lambda: a.append_tokens_into([0, 1], tables, lens),   # 0 would pass width 2
+                 lambda: a.append_tokens_into([1, 1], tables, lens),   # named twice
+                 lambda: a.append_tokens_into([1, 7], tables, lens),   # unknown sequence
+                 lambda: a.append_tokens_into([0], tables, lens),      # rows != sequences
+                 lambda: a.append_tokens_into([0, 1], tables.astype(np.int64), lens),
+                 lambda: a.append_tokens_into([0, 1], tables[:, :1], lens)):  # not contiguous
+        with pytest.raises(AllocError):
+            call()
+        assert np.array_equal(tables, keep[0]) and np.array_equal(lens, keep[1])
+        assert a.free_blocks() == keep[2]
+    b = BlockAllocator(2)
+    b.add_seq(0, 16)
+    b.add_seq(1, 16)  # both blocks full, the pool empty
+    t, ln = b.export([0, 1], 4)
+    k = (t.copy(), ln.copy())
+    with pytest.raises(AllocError) as e:
+        b.append_tokens_into([0, 1], t, ln)
+    assert e.value.kind == "oom" and np.array_equal(t, k[0]) and np.array_equal(ln, k[1])
+
+
 @pytest.mark.parametrize("name,kw", [("tiny", {}), ("llama", {}), ("qwen", {}), ("prefix", {}),
                                      ("long", {})])
 def test_workload_tables_match_model(name, kw):
