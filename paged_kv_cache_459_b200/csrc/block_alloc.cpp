@@ -8,12 +8,13 @@
 // returned when the request finishes).  Reference counts reconcile sharing
 // with release: a block goes back to the pool when its last holder lets go.
 //
-// The free list is a deque: blocks are taken from the front and returned to
-// the back, starting from a caller-given permutation, so tables are
-// reproducible for a seed.  Every call validates first and mutates only once
-// it cannot fail, so an error leaves the state unchanged.
+// The free list is a first-in first-out queue: blocks are taken from the
+// front and returned to the back, starting from a caller-given permutation, so
+// tables are reproducible for a seed.  Every call validates first and mutates
+// only once it cannot fail, so an error leaves the state unchanged; the free
+// lists are rings sized once for the whole pool, so returning blocks never
+// allocates.
 #include <algorithm>
-#include <deque>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -38,18 +39,45 @@ struct Sequence {
 // partly filled last block that other tables also hold.
 enum class AppendKind : uint8_t { kInPlace, kNewBlock, kCopyOnWrite };
 
+// Fixed-capacity FIFO of block (or host slot) ids.  A pool never has more
+// free entries than entries, so the ring is sized once (init, which may
+// throw) and push_back never allocates.
+class BlockFifo {
+public:
+    void init(size_t capacity) {
+        buf_.assign(std::max<size_t>(capacity, 1), 0);
+        head_ = size_ = 0;
+    }
+    size_t size() const { return size_; }
+    bool empty() const { return size_ == 0; }
+    int32_t front() const { return buf_[head_]; }
+    int32_t operator[](size_t i) const { return buf_[(head_ + i) % buf_.size()]; }
+    void pop_front() {
+        head_ = (head_ + 1) % buf_.size();
+        --size_;
+    }
+    void push_back(int32_t v) {  // the caller keeps size() below the capacity
+        buf_[(head_ + size_) % buf_.size()] = v;
+        ++size_;
+    }
+
+private:
+    std::vector<int32_t> buf_;
+    size_t head_ = 0, size_ = 0;
+};
+
 }  // namespace
 
 struct pkv_alloc {
     int64_t num_blocks = 0;
-    std::deque<int32_t> free_list;
+    BlockFifo free_list;  // capacity num_blocks
     std::vector<int32_t> refcount;
     std::unordered_map<int64_t, Sequence> seqs;
     // Copy-on-write block copies (src, dst) not yet taken by the caller.
     std::vector<std::pair<int32_t, int32_t>> pending_copies;
     // Host swap space: free host block slots, and queued moves (GPU block,
     // host slot) out of and into the GPU pool.
-    std::deque<int32_t> host_free;
+    BlockFifo host_free;  // capacity num_host_blocks
     int64_t num_host_blocks = 0;
     std::vector<std::pair<int32_t, int32_t>> pending_out, pending_in;
     // Scratch of the batch append, kept between calls (no allocation per step).
@@ -57,6 +85,10 @@ struct pkv_alloc {
     std::vector<Sequence *> batch_seqs;
     std::vector<AppendKind> batch_kinds;
 };
+
+static pkv_status prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, int n,
+                                int32_t *prefix_blocks_out, int32_t *group_offsets_out,
+                                int32_t *group_seqs_out, int32_t *num_groups_out);
 
 extern "C" {
 
@@ -68,6 +100,8 @@ pkv_status pkv_alloc_create(int64_t num_blocks, const int64_t *free_order, pkv_a
     try {
         a->num_blocks = num_blocks;
         a->refcount.assign(static_cast<size_t>(num_blocks), 0);
+        a->free_list.init(static_cast<size_t>(num_blocks));
+        a->host_free.init(0);
         if (free_order) {
             std::vector<char> seen(static_cast<size_t>(num_blocks), 0);
             for (int64_t i = 0; i < num_blocks; ++i) {
@@ -118,15 +152,16 @@ pkv_status pkv_alloc_fork(pkv_alloc *a, int64_t parent, int64_t child, int64_t n
     if (it == a->seqs.end() || it->second.swapped || a->seqs.count(child)) return PKV_ERR_INVALID_ARG;
     int64_t n = num_tokens < 0 ? it->second.len : num_tokens;
     if (n > it->second.len) return PKV_ERR_INVALID_ARG;
+    Sequence *made = nullptr;
     try {
         Sequence s;
         s.len = n;
         s.blocks.assign(it->second.blocks.begin(), it->second.blocks.begin() + blocks_for(n));
-        for (int32_t b : s.blocks) a->refcount[b] += 1;
-        a->seqs.emplace(child, std::move(s));
+        made = &a->seqs.emplace(child, std::move(s)).first->second;  // may rehash: `it` is stale after
     } catch (const std::bad_alloc &) {
         return PKV_ERR_OOM;
     }
+    for (int32_t b : made->blocks) a->refcount[b] += 1;  // only once the child exists
     return PKV_OK;
 }
 
@@ -300,9 +335,10 @@ pkv_status pkv_alloc_set_host_pool(pkv_alloc *a, int64_t num_host_blocks) {
     for (const auto &kv : a->seqs)
         if (kv.second.swapped) return PKV_ERR_INVALID_ARG;  // host slots in use
     try {
-        std::deque<int32_t> fresh;
+        BlockFifo fresh;
+        fresh.init(static_cast<size_t>(num_host_blocks));
         for (int64_t i = 0; i < num_host_blocks; ++i) fresh.push_back(static_cast<int32_t>(i));
-        a->host_free.swap(fresh);
+        a->host_free = std::move(fresh);
     } catch (const std::bad_alloc &) {
         return PKV_ERR_OOM;
     }
@@ -423,7 +459,12 @@ pkv_status pkv_alloc_stats(const pkv_alloc *a, int64_t *free_blocks, int64_t *us
     for (int32_t r : a->refcount) shared += r > 1;
     double util = 0.0;
     if (used > 0) {
-        std::vector<int16_t> fill(static_cast<size_t>(a->num_blocks), 0);
+        std::vector<int16_t> fill;
+        try {
+            fill.assign(static_cast<size_t>(a->num_blocks), 0);
+        } catch (const std::bad_alloc &) {
+            return PKV_ERR_OOM;
+        }
         for (const auto &kv : a->seqs) {
             const Sequence &s = kv.second;
             if (s.swapped) continue;
@@ -459,6 +500,19 @@ pkv_status pkv_alloc_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, i
     if (!a || n < 0 || !num_groups_out ||
         (n > 0 && (!seq_ids || !prefix_blocks_out || !group_offsets_out || !group_seqs_out)))
         return PKV_ERR_INVALID_ARG;
+    try {
+        return prefix_groups(a, seq_ids, n, prefix_blocks_out, group_offsets_out, group_seqs_out,
+                             num_groups_out);
+    } catch (const std::bad_alloc &) {  // before any output is written
+        return PKV_ERR_OOM;
+    }
+}
+
+}  // extern "C"
+
+static pkv_status prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, int n,
+                                int32_t *prefix_blocks_out, int32_t *group_offsets_out,
+                                int32_t *group_seqs_out, int32_t *num_groups_out) {
     std::vector<const Sequence *> seqs(static_cast<size_t>(n));
     for (int i = 0; i < n; ++i) {
         auto it = a->seqs.find(seq_ids[i]);
@@ -503,6 +557,8 @@ pkv_status pkv_alloc_prefix_groups(const pkv_alloc *a, const int64_t *seq_ids, i
     *num_groups_out = groups;
     return PKV_OK;
 }
+
+extern "C" {
 
 pkv_status pkv_alloc_refcount(const pkv_alloc *a, int64_t block, int32_t *out) {
     if (!a || !out || block < 0 || block >= a->num_blocks) return PKV_ERR_INVALID_ARG;
