@@ -68,7 +68,7 @@ def parse_args():
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 256 MB buffer between timed steps (automatic when the "
                          "step's K/V fit in L2) and time the step from per-step events")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     return ap.parse_args()
 
@@ -247,6 +247,7 @@ def cpu_baseline(w, budget_s: float) -> dict:
     """Bounded sample of the oracle on this host: about `budget_s` seconds on
     all the process's cores, then about a quarter of that on one thread."""
     st = OracleStep(w)
+    st.seconds_per_seq()  # the first call pays page faults and cold caches
     per_seq = st.seconds_per_seq()
     b = w.cfg["batch"]
     nseq = int(min(b, max(1, budget_s / 3 / per_seq)))
