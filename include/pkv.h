@@ -171,6 +171,10 @@ PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *q, const vo
  * length chosen by the caller.  partition_tokens: a multiple of 16 in
  * [16, 65536] (used by PKV_DECODE_SPLIT only).  PKV_DECODE_SPLIT or
  * PKV_DECODE_STREAM without enough workspace returns PKV_ERR_WORKSPACE.
+ * For tuning sweeps, the environment variables PKV_DECODE_WARPS and
+ * PKV_DECODE_STAGES (read at each call) pick the decode CTA shape of the
+ * single-pass and split-K kernels: 4 warps x 2 ring stages (the default,
+ * measured fastest), 4 x 3 or 2 x 2; other values give the default.
  */
 PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,

@@ -95,3 +95,15 @@ def test_recorded_ncu_commands_leave_the_clocks_alone():
                 found += 1
                 assert "--clock-control none" in line, f"{md.name}: {line.strip()}"
     assert found > 0
+
+
+def test_every_environment_switch_is_documented():
+    """Each environment variable the library reads is described in the public
+    header (the kernels it selects, their defaults)."""
+    header = (ROOT / "include" / "pkv.h").read_text()
+    names = set()
+    for path in SOURCES:
+        names |= set(re.findall(r'(?:env_int|getenv)\(\s*"([A-Z0-9_]+)"', _code(path)))
+    assert names, "no environment switch found"
+    missing = sorted(n for n in names if n not in header)
+    assert not missing, missing
