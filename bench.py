@@ -269,7 +269,7 @@ def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     from oracle.alloc_model import BlockManager
-    from paged_kv_cache_459_b200 import workloads as wl
+    import workloads as wl
     w = wl.build(args.config, args.seed, BlockManager)
     st = OracleStep(w)
     per_seq = st.seconds_per_seq()
@@ -313,7 +313,7 @@ def run_gpu(args):
                                 device_id=dev)
 
     from paged_kv_cache_459_b200 import pkv
-    from paged_kv_cache_459_b200 import workloads as wl
+    import workloads as wl
 
     w = wl.build(args.config, args.seed + rank, pkv.BlockAllocator, batch=args.batch)
     cfg = w.cfg
@@ -694,7 +694,7 @@ def run_alloc_row(args):
     every sequence of the workload, then the tables and lengths exported), on
     the CPU: what the engine pays before each decode call."""
     from paged_kv_cache_459_b200 import pkv
-    from paged_kv_cache_459_b200 import workloads as wl
+    import workloads as wl
 
     cfg = wl.config("qwen" if args.config == "qwen" else "llama")
     B = cfg["batch"]
@@ -748,7 +748,7 @@ def run_row(args):
         return run_alloc_row(args)
     import torch
     from paged_kv_cache_459_b200 import pkv
-    from paged_kv_cache_459_b200 import workloads as wl
+    import workloads as wl
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)

@@ -152,9 +152,13 @@ PKV_API int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads
  * head_dim: 64 or 128.  num_heads % num_kv_heads == 0.  Pointers 16-byte
  * aligned.  num_blocks * num_kv_heads * 16 must be < 2^31.
  * This entry point takes PKV_DECODE_AUTO with 512-token partitions: split-K
- * when a sequence may span more than one partition, the single-pass grid
- * would be short of CTAs (fewer than ~4 waves) and `workspace` holds
- * pkv_decode_workspace_bytes(...) bytes; the single-pass variant otherwise.
+ * when a sequence may span more than one partition, `workspace` holds
+ * pkv_decode_workspace_bytes(...) bytes, and the single-pass grid would be
+ * short of CTAs -- its (sequence, KV head [, group of 8 query heads]) units
+ * fill fewer than 1.5 waves at 3 CTAs per SM when the workspace also holds
+ * the longest-first order (pkv_decode_workspace_bytes_for(PKV_DECODE_SINGLE,
+ * ...) bytes), fewer than 4 waves without it; the single-pass variant
+ * otherwise.  pkv_decode_variant_for() reports the choice.
  * The workspace is scratch owned by the caller; calls that share one
  * workspace must be ordered on the GPU (the same stream, or events).
  */

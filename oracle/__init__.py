@@ -2,9 +2,9 @@
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg may import this package.  It shares no code with
-the CUDA library (``paged_kv_cache_459_b200``) and never imports it; the only
-common module is the seeded input generator, which holds no attention
-arithmetic.
+the CUDA library package and never imports it; the only module both sides use
+is the seeded input generator (``workloads.py`` at the repository root), which
+holds no attention arithmetic and imports neither side.
 
 * ``paged_decode``          -- softmax(scale * q K^T) V per (sequence, query head),
                                K and V gathered through the block table (C, fp64).

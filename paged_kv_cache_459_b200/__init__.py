@@ -2,12 +2,11 @@
 
 The compute path lives in ``libpkv.so`` (CUDA for sm_100a plus the host block
 allocator, behind the C ABI declared in ``include/pkv.h``).  ``pkv`` is the
-thin ctypes binding over it; it is imported lazily so that the seeded input
-generator (``workloads``) can be used without loading the CUDA library.
+thin ctypes binding over it, imported on first use.
 """
 from importlib import import_module as _import_module
 
-__all__ = ["pkv", "workloads"]
+__all__ = ["pkv"]
 
 
 def __getattr__(name):

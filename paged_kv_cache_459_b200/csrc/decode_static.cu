@@ -18,6 +18,7 @@
 #include <mutex>
 
 #include "../../include/pkv.h"
+#include "internal.h"
 
 namespace {
 
@@ -29,27 +30,33 @@ constexpr int kMaxDevices = 64;
 // reads no other partition.
 __device__ __align__(256) unsigned char pkv_static_scratch[PKV_STATIC_SCRATCH_BYTES];
 
+// The array's device address on each device, set only by a successful
+// lookup: a failed one (e.g. an error left behind by an unrelated earlier
+// launch) is retried by the next call instead of disabling the entry point.
 struct ScratchSlot {
-    std::once_flag once;
-    cudaError_t status = cudaErrorNotReady;
+    std::mutex lock;
     void *addr = nullptr;
 };
 ScratchSlot g_slots[kMaxDevices];
 
-// Device address of the scratch array on the current device; the first call
-// on a device does the lookup.
+// Device address of the scratch array on the current device; the first
+// successful call on a device does the lookup.
 cudaError_t scratch_address(void **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     ScratchSlot &s = g_slots[dev];
-    std::call_once(s.once, [&s] {
-        s.status = cudaGetSymbolAddress(&s.addr, pkv_static_scratch);
-        if (s.status != cudaSuccess) s.addr = nullptr;
-    });
+    std::lock_guard<std::mutex> guard(s.lock);
+    if (s.addr == nullptr) {
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, pkv_static_scratch);
+        if (e != cudaSuccess) return e;
+        if (addr == nullptr) return cudaErrorInvalidSymbol;
+        s.addr = addr;
+    }
     *out = s.addr;
-    return s.status;
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -70,7 +77,8 @@ pkv_status pkv_paged_attention_decode_static(void *out, const void *q, const voi
     if (need == 0) return PKV_ERR_INVALID_ARG;
     if (need > static_cast<size_t>(PKV_STATIC_SCRATCH_BYTES)) return PKV_ERR_WORKSPACE;
     void *scratch = nullptr;
-    if (scratch_address(&scratch) != cudaSuccess || scratch == nullptr) return PKV_ERR_CUDA;
+    const cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess) return static_cast<pkv_status>(pkv::cuda_status(e));
     return pkv_paged_attention_decode_ex(out, q, k_cache, v_cache, block_tables,
                                          max_blocks_per_seq, seq_lens, num_seqs, num_heads,
                                          num_kv_heads, head_dim, num_blocks, scale,

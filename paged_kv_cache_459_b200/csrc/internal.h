@@ -11,6 +11,10 @@ namespace pkv {
 
 constexpr int kBlockTokens = 16;
 
+// Maps a CUDA error to PKV_ERR_CUDA (PKV_OK for cudaSuccess) and records it
+// as the calling thread's last error for pkv_last_cuda_error().
+int cuda_status(cudaError_t e);
+
 struct DecodeParams {
     __nv_bfloat16 *out;           // [B][Hq][D]
     const __nv_bfloat16 *q;       // [B][Hq][D]

@@ -56,11 +56,7 @@ int env_int(const char *name, int fallback) {
 // The CUDA error behind the last PKV_ERR_CUDA returned on this thread.
 thread_local int g_last_cuda_error = 0;
 
-pkv_status cuda_status(cudaError_t e) {
-    if (e == cudaSuccess) return PKV_OK;
-    g_last_cuda_error = static_cast<int>(e);
-    return PKV_ERR_CUDA;
-}
+pkv_status cuda_status(cudaError_t e) { return static_cast<pkv_status>(pkv::cuda_status(e)); }
 
 // Streaming multiprocessors of the current device (148 on B200).
 int sm_count() {
@@ -77,6 +73,12 @@ int num_parts_for(int max_blocks_per_seq, int partition_tokens) {
 }
 
 }  // namespace
+
+int pkv::cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return PKV_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return PKV_ERR_CUDA;
+}
 
 extern "C" {
 

@@ -24,6 +24,7 @@
 #include <algorithm>
 
 #include "decode_common.cuh"
+#include "tcgen05.cuh"
 
 namespace pkv {
 
@@ -40,97 +41,6 @@ constexpr int kSoftmaxWarps = kTiles * kWarpsPerTile;
 constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-
-__device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    // start >> 4 [0,14), leading byte offset >> 4 [16,30), stride byte offset
-    // >> 4 [32,46), version 1 [46,48), layout 128-byte swizzle (2) [61,64)
-    return static_cast<uint64_t>((addr & 0x3FFFF) >> 4) |
-           (static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16) |
-           (static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, A K-major,
-// B K-major (b_mn = 0) or MN-major (b_mn = 1), N >> 3 at bit 17, M >> 4 at 24.
-__host__ __device__ constexpr uint32_t umma_idesc(int M, int N, int b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn) << 16) |
-           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                     bool accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(static_cast<int>(accumulate))
-        : "memory");
-}
-
-// The same with A read from tensor memory (K-major: row = lane, two 16-bit
-// elements per 32-bit column).
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                        bool accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b), "r"(idesc), "r"(static_cast<int>(accumulate))
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 32 lanes x 32 consecutive 32-bit TMEM columns: this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-        "%30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// The same without the wait: several loads may be in flight before one
-// tcgen05.wait::ld.
-__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t *r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-        "%30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
-        "%29, %30, %31, %32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-        "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
 
 // ------------------------------------------------ packed f32x2 arithmetic
 // Two floats in one 64-bit register pair for the sm_100 f32x2 instructions.
@@ -286,15 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmv);
     }
     if (warp == kMmaWarp) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(tmem_slot)),
-                     "n"(Geo::kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc::alloc<Geo::kTmemCols>(smem_u32(tmem_slot));
     }
-    tc_fence_before();
+    tc::fence_before();
     __syncthreads();
-    tc_fence_after();
+    tc::fence_after();
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kProducerWarp) {
@@ -381,25 +287,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // of TMEM; it overwrites P_x(j) (which aliases S_x) only after PV_x(j),
         // issued before it, has read it; and its completion tells the
         // softmax that PV_x(j) is done.
-        constexpr uint32_t kIdS = umma_idesc(kRows, kKeys, 0);
-        constexpr uint32_t kIdO = umma_idesc(kRows, D, 1);
+        constexpr uint32_t kIdS = tc::idesc_bf16(kRows, kKeys, 0);
+        constexpr uint32_t kIdO = tc::idesc_bf16(kRows, D, 1);
         const auto issue_s = [&](int x, int stage) {  // S_x = Q_x . K^T
             const uint32_t kbase = smem_u32(smem + Geo::kK + stage * Geo::kKVBytes);
             const uint32_t qbase = smem_u32(smem + Geo::kQ + x * Geo::kQBytes);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const int hh = k >> 2, kk = k & 3;
-                umma(tmem + kKeys * x, umma_desc(qbase + hh * (kRows * 128) + kk * 32, 16, 1024),
-                     umma_desc(kbase + hh * (kKeys * 128) + kk * 32, 16, 1024), kIdS, k > 0);
+                tc::mma_ss(tmem + kKeys * x, tc::smem_desc(qbase + hh * (kRows * 128) + kk * 32, 16, 1024),
+                     tc::smem_desc(kbase + hh * (kKeys * 128) + kk * 32, 16, 1024), kIdS, k > 0);
             }
-            umma_commit(s_full(x));
+            tc::commit(s_full(x));
         };
         const auto issue_pv = [&](int x, int stage, bool acc) {  // O_x (+)= P_x . V, P_x from TMEM
             const uint32_t vbase = smem_u32(smem + Geo::kV + stage * Geo::kKVBytes);
 #pragma unroll
             for (int k = 0; k < kKeys / 16; ++k)
-                umma_ts(tmem + Geo::kO + D * x, tmem + kKeys * x + 8 * k,
-                        umma_desc(vbase + k * (16 * 128), kKeys * 128, 1024), kIdO, acc || k > 0);
+                tc::mma_ts(tmem + Geo::kO + D * x, tmem + kKeys * x + 8 * k,
+                        tc::smem_desc(vbase + k * (16 * 128), kKeys * 128, 1024), kIdO, acc || k > 0);
         };
         bool ok = true;
         const auto wait = [&](uint32_t bar, uint32_t parity) {
@@ -427,11 +333,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int x = 0; x < kTiles; ++x) {
                 if (nk_t[x] == 0) continue;
                 wait(q_full(x), static_cast<uint32_t>(n_it & 1));
-                tc_fence_after();
+                tc::fence_after();
                 if (ok && lane == 0) issue_s(x, gk % KS);
                 __syncwarp();
             }
-            if (ok && lane == 0) umma_commit(k_empty(gk % KS));
+            if (ok && lane == 0) tc::commit(k_empty(gk % KS));
             __syncwarp();
             ++gk;
             for (int j = 0; j < nk && ok; ++j, ++gv) {
@@ -459,22 +365,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j >= nk_t[x]) continue;
                     wait(p_full(x), static_cast<uint32_t>(ns[x] & 1));
                     if (j == 0 && n_it > 0) wait(o_free(x), static_cast<uint32_t>((n_it - 1) & 1));
-                    tc_fence_after();
+                    tc::fence_after();
                     if (ok && lane == 0) {
                         issue_pv(x, sv, j > 0);
-                        if (x == last_v) umma_commit(v_empty(sv));
-                        if (j + 1 >= nk_t[x]) umma_commit(o_done(x));
+                        if (x == last_v) tc::commit(v_empty(sv));
+                        if (j + 1 >= nk_t[x]) tc::commit(o_done(x));
                     }
                     ++ns[x];
                     if (j + 1 < nk_t[x]) {
                         if (!next_ready) {
                             wait(k_full(gk % KS), static_cast<uint32_t>((gk / KS) & 1));
-                            tc_fence_after();
+                            tc::fence_after();
                             next_ready = true;
                         }
                         if (ok && lane == 0) {
                             issue_s(x, gk % KS);
-                            if (x == last_k) umma_commit(k_empty(gk % KS));
+                            if (x == last_k) tc::commit(k_empty(gk % KS));
                         }
                     }
                     __syncwarp();
@@ -486,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (nk_t[x] > 0) continue;
                 wait(q_full(x), static_cast<uint32_t>(n_it & 1));
                 if (n_it > 0) wait(o_free(x), static_cast<uint32_t>((n_it - 1) & 1));
-                if (ok && lane == 0) umma_commit(o_done(x));
+                if (ok && lane == 0) tc::commit(o_done(x));
                 __syncwarp();
             }
             k = kn;
@@ -545,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                tc_fence_after();
+                tc::fence_after();
                 // the last S product of this item has read Q_x: fetch the next item's rows
                 if (j + 1 == my_nk && kn >= 0) fetch_q(nx);
                 // Two passes over S in TMEM, 64 columns at a time, so that a row
@@ -557,9 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1  // one half's 64 registers live at a time
                 for (int h = 0; h < kKeys / 64; ++h) {
                     uint32_t sr[64];
-                    tmem_ld32_nowait(t_s + 64 * h, sr);
-                    tmem_ld32_nowait(t_s + 64 * h + 32, sr + 32);
-                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    tc::ld32(t_s + 64 * h, sr);
+                    tc::ld32(t_s + 64 * h + 32, sr + 32);
+                    tc::wait_ld();
                     // causal mask by position (only tiles that reach past some row need it)
                     if (masked) {
 #pragma unroll
@@ -585,9 +491,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1  // one half's 64 registers live at a time
                 for (int h = 0; h < kKeys / 64; ++h) {
                     uint32_t sr[64];
-                    tmem_ld32_nowait(t_s + 64 * h, sr);
-                    tmem_ld32_nowait(t_s + 64 * h + 32, sr + 32);
-                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    tc::ld32(t_s + 64 * h, sr);
+                    tc::ld32(t_s + 64 * h + 32, sr + 32);
+                    tc::wait_ld();
                     uint32_t pk[32];
                     if (masked) {  // diagonal tiles: -inf scores (2^-inf = 0)
 #pragma unroll
@@ -604,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
                         pk[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
                     }
-                    tmem_st32(t_s + 32 * h, pk);
+                    tc::st32(t_s + 32 * h, pk);
                 }
                 float s_lo, s_hi, s_lo2, s_hi2;
                 f2unpack(sum2[0], s_lo, s_hi);
@@ -616,18 +522,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int cc = 0; cc < D / 32; ++cc) {
                             uint32_t o[32];
-                            tmem_ld32(t_o + 32 * cc, o);
+                            tc::ld32(t_o + 32 * cc, o);
+                            tc::wait_ld();
 #pragma unroll
                             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                            tmem_st32(t_o + 32 * cc, o);
+                            tc::st32(t_o + 32 * cc, o);
                         }
                     }
                     l_run *= alpha;
                 }
                 l_run += rowsum;
                 m_run = m_new;
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                tc_fence_before();
+                tc::wait_st();
+                tc::fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full(tile));
                 // This tile's S products of the item are all done, so the tensor
@@ -640,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            tc_fence_after();
+            tc::fence_after();
             if (my_nk == 0 && kn >= 0) publish_q();  // after o_done: at most one phase ahead
             ++n_it;
             if (my_nk == 0) {
@@ -657,9 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int h = 0; h < D / 64; ++h) {
                 uint32_t o[64];
-                tmem_ld32_nowait(t_o + 64 * h, o);
-                tmem_ld32_nowait(t_o + 64 * h + 32, o + 32);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                tc::ld32(t_o + 64 * h, o);
+                tc::ld32(t_o + 64 * h + 32, o + 32);
+                tc::wait_ld();
                 if (row_pos >= 0) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -674,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            tc_fence_before();
+            tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(o_free(tile));
             it = nx;
@@ -687,13 +594,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.wait_all;" ::: "memory");
     }
     // everyone (the producer's copies included) is done with TMEM and shared memory
-    tc_fence_before();
+    tc::fence_before();
     __syncthreads();
-    tc_fence_after();
+    tc::fence_after();
     if (warp == kMmaWarp)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "n"(Geo::kTmemCols)
-                     : "memory");
+        tc::dealloc<Geo::kTmemCols>(tmem);
 }
 
 template <int D>

@@ -1,7 +1,7 @@
 // 5th-generation tensor core (tcgen05) and tensor memory (TMEM) helpers for
 // sm_100a: shared-memory matrix descriptors, the kind::f16 instruction
 // descriptor, MMA issue and commit, TMEM allocation, loads and stores.
-// Used by the shared-prefix decode; the prefill kernel carries its own copy.
+// Used by the shared-prefix decode and the prefill kernel.
 #pragma once
 
 #include <cstdint>
@@ -24,6 +24,17 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn) << 16) |
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D (TMEM) (+)= A (shared memory) x B (shared memory), both by descriptor.
+// Issued by one thread.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(static_cast<int>(accumulate))
+        : "memory");
 }
 
 // D (TMEM) (+)= A (TMEM, K-major: row = lane, two bf16 per 32-bit column) x B

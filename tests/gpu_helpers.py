@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from oracle.alloc_model import BlockManager
-from paged_kv_cache_459_b200 import workloads as wl
+import workloads as wl
 
 # Tolerance for bf16 attention outputs accumulated in fp32, against the fp64
 # oracle: an element passes when |gpu - ref| <= ATOL + RTOL * |ref|.

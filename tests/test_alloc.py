@@ -9,7 +9,7 @@ import pytest
 
 from oracle.alloc_model import AllocError as ModelError, BlockManager
 from paged_kv_cache_459_b200 import build as pkv_build
-from paged_kv_cache_459_b200 import workloads as wl
+import workloads as wl
 
 pkv_build.build()
 from paged_kv_cache_459_b200.pkv import AllocError, BlockAllocator  # noqa: E402

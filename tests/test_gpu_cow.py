@@ -16,7 +16,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 from paged_kv_cache_459_b200 import pkv  # noqa: E402
-from paged_kv_cache_459_b200 import workloads as wl  # noqa: E402
+import workloads as wl  # noqa: E402
 
 
 @pytest.mark.parametrize("hq,hkv,d,parent_len,beams", [(8, 8, 128, 1000, 4), (28, 4, 128, 77, 6),

@@ -16,7 +16,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 from paged_kv_cache_459_b200 import pkv  # noqa: E402
-from paged_kv_cache_459_b200 import workloads as wl  # noqa: E402
+import workloads as wl  # noqa: E402
 
 
 def capture(step):

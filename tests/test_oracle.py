@@ -17,7 +17,8 @@ import torch.nn.functional as F
 
 import oracle
 from oracle.alloc_model import BlockManager
-from paged_kv_cache_459_b200 import workloads as wl
+import workloads as wl
+from relabel import permute_pool
 
 BT = 16
 
@@ -267,7 +268,7 @@ def test_block_relabelling_invariance_is_bit_exact():
     base = oracle.paged_decode(w.q, kc, vc, w.block_tables, w.lens, w.cfg["scale"])
     for seed in range(3):
         perm = wl.rng(100 + seed).permutation(w.num_blocks)
-        t2, _, kc2, vc2 = wl.permute_pool(perm, w.block_tables, w.slot_mapping, kc, vc)
+        t2, _, kc2, vc2 = permute_pool(perm, w.block_tables, w.slot_mapping, kc, vc)
         out = oracle.paged_decode(w.q, kc2, vc2, t2, w.lens, w.cfg["scale"])
         assert np.array_equal(out, base)
 

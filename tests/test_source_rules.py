@@ -107,3 +107,37 @@ def test_every_environment_switch_is_documented():
     assert names, "no environment switch found"
     missing = sorted(n for n in names if n not in header)
     assert not missing, missing
+
+
+def _imports(path: pathlib.Path) -> set[str]:
+    """Top-level names of the modules a Python file imports."""
+    names = set()
+    for m in re.finditer(r"^\s*(?:from\s+([\w.]+)\s+import|import\s+([\w., ]+))", path.read_text(),
+                         flags=re.M):
+        if m.group(1):
+            names.add(m.group(1).split(".")[0])
+        else:
+            names |= {n.strip().split(" ")[0].split(".")[0] for n in m.group(2).split(",")}
+    return names
+
+
+def test_oracle_side_never_imports_the_library():
+    """The oracle and its pins share no code with the CUDA path: nothing under
+    oracle/, no oracle pin and not the input generator imports the library
+    package (the generator is a module of its own at the repository root)."""
+    files = sorted((ROOT / "oracle").glob("*.py")) + [ROOT / "tests" / "test_oracle.py",
+                                                        ROOT / "tests" / "relabel.py",
+                                                        ROOT / "workloads.py"]
+    for path in files:
+        assert "paged_kv_cache_459_b200" not in _imports(path), path.name
+        assert "paged_kv_cache_459_b200" not in path.read_text(), path.name
+    assert "oracle" not in _imports(ROOT / "workloads.py")
+
+
+def test_library_never_imports_the_oracle():
+    """No product file (the package's Python or C/CUDA sources) reaches oracle/."""
+    pkg = ROOT / "paged_kv_cache_459_b200"
+    for path in sorted(pkg.rglob("*.py")):
+        assert "oracle" not in _imports(path), path.name
+    for path in SOURCES:
+        assert "oracle" not in _code(path).lower(), path.name

@@ -4,15 +4,18 @@ may not allocate, a server that reserves all memory at start-up, code that
 avoids cudaMalloc/cudaFree because they can synchronise the device).  Its
 scratch is a fixed array inside the library instead of a caller workspace.
 
-Called through the C ABI and compared with the regular entry point
-(pkv_paged_attention_decode_ex, split-K, caller-owned workspace) on the same
-inputs, two calls in a row, with the tolerance of the parity tests.  This file
-sorts last so that a failure here comes after every other test has run."""
+Called through the C ABI on two calls in a row and compared with the regular
+entry point (pkv_paged_attention_decode_ex, split-K, same partition, caller-
+owned workspace): both run the same kernels on the same inputs, so the outputs
+must be the same bits -- a stale or misaddressed scratch would shift them.
+The output is also checked against the fp64 oracle with the tolerance of the
+parity tests, and the device's free memory must not change across a call.
+This file sorts last so that a failure here comes after every other test."""
 import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import ATOL, RTOL, DeviceStep, bits_to_f64, build, host_bits
+from gpu_helpers import DeviceStep, build, check_close, host_bits, oracle_after_write
 
 pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():
@@ -51,27 +54,32 @@ def call_regular(d: DeviceStep, partition=512):
     return rc, host_bits(d.out)
 
 
-def assert_match(got_bits, want_bits):
-    got, want = bits_to_f64(got_bits), bits_to_f64(want_bits)
-    assert np.isfinite(got).all() and np.isfinite(want).all()
-    assert np.all(np.abs(got - want) <= ATOL + RTOL * np.abs(want))
+CASES = [("qwen", 21, dict(batch=6, len_lo=1, len_hi=1500), 512),
+         ("llama", 22, dict(batch=5, len_lo=1, len_hi=900, head_dim=64), 64),
+         ("long", 24, dict(batch=2, len_fixed=3000, num_blocks=420), 128)]
 
 
-def test_static_scratch_matches_regular_entry_twice_in_a_row():
-    cases = [build("qwen", 21, batch=6, len_lo=1, len_hi=1500),
-             build("llama", 22, batch=5, len_lo=1, len_hi=900, head_dim=64)]
-    steps = [DeviceStep(w) for w in cases]
-    for d in steps:
-        d.write()
-    for d, part in ((steps[0], 512), (steps[1], 64)):
-        rc, want = call_regular(d, part)
+@pytest.mark.parametrize("name,seed,kw,part", CASES, ids=[c[0] for c in CASES])
+def test_static_scratch_matches_regular_entry_twice_in_a_row(name, seed, kw, part):
+    w = build(name, seed, **kw)
+    d = DeviceStep(w)
+    d.write()
+    _, _, ref = oracle_after_write(w)
+    rc, want = call_regular(d, part)
+    assert rc == pkv.OK
+    for call in range(2):  # the second call starts from the first call's scratch contents
+        d.out.fill_(float("nan"))
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
+        held_before = torch.cuda.memory_allocated()
+        rc, got = call_static(d, part)
         assert rc == pkv.OK
-        for _ in range(2):  # the second call starts from the first call's scratch contents
-            d.out.fill_(float("nan"))
-            rc, got = call_static(d, part)
-            assert rc == pkv.OK
-            assert_match(got, want)
-        assert d.err_word() == 0
+        assert np.array_equal(got, want), f"call {call}: differs from the regular split-K entry"
+        check_close(got, ref, f"static scratch {name}, call {call}")
+        if call == 1:  # the first call may load the library's kernels; later calls take nothing
+            assert torch.cuda.mem_get_info()[0] == free_before
+            assert torch.cuda.memory_allocated() == held_before
+    assert d.err_word() == 0
 
 
 def test_static_scratch_rejects_sizes_past_its_limit():

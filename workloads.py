@@ -5,7 +5,8 @@ the order of the free-block list, bf16 Q/K/V values and NaN poison.  It holds
 no attention arithmetic and no allocation policy.  Block tables and slots come
 from an allocator object that the caller passes in (the library's C++ block
 allocator, or the reference model under ``oracle/``), which is how both the
-CUDA path and the oracle are fed the same inputs without sharing code.
+CUDA path and the oracle are fed the same inputs without sharing code.  It
+sits outside both the library package and ``oracle/`` and imports neither.
 
 Workloads (the shapes come from the decode configurations this library is
 measured on):
@@ -235,19 +236,3 @@ def poison_cache(kc, vc, free_blocks, tables, lens, new_slots) -> None:
         if s >= 0:
             kc[s // BLOCK_TOKENS, :, s % BLOCK_TOKENS, :] = BF16_NAN
             vc[s // BLOCK_TOKENS, :, s % BLOCK_TOKENS, :] = BF16_NAN
-
-
-def permute_pool(perm: np.ndarray, tables: np.ndarray, slots: np.ndarray, *caches):
-    """Relabel physical blocks: block i moves to perm[i].  Returns the new
-    tables, slots and caches; the logical content of every sequence is
-    unchanged."""
-    perm = np.asarray(perm, dtype=np.int64)
-    t2 = np.where(tables >= 0, perm[np.clip(tables, 0, None)], tables).astype(np.int32)
-    s2 = np.where(slots >= 0, perm[np.clip(slots, 0, None) // BLOCK_TOKENS] * BLOCK_TOKENS
-                  + np.clip(slots, 0, None) % BLOCK_TOKENS, slots).astype(np.int64)
-    out = []
-    for c in caches:
-        c2 = np.empty_like(c)
-        c2[perm] = c
-        out.append(c2)
-    return (t2, s2, *out)
