@@ -2,13 +2,21 @@
 """Benchmark of the paged KV-cache decode step on B200.
 
 One step = the whole hot path over one batch: the cache write of every
-sequence's new token (pkv_paged_kv_write) and single-query decode attention
-over the paged cache (pkv_paged_attention_decode).  Block tables and slots
-come from the library's C++ block allocator; values are seeded synthetic bf16
-N(0,1) draws.  Prints ONE JSON line (rank 0).
+sequence's new token and single-query decode attention over the paged cache,
+in one library call (pkv_paged_decode_step; the write fused into the decode
+kernel).  Block tables and slots come from the library's C++ block
+allocator; values are seeded synthetic bf16 N(0,1) draws.  Prints ONE JSON
+line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config llama]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen]
     python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
+    python bench.py --row prefill|cow|swap|alloc   # the rows beside the decode step
+
+The headline workload is the Qwen2.5-7B-shaped GQA decode (batch 256, 28/4
+heads).  At N = 1 the same line also carries the Llama-2-7B-shaped and the
+long-context (8 x 32768, split-K) workloads, the shared-prefix cascade, a
+batch sweep and the paged prefill, each with its own roofline and clocks
+(--no-extras leaves them out).
 
 Multi-GPU (torchrun, one process per GPU): every rank decodes its own batch
 (seed + rank) -- independent problems, no collective on the data path -- and
@@ -51,11 +59,11 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
-    ap.add_argument("--config", choices=sorted(WORKLOAD_NAMES), default="llama")
+    ap.add_argument("--config", choices=sorted(WORKLOAD_NAMES), default="qwen")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for ncu captures)")
-    ap.add_argument("--variant", choices=["auto", "single", "split", "stream"], default="auto")
+    ap.add_argument("--variant", choices=["auto", "single", "split", "cluster"], default="auto")
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--row", choices=["decode", "prefill", "cow", "swap", "alloc"], default="decode",
                     help="which part of the path to measure (decode: the default step)")
@@ -70,6 +78,9 @@ def parse_args():
                          "step's K/V fit in L2) and time the step from per-step events")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="only the headline workload (no llama / long / cascade keys, batch "
+                         "sweep or prefill; these run by default at N = 1)")
     return ap.parse_args()
 
 
@@ -296,6 +307,341 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------- GPU path
+# The host keeps ahead of the device in every timed loop: a spin kernel
+# (torch.cuda._sleep) holds the stream while the first steps are enqueued, so
+# the per-step events see the step's own device time rather than gaps left by
+# the host issuing launches.  Spins sit outside the per-step events.
+SPIN_CYCLES_LEAD = 20_000_000   # ~10 ms at the B200's clocks
+SPIN_CYCLES_CHUNK = 4_000_000   # ~2 ms, before every FLUSH_CHUNK flushed steps
+FLUSH_CHUNK = 16
+
+
+class Resident:
+    """One decode workload resident on the GPU (caches, step inputs, tables,
+    workspace) with the step's library calls bound to it."""
+
+    def __init__(self, args, name: str, seed: int, dev, *, batch=None, cascade=False,
+                 variant="auto", partition=512, host_copies=False):
+        import torch
+
+        from paged_kv_cache_459_b200 import pkv
+        import workloads as wl
+
+        self.pkv, self.dev, self.name, self.cascade = pkv, dev, name, cascade
+        self.partition = partition
+        w = self.w = wl.build(name, seed, pkv.BlockAllocator, batch=batch)
+        cfg = w.cfg
+        self.B, self.hq, self.hkv, self.d = cfg["batch"], cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"]
+        self.scale = cfg["scale"]
+
+        def up(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+        q_h, k_h, v_h = (up(x) for x in (w.q, w.k_new, w.v_new))
+        tables_h = torch.from_numpy(w.block_tables)
+        lens_h = torch.from_numpy(w.lens.astype(np.int32))
+        slots_h = torch.from_numpy(w.slot_mapping)
+        if host_copies:  # pinned host inputs of the end-to-end loop
+            q_h, k_h, v_h, tables_h, lens_h, slots_h = (
+                t.pin_memory() for t in (q_h, k_h, v_h, tables_h, lens_h, slots_h))
+            self.host = {"q": q_h, "k": k_h, "v": v_h, "tables": tables_h, "lens": lens_h,
+                         "slots": slots_h}
+        self.kc = up(w.k_cache).to(dev)
+        self.vc = up(w.v_cache).to(dev)
+        if not host_copies:  # the device holds them now
+            w.k_cache = w.v_cache = None
+        self.q, self.k_new, self.v_new = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        self.tables, self.lens, self.slots = tables_h.to(dev), lens_h.to(dev), slots_h.to(dev)
+        self.out = torch.empty_like(self.q)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.variant = {"auto": pkv.DECODE_AUTO, "single": pkv.DECODE_SINGLE,
+                        "split": pkv.DECODE_SPLIT, "cluster": pkv.DECODE_CLUSTER}[variant]
+        W = self.W = w.block_tables.shape[1]
+        if cascade:
+            pb_h, offs_h, mem_h = w.alloc.prefix_groups(list(range(self.B)))
+            self.pb_h, self.offs_h, self.mem_h = pb_h, offs_h, mem_h
+            self.pb, self.offs_g, self.mem = (torch.from_numpy(x).to(dev) for x in (pb_h, offs_h, mem_h))
+            self.suffix_bound = pkv.suffix_blocks_bound(w.lens, pb_h)  # the allocator's host view
+            ws_bytes = pkv.decode_prefix_workspace_bytes(self.B, self.hq, self.d, W, partition)
+        else:
+            ws_bytes = pkv.decode_workspace_bytes_for(self.variant, self.B, self.hq, self.hkv,
+                                                      self.d, W, partition)
+        self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.chosen = self.variant if self.variant != pkv.DECODE_AUTO else pkv.decode_variant_for(
+            self.B, self.hq, self.hkv, self.d, W, partition, self.ws.numel())
+        self.parts = pkv.decode_cluster_parts_for(self.B, self.hq, self.hkv, self.d, W, self.variant,
+                                                  partition, self.ws.numel()) if not cascade else 0
+        self.fused = not args.unfused
+
+    # -- the library calls of one step
+    def write(self, c=None, o=None):
+        c = c or {"k": self.k_new, "v": self.v_new, "slots": self.slots}
+        self.pkv.paged_kv_write(c["k"], c["v"], self.kc, self.vc, c["slots"], err=self.err)
+
+    def decode(self, c=None, o=None):
+        c = c or {"q": self.q, "tables": self.tables, "lens": self.lens}
+        o = self.out if o is None else o
+        if self.cascade:
+            self.pkv.paged_attention_decode_prefix(
+                o, c["q"], self.kc, self.vc, c["tables"], c["lens"], self.scale, self.hkv, self.pb,
+                self.offs_g, self.mem, max_suffix_blocks=self.suffix_bound,
+                partition_tokens=self.partition, workspace=self.ws, err=self.err)
+        else:
+            self.pkv.paged_attention_decode(o, c["q"], self.kc, self.vc, c["tables"], c["lens"],
+                                            self.scale, self.hkv, variant=self.variant,
+                                            partition_tokens=self.partition, workspace=self.ws,
+                                            err=self.err)
+
+    def fused_step(self, c=None, o=None):
+        """The write of each sequence's new token fused into the decode kernel."""
+        c = c or {"q": self.q, "k": self.k_new, "v": self.v_new, "tables": self.tables,
+                  "lens": self.lens}
+        o = self.out if o is None else o
+        if self.cascade:
+            self.pkv.paged_decode_prefix_step(
+                o, c["q"], c["k"], c["v"], self.kc, self.vc, c["tables"], c["lens"], self.scale,
+                self.hkv, self.pb, self.offs_g, self.mem, max_suffix_blocks=self.suffix_bound,
+                partition_tokens=self.partition, workspace=self.ws, err=self.err)
+        else:
+            self.pkv.paged_decode_step(o, c["q"], c["k"], c["v"], self.kc, self.vc, c["tables"],
+                                       c["lens"], self.scale, self.hkv, variant=self.variant,
+                                       partition_tokens=self.partition, workspace=self.ws,
+                                       err=self.err)
+
+    def step(self, c=None, o=None):
+        if self.fused:
+            self.fused_step(c, o)
+        else:
+            self.write(c, o)
+            self.decode(c, o)
+
+    def two_calls(self):
+        self.write()
+        self.decode()
+
+    # -- accounting
+    def bytes(self) -> dict:
+        ab = algorithmic_bytes(self.w)
+        dec = ab["kv"] + ab["q"]
+        if self.cascade:
+            # what the cascade must read: each group's prefix once, every suffix once
+            w = self.w
+            uniq = int((np.asarray(w.lens, np.int64) - 16 * self.pb_h.astype(np.int64)).sum())
+            uniq += sum(16 * int(self.pb_h[self.mem_h[self.offs_h[g]]])
+                        for g in range(len(self.offs_h) - 1))
+            dec = uniq * self.hkv * self.d * 2 * 2 + ab["q"]
+        if self.fused:  # the new tokens' K/V: read once, written once
+            dec += 2 * self.B * self.hkv * self.d * 2 * 2
+        ab["decode"] = dec
+        return ab
+
+    def ordered(self) -> bool:
+        """Whether the decode runs its sequences longest first (an order kernel)."""
+        if self.cascade:
+            return False
+        if self.chosen == self.pkv.DECODE_CLUSTER:
+            return self.B >= 16 and self.ws.numel() >= (4 * self.B + 255) // 256 * 256
+        return self.chosen == self.pkv.DECODE_SINGLE and self.ws.numel() >= 4 * self.B
+
+    def launches_per_step(self) -> int:
+        pkv = self.pkv
+        if self.cascade:  # (write;) prefix chunks + suffix split-K in one launch, merge
+            return 2 if self.fused else 3
+        return (1 if self.fused else 2) + \
+            (1 if self.chosen == pkv.DECODE_SPLIT or self.ordered() else 0)
+
+    def variant_text(self) -> str:
+        pkv = self.pkv
+        if self.cascade:
+            return "shared-prefix cascade (prefix once per group x KV head, split-K suffixes, merge)"
+        return {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head, longest first)"
+                if self.ordered() else "single pass (one CTA per sequence x KV head)",
+                pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % self.partition,
+                pkv.DECODE_CLUSTER: f"cluster split ({self.parts} equal parts per sequence, one "
+                                    f"CTA each, merged in distributed shared memory" +
+                                    (", longest first)" if self.ordered() else ")"),
+                }[self.chosen]
+
+    def kernel_text(self) -> str:
+        pkv = self.pkv
+        if self.cascade:
+            return ("cascade_kernel (prefix chunks + suffix units" +
+                    (", fused write" if self.fused else "") + ") + cascade_merge_kernel")
+        return (("paged_decode_kernel with the fused write" if self.fused else "paged_decode_kernel")
+                + (" (cluster mode)" if self.chosen == pkv.DECODE_CLUSTER else "")
+                + (" + merge kernel" if self.chosen == pkv.DECODE_SPLIT else
+                   " + order kernel" if self.ordered() else ""))
+
+    def check_err(self, when: str):
+        import torch
+        torch.cuda.synchronize(self.dev)
+        if int(self.err.item()) != 0:
+            raise SystemExit(f"{self.name}: device error word {int(self.err.item())} {when}")
+
+
+def device_steps(step, K: int, dev, flush_buf=None):
+    """Device time of K calls of step(): per-step CUDA events (ms each) and the
+    whole loop (ms).  With flush_buf, L2 is flushed (a write larger than L2)
+    before every step, outside its events."""
+    import torch
+
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    torch.cuda._sleep(SPIN_CYCLES_LEAD)
+    t0.record(stream)
+    for i in range(K):
+        if flush_buf is not None:
+            if i and i % FLUSH_CHUNK == 0:
+                torch.cuda._sleep(SPIN_CYCLES_CHUNK)
+            flush_buf.zero_()  # L2 holds none of this step's inputs
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in ev], t0.elapsed_time(t1)
+
+
+def timed_decode(r: Resident, K: int, W: int, *, world: int, sampler=None, flush=None) -> dict:
+    """W warm-up steps, then K timed steps of the resident workload; returns the
+    line's numbers for it (and its clocks when a sampler runs)."""
+    import torch
+
+    for _ in range(W):
+        r.step()
+        if r.fused:
+            r.two_calls()
+    r.check_err("after warm-up")
+    ab = r.bytes()
+    if flush is None:
+        flush = ab["kv"] <= L2_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=r.dev) if flush else None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    per, loop_ms = device_steps(r.step, K, r.dev, flush_buf)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    total_ms = sum(per) if flush else loop_ms  # the flushes are not the step's work
+    clocks = None
+    if sampler is not None:  # keep the GPU loaded long enough for the sampler to see it
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 1.0:
+            for _ in range(50):
+                r.step()
+            torch.cuda.synchronize(r.dev)
+        clocks = sampler.stop()
+    r.check_err("after the timed steps")
+    total_ms = max_over_ranks([total_ms], device=r.dev)[0]
+    step_us = 1e3 * statistics.fmean(per)
+    peak, peak_kind = measured_peak_hbm()
+    achieved = ab["decode"] / (step_us * 1e-6) / 1e9
+    return {
+        "step_us": step_us, "total_ms": total_ms, "flush": flush, "bytes": ab,
+        "value": job_throughput(r.B, K, world, total_ms),
+        "kv_hbm_gbs": achieved,
+        "kv_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+        "kv_frac_of_measured_copy": achieved / peak,
+        "roofline": {
+            "bound": "hbm", "kernel": r.kernel_text(),
+            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_kind": peak_kind,
+            "traffic": committed_traffic("cascade_kernel" if r.cascade else "paged_decode_kernel",
+                                         ("prefix_cascade" if r.cascade else r.name)
+                                         if r.B == CONFIG_BATCH.get(r.name) else None),
+            "algorithmic_bytes_per_launch": ab["decode"],
+        },
+        "clocks": clocks,
+    }
+
+
+CONFIG_BATCH = {"tiny": 4, "llama": 64, "qwen": 256, "prefix": 128, "long": 8}
+
+
+def workload_key(args, name, *, dev, cascade=False, batch=None, clocks=True) -> dict:
+    """One extra workload of the bench line: the fused step timed like the
+    headline, its roofline against the measured copy rate, and its clocks."""
+    import torch
+
+    r = Resident(args, name, args.seed, dev, batch=batch, cascade=cascade)
+    sampler = ClockSampler(device_pci_id(dev)) if clocks else None
+    m = timed_decode(r, args.steps, max(3, args.warmup), world=1, sampler=sampler)
+    out = {
+        "workload": WORKLOAD_NAMES[name] if batch is None else
+        f"{WORKLOAD_NAMES[name]} (batch {r.B})",
+        "variant": r.variant_text(), "step": "fused write + decode (one call)" if r.fused else
+        "write, then decode", "tokens": m["bytes"]["tokens"],
+        "decode_us": m["step_us"], "value": m["value"], "unit": UNIT,
+        "kv_hbm_gbs": m["kv_hbm_gbs"], "kv_frac_of_8tbs": m["kv_frac_of_8tbs"],
+        "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
+        "l2": "flushed between steps (256 MB write), step time from per-step events"
+        if m["flush"] else "inputs larger than L2, no flush",
+        "roofline": m["roofline"], "gpu_launches": args.steps * r.launches_per_step(),
+    }
+    if clocks:
+        out["clocks"] = m["clocks"]
+    if cascade:
+        out["logical_kv_bytes"] = m["bytes"]["kv"]
+        out["unique_kv_bytes"] = m["bytes"]["decode"] - m["bytes"]["q"] - \
+            (2 * r.B * r.hkv * r.d * 2 * 2 if r.fused else 0)
+        # the prefix chunks on mma.sync (default) and on tcgen05, one loop each
+        cmp = {"default_step_us": 1e3 * _events_time(r.step, args.steps, 3)}
+        os.environ["PKV_CASCADE_TC"] = "1"
+        try:
+            cmp["tcgen05_step_us"] = 1e3 * _events_time(r.step, args.steps, 3)
+        finally:
+            os.environ.pop("PKV_CASCADE_TC")
+        os.environ["PKV_CASCADE_WIDE"] = "0"
+        try:
+            cmp["narrow_suffix_step_us"] = 1e3 * _events_time(r.step, args.steps, 3)
+        finally:
+            os.environ.pop("PKV_CASCADE_WIDE")
+        cmp["how"] = ("K steps back to back between two events: the default prefix chunks and "
+                      "suffix units, then PKV_CASCADE_TC=1 (tcgen05 prefix chunks), then "
+                      "PKV_CASCADE_WIDE=0 (one head segment per suffix CTA)")
+        out["prefix_paths"] = cmp
+    del r
+    torch.cuda.empty_cache()
+    return out
+
+
+def batch_sweep_key(args, dev) -> dict:
+    """Llama-2-7B-shaped decode at batch 1 .. 128 (the pages' own batch sweep
+    runs 1, 8, 32, 64, 128): small batches are latency-bound, large ones read
+    at the copy rate."""
+    import torch
+
+    rows = []
+    sampler = ClockSampler(device_pci_id(dev))
+    for B in (1, 8, 32, 64, 128):
+        r = Resident(args, "llama", args.seed, dev, batch=B)
+        m = timed_decode(r, args.steps, max(3, args.warmup), world=1)
+        rows.append({"batch": B, "variant": r.variant_text(), "decode_us": m["step_us"],
+                     "kv_hbm_gbs": m["kv_hbm_gbs"],
+                     "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
+                     "value": m["value"], "l2": "flushed" if m["flush"] else "larger than L2",
+                     "algorithmic_bytes_per_launch": m["bytes"]["decode"]})
+        last = r
+        if B != 128:
+            del r
+            torch.cuda.empty_cache()
+    t0 = time.perf_counter()  # the clock sampler sees the largest batch under load
+    while time.perf_counter() - t0 < 1.0:
+        for _ in range(20):
+            last.step()
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    del last
+    torch.cuda.empty_cache()
+    return {"workload": "Llama-2-7B-shaped MHA decode, 32/32 heads, d 128, len U[128,2048], "
+                        "fused write + decode step", "unit": UNIT, "rows": rows,
+            "clocks": clocks}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -312,164 +658,35 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    from paged_kv_cache_459_b200 import pkv
-    import workloads as wl
-
-    w = wl.build(args.config, args.seed + rank, pkv.BlockAllocator, batch=args.batch)
-    cfg = w.cfg
-    B, hq, hkv, d = cfg["batch"], cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"]
-
-    def up(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
-
-    q_h, k_h, v_h = (up(x).pin_memory() for x in (w.q, w.k_new, w.v_new))
-    tables_h = torch.from_numpy(w.block_tables).pin_memory()
-    lens_h = torch.from_numpy(w.lens.astype(np.int32)).pin_memory()
-    slots_h = torch.from_numpy(w.slot_mapping).pin_memory()
-    kc = up(w.k_cache).to(dev)
-    vc = up(w.v_cache).to(dev)
-    q, k_new, v_new = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    tables, lens, slots = tables_h.to(dev), lens_h.to(dev), slots_h.to(dev)
-    out = torch.empty_like(q)
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-    variant = {"auto": pkv.DECODE_AUTO, "single": pkv.DECODE_SINGLE, "split": pkv.DECODE_SPLIT,
-               "stream": pkv.DECODE_STREAM}[args.variant]
-    W = w.block_tables.shape[1]
-    ws_bytes = pkv.decode_workspace_bytes_for(variant, B, hq, hkv, d, W, args.partition)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    chosen = variant if variant != pkv.DECODE_AUTO else pkv.decode_variant_for(
-        B, hq, hkv, d, W, args.partition, ws.numel())
-    if args.cascade:
-        pb_h, offs_h, mem_h = w.alloc.prefix_groups(list(range(B)))
-        pb, offs_g, mem = (torch.from_numpy(x).to(dev) for x in (pb_h, offs_h, mem_h))
-        suffix_bound = pkv.suffix_blocks_bound(w.lens, pb_h)  # the allocator's host view
-        ws = torch.empty(pkv.decode_prefix_workspace_bytes(B, hq, d, W, args.partition),
-                         dtype=torch.uint8, device=dev)
-    scale = cfg["scale"]
-
-    def write():
-        pkv.paged_kv_write(k_new, v_new, kc, vc, slots, err=err)
-
-    def decode():
-        if args.cascade:
-            pkv.paged_attention_decode_prefix(out, q, kc, vc, tables, lens, scale, hkv, pb, offs_g, mem,
-                                              max_suffix_blocks=suffix_bound,
-                                              partition_tokens=args.partition, workspace=ws,
-                                              err=err)
-        else:
-            pkv.paged_attention_decode(out, q, kc, vc, tables, lens, scale, hkv, variant=variant,
-                                       partition_tokens=args.partition, workspace=ws, err=err)
-
-    # The step: the new token's K/V write fused into the decode kernel
-    # (pkv_paged_decode_step), or the write and the decode as two calls.
-    fused = not args.unfused and (args.cascade or chosen != pkv.DECODE_STREAM)
-
-    def fused_step(o=None, c=None):
-        c = c or {"q": q, "k": k_new, "v": v_new, "tables": tables, "lens": lens}
-        if args.cascade:
-            pkv.paged_decode_prefix_step(out if o is None else o, c["q"], c["k"], c["v"], kc, vc,
-                                         c["tables"], c["lens"], scale, hkv, pb, offs_g, mem,
-                                         max_suffix_blocks=suffix_bound,
-                                         partition_tokens=args.partition, workspace=ws, err=err)
-        else:
-            pkv.paged_decode_step(out if o is None else o, c["q"], c["k"], c["v"], kc, vc,
-                                  c["tables"], c["lens"], scale, hkv, variant=variant,
-                                  partition_tokens=args.partition, workspace=ws, err=err)
-
-    def step():
-        if fused:
-            fused_step()
-        else:
-            write()
-            decode()
-
-    stream = torch.cuda.current_stream(dev)
+    r = Resident(args, args.config, args.seed + rank, dev, batch=args.batch, cascade=args.cascade,
+                 variant=args.variant, partition=args.partition, host_copies=True)
+    B, hq, hkv, d, W = r.B, r.hq, r.hkv, r.d, r.W
     K, Wm = args.steps, args.warmup
-    for _ in range(Wm):
-        step()
-        if fused:
-            write()
-            decode()
-    torch.cuda.synchronize(dev)
-    if int(err.item()) != 0:
-        raise SystemExit(f"device error word {int(err.item())} after warm-up")
-
+    stream = torch.cuda.current_stream(dev)
     sampler = ClockSampler(device_pci_id(dev)) if rank == 0 else None
-    flush = args.flush_l2 or algorithmic_bytes(w)["kv"] <= L2_BYTES
-    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    t_start.record(stream)
-    for i in range(K):
-        if flush:
-            flush_buf.zero_()  # L2 holds none of this step's inputs
-        ev[i][0].record(stream)
-        if fused:
-            fused_step()
-        else:
-            write()
-            ev[i][1].record(stream)
-            decode()
-        ev[i][2].record(stream)
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    if flush:  # the flushes are not the step's work: sum the steps' own events
-        total_ms = sum(e[0].elapsed_time(e[2]) for e in ev)
-    if fused:  # one call: the decode kernel's time includes the write
-        write_ms = None
-        decode_ms = statistics.fmean(e[0].elapsed_time(e[2]) for e in ev)
-    else:
-        write_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
-        decode_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev)
+    m = timed_decode(r, K, Wm, world=world, sampler=sampler,
+                     flush=True if args.flush_l2 else None)
+    total_ms = m["total_ms"]
+    clocks = m["clocks"]
+    fused = r.fused
     unfused = None
-    if fused:  # the same step as two calls, for comparison
-        uev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-        torch.cuda.synchronize(dev)
-        for i in range(K):
-            if flush:
-                flush_buf.zero_()
-            uev[i][0].record(stream)
-            write()
-            uev[i][1].record(stream)
-            decode()
-            uev[i][2].record(stream)
-        torch.cuda.synchronize(dev)
-        unfused = {"write_us": 1e3 * statistics.fmean(e[0].elapsed_time(e[1]) for e in uev),
-                   "decode_us": 1e3 * statistics.fmean(e[1].elapsed_time(e[2]) for e in uev),
-                   "total_ms": sum(e[0].elapsed_time(e[2]) for e in uev)}
-    prefix_tc = None
-    if args.cascade and fused:  # the prefix chunks on mma.sync (default) and on tcgen05, one loop each
-        prefix_tc = {"default_step_us": 1e3 * _events_time(step, K, Wm)}
-        os.environ["PKV_CASCADE_TC"] = "1"
-        try:
-            prefix_tc["step_us"] = 1e3 * _events_time(step, K, Wm)
-        finally:
-            os.environ.pop("PKV_CASCADE_TC")
-        prefix_tc["how"] = ("K steps back to back between two events, mma.sync prefix chunks "
-                            "(default_step_us) then PKV_CASCADE_TC=1 (step_us)")
-    # keep the GPU loaded long enough for the clock sampler to see it
-    if sampler is not None:
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < 1.0:
-            for _ in range(50):
-                step()
-            torch.cuda.synchronize(dev)
-    clocks = sampler.stop() if sampler is not None else None
+    if fused:  # the same step as two calls (write, then decode), for comparison
+        flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if m["flush"] else None
+        uw, _ = device_steps(r.write, K, dev, flush_buf)  # the write call alone
+        per, loop = device_steps(r.two_calls, K, dev, flush_buf)
+        u_ms = max_over_ranks([sum(per) if m["flush"] else loop], device=dev)[0]
+        unfused = {"step_us": 1e3 * statistics.fmean(per), "write_us": 1e3 * statistics.fmean(uw),
+                   "value": job_throughput(B, K, world, u_ms),
+                   "how": "write + decode calls per step; write_us from a loop of the write alone"}
+        del flush_buf
 
     # End to end through the public API: every step's inputs (q, new K/V, tables, lengths,
     # slots) go host -> device from one pinned staging buffer, and its output comes back.
     # Two device input/output sets and a copy stream let step i+1's upload and step i's
     # download overlap step i's kernels.
-    parts = [("q", q_h), ("k", k_h), ("v", v_h), ("tables", tables_h), ("lens", lens_h)]
+    parts = [(n, r.host[n]) for n in ("q", "k", "v", "tables", "lens")]
     if not fused:  # the fused step takes each token's slot from its table
-        parts.append(("slots", slots_h))
+        parts.append(("slots", r.host["slots"]))
     offs, total = {}, 0
     for name, t in parts:
         offs[name] = total
@@ -489,29 +706,15 @@ def run_gpu(args):
 
     stage_d = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
     sets = [views(b) for b in stage_d]
-    outs = [torch.empty_like(out) for _ in range(2)]
-    outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    outs = [torch.empty_like(r.out) for _ in range(2)]
+    outs_h = [torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory() for _ in range(2)]
     d2h = outs_h[0].numel() * outs_h[0].element_size()
     copy_stream = torch.cuda.Stream(dev)   # uploads
     d2h_stream = torch.cuda.Stream(dev)    # downloads, on the other copy engine
     h2d_done, comp_done, d2h_done = ([torch.cuda.Event(), torch.cuda.Event()] for _ in range(3))
 
     def step_on(i):
-        c = sets[i % 2]
-        o = outs[i % 2]
-        if fused:
-            fused_step(o, c)
-            return
-        pkv.paged_kv_write(c["k"], c["v"], kc, vc, c["slots"], err=err)
-        if args.cascade:
-            pkv.paged_attention_decode_prefix(o, c["q"], kc, vc, c["tables"], c["lens"], scale, hkv,
-                                              pb, offs_g, mem, max_suffix_blocks=suffix_bound,
-                                              partition_tokens=args.partition, workspace=ws,
-                                              err=err)
-        else:
-            pkv.paged_attention_decode(o, c["q"], kc, vc, c["tables"], c["lens"], scale, hkv,
-                                       variant=variant, partition_tokens=args.partition,
-                                       workspace=ws, err=err)
+        r.step(sets[i % 2], outs[i % 2])
 
     def pipelined(run_step) -> float:
         """K steps: upload of step i+1 and download of step i (two copy streams,
@@ -547,12 +750,11 @@ def run_gpu(args):
         stream.wait_stream(d2h_stream)
         e2e_ev[1].record(stream)
         torch.cuda.synchronize(dev)
-        if int(err.item()) != 0:
-            raise SystemExit(f"device error word {int(err.item())} after the timed steps")
+        r.check_err("after the end-to-end steps")
         # the end-to-end steps ran the same inputs through staged copies: the
         # kernels are deterministic, so the output read back must match bit for bit
         if K > 0 and not torch.equal(outs_h[(K - 1) % 2].view(torch.int16),
-                                     out.cpu().view(torch.int16)):
+                                     r.out.cpu().view(torch.int16)):
             raise SystemExit("end-to-end output differs from the device-timed output")
         return e2e_ev[0].elapsed_time(e2e_ev[1])
 
@@ -568,80 +770,40 @@ def run_gpu(args):
         graphs.append(g)
     e2e_graph_ms = pipelined(lambda i: graphs[i % 2].replay())
     del graphs
+    e2e_ms, e2e_graph_ms = max_over_ranks([e2e_ms, e2e_graph_ms], device=dev)
 
-    total_ms, e2e_ms, e2e_graph_ms, u_ms = max_over_ranks(
-        [total_ms, e2e_ms, e2e_graph_ms, unfused["total_ms"] if unfused else 0.0], device=dev)
-    if unfused:
-        unfused = {"write_us": unfused["write_us"], "decode_us": unfused["decode_us"],
-                   "value": job_throughput(B, K, world, u_ms)}
-
-    ab = algorithmic_bytes(w)
-    peak, peak_kind = measured_peak_hbm()
-    dec_bytes = ab["kv"] + ab["q"]
-    if args.cascade:
-        # what the cascade must read: each group's prefix once, every suffix once
-        unique_tokens = int((np.asarray(w.lens, np.int64) - 16 * pb_h.astype(np.int64)).sum())
-        unique_tokens += sum(16 * int(pb_h[mem_h[offs_h[g]]]) for g in range(len(offs_h) - 1))
-        dec_bytes = unique_tokens * hkv * d * 2 * 2 + ab["q"]
-    if fused:  # the new tokens' K/V: read once, written once
-        dec_bytes += 2 * B * hkv * d * 2 * 2
-    achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
-    value = job_throughput(B, K, world, total_ms)
-    e2e_value = job_throughput(B, K, world, e2e_ms)
-    # write + decode, + the merge (split-K, balanced) or the longest-first order (single pass)
-    ordered = chosen == pkv.DECODE_SINGLE and ws.numel() >= 4 * B
-    launches_per_step = (1 if fused else 2) + \
-        (1 if chosen in (pkv.DECODE_SPLIT, pkv.DECODE_STREAM) or ordered else 0)
-    if args.cascade:  # (write;) prefix chunks + suffix split-K in one launch, merge
-        launches_per_step = 2 if fused else 3
+    ab = m["bytes"]
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": METRIC, "value": m["value"], "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
             "workload": WORKLOAD_NAMES[args.config], "name": args.config, "batch": B,
             "num_heads": hq, "num_kv_heads": hkv, "head_dim": d, "block_tokens": 16,
-            "tokens": ab["tokens"], "num_blocks": w.num_blocks, "table_width": W,
-            "variant": {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head, longest "
-                                            "first)" if ordered else
-                        "single pass (one CTA per sequence x KV head)",
-                        pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % args.partition,
-                        pkv.DECODE_STREAM: "balanced stream-K (equal tile ranges per warp) + merge",
-                        }[chosen] if not args.cascade else
-            "shared-prefix cascade (prefix once per group x KV head, split-K suffixes, merge)",
+            "tokens": ab["tokens"], "num_blocks": r.w.num_blocks, "table_width": W,
+            "variant": r.variant_text(),
             "logical_kv_bytes": ab["kv"],
             "l2": (f"L2 flushed between steps (256 MB write); step time from per-step events "
-                   f"(KV {ab['kv'] / 1e9:.3f} GB per step)") if flush else
+                   f"(KV {ab['kv'] / 1e9:.3f} GB per step)") if m["flush"] else
                   f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), no flush",
+            "timing": "CUDA events on the launching stream; a spin kernel lets the host enqueue "
+                      "ahead of the device, outside the steps' events",
             "parallelism": f"{world} independent replicas (batch per GPU fixed)",
             "seed": args.seed,
         },
-        "kv_hbm_gbs": achieved,
-        "kv_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
-        "kv_frac_of_measured_copy": achieved / peak,
-        "write_us": write_ms * 1e3 if write_ms is not None else None,
-        "decode_us": decode_ms * 1e3,
+        "kv_hbm_gbs": m["kv_hbm_gbs"],
+        "kv_frac_of_8tbs": m["kv_frac_of_8tbs"],
+        "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
+        "write_us": None if fused else unfused and unfused["write_us"],
+        "decode_us": m["step_us"],
         "step": ("pkv_paged_decode_prefix_step" if args.cascade else "pkv_paged_decode_step") +
                 ": the write fused into the decode kernel" if fused else
                 "pkv_paged_kv_write, then the decode call",
         "unfused": unfused,
-        **({"prefix_tcgen05": prefix_tc} if prefix_tc else {}),
-        "roofline": {
-            "bound": "hbm",
-            "kernel": ("cascade_kernel (prefix chunks + suffix units" +
-                       (", fused write" if fused else "") + ") + cascade_merge_kernel")
-                      if args.cascade else
-                      ("paged_decode_kernel with the fused write" if fused else "paged_decode_kernel")
-                      + (" + merge kernel" if chosen == pkv.DECODE_SPLIT else
-                         " + order kernel" if ordered else ""),
-            "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "peak_kind": peak_kind,
-            "traffic": committed_traffic("paged_decode_kernel", args.config),
-            "algorithmic_bytes_per_launch": dec_bytes,
-        },
-        "gpu_launches": K * launches_per_step,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
+        "roofline": m["roofline"],
+        "gpu_launches": K * r.launches_per_step(),
+        "e2e": {"value": job_throughput(B, K, world, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                 "how": "one pinned staging buffer per step in, output out; double-buffered, "
                        "uploads and downloads on their own streams, overlapping the kernels"},
         "e2e_graph": {"value": job_throughput(B, K, world, e2e_graph_ms), "unit": UNIT,
@@ -649,13 +811,83 @@ def run_gpu(args):
                       "how": "the same loop, each step replayed from a CUDA graph"},
         "clocks": clocks,
     }
+    w_host = r.w
+    del r, stage_d, sets, outs
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_extras and args.batch is None \
+            and not args.cascade and args.variant == "auto":
+        extra = {}
+        for name in ("llama", "long"):
+            if name != args.config:
+                extra[name] = workload_key(args, name, dev=dev)
+        extra["prefix_cascade"] = workload_key(args, "prefix", dev=dev, cascade=True)
+        line["workloads"] = extra
+        line["batch_sweep"] = batch_sweep_key(args, dev)
+        line["prefill"] = {c: prefill_numbers(args, c, dev) for c in ("llama", "qwen")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(w_host, args.cpu_seconds)
+    del w_host
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def prefill_numbers(args, config: str, dev) -> dict:
+    """Paged prefill attention (tcgen05) on 4 prompts x 2048 tokens with
+    Llama-2-7B-shaped (32/32) or Qwen2.5-7B-shaped (28/4) heads: TFLOP/s of the
+    causal attention against the measured bf16 matmul peak, and the prompt's
+    K/V write."""
+    import torch
+
+    from paged_kv_cache_459_b200 import pkv
+    import workloads as wl
+
+    steps, warm = args.steps, max(3, args.warmup)
+    up = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    cfg = wl.config(config)
+    hq, hkv, d, B, n = cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"], 4, 2048
+    alloc = pkv.BlockAllocator(B * n // 16 + 8, wl.rng(args.seed).permutation(B * n // 16 + 8))
+    slots = []
+    for b in range(B):
+        alloc.add_seq(b, 0)
+        slots.append(alloc.extend(b, n))
+    tables, lens = alloc.export(list(range(B)), n // 16)
+    nb = alloc.num_blocks
+    kc, vc = up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 1)), up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 2))
+    T = B * n
+    q = up(wl.bf16_normal((T, hq, d), args.seed, 3))
+    k_new, v_new = up(wl.bf16_normal((T, hkv, d), args.seed, 4)), up(wl.bf16_normal((T, hkv, d), args.seed, 5))
+    out = torch.empty_like(q)
+    t_d, l_d = torch.from_numpy(tables).to(dev), torch.from_numpy(lens).to(dev)
+    qs = torch.tensor([b * n for b in range(B + 1)], dtype=torch.int32, device=dev)
+    sl = torch.from_numpy(np.concatenate(slots)).to(dev)
+    wr_ms = _events_time(lambda: pkv.paged_kv_write(k_new, v_new, kc, vc, sl), steps, warm)
+    run = lambda: pkv.paged_attention_prefill(out, q, kc, vc, t_d, l_d, qs, cfg["scale"], hkv, n)  # noqa: E731
+    sampler = ClockSampler(device_pci_id(dev))
+    ms = _events_time(run, steps, warm)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < 1.0:
+        for _ in range(20):
+            run()
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    flops = B * 4.0 * d * hq * n * (n + 1) / 2  # causal: row i sees i + 1 keys
+    peak, kind = measured_peak_tensor()
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"metric": "paged prefill attention TFLOP/s (causal, bf16 in / fp32 accumulate)",
+            "value": ach, "unit": "TFLOP/s", "ms_per_step": ms, "steps": steps,
+            "workload": f"{B} prompts x {n} tokens, {hq}/{hkv} heads, d {d}",
+            "prompt_write_gbs": T * hkv * d * 2 * 2 * 2 / (wr_ms * 1e-3) / 1e9,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                         "frac": ach / peak, "peak_kind": kind,
+                         "frac_of_sustained": ach / measured_peak_tensor_sustained(),
+                         "kernel": "paged_prefill_tc_kernel (tcgen05, TMEM accumulators)",
+                         "traffic": committed_traffic("paged_prefill_tc_kernel",
+                                                      f"prefill_{config}_4x2048"),
+                         "algorithmic_flops_per_launch": flops},
+            "clocks": clocks, "gpu_launches": steps}
 
 
 def measured_peak_tensor_sustained() -> float:
@@ -756,45 +988,9 @@ def run_row(args):
     up = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     line = {"row": args.row, "n_gpus": 1, "steps": steps, "warmup": warm, "data": "synthetic"}
     if args.row == "prefill":
-        # Llama-2-7B-shaped heads (or Qwen2.5-7B-shaped with --config qwen), 4 prompts x 2048
-        cfg = wl.config("qwen" if args.config == "qwen" else "llama")
-        hq, hkv, d, B, n = cfg["num_heads"], cfg["num_kv_heads"], cfg["head_dim"], 4, 2048
-        alloc = pkv.BlockAllocator(B * n // 16 + 8, wl.rng(args.seed).permutation(B * n // 16 + 8))
-        slots = []
-        for b in range(B):
-            alloc.add_seq(b, 0)
-            slots.append(alloc.extend(b, n))
-        tables, lens = alloc.export(list(range(B)), n // 16)
-        nb = alloc.num_blocks
-        kc, vc = up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 1)), up(wl.bf16_normal((nb, hkv, 16, d), args.seed, 2))
-        T = B * n
-        q = up(wl.bf16_normal((T, hq, d), args.seed, 3))
-        k_new, v_new = up(wl.bf16_normal((T, hkv, d), args.seed, 4)), up(wl.bf16_normal((T, hkv, d), args.seed, 5))
-        out = torch.empty_like(q)
-        t_d, l_d = torch.from_numpy(tables).to(dev), torch.from_numpy(lens).to(dev)
-        qs = torch.tensor([b * n for b in range(B + 1)], dtype=torch.int32, device=dev)
-        sl = torch.from_numpy(np.concatenate(slots)).to(dev)
-        wr_ms = _events_time(lambda: pkv.paged_kv_write(k_new, v_new, kc, vc, sl), steps, warm)
-        run = lambda: pkv.paged_attention_prefill(out, q, kc, vc, t_d, l_d, qs, cfg["scale"], hkv, n)  # noqa: E731
-        os.environ["PKV_PREFILL_WARP_MMA"] = "1"
-        ms_warp = _events_time(run, steps, warm)
-        os.environ.pop("PKV_PREFILL_WARP_MMA")
-        ms = _events_time(run, steps, warm)
-        flops = B * 4.0 * d * hq * n * (n + 1) / 2  # causal: row i sees i + 1 keys
-        peak, kind = measured_peak_tensor()
-        ach = flops / (ms * 1e-3) / 1e12
-        line.update(metric="paged prefill attention TFLOP/s (causal, bf16 in / fp32 accumulate)",
-                    value=ach, unit="TFLOP/s", ms_per_step=ms, higher_is_better=True,
-                    config={"workload": f"{B} prompts x {n} tokens, {hq}/{hkv} heads, d {d}"},
-                    prompt_write_gbs=T * hkv * d * 2 * 2 * 2 / (wr_ms * 1e-3) / 1e9,
-                    warp_mma_tflops=flops / (ms_warp * 1e-3) / 1e12,
-                    roofline={"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                              "frac": ach / peak, "peak_kind": kind,
-                              "frac_of_sustained": ach / measured_peak_tensor_sustained(),
-                              "kernel": "paged_prefill_tc_kernel (tcgen05, TMEM accumulators)",
-                              "traffic": committed_traffic(
-                                  "paged_prefill_tc_kernel",
-                                  "prefill_qwen_4x2048" if args.config == "qwen" else "prefill_llama_4x2048")})
+        # Qwen2.5-7B-shaped heads (default) or Llama-2-7B-shaped with --config llama, 4 x 2048
+        line.update(prefill_numbers(args, "llama" if args.config == "llama" else "qwen", dev))
+        line["higher_is_better"] = True
     elif args.row == "cow":
         cfg = wl.config("llama")
         hkv, d, nb, n = cfg["num_kv_heads"], cfg["head_dim"], 8192, 2048

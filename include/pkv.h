@@ -76,11 +76,14 @@ typedef enum {
 #define PKV_SWAP_IN 1  /* host slot -> GPU block */
 
 typedef enum {
-    PKV_DECODE_AUTO = 0,   /* choose from the shapes (see pkv_paged_attention_decode) */
-    PKV_DECODE_SINGLE = 1, /* one CTA per (sequence, KV head [, group of 8 query heads]) */
-    PKV_DECODE_SPLIT = 2,  /* split-K token partitions + log-sum-exp merge kernel */
-    PKV_DECODE_STREAM = 3  /* balanced: every warp of a persistent grid takes an equal share of
-                              all (sequence, head, block) tiles; cut segments merged by LSE */
+    PKV_DECODE_AUTO = 0,    /* choose from the shapes (see pkv_paged_attention_decode) */
+    PKV_DECODE_SINGLE = 1,  /* one CTA per (sequence, KV head [, group of 8 query heads]) */
+    PKV_DECODE_SPLIT = 2,   /* split-K token partitions + log-sum-exp merge kernel */
+    /* 3: not used (rejected with PKV_ERR_INVALID_ARG) */
+    PKV_DECODE_CLUSTER = 4  /* each sequence cut into P <= 8 equal parts, one CTA each; the P
+                               CTAs of a (sequence, KV head) form a thread-block cluster and
+                               merge their log-sum-exp partials in distributed shared memory
+                               (no workspace, no second kernel) */
 } pkv_decode_variant;
 
 /* Human-readable name of a pkv_status value (static storage). */
@@ -121,23 +124,36 @@ PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_
                                   int max_blocks_per_seq, int partition_tokens);
 
 /*
- * Workspace (device bytes) that `variant` needs for these sizes on the
- * current device (PKV_DECODE_AUTO: enough for any variant it may pick;
- * PKV_DECODE_SINGLE: 0); 0 if a size is invalid.  partition_tokens <= 0
- * means 512.
+ * Workspace (device bytes) that `variant` can use for these sizes
+ * (PKV_DECODE_AUTO: enough for any variant it may pick; PKV_DECODE_SPLIT:
+ * what it needs; PKV_DECODE_SINGLE and PKV_DECODE_CLUSTER: room for the
+ * optional longest-first order of the sequences, 4 bytes per sequence
+ * rounded up to 256 -- they also run without any workspace); 0 if a size is
+ * invalid.  partition_tokens <= 0 means 512.
  */
 PKV_API size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads,
                                               int num_kv_heads, int head_dim,
                                               int max_blocks_per_seq, int partition_tokens);
 
 /*
- * The variant PKV_DECODE_AUTO picks for these sizes given `workspace_bytes`
- * of workspace (PKV_DECODE_SINGLE, _SPLIT or _STREAM); -1 if a size is
- * invalid.
+ * The variant PKV_DECODE_AUTO picks for these sizes on the current device
+ * given `workspace_bytes` of workspace (PKV_DECODE_SINGLE, _SPLIT or
+ * _CLUSTER); -1 if a size is invalid.
  */
 PKV_API int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                    int max_blocks_per_seq, int partition_tokens,
                                    size_t workspace_bytes);
+
+/*
+ * The number of parts P each sequence is cut into when `variant` runs as the
+ * cluster variant: PKV_DECODE_CLUSTER gives ceil(max_blocks_per_seq * 16 /
+ * partition_tokens) capped at 8; PKV_DECODE_AUTO gives its own P when it
+ * picks the cluster variant for these sizes and workspace, else 0; other
+ * variants 0.  -1 if a size is invalid.
+ */
+PKV_API int pkv_decode_cluster_parts_for(int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int max_blocks_per_seq, int variant,
+                                         int partition_tokens, size_t workspace_bytes);
 
 /*
  * Single-query decode attention over the paged cache (section 三, step 三:
@@ -151,14 +167,18 @@ PKV_API int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads
  *
  * head_dim: 64 or 128.  num_heads % num_kv_heads == 0.  Pointers 16-byte
  * aligned.  num_blocks * num_kv_heads * 16 must be < 2^31.
- * This entry point takes PKV_DECODE_AUTO with 512-token partitions: split-K
- * when a sequence may span more than one partition, `workspace` holds
- * pkv_decode_workspace_bytes(...) bytes, and the single-pass grid would be
- * short of CTAs -- its (sequence, KV head [, group of 8 query heads]) units
- * fill fewer than 1.5 waves at 3 CTAs per SM when the workspace also holds
- * the longest-first order (pkv_decode_workspace_bytes_for(PKV_DECODE_SINGLE,
- * ...) bytes), fewer than 4 waves without it; the single-pass variant
- * otherwise.  pkv_decode_variant_for() reports the choice.
+ * This entry point takes PKV_DECODE_AUTO with 512-token partitions.  The
+ * work units are (sequence, KV head [, group of 8 query heads]).  When they
+ * fill at least 1.5 waves of the GPU at 3 CTAs per SM (4 waves if the
+ * workspace cannot hold the longest-first order,
+ * pkv_decode_workspace_bytes_for(PKV_DECODE_SINGLE, ...) bytes): the
+ * single-pass variant.  Otherwise each sequence is cut into parts: the
+ * cluster variant with P = min(8, ceil(2 waves / units), longest table / 4
+ * blocks) parts while a part of the longest sequence stays at most 64 blocks;
+ * else split-K when a sequence may span more than one partition and
+ * `workspace` holds pkv_decode_workspace_bytes(...) bytes; else the cluster
+ * variant (P >= 2) or the single pass.  pkv_decode_variant_for() and
+ * pkv_decode_cluster_parts_for() report the choice.
  * The workspace is scratch owned by the caller; calls that share one
  * workspace must be ordered on the GPU (the same stream, or events).
  */
@@ -173,8 +193,11 @@ PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *q, const vo
 /*
  * As pkv_paged_attention_decode, with the variant and the split-K partition
  * length chosen by the caller.  partition_tokens: a multiple of 16 in
- * [16, 65536] (used by PKV_DECODE_SPLIT only).  PKV_DECODE_SPLIT or
- * PKV_DECODE_STREAM without enough workspace returns PKV_ERR_WORKSPACE.
+ * [16, 65536] (used by PKV_DECODE_SPLIT and PKV_DECODE_CLUSTER).
+ * PKV_DECODE_SPLIT without enough workspace returns PKV_ERR_WORKSPACE.
+ * PKV_DECODE_CLUSTER cuts every sequence into P = ceil(max_blocks_per_seq *
+ * 16 / partition_tokens) (at most 8) equal parts; its workspace is optional
+ * (the longest-first order when num_seqs >= 16).
  * For tuning sweeps, the environment variables PKV_DECODE_WARPS and
  * PKV_DECODE_STAGES (read at each call) pick the decode CTA shape of the
  * single-pass and split-K kernels: 4 warps x 2 ring stages (the default,
@@ -202,8 +225,8 @@ PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const
  * that reads a sequence's last block stores the token there before reading
  * it.  Sequences with seq_lens[b] <= 0 write nothing.  A table entry outside
  * the pool for that block is not written and is flagged
- * PKV_DEV_ERR_BAD_BLOCK.  Variants: PKV_DECODE_AUTO, _SINGLE, _SPLIT
- * (PKV_DECODE_STREAM: PKV_ERR_UNSUPPORTED).  Workspace as for
+ * PKV_DEV_ERR_BAD_BLOCK.  Variants: PKV_DECODE_AUTO, _SINGLE, _SPLIT,
+ * _CLUSTER.  Workspace as for
  * pkv_paged_attention_decode_ex.
  */
 PKV_API pkv_status pkv_paged_decode_step(void *out, const void *q, const void *k_new,
@@ -268,7 +291,14 @@ PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, c
  * prefix; a merge kernel combines the partials.  The prefix chunks run on
  * warp-level mma.sync by default; the environment variable PKV_CASCADE_TC=1
  * selects tcgen05 MMAs with TMEM accumulators instead (same results up to
- * fp32 rounding order; measured slower beside the suffix stream).  Workspace:
+ * fp32 rounding order; measured slower beside the suffix stream).  The
+ * suffix units cover one head segment each, or -- "wide" units -- 4 head
+ * segments of a sequence with one warp streaming each segment's suffix alone
+ * (suffixes are short); wide units are used when the segments (query heads,
+ * or KV heads with at most 8 query heads each) come in groups of 4 and the
+ * wide grid still holds two waves of CTAs at 3 per SM.  The environment
+ * variable PKV_CASCADE_WIDE=0 or =1 turns them off, or on wherever the heads
+ * allow (same results up to fp32 rounding order).  Workspace:
  * pkv_decode_prefix_workspace_bytes(...), else PKV_ERR_WORKSPACE.
  * max_suffix_blocks: an upper bound on ceil(len / 16) - prefix_blocks over the
  * batch (the blocks past each sequence's prefix), or <= 0 for "unknown"
@@ -353,8 +383,7 @@ PKV_API pkv_status pkv_swap_blocks(void *k_cache, void *v_cache, void *host_k, v
  * in the cache already.  max_query_len >= every sequence's row count.
  * 5th-generation tensor cores (tcgen05.mma, bf16 -> fp32 in tensor memory),
  * a persistent grid of one CTA per SM over 256-row work items, TMA-fed K and
- * V rings.  The environment variable PKV_PREFILL_WARP_MMA=1 selects the
- * warp-level mma.m16n8k16 kernel instead (same result; kept for comparison).
+ * V rings.
  * A sequence with seq_lens[b] < its rows or past its table is skipped
  * (rows not written) and flagged PKV_DEV_ERR_BAD_LEN; a table entry outside
  * the pool is read as zeros and flagged PKV_DEV_ERR_BAD_BLOCK.

@@ -41,7 +41,7 @@ namespace {
 
 using namespace dev;
 
-template <int D, int NW, int S, bool MMA, bool SPLIT>
+template <int D, int NW, int S, bool MMA, int MODE>
 __global__ void __launch_bounds__(NW * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(NW * 32)
         pdl_wait_primary();  // the order kernel's output
         b = __ldg(p.order + b);
     }
-    decode_unit<D, NW, S, MMA, SPLIT>(tmk, tmv, p, blockIdx.x, blockIdx.y, b);
+    decode_unit<D, NW, S, MMA, MODE>(tmk, tmv, p, blockIdx.x, blockIdx.y, b);
 }
 
 // Longest-first order of the sequences by block count (counting sort; ties in
@@ -166,58 +166,71 @@ __global__ void __launch_bounds__(D) splitk_merge_kernel(const DecodeParams p) {
     p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
 }
 
-template <int D, int NW, int S, bool MMA, bool SPLIT>
+template <int D, int NW, int S, bool MMA, int MODE>
 cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                        cudaStream_t stream) {
     using G = Geometry<D, NW, S>;
-    auto kern = paged_decode_kernel<D, NW, S, MMA, SPLIT>;
+    auto kern = paged_decode_kernel<D, NW, S, MMA, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          G::kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(p.num_parts),
                     static_cast<unsigned>(MMA ? p.Hkv * p.chunks : p.Hq),
                     static_cast<unsigned>(p.B));
-    if (p.order != nullptr) {
+    if (p.order != nullptr || MODE == kModeCluster) {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = grid;
         cfg.blockDim = dim3(NW * 32);
         cfg.dynamicSmemBytes = G::kSmemBytes;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchAttribute attr[2];
+        unsigned n = 0;
+        if (p.order != nullptr) {  // waits (griddepcontrol.wait) for the order kernel
+            attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[n++].val.programmaticStreamSerializationAllowed = 1;
+        }
+        if (MODE == kModeCluster) {  // the parts of one (sequence, head) form a cluster
+            attr[n].id = cudaLaunchAttributeClusterDimension;
+            attr[n].val.clusterDim.x = static_cast<unsigned>(p.num_parts);
+            attr[n].val.clusterDim.y = 1;
+            attr[n++].val.clusterDim.z = 1;
+        }
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = n;
         e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p);
     } else {
         kern<<<grid, NW * 32, G::kSmemBytes, stream>>>(tmk, tmv, p);
         e = cudaGetLastError();
     }
-    if (e != cudaSuccess || !SPLIT || p.skip_merge) return e;
+    if (e != cudaSuccess || MODE != kModeSplit || p.skip_merge) return e;
     return launch_dependent(splitk_merge_kernel<D>, dim3(static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B)),
                             dim3(D), stream, p);
 }
 
-template <int D, bool MMA, bool SPLIT>
+template <int D, bool MMA, int MODE>
 cudaError_t launch_tuned(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                          DecodeTuning t, cudaStream_t stream) {
     // 4 warps x 2 stages (64 KB of ring at d = 128, three CTAs per SM) measured
     // fastest on every workload (against 1, 2 and 8 warps and 3-4 stages); the
     // other shapes stay for tuning sweeps.
-    if (t.warps == 4 && t.stages == 3) return launch_one<D, 4, 3, MMA, SPLIT>(tmk, tmv, p, stream);
-    if (t.warps == 2 && t.stages == 2) return launch_one<D, 2, 2, MMA, SPLIT>(tmk, tmv, p, stream);
-    return launch_one<D, 4, 2, MMA, SPLIT>(tmk, tmv, p, stream);
+    if (t.warps == 4 && t.stages == 3) return launch_one<D, 4, 3, MMA, MODE>(tmk, tmv, p, stream);
+    if (t.warps == 2 && t.stages == 2) return launch_one<D, 2, 2, MMA, MODE>(tmk, tmv, p, stream);
+    return launch_one<D, 4, 2, MMA, MODE>(tmk, tmv, p, stream);
+}
+
+template <int D, bool MMA>
+cudaError_t launch_m(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
+                     int mode, DecodeTuning t, cudaStream_t stream) {
+    if (mode == kModeSplit) return launch_tuned<D, MMA, kModeSplit>(tmk, tmv, p, t, stream);
+    if (mode == kModeCluster) return launch_tuned<D, MMA, kModeCluster>(tmk, tmv, p, t, stream);
+    return launch_tuned<D, MMA, kModeSingle>(tmk, tmv, p, t, stream);
 }
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
-                     bool split, DecodeTuning t, cudaStream_t stream) {
-    const bool mma = p.group > 1;
-    if (mma)
-        return split ? launch_tuned<D, true, true>(tmk, tmv, p, t, stream)
-                     : launch_tuned<D, true, false>(tmk, tmv, p, t, stream);
-    return split ? launch_tuned<D, false, true>(tmk, tmv, p, t, stream)
-                 : launch_tuned<D, false, false>(tmk, tmv, p, t, stream);
+                     int mode, DecodeTuning t, cudaStream_t stream) {
+    return p.group > 1 ? launch_m<D, true>(tmk, tmv, p, mode, t, stream)
+                       : launch_m<D, false>(tmk, tmv, p, mode, t, stream);
 }
 
 }  // namespace
@@ -230,9 +243,13 @@ cudaError_t launch_order(const int32_t *seq_lens, int B, int W, int32_t *order, 
 }
 
 cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
-                          int head_dim, bool split, DecodeTuning tuning, cudaStream_t stream) {
-    if (head_dim == 128) return launch_d<128>(tmk, tmv, p, split, tuning, stream);
-    if (head_dim == 64) return launch_d<64>(tmk, tmv, p, split, tuning, stream);
+                          int head_dim, int mode, DecodeTuning tuning, cudaStream_t stream) {
+    if (mode != dev::kModeSingle && mode != dev::kModeSplit && mode != dev::kModeCluster)
+        return cudaErrorInvalidValue;
+    if (mode == dev::kModeCluster && (p.num_parts < 1 || p.num_parts > kMaxClusterParts))
+        return cudaErrorInvalidValue;
+    if (head_dim == 128) return launch_d<128>(tmk, tmv, p, mode, tuning, stream);
+    if (head_dim == 64) return launch_d<64>(tmk, tmv, p, mode, tuning, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -613,8 +613,11 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
 // evenly through the grid, so that every SM runs the short, latency-bound
 // prefix work beside the bandwidth-bound suffix stream; the other CTAs take
 // suffix units in order (partition fastest, then head segment, then
-// sequence).  TC: the prefix chunks on tcgen05 (else mma.sync).
-template <int D, bool MMA, bool TC>
+// sequence).  TC: the prefix chunks on tcgen05 (else mma.sync).  WIDE: each
+// suffix CTA covers kPrefixWarps head segments of one sequence, a warp each
+// (suffixes are short: one warp per segment keeps every ring busy for the
+// whole suffix instead of a quarter of it).
+template <int D, bool MMA, bool TC, bool WIDE>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const PrefixParams pp, const DecodeParams dp, int n_pre) {
@@ -637,7 +640,7 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
     // twice as long).
     if (TC && n_pre > 0 && threadIdx.x < 32) tc::relinquish();
     if (n_pre > 0) id -= min(id / stride + 1, n_pre);  // prefix CTAs at or before this one
-    const int ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
+    const int ny = (MMA ? dp.Hkv * dp.chunks : dp.Hq) / (WIDE ? kPrefixWarps : 1);
     const int part = id % dp.num_parts;
     id /= dp.num_parts;
     const int b = id / ny;
@@ -649,20 +652,20 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
         if (start + dp.num_parts * dp.part_blocks < (len + kBlockTokens - 1) / kBlockTokens)
             flag(dp.err, PKV_DEV_ERR_BAD_LEN);
     }
-    decode_unit<D, kPrefixWarps, 2, MMA, true>(tmk, tmv, dp, part, id % ny, b);
+    decode_unit<D, kPrefixWarps, 2, MMA, kModeSplit, WIDE>(tmk, tmv, dp, part, id % ny, b);
 }
 
-template <int D, bool MMA, bool TC>
+template <int D, bool MMA, bool TC, bool WIDE>
 cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                              const DecodeParams &dp, int num_groups, cudaStream_t stream) {
     constexpr int kPre = TC ? PrefixTcGeometry<D, kPrefixChunkBlocks>::kSmemBytes
                             : PrefixMmaGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
     constexpr int kSmem = std::max(kPre, Geometry<D, kPrefixWarps, 2>::kSmemBytes);
-    auto kern = cascade_kernel<D, MMA, TC>;
+    auto kern = cascade_kernel<D, MMA, TC, WIDE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const long long n_pre = static_cast<long long>(pp.prefix_parts) * pp.Hkv * num_groups;
-    const long long ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
+    const long long ny = (MMA ? dp.Hkv * dp.chunks : dp.Hq) / (WIDE ? kPrefixWarps : 1);
     const long long n_suf = static_cast<long long>(dp.num_parts) * ny * dp.B;
     if (n_pre + n_suf >= (1ll << 31)) return cudaErrorInvalidValue;
     kern<<<static_cast<unsigned>(n_pre + n_suf), kPrefixWarps * 32, kSmem, stream>>>(
@@ -673,24 +676,37 @@ cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, con
                             stream, pp);
 }
 
+template <int D, bool TC, bool WIDE>
+cudaError_t launch_cascade_w(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
+                             const DecodeParams &dp, int num_groups, cudaStream_t stream) {
+    return dp.group > 1 ? launch_cascade_d<D, true, TC, WIDE>(tmk, tmv, pp, dp, num_groups, stream)
+                        : launch_cascade_d<D, false, TC, WIDE>(tmk, tmv, pp, dp, num_groups, stream);
+}
+
 template <int D>
 cudaError_t launch_cascade_h(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
-                             const DecodeParams &dp, int num_groups, bool prefix_tc, cudaStream_t stream) {
-    const bool mma = dp.group > 1;
+                             const DecodeParams &dp, int num_groups, bool prefix_tc, bool wide,
+                             cudaStream_t stream) {
     if (prefix_tc)
-        return mma ? launch_cascade_d<D, true, true>(tmk, tmv, pp, dp, num_groups, stream)
-                   : launch_cascade_d<D, false, true>(tmk, tmv, pp, dp, num_groups, stream);
-    return mma ? launch_cascade_d<D, true, false>(tmk, tmv, pp, dp, num_groups, stream)
-               : launch_cascade_d<D, false, false>(tmk, tmv, pp, dp, num_groups, stream);
+        return wide ? launch_cascade_w<D, true, true>(tmk, tmv, pp, dp, num_groups, stream)
+                    : launch_cascade_w<D, true, false>(tmk, tmv, pp, dp, num_groups, stream);
+    return wide ? launch_cascade_w<D, false, true>(tmk, tmv, pp, dp, num_groups, stream)
+                : launch_cascade_w<D, false, false>(tmk, tmv, pp, dp, num_groups, stream);
 }
 
 }  // namespace
 
+bool cascade_wide_fits(const DecodeParams &dp) {
+    const int segments = dp.group > 1 ? dp.Hkv * dp.chunks : dp.Hq;
+    return segments % kPrefixWarps == 0 && dp.chunks == 1;
+}
+
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                            const DecodeParams &dp, int head_dim, int num_groups, bool prefix_tc,
-                           cudaStream_t stream) {
-    if (head_dim == 128) return launch_cascade_h<128>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
-    if (head_dim == 64) return launch_cascade_h<64>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
+                           bool wide, cudaStream_t stream) {
+    if (wide && !cascade_wide_fits(dp)) return cudaErrorInvalidValue;
+    if (head_dim == 128) return launch_cascade_h<128>(tmk, tmv, pp, dp, num_groups, prefix_tc, wide, stream);
+    if (head_dim == 64) return launch_cascade_h<64>(tmk, tmv, pp, dp, num_groups, prefix_tc, wide, stream);
     return cudaErrorInvalidValue;
 }
 

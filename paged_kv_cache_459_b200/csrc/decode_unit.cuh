@@ -8,20 +8,39 @@
 namespace pkv {
 namespace dev {
 
+// How a decode unit's result leaves the CTA.
+constexpr int kModeSingle = 0;   // the whole sequence: normalised row to `out`
+constexpr int kModeSplit = 1;    // one token partition: (m, l, o) partial to the workspace
+constexpr int kModeCluster = 2;  // one of p.num_parts equal parts of the sequence, the parts
+                                 // a thread-block cluster, merged through its shared memory
+
 // One work unit (partition `part` of sequence b, KV head / head chunk `by`)
-// of the per-unit decode kernel, run by a CTA of NW warps.
-template <int D, int NW, int S, bool MMA, bool SPLIT>
+// of the per-unit decode kernel, run by a CTA of NW warps.  The warps take
+// the unit's blocks round-robin and are combined in shared memory at the end.
+// WIDE: the unit is NW head segments instead (by = group of NW: MHA query
+// heads, or KV heads with one chunk of <= 8 query heads each); warp w takes
+// every block of segment by * NW + w alone, so short sequences keep each
+// warp's ring busy for NW times as many tiles, and no cross-warp combine is
+// needed (each warp's result is final).
+template <int D, int NW, int S, bool MMA, int MODE, bool WIDE = false>
 __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtensorMap &tmv,
                                             const DecodeParams &p, int part, int by, int b) {
     using G = Geometry<D, NW, S>;
+    constexpr bool SPLIT = MODE == kModeSplit;
+    constexpr bool CLUSTER = MODE == kModeCluster;
+    static_assert(!(WIDE && CLUSTER), "wide units run single pass or split-K");
     // The merge kernel may be scheduled as soon as every unit has started; it
     // waits for this grid to finish before reading the partials.
     if constexpr (SPLIT) pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kvh = MMA ? by / p.chunks : by;
-    const int chunk = MMA ? by % p.chunks : 0;
-    const int h0 = MMA ? kvh * p.group + chunk * 8 : kvh;  // first query head of this CTA
+    const int seg = WIDE ? by * NW + warp : by;  // head segment: query head, or KV head [x chunk]
+    const int kvh = MMA ? seg / p.chunks : seg;
+    const int chunk = MMA ? seg % p.chunks : 0;
+    const int h0 = MMA ? kvh * p.group + chunk * 8 : kvh;  // first query head of this warp's segment
     const int heads = MMA ? min(8, p.group - chunk * 8) : 1;
+    // query heads of the whole CTA (wide: NW segments; chunks == 1 for MMA) from h0_cta
+    const int h0_cta = WIDE ? (MMA ? by * NW * p.group : by * NW) : h0;
+    const int heads_cta = WIDE ? NW * heads : heads;
 
     int len = __ldg(p.seq_lens + b);
     if (len < 0 || len > p.W * kBlockTokens) {
@@ -31,20 +50,24 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
     int start = 0;
     if (p.start_blocks != nullptr) start = min(max(__ldg(p.start_blocks + b), 0), len / kBlockTokens);
-    // Partitions are counted from the start block.
-    const int blk_begin = start + part * p.part_blocks;
-    const int blk_end = min(nblk, start + (part + 1) * p.part_blocks);
-    if (blk_begin >= blk_end) {
+    // Partitions are counted from the start block.  Cluster mode: the
+    // sequence's blocks are cut into p.num_parts equal parts, one per CTA.
+    const int pblk = CLUSTER ? (nblk - start + p.num_parts - 1) / p.num_parts : p.part_blocks;
+    const int blk_begin = min(nblk, start + part * pblk);
+    const int blk_end = min(nblk, blk_begin + pblk);
+    // Cluster mode: an empty part still takes part in the merge (every CTA of
+    // the cluster must reach its barriers); it contributes nothing.
+    if (blk_begin >= blk_end && !CLUSTER) {
         // Nothing to read.  Single pass: the (empty) sequence's rows are zero.
         // Split-K: the merge kernel only reads partitions that hold tokens.
         // A fused write whose token lies before the start block (inside a
         // shared prefix) cannot be done here: flagged.
         if (p.k_new != nullptr && part == 0 && len > 0 && start >= nblk && threadIdx.x == 0 &&
-            (!MMA || by % p.chunks == 0))
+            (WIDE || !MMA || by % p.chunks == 0))
             flag(p.err, PKV_DEV_ERR_BAD_LEN);
         if (!SPLIT)
-            for (int i = threadIdx.x; i < heads * D; i += NW * 32)
-                p.out[(static_cast<size_t>(b) * p.Hq + h0 + i / D) * D + i % D] = __float2bfloat16(0.f);
+            for (int i = threadIdx.x; i < heads_cta * D; i += NW * 32)
+                p.out[(static_cast<size_t>(b) * p.Hq + h0_cta + i / D) * D + i % D] = __float2bfloat16(0.f);
         return;
     }
 
@@ -64,11 +87,14 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     }
     __syncthreads();
 
-    const int n_mine = blk_end - blk_begin > warp ? (blk_end - blk_begin - warp + NW - 1) / NW : 0;
+    // Round-robin: warp w takes blocks blk_begin + w, + NW, ...; wide: all of them.
+    constexpr int kStride = WIDE ? 1 : NW;
+    const int lead = WIDE ? 0 : warp;
+    const int n_mine = blk_end - blk_begin > lead ? (blk_end - blk_begin - lead + kStride - 1) / kStride : 0;
     TableWindow tw;
     tw.row = p.block_tables + static_cast<size_t>(b) * p.W;
-    tw.first = blk_begin + warp;
-    tw.stride = NW;
+    tw.first = blk_begin + lead;
+    tw.stride = kStride;
     tw.count = n_mine;
     tw.init(lane);
     const uint64_t policy = l2_policy_evict_first();
@@ -107,9 +133,11 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     // registers now, the store and the proxy fence (then __syncwarp, so lane
     // 0's TMA read is ordered after them) wait until then.  Several
     // head-chunk CTAs of one KV head store the same bytes.
+    // (Wide units: every warp holds its own segment's last block.)
     const int last_local = nblk - 1 - blk_begin;
-    const bool writer = p.k_new != nullptr && blk_end == nblk && len > 0 && warp == last_local % NW;
-    const int i_write = last_local / NW;
+    const bool writer = p.k_new != nullptr && blk_end == nblk && len > 0 &&
+                        (WIDE || warp == last_local % NW);
+    const int i_write = last_local / kStride;
     uint4 new_val = make_uint4(0, 0, 0, 0);
     __nv_bfloat16 *new_dst = nullptr;
     if (writer && lane < 2 * (D / 8)) {
@@ -147,7 +175,7 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         }
         const int32_t phys = tw.get(i);
         if (phys >= 0 && phys < p.num_blocks) {
-            const int lb = blk_begin + warp + NW * i;
+            const int lb = blk_begin + lead + kStride * i;
             const int nvalid = min(kBlockTokens, len - lb * kBlockTokens);
             const uint8_t *kt = ring + s * G::kStageBytes;
             if constexpr (MMA)
@@ -169,12 +197,47 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
             mbar_wait(bars + 8 * (j % S), static_cast<uint32_t>((j / S) & 1), kWaitLimitNs);
     }
 
+    constexpr int kRed = MMA ? 16 + 8 * D : D + 2;
+    if constexpr (WIDE) {
+        // This warp's result is final for its segment: its (m, l, o) go
+        // through its own (drained) ring slice and out.
+        __syncwarp();
+        float *wr = reinterpret_cast<float *>(ring);
+        st.finish(wr, lane);
+        __syncwarp();
+        for (int idx = lane; idx < heads * D; idx += 32) {
+            const int n = idx / D, e = idx % D;
+            const float M = MMA ? wr[n] : wr[D];
+            const float L = MMA ? wr[8 + n] : wr[D + 1];
+            const float O = MMA ? wr[16 + n * D + e] : wr[e];
+            const size_t row = static_cast<size_t>(b) * p.Hq + h0 + n;
+            if constexpr (SPLIT) {
+                const size_t pr = row * p.ws_parts + p.ws_part0 + part;
+                p.ws_o[pr * D + e] = O;
+                if (e == 0) {
+                    p.ws_ml[2 * pr] = M;
+                    p.ws_ml[2 * pr + 1] = L;
+                }
+            } else {
+                p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
+            }
+        }
+        return;
+    }
+
     // ---- combine the warps of this CTA (all rings are drained) ----
     __syncthreads();
-    constexpr int kRed = MMA ? 16 + 8 * D : D + 2;
     float *red = reinterpret_cast<float *>(smem);
+    // cluster mode: this CTA's combined rows for the other CTAs of the
+    // cluster -- m of head n at [n], l at [8 + n], o at [16 + n * D + e]
+    float *xch = red + NW * kRed;
     st.finish(red + warp * kRed, lane);
     __syncthreads();
+    if constexpr (CLUSTER) {
+        if (blk_begin >= blk_end && p.k_new != nullptr && len > 0 && start >= nblk && part == 0 &&
+            threadIdx.x == 0 && (!MMA || by % p.chunks == 0))
+            flag(p.err, PKV_DEV_ERR_BAD_LEN);  // the fused write's token lies inside the skipped prefix
+    }
     for (int idx = threadIdx.x; idx < heads * D; idx += NW * 32) {
         const int n = idx / D, e = idx % D;
         float mw[NW];
@@ -201,9 +264,43 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
                 p.ws_ml[2 * pr] = M;
                 p.ws_ml[2 * pr + 1] = L;
             }
+        } else if constexpr (CLUSTER) {
+            xch[16 + n * D + e] = O;
+            if (e == 0) {
+                xch[n] = M;
+                xch[8 + n] = L;
+            }
         } else {
             p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
         }
+    }
+    if constexpr (CLUSTER) {
+        // Log-sum-exp merge of the cluster's parts, in part order (the same
+        // arithmetic as the split-K merge kernel): each CTA merges an equal
+        // slice of the (head, column) elements, reading every part's m, l and
+        // o from the owning CTA's shared memory.
+        cluster_sync();
+        const int P = p.num_parts;
+        const int total = heads * D;
+        const int per = (total + P - 1) / P;
+        const int lo = static_cast<int>(cluster_ctarank()) * per, hi = min(total, lo + per);
+        for (int idx = lo + threadIdx.x; idx < hi; idx += NW * 32) {
+            const int n = idx / D, e = idx % D;
+            float M = -INFINITY;
+            for (int c = 0; c < P; ++c) M = fmaxf(M, ld_dsmem_f32(xch + n, c));
+            float L = 0.f, O = 0.f;
+            if (M != -INFINITY) {
+                for (int c = 0; c < P; ++c) {
+                    const float mc = ld_dsmem_f32(xch + n, c);
+                    const float wgt = mc == -INFINITY ? 0.f : exp2f(mc - M);
+                    L = fmaf(ld_dsmem_f32(xch + 8 + n, c), wgt, L);
+                    O = fmaf(ld_dsmem_f32(xch + 16 + n * D + e, c), wgt, O);
+                }
+            }
+            p.out[(static_cast<size_t>(b) * p.Hq + h0 + n) * D + e] =
+                __float2bfloat16(L > 0.f ? O / L : 0.f);
+        }
+        cluster_sync();  // no CTA leaves while the others still read its shared memory
     }
 }
 

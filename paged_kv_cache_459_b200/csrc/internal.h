@@ -59,39 +59,16 @@ struct DecodeTuning {
     int stages;  // TMA stages per warp (one K tile + one V tile each)
 };
 
-// Balanced (stream-K) decode: a persistent grid whose warps each take an
-// equal contiguous range of the flattened (sequence, head segment, block)
-// tile order; segments cut between warps are merged by a second kernel.
-constexpr int kStreamMaxCtasPerSm = 8;
-constexpr int kStreamWarps = 4;
+// Most parts of one sequence in cluster mode: the portable cluster size.
+constexpr int kMaxClusterParts = 8;
 
-struct StreamParams {
-    __nv_bfloat16 *out;
-    const __nv_bfloat16 *q;
-    const int32_t *block_tables;
-    const int32_t *seq_lens;
-    long long *ws_total;  // total tiles of the launch (read by the merge kernel)
-    int2 *ws_dir;     // [B * Y] (first worker, last worker) of each segment
-    float *ws_piece;  // [max_workers + B * Y][HP][D + 2]: o, then m[HP], then l[HP]
-    unsigned int *err;
-    long long num_blocks;
-    long long max_workers;  // piece slots reserved for workers
-    long long num_workers;  // warps of the launched grid
-    int W, B, Hq, Hkv;
-    int group, chunks;
-    int Y;   // head segments per sequence: Hkv (one query row per KV head) or Hkv * chunks
-    int HP;  // query heads per segment slot: 1, or min(8, group)
-    float scale_log2;
-};
-
-cudaError_t launch_decode_stream(const CUtensorMap &tmk, const CUtensorMap &tmv,
-                                 const StreamParams &p, int head_dim, cudaStream_t stream);
-
-// Launches the decode kernel (and the merge kernel when split) on `stream`;
-// when p.order is set the decode grid is launched as a programmatic dependent
-// of the order kernel and waits for it.
+// Launches the decode kernel on `stream` in one of three modes (0: single
+// pass, 1: split-K + the merge kernel, 2: p.num_parts parts per sequence as
+// one thread-block cluster, merged in distributed shared memory); when
+// p.order is set the decode grid is launched as a programmatic dependent of
+// the order kernel and waits for it.
 cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
-                          int head_dim, bool split, DecodeTuning tuning, cudaStream_t stream);
+                          int head_dim, int mode, DecodeTuning tuning, cudaStream_t stream);
 
 // Shared-prefix (cascade) decode: prefix blocks read once per (group, KV
 // head) by a dense tensor-core kernel; suffixes by split-K; LSE merge.
@@ -118,10 +95,15 @@ struct PrefixParams {
 
 // One launch running prefix chunks and suffix split-K units side by side,
 // then the merge.  dp must describe split-K with start_blocks = prefix_blocks.
-// prefix_tc: the prefix chunks on tcgen05/TMEM instead of mma.sync.
+// prefix_tc: the prefix chunks on tcgen05/TMEM instead of mma.sync.  wide:
+// each suffix CTA covers 4 head segments of a sequence, one warp each (needs
+// cascade_wide_fits).
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                            const DecodeParams &dp, int head_dim, int num_groups, bool prefix_tc,
-                           cudaStream_t stream);
+                           bool wide, cudaStream_t stream);
+// Wide suffix units need the head segments in whole groups of 4 (and one
+// chunk of <= 8 query heads per KV head).
+bool cascade_wide_fits(const DecodeParams &dp);
 
 // Causal prefill attention of each sequence's new tokens over its paged K/V.
 struct PrefillParams {
@@ -137,10 +119,8 @@ struct PrefillParams {
     int items;  // work items of the persistent tcgen05 kernel (set by its launcher)
 };
 
-cudaError_t launch_prefill(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
-                           int head_dim, int max_query_len, cudaStream_t stream);
-// The same on tcgen05 / TMEM: a persistent kernel, one CTA per SM, work
-// items of two 128-row Q tiles.
+// On tcgen05 / TMEM: a persistent kernel, one CTA per SM, work items of two
+// 128-row Q tiles.
 cudaError_t launch_prefill_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefillParams &p,
                               int head_dim, int max_query_len, int num_sms, cudaStream_t stream);
 

@@ -180,24 +180,61 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
 
 namespace {
 
-struct StreamLayout {
-    int Y, HP;
-    long long max_workers;
-    size_t dir_bytes, piece_bytes;
+size_t order_bytes(int num_seqs) {
+    return (static_cast<size_t>(num_seqs) * sizeof(int32_t) + 255) / 256 * 256;
+}
+
+// (sequence, KV head [, group of 8 query heads]) work units of one decode.
+int64_t decode_units(int num_seqs, int num_heads, int num_kv_heads) {
+    return static_cast<int64_t>(num_seqs) * num_kv_heads * ((num_heads / num_kv_heads + 7) / 8);
+}
+
+// Cluster variant, automatic: parts per sequence so that the grid holds about
+// two waves of CTAs at three per SM, at most kMaxClusterParts, and at least
+// one block per consumer warp (4) in a part of the longest sequence.
+int cluster_parts_auto(int64_t units, int max_blocks_per_seq) {
+    const int64_t target = 2 * 3 * static_cast<int64_t>(sm_count());
+    int64_t parts = (target + units - 1) / std::max<int64_t>(units, 1);
+    parts = std::min<int64_t>(parts, pkv::kMaxClusterParts);
+    parts = std::min<int64_t>(parts, std::max(1, max_blocks_per_seq / 4));
+    return static_cast<int>(std::max<int64_t>(parts, 1));
+}
+
+// Cluster variant, explicit: the longest sequence cut into partition_tokens
+// pieces, at most kMaxClusterParts.
+int cluster_parts_for(int max_blocks_per_seq, int partition_tokens) {
+    return std::min(num_parts_for(max_blocks_per_seq, partition_tokens), pkv::kMaxClusterParts);
+}
+
+// A cluster part longer than this (blocks of the longest sequence) leaves too
+// few CTAs for a long context: split-K with the merge kernel balances better.
+constexpr int kClusterMaxPartBlocks = 64;
+
+struct DecodePlan {
+    int variant;  // PKV_DECODE_SINGLE, _SPLIT or _CLUSTER
+    int parts;    // cluster parts per sequence (cluster variant)
 };
 
-StreamLayout stream_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim) {
-    StreamLayout l{};
-    const int group = num_heads / num_kv_heads;
-    const int chunks = (group + 7) / 8;
-    l.Y = group > 1 ? num_kv_heads * chunks : num_kv_heads;
-    l.HP = group > 1 ? (group < 8 ? group : 8) : 1;
-    l.max_workers = static_cast<long long>(sm_count()) * pkv::kStreamMaxCtasPerSm * pkv::kStreamWarps;
-    const size_t segs = static_cast<size_t>(num_seqs) * l.Y;
-    l.dir_bytes = (256 + segs * 8 + 255) / 256 * 256;  // total-tile word, then the directory
-    l.piece_bytes = (static_cast<size_t>(l.max_workers) + segs) * l.HP *
-                    (static_cast<size_t>(head_dim) + 2) * sizeof(float);
-    return l;
+// The automatic choice.  Single pass, its units run longest first when the
+// workspace holds the order (measured best when the units fill the GPU);
+// when one pass would leave the GPU short of CTAs -- fewer than ~1.5 waves of
+// units at 3 CTAs per SM (4 waves without the order, whose tail is longer) --
+// each sequence is cut into parts: one cluster of up to 8 CTAs per unit,
+// merged on chip, while a part stays short (kClusterMaxPartBlocks), else
+// 512-token split-K partitions and the merge kernel (long contexts).
+DecodePlan plan_auto(int num_seqs, int num_heads, int num_kv_heads, int max_blocks_per_seq,
+                     int partition_tokens, size_t workspace_bytes, size_t split_bytes) {
+    const int64_t units = decode_units(num_seqs, num_heads, num_kv_heads);
+    const bool ordered = workspace_bytes >= order_bytes(num_seqs);
+    const int64_t min_units = ordered ? 3 * 3 * sm_count() / 2 : 4 * 3 * sm_count();
+    if (units >= min_units) return {PKV_DECODE_SINGLE, 1};
+    const int parts = cluster_parts_auto(units, max_blocks_per_seq);
+    const bool short_parts = (max_blocks_per_seq + parts - 1) / parts <= kClusterMaxPartBlocks;
+    if (parts >= 2 && short_parts) return {PKV_DECODE_CLUSTER, parts};
+    if (max_blocks_per_seq > partition_tokens / PKV_BLOCK_TOKENS && workspace_bytes >= split_bytes)
+        return {PKV_DECODE_SPLIT, 1};
+    if (parts >= 2) return {PKV_DECODE_CLUSTER, parts};
+    return {PKV_DECODE_SINGLE, 1};
 }
 
 }  // namespace
@@ -209,14 +246,12 @@ size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads, 
         return 0;
     const size_t split = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
                                                     max_blocks_per_seq, partition_tokens);
-    const StreamLayout l = stream_layout(num_seqs, num_heads, num_kv_heads, head_dim);
-    const size_t stream = l.dir_bytes + l.piece_bytes;
-    const size_t order = (static_cast<size_t>(num_seqs) * sizeof(int32_t) + 255) / 256 * 256;
+    const size_t order = order_bytes(num_seqs);
     switch (variant) {
-        case PKV_DECODE_SINGLE: return order;  // optional: longest-first scheduling
+        case PKV_DECODE_SINGLE:   // optional: longest-first scheduling
+        case PKV_DECODE_CLUSTER: return order;
         case PKV_DECODE_SPLIT: return split;
-        case PKV_DECODE_STREAM: return stream;
-        case PKV_DECODE_AUTO: return std::max(std::max(split, stream), order);
+        case PKV_DECODE_AUTO: return std::max(split, order);
         default: return 0;
     }
 }
@@ -228,24 +263,28 @@ int pkv_decode_variant_for(int num_seqs, int num_heads, int num_kv_heads, int he
         return -1;
     if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
     if (partition_tokens % PKV_BLOCK_TOKENS) return -1;
-    const auto need = [&](int v) {
-        return pkv_decode_workspace_bytes_for(v, num_seqs, num_heads, num_kv_heads, head_dim,
-                                              max_blocks_per_seq, partition_tokens);
-    };
-    // Single pass, its units run longest first when the workspace holds the
-    // order (measured best on the Llama and Qwen shapes); split-K only when
-    // one pass would leave the GPU short of CTAs -- fewer than ~1.5 waves of
-    // (sequence, KV head) units at 3 CTAs per SM (without the order: 4 waves,
-    // since the tail of an unordered grid is longer).  The balanced variant
-    // measured slower than both everywhere, so it is only used when asked for.
-    const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads *
-                          ((num_heads / num_kv_heads + 7) / 8);
-    const bool ordered = workspace_bytes >= need(PKV_DECODE_SINGLE);
-    const int64_t min_units = ordered ? 3 * 3 * sm_count() / 2 : 4 * 3 * sm_count();
-    if (max_blocks_per_seq > partition_tokens / PKV_BLOCK_TOKENS &&
-        workspace_bytes >= need(PKV_DECODE_SPLIT) && units < min_units)
-        return PKV_DECODE_SPLIT;
-    return PKV_DECODE_SINGLE;
+    const size_t split = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                    max_blocks_per_seq, partition_tokens);
+    return plan_auto(num_seqs, num_heads, num_kv_heads, max_blocks_per_seq, partition_tokens,
+                     workspace_bytes, split)
+        .variant;
+}
+
+int pkv_decode_cluster_parts_for(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int max_blocks_per_seq, int variant, int partition_tokens,
+                                 size_t workspace_bytes) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
+        head_dim <= 0 || max_blocks_per_seq <= 0)
+        return -1;
+    if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
+    if (partition_tokens % PKV_BLOCK_TOKENS) return -1;
+    if (variant == PKV_DECODE_CLUSTER) return cluster_parts_for(max_blocks_per_seq, partition_tokens);
+    if (variant != PKV_DECODE_AUTO) return 0;
+    const size_t split = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                    max_blocks_per_seq, partition_tokens);
+    const DecodePlan plan = plan_auto(num_seqs, num_heads, num_kv_heads, max_blocks_per_seq,
+                                      partition_tokens, workspace_bytes, split);
+    return plan.variant == PKV_DECODE_CLUSTER ? plan.parts : 0;
 }
 
 static pkv_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -259,7 +298,9 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
         num_heads % num_kv_heads || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
         !std::isfinite(scale))
         return PKV_ERR_INVALID_ARG;
-    if (variant < PKV_DECODE_AUTO || variant > PKV_DECODE_STREAM) return PKV_ERR_INVALID_ARG;
+    if (variant != PKV_DECODE_AUTO && variant != PKV_DECODE_SINGLE && variant != PKV_DECODE_SPLIT &&
+        variant != PKV_DECODE_CLUSTER)
+        return PKV_ERR_INVALID_ARG;
     if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
     if (partition_tokens % PKV_BLOCK_TOKENS || partition_tokens > 65536) return PKV_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
@@ -275,48 +316,20 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
     const int part_blocks = partition_tokens / PKV_BLOCK_TOKENS;
     const bool ws_aligned = workspace != nullptr && aligned16(workspace);
     const size_t have = ws_aligned ? workspace_bytes : 0;
+    const size_t split_bytes = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                          max_blocks_per_seq, partition_tokens);
+    DecodePlan plan{variant, 1};
     if (variant == PKV_DECODE_AUTO)
-        variant = pkv_decode_variant_for(num_seqs, num_heads, num_kv_heads, head_dim,
-                                         max_blocks_per_seq, partition_tokens, have);
-    if (variant != PKV_DECODE_SINGLE &&
-        have < pkv_decode_workspace_bytes_for(variant, num_seqs, num_heads, num_kv_heads, head_dim,
-                                              max_blocks_per_seq, partition_tokens))
-        return PKV_ERR_WORKSPACE;
-    const bool stream_k = variant == PKV_DECODE_STREAM;
-    const bool split = variant == PKV_DECODE_SPLIT;
-    if (k_new != nullptr && stream_k) return PKV_ERR_UNSUPPORTED;  // fused write: per-unit kernels only
-    const StreamLayout sl = stream_layout(num_seqs, num_heads, num_kv_heads, head_dim);
+        plan = plan_auto(num_seqs, num_heads, num_kv_heads, max_blocks_per_seq, partition_tokens,
+                         have, split_bytes);
+    else if (variant == PKV_DECODE_CLUSTER)
+        plan.parts = cluster_parts_for(max_blocks_per_seq, partition_tokens);
+    if (plan.variant == PKV_DECODE_SPLIT && have < split_bytes) return PKV_ERR_WORKSPACE;
 
     CUtensorMap tmk, tmv;
     if (!encode_cache_map(&tmk, k_cache, rows, head_dim) ||
         !encode_cache_map(&tmv, v_cache, rows, head_dim))
         return PKV_ERR_CUDA;
-
-    if (stream_k) {
-        pkv::StreamParams sp{};
-        sp.out = static_cast<__nv_bfloat16 *>(out);
-        sp.q = static_cast<const __nv_bfloat16 *>(q);
-        sp.block_tables = block_tables;
-        sp.seq_lens = seq_lens;
-        sp.ws_total = static_cast<long long *>(workspace);
-        sp.ws_dir = reinterpret_cast<int2 *>(static_cast<char *>(workspace) + 256);
-        sp.ws_piece = reinterpret_cast<float *>(static_cast<char *>(workspace) + sl.dir_bytes);
-        sp.err = err_word;
-        sp.num_blocks = num_blocks;
-        sp.max_workers = sl.max_workers;
-        sp.W = max_blocks_per_seq;
-        sp.B = num_seqs;
-        sp.Hq = num_heads;
-        sp.Hkv = num_kv_heads;
-        sp.group = num_heads / num_kv_heads;
-        sp.chunks = (sp.group + 7) / 8;
-        sp.Y = sl.Y;
-        sp.HP = sl.HP;
-        sp.scale_log2 = scale * 1.4426950408889634f;
-        cudaError_t e = pkv::launch_decode_stream(tmk, tmv, sp, head_dim,
-                                                  static_cast<cudaStream_t>(stream));
-        return cuda_status(e);
-    }
 
     pkv::DecodeParams p{};
     p.out = static_cast<__nv_bfloat16 *>(out);
@@ -336,28 +349,37 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
     p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
     p.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
     p.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
-    if (split) {
+    int mode = 0;  // single pass
+    bool use_order = false;
+    if (plan.variant == PKV_DECODE_SPLIT) {
+        mode = 1;
         p.part_blocks = part_blocks;
         p.num_parts = num_parts_for(max_blocks_per_seq, partition_tokens);
         const size_t rows_ws = static_cast<size_t>(num_seqs) * num_heads * p.num_parts;
         p.ws_o = static_cast<float *>(workspace);
         p.ws_ml = p.ws_o + rows_ws * head_dim;
         p.ws_parts = p.num_parts;
+    } else if (plan.variant == PKV_DECODE_CLUSTER) {
+        mode = 2;
+        p.part_blocks = 0;  // per sequence: its blocks / num_parts
+        p.num_parts = plan.parts;
+        // longest sequences first when there are enough of them to matter
+        use_order = num_seqs >= 16 && have >= order_bytes(num_seqs);
     } else {
         p.part_blocks = max_blocks_per_seq;
         p.num_parts = 1;
         // longest sequences first, when the workspace has room for the order
-        if (workspace != nullptr && aligned16(workspace) &&
-            workspace_bytes >= static_cast<size_t>(num_seqs) * sizeof(int32_t)) {
-            int32_t *order = static_cast<int32_t *>(workspace);
-            cudaError_t e = pkv::launch_order(seq_lens, num_seqs, max_blocks_per_seq, order,
-                                              static_cast<cudaStream_t>(stream));
-            if (e != cudaSuccess) return cuda_status(e);
-            p.order = order;
-        }
+        use_order = have >= static_cast<size_t>(num_seqs) * sizeof(int32_t);
+    }
+    if (use_order) {
+        int32_t *order = static_cast<int32_t *>(workspace);
+        cudaError_t e = pkv::launch_order(seq_lens, num_seqs, max_blocks_per_seq, order,
+                                          static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_status(e);
+        p.order = order;
     }
     pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
-    cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, split, t,
+    cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, mode, t,
                                        static_cast<cudaStream_t>(stream));
     return cuda_status(e);
 }
@@ -501,10 +523,18 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     dp.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
     dp.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
 
+    // Suffix units: one warp per head segment (wide) when the segments come in
+    // groups of 4 and the wide grid still holds two waves of CTAs at 3 per
+    // SM; PKV_CASCADE_WIDE=0 / 1 turns it off / on (where it fits).
+    const int64_t segments = pp.group > 1 ? static_cast<int64_t>(num_kv_heads) * dp.chunks : num_heads;
+    const int64_t wide_ctas = static_cast<int64_t>(suffix_parts) * (segments / 4) * num_seqs;
+    const int wide_env = env_int("PKV_CASCADE_WIDE", -1);
+    const bool wide = pkv::cascade_wide_fits(dp) &&
+                      (wide_env == 1 || (wide_env < 0 && wide_ctas >= 2 * 3 * sm_count()));
     // mma.sync prefix chunks by default (measured faster beside the suffix
     // stream); PKV_CASCADE_TC=1 selects the tcgen05 ones
     cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
-                                        env_int("PKV_CASCADE_TC", 0) != 0,
+                                        env_int("PKV_CASCADE_TC", 0) != 0, wide,
                                         static_cast<cudaStream_t>(stream));
     return cuda_status(e);
 }
@@ -586,13 +616,8 @@ pkv_status pkv_paged_attention_prefill(void *out, const void *q, const void *k_c
     p.Hkv = num_kv_heads;
     p.group = num_heads / num_kv_heads;
     p.scale_log2 = scale * 1.4426950408889634f;
-    // tcgen05 kernel by default; PKV_PREFILL_WARP_MMA=1 selects the warp-level
-    // mma.sync kernel (kept for comparison).
-    cudaError_t e = env_int("PKV_PREFILL_WARP_MMA", 0)
-                        ? pkv::launch_prefill(tmk, tmv, p, head_dim, max_query_len,
-                                              static_cast<cudaStream_t>(stream))
-                        : pkv::launch_prefill_tc(tmk, tmv, p, head_dim, max_query_len, sm_count(),
-                                                 static_cast<cudaStream_t>(stream));
+    cudaError_t e = pkv::launch_prefill_tc(tmk, tmv, p, head_dim, max_query_len, sm_count(),
+                                           static_cast<cudaStream_t>(stream));
     return cuda_status(e);
 }
 

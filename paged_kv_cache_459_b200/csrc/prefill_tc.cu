@@ -1,8 +1,7 @@
 // Paged prefill attention on the 5th-generation tensor cores (tcgen05, TMEM).
 //
-// Same result as paged_prefill_kernel (prefill.cu): causal attention of each
-// sequence's new tokens over its paged K/V ("vLLM 與 PagedAttention：高吞吐推理
-// 的關鍵", section 三 step 二).  A persistent CTA (one per SM) walks work
+// Causal attention of each sequence's new tokens over its paged K/V ("vLLM 與
+// PagedAttention：高吞吐推理的關鍵", section 三 step 二).  A persistent CTA (one per SM) walks work
 // items; an item is two Q tiles of 128 query rows each -- (token, query head
 // of one KV head) pairs of one sequence -- whose keys are walked in tiles of
 // 128 (eight 16-token blocks); both Q tiles share each K/V tile.  Per Q tile x:

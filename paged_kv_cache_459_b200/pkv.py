@@ -29,7 +29,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_OOM, ERR_CUDA = range(6)
 DEV_ERR_BAD_SLOT, DEV_ERR_BAD_BLOCK, DEV_ERR_BAD_LEN, DEV_ERR_TIMEOUT = 1, 2, 4, 8
-DECODE_AUTO, DECODE_SINGLE, DECODE_SPLIT, DECODE_STREAM = 0, 1, 2, 3
+DECODE_AUTO, DECODE_SINGLE, DECODE_SPLIT, DECODE_CLUSTER = 0, 1, 2, 4
 SWAP_OUT, SWAP_IN = 0, 1
 BLOCK_TOKENS = 16
 DEFAULT_PARTITION_TOKENS = 512
@@ -45,6 +45,7 @@ _sigs = {
     "pkv_decode_workspace_bytes": ([_i32, _i32, _i32, _i32, _i32], _sz),
     "pkv_decode_workspace_bytes_for": ([_i32, _i32, _i32, _i32, _i32, _i32, _i32], _sz),
     "pkv_decode_variant_for": ([_i32, _i32, _i32, _i32, _i32, _i32, _sz], _i32),
+    "pkv_decode_cluster_parts_for": ([_i32, _i32, _i32, _i32, _i32, _i32, _i32, _sz], _i32),
     "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
                                     _f32, _P, _sz, _P, _P], _i32),
     "pkv_paged_attention_decode_ex": ([_P, _P, _P, _P, _P, _i32, _P, _i32, _i32, _i32, _i32, _i64,
@@ -256,6 +257,16 @@ def decode_variant_for(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_p
     """The variant the automatic choice takes for these sizes and workspace."""
     return int(_lib.pkv_decode_variant_for(num_seqs, num_heads, num_kv_heads, head_dim,
                                            max_blocks_per_seq, partition_tokens, workspace_bytes))
+
+
+def decode_cluster_parts_for(num_seqs, num_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                             variant=DECODE_AUTO, partition_tokens=DEFAULT_PARTITION_TOKENS,
+                             workspace_bytes=0) -> int:
+    """Parts per sequence of the cluster variant for these sizes (0 when the
+    variant does not run as the cluster variant)."""
+    return int(_lib.pkv_decode_cluster_parts_for(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                 max_blocks_per_seq, variant, partition_tokens,
+                                                 workspace_bytes))
 
 
 def _decode_args(out, q, new_kv, k_cache, v_cache, block_tables, seq_lens, num_kv_heads, variant,

@@ -86,7 +86,7 @@ def step(**kw):
     (dict(vn=None), pkv.ERR_INVALID_ARG),
     (dict(kn=FAKE + 4), pkv.ERR_INVALID_ARG),
     (dict(D=96), pkv.ERR_UNSUPPORTED),
-    (dict(variant=3, ws=FAKE, wsb=1 << 40), pkv.ERR_UNSUPPORTED),   # stream-K: no fused write
+    (dict(variant=3, ws=FAKE, wsb=1 << 40), pkv.ERR_INVALID_ARG),   # 3 is not a variant
     (dict(variant=2), pkv.ERR_WORKSPACE),
 ])
 def test_fused_step_argument_checks(kw, code):
@@ -135,20 +135,35 @@ def test_write_argument_checks(args, code):
 
 def test_variant_choice_and_workspace_sizes():
     B, hq, hkv, d, W = 64, 32, 32, 128, 128
-    stream = pkv.decode_workspace_bytes_for(pkv.DECODE_STREAM, B, hq, hkv, d, W)
     split = pkv.decode_workspace_bytes_for(pkv.DECODE_SPLIT, B, hq, hkv, d, W)
     assert split == pkv.decode_workspace_bytes(B, hq, d, W)
-    assert pkv.decode_workspace_bytes_for(pkv.DECODE_AUTO, B, hq, hkv, d, W) == max(split, stream, 256)
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_AUTO, B, hq, hkv, d, W) == max(split, 256)
     assert pkv.decode_workspace_bytes_for(pkv.DECODE_SINGLE, B, hq, hkv, d, W) == 256  # the order
-    assert pkv.decode_workspace_bytes_for(pkv.DECODE_STREAM, B, 28, 5, d, W) == 0  # 28 % 5
-    # no workspace: single pass; enough for the balanced variant: balanced
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_CLUSTER, B, hq, hkv, d, W) == 256
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_CLUSTER, B, 28, 5, d, W) == 0  # 28 % 5
+    assert pkv.decode_workspace_bytes_for(3, B, hq, hkv, d, W) == 0  # 3 is not a variant
+    # enough units to fill the GPU: single pass, with or without workspace
     assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, 0) == pkv.DECODE_SINGLE
-    # the automatic choice never takes the balanced variant (it measured slower)
     assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, 1 << 40) == pkv.DECODE_SINGLE
-    # only split-K workspace: split when short of CTAs (8 x 8 units), single pass otherwise
+    # long context (8 sequences x 2048 blocks, 8 x 8 units): a cluster part would span
+    # 256 blocks, so split-K when the workspace holds its partials; the cluster
+    # variant (8 parts) without it
     long_split = pkv.decode_workspace_bytes(8, 32, d, 2048)
     assert pkv.decode_variant_for(8, 32, 8, d, 2048, 512, long_split) == pkv.DECODE_SPLIT
-    assert pkv.decode_variant_for(8, 32, 8, d, 2048, 512, long_split - 1) == pkv.DECODE_SINGLE
-    assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, 0) == pkv.DECODE_SINGLE
+    assert pkv.decode_variant_for(8, 32, 8, d, 2048, 512, long_split - 1) == pkv.DECODE_CLUSTER
+    assert pkv.decode_cluster_parts_for(8, 32, 8, d, 2048, pkv.DECODE_AUTO, 512, 0) == 8
+    # a few short sequences: the cluster variant, parts sized to about two waves
+    assert pkv.decode_variant_for(1, 32, 32, d, 128, 512, 0) == pkv.DECODE_CLUSTER
+    assert pkv.decode_cluster_parts_for(1, 32, 32, d, 128, pkv.DECODE_AUTO, 512, 0) == 8
+    assert pkv.decode_cluster_parts_for(8, 32, 32, d, 128, pkv.DECODE_AUTO, 512, 0) == 4
+    # ... never more parts than a quarter of the longest table's blocks
+    assert pkv.decode_cluster_parts_for(1, 32, 32, d, 12, pkv.DECODE_AUTO, 512, 0) == 3
+    assert pkv.decode_variant_for(1, 32, 32, d, 4, 512, 1 << 30) == pkv.DECODE_SINGLE
+    # explicit cluster variant: the longest table cut into partition_tokens pieces, at most 8
+    assert pkv.decode_cluster_parts_for(B, hq, hkv, d, W, pkv.DECODE_CLUSTER, 512, 0) == 4
+    assert pkv.decode_cluster_parts_for(B, hq, hkv, d, W, pkv.DECODE_CLUSTER, 64, 0) == 8
+    assert pkv.decode_cluster_parts_for(B, hq, hkv, d, 5, pkv.DECODE_CLUSTER, 512, 0) == 1
+    assert pkv.decode_cluster_parts_for(B, hq, hkv, d, W, pkv.DECODE_SPLIT, 512, 0) == 0
     assert pkv.decode_variant_for(B, 5, 2, d, W, 512, 0) == -1
-    assert decode(variant=3) == pkv.ERR_WORKSPACE
+    assert decode(variant=3) == pkv.ERR_INVALID_ARG
+    assert decode(variant=pkv.DECODE_SPLIT) == pkv.ERR_WORKSPACE

@@ -13,7 +13,7 @@ if not torch.cuda.is_available():
 
 from paged_kv_cache_459_b200 import pkv  # noqa: E402
 
-VARIANTS = [(pkv.DECODE_SINGLE, 512), (pkv.DECODE_SPLIT, 32), (pkv.DECODE_STREAM, 512)]
+VARIANTS = [(pkv.DECODE_SINGLE, 512), (pkv.DECODE_SPLIT, 32), (pkv.DECODE_CLUSTER, 32)]
 
 
 @pytest.mark.parametrize("name", ["llama", "qwen"])

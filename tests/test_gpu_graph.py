@@ -38,7 +38,7 @@ def same(a: torch.Tensor, b: torch.Tensor) -> bool:
 
 
 @pytest.mark.parametrize("variant", [pkv.DECODE_AUTO, pkv.DECODE_SINGLE, pkv.DECODE_SPLIT,
-                                     pkv.DECODE_STREAM])
+                                     pkv.DECODE_CLUSTER])
 def test_decode_step_replays_from_a_graph(variant):
     w = build("qwen", 4, batch=12, len_lo=40, len_hi=1200)
     d = DeviceStep(w)
@@ -136,8 +136,7 @@ def test_cascade_replays_from_a_graph():
     assert d.err_word() == 0
 
 
-def test_prefill_replays_from_a_graph(monkeypatch):
-    monkeypatch.delenv("PKV_PREFILL_WARP_MMA", raising=False)
+def test_prefill_replays_from_a_graph():
     hq, hkv, dh, new = 16, 4, 128, [300, 77, 520]
     B = len(new)
     nb = sum(-(-n // 16) for n in new) + 8

@@ -23,7 +23,7 @@ from paged_kv_cache_459_b200 import pkv  # noqa: E402
 import workloads as wl  # noqa: E402
 from relabel import permute_pool  # noqa: E402
 
-SINGLE, SPLIT, STREAM = pkv.DECODE_SINGLE, pkv.DECODE_SPLIT, pkv.DECODE_STREAM
+SINGLE, SPLIT, CLUSTER = pkv.DECODE_SINGLE, pkv.DECODE_SPLIT, pkv.DECODE_CLUSTER
 
 
 def test_tiny_end_to_end():
@@ -32,7 +32,8 @@ def test_tiny_end_to_end():
     d.write()
     kc, vc, ref = oracle_after_write(w)
     assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
-    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 16), (SPLIT, 32), (STREAM, 512)):
+    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 16), (SPLIT, 32), (CLUSTER, 512),
+                          (CLUSTER, 16)):
         out = d.decode(variant, part)
         check_close(out, ref, f"tiny variant {variant} partition {part}")
     assert d.err_word() == 0
@@ -61,7 +62,7 @@ def test_parity_small(name, kw):
     kc, vc, ref = oracle_after_write(w)
     assert np.array_equal(host_bits(d.kc), kc), "write not bit-exact (K)"
     assert np.array_equal(host_bits(d.vc), vc), "write not bit-exact (V)"
-    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 64), (STREAM, 512),
+    for variant, part in ((SINGLE, 512), (SPLIT, 512), (SPLIT, 64), (CLUSTER, 512), (CLUSTER, 64),
                           (pkv.DECODE_AUTO, 512)):
         check_close(d.decode(variant, part), ref, f"{name} {kw} variant {variant}/{part}")
     assert d.err_word() == 0
@@ -79,7 +80,7 @@ def test_parity_full_size(name):
     d.write()
     kc, vc, ref = oracle_after_write(w)
     assert np.array_equal(host_bits(d.kc), kc) and np.array_equal(host_bits(d.vc), vc)
-    for variant in (pkv.DECODE_AUTO, SINGLE, SPLIT, STREAM):
+    for variant in (pkv.DECODE_AUTO, SINGLE, SPLIT, CLUSTER):
         check_close(d.decode(variant, 512), ref, f"{name} full, variant {variant}")
     assert d.err_word() == 0
 
@@ -89,14 +90,14 @@ def test_len_one_is_v_exactly():
     d = DeviceStep(w)
     d.write()
     g = w.cfg["num_heads"] // w.cfg["num_kv_heads"]
-    for variant in (SINGLE, SPLIT, STREAM):
+    for variant in (SINGLE, SPLIT, CLUSTER):
         out = d.decode(variant, 512)
         assert np.array_equal(out, np.repeat(w.v_new, g, axis=1))
     w = build("llama", 2, batch=3, len_lo=1, len_hi=1)
     d = DeviceStep(w)
     d.write()
     assert np.array_equal(d.decode(SINGLE), w.v_new)
-    assert np.array_equal(d.decode(STREAM), w.v_new)
+    assert np.array_equal(d.decode(CLUSTER, 16), w.v_new)
 
 
 def test_block_relabelling_is_bit_exact_on_gpu():
@@ -105,7 +106,7 @@ def test_block_relabelling_is_bit_exact_on_gpu():
         w = build(name, 3, **kw)
         d = DeviceStep(w)
         d.write()
-        outs = {v: d.decode(v, 128) for v in (SINGLE, SPLIT, STREAM)}
+        outs = {v: d.decode(v, 128) for v in (SINGLE, SPLIT, CLUSTER)}
         perm = wl.rng(4).permutation(w.num_blocks)
         t2, s2, kc2, vc2 = permute_pool(perm, w.block_tables, w.slot_mapping,
                                            host_bits(d.kc), host_bits(d.vc))
@@ -113,7 +114,7 @@ def test_block_relabelling_is_bit_exact_on_gpu():
         d2.kc.copy_(torch.from_numpy(kc2.view(np.int16)).view(torch.bfloat16))
         d2.vc.copy_(torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16))
         d2.tables = torch.from_numpy(t2).cuda()
-        for v in (SINGLE, SPLIT, STREAM):
+        for v in (SINGLE, SPLIT, CLUSTER):
             assert np.array_equal(d2.decode(v, 128), outs[v])
 
 
@@ -137,25 +138,30 @@ def test_shared_prefix_matches_private_copy_on_gpu():
     d2.vc = torch.from_numpy(vc2.view(np.int16)).view(torch.bfloat16).cuda()
     d2.tables = torch.from_numpy(t2).cuda()
     assert np.array_equal(d2.decode(SPLIT, 128), base)
-    assert np.array_equal(d2.decode(STREAM), d.decode(STREAM))
+    assert np.array_equal(d2.decode(CLUSTER, 64), d.decode(CLUSTER, 64))
 
 
-STREAM_SHAPES = [
-    ("llama", dict(batch=200, len_lo=1, len_hi=40, head_dim=64)),   # many short segments per worker
-    ("long", dict(batch=1, len_fixed=32768)),                       # segments cut across ~200 workers
-    ("qwen", dict(batch=1, len_lo=1, len_hi=1)),                    # fewer tiles than workers
-    ("qwen", dict(batch=300, len_lo=1, len_hi=300, num_heads=24, num_kv_heads=2)),  # 12-head groups
+CLUSTER_SHAPES = [
+    # (workload, overrides, partition): parts per sequence = the longest table / partition, <= 8
+    ("llama", dict(batch=200, len_lo=1, len_hi=40, head_dim=64), 16),      # 3 parts, many clusters
+    ("long", dict(batch=1, len_fixed=32768), 512),                         # 8 parts of 256 blocks
+    ("qwen", dict(batch=3, len_lo=1, len_hi=300), 16),                     # short rows: empty parts
+    ("qwen", dict(batch=1, len_lo=1, len_hi=1), 16),                       # one block, one part
+    ("qwen", dict(batch=40, len_lo=1, len_hi=300, num_heads=24, num_kv_heads=2), 64),  # 2 chunks
+    ("qwen", dict(batch=7, len_lo=100, len_hi=900, head_dim=64, num_heads=16, num_kv_heads=2), 32),
 ]
 
 
-@pytest.mark.parametrize("name,kw", STREAM_SHAPES, ids=[f"{n}-{i}" for i, (n, _) in enumerate(STREAM_SHAPES)])
-def test_stream_variant_shapes(name, kw):
+@pytest.mark.parametrize("name,kw,part", CLUSTER_SHAPES,
+                         ids=[f"{n}-{i}" for i, (n, _, _) in enumerate(CLUSTER_SHAPES)])
+def test_cluster_variant_shapes(name, kw, part):
+    """The cluster variant where its parts are many, long, empty or single."""
     w = build(name, 11, **kw)
     d = DeviceStep(w)
     d.write()
     kc, vc, ref = oracle_after_write(w)
-    out = d.decode(STREAM)
-    check_close(out, ref, f"stream {name} {kw}")
+    out = d.decode(CLUSTER, part)
+    check_close(out, ref, f"cluster {name} {kw} partition {part}")
     assert d.err_word() == 0
 
 

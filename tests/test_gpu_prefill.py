@@ -55,14 +55,10 @@ def run_prefill(hq, hkv, d, cached, new, seed):
     return host_bits(out), ref
 
 
-@pytest.fixture(params=["tcgen05", "warp_mma"])
-def prefill_impl(request, monkeypatch):
-    """The tcgen05/TMEM kernel (default) and the warp-level mma.sync kernel."""
-    if request.param == "warp_mma":
-        monkeypatch.setenv("PKV_PREFILL_WARP_MMA", "1")
-    else:
-        monkeypatch.delenv("PKV_PREFILL_WARP_MMA", raising=False)
-    return request.param
+@pytest.fixture
+def prefill_impl():
+    """The tcgen05/TMEM prefill kernel."""
+    return "tcgen05"
 
 
 @pytest.mark.parametrize("hq,hkv,d,cached,new", [

@@ -59,8 +59,16 @@ def prefix_impl(request, monkeypatch):
     return request.param
 
 
+@pytest.fixture(params=["narrow", "wide"])
+def suffix_units(request, monkeypatch):
+    """Suffix units of one head segment each, or four per CTA with a warp each
+    (wide; used where the heads come in groups of four)."""
+    monkeypatch.setenv("PKV_CASCADE_WIDE", "1" if request.param == "wide" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("name,kw", CASES, ids=[str(i) for i in range(len(CASES))])
-def test_cascade_matches_oracle(name, kw, prefix_impl):
+def test_cascade_matches_oracle(name, kw, prefix_impl, suffix_units):
     w = build(name, 13, **kw)
     d = DeviceStep(w)
     d.write()
@@ -83,7 +91,7 @@ def test_cascade_suffix_bound_too_small_is_flagged():
     assert d.err_word() & 4
 
 
-def test_cascade_full_size(prefix_impl):
+def test_cascade_full_size(prefix_impl, suffix_units):
     """The prefix workload at full size (128 sequences sharing a 2000-token
     prefix): every output row against the oracle."""
     w = build("prefix", 0)
@@ -97,7 +105,7 @@ def test_cascade_full_size(prefix_impl):
     assert d.err_word() == 0
 
 
-def test_cascade_block_relabelling_is_bit_exact(prefix_impl):
+def test_cascade_block_relabelling_is_bit_exact(prefix_impl, suffix_units):
     w = build("prefix", 14, batch=10, prefix_len=256, suffix_lo=1, suffix_hi=80, prefix_groups=2)
     d = DeviceStep(w)
     d.write()
@@ -112,7 +120,7 @@ def test_cascade_block_relabelling_is_bit_exact(prefix_impl):
 
 
 @pytest.mark.parametrize("idx", [0, 1, 2, 3])
-def test_cascade_fused_step(idx, prefix_impl):
+def test_cascade_fused_step(idx, prefix_impl, suffix_units):
     """pkv_paged_decode_prefix_step: the step's write fused into the cascade --
     caches bit-exact with the oracle's write, output within tolerance, and
     bit-identical to the separate write + cascade."""

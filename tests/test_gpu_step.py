@@ -17,7 +17,7 @@ from paged_kv_cache_459_b200 import pkv  # noqa: E402
 import workloads as wl  # noqa: E402
 
 VARIANTS = [(pkv.DECODE_AUTO, 512), (pkv.DECODE_SINGLE, 512), (pkv.DECODE_SPLIT, 512),
-            (pkv.DECODE_SPLIT, 64)]
+            (pkv.DECODE_SPLIT, 64), (pkv.DECODE_CLUSTER, 512), (pkv.DECODE_CLUSTER, 32)]
 
 
 def fused(d: DeviceStep, variant, part, kc=None, vc=None, tables=None, lens=None):
@@ -97,9 +97,9 @@ def test_fused_step_bad_last_block_is_flagged():
     assert d.err_word() & 2  # PKV_DEV_ERR_BAD_BLOCK
 
 
-def test_fused_step_refuses_stream_variant():
+def test_fused_step_refuses_an_unknown_variant():
     w = build("tiny", 24)
     d = DeviceStep(w)
     with pytest.raises(pkv.PkvError) as ex:
-        fused(d, pkv.DECODE_STREAM, 512)
-    assert ex.value.code == pkv.ERR_UNSUPPORTED
+        fused(d, 3, 512)
+    assert ex.value.code == pkv.ERR_INVALID_ARG
