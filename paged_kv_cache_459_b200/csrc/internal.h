@@ -72,7 +72,7 @@ cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const 
 
 // Shared-prefix (cascade) decode: prefix blocks read once per (group, KV
 // head) by a dense tensor-core kernel; suffixes by split-K; LSE merge.
-constexpr int kPrefixChunkBlocks = 8;  // prefix blocks per CTA
+constexpr int kPrefixChunkBlocks = 8;  // prefix blocks per chunk (one 128-key tile)
 
 struct PrefixParams {
     __nv_bfloat16 *out;
@@ -88,13 +88,15 @@ struct PrefixParams {
     long long num_blocks;
     int W, B, Hq, Hkv, group;
     int ws_parts;      // prefix_parts + suffix partitions
-    int prefix_parts;  // ceil(W / kPrefixChunkBlocks): slots 0.. hold prefix chunks
+    int prefix_parts;  // prefix ranges per (group, KV head): slots 0.. hold their partials
+    int range_chunks;  // chunks of kPrefixChunkBlocks blocks per prefix range (1 on mma.sync)
     int part_blocks;   // suffix split-K partition (blocks)
     float scale_log2;
 };
 
-// One launch running prefix chunks and suffix split-K units side by side,
-// then the merge.  dp must describe split-K with start_blocks = prefix_blocks.
+// The prefix grid, the suffix split-K grid beside it (a programmatic
+// dependent), then the merge.  dp must describe split-K with start_blocks =
+// prefix_blocks.
 // prefix_tc: the prefix chunks on tcgen05/TMEM instead of mma.sync.  wide:
 // each suffix CTA covers 4 head segments of a sequence, one warp each (needs
 // cascade_wide_fits).

@@ -469,7 +469,26 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
                                   ? max_suffix_blocks
                                   : max_blocks_per_seq;
     const int suffix_parts = num_parts_for(suffix_blocks, partition_tokens);
-    const int prefix_parts = (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+    // Prefix work: 8-block chunks; on tcgen05 each CTA takes a range of
+    // chunks with O held in TMEM across them, sized so that the prefix grid
+    // is about 64 CTAs (the (group, KV head, 128-row tile, chunk) steps spread
+    // evenly, rows per group estimated from an even split of the batch); on
+    // mma.sync one chunk per CTA.
+    const bool prefix_tc = env_int("PKV_CASCADE_TC", 0) != 0;
+    const int chunks = (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+    int range_chunks = 1;
+    if (prefix_tc) {
+        const int64_t groups = std::max(num_groups, 1);
+        const int64_t rows = static_cast<int64_t>(num_seqs) * (num_heads / num_kv_heads);
+        const int64_t row_tiles = std::max<int64_t>(1, (rows / groups + 127) / 128);
+        const int64_t steps = groups * num_kv_heads * row_tiles * chunks;
+        const int64_t per_cta = (steps + 63) / 64;
+        range_chunks = static_cast<int>(std::min<int64_t>(
+            chunks, std::max<int64_t>(1, (per_cta + row_tiles - 1) / row_tiles)));
+        const int forced = env_int("PKV_CASCADE_RANGE_CHUNKS", 0);
+        if (forced > 0) range_chunks = std::min(forced, chunks);
+    }
+    const int prefix_parts = (chunks + range_chunks - 1) / range_chunks;
     const size_t ws_rows = static_cast<size_t>(num_seqs) * num_heads * (prefix_parts + suffix_parts);
     float *ws_o = static_cast<float *>(workspace);
     float *ws_ml = ws_o + ws_rows * head_dim;
@@ -493,6 +512,7 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     pp.group = num_heads / num_kv_heads;
     pp.ws_parts = prefix_parts + suffix_parts;
     pp.prefix_parts = prefix_parts;
+    pp.range_chunks = range_chunks;
     pp.part_blocks = partition_tokens / PKV_BLOCK_TOKENS;
     pp.scale_log2 = scale * 1.4426950408889634f;
 
@@ -531,10 +551,9 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     const int wide_env = env_int("PKV_CASCADE_WIDE", -1);
     const bool wide = pkv::cascade_wide_fits(dp) &&
                       (wide_env == 1 || (wide_env < 0 && wide_ctas >= 2 * 3 * sm_count()));
-    // mma.sync prefix chunks by default (measured faster beside the suffix
-    // stream); PKV_CASCADE_TC=1 selects the tcgen05 ones
-    cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
-                                        env_int("PKV_CASCADE_TC", 0) != 0, wide,
+    // mma.sync prefix chunks by default; PKV_CASCADE_TC=1 selects the
+    // tcgen05 prefix ranges
+    cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups, prefix_tc, wide,
                                         static_cast<cudaStream_t>(stream));
     return cuda_status(e);
 }

@@ -328,6 +328,38 @@ def paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_
            "pkv_paged_decode_step")
 
 
+class PreparedDecodeStep:
+    """paged_decode_step bound to fixed tensors: the checks and the pointer
+    marshalling run once, here; each call passes the stored pointers and
+    the current stream to pkv_paged_decode_step.  For serving loops that
+    reuse the same device buffers every step (the tensors must stay alive
+    and keep their shapes; their contents may change between calls)."""
+
+    def __init__(self, out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale,
+                 num_kv_heads, *, variant: int = DECODE_AUTO,
+                 partition_tokens: int = DEFAULT_PARTITION_TOKENS, workspace=None, err=None):
+        ptrs, sizes, tail = _decode_args(out, q, (k_new, v_new), k_cache, v_cache, block_tables,
+                                         seq_lens, num_kv_heads, variant, partition_tokens,
+                                         workspace, err)
+        self._keep = (out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, workspace,
+                      err, _workspaces.get((q.device.type, q.device.index)))
+        self._args = (*ptrs, *sizes, float(scale), variant, partition_tokens, *tail)
+        self._device = q.device
+        self._fn = _lib.pkv_paged_decode_step
+
+    def __call__(self) -> None:
+        code = self._fn(*self._args, _stream_ptr(self._device))
+        if code != OK:
+            raise PkvError(code, "pkv_paged_decode_step")
+
+
+def prepare_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale,
+                        num_kv_heads, **kw) -> PreparedDecodeStep:
+    """A PreparedDecodeStep: paged_decode_step with its argument checks done once."""
+    return PreparedDecodeStep(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens,
+                              scale, num_kv_heads, **kw)
+
+
 def decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks_per_seq,
                                   partition_tokens=DEFAULT_PARTITION_TOKENS) -> int:
     return int(_lib.pkv_decode_prefix_workspace_bytes(num_seqs, num_heads, head_dim,

@@ -81,6 +81,24 @@ def test_cascade_matches_oracle(name, kw, prefix_impl, suffix_units):
     assert d.err_word() == 0
 
 
+@pytest.mark.parametrize("range_chunks", [1, 2, 100])
+@pytest.mark.parametrize("idx", [0, 2, 6])
+def test_cascade_tcgen05_prefix_ranges(idx, range_chunks, monkeypatch):
+    """tcgen05 prefix ranges of one chunk, two chunks, and the whole prefix:
+    the output accumulated in TMEM across chunks with the running max, over
+    one or several 128-row tiles."""
+    monkeypatch.setenv("PKV_CASCADE_TC", "1")
+    monkeypatch.setenv("PKV_CASCADE_RANGE_CHUNKS", str(range_chunks))
+    name, kw = CASES[idx]
+    w = build(name, 17, **kw)
+    d = DeviceStep(w)
+    d.write()
+    kc, vc, ref = oracle_after_write(w)
+    out, pb, offs = cascade(d, bound="exact")
+    check_close(out, ref, f"tcgen05 prefix ranges of {range_chunks} chunks, {kw}")
+    assert d.err_word() == 0
+
+
 def test_cascade_suffix_bound_too_small_is_flagged():
     """A max_suffix_blocks below a real suffix leaves it incomplete and sets the
     bad-length bit (no out-of-range workspace use)."""

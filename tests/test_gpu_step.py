@@ -103,3 +103,25 @@ def test_fused_step_refuses_an_unknown_variant():
     with pytest.raises(pkv.PkvError) as ex:
         fused(d, 3, 512)
     assert ex.value.code == pkv.ERR_INVALID_ARG
+
+
+def test_prepared_step_matches_the_plain_call():
+    """pkv.prepare_decode_step checks its tensors once; each call then runs the
+    same library call on the same buffers: identical output and caches, and a
+    change of the buffers' contents between calls is seen by the next call."""
+    w = build("qwen", 25, batch=6, len_lo=1, len_hi=700)
+    kc, vc, ref = oracle_after_write(w)
+    d, e = DeviceStep(w), DeviceStep(w)
+    out = fused(d, pkv.DECODE_AUTO, 512)
+    step = pkv.prepare_decode_step(e.out, e.q, e.k_new, e.v_new, e.kc, e.vc, e.tables, e.lens,
+                                   w.cfg["scale"], w.cfg["num_kv_heads"], err=e.err)
+    step()
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(e.out), out)
+    assert np.array_equal(host_bits(e.kc), kc) and np.array_equal(host_bits(e.vc), vc)
+    e.q.copy_(torch.flip(e.q, dims=[0]))  # new queries in the same buffer
+    step()
+    torch.cuda.synchronize()
+    d.q.copy_(torch.flip(d.q, dims=[0]))
+    assert np.array_equal(host_bits(e.out), fused(d, pkv.DECODE_AUTO, 512))
+    assert e.err_word() == 0
