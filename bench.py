@@ -479,10 +479,26 @@ class Resident:
             raise SystemExit(f"{self.name}: device error word {int(self.err.item())} {when}")
 
 
+class L2Flush:
+    """Empties L2 between timed steps: a 256 MB buffer is written (L2 then
+    holds none of the step's inputs), then another 256 MB is read, so that the
+    dirty lines of that write go back to HBM here rather than inside the next
+    step (whose misses would otherwise pay for their write-back)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+
 def device_steps(step, K: int, dev, flush_buf=None):
     """Device time of K calls of step(): per-step CUDA events (ms each) and the
-    whole loop (ms).  With flush_buf, L2 is flushed (a write larger than L2)
-    before every step, outside its events."""
+    whole loop (ms).  With flush_buf (an L2Flush), L2 is emptied before every
+    step, outside its events."""
     import torch
 
     stream = torch.cuda.current_stream(dev)
@@ -496,7 +512,7 @@ def device_steps(step, K: int, dev, flush_buf=None):
         if flush_buf is not None:
             if i and i % FLUSH_CHUNK == 0:
                 torch.cuda._sleep(SPIN_CYCLES_CHUNK)
-            flush_buf.zero_()  # L2 holds none of this step's inputs
+            flush_buf()  # L2 holds none of this step's inputs and no dirty lines
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
@@ -518,7 +534,7 @@ def timed_decode(r: Resident, K: int, W: int, *, world: int, sampler=None, flush
     ab = r.bytes()
     if flush is None:
         flush = ab["kv"] <= L2_BYTES
-    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=r.dev) if flush else None
+    flush_buf = L2Flush(r.dev) if flush else None
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -578,7 +594,7 @@ def workload_key(args, name, *, dev, cascade=False, batch=None, clocks=True) -> 
         "decode_us": m["step_us"], "value": m["value"], "unit": UNIT,
         "kv_hbm_gbs": m["kv_hbm_gbs"], "kv_frac_of_8tbs": m["kv_frac_of_8tbs"],
         "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
-        "l2": "flushed between steps (256 MB write), step time from per-step events"
+        "l2": "flushed between steps (256 MB write, then 256 MB read), step time from per-step events"
         if m["flush"] else "inputs larger than L2, no flush",
         "roofline": m["roofline"], "gpu_launches": args.steps * r.launches_per_step(),
     }
@@ -673,7 +689,7 @@ def run_gpu(args):
     fused = r.fused
     unfused = None
     if fused:  # the same step as two calls (write, then decode), for comparison
-        flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if m["flush"] else None
+        flush_buf = L2Flush(dev) if m["flush"] else None
         uw, _ = device_steps(r.write, K, dev, flush_buf)  # the write call alone
         per, loop = device_steps(r.two_calls, K, dev, flush_buf)
         u_ms = max_over_ranks([sum(per) if m["flush"] else loop], device=dev)[0]
@@ -797,7 +813,8 @@ def run_gpu(args):
             "tokens": ab["tokens"], "num_blocks": r.w.num_blocks, "table_width": W,
             "variant": r.variant_text(),
             "logical_kv_bytes": ab["kv"],
-            "l2": (f"L2 flushed between steps (256 MB write); step time from per-step events "
+            "l2": (f"L2 flushed between steps (a 256 MB write, then a 256 MB read, so no dirty "
+                   f"lines either); step time from per-step events "
                    f"(KV {ab['kv'] / 1e9:.3f} GB per step)") if m["flush"] else
                   f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), no flush",
             "timing": "CUDA events on the launching stream; a spin kernel lets the host enqueue "

@@ -173,8 +173,9 @@ PKV_API int pkv_decode_cluster_parts_for(int num_seqs, int num_heads, int num_kv
  * workspace cannot hold the longest-first order,
  * pkv_decode_workspace_bytes_for(PKV_DECODE_SINGLE, ...) bytes): the
  * single-pass variant.  Otherwise each sequence is cut into parts: the
- * cluster variant with P = min(8, ceil(2 waves / units), longest table / 4
- * blocks) parts while a part of the longest sequence stays at most 64 blocks;
+ * cluster variant with P = min(8, units that fit one wave at 3 CTAs per SM /
+ * units, longest table / 4 blocks) parts (P >= 2) while a part of the longest
+ * sequence stays at most 64 blocks;
  * else split-K when a sequence may span more than one partition and
  * `workspace` holds pkv_decode_workspace_bytes(...) bytes; else the cluster
  * variant (P >= 2) or the single pass.  pkv_decode_variant_for() and

@@ -189,12 +189,15 @@ int64_t decode_units(int num_seqs, int num_heads, int num_kv_heads) {
     return static_cast<int64_t>(num_seqs) * num_kv_heads * ((num_heads / num_kv_heads + 7) / 8);
 }
 
-// Cluster variant, automatic: parts per sequence so that the grid holds about
-// two waves of CTAs at three per SM, at most kMaxClusterParts, and at least
-// one block per consumer warp (4) in a part of the longest sequence.
+// Cluster variant, automatic: as many parts per sequence as keep the whole
+// grid resident at once (three CTAs per SM) -- a CTA that waits at the
+// cluster barrier for a peer still queued would hold its slot idle; measured:
+// 8 parts at batch 32 ran 2x slower than the single pass -- at most
+// kMaxClusterParts, and at least one block per consumer warp (4) in a part of
+// the longest sequence.
 int cluster_parts_auto(int64_t units, int max_blocks_per_seq) {
-    const int64_t target = 2 * 3 * static_cast<int64_t>(sm_count());
-    int64_t parts = (target + units - 1) / std::max<int64_t>(units, 1);
+    const int64_t slots = 3 * static_cast<int64_t>(sm_count());
+    int64_t parts = slots / std::max<int64_t>(units, 1);
     parts = std::min<int64_t>(parts, pkv::kMaxClusterParts);
     parts = std::min<int64_t>(parts, std::max(1, max_blocks_per_seq / 4));
     return static_cast<int>(std::max<int64_t>(parts, 1));

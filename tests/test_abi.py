@@ -146,16 +146,19 @@ def test_variant_choice_and_workspace_sizes():
     assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, 0) == pkv.DECODE_SINGLE
     assert pkv.decode_variant_for(B, hq, hkv, d, W, 512, 1 << 40) == pkv.DECODE_SINGLE
     # long context (8 sequences x 2048 blocks, 8 x 8 units): a cluster part would span
-    # 256 blocks, so split-K when the workspace holds its partials; the cluster
-    # variant (8 parts) without it
+    # 342 blocks, so split-K when the workspace holds its partials; the cluster
+    # variant (6 parts: 64 x 6 CTAs in one wave of 3 per SM) without it
     long_split = pkv.decode_workspace_bytes(8, 32, d, 2048)
     assert pkv.decode_variant_for(8, 32, 8, d, 2048, 512, long_split) == pkv.DECODE_SPLIT
     assert pkv.decode_variant_for(8, 32, 8, d, 2048, 512, long_split - 1) == pkv.DECODE_CLUSTER
-    assert pkv.decode_cluster_parts_for(8, 32, 8, d, 2048, pkv.DECODE_AUTO, 512, 0) == 8
-    # a few short sequences: the cluster variant, parts sized to about two waves
+    assert pkv.decode_cluster_parts_for(8, 32, 8, d, 2048, pkv.DECODE_AUTO, 512, 0) == 6
+    # one short sequence: the cluster variant, as many parts as one wave holds (<= 8)
     assert pkv.decode_variant_for(1, 32, 32, d, 128, 512, 0) == pkv.DECODE_CLUSTER
     assert pkv.decode_cluster_parts_for(1, 32, 32, d, 128, pkv.DECODE_AUTO, 512, 0) == 8
-    assert pkv.decode_cluster_parts_for(8, 32, 32, d, 128, pkv.DECODE_AUTO, 512, 0) == 4
+    assert pkv.decode_cluster_parts_for(4, 32, 32, d, 128, pkv.DECODE_AUTO, 512, 0) == 3
+    # 8 sequences (256 units) leave no room for two parts each in one wave: split-K
+    assert pkv.decode_cluster_parts_for(8, 32, 32, d, 128, pkv.DECODE_AUTO, 512, 0) == 0
+    assert pkv.decode_variant_for(8, 32, 32, d, 128, 512, 1 << 30) == pkv.DECODE_SPLIT
     # ... never more parts than a quarter of the longest table's blocks
     assert pkv.decode_cluster_parts_for(1, 32, 32, d, 12, pkv.DECODE_AUTO, 512, 0) == 3
     assert pkv.decode_variant_for(1, 32, 32, d, 4, 512, 1 << 30) == pkv.DECODE_SINGLE

@@ -11,6 +11,8 @@ must be the same bits -- a stale or misaddressed scratch would shift them.
 The output is also checked against the fp64 oracle with the tolerance of the
 parity tests, and the device's free memory must not change across a call.
 This file sorts last so that a failure here comes after every other test."""
+import gc
+
 import numpy as np
 import pytest
 import torch
@@ -69,6 +71,7 @@ def test_static_scratch_matches_regular_entry_twice_in_a_row(name, seed, kw, par
     assert rc == pkv.OK
     for call in range(2):  # the second call starts from the first call's scratch contents
         d.out.fill_(float("nan"))
+        gc.collect()  # tensors freed late by the collector would show as a drop below
         torch.cuda.synchronize()
         free_before = torch.cuda.mem_get_info()[0]
         held_before = torch.cuda.memory_allocated()
@@ -77,8 +80,8 @@ def test_static_scratch_matches_regular_entry_twice_in_a_row(name, seed, kw, par
         assert np.array_equal(got, want), f"call {call}: differs from the regular split-K entry"
         check_close(got, ref, f"static scratch {name}, call {call}")
         if call == 1:  # the first call may load the library's kernels; later calls take nothing
-            assert torch.cuda.mem_get_info()[0] == free_before
-            assert torch.cuda.memory_allocated() == held_before
+            assert torch.cuda.mem_get_info()[0] == free_before     # no cudaMalloc
+            assert torch.cuda.memory_allocated() <= held_before    # nothing through torch
     assert d.err_word() == 0
 
 
