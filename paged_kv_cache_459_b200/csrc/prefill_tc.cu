@@ -105,15 +105,28 @@ struct TcItem {
     int nk0, nk1;  // key tiles Q tile 0 / 1 can see (tile 1 may be empty: 0)
 };
 
-// Items are numbered z-major -- z counts 256-row tiles from the END of each
-// sequence, so low numbers see the most keys -- then sequence, then KV head.
+// z counts 256-row tiles from the END of each sequence, so low z sees the
+// most keys.  Items are numbered heaviest first in groups of kZGroup z levels:
+// group-major, then (sequence, KV head), then z within the group -- so the
+// items of one (sequence, head) that read nearly the same keys are dealt to
+// neighbouring CTAs, run at the same time and share their K/V tiles in L2,
+// while the order stays heaviest first.
+constexpr int kZGroup = 2;
+
+__device__ __forceinline__ void tc_item_coords(const PrefillParams &p, int i, int &z, int &b, int &kvh) {
+    const int per_group = kZGroup * p.Hkv * p.B;
+    const int zg = i / per_group, rem = i - zg * per_group;
+    const int pair = rem / kZGroup;
+    z = zg * kZGroup + (rem - pair * kZGroup);
+    b = pair / p.Hkv;
+    kvh = pair - b * p.Hkv;
+}
+
 // Returns false for items past a sequence's rows or of a sequence whose
 // lengths are inconsistent (*bad set for the latter).
 __device__ __forceinline__ bool tc_item(const PrefillParams &p, int i, TcItem &it, bool *bad) {
-    const int per_z = p.Hkv * p.B;
-    const int z = i / per_z, rem = i - z * per_z;
-    it.b = rem / p.Hkv;
-    it.kvh = rem - it.b * p.Hkv;
+    int z;
+    tc_item_coords(p, i, z, it.b, it.kvh);
     it.q0 = __ldg(p.query_start + it.b);
     const int nq = __ldg(p.query_start + it.b + 1) - it.q0;
     it.ctx = __ldg(p.seq_lens + it.b);
@@ -279,7 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0;; ++k) {
                 const int i = tc_item_index(k, blockIdx.x, gridDim.x);
                 if (i >= p.items) break;
-                if (i < p.Hkv * p.B && i % p.Hkv == 0) {
+                int z, b, kvh;
+                tc_item_coords(p, i, z, b, kvh);
+                if (z == 0 && kvh == 0) {
                     TcItem bad_it;
                     bool bad;
                     tc_item(p, i, bad_it, &bad);
@@ -656,7 +671,8 @@ cudaError_t launch_prefill_tc_d(const CUtensorMap &tmk, const CUtensorMap &tmv, 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const long long rows = static_cast<long long>(max_query_len) * p.group;
-    const long long items = (rows + kCtaRows - 1) / kCtaRows * p.Hkv * p.B;
+    const long long zlevels = (rows + kCtaRows - 1) / kCtaRows;
+    const long long items = (zlevels + kZGroup - 1) / kZGroup * kZGroup * p.Hkv * p.B;
     if (items == 0) return cudaSuccess;
     if (items > 0x7FFFFFFFLL - 2LL * num_sms) return cudaErrorInvalidValue;
     p.items = static_cast<int>(items);
