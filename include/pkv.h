@@ -163,7 +163,8 @@ PKV_API int pkv_decode_cluster_parts_for(int num_seqs, int num_heads, int num_kv
  * (query heads grouped contiguously over KV heads) and the same for V.
  * bf16 inputs, fp32 accumulation and softmax, bf16 output (round to nearest
  * even).  seq_lens[b] == 0 gives a zero row.  Table entries at or past
- * ceil(seq_lens[b] / 16) are never read.
+ * ceil(seq_lens[b] / 16) are never used: they may be read (every row holds
+ * max_blocks_per_seq entries) but are never taken as block numbers.
  *
  * head_dim: 64 or 128.  num_heads % num_kv_heads == 0.  Pointers 16-byte
  * aligned.  num_blocks * num_kv_heads * 16 must be < 2^31.

@@ -42,6 +42,26 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     const int h0_cta = WIDE ? (MMA ? by * NW * p.group : by * NW) : h0;
     const int heads_cta = WIDE ? NW * heads : heads;
 
+    // Round-robin: warp w takes blocks blk_begin + w, + NW, ...; wide: all of them.
+    constexpr int kStride = WIDE ? 1 : NW;
+    const int lead = WIDE ? 0 : warp;
+    // Block-table entries of this warp's blocks, 32 per lane-load.  Where the
+    // unit's first block does not depend on the length (no skipped prefix, not
+    // cluster mode), they are loaded now, beside the length, for every block
+    // the table row holds in this unit's range; entries past the sequence are
+    // read but never used.  Otherwise after the length, below.
+    const bool early_table = !CLUSTER && p.start_blocks == nullptr;
+    TableWindow tw;
+    tw.row = p.block_tables + static_cast<size_t>(b) * p.W;
+    tw.stride = kStride;
+    if (early_table) {
+        const int first_blk = part * p.part_blocks;
+        const int last_blk = min(p.W, first_blk + p.part_blocks);  // exclusive, within the row
+        tw.first = first_blk + lead;
+        tw.count = last_blk - tw.first > 0 ? (last_blk - tw.first + kStride - 1) / kStride : 0;
+        tw.init(lane);
+    }
+
     int len = __ldg(p.seq_lens + b);
     if (len < 0 || len > p.W * kBlockTokens) {
         if (threadIdx.x == 0 && part == 0 && by == 0) flag(p.err, PKV_DEV_ERR_BAD_LEN);
@@ -87,16 +107,12 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     }
     __syncthreads();
 
-    // Round-robin: warp w takes blocks blk_begin + w, + NW, ...; wide: all of them.
-    constexpr int kStride = WIDE ? 1 : NW;
-    const int lead = WIDE ? 0 : warp;
     const int n_mine = blk_end - blk_begin > lead ? (blk_end - blk_begin - lead + kStride - 1) / kStride : 0;
-    TableWindow tw;
-    tw.row = p.block_tables + static_cast<size_t>(b) * p.W;
-    tw.first = blk_begin + lead;
-    tw.stride = kStride;
-    tw.count = n_mine;
-    tw.init(lane);
+    if (!early_table) {
+        tw.first = blk_begin + lead;
+        tw.count = n_mine;
+        tw.init(lane);
+    }
     const uint64_t policy = l2_policy_evict_first();
     const int y_head = kvh * kBlockTokens;
 
