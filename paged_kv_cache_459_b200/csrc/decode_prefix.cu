@@ -265,20 +265,22 @@ struct PrefixTcGeometry {
     static constexpr int kMeta = 64;                    // 3 mbarriers, TMEM base, keep bits x 2
     static constexpr int kSmemBytes = 2 * kKV + kQ + kMeta + 1024;
     static constexpr int kTmemCols = 256;               // S (P over its first half) | O
-    static_assert(kKeys == 128 && CB <= 32, "chunk layout");
+    static_assert(kKeys % 64 == 0 && kKeys <= 128 && CB <= 32, "chunk layout");
     static_assert(kKeys + D <= kTmemCols, "tensor memory columns");
 };
 
 // Prefix range c of group g's shared prefix -- chunks [c * RC, (c + 1) * RC)
-// of CB blocks each, RC = p.range_chunks -- for KV head kvh, on the tcgen05
+// of CB blocks each, RC = p.range_blocks / CB -- for KV head kvh, on the tcgen05
 // tensor cores.  The rows, (member, query head) pairs, go in tiles of 128,
 // one row per thread (= TMEM lane); for each row tile the range's chunks run
 // one after another with an online softmax:
-//   S[128 x 128] = Q K^T          tcgen05.mma, Q tile and K chunk in shared memory
+//   S[128 x 16 CB] = Q K^T        tcgen05.mma, Q tile and K chunk in shared memory
 //   m = running row max (moved only when it grows by more than 2^8),
 //   P = 2^(S * scale - m) as bf16 into TMEM over S, l += sum P,
 //   O in TMEM rescaled by 2^(m_old - m) when the max moves
 //   O[128 x d] (+)= P V           tcgen05.mma, P from TMEM, V chunk in shared memory
+// (chunks of 4 blocks keep the CTA's shared memory -- K chunk, V chunk, Q
+// tile -- near a suffix CTA's, so that a prefix CTA displaces one of them)
 // and leaves one partial (m, l, O) per row for the range.  The next chunk's K
 // is loaded as soon as S has read this one, its V as soon as P.V has, so the
 // loads overlap the softmax.  Keys of blocks past the prefix or with a bad
@@ -306,7 +308,8 @@ __device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CU
     int len0 = __ldg(p.seq_lens + b0);
     len0 = len0 < 0 ? 0 : min(len0, p.W * kBlockTokens);
     const int nb = min(max(__ldg(p.prefix_blocks + b0), 0), len0 / kBlockTokens);  // full blocks
-    const int c0 = c * p.range_chunks, c1 = min((nb + CB - 1) / CB, c0 + p.range_chunks);
+    const int rc = p.range_blocks / CB;  // chunks per range
+    const int c0 = c * rc, c1 = min((nb + CB - 1) / CB, c0 + rc);
     if (c0 >= c1) return;
     const int nc = c1 - c0;          // chunks of the range
     const int G = p.group;           // query heads per KV head
@@ -554,7 +557,7 @@ __device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CU
     if (warp == 1) tc::dealloc<Geo::kTmemCols>(tmem);
 }
 
-// Merge of one (sequence, query head): prefix ranges [0, ceil(pb / (CB * RC))) and
+// Merge of one (sequence, query head): prefix slots [0, ceil(pb / range_blocks)) and
 // the suffix split-K partitions that hold tokens past the prefix (counted
 // from the prefix end), in slot order, by log-sum-exp.  As in the split-K
 // merge: all (m, l) read at once, weights computed once, output loads batched.
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
     len = len < 0 ? 0 : min(len, p.W * kBlockTokens);
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
     const int pb = min(max(__ldg(p.prefix_blocks + b), 0), len / kBlockTokens);
-    const int nchunks = (pb + CB * p.range_chunks - 1) / (CB * p.range_chunks);  // prefix slots
+    const int nchunks = (pb + p.range_blocks - 1) / p.range_blocks;  // prefix slots
     // suffix partitions with tokens, at most those the launch computed (a
     // longer suffix was flagged by the cascade kernel)
     const int ntot = nchunks + min((nblk - pb + p.part_blocks - 1) / p.part_blocks,
@@ -632,7 +635,7 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
     const int c = id % pp.prefix_parts;
     id /= pp.prefix_parts;
     if constexpr (TC)
-        prefix_range_tc<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
+        prefix_range_tc<D, kPrefixTcChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
     else
         prefix_unit_mma<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
 }
@@ -674,7 +677,7 @@ cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, con
     if (n_pre >= (1ll << 31) || n_suf >= (1ll << 31)) return cudaErrorInvalidValue;
     cudaError_t e;
     if (n_pre > 0) {
-        constexpr int kPre = TC ? PrefixTcGeometry<D, kPrefixChunkBlocks>::kSmemBytes
+        constexpr int kPre = TC ? PrefixTcGeometry<D, kPrefixTcChunkBlocks>::kSmemBytes
                                 : PrefixMmaGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
         auto pre = cascade_prefix_kernel<D, TC>;
         if ((e = cudaFuncSetAttribute(pre, cudaFuncAttributeMaxDynamicSharedMemorySize, kPre)) != cudaSuccess)

@@ -72,7 +72,8 @@ cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const 
 
 // Shared-prefix (cascade) decode: prefix blocks read once per (group, KV
 // head) by a dense tensor-core kernel; suffixes by split-K; LSE merge.
-constexpr int kPrefixChunkBlocks = 8;  // prefix blocks per chunk (one 128-key tile)
+constexpr int kPrefixChunkBlocks = 8;    // prefix blocks per chunk on mma.sync (128 keys)
+constexpr int kPrefixTcChunkBlocks = 4;  // prefix blocks per chunk on tcgen05 (64 keys)
 
 struct PrefixParams {
     __nv_bfloat16 *out;
@@ -89,7 +90,7 @@ struct PrefixParams {
     int W, B, Hq, Hkv, group;
     int ws_parts;      // prefix_parts + suffix partitions
     int prefix_parts;  // prefix ranges per (group, KV head): slots 0.. hold their partials
-    int range_chunks;  // chunks of kPrefixChunkBlocks blocks per prefix range (1 on mma.sync)
+    int range_blocks;  // prefix blocks per slot: a chunk (mma.sync) or a range of chunks (tcgen05)
     int part_blocks;   // suffix split-K partition (blocks)
     float scale_log2;
 };

@@ -421,9 +421,11 @@ size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_d
     if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0) return 0;
     if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
     if (partition_tokens % PKV_BLOCK_TOKENS) return 0;
+    // suffix partitions + prefix slots (at most one per chunk of the smaller chunk size)
+    const int chunk = std::min(pkv::kPrefixChunkBlocks, pkv::kPrefixTcChunkBlocks);
     const size_t parts =
         static_cast<size_t>(num_parts_for(max_blocks_per_seq, partition_tokens)) +
-        (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+        (max_blocks_per_seq + chunk - 1) / chunk;
     return static_cast<size_t>(num_seqs) * num_heads * parts * (static_cast<size_t>(head_dim) + 2) *
            sizeof(float);
 }
@@ -472,13 +474,14 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
                                   ? max_suffix_blocks
                                   : max_blocks_per_seq;
     const int suffix_parts = num_parts_for(suffix_blocks, partition_tokens);
-    // Prefix work: 8-block chunks; on tcgen05 each CTA takes a range of
-    // chunks with O held in TMEM across them, sized so that the prefix grid
-    // is about 64 CTAs (the (group, KV head, 128-row tile, chunk) steps spread
+    // Prefix work: 8-block chunks on mma.sync, one per CTA; 4-block chunks on
+    // tcgen05, each CTA taking a range of them with O held in TMEM across
+    // the range, sized so that the prefix grid is about 64 CTAs (the (group, KV head, 128-row tile, chunk) steps spread
     // evenly, rows per group estimated from an even split of the batch); on
     // mma.sync one chunk per CTA.
     const bool prefix_tc = env_int("PKV_CASCADE_TC", 0) != 0;
-    const int chunks = (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+    const int chunk_blocks = prefix_tc ? pkv::kPrefixTcChunkBlocks : pkv::kPrefixChunkBlocks;
+    const int chunks = (max_blocks_per_seq + chunk_blocks - 1) / chunk_blocks;
     int range_chunks = 1;
     if (prefix_tc) {
         const int64_t groups = std::max(num_groups, 1);
@@ -515,7 +518,7 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     pp.group = num_heads / num_kv_heads;
     pp.ws_parts = prefix_parts + suffix_parts;
     pp.prefix_parts = prefix_parts;
-    pp.range_chunks = range_chunks;
+    pp.range_blocks = range_chunks * chunk_blocks;
     pp.part_blocks = partition_tokens / PKV_BLOCK_TOKENS;
     pp.scale_log2 = scale * 1.4426950408889634f;
 
