@@ -45,6 +45,10 @@ constexpr int kSoftmaxWarps = kTiles * 2 * kWarpsPerTile;  // two warpgroups (ke
 constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 16 score pairs a softmax thread turns into P, this many take 2^x
+// on the FMA pipe (exp2_fma2) instead of the special-function unit, which
+// the two Q tiles' softmaxes otherwise share.
+constexpr int kFmaExpPairs = 0;
 
 // ------------------------------------------------ packed f32x2 arithmetic
 // Two floats in one 64-bit register pair for the sm_100 f32x2 instructions.
@@ -66,6 +70,34 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for two values on the FMA pipe instead of the special-function unit:
+// 2^x = 2^floor(x) * 2^f, f in [0, 1), with 2^f from a cubic fitted here to
+// 2^f on [0, 1) by least squares on the relative error (largest relative
+// error 2.2e-4, under the bf16 rounding of P); the integer part is added to
+// the exponent bits.  x is clamped at -126 (2^-126 instead of 0 below it);
+// the softmax never passes more than +8.
+__device__ __forceinline__ void exp2_fma2(float &a, float &b) {
+    constexpr float c0 = 0.99998891353607178f, c1 = 0.69449967145919800f;
+    constexpr float c2 = 0.23030571639537811f, c3 = 0.07476584613323212f;
+    a = fmaxf(a, -126.f);
+    b = fmaxf(b, -126.f);
+    const float fa = floorf(a), fb = floorf(b);
+    const uint64_t f = fsub2(f2pack(a, b), f2pack(fa, fb));
+    uint64_t p = ffma2(f2pack(c3, c3), f, f2pack(c2, c2));
+    p = ffma2(p, f, f2pack(c1, c1));
+    p = ffma2(p, f, f2pack(c0, c0));
+    float pa, pb;
+    f2unpack(p, pa, pb);
+    a = __uint_as_float(__float_as_uint(pa) + (static_cast<uint32_t>(static_cast<int>(fa)) << 23));
+    b = __uint_as_float(__float_as_uint(pb) + (static_cast<uint32_t>(static_cast<int>(fb)) << 23));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -560,8 +592,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < 32; c += 2) {  // scale and shift two at a time, 2^x on the SFU
                         float a, bb;
                         f2unpack(ffma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), scale2, nbase2), a, bb);
-                        a = ex2_approx(a);
-                        bb = ex2_approx(bb);
+                        if ((c >> 1) % 16 < kFmaExpPairs) {
+                            exp2_fma2(a, bb);
+                        } else {
+                            a = ex2_approx(a);
+                            bb = ex2_approx(bb);
+                        }
                         sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], f2pack(a, bb));
                         __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
                         pk[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
