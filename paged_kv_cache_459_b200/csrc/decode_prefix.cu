@@ -371,6 +371,12 @@ __device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CU
     tc::fence_before();
     __syncthreads();  // barriers, keep bits and the TMEM base
     tc::fence_after();
+    // Only now may the suffix grid launch: every prefix CTA holds its TMEM
+    // before any suffix or merge CTA exists.  (A co-resident CTA that keeps
+    // its right to allocate can hold up tcgen05.alloc, and suffix CTAs wait
+    // for this grid before they exit: allocating after them could wait for
+    // ever.)
+    pdl_launch_dependents();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // this thread's lane
 
@@ -622,15 +628,17 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
 
 // The prefix grid: CTA k is prefix range k % prefix_parts of KV head
 // (k / prefix_parts) % Hkv of group k / (prefix_parts * Hkv).  It lets the
-// suffix grid, launched after it as a programmatic dependent, start at once:
+// suffix grid, launched after it as a programmatic dependent, start early:
 // the two run side by side, the short tensor-core prefix work beside the
 // bandwidth-bound suffix stream.  TC: ranges on tcgen05 (else one chunk per
-// CTA on mma.sync).
+// CTA on mma.sync); a tcgen05 CTA lets the suffix grid launch only once it
+// holds its tensor memory (in prefix_range_tc), a CTA without prefix work by
+// exiting.
 template <int D, bool TC>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_prefix_kernel(const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv, const PrefixParams pp) {
-    pdl_launch_dependents();
+    if constexpr (!TC) pdl_launch_dependents();
     int id = blockIdx.x;
     const int c = id % pp.prefix_parts;
     id /= pp.prefix_parts;
@@ -651,6 +659,9 @@ template <int D, bool MMA, bool WIDE>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_suffix_kernel(const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv, const DecodeParams dp) {
+    // These CTAs use no tensor memory: they give up the right to allocate at
+    // once, so that they can never hold up a tcgen05.alloc on their SM.
+    if (threadIdx.x < 32) tc::relinquish();
     int id = blockIdx.x;
     const int ny = (MMA ? dp.Hkv * dp.chunks : dp.Hq) / (WIDE ? kPrefixWarps : 1);
     const int part = id % dp.num_parts;
