@@ -611,14 +611,8 @@ def workload_key(args, name, *, dev, cascade=False, batch=None, clocks=True) -> 
             cmp["tcgen05_step_us"] = 1e3 * _events_time(r.step, args.steps, 3)
         finally:
             os.environ.pop("PKV_CASCADE_TC")
-        os.environ["PKV_CASCADE_WIDE"] = "0"
-        try:
-            cmp["narrow_suffix_step_us"] = 1e3 * _events_time(r.step, args.steps, 3)
-        finally:
-            os.environ.pop("PKV_CASCADE_WIDE")
-        cmp["how"] = ("K steps back to back between two events: the default prefix chunks and "
-                      "suffix units, then PKV_CASCADE_TC=1 (tcgen05 prefix chunks), then "
-                      "PKV_CASCADE_WIDE=0 (one head segment per suffix CTA)")
+        cmp["how"] = ("K steps back to back between two events: the default prefix chunks, then "
+                      "PKV_CASCADE_TC=1 (tcgen05 prefix chunks)")
         out["prefix_paths"] = cmp
     del r
     torch.cuda.empty_cache()

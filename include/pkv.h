@@ -287,23 +287,13 @@ PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, c
  * prefix_blocks[b] = 0.  The group's shared block ids are read from its first
  * member's table row.  pkv_alloc_prefix_groups builds all three arrays from
  * the allocator's state.  All five arrays are device int32.
- * Work: three launches on the stream.  A tensor-core kernel computes each
- * group's prefix attention (queries of all members x heads as MMA rows) in
- * chunks of 8 blocks; the split-K kernel (partition_tokens, <= 0: 512),
- * launched as its programmatic dependent so that the two run side by side,
- * covers each sequence past its prefix; a merge kernel combines the
- * partials.  The prefix runs on warp-level mma.sync, one chunk per CTA, by
- * default; the environment variable PKV_CASCADE_TC=1 selects tcgen05 MMAs
- * instead, each CTA taking a range of chunks with its output accumulated in
- * tensor memory across them (range length chosen from the sizes, or forced
- * with PKV_CASCADE_RANGE_CHUNKS=n; same results up to fp32 rounding order).  The
- * suffix units cover one head segment each, or -- "wide" units -- 4 head
- * segments of a sequence with one warp streaming each segment's suffix alone
- * (suffixes are short); wide units are used when the segments (query heads,
- * or KV heads with at most 8 query heads each) come in groups of 4 and the
- * wide grid still holds two waves of CTAs at 3 per SM.  The environment
- * variable PKV_CASCADE_WIDE=0 or =1 turns them off, or on wherever the heads
- * allow (same results up to fp32 rounding order).  Workspace:
+ * Work: a tensor-core kernel computes each group's prefix attention in
+ * chunks of 8 blocks (queries of all members x heads as MMA rows); the
+ * split-K kernel (partition_tokens, <= 0: 512) covers each sequence past its
+ * prefix; a merge kernel combines the partials.  The prefix chunks run on
+ * warp-level mma.sync by default; the environment variable PKV_CASCADE_TC=1
+ * selects tcgen05 MMAs with TMEM accumulators instead (same results up to
+ * fp32 rounding order).  Workspace:
  * pkv_decode_prefix_workspace_bytes(...), else PKV_ERR_WORKSPACE.
  * max_suffix_blocks: an upper bound on ceil(len / 16) - prefix_blocks over the
  * batch (the blocks past each sequence's prefix), or <= 0 for "unknown"

@@ -261,35 +261,30 @@ template <int D, int CB>
 struct PrefixTcGeometry {
     static constexpr int kKeys = CB * kBlockTokens;     // keys of one chunk: MMA N of S, K of P.V
     static constexpr int kKV = (D / 64) * kKeys * 128;  // one K or V chunk [d half][key][128 B]
-    static constexpr int kQ = (D / 64) * 128 * 128;     // one 128-row Q tile [d half][row][128 B]
-    static constexpr int kMeta = 64;                    // 3 mbarriers, TMEM base, keep bits x 2
-    static constexpr int kSmemBytes = 2 * kKV + kQ + kMeta + 1024;
-    static constexpr int kTmemCols = 256;               // S (P over its first half) | O
-    static_assert(kKeys % 64 == 0 && kKeys <= 128 && CB <= 32, "chunk layout");
+    static constexpr int kMeta = 64;                    // 3 mbarriers, TMEM base, valid[CB]
+    static constexpr int kSmemBytes = 2 * kKV + kMeta + 1024;
+    static constexpr int kTmemCols = 256;               // S (P over its first half) | O (Q before it)
+    static_assert(kKeys == 128 && 32 + 4 * CB <= kMeta, "chunk layout");
     static_assert(kKeys + D <= kTmemCols, "tensor memory columns");
 };
 
-// Prefix range c of group g's shared prefix -- chunks [c * RC, (c + 1) * RC)
-// of CB blocks each, RC = p.range_blocks / CB -- for KV head kvh, on the tcgen05
-// tensor cores.  The rows, (member, query head) pairs, go in tiles of 128,
-// one row per thread (= TMEM lane); for each row tile the range's chunks run
-// one after another with an online softmax:
-//   S[128 x 16 CB] = Q K^T        tcgen05.mma, Q tile and K chunk in shared memory
-//   m = running row max (moved only when it grows by more than 2^8),
-//   P = 2^(S * scale - m) as bf16 into TMEM over S, l += sum P,
-//   O in TMEM rescaled by 2^(m_old - m) when the max moves
-//   O[128 x d] (+)= P V           tcgen05.mma, P from TMEM, V chunk in shared memory
-// (chunks of 4 blocks keep the CTA's shared memory -- K chunk, V chunk, Q
-// tile -- near a suffix CTA's, so that a prefix CTA displaces one of them)
-// and leaves one partial (m, l, O) per row for the range.  The next chunk's K
-// is loaded as soon as S has read this one, its V as soon as P.V has, so the
-// loads overlap the softmax.  Keys of blocks past the prefix or with a bad
-// table entry load as zeros (a row past the tensor) and are masked.  Every
-// wait is bounded; on a timeout the CTA flags it, waits (bounded) for its
-// copies and MMAs, and frees its TMEM.
+// Prefix chunk c (blocks [c*CB, (c+1)*CB) of group g's shared prefix) for KV
+// head kvh on the tcgen05 tensor cores.  The chunk's K and V (128 keys) are
+// loaded once by TMA; the rows, (member, query head) pairs, go in tiles of
+// 128, one row per thread (= TMEM lane).  Per row tile:
+//   Q rows (bf16) -> TMEM, in O's columns (O is not written before P.V)
+//   S[128 x 128] = Q K^T    tcgen05.mma, A from TMEM, K from shared memory
+//   m = max S * scale, P = 2^(S * scale - m) as bf16 into TMEM over S,
+//   l = sum P (fp32)
+//   O[128 x d]   = P V      tcgen05.mma, A from TMEM, V from shared memory
+// and the row's partial (m, l, O) goes to its workspace slot.  A chunk is one
+// key tile, so the softmax is a single pass with no running max.  Keys of
+// blocks past the prefix or with a bad table entry are loaded as zeros (a row
+// past the tensor) and masked to -inf.  Every wait is bounded; on a timeout the
+// CTA flags it, waits (bounded) for its copies and MMAs, and frees its TMEM.
 template <int D, int CB>
-__device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CUtensorMap &tmv,
-                                                const PrefixParams &p, int c, int kvh, int g) {
+__device__ __forceinline__ void prefix_unit_tc(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                            const PrefixParams &p, int c, int kvh, int g) {
     using Geo = PrefixTcGeometry<D, CB>;
     constexpr int kKeys = Geo::kKeys;
     constexpr int kColS = 0, kColO = kKeys;  // TMEM columns
@@ -308,54 +303,18 @@ __device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CU
     int len0 = __ldg(p.seq_lens + b0);
     len0 = len0 < 0 ? 0 : min(len0, p.W * kBlockTokens);
     const int nb = min(max(__ldg(p.prefix_blocks + b0), 0), len0 / kBlockTokens);  // full blocks
-    const int rc = p.range_blocks / CB;  // chunks per range
-    const int c0 = c * rc, c1 = min((nb + CB - 1) / CB, c0 + rc);
-    if (c0 >= c1) return;
-    const int nc = c1 - c0;          // chunks of the range
-    const int G = p.group;           // query heads per KV head
-    const int R = members * G;       // rows of this group and KV head
-    const int steps = ((R + 127) / 128) * nc;  // (row tile, chunk), chunk fastest
+    const int j0 = c * CB, j1 = min(nb, j0 + CB);
+    if (j0 >= j1) return;
+    const int nt = j1 - j0;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t k_smem = smem_u32(smem), v_smem = smem_u32(smem + Geo::kKV);
-    uint8_t *q_tile = smem + 2 * Geo::kKV;
-    uint8_t *meta = q_tile + Geo::kQ;
-    const uint32_t k_bar = smem_u32(meta);  // a K chunk landed
-    const uint32_t v_bar = k_bar + 8;       // a V chunk landed
-    const uint32_t m_bar = k_bar + 16;      // the MMAs issued so far are done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(meta + 24);
-    volatile uint32_t *keep_bits = reinterpret_cast<volatile uint32_t *>(meta + 32);  // [2], by step parity
-
-    const int32_t *trow = p.block_tables + static_cast<size_t>(b0) * p.W;
-    // Thread 0: the TMA loads of chunk `ch` into one buffer; bit i of the
-    // return value: block i of the chunk is there.
-    const auto load_chunk = [&](int ch, uint32_t dst, uint32_t bar, const CUtensorMap *tm) {
-        const int j0 = ch * CB;
-        uint32_t keep = 0;
-        mbar_arrive_expect_tx(bar, Geo::kKV);
-        const uint64_t policy = l2_policy_evict_first();
-        const long long y_none = p.num_blocks * p.Hkv * kBlockTokens;  // past the tensor: zeros
-#pragma unroll 1
-        for (int i = 0; i < CB; ++i) {
-            long long y = y_none;
-            if (j0 + i < nb) {
-                const int32_t phys = __ldg(trow + j0 + i);
-                if (phys >= 0 && phys < p.num_blocks) {
-                    y = (static_cast<long long>(phys) * p.Hkv + kvh) * kBlockTokens;
-                    keep |= 1u << i;
-                } else if (tm == &tmk) {
-                    flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
-                }
-            }
-#pragma unroll
-            for (int hh = 0; hh < D / 64; ++hh)
-                tma_load_2d(dst + hh * (kKeys * 128) + i * (kBlockTokens * 128), tm, hh * 64,
-                            static_cast<int>(y), bar, policy);
-        }
-        return keep;
-    };
-    const auto chunk_of = [&](int st) { return c0 + st % nc; };
+    const uint32_t k_bar = smem_u32(smem + 2 * Geo::kKV);  // K landed
+    const uint32_t v_bar = k_bar + 8;                       // V landed
+    const uint32_t m_bar = k_bar + 16;                      // the MMAs issued so far are done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 2 * Geo::kKV + 24);
+    int *valid = reinterpret_cast<int *>(smem + 2 * Geo::kKV + 32);  // [CB]
 
     if (t == 0) {
         mbar_init(k_bar, 1);
@@ -364,61 +323,84 @@ __device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CU
         fence_mbar_init();
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
-        keep_bits[0] = load_chunk(c0, k_smem, k_bar, &tmk);
-        load_chunk(c0, v_smem, v_bar, &tmv);
+        const int32_t *row = p.block_tables + static_cast<size_t>(b0) * p.W;
+        const int y_none = static_cast<int>(p.num_blocks * p.Hkv * kBlockTokens);  // past the tensor: zeros
+        int y[CB];
+#pragma unroll
+        for (int i = 0; i < CB; ++i) {
+            valid[i] = -1;
+            y[i] = y_none;
+            if (i < nt) {
+                const int32_t phys = __ldg(row + j0 + i);
+                if (phys >= 0 && phys < p.num_blocks) {
+                    valid[i] = phys;
+                    y[i] = (phys * p.Hkv + kvh) * kBlockTokens;
+                } else {
+                    flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
+                }
+            }
+        }
+        const uint64_t policy = l2_policy_evict_first();
+        // [d half][key][128 B]: key k of half hh at hh * 128 keys * 128 B + k * 128 B
+        mbar_arrive_expect_tx(k_bar, Geo::kKV);
+#pragma unroll
+        for (int i = 0; i < CB; ++i)
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh)
+                tma_load_2d(k_smem + hh * (kKeys * 128) + i * (kBlockTokens * 128), &tmk, hh * 64, y[i], k_bar,
+                            policy);
+        mbar_arrive_expect_tx(v_bar, Geo::kKV);
+#pragma unroll
+        for (int i = 0; i < CB; ++i)
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh)
+                tma_load_2d(v_smem + hh * (kKeys * 128) + i * (kBlockTokens * 128), &tmv, hh * 64, y[i], v_bar,
+                            policy);
     }
     if (warp == 1) tc::alloc<Geo::kTmemCols>(smem_u32(tmem_slot));  // beside thread 0's TMA issue
     tc::fence_before();
-    __syncthreads();  // barriers, keep bits and the TMEM base
+    __syncthreads();  // barriers, valid[] and the TMEM base
     tc::fence_after();
-    // Only now may the suffix grid launch: every prefix CTA holds its TMEM
-    // before any suffix or merge CTA exists.  (A co-resident CTA that keeps
-    // its right to allocate can hold up tcgen05.alloc, and suffix CTAs wait
-    // for this grid before they exit: allocating after them could wait for
-    // ever.)
-    pdl_launch_dependents();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // this thread's lane
-
-    bool ok = true;
-    bool mma_pending = false;  // an MMA batch committed to m_bar and not yet seen done
-    uint32_t m_phase = 0;
-    int k_issued = 1, k_done = 0, v_issued = 1, v_done = 0;  // chunk loads per buffer (thread 0's view)
-    int b = -1, h = 0;  // this thread's row of the current row tile
-    float m_run = -INFINITY, l_run = 0.f;
-    for (int st = 0; st < steps && ok; ++st) {
-        const int ci = st % nc;  // chunk index within the range
-        const int ch = c0 + ci;
-        const bool new_k = st == 0 || ch != chunk_of(st - 1);  // a load was issued for this step
-        const bool new_v = new_k;
-        if (ci == 0) {
-            // A new row tile: this thread's Q row into the swizzled Q tile (the
-            // S product that read the previous tile is done), zeros for rows
-            // without a sequence.
-            const int r = (st / nc) * 128 + t;
-            b = -1;
-            h = 0;
-            if (r < R) {
-                const int bb = __ldg(p.group_seqs + off + r / G);
-                if (bb >= 0 && bb < p.B) {
-                    b = bb;
-                    h = kvh * G + r % G;
-                }
-            }
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.q + (static_cast<size_t>(b < 0 ? 0 : b) * p.Hq + h) * D);
-            uint8_t *qrow = q_tile + t * 128;
+    uint32_t keep = 0;  // bit i: block i of the chunk is there
 #pragma unroll
-            for (int cc = 0; cc < D / 8; ++cc) {
-                const uint4 v = b >= 0 ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4 *>(qrow + (cc >> 3) * (128 * 128) + (((cc & 7) ^ (t & 7)) << 4)) = v;
+    for (int i = 0; i < CB; ++i) keep |= (valid[i] >= 0 ? 1u : 0u) << i;
+
+    const int G = p.group;      // query heads per KV head
+    const int R = members * G;  // rows of this group and KV head
+    bool ok = true;
+    bool mma_pending = false;   // an MMA batch committed to m_bar and not yet seen done
+    uint32_t phase = 0;         // m_bar phase
+    for (int r0 = 0; r0 < R; r0 += 128) {
+        const int r = r0 + t;
+        int b = -1, h = 0;
+        if (r < R) {
+            const int bb = __ldg(p.group_seqs + off + r / G);
+            if (bb >= 0 && bb < p.B) {
+                b = bb;
+                h = kvh * G + r % G;
             }
-            fence_proxy_async_smem();  // the generic-proxy stores, before the MMA's reads
-            m_run = -INFINITY;
-            l_run = 0.f;
         }
-        const bool k_ok = !new_k || mbar_wait(k_bar, static_cast<uint32_t>(k_done & 1), kWaitLimitNs);
-        if (new_k && k_ok) ++k_done;
+        // Q row -> TMEM columns [kColO, kColO + D / 2), zeros for rows without
+        // a sequence; all of the row's loads in flight before the stores
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.q + (static_cast<size_t>(b < 0 ? 0 : b) * p.Hq + h) * D);
+            uint32_t w[D / 2];
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                const uint4 v = b >= 0 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+                w[4 * i] = v.x;
+                w[4 * i + 1] = v.y;
+                w[4 * i + 2] = v.z;
+                w[4 * i + 3] = v.w;
+            }
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) tc::st32(lane_base + kColO + 32 * cc, w + 32 * cc);
+            tc::wait_st();
+        }
+        tc::fence_before();
+        const bool k_ok = r0 > 0 || mbar_wait(k_bar, 0, kWaitLimitNs);
         if (__syncthreads_or(!k_ok)) {
             ok = false;
             break;
@@ -426,136 +408,136 @@ __device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CU
         tc::fence_after();
         if (t == 0) {  // S = Q K^T
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const int hh = k >> 2, kk = k & 3;
-                tc::mma_ss(tmem + kColS,
-                           tc::smem_desc(smem_u32(q_tile) + hh * (128 * 128) + kk * 32, 16, 1024),
-                           tc::smem_desc(k_smem + hh * (kKeys * 128) + kk * 32, 16, 1024), kIdS, k > 0);
-            }
+            for (int k = 0; k < D / 16; ++k)
+                tc::mma_ts(tmem + kColS, tmem + kColO + 8 * k,
+                           tc::smem_desc(k_smem + (k >> 2) * (kKeys * 128) + (k & 3) * 32, 16, 1024), kIdS, k > 0);
             tc::commit(m_bar);
         }
         mma_pending = true;
-        if (__syncthreads_or(!mbar_wait(m_bar, m_phase, kWaitLimitNs))) {
+        if (__syncthreads_or(!mbar_wait(m_bar, phase, kWaitLimitNs))) {
             ok = false;
             break;
         }
         mma_pending = false;
-        m_phase ^= 1;
+        phase ^= 1;
         tc::fence_after();
-        // S has read this K chunk: the next step's K may come in now
-        if (st + 1 < steps && chunk_of(st + 1) != ch) {
-            if (t == 0) keep_bits[(st + 1) & 1] = load_chunk(chunk_of(st + 1), k_smem, k_bar, &tmk);
-            ++k_issued;
-        } else if (t == 0 && st + 1 < steps) {
-            keep_bits[(st + 1) & 1] = keep_bits[st & 1];
-        }
-        const uint32_t keep = keep_bits[st & 1];
 
         // softmax of the row, two passes over S (64 columns at a time): max, then P
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // one chain per block of 16
 #pragma unroll 1
         for (int hf = 0; hf < kKeys / 64; ++hf) {
-            uint32_t sv[64];
-            tc::ld32(lane_base + kColS + 64 * hf, sv);
-            tc::ld32(lane_base + kColS + 64 * hf + 32, sv + 32);
+            uint32_t s[64];
+            tc::ld32(lane_base + kColS + 64 * hf, s);
+            tc::ld32(lane_base + kColS + 64 * hf + 32, s + 32);
             tc::wait_ld();
 #pragma unroll
             for (int i = 0; i < 64; ++i)
                 if (keep >> (4 * hf + i / kBlockTokens) & 1u)
-                    mx4[i / kBlockTokens] = fmaxf(mx4[i / kBlockTokens], __uint_as_float(sv[i]) * p.scale_log2);
+                    mx4[i / kBlockTokens] = fmaxf(mx4[i / kBlockTokens], __uint_as_float(s[i]) * p.scale_log2);
         }
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        const bool grow = mx > m_run + kLazyRescale || (m_run == -INFINITY && mx != -INFINITY);
-        const float m_new = grow ? mx : m_run;
-        const float nbase = m_new == -INFINITY ? 0.f : m_new;
+        const float nbase = mx == -INFINITY ? 0.f : mx;
         float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
         for (int hf = 0; hf < kKeys / 64; ++hf) {
-            uint32_t sv[64];
-            tc::ld32(lane_base + kColS + 64 * hf, sv);
-            tc::ld32(lane_base + kColS + 64 * hf + 32, sv + 32);
+            uint32_t s[64];
+            tc::ld32(lane_base + kColS + 64 * hf, s);
+            tc::ld32(lane_base + kColS + 64 * hf + 32, s + 32);
             tc::wait_ld();
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
                 const bool there = keep >> (4 * hf + i / kBlockTokens) & 1u;  // i, i + 1: one block
-                const float p0 = there ? ex2_approx(fmaf(__uint_as_float(sv[i]), p.scale_log2, -nbase)) : 0.f;
-                const float p1 = there ? ex2_approx(fmaf(__uint_as_float(sv[i + 1]), p.scale_log2, -nbase)) : 0.f;
+                const float p0 = there ? ex2_approx(fmaf(__uint_as_float(s[i]), p.scale_log2, -nbase)) : 0.f;
+                const float p1 = there ? ex2_approx(fmaf(__uint_as_float(s[i + 1]), p.scale_log2, -nbase)) : 0.f;
                 l4[i / kBlockTokens] += p0 + p1;
                 pk[i / 2] = pack_bf16x2(p0, p1);
             }
             tc::st32(lane_base + kColS + 32 * hf, pk);  // P columns over S columns already read
         }
-        const float alpha = (ci > 0 && grow && m_run != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {  // O of the earlier chunks, to the new max
-#pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                tc::ld32(lane_base + kColO + 32 * cc, o);
-                tc::wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                tc::st32(lane_base + kColO + 32 * cc, o);
-            }
-        }
-        l_run = l_run * alpha + ((l4[0] + l4[1]) + (l4[2] + l4[3]));
-        m_run = m_new;
+        const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
         tc::wait_st();
         tc::fence_before();
-        const bool v_ok = !new_v || mbar_wait(v_bar, static_cast<uint32_t>(v_done & 1), kWaitLimitNs);
-        if (new_v && v_ok) ++v_done;
+        const bool v_ok = r0 > 0 || mbar_wait(v_bar, 0, kWaitLimitNs);
         if (__syncthreads_or(!v_ok)) {
             ok = false;
             break;
         }
         tc::fence_after();
-        if (t == 0) {  // O (+)= P V (V MN-major: d contiguous)
+        if (t == 0) {  // O = P V (V MN-major: d contiguous)
 #pragma unroll
             for (int k = 0; k < kKeys / 16; ++k)
                 tc::mma_ts(tmem + kColO, tmem + kColS + 8 * k,
-                           tc::smem_desc(v_smem + k * (16 * 128), kKeys * 128, 1024), kIdO, ci > 0 || k > 0);
+                           tc::smem_desc(v_smem + k * (16 * 128), kKeys * 128, 1024), kIdO, k > 0);
             tc::commit(m_bar);
         }
         mma_pending = true;
-        if (__syncthreads_or(!mbar_wait(m_bar, m_phase, kWaitLimitNs))) {
+        if (__syncthreads_or(!mbar_wait(m_bar, phase, kWaitLimitNs))) {
             ok = false;
             break;
         }
         mma_pending = false;
-        m_phase ^= 1;
+        phase ^= 1;
         tc::fence_after();
-        // P.V has read this V chunk: the next step's V may come in now
-        if (st + 1 < steps && chunk_of(st + 1) != ch) {
-            if (t == 0) load_chunk(chunk_of(st + 1), v_smem, v_bar, &tmv);
-            ++v_issued;
-        }
 
-        if (ci == nc - 1 && b >= 0) {
-            // the row's partial for range c: (m, l) and O from TMEM
-            const size_t slot = (static_cast<size_t>(b) * p.Hq + h) * p.ws_parts + c;
-            p.ws_ml[2 * slot] = m_run;
-            p.ws_ml[2 * slot + 1] = l_run;
-            float4 *dst = reinterpret_cast<float4 *>(p.ws_o + slot * D);
-#pragma unroll 1
+        // the row's partial for chunk c
+        const size_t slot = (static_cast<size_t>(b < 0 ? 0 : b) * p.Hq + h) * p.ws_parts + c;
+        if (b >= 0) {
+            p.ws_ml[2 * slot] = mx;
+            p.ws_ml[2 * slot + 1] = l;
+        }
+        if (R <= 128) {
+            // The only row tile: K and V are no longer read, so the rows go
+            // through their shared memory ([row][D floats], 16-byte chunk j of
+            // row t at j ^ (t % chunks per row)) and each warp then writes its
+            // lanes' rows whole, one 16-byte chunk per lane.
+            constexpr int kChunks = D / 4;  // 16-byte chunks of a row
+            float4 *stage = reinterpret_cast<float4 *>(smem);
+#pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
                 tc::ld32(lane_base + kColO + 32 * cc, o);
                 tc::wait_ld();
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    dst[8 * cc + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                                  __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                    stage[t * kChunks + ((8 * cc + i) ^ (t & (kChunks - 1)))] =
+                        make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                    __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            }
+            __syncwarp();  // a warp writes out its own lanes' rows
+            const int lane = t & 31;
+#pragma unroll 1
+            for (int i = 0; i < 32; ++i) {
+                const int rr = 32 * warp + i;
+                const unsigned long long rslot = __shfl_sync(0xffffffffu, static_cast<unsigned long long>(slot), i);
+                if (!__shfl_sync(0xffffffffu, b >= 0, i)) continue;
+                float4 *rdst = reinterpret_cast<float4 *>(p.ws_o + rslot * D);
+                for (int j = lane; j < kChunks; j += 32)
+                    rdst[j] = stage[rr * kChunks + (j ^ (rr & (kChunks - 1)))];
+            }
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(p.ws_o + slot * D);
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tc::ld32(lane_base + kColO + 32 * cc, o);
+                tc::wait_ld();
+                if (b >= 0) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[8 * cc + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                                      __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                }
             }
         }
-        tc::fence_before();  // the O reads above, before the next tile's P.V overwrites O
     }
     if (!ok && t == 0) {
         flag(p.err, PKV_DEV_ERR_TIMEOUT);
-        if (mma_pending) mbar_wait(m_bar, m_phase, kWaitLimitNs);  // the batch still running
+        if (mma_pending) mbar_wait(m_bar, phase, kWaitLimitNs);  // the batch still running
     }
-    if (t == 0) {  // a load issued and not waited for (only after a wait gave up): let it land
-        if (k_issued > k_done) mbar_wait(k_bar, static_cast<uint32_t>(k_done & 1), kWaitLimitNs);
-        if (v_issued > v_done) mbar_wait(v_bar, static_cast<uint32_t>(v_done & 1), kWaitLimitNs);
+    if (t == 0) {  // copies still landing (done already unless a wait gave up)
+        mbar_wait(k_bar, 0, kWaitLimitNs);
+        mbar_wait(v_bar, 0, kWaitLimitNs);
     }
     tc::fence_before();
     __syncthreads();
@@ -563,7 +545,7 @@ __device__ __forceinline__ void prefix_range_tc(const CUtensorMap &tmk, const CU
     if (warp == 1) tc::dealloc<Geo::kTmemCols>(tmem);
 }
 
-// Merge of one (sequence, query head): prefix slots [0, ceil(pb / range_blocks)) and
+// Merge of one (sequence, query head): prefix chunks [0, ceil(pb / CB)) and
 // the suffix split-K partitions that hold tokens past the prefix (counted
 // from the prefix end), in slot order, by log-sum-exp.  As in the split-K
 // merge: all (m, l) read at once, weights computed once, output loads batched.
@@ -578,7 +560,7 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
     len = len < 0 ? 0 : min(len, p.W * kBlockTokens);
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
     const int pb = min(max(__ldg(p.prefix_blocks + b), 0), len / kBlockTokens);
-    const int nchunks = (pb + p.range_blocks - 1) / p.range_blocks;  // prefix slots
+    const int nchunks = (pb + CB - 1) / CB;
     // suffix partitions with tokens, at most those the launch computed (a
     // longer suffix was flagged by the cascade kernel)
     const int ntot = nchunks + min((nblk - pb + p.part_blocks - 1) / p.part_blocks,
@@ -626,44 +608,36 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
     p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
 }
 
-// The prefix grid: CTA k is prefix range k % prefix_parts of KV head
-// (k / prefix_parts) % Hkv of group k / (prefix_parts * Hkv).  It lets the
-// suffix grid, launched after it as a programmatic dependent, start early:
-// the two run side by side, the short tensor-core prefix work beside the
-// bandwidth-bound suffix stream.  TC: ranges on tcgen05 (else one chunk per
-// CTA on mma.sync); a tcgen05 CTA lets the suffix grid launch only once it
-// holds its tensor memory (in prefix_range_tc), a CTA without prefix work by
-// exiting.
-template <int D, bool TC>
+// One launch for the prefix chunks and the suffix split-K units.  Prefix
+// chunk k (chunk fastest, then KV head, then group) is CTA k * stride, spread
+// evenly through the grid, so that every SM runs the short, latency-bound
+// prefix work beside the bandwidth-bound suffix stream; the other CTAs take
+// suffix units in order (partition fastest, then head segment, then
+// sequence).  TC: the prefix chunks on tcgen05 (else mma.sync).
+template <int D, bool MMA, bool TC>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
-    cascade_prefix_kernel(const __grid_constant__ CUtensorMap tmk,
-                          const __grid_constant__ CUtensorMap tmv, const PrefixParams pp) {
-    if constexpr (!TC) pdl_launch_dependents();
+    cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                   const PrefixParams pp, const DecodeParams dp, int n_pre) {
+    pdl_launch_dependents();
     int id = blockIdx.x;
-    const int c = id % pp.prefix_parts;
-    id /= pp.prefix_parts;
-    if constexpr (TC)
-        prefix_range_tc<D, kPrefixTcChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
-    else
-        prefix_unit_mma<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
-}
-
-// The suffix grid: split-K units from each sequence's prefix end (partition
-// fastest, then head segment, then sequence).  WIDE: each CTA covers
-// kPrefixWarps head segments of one sequence, a warp each (suffixes are
-// short: one warp per segment keeps every ring busy for the whole suffix
-// instead of a quarter of it).  Before it exits, each CTA waits for the
-// prefix grid, so that this grid's completion -- which the merge waits for --
-// also covers the prefix partials.
-template <int D, bool MMA, bool WIDE>
-__global__ void __launch_bounds__(kPrefixWarps * 32)
-    cascade_suffix_kernel(const __grid_constant__ CUtensorMap tmk,
-                          const __grid_constant__ CUtensorMap tmv, const DecodeParams dp) {
-    // These CTAs use no tensor memory: they give up the right to allocate at
-    // once, so that they can never hold up a tcgen05.alloc on their SM.
-    if (threadIdx.x < 32) tc::relinquish();
-    int id = blockIdx.x;
-    const int ny = (MMA ? dp.Hkv * dp.chunks : dp.Hq) / (WIDE ? kPrefixWarps : 1);
+    const int stride = n_pre > 0 ? static_cast<int>(gridDim.x) / n_pre : 1;
+    if (n_pre > 0 && id % stride == 0 && id / stride < n_pre) {
+        id /= stride;
+        const int c = id % pp.prefix_parts;
+        id /= pp.prefix_parts;
+        if constexpr (TC)
+            prefix_unit_tc<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
+        else
+            prefix_unit_mma<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
+        return;
+    }
+    // Suffix units use no TMEM: they give up the right to allocate at once.
+    // A CTA that keeps it (until it exits) holds up the TMEM allocation of a
+    // prefix CTA that starts after it on the same SM (measured: the step took
+    // twice as long).
+    if (TC && n_pre > 0 && threadIdx.x < 32) tc::relinquish();
+    if (n_pre > 0) id -= min(id / stride + 1, n_pre);  // prefix CTAs at or before this one
+    const int ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
     const int part = id % dp.num_parts;
     id /= dp.num_parts;
     const int b = id / ny;
@@ -675,80 +649,48 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
         if (start + dp.num_parts * dp.part_blocks < (len + kBlockTokens - 1) / kBlockTokens)
             flag(dp.err, PKV_DEV_ERR_BAD_LEN);
     }
-    decode_unit<D, kPrefixWarps, 2, MMA, kModeSplit, WIDE>(tmk, tmv, dp, part, id % ny, b);
-    pdl_wait_primary();
+    decode_unit<D, kPrefixWarps, 2, MMA, kModeSplit>(tmk, tmv, dp, part, id % ny, b);
 }
 
-template <int D, bool MMA, bool TC, bool WIDE>
+template <int D, bool MMA, bool TC>
 cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                              const DecodeParams &dp, int num_groups, cudaStream_t stream) {
+    constexpr int kPre = TC ? PrefixTcGeometry<D, kPrefixChunkBlocks>::kSmemBytes
+                            : PrefixMmaGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
+    constexpr int kSmem = std::max(kPre, Geometry<D, kPrefixWarps, 2>::kSmemBytes);
+    auto kern = cascade_kernel<D, MMA, TC>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
     const long long n_pre = static_cast<long long>(pp.prefix_parts) * pp.Hkv * num_groups;
-    const long long ny = (MMA ? dp.Hkv * dp.chunks : dp.Hq) / (WIDE ? kPrefixWarps : 1);
+    const long long ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
     const long long n_suf = static_cast<long long>(dp.num_parts) * ny * dp.B;
-    if (n_pre >= (1ll << 31) || n_suf >= (1ll << 31)) return cudaErrorInvalidValue;
-    cudaError_t e;
-    if (n_pre > 0) {
-        constexpr int kPre = TC ? PrefixTcGeometry<D, kPrefixTcChunkBlocks>::kSmemBytes
-                                : PrefixMmaGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
-        auto pre = cascade_prefix_kernel<D, TC>;
-        if ((e = cudaFuncSetAttribute(pre, cudaFuncAttributeMaxDynamicSharedMemorySize, kPre)) != cudaSuccess)
-            return e;
-        pre<<<static_cast<unsigned>(n_pre), kPrefixWarps * 32, kPre, stream>>>(tmk, tmv, pp);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    constexpr int kSuf = Geometry<D, kPrefixWarps, 2>::kSmemBytes;
-    auto suf = cascade_suffix_kernel<D, MMA, WIDE>;
-    if ((e = cudaFuncSetAttribute(suf, cudaFuncAttributeMaxDynamicSharedMemorySize, kSuf)) != cudaSuccess)
-        return e;
-    if (n_suf > 0) {
-        cudaLaunchConfig_t cfg{};
-        cfg.gridDim = dim3(static_cast<unsigned>(n_suf));
-        cfg.blockDim = dim3(kPrefixWarps * 32);
-        cfg.dynamicSmemBytes = kSuf;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = n_pre > 0 ? 1 : 0;  // beside the prefix grid
-        if ((e = cudaLaunchKernelEx(&cfg, suf, tmk, tmv, dp)) != cudaSuccess) return e;
-    }
+    if (n_pre + n_suf >= (1ll << 31)) return cudaErrorInvalidValue;
+    kern<<<static_cast<unsigned>(n_pre + n_suf), kPrefixWarps * 32, kSmem, stream>>>(
+        tmk, tmv, pp, dp, static_cast<int>(n_pre));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return launch_dependent(cascade_merge_kernel<D, kPrefixChunkBlocks>,
                             dim3(static_cast<unsigned>(pp.Hq), static_cast<unsigned>(pp.B)), dim3(D),
                             stream, pp);
 }
 
-template <int D, bool TC, bool WIDE>
-cudaError_t launch_cascade_w(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
-                             const DecodeParams &dp, int num_groups, cudaStream_t stream) {
-    return dp.group > 1 ? launch_cascade_d<D, true, TC, WIDE>(tmk, tmv, pp, dp, num_groups, stream)
-                        : launch_cascade_d<D, false, TC, WIDE>(tmk, tmv, pp, dp, num_groups, stream);
-}
-
 template <int D>
 cudaError_t launch_cascade_h(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
-                             const DecodeParams &dp, int num_groups, bool prefix_tc, bool wide,
-                             cudaStream_t stream) {
+                             const DecodeParams &dp, int num_groups, bool prefix_tc, cudaStream_t stream) {
+    const bool mma = dp.group > 1;
     if (prefix_tc)
-        return wide ? launch_cascade_w<D, true, true>(tmk, tmv, pp, dp, num_groups, stream)
-                    : launch_cascade_w<D, true, false>(tmk, tmv, pp, dp, num_groups, stream);
-    return wide ? launch_cascade_w<D, false, true>(tmk, tmv, pp, dp, num_groups, stream)
-                : launch_cascade_w<D, false, false>(tmk, tmv, pp, dp, num_groups, stream);
+        return mma ? launch_cascade_d<D, true, true>(tmk, tmv, pp, dp, num_groups, stream)
+                   : launch_cascade_d<D, false, true>(tmk, tmv, pp, dp, num_groups, stream);
+    return mma ? launch_cascade_d<D, true, false>(tmk, tmv, pp, dp, num_groups, stream)
+               : launch_cascade_d<D, false, false>(tmk, tmv, pp, dp, num_groups, stream);
 }
 
 }  // namespace
 
-bool cascade_wide_fits(const DecodeParams &dp) {
-    const int segments = dp.group > 1 ? dp.Hkv * dp.chunks : dp.Hq;
-    return segments % kPrefixWarps == 0 && dp.chunks == 1;
-}
-
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                            const DecodeParams &dp, int head_dim, int num_groups, bool prefix_tc,
-                           bool wide, cudaStream_t stream) {
-    if (wide && !cascade_wide_fits(dp)) return cudaErrorInvalidValue;
-    if (head_dim == 128) return launch_cascade_h<128>(tmk, tmv, pp, dp, num_groups, prefix_tc, wide, stream);
-    if (head_dim == 64) return launch_cascade_h<64>(tmk, tmv, pp, dp, num_groups, prefix_tc, wide, stream);
+                           cudaStream_t stream) {
+    if (head_dim == 128) return launch_cascade_h<128>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
+    if (head_dim == 64) return launch_cascade_h<64>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
     return cudaErrorInvalidValue;
 }
 

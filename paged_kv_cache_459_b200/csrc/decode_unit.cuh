@@ -17,34 +17,24 @@ constexpr int kModeCluster = 2;  // one of p.num_parts equal parts of the sequen
 // One work unit (partition `part` of sequence b, KV head / head chunk `by`)
 // of the per-unit decode kernel, run by a CTA of NW warps.  The warps take
 // the unit's blocks round-robin and are combined in shared memory at the end.
-// WIDE: the unit is NW head segments instead (by = group of NW: MHA query
-// heads, or KV heads with one chunk of <= 8 query heads each); warp w takes
-// every block of segment by * NW + w alone, so short sequences keep each
-// warp's ring busy for NW times as many tiles, and no cross-warp combine is
-// needed (each warp's result is final).
-template <int D, int NW, int S, bool MMA, int MODE, bool WIDE = false>
+template <int D, int NW, int S, bool MMA, int MODE>
 __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtensorMap &tmv,
                                             const DecodeParams &p, int part, int by, int b) {
     using G = Geometry<D, NW, S>;
     constexpr bool SPLIT = MODE == kModeSplit;
     constexpr bool CLUSTER = MODE == kModeCluster;
-    static_assert(!(WIDE && CLUSTER), "wide units run single pass or split-K");
     // The merge kernel may be scheduled as soon as every unit has started; it
     // waits for this grid to finish before reading the partials.
     if constexpr (SPLIT) pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int seg = WIDE ? by * NW + warp : by;  // head segment: query head, or KV head [x chunk]
-    const int kvh = MMA ? seg / p.chunks : seg;
-    const int chunk = MMA ? seg % p.chunks : 0;
-    const int h0 = MMA ? kvh * p.group + chunk * 8 : kvh;  // first query head of this warp's segment
+    const int kvh = MMA ? by / p.chunks : by;
+    const int chunk = MMA ? by % p.chunks : 0;
+    const int h0 = MMA ? kvh * p.group + chunk * 8 : kvh;  // first query head of this CTA
     const int heads = MMA ? min(8, p.group - chunk * 8) : 1;
-    // query heads of the whole CTA (wide: NW segments; chunks == 1 for MMA) from h0_cta
-    const int h0_cta = WIDE ? (MMA ? by * NW * p.group : by * NW) : h0;
-    const int heads_cta = WIDE ? NW * heads : heads;
 
-    // Round-robin: warp w takes blocks blk_begin + w, + NW, ...; wide: all of them.
-    constexpr int kStride = WIDE ? 1 : NW;
-    const int lead = WIDE ? 0 : warp;
+    // Round-robin: warp w takes blocks blk_begin + w, + NW, ...
+    constexpr int kStride = NW;
+    const int lead = warp;
     // Block-table entries of this warp's blocks, 32 per lane-load.  Where the
     // unit's first block does not depend on the length (no skipped prefix, not
     // cluster mode), they are loaded now, beside the length, for every block
@@ -83,11 +73,11 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         // A fused write whose token lies before the start block (inside a
         // shared prefix) cannot be done here: flagged.
         if (p.k_new != nullptr && part == 0 && len > 0 && start >= nblk && threadIdx.x == 0 &&
-            (WIDE || !MMA || by % p.chunks == 0))
+            (!MMA || by % p.chunks == 0))
             flag(p.err, PKV_DEV_ERR_BAD_LEN);
         if (!SPLIT)
-            for (int i = threadIdx.x; i < heads_cta * D; i += NW * 32)
-                p.out[(static_cast<size_t>(b) * p.Hq + h0_cta + i / D) * D + i % D] = __float2bfloat16(0.f);
+            for (int i = threadIdx.x; i < heads * D; i += NW * 32)
+                p.out[(static_cast<size_t>(b) * p.Hq + h0 + i / D) * D + i % D] = __float2bfloat16(0.f);
         return;
     }
 
@@ -149,10 +139,8 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     // registers now, the store and the proxy fence (then __syncwarp, so lane
     // 0's TMA read is ordered after them) wait until then.  Several
     // head-chunk CTAs of one KV head store the same bytes.
-    // (Wide units: every warp holds its own segment's last block.)
     const int last_local = nblk - 1 - blk_begin;
-    const bool writer = p.k_new != nullptr && blk_end == nblk && len > 0 &&
-                        (WIDE || warp == last_local % NW);
+    const bool writer = p.k_new != nullptr && blk_end == nblk && len > 0 && warp == last_local % NW;
     const int i_write = last_local / kStride;
     uint4 new_val = make_uint4(0, 0, 0, 0);
     __nv_bfloat16 *new_dst = nullptr;
@@ -214,33 +202,6 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     }
 
     constexpr int kRed = MMA ? 16 + 8 * D : D + 2;
-    if constexpr (WIDE) {
-        // This warp's result is final for its segment: its (m, l, o) go
-        // through its own (drained) ring slice and out.
-        __syncwarp();
-        float *wr = reinterpret_cast<float *>(ring);
-        st.finish(wr, lane);
-        __syncwarp();
-        for (int idx = lane; idx < heads * D; idx += 32) {
-            const int n = idx / D, e = idx % D;
-            const float M = MMA ? wr[n] : wr[D];
-            const float L = MMA ? wr[8 + n] : wr[D + 1];
-            const float O = MMA ? wr[16 + n * D + e] : wr[e];
-            const size_t row = static_cast<size_t>(b) * p.Hq + h0 + n;
-            if constexpr (SPLIT) {
-                const size_t pr = row * p.ws_parts + p.ws_part0 + part;
-                p.ws_o[pr * D + e] = O;
-                if (e == 0) {
-                    p.ws_ml[2 * pr] = M;
-                    p.ws_ml[2 * pr + 1] = L;
-                }
-            } else {
-                p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
-            }
-        }
-        return;
-    }
-
     // ---- combine the warps of this CTA (all rings are drained) ----
     __syncthreads();
     float *red = reinterpret_cast<float *>(smem);

@@ -72,8 +72,7 @@ cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const 
 
 // Shared-prefix (cascade) decode: prefix blocks read once per (group, KV
 // head) by a dense tensor-core kernel; suffixes by split-K; LSE merge.
-constexpr int kPrefixChunkBlocks = 8;    // prefix blocks per chunk on mma.sync (128 keys)
-constexpr int kPrefixTcChunkBlocks = 4;  // prefix blocks per chunk on tcgen05 (64 keys)
+constexpr int kPrefixChunkBlocks = 8;  // prefix blocks per CTA
 
 struct PrefixParams {
     __nv_bfloat16 *out;
@@ -89,24 +88,17 @@ struct PrefixParams {
     long long num_blocks;
     int W, B, Hq, Hkv, group;
     int ws_parts;      // prefix_parts + suffix partitions
-    int prefix_parts;  // prefix ranges per (group, KV head): slots 0.. hold their partials
-    int range_blocks;  // prefix blocks per slot: a chunk (mma.sync) or a range of chunks (tcgen05)
+    int prefix_parts;  // ceil(W / kPrefixChunkBlocks): slots 0.. hold prefix chunks
     int part_blocks;   // suffix split-K partition (blocks)
     float scale_log2;
 };
 
-// The prefix grid, the suffix split-K grid beside it (a programmatic
-// dependent), then the merge.  dp must describe split-K with start_blocks =
-// prefix_blocks.
-// prefix_tc: the prefix chunks on tcgen05/TMEM instead of mma.sync.  wide:
-// each suffix CTA covers 4 head segments of a sequence, one warp each (needs
-// cascade_wide_fits).
+// One launch running prefix chunks and suffix split-K units side by side,
+// then the merge.  dp must describe split-K with start_blocks = prefix_blocks.
+// prefix_tc: the prefix chunks on tcgen05/TMEM instead of mma.sync.
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                            const DecodeParams &dp, int head_dim, int num_groups, bool prefix_tc,
-                           bool wide, cudaStream_t stream);
-// Wide suffix units need the head segments in whole groups of 4 (and one
-// chunk of <= 8 query heads per KV head).
-bool cascade_wide_fits(const DecodeParams &dp);
+                           cudaStream_t stream);
 
 // Causal prefill attention of each sequence's new tokens over its paged K/V.
 struct PrefillParams {

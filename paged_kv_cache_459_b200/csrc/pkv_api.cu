@@ -421,11 +421,9 @@ size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_d
     if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0) return 0;
     if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
     if (partition_tokens % PKV_BLOCK_TOKENS) return 0;
-    // suffix partitions + prefix slots (at most one per chunk of the smaller chunk size)
-    const int chunk = std::min(pkv::kPrefixChunkBlocks, pkv::kPrefixTcChunkBlocks);
     const size_t parts =
         static_cast<size_t>(num_parts_for(max_blocks_per_seq, partition_tokens)) +
-        (max_blocks_per_seq + chunk - 1) / chunk;
+        (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
     return static_cast<size_t>(num_seqs) * num_heads * parts * (static_cast<size_t>(head_dim) + 2) *
            sizeof(float);
 }
@@ -474,27 +472,7 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
                                   ? max_suffix_blocks
                                   : max_blocks_per_seq;
     const int suffix_parts = num_parts_for(suffix_blocks, partition_tokens);
-    // Prefix work: 8-block chunks on mma.sync, one per CTA; 4-block chunks on
-    // tcgen05, each CTA taking a range of them with O held in TMEM across
-    // the range, sized so that the prefix grid is about 64 CTAs (the (group, KV head, 128-row tile, chunk) steps spread
-    // evenly, rows per group estimated from an even split of the batch); on
-    // mma.sync one chunk per CTA.
-    const bool prefix_tc = env_int("PKV_CASCADE_TC", 0) != 0;
-    const int chunk_blocks = prefix_tc ? pkv::kPrefixTcChunkBlocks : pkv::kPrefixChunkBlocks;
-    const int chunks = (max_blocks_per_seq + chunk_blocks - 1) / chunk_blocks;
-    int range_chunks = 1;
-    if (prefix_tc) {
-        const int64_t groups = std::max(num_groups, 1);
-        const int64_t rows = static_cast<int64_t>(num_seqs) * (num_heads / num_kv_heads);
-        const int64_t row_tiles = std::max<int64_t>(1, (rows / groups + 127) / 128);
-        const int64_t steps = groups * num_kv_heads * row_tiles * chunks;
-        const int64_t per_cta = (steps + 63) / 64;
-        range_chunks = static_cast<int>(std::min<int64_t>(
-            chunks, std::max<int64_t>(1, (per_cta + row_tiles - 1) / row_tiles)));
-        const int forced = env_int("PKV_CASCADE_RANGE_CHUNKS", 0);
-        if (forced > 0) range_chunks = std::min(forced, chunks);
-    }
-    const int prefix_parts = (chunks + range_chunks - 1) / range_chunks;
+    const int prefix_parts = (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
     const size_t ws_rows = static_cast<size_t>(num_seqs) * num_heads * (prefix_parts + suffix_parts);
     float *ws_o = static_cast<float *>(workspace);
     float *ws_ml = ws_o + ws_rows * head_dim;
@@ -518,7 +496,6 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     pp.group = num_heads / num_kv_heads;
     pp.ws_parts = prefix_parts + suffix_parts;
     pp.prefix_parts = prefix_parts;
-    pp.range_blocks = range_chunks * chunk_blocks;
     pp.part_blocks = partition_tokens / PKV_BLOCK_TOKENS;
     pp.scale_log2 = scale * 1.4426950408889634f;
 
@@ -549,17 +526,9 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     dp.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
     dp.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
 
-    // Suffix units: one warp per head segment (wide) when the segments come in
-    // groups of 4 and the wide grid still holds two waves of CTAs at 3 per
-    // SM; PKV_CASCADE_WIDE=0 / 1 turns it off / on (where it fits).
-    const int64_t segments = pp.group > 1 ? static_cast<int64_t>(num_kv_heads) * dp.chunks : num_heads;
-    const int64_t wide_ctas = static_cast<int64_t>(suffix_parts) * (segments / 4) * num_seqs;
-    const int wide_env = env_int("PKV_CASCADE_WIDE", -1);
-    const bool wide = pkv::cascade_wide_fits(dp) &&
-                      (wide_env == 1 || (wide_env < 0 && wide_ctas >= 2 * 3 * sm_count()));
-    // mma.sync prefix chunks by default; PKV_CASCADE_TC=1 selects the
-    // tcgen05 prefix ranges
-    cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups, prefix_tc, wide,
+    // mma.sync prefix chunks by default; PKV_CASCADE_TC=1 selects the tcgen05 ones
+    cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
+                                        env_int("PKV_CASCADE_TC", 0) != 0,
                                         static_cast<cudaStream_t>(stream));
     return cuda_status(e);
 }

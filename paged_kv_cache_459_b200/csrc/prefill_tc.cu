@@ -1,8 +1,8 @@
 // Paged prefill attention on the 5th-generation tensor cores (tcgen05, TMEM).
 //
 // Causal attention of each sequence's new tokens over its paged K/V ("vLLM 與
-// PagedAttention：高吞吐推理的關鍵", section 三 step 二).  A persistent CTA (one per
-// SM) walks work items; an item is two Q tiles of 128 query rows each -- (token, query head
+// PagedAttention：高吞吐推理的關鍵", section 三 step 二).  A persistent CTA (one per SM) walks work
+// items; an item is two Q tiles of 128 query rows each -- (token, query head
 // of one KV head) pairs of one sequence -- whose keys are walked in tiles of
 // 128 (eight 16-token blocks); both Q tiles share each K/V tile.  Per Q tile x:
 //   S_x[128 x 128] = Q_x[128 x d] K_tile^T   tcgen05.mma (A, B in shared memory)
@@ -12,19 +12,14 @@
 // Roles: a producer warp streams K and V tiles (TMA, 128-byte swizzle, K and
 // V in separate rings; blocks past the table or the pool load as zeros from
 // out-of-range coordinates); one thread of the MMA warp issues the products
-// and commits them to mbarriers; two softmax warpgroups per Q tile each own
-// half of every key tile (64 keys) for one row per thread (TMEM lane = row):
-// they read S with tcgen05.ld, mask (causal, sequence end), trade their row
-// maxima through shared memory behind the tile's named barrier, keep the
-// running max and sum, store P with tcgen05.st, and rescale their half of O
-// in TMEM only when a row's max grows by more than 2^8 (otherwise the old max
-// is kept: P stays <= 2^8).  Halving each tile's softmax shortens its chain
-// S -> softmax -> P.V -> next S, which bounds the step.  The two Q tiles
-// ping-pong: the tensor core computes one tile's products while the other
-// tile's softmax runs.  Every mbarrier wait is bounded; a wait that gives up
-// is voted on at the tile's next named barrier so that all its warps stop
-// together; the kernel flags PKV_DEV_ERR_TIMEOUT, stops issuing, and still
-// frees its TMEM.
+// and commits them to mbarriers; one softmax warpgroup per Q tile owns one
+// row per thread (TMEM lane = row), reads S with tcgen05.ld, masks (causal,
+// sequence end), keeps the running max and sum, stores P with tcgen05.st, and
+// rescales O in TMEM only when a row's max grows by more than 2^8 (otherwise
+// the old max is kept: P stays <= 2^8).  The two Q tiles ping-pong: the tensor
+// core computes one tile's products while the other tile's softmax runs.
+// Every wait is bounded; on a timeout the kernel flags PKV_DEV_ERR_TIMEOUT,
+// stops issuing, and still frees its TMEM.
 #include <algorithm>
 
 #include "decode_common.cuh"
@@ -40,15 +35,11 @@ constexpr int kRows = 128;                 // query rows per Q tile (MMA M)
 constexpr int kTiles = 2;                  // Q tiles per CTA, ping-ponged on the tensor core
 constexpr int kCtaRows = kTiles * kRows;
 constexpr int kKeys = 128;                 // keys per tile (MMA N of S, K of P.V)
-constexpr int kWarpsPerTile = 4;           // warps of one softmax warpgroup (all 128 TMEM lanes)
-constexpr int kSoftmaxWarps = kTiles * 2 * kWarpsPerTile;  // two warpgroups (key halves) per Q tile
+constexpr int kWarpsPerTile = 4;           // one softmax warpgroup per Q tile
+constexpr int kSoftmaxWarps = kTiles * kWarpsPerTile;
 constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Of every 16 score pairs a softmax thread turns into P, this many take 2^x
-// on the FMA pipe (exp2_fma2) instead of the special-function unit, which
-// the two Q tiles' softmaxes otherwise share.
-constexpr int kFmaExpPairs = 0;
 
 // ------------------------------------------------ packed f32x2 arithmetic
 // Two floats in one 64-bit register pair for the sm_100 f32x2 instructions.
@@ -70,34 +61,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
-__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-// 2^x for two values on the FMA pipe instead of the special-function unit:
-// 2^x = 2^floor(x) * 2^f, f in [0, 1), with 2^f from a cubic fitted here to
-// 2^f on [0, 1) by least squares on the relative error (largest relative
-// error 2.2e-4, under the bf16 rounding of P); the integer part is added to
-// the exponent bits.  x is clamped at -126 (2^-126 instead of 0 below it);
-// the softmax never passes more than +8.
-__device__ __forceinline__ void exp2_fma2(float &a, float &b) {
-    constexpr float c0 = 0.99998891353607178f, c1 = 0.69449967145919800f;
-    constexpr float c2 = 0.23030571639537811f, c3 = 0.07476584613323212f;
-    a = fmaxf(a, -126.f);
-    b = fmaxf(b, -126.f);
-    const float fa = floorf(a), fb = floorf(b);
-    const uint64_t f = fsub2(f2pack(a, b), f2pack(fa, fb));
-    uint64_t p = ffma2(f2pack(c3, c3), f, f2pack(c2, c2));
-    p = ffma2(p, f, f2pack(c1, c1));
-    p = ffma2(p, f, f2pack(c0, c0));
-    float pa, pb;
-    f2unpack(p, pa, pb);
-    a = __uint_as_float(__float_as_uint(pa) + (static_cast<uint32_t>(static_cast<int>(fa)) << 23));
-    b = __uint_as_float(__float_as_uint(pb) + (static_cast<uint32_t>(static_cast<int>(fb)) << 23));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -107,7 +70,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 template <int D>
 struct TcGeometry {
     static constexpr int kHalves = D / 64;
-    static constexpr int kKStages = D == 128 ? 2 : 4;           // K ring depth
+    static constexpr int kKStages = D == 128 ? 3 : 4;           // K ring depth
     static constexpr int kVStages = D == 128 ? 2 : 4;           // V ring depth
     static constexpr int kQBytes = kHalves * kRows * 128;      // one Q tile [half][row][128 B]
     static constexpr int kKVBytes = kHalves * kKeys * 128;     // K or V tile [half][key][128 B]
@@ -116,15 +79,10 @@ struct TcGeometry {
     static constexpr int kV = kK + kKStages * kKVBytes;
     static constexpr int kBars = kV + kVStages * kKVBytes;     // up to 32 mbarriers
     static constexpr int kTmemSlot = kBars + 32 * 8;
-    // per Q tile: the key halves' row maxima and row sums (2 parities each)
-    // and the warps' votes (2 step parities, 2 item parities, 8 warps each)
-    static constexpr int kXchPerTile = 8 * kRows + 32;        // floats
-    static constexpr int kXch = kTmemSlot + 16;
-    static constexpr int kSmemBytes = kXch + kTiles * kXchPerTile * 4 + 1024;
+    static constexpr int kSmemBytes = kTmemSlot + 16 + 1024;
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
     static_assert(2 * (kKStages + kVStages) + 10 <= 32, "barrier slots");
-    // TMEM columns: S of tile x at kKeys x (P, bf16, over columns [0, 32) and
-    // [64, 96) of it: each softmax half's keys over its own scores),
+    // TMEM columns: S of tile x at kKeys x (P, bf16, over its first half),
     // O of tile x at kO + D x.
     static constexpr int kO = kTiles * kKeys;
     static constexpr int kTmemCols = 512;
@@ -137,28 +95,15 @@ struct TcItem {
     int nk0, nk1;  // key tiles Q tile 0 / 1 can see (tile 1 may be empty: 0)
 };
 
-// z counts 256-row tiles from the END of each sequence, so low z sees the
-// most keys.  Items are numbered heaviest first in groups of kZGroup z levels:
-// group-major, then (sequence, KV head), then z within the group -- so the
-// items of one (sequence, head) that read nearly the same keys are dealt to
-// neighbouring CTAs, run at the same time and share their K/V tiles in L2,
-// while the order stays heaviest first.
-constexpr int kZGroup = 2;
-
-__device__ __forceinline__ void tc_item_coords(const PrefillParams &p, int i, int &z, int &b, int &kvh) {
-    const int per_group = kZGroup * p.Hkv * p.B;
-    const int zg = i / per_group, rem = i - zg * per_group;
-    const int pair = rem / kZGroup;
-    z = zg * kZGroup + (rem - pair * kZGroup);
-    b = pair / p.Hkv;
-    kvh = pair - b * p.Hkv;
-}
-
+// Items are numbered z-major -- z counts 256-row tiles from the END of each
+// sequence, so low numbers see the most keys -- then sequence, then KV head.
 // Returns false for items past a sequence's rows or of a sequence whose
 // lengths are inconsistent (*bad set for the latter).
 __device__ __forceinline__ bool tc_item(const PrefillParams &p, int i, TcItem &it, bool *bad) {
-    int z;
-    tc_item_coords(p, i, z, it.b, it.kvh);
+    const int per_z = p.Hkv * p.B;
+    const int z = i / per_z, rem = i - z * per_z;
+    it.b = rem / p.Hkv;
+    it.kvh = rem - it.b * p.Hkv;
     it.q0 = __ldg(p.query_start + it.b);
     const int nq = __ldg(p.query_start + it.b + 1) - it.q0;
     it.ctx = __ldg(p.seq_lens + it.b);
@@ -239,10 +184,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int x = 0; x < kTiles; ++x) {
             mbar_init(s_full(x), 1);
-            mbar_init(p_full(x), 2 * kWarpsPerTile);
+            mbar_init(p_full(x), kWarpsPerTile);
             mbar_init(o_done(x), 1);
-            mbar_init(q_full(x), 2 * kWarpsPerTile);
-            mbar_init(o_free(x), 2 * kWarpsPerTile);
+            mbar_init(q_full(x), kWarpsPerTile);
+            mbar_init(o_free(x), kWarpsPerTile);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -324,9 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0;; ++k) {
                 const int i = tc_item_index(k, blockIdx.x, gridDim.x);
                 if (i >= p.items) break;
-                int z, b, kvh;
-                tc_item_coords(p, i, z, b, kvh);
-                if (z == 0 && kvh == 0) {
+                if (i < p.Hkv * p.B && i % p.Hkv == 0) {
                     TcItem bad_it;
                     bool bad;
                     tc_item(p, i, bad_it, &bad);
@@ -356,13 +299,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc::commit(s_full(x));
         };
-        // O_x (+)= P_x . V, P_x from TMEM: the P of keys [64 h, 64 h + 64) sits at
-        // columns [64 h, 64 h + 32) of S_x (each softmax half over its own scores)
-        const auto issue_pv = [&](int x, int stage, bool acc) {
+        const auto issue_pv = [&](int x, int stage, bool acc) {  // O_x (+)= P_x . V, P_x from TMEM
             const uint32_t vbase = smem_u32(smem + Geo::kV + stage * Geo::kKVBytes);
 #pragma unroll
             for (int k = 0; k < kKeys / 16; ++k)
-                tc::mma_ts(tmem + Geo::kO + D * x, tmem + kKeys * x + 64 * (k / 4) + 8 * (k % 4),
+                tc::mma_ts(tmem + Geo::kO + D * x, tmem + kKeys * x + 8 * k,
                         tc::smem_desc(vbase + k * (16 * 128), kKeys * 128, 1024), kIdO, acc || k > 0);
         };
         bool ok = true;
@@ -456,44 +397,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             k = kn;
         }
     } else {
-        // ---------------- softmax warps.  Tile x has two warpgroups: half hf
-        // takes keys [64 hf, 64 hf + 64) of every key tile (P columns
-        // [32 hf, 32 hf + 32)) and O columns [hf D / 2, (hf + 1) D / 2) for
-        // the rescale and the epilogue; thread t of either half = TMEM lane t
-        // = row r_begin + 128 x + t.  Per key tile the halves exchange their
-        // row maxima (and at the end of an item their row sums) through
-        // shared memory behind the tile's named barrier, which also carries
-        // each warp's "wait gave up" vote so that all eight warps of a tile
-        // leave the loop at the same step.
-        const int tile = warp / (2 * kWarpsPerTile);
-        const int hf = (warp / kWarpsPerTile) & 1;
+        // ---------------- softmax warps: thread t of tile x = TMEM lane t = row r_begin + 128 x + t
+        const int tile = warp / kWarpsPerTile;
         const int t = threadIdx.x & (kRows - 1);
-        const int wq = warp & (2 * kWarpsPerTile - 1);  // warp within the tile: vote slot
         const uint32_t lane_addr = static_cast<uint32_t>((warp % kWarpsPerTile) * 32) << 16;
         const uint32_t t_s = tmem + lane_addr + kKeys * tile;
         const uint32_t t_o = tmem + lane_addr + Geo::kO + D * tile;
         uint8_t *qrow = smem + Geo::kQ + tile * Geo::kQBytes + t * 128;
-        float *xch = reinterpret_cast<float *>(smem + Geo::kXch) + tile * Geo::kXchPerTile;
-        // xch: max [2 step parities][2 halves][128 rows], sum [2 item parities][2 halves][128
-        // rows], votes [2 step parities + 2 item parities][8 warps].  Alternate slots: a
-        // slot is written again only after a later barrier that the partner half passes
-        // after reading it.
-        float *x_max = xch, *x_sum = xch + 4 * kRows;
-        volatile int *x_vote = reinterpret_cast<volatile int *>(xch + 8 * kRows);
-        const auto tile_bar = [&]() {  // the 256 threads of this tile's two halves
-            asm volatile("bar.sync %0, %1;" ::"r"(1 + tile), "r"(2 * kWarpsPerTile * 32) : "memory");
-        };
-        // every warp of the tile votes in vote slot `slot`; true if all eight are still fine
-        const auto tile_vote = [&](bool fine, int slot) {
-            if (lane == 0) x_vote[8 * slot + wq] = fine ? 1 : 0;
-            tile_bar();
-            bool all = true;
-#pragma unroll
-            for (int w = 0; w < 2 * kWarpsPerTile; ++w) all = all && x_vote[8 * slot + w] != 0;
-            return all;
-        };
-        // this thread's half of its Q row of an item into shared memory
-        // (K-major, 128-byte swizzle; rows past the item's rows are zero-filled)
+        // this thread's Q row of an item into shared memory (K-major, 128-byte
+        // swizzle; rows past the item's rows are zero-filled)
         const auto fetch_q = [&](const TcItem &nx) {
             const int r = nx.r_begin + tile * kRows + t;
             const __nv_bfloat16 *src = p.q;
@@ -503,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bytes = 16;
             }
 #pragma unroll
-            for (int c = hf * (D / 16); c < (hf + 1) * (D / 16); ++c)
+            for (int c = 0; c < D / 8; ++c)
                 cp_async16(smem_u32(qrow + (c >> 3) * (kRows * 128) + (((c & 7) ^ (t & 7)) << 4)),
                            src + (bytes ? c * 8 : 0), bytes);
             asm volatile("cp.async.commit_group;" ::: "memory");
@@ -515,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(q_full(tile));
         };
         bool ok = true;
-        int ns = 0;    // S products seen (s_full / p_full phases; vote parity)
+        int ns = 0;    // S products seen (s_full / p_full phases)
         int n_it = 0;  // items done (o_done phases)
         TcItem it, nx;  // the current and the next item
         int k = tc_next_item(p, 0, it);
@@ -530,81 +442,74 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int my_nk = tile == 0 ? it.nk0 : it.nk1;
             __nv_bfloat16 *out_row =
                 p.out + (static_cast<size_t>(it.q0 + r / G) * p.Hq + it.kvh * G + r % G) * D;
-            float m_run = -INFINITY, l_run = 0.f;  // l_run: this half's keys
+            float m_run = -INFINITY, l_run = 0.f;
             if (my_nk == 0 && kn >= 0) fetch_q(nx);
             for (int j = 0; j < my_nk; ++j, ++ns) {
                 // S_x(j) done; it was issued after PV_x(j - 1), so O_x is free too
-                const bool got = mbar_wait(s_full(tile), static_cast<uint32_t>(ns & 1), kWaitLimitNs) &&
-                                 !*abort_flag;
-                tc::fence_after();
-                // this half's 64 scores of the row, 32 at a time (two passes: the
-                // row max, then P), causal mask by position
-                const int k0 = j * kKeys + 64 * hf;
-                const bool masked = __any_sync(0xffffffffu, k0 + 63 > row_pos);
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                if (got) {
-#pragma unroll 1
-                    for (int q = 0; q < 2; ++q) {
-                        uint32_t sr[32];
-                        tc::ld32(t_s + 64 * hf + 32 * q, sr);
-                        tc::wait_ld();
-                        if (masked) {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                if (k0 + 32 * q + c > row_pos) sr[c] = 0xFF800000u;  // -inf
-                        }
-#pragma unroll
-                        for (int c = 0; c < 32; c += 2)
-                            mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                    }
-                }
-                x_max[(2 * (ns & 1) + hf) * kRows + t] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-                if (!tile_vote(got, ns & 1)) {
+                if (!mbar_wait(s_full(tile), static_cast<uint32_t>(ns & 1), kWaitLimitNs) || *abort_flag) {
                     ok = false;
                     break;
                 }
+                tc::fence_after();
                 // the last S product of this item has read Q_x: fetch the next item's rows
                 if (j + 1 == my_nk && kn >= 0) fetch_q(nx);
-                // row max of the raw scores (scale > 0), both halves
-                const float mx = fmaxf(x_max[(2 * (ns & 1)) * kRows + t], x_max[(2 * (ns & 1) + 1) * kRows + t]) *
-                                 p.scale_log2;
-                // keep the running max unless it grows by more than 2^8 (the same
-                // decision in both halves: the same inputs)
+                // Two passes over S in TMEM, 64 columns at a time, so that a row
+                // never sits in registers whole (ten warps leave 168 registers
+                // a thread): the row max first, then exp2 and P.
+                const int k0 = j * kKeys;
+                const bool masked = __any_sync(0xffffffffu, k0 + kKeys - 1 > row_pos);
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1  // one half's 64 registers live at a time
+                for (int h = 0; h < kKeys / 64; ++h) {
+                    uint32_t sr[64];
+                    tc::ld32(t_s + 64 * h, sr);
+                    tc::ld32(t_s + 64 * h + 32, sr + 32);
+                    tc::wait_ld();
+                    // causal mask by position (only tiles that reach past some row need it)
+                    if (masked) {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;  // -inf
+                    }
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2)
+                        mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                }
+                // row max of the raw scores (scale > 0)
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
+                // keep the running max unless it grows by more than 2^8
                 const bool grow = mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx != -INFINITY);
                 const float m_new = grow ? mx : m_run;
                 const float nbase = m_new == -INFINITY ? 0.f : -m_new;
-                // P of this half's 64 keys, 32 columns (two keys per column), 16 at a time
+                // P_x over the first half of S_x's columns (two keys per column),
+                // 64 keys at a time; P's columns [32 h, 32 h + 32) overwrite S
+                // columns already read
                 const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
                 const uint64_t nbase2 = f2pack(nbase, nbase);
                 uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
-#pragma unroll 1
-                for (int q = 0; q < 2; ++q) {
-                    uint32_t sr[32];
-                    tc::ld32(t_s + 64 * hf + 32 * q, sr);
+#pragma unroll 1  // one half's 64 registers live at a time
+                for (int h = 0; h < kKeys / 64; ++h) {
+                    uint32_t sr[64];
+                    tc::ld32(t_s + 64 * h, sr);
+                    tc::ld32(t_s + 64 * h + 32, sr + 32);
                     tc::wait_ld();
+                    uint32_t pk[32];
                     if (masked) {  // diagonal tiles: -inf scores (2^-inf = 0)
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (k0 + 32 * q + c > row_pos) sr[c] = 0xFF800000u;
+                        for (int c = 0; c < 64; ++c)
+                            if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;
                     }
-                    uint32_t pk[16];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {  // scale and shift two at a time, 2^x on the SFU
+                    for (int c = 0; c < 64; c += 2) {  // scale and shift two at a time, 2^x on the SFU
                         float a, bb;
                         f2unpack(ffma2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), scale2, nbase2), a, bb);
-                        if ((c >> 1) % 16 < kFmaExpPairs) {
-                            exp2_fma2(a, bb);
-                        } else {
-                            a = ex2_approx(a);
-                            bb = ex2_approx(bb);
-                        }
+                        a = ex2_approx(a);
+                        bb = ex2_approx(bb);
                         sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], f2pack(a, bb));
                         __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
                         pk[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
                     }
-                    // P over this half's own S columns, already read: keys [64 hf, 64 hf + 64)
-                    // at columns [64 hf, 64 hf + 32) -- never over the other half's scores
-                    tc::st16(t_s + 64 * hf + 16 * q, pk);
+                    tc::st32(t_s + 32 * h, pk);
                 }
                 float s_lo, s_hi, s_lo2, s_hi2;
                 f2unpack(sum2[0], s_lo, s_hi);
@@ -612,15 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float rowsum = (s_lo + s_hi) + (s_lo2 + s_hi2);
                 if (j > 0) {
                     const float alpha = (grow && m_run != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
-                    if (__any_sync(0xffffffffu, alpha != 1.f)) {  // this half's columns of O
+                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                        for (int cc = 0; cc < D / 64; ++cc) {
+                        for (int cc = 0; cc < D / 32; ++cc) {
                             uint32_t o[32];
-                            tc::ld32(t_o + hf * (D / 2) + 32 * cc, o);
+                            tc::ld32(t_o + 32 * cc, o);
                             tc::wait_ld();
 #pragma unroll
                             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                            tc::st32(t_o + hf * (D / 2) + 32 * cc, o);
+                            tc::st32(t_o + 32 * cc, o);
                         }
                     }
                     l_run *= alpha;
@@ -637,16 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             // O_x of this item complete (a tile without rows gets a bare commit)
-            const bool done = mbar_wait(o_done(tile), static_cast<uint32_t>(n_it & 1), kWaitLimitNs) &&
-                              !*abort_flag;
-            tc::fence_after();
-            float *sums = x_sum + 2 * kRows * (n_it & 1);
-            sums[hf * kRows + t] = l_run;
-            if (!tile_vote(done, 2 + (n_it & 1))) {
+            if (!mbar_wait(o_done(tile), static_cast<uint32_t>(n_it & 1), kWaitLimitNs) || *abort_flag) {
                 ok = false;
                 break;
             }
-            const float l_row = sums[t] + sums[kRows + t];
+            tc::fence_after();
             if (my_nk == 0 && kn >= 0) publish_q();  // after o_done: at most one phase ahead
             ++n_it;
             if (my_nk == 0) {
@@ -656,18 +556,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 k = kn;
                 continue;
             }
-            // this half's O columns of the row, normalised, packed to bf16 and
-            // stored; then O_x is handed back
-            const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
-            uint4 *dst = reinterpret_cast<uint4 *>(out_row) + hf * (D / 16);
-#pragma unroll 1
-            for (int cc = 0; cc < D / 64; ++cc) {
-                uint32_t o[32];
-                tc::ld32(t_o + hf * (D / 2) + 32 * cc, o);
+            // O row, normalised, packed to bf16 and stored 64 columns at a
+            // time; then O_x is handed back
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            uint4 *dst = reinterpret_cast<uint4 *>(out_row);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) {
+                uint32_t o[64];
+                tc::ld32(t_o + 64 * h, o);
+                tc::ld32(t_o + 64 * h + 32, o + 32);
                 tc::wait_ld();
                 if (row_pos >= 0) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < 8; ++i) {
                         uint32_t w[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -675,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                       __uint_as_float(o[8 * i + 2 * e + 1]) * inv);
                             w[e] = *reinterpret_cast<uint32_t *>(&h2);
                         }
-                        dst[4 * cc + i] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[8 * h + i] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
             }
@@ -685,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             it = nx;
             k = kn;
         }
-        if (!ok && t == 0 && hf == 0) {
+        if (!ok && t == 0) {
             flag(p.err, PKV_DEV_ERR_TIMEOUT);
             *abort_flag = 1;
         }
@@ -707,8 +608,7 @@ cudaError_t launch_prefill_tc_d(const CUtensorMap &tmk, const CUtensorMap &tmv, 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const long long rows = static_cast<long long>(max_query_len) * p.group;
-    const long long zlevels = (rows + kCtaRows - 1) / kCtaRows;
-    const long long items = (zlevels + kZGroup - 1) / kZGroup * kZGroup * p.Hkv * p.B;
+    const long long items = (rows + kCtaRows - 1) / kCtaRows * p.Hkv * p.B;
     if (items == 0) return cudaSuccess;
     if (items > 0x7FFFFFFFLL - 2LL * num_sms) return cudaErrorInvalidValue;
     p.items = static_cast<int>(items);

@@ -59,16 +59,8 @@ def prefix_impl(request, monkeypatch):
     return request.param
 
 
-@pytest.fixture(params=["narrow", "wide"])
-def suffix_units(request, monkeypatch):
-    """Suffix units of one head segment each, or four per CTA with a warp each
-    (wide; used where the heads come in groups of four)."""
-    monkeypatch.setenv("PKV_CASCADE_WIDE", "1" if request.param == "wide" else "0")
-    return request.param
-
-
 @pytest.mark.parametrize("name,kw", CASES, ids=[str(i) for i in range(len(CASES))])
-def test_cascade_matches_oracle(name, kw, prefix_impl, suffix_units):
+def test_cascade_matches_oracle(name, kw, prefix_impl):
     w = build(name, 13, **kw)
     d = DeviceStep(w)
     d.write()
@@ -78,24 +70,6 @@ def test_cascade_matches_oracle(name, kw, prefix_impl, suffix_units):
             out, pb, offs = cascade(d, part, bound=bound)
             assert len(offs) - 1 == kw.get("prefix_groups", 1) and pb.max() > 0
             check_close(out, ref, f"cascade {kw} partition {part} suffix bound {bound}")
-    assert d.err_word() == 0
-
-
-@pytest.mark.parametrize("range_chunks", [1, 2, 100])
-@pytest.mark.parametrize("idx", [0, 2, 6])
-def test_cascade_tcgen05_prefix_ranges(idx, range_chunks, monkeypatch):
-    """tcgen05 prefix ranges of one chunk, two chunks, and the whole prefix:
-    the output accumulated in TMEM across chunks with the running max, over
-    one or several 128-row tiles."""
-    monkeypatch.setenv("PKV_CASCADE_TC", "1")
-    monkeypatch.setenv("PKV_CASCADE_RANGE_CHUNKS", str(range_chunks))
-    name, kw = CASES[idx]
-    w = build(name, 17, **kw)
-    d = DeviceStep(w)
-    d.write()
-    kc, vc, ref = oracle_after_write(w)
-    out, pb, offs = cascade(d, bound="exact")
-    check_close(out, ref, f"tcgen05 prefix ranges of {range_chunks} chunks, {kw}")
     assert d.err_word() == 0
 
 
@@ -109,7 +83,7 @@ def test_cascade_suffix_bound_too_small_is_flagged():
     assert d.err_word() & 4
 
 
-def test_cascade_full_size(prefix_impl, suffix_units):
+def test_cascade_full_size(prefix_impl):
     """The prefix workload at full size (128 sequences sharing a 2000-token
     prefix): every output row against the oracle."""
     w = build("prefix", 0)
@@ -123,7 +97,7 @@ def test_cascade_full_size(prefix_impl, suffix_units):
     assert d.err_word() == 0
 
 
-def test_cascade_block_relabelling_is_bit_exact(prefix_impl, suffix_units):
+def test_cascade_block_relabelling_is_bit_exact(prefix_impl):
     w = build("prefix", 14, batch=10, prefix_len=256, suffix_lo=1, suffix_hi=80, prefix_groups=2)
     d = DeviceStep(w)
     d.write()
@@ -138,7 +112,7 @@ def test_cascade_block_relabelling_is_bit_exact(prefix_impl, suffix_units):
 
 
 @pytest.mark.parametrize("idx", [0, 1, 2, 3])
-def test_cascade_fused_step(idx, prefix_impl, suffix_units):
+def test_cascade_fused_step(idx, prefix_impl):
     """pkv_paged_decode_prefix_step: the step's write fused into the cascade --
     caches bit-exact with the oracle's write, output within tolerance, and
     bit-identical to the separate write + cascade."""
