@@ -604,16 +604,6 @@ def workload_key(args, name, *, dev, cascade=False, batch=None, clocks=True) -> 
         out["logical_kv_bytes"] = m["bytes"]["kv"]
         out["unique_kv_bytes"] = m["bytes"]["decode"] - m["bytes"]["q"] - \
             (2 * r.B * r.hkv * r.d * 2 * 2 if r.fused else 0)
-        # the prefix chunks on mma.sync (default) and on tcgen05, one loop each
-        cmp = {"default_step_us": 1e3 * _events_time(r.step, args.steps, 3)}
-        os.environ["PKV_CASCADE_TC"] = "1"
-        try:
-            cmp["tcgen05_step_us"] = 1e3 * _events_time(r.step, args.steps, 3)
-        finally:
-            os.environ.pop("PKV_CASCADE_TC")
-        cmp["how"] = ("K steps back to back between two events: the default prefix chunks, then "
-                      "PKV_CASCADE_TC=1 (tcgen05 prefix chunks)")
-        out["prefix_paths"] = cmp
     del r
     torch.cuda.empty_cache()
     return out

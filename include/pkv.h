@@ -287,13 +287,11 @@ PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, c
  * prefix_blocks[b] = 0.  The group's shared block ids are read from its first
  * member's table row.  pkv_alloc_prefix_groups builds all three arrays from
  * the allocator's state.  All five arrays are device int32.
- * Work: a tensor-core kernel computes each group's prefix attention in
- * chunks of 8 blocks (queries of all members x heads as MMA rows); the
- * split-K kernel (partition_tokens, <= 0: 512) covers each sequence past its
- * prefix; a merge kernel combines the partials.  The prefix chunks run on
- * warp-level mma.sync by default; the environment variable PKV_CASCADE_TC=1
- * selects tcgen05 MMAs with TMEM accumulators instead (same results up to
- * fp32 rounding order).  Workspace:
+ * Work: one launch computes each group's prefix attention in chunks of 8
+ * blocks on the 5th-generation tensor cores (tcgen05.mma, queries of all
+ * members x heads as the MMA rows, products in tensor memory) beside split-K
+ * units (partition_tokens, <= 0: 512) that cover each sequence past its
+ * prefix; a merge kernel combines the partials.  Workspace:
  * pkv_decode_prefix_workspace_bytes(...), else PKV_ERR_WORKSPACE.
  * max_suffix_blocks: an upper bound on ceil(len / 16) - prefix_blocks over the
  * batch (the blocks past each sequence's prefix), or <= 0 for "unknown"

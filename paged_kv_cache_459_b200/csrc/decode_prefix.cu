@@ -5,17 +5,17 @@
 // requests with a common prefix point at one set of blocks) need the same
 // prefix K/V.  Plain decode streams those shared blocks once per sequence;
 // here they are read once per (group, KV head) and the attention of every
-// member's query against them is computed as one dense product:
-//   rows = (member, query head of this KV head) pairs, 16 per warp tile,
-//   S[16 rows x 16 tokens] = Q . K_blk^T  and  O[16 x d] += P . V_blk
-// on mma.m16n8k16 (bf16 in, fp32 accumulate) -- with 128 members this is a
-// 128-row tile per KV head, a real dense contraction.  (The same chunk runs
-// on tcgen05 with TMEM accumulators when selected: prefix_unit_tc below.)
-// Each CTA takes a chunk of CB prefix blocks, loads its K and V tiles once
-// with TMA, and leaves one partial (m, l, o) per row.  The private suffixes go through the split-K
-// kernel starting past the prefix, and the merge below combines prefix and
-// suffix partials of each (sequence, query head) by log-sum-exp.  The result
-// equals plain decode over the whole sequence.
+// member's query against them is computed as one dense product -- rows =
+// (member, query head of this KV head) pairs, 128 per tile, against a chunk
+// of the prefix's keys -- on the tcgen05 tensor cores with the products in
+// TMEM (prefix_unit_tc below); with 128 members that is a 128-row tile per KV
+// head, a real dense contraction.  (A warp-level mma.sync version of the
+// chunk measured 1-2.5 % slower per step beside the suffix stream.)  Each
+// prefix CTA takes a chunk of CB prefix blocks, loads its K and V tiles once
+// with TMA, and leaves one partial (m, l, o) per row.  The private suffixes go
+// through the split-K kernel starting past the prefix, and the merge below
+// combines prefix and suffix partials of each (sequence, query head) by
+// log-sum-exp.  The result equals plain decode over the whole sequence.
 #include <algorithm>
 
 #include "decode_unit.cuh"
@@ -28,234 +28,6 @@ namespace {
 using namespace dev;
 
 constexpr int kPrefixWarps = 4;
-constexpr float kLazyRescale = 8.0f;  // log2 units: the running max moves past this growth only
-
-template <int D, int CB>
-struct PrefixMmaGeometry {
-    static constexpr int kTile = (D / 64) * kBoxBytes;  // one K or V tile of a block
-    static constexpr int kSmemBytes = 2 * CB * kTile + 8 + CB * 4 + 1024;
-};
-
-// Prefix chunk c (blocks [c*CB, (c+1)*CB) of group g's shared prefix) for KV
-// head kvh: all member rows against the chunk's K/V, one partial per row.
-template <int D, int CB>
-__device__ __forceinline__ void prefix_unit_mma(const CUtensorMap &tmk, const CUtensorMap &tmv,
-                                            const PrefixParams &p, int c, int kvh, int g) {
-    constexpr int KS = D / 16;                     // k-steps of S = Q K^T over d
-    constexpr int NT = D / 8;                      // 8-column tiles of O
-    constexpr int kTile = PrefixMmaGeometry<D, CB>::kTile;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tig = lane & 3, gid = lane >> 2;
-
-    const int off = __ldg(p.group_offsets + g);
-    const int members = __ldg(p.group_offsets + g + 1) - off;
-    if (members <= 0) return;
-    const int b0 = __ldg(p.group_seqs + off);
-    if (b0 < 0 || b0 >= p.B) {
-        if (threadIdx.x == 0) flag(p.err, PKV_DEV_ERR_BAD_LEN);
-        return;
-    }
-    int len0 = __ldg(p.seq_lens + b0);
-    len0 = len0 < 0 ? 0 : min(len0, p.W * kBlockTokens);
-    const int nb = min(max(__ldg(p.prefix_blocks + b0), 0), len0 / kBlockTokens);  // full blocks
-    const int j0 = c * CB, j1 = min(nb, j0 + CB);
-    if (j0 >= j1) return;
-    const int nt = j1 - j0;
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *ktiles = smem;                    // [CB][kTile]
-    uint8_t *vtiles = smem + CB * kTile;       // [CB][kTile]
-    const uint32_t bar = smem_u32(smem + 2 * CB * kTile);
-    int *valid = reinterpret_cast<int *>(smem + 2 * CB * kTile + 8);  // [CB]
-
-    if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-        prefetch_tmap(&tmk);
-        prefetch_tmap(&tmv);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int32_t *row = p.block_tables + static_cast<size_t>(b0) * p.W;
-        uint32_t bytes = 0;
-        for (int t = 0; t < nt; ++t) {
-            const int32_t phys = __ldg(row + j0 + t);
-            valid[t] = phys >= 0 && phys < p.num_blocks ? phys : -1;
-            if (valid[t] >= 0) bytes += 2 * kTile;
-        }
-        mbar_arrive_expect_tx(bar, bytes);
-        const uint64_t policy = l2_policy_evict_first();
-        for (int t = 0; t < nt; ++t) {
-            if (valid[t] < 0) {
-                flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
-                continue;
-            }
-            const int y = valid[t] * (p.Hkv * kBlockTokens) + kvh * kBlockTokens;
-#pragma unroll
-            for (int hh = 0; hh < D / 64; ++hh) {
-                tma_load_2d(smem_u32(ktiles + t * kTile) + hh * kBoxBytes, &tmk, hh * 64, y, bar, policy);
-                tma_load_2d(smem_u32(vtiles + t * kTile) + hh * kBoxBytes, &tmv, hh * 64, y, bar, policy);
-            }
-        }
-    }
-    __syncthreads();  // valid[] written
-    if (!mbar_wait(bar, 0, kWaitLimitNs)) {
-        if (threadIdx.x == 0) flag(p.err, PKV_DEV_ERR_TIMEOUT);
-        mbar_wait(bar, 0, kWaitLimitNs);  // let copies in flight land before exiting
-        return;
-    }
-
-    const int G = p.group;        // query heads per KV head
-    const int R = members * G;    // query rows of this group and KV head
-    for (int rt = warp; rt * 16 < R; rt += kPrefixWarps) {
-        // Q rows (member, head) as mma A fragments: rows gid and gid + 8.
-        int rb[2], rh[2];
-        const uint32_t *qr[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = rt * 16 + gid + 8 * i;
-            rb[i] = -1;
-            rh[i] = 0;
-            qr[i] = nullptr;
-            if (r < R) {
-                const int b = __ldg(p.group_seqs + off + r / G);
-                if (b >= 0 && b < p.B) {
-                    rb[i] = b;
-                    rh[i] = kvh * G + r % G;
-                    qr[i] = reinterpret_cast<const uint32_t *>(p.q + (static_cast<size_t>(b) * p.Hq + rh[i]) * D);
-                }
-            }
-        }
-        uint32_t qa[KS][4];
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qa[ks][0] = qr[0] ? __ldg(qr[0] + (16 * ks + 2 * tig) / 2) : 0u;
-            qa[ks][1] = qr[1] ? __ldg(qr[1] + (16 * ks + 2 * tig) / 2) : 0u;
-            qa[ks][2] = qr[0] ? __ldg(qr[0] + (16 * ks + 8 + 2 * tig) / 2) : 0u;
-            qa[ks][3] = qr[1] ? __ldg(qr[1] + (16 * ks + 8 + 2 * tig) / 2) : 0u;
-        }
-        float o[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) o[n][i] = 0.f;
-        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-
-        // Two blocks (32 tokens) per step: S for both, one row-max update,
-        // one (rare) rescale, then P.V for each block.  The running max only
-        // moves when a row's max grows by more than 2^8, so O is rescaled
-        // seldom and P stays <= 2^8; the partial's m is that base.
-        for (int t0 = 0; t0 < nt; t0 += 2) {
-            const bool v0 = valid[t0] >= 0, v1 = t0 + 1 < nt && valid[t0 + 1] >= 0;
-            float s[4][4];  // 8-token column tiles: block t0 tokens 0-7, 8-15, block t0+1 0-7, 8-15
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) s[n][i] = 0.f;
-            {
-                const int tok = (lane & 7) + (lane >> 4) * 8;
-                const int cb = (lane >> 3) & 1;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    if (!(half ? v1 : v0)) continue;
-                    const uint32_t kt = smem_u32(ktiles + (t0 + half) * kTile);
-#pragma unroll
-                    for (int ks = 0; ks < KS; ++ks) {
-                        uint32_t b00, b01, b10, b11;
-                        ldmatrix_x4(kt + tile_off(tok, 2 * ks + cb), b00, b01, b10, b11);
-                        mma_bf16_16816(s[2 * half], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
-                        mma_bf16_16816(s[2 * half + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
-                    }
-                }
-            }
-            // scores in the exp2 domain; a block that is not there scores -inf
-#pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const bool there = n < 2 ? v0 : v1;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) s[n][i] = there ? s[n][i] * p.scale_log2 : -INFINITY;
-            }
-            // row gid: s[n][0], s[n][1]; row gid + 8: s[n][2], s[n][3]
-            float mx0 = fmaxf(fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1])),
-                              fmaxf(fmaxf(s[2][0], s[2][1]), fmaxf(s[3][0], s[3][1])));
-            float mx1 = fmaxf(fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3])),
-                              fmaxf(fmaxf(s[2][2], s[2][3]), fmaxf(s[3][2], s[3][3])));
-#pragma unroll
-            for (int m = 1; m < 4; m <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, m));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, m));
-            }
-            const bool g0 = mx0 > m_run[0] + kLazyRescale || (m_run[0] == -INFINITY && mx0 != -INFINITY);
-            const bool g1 = mx1 > m_run[1] + kLazyRescale || (m_run[1] == -INFINITY && mx1 != -INFINITY);
-            const float al0 = g0 && m_run[0] != -INFINITY ? ex2_approx(m_run[0] - mx0) : 1.f;
-            const float al1 = g1 && m_run[1] != -INFINITY ? ex2_approx(m_run[1] - mx1) : 1.f;
-            if (g0) m_run[0] = mx0;
-            if (g1) m_run[1] = mx1;
-            if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    o[n][0] *= al0;
-                    o[n][1] *= al0;
-                    o[n][2] *= al1;
-                    o[n][3] *= al1;
-                }
-            }
-            const float nb0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
-            const float nb1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
-            float pr[4][4];
-            float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                pr[n][0] = ex2_approx(s[n][0] - nb0);
-                pr[n][1] = ex2_approx(s[n][1] - nb0);
-                pr[n][2] = ex2_approx(s[n][2] - nb1);
-                pr[n][3] = ex2_approx(s[n][3] - nb1);
-                sum0 += pr[n][0] + pr[n][1];
-                sum1 += pr[n][2] + pr[n][3];
-            }
-            l_run[0] = l_run[0] * al0 + sum0;
-            l_run[1] = l_run[1] * al1 + sum1;
-            const int tok = (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int cb = lane >> 4;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                if (!(half ? v1 : v0)) continue;
-                const uint32_t vt = smem_u32(vtiles + (t0 + half) * kTile);
-                const uint32_t pa0 = pack_bf16x2(pr[2 * half][0], pr[2 * half][1]);
-                const uint32_t pa1 = pack_bf16x2(pr[2 * half][2], pr[2 * half][3]);
-                const uint32_t pa2 = pack_bf16x2(pr[2 * half + 1][0], pr[2 * half + 1][1]);
-                const uint32_t pa3 = pack_bf16x2(pr[2 * half + 1][2], pr[2 * half + 1][3]);
-#pragma unroll
-                for (int i = 0; i < NT / 2; ++i) {
-                    uint32_t w0, w1, w2, w3;
-                    ldmatrix_x4_trans(vt + tile_off(tok, 2 * i + cb), w0, w1, w2, w3);
-                    mma_bf16_16816(o[2 * i], pa0, pa1, pa2, pa3, w0, w1);
-                    mma_bf16_16816(o[2 * i + 1], pa0, pa1, pa2, pa3, w2, w3);
-                }
-            }
-        }
-#pragma unroll
-        for (int m = 1; m < 4; m <<= 1) {
-            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], m);
-            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], m);
-        }
-        // partial of (sequence, head) for prefix chunk c
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            if (rb[i] < 0) continue;
-            const size_t slot = (static_cast<size_t>(rb[i]) * p.Hq + rh[i]) * p.ws_parts + c;
-            float *dst = p.ws_o + slot * D;
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-                *reinterpret_cast<float2 *>(dst + 8 * n + 2 * tig) = make_float2(o[n][2 * i], o[n][2 * i + 1]);
-            if (tig == 0) {
-                p.ws_ml[2 * slot] = m_run[i];
-                p.ws_ml[2 * slot + 1] = l_run[i];
-            }
-        }
-    }
-}
 
 template <int D, int CB>
 struct PrefixTcGeometry {
@@ -613,8 +385,8 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
 // evenly through the grid, so that every SM runs the short, latency-bound
 // prefix work beside the bandwidth-bound suffix stream; the other CTAs take
 // suffix units in order (partition fastest, then head segment, then
-// sequence).  TC: the prefix chunks on tcgen05 (else mma.sync).
-template <int D, bool MMA, bool TC>
+// sequence).
+template <int D, bool MMA>
 __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const PrefixParams pp, const DecodeParams dp, int n_pre) {
@@ -625,17 +397,14 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
         id /= stride;
         const int c = id % pp.prefix_parts;
         id /= pp.prefix_parts;
-        if constexpr (TC)
-            prefix_unit_tc<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
-        else
-            prefix_unit_mma<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
+        prefix_unit_tc<D, kPrefixChunkBlocks>(tmk, tmv, pp, c, id % pp.Hkv, id / pp.Hkv);
         return;
     }
     // Suffix units use no TMEM: they give up the right to allocate at once.
     // A CTA that keeps it (until it exits) holds up the TMEM allocation of a
     // prefix CTA that starts after it on the same SM (measured: the step took
     // twice as long).
-    if (TC && n_pre > 0 && threadIdx.x < 32) tc::relinquish();
+    if (n_pre > 0 && threadIdx.x < 32) tc::relinquish();
     if (n_pre > 0) id -= min(id / stride + 1, n_pre);  // prefix CTAs at or before this one
     const int ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
     const int part = id % dp.num_parts;
@@ -652,13 +421,12 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
     decode_unit<D, kPrefixWarps, 2, MMA, kModeSplit>(tmk, tmv, dp, part, id % ny, b);
 }
 
-template <int D, bool MMA, bool TC>
+template <int D, bool MMA>
 cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                              const DecodeParams &dp, int num_groups, cudaStream_t stream) {
-    constexpr int kPre = TC ? PrefixTcGeometry<D, kPrefixChunkBlocks>::kSmemBytes
-                            : PrefixMmaGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
+    constexpr int kPre = PrefixTcGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
     constexpr int kSmem = std::max(kPre, Geometry<D, kPrefixWarps, 2>::kSmemBytes);
-    auto kern = cascade_kernel<D, MMA, TC>;
+    auto kern = cascade_kernel<D, MMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const long long n_pre = static_cast<long long>(pp.prefix_parts) * pp.Hkv * num_groups;
@@ -675,22 +443,17 @@ cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, con
 
 template <int D>
 cudaError_t launch_cascade_h(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
-                             const DecodeParams &dp, int num_groups, bool prefix_tc, cudaStream_t stream) {
-    const bool mma = dp.group > 1;
-    if (prefix_tc)
-        return mma ? launch_cascade_d<D, true, true>(tmk, tmv, pp, dp, num_groups, stream)
-                   : launch_cascade_d<D, false, true>(tmk, tmv, pp, dp, num_groups, stream);
-    return mma ? launch_cascade_d<D, true, false>(tmk, tmv, pp, dp, num_groups, stream)
-               : launch_cascade_d<D, false, false>(tmk, tmv, pp, dp, num_groups, stream);
+                             const DecodeParams &dp, int num_groups, cudaStream_t stream) {
+    return dp.group > 1 ? launch_cascade_d<D, true>(tmk, tmv, pp, dp, num_groups, stream)
+                        : launch_cascade_d<D, false>(tmk, tmv, pp, dp, num_groups, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
-                           const DecodeParams &dp, int head_dim, int num_groups, bool prefix_tc,
-                           cudaStream_t stream) {
-    if (head_dim == 128) return launch_cascade_h<128>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
-    if (head_dim == 64) return launch_cascade_h<64>(tmk, tmv, pp, dp, num_groups, prefix_tc, stream);
+                           const DecodeParams &dp, int head_dim, int num_groups, cudaStream_t stream) {
+    if (head_dim == 128) return launch_cascade_h<128>(tmk, tmv, pp, dp, num_groups, stream);
+    if (head_dim == 64) return launch_cascade_h<64>(tmk, tmv, pp, dp, num_groups, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -93,12 +93,11 @@ struct PrefixParams {
     float scale_log2;
 };
 
-// One launch running prefix chunks and suffix split-K units side by side,
-// then the merge.  dp must describe split-K with start_blocks = prefix_blocks.
-// prefix_tc: the prefix chunks on tcgen05/TMEM instead of mma.sync.
+// One launch running prefix chunks (tcgen05/TMEM) and suffix split-K units
+// side by side, then the merge.  dp must describe split-K with start_blocks
+// = prefix_blocks.
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
-                           const DecodeParams &dp, int head_dim, int num_groups, bool prefix_tc,
-                           cudaStream_t stream);
+                           const DecodeParams &dp, int head_dim, int num_groups, cudaStream_t stream);
 
 // Causal prefill attention of each sequence's new tokens over its paged K/V.
 struct PrefillParams {

@@ -526,9 +526,7 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     dp.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
     dp.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
 
-    // mma.sync prefix chunks by default; PKV_CASCADE_TC=1 selects the tcgen05 ones
     cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
-                                        env_int("PKV_CASCADE_TC", 0) != 0,
                                         static_cast<cudaStream_t>(stream));
     return cuda_status(e);
 }

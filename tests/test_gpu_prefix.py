@@ -49,18 +49,8 @@ CASES = [
 ]
 
 
-@pytest.fixture(params=["mma_sync", "tcgen05"])
-def prefix_impl(request, monkeypatch):
-    """The prefix chunks on warp-level mma.sync (default) or on tcgen05/TMEM."""
-    if request.param == "tcgen05":
-        monkeypatch.setenv("PKV_CASCADE_TC", "1")
-    else:
-        monkeypatch.delenv("PKV_CASCADE_TC", raising=False)
-    return request.param
-
-
 @pytest.mark.parametrize("name,kw", CASES, ids=[str(i) for i in range(len(CASES))])
-def test_cascade_matches_oracle(name, kw, prefix_impl):
+def test_cascade_matches_oracle(name, kw):
     w = build(name, 13, **kw)
     d = DeviceStep(w)
     d.write()
@@ -83,7 +73,7 @@ def test_cascade_suffix_bound_too_small_is_flagged():
     assert d.err_word() & 4
 
 
-def test_cascade_full_size(prefix_impl):
+def test_cascade_full_size():
     """The prefix workload at full size (128 sequences sharing a 2000-token
     prefix): every output row against the oracle."""
     w = build("prefix", 0)
@@ -97,7 +87,7 @@ def test_cascade_full_size(prefix_impl):
     assert d.err_word() == 0
 
 
-def test_cascade_block_relabelling_is_bit_exact(prefix_impl):
+def test_cascade_block_relabelling_is_bit_exact():
     w = build("prefix", 14, batch=10, prefix_len=256, suffix_lo=1, suffix_hi=80, prefix_groups=2)
     d = DeviceStep(w)
     d.write()
@@ -112,7 +102,7 @@ def test_cascade_block_relabelling_is_bit_exact(prefix_impl):
 
 
 @pytest.mark.parametrize("idx", [0, 1, 2, 3])
-def test_cascade_fused_step(idx, prefix_impl):
+def test_cascade_fused_step(idx):
     """pkv_paged_decode_prefix_step: the step's write fused into the cascade --
     caches bit-exact with the oracle's write, output within tolerance, and
     bit-identical to the separate write + cascade."""
