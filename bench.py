@@ -408,6 +408,20 @@ class Resident:
                                        partition_tokens=self.partition, workspace=self.ws,
                                        err=self.err)
 
+    def add_cache_copies(self, n: int):
+        """n more copies of the K/V pool -- the caches of a model's other layers:
+        steps that rotate over them find none of their K/V in L2."""
+        self.caches = [(self.kc, self.vc)] + [(self.kc.clone(), self.vc.clone()) for _ in range(n)]
+        self.cur = 0
+
+    def next_cache(self):
+        self.cur = (self.cur + 1) % len(self.caches)
+        self.kc, self.vc = self.caches[self.cur]
+
+    def drop_cache_copies(self):
+        self.kc, self.vc = self.caches[0]
+        self.caches, self.cur = [(self.kc, self.vc)], 0
+
     def step(self, c=None, o=None):
         if self.fused:
             self.fused_step(c, o)
@@ -521,9 +535,36 @@ def device_steps(step, K: int, dev, flush_buf=None):
     return [a.elapsed_time(b) for a, b in ev], t0.elapsed_time(t1)
 
 
+def rotating_steps(r: Resident, K: int, dev, fn=None) -> float:
+    """Device time (ms) of K steps (fn, default r.step) back to back, each on
+    the next copy of the K/V pool (Resident.add_cache_copies)."""
+    import torch
+
+    fn = fn or r.step
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    torch.cuda._sleep(SPIN_CYCLES_LEAD)
+    t0.record()
+    for _ in range(K):
+        r.next_cache()
+        fn()
+    t1.record()
+    torch.cuda.synchronize(dev)
+    return t0.elapsed_time(t1)
+
+
 def timed_decode(r: Resident, K: int, W: int, *, world: int, sampler=None, flush=None) -> dict:
     """W warm-up steps, then K timed steps of the resident workload; returns the
-    line's numbers for it (and its clocks when a sampler runs)."""
+    line's numbers for it (and its clocks when a sampler runs).
+
+    A workload whose K/V fits in L2 is timed two ways.  Rotating (the step
+    time reported): the pool is copied until the copies hold over 3 L2 sizes
+    and each step runs on the next copy, K steps back to back between two
+    events -- as in a model, whose layers each read their own cache, so that a
+    step's K/V were last touched two L2 sizes of traffic ago.  Flushed
+    (reported beside it): L2 emptied before every step and each step timed
+    alone by its own events, which adds the launch and event overhead of an
+    isolated kernel (about 5 us on a B200 for an empty kernel)."""
     import torch
 
     for _ in range(W):
@@ -532,8 +573,8 @@ def timed_decode(r: Resident, K: int, W: int, *, world: int, sampler=None, flush
             r.two_calls()
     r.check_err("after warm-up")
     ab = r.bytes()
-    if flush is None:
-        flush = ab["kv"] <= L2_BYTES
+    if flush is None:  # the same choice on every rank
+        flush = max_over_ranks([float(ab["kv"])], device=r.dev)[0] <= L2_BYTES
     flush_buf = L2Flush(r.dev) if flush else None
     if world > 1:
         import torch.distributed as dist
@@ -543,6 +584,28 @@ def timed_decode(r: Resident, K: int, W: int, *, world: int, sampler=None, flush
         import torch.distributed as dist
         dist.barrier()
     total_ms = sum(per) if flush else loop_ms  # the flushes are not the step's work
+    flushed_us, copies = None, 1
+    if flush:
+        del flush_buf
+        pool = 2 * r.kc.numel() * r.kc.element_size()
+        copies = max(2, -(-3 * L2_BYTES // max(ab["kv"], 1)))
+        free = torch.cuda.mem_get_info(r.dev)[0]
+        copies = int(min(copies, 1 + (free // 2) // max(pool, 1)))
+        r.add_cache_copies(copies - 1)
+        for _ in range(2 * copies):  # every copy written and read once
+            r.next_cache()
+            r.step()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        loop_ms = rotating_steps(r, K, r.dev)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        r.drop_cache_copies()
+        flushed_us = 1e3 * statistics.fmean(per)
+        per = [loop_ms / K] * K
+        total_ms = loop_ms
     clocks = None
     if sampler is not None:  # keep the GPU loaded long enough for the sampler to see it
         t0 = time.perf_counter()
@@ -558,6 +621,9 @@ def timed_decode(r: Resident, K: int, W: int, *, world: int, sampler=None, flush
     achieved = ab["decode"] / (step_us * 1e-6) / 1e9
     return {
         "step_us": step_us, "total_ms": total_ms, "flush": flush, "bytes": ab,
+        "flushed_step_us": flushed_us, "cache_copies": copies,
+        "flushed_frac_of_measured_copy": None if flushed_us is None else
+        ab["decode"] / (flushed_us * 1e-6) / 1e9 / peak,
         "value": job_throughput(r.B, K, world, total_ms),
         "kv_hbm_gbs": achieved,
         "kv_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
@@ -594,10 +660,13 @@ def workload_key(args, name, *, dev, cascade=False, batch=None, clocks=True) -> 
         "decode_us": m["step_us"], "value": m["value"], "unit": UNIT,
         "kv_hbm_gbs": m["kv_hbm_gbs"], "kv_frac_of_8tbs": m["kv_frac_of_8tbs"],
         "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
-        "l2": "flushed between steps (256 MB write, then 256 MB read), step time from per-step events"
+        "l2": (f"inputs smaller than L2: each step on the next of {m['cache_copies']} copies of "
+               f"the K/V pool (over 3 L2 sizes, as a model's layers), K steps back to back")
         if m["flush"] else "inputs larger than L2, no flush",
         "roofline": m["roofline"], "gpu_launches": args.steps * r.launches_per_step(),
     }
+    if m["flush"]:
+        out["flushed"] = flushed_key(m)
     if clocks:
         out["clocks"] = m["clocks"]
     if cascade:
@@ -607,6 +676,14 @@ def workload_key(args, name, *, dev, cascade=False, batch=None, clocks=True) -> 
     del r
     torch.cuda.empty_cache()
     return out
+
+
+def flushed_key(m: dict) -> dict:
+    """The same step timed alone: L2 flushed before it, its own two events."""
+    return {"step_us": m["flushed_step_us"],
+            "kv_frac_of_measured_copy": m["flushed_frac_of_measured_copy"],
+            "how": "L2 flushed before every step (256 MB write, then 256 MB read), each step "
+                   "between its own two events; an empty kernel measures ~5 us this way"}
 
 
 def batch_sweep_key(args, dev) -> dict:
@@ -620,11 +697,16 @@ def batch_sweep_key(args, dev) -> dict:
     for B in (1, 8, 32, 64, 128):
         r = Resident(args, "llama", args.seed, dev, batch=B)
         m = timed_decode(r, args.steps, max(3, args.warmup), world=1)
-        rows.append({"batch": B, "variant": r.variant_text(), "decode_us": m["step_us"],
-                     "kv_hbm_gbs": m["kv_hbm_gbs"],
-                     "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
-                     "value": m["value"], "l2": "flushed" if m["flush"] else "larger than L2",
-                     "algorithmic_bytes_per_launch": m["bytes"]["decode"]})
+        row = {"batch": B, "variant": r.variant_text(), "decode_us": m["step_us"],
+               "kv_hbm_gbs": m["kv_hbm_gbs"],
+               "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
+               "value": m["value"],
+               "l2": f"rotating over {m['cache_copies']} pool copies" if m["flush"] else
+               "larger than L2",
+               "algorithmic_bytes_per_launch": m["bytes"]["decode"]}
+        if m["flush"]:
+            row["flushed"] = flushed_key(m)
+        rows.append(row)
         last = r
         if B != 128:
             del r
@@ -673,14 +755,23 @@ def run_gpu(args):
     fused = r.fused
     unfused = None
     if fused:  # the same step as two calls (write, then decode), for comparison
-        flush_buf = L2Flush(dev) if m["flush"] else None
-        uw, _ = device_steps(r.write, K, dev, flush_buf)  # the write call alone
-        per, loop = device_steps(r.two_calls, K, dev, flush_buf)
-        u_ms = max_over_ranks([sum(per) if m["flush"] else loop], device=dev)[0]
+        if m["flush"]:  # timed as the fused step was: rotating over copies of the pool
+            r.add_cache_copies(m["cache_copies"] - 1)
+            for _ in range(2 * m["cache_copies"]):
+                r.next_cache()
+                r.two_calls()
+            uw_ms = rotating_steps(r, K, dev, r.write)
+            loop = rotating_steps(r, K, dev, r.two_calls)
+            r.drop_cache_copies()
+            uw, per = [uw_ms / K] * K, [loop / K] * K
+        else:
+            _, uw_ms = device_steps(r.write, K, dev)  # the write call alone
+            uw = [uw_ms / K] * K
+            per, loop = device_steps(r.two_calls, K, dev)
+        u_ms = max_over_ranks([loop], device=dev)[0]
         unfused = {"step_us": 1e3 * statistics.fmean(per), "write_us": 1e3 * statistics.fmean(uw),
                    "value": job_throughput(B, K, world, u_ms),
-                   "how": "write + decode calls per step; write_us from a loop of the write alone"}
-        del flush_buf
+                   "how": "write + decode calls per step; write_us from K writes alone back to back"}
 
     # End to end through the public API: every step's inputs (q, new K/V, tables, lengths,
     # slots) go host -> device from one pinned staging buffer, and its output comes back.
@@ -797,9 +888,10 @@ def run_gpu(args):
             "tokens": ab["tokens"], "num_blocks": r.w.num_blocks, "table_width": W,
             "variant": r.variant_text(),
             "logical_kv_bytes": ab["kv"],
-            "l2": (f"L2 flushed between steps (a 256 MB write, then a 256 MB read, so no dirty "
-                   f"lines either); step time from per-step events "
-                   f"(KV {ab['kv'] / 1e9:.3f} GB per step)") if m["flush"] else
+            "l2": (f"inputs smaller than L2 (KV {ab['kv'] / 1e9:.3f} GB per step): each step runs "
+                   f"on the next of {m['cache_copies']} copies of the K/V pool (over 3 L2 sizes, "
+                   f"as a model's layers each read their own cache), K steps back to back; the "
+                   f"'flushed' key times each step alone after an L2 flush") if m["flush"] else
                   f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), no flush",
             "timing": "CUDA events on the launching stream; a spin kernel lets the host enqueue "
                       "ahead of the device, outside the steps' events",
@@ -815,6 +907,7 @@ def run_gpu(args):
                 ": the write fused into the decode kernel" if fused else
                 "pkv_paged_kv_write, then the decode call",
         "unfused": unfused,
+        "flushed": flushed_key(m) if m["flush"] else None,
         "roofline": m["roofline"],
         "gpu_launches": K * r.launches_per_step(),
         "e2e": {"value": job_throughput(B, K, world, e2e_ms), "unit": UNIT,

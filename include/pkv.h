@@ -204,6 +204,10 @@ PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *q, const vo
  * PKV_DECODE_STAGES (read at each call) pick the decode CTA shape of the
  * single-pass and split-K kernels: 4 warps x 2 ring stages (the default,
  * measured fastest), 4 x 3 or 2 x 2; other values give the default.
+ * PKV_DECODE_L2_AHEAD (0..16, read at each call, also by the shared-prefix
+ * calls) makes every decode warp ask L2 for that many of its blocks beyond
+ * its ring (bulk L2 prefetches), so that short work units put all their
+ * reads to DRAM at once.
  */
 PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,

@@ -170,9 +170,9 @@ template <int D, int NW, int S, bool MMA, int MODE>
 cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                        cudaStream_t stream) {
     using G = Geometry<D, NW, S>;
+    constexpr int kSmem = MODE == kModeCluster ? G::kClusterSmemBytes : G::kSmemBytes;
     auto kern = paged_decode_kernel<D, NW, S, MMA, MODE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         G::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     const dim3 grid(static_cast<unsigned>(p.num_parts),
                     static_cast<unsigned>(MMA ? p.Hkv * p.chunks : p.Hq),
@@ -181,7 +181,7 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = grid;
         cfg.blockDim = dim3(NW * 32);
-        cfg.dynamicSmemBytes = G::kSmemBytes;
+        cfg.dynamicSmemBytes = kSmem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[2];
         unsigned n = 0;
@@ -199,7 +199,7 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
         cfg.numAttrs = n;
         e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p);
     } else {
-        kern<<<grid, NW * 32, G::kSmemBytes, stream>>>(tmk, tmv, p);
+        kern<<<grid, NW * 32, kSmem, stream>>>(tmk, tmv, p);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess || MODE != kModeSplit || p.skip_merge) return e;

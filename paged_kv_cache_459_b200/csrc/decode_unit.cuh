@@ -40,16 +40,35 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     // cluster mode), they are loaded now, beside the length, for every block
     // the table row holds in this unit's range; entries past the sequence are
     // read but never used.  Otherwise after the length, below.
+    // Cluster mode with a table row of at most kStagedTable entries: the whole
+    // row is read into shared memory beside the length (the part's range needs
+    // the length), and the window reads it there.
     const bool early_table = !CLUSTER && p.start_blocks == nullptr;
     TableWindow tw;
     tw.row = p.block_tables + static_cast<size_t>(b) * p.W;
     tw.stride = kStride;
+    tw.shared_row = false;
     if (early_table) {
         const int first_blk = part * p.part_blocks;
         const int last_blk = min(p.W, first_blk + p.part_blocks);  // exclusive, within the row
         tw.first = first_blk + lead;
         tw.count = last_blk - tw.first > 0 ? (last_blk - tw.first + kStride - 1) / kStride : 0;
         tw.init(lane);
+    }
+    extern __shared__ uint8_t smem_raw[];
+    // Stage buffers must sit on 1024-byte boundaries for the 128-byte swizzle.
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    constexpr int kTabPer = CLUSTER ? kStagedTable / (NW * 32) : 1;
+    const bool staged = CLUSTER && p.W <= kStagedTable;
+    int32_t tab[kTabPer];
+    if constexpr (CLUSTER) {
+        if (staged) {
+#pragma unroll
+            for (int k = 0; k < kTabPer; ++k) {
+                const int j = threadIdx.x + k * NW * 32;
+                tab[k] = j < p.W ? __ldg(tw.row + j) : -1;
+            }
+        }
     }
 
     int len = __ldg(p.seq_lens + b);
@@ -81,11 +100,20 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         return;
     }
 
-    extern __shared__ uint8_t smem_raw[];
-    // Stage buffers must sit on 1024-byte boundaries for the 128-byte swizzle.
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *ring = smem + warp * S * G::kStageBytes;
     const uint32_t bars = smem_u32(smem + G::kRingBytes) + warp * S * 8;
+    if constexpr (CLUSTER) {
+        if (staged) {
+            int32_t *tab_s = reinterpret_cast<int32_t *>(smem + G::kRingBytes + NW * S * 8);
+#pragma unroll
+            for (int k = 0; k < kTabPer; ++k) {
+                const int j = threadIdx.x + k * NW * 32;
+                if (j < p.W) tab_s[j] = tab[k];
+            }
+            tw.row = tab_s;
+            tw.shared_row = true;
+        }
+    }
 
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(bars + 8 * s, 1);
@@ -125,6 +153,24 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
             }
         }
     };
+
+    // L2 read-ahead: block i + S + ahead is asked for when block i + S is
+    // loaded, and blocks S .. S + ahead - 1 at the start (lane j takes block
+    // S + j, its table entry fetched from the window by shuffle).
+    const int ahead = p.l2_ahead;
+    auto prefetch_l2 = [&](int32_t phys) {  // one lane
+        if (phys >= 0 && phys < p.num_blocks) {
+            const size_t off = (static_cast<size_t>(phys) * p.Hkv + kvh) * kBlockTokens * D;
+            bulk_prefetch_l2(p.k_cache + off, kBlockTokens * D * 2);
+            bulk_prefetch_l2(p.v_cache + off, kBlockTokens * D * 2);
+        }
+    };
+    if (ahead > 0) {
+        const int i = S + lane;  // < 64: in the window's first two chunks
+        const int32_t a = __shfl_sync(0xffffffffu, tw.cur, i & 31);
+        const int32_t c = __shfl_sync(0xffffffffu, tw.nxt, i & 31);
+        if (lane < ahead && i < n_mine) prefetch_l2(i < 32 ? a : c);
+    }
 
     using Head = typename std::conditional<MMA, GroupHeads<D>, ScalarHead<D>>::type;
     Head st;
@@ -192,6 +238,10 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         if (i + S < n_mine) {
             if (writer && i + S == i_write) store_new();
             issue(i + S);
+            if (ahead > 0 && i + S + ahead < n_mine) {
+                const int32_t ph = tw.get(i + S + ahead);
+                if (lane == 1) prefetch_l2(ph);
+            }
         }
     }
     if (i < n_mine) {
@@ -263,15 +313,26 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         const int lo = static_cast<int>(cluster_ctarank()) * per, hi = min(total, lo + per);
         for (int idx = lo + threadIdx.x; idx < hi; idx += NW * 32) {
             const int n = idx / D, e = idx % D;
+            // every part's m, l and o requested at once (one round trip through
+            // the cluster), then combined in part order
+            float mc[kMaxClusterParts], lc[kMaxClusterParts], oc[kMaxClusterParts];
+#pragma unroll
+            for (int c = 0; c < kMaxClusterParts; ++c) {
+                mc[c] = c < P ? ld_dsmem_f32(xch + n, c) : -INFINITY;
+                lc[c] = c < P ? ld_dsmem_f32(xch + 8 + n, c) : 0.f;
+                oc[c] = c < P ? ld_dsmem_f32(xch + 16 + n * D + e, c) : 0.f;
+            }
             float M = -INFINITY;
-            for (int c = 0; c < P; ++c) M = fmaxf(M, ld_dsmem_f32(xch + n, c));
+#pragma unroll
+            for (int c = 0; c < kMaxClusterParts; ++c) M = fmaxf(M, mc[c]);
             float L = 0.f, O = 0.f;
             if (M != -INFINITY) {
-                for (int c = 0; c < P; ++c) {
-                    const float mc = ld_dsmem_f32(xch + n, c);
-                    const float wgt = mc == -INFINITY ? 0.f : exp2f(mc - M);
-                    L = fmaf(ld_dsmem_f32(xch + 8 + n, c), wgt, L);
-                    O = fmaf(ld_dsmem_f32(xch + 16 + n * D + e, c), wgt, O);
+#pragma unroll
+                for (int c = 0; c < kMaxClusterParts; ++c) {
+                    if (c >= P) break;
+                    const float wgt = mc[c] == -INFINITY ? 0.f : exp2f(mc[c] - M);
+                    L = fmaf(lc[c], wgt, L);
+                    O = fmaf(oc[c], wgt, O);
                 }
             }
             p.out[(static_cast<size_t>(b) * p.Hq + h0 + n) * D + e] =

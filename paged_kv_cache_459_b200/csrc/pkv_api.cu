@@ -213,6 +213,11 @@ int cluster_parts_for(int max_blocks_per_seq, int partition_tokens) {
 // few CTAs for a long context: split-K with the merge kernel balances better.
 constexpr int kClusterMaxPartBlocks = 64;
 
+// L2 read-ahead of the decode units (blocks per warp beyond the TMA ring).
+int l2_ahead_for(int fallback) {
+    return std::clamp(env_int("PKV_DECODE_L2_AHEAD", fallback), 0, pkv::kMaxL2Ahead);
+}
+
 struct DecodePlan {
     int variant;  // PKV_DECODE_SINGLE, _SPLIT or _CLUSTER
     int parts;    // cluster parts per sequence (cluster variant)
@@ -382,6 +387,7 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
         p.order = order;
     }
     pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
+    p.l2_ahead = l2_ahead_for(0);
     cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, mode, t,
                                        static_cast<cudaStream_t>(stream));
     return cuda_status(e);
@@ -525,6 +531,7 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     dp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
     dp.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
     dp.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
+    dp.l2_ahead = l2_ahead_for(0);
 
     cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
                                         static_cast<cudaStream_t>(stream));
