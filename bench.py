@@ -371,6 +371,7 @@ class Resident:
             self.B, self.hq, self.hkv, self.d, W, partition, self.ws.numel())
         self.parts = pkv.decode_cluster_parts_for(self.B, self.hq, self.hkv, self.d, W, self.variant,
                                                   partition, self.ws.numel()) if not cascade else 0
+
         self.fused = not args.unfused
 
     # -- the library calls of one step
@@ -453,16 +454,20 @@ class Resident:
         """Whether the decode runs its sequences longest first (an order kernel)."""
         if self.cascade:
             return False
+        order = (4 * self.B + 255) // 256 * 256
         if self.chosen == self.pkv.DECODE_CLUSTER:
-            return self.B >= 16 and self.ws.numel() >= (4 * self.B + 255) // 256 * 256
+            return self.B >= 16 and self.ws.numel() >= order
+        if self.chosen == self.pkv.DECODE_SPLIT:
+            split = self.pkv.decode_workspace_bytes(self.B, self.hq, self.d, self.W, self.partition)
+            return self.B >= 2 and self.ws.numel() >= (split + 255) // 256 * 256 + order
         return self.chosen == self.pkv.DECODE_SINGLE and self.ws.numel() >= 4 * self.B
 
     def launches_per_step(self) -> int:
         pkv = self.pkv
         if self.cascade:  # (write;) prefix chunks + suffix split-K in one launch, merge
             return 2 if self.fused else 3
-        return (1 if self.fused else 2) + \
-            (1 if self.chosen == pkv.DECODE_SPLIT or self.ordered() else 0)
+        return (1 if self.fused else 2) + (1 if self.chosen == pkv.DECODE_SPLIT else 0) + \
+            (1 if self.ordered() else 0)
 
     def variant_text(self) -> str:
         pkv = self.pkv
@@ -470,7 +475,8 @@ class Resident:
             return "shared-prefix cascade (prefix once per group x KV head, split-K suffixes, merge)"
         return {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head, longest first)"
                 if self.ordered() else "single pass (one CTA per sequence x KV head)",
-                pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % self.partition,
+                pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % self.partition +
+                (", longest first" if self.ordered() else ""),
                 pkv.DECODE_CLUSTER: f"cluster split ({self.parts} equal parts per sequence, one "
                                     f"CTA each, merged in distributed shared memory" +
                                     (", longest first)" if self.ordered() else ")"),
@@ -483,8 +489,8 @@ class Resident:
                     (", fused write" if self.fused else "") + ") + cascade_merge_kernel")
         return (("paged_decode_kernel with the fused write" if self.fused else "paged_decode_kernel")
                 + (" (cluster mode)" if self.chosen == pkv.DECODE_CLUSTER else "")
-                + (" + merge kernel" if self.chosen == pkv.DECODE_SPLIT else
-                   " + order kernel" if self.ordered() else ""))
+                + (" + merge kernel" if self.chosen == pkv.DECODE_SPLIT else "")
+                + (" + order kernel" if self.ordered() else ""))
 
     def check_err(self, when: str):
         import torch

@@ -125,11 +125,14 @@ PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_
 
 /*
  * Workspace (device bytes) that `variant` can use for these sizes
- * (PKV_DECODE_AUTO: enough for any variant it may pick; PKV_DECODE_SPLIT:
- * what it needs; PKV_DECODE_SINGLE and PKV_DECODE_CLUSTER: room for the
- * optional longest-first order of the sequences, 4 bytes per sequence
- * rounded up to 256 -- they also run without any workspace); 0 if a size is
- * invalid.  partition_tokens <= 0 means 512.
+ * (PKV_DECODE_AUTO: enough for any variant it may pick -- the split-K
+ * partials rounded up to 256 bytes, then the order; PKV_DECODE_SPLIT: what
+ * it needs, pkv_decode_workspace_bytes(...); PKV_DECODE_SINGLE and
+ * PKV_DECODE_CLUSTER: room for the optional longest-first order of the
+ * sequences, 4 bytes per sequence rounded up to 256 -- they also run without
+ * any workspace); 0 if a size is invalid.  partition_tokens <= 0 means 512.
+ * Split-K runs its sequences longest first when the workspace holds the
+ * partials and the order behind them (the PKV_DECODE_AUTO size).
  */
 PKV_API size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads,
                                               int num_kv_heads, int head_dim,
@@ -204,10 +207,6 @@ PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *q, const vo
  * PKV_DECODE_STAGES (read at each call) pick the decode CTA shape of the
  * single-pass and split-K kernels: 4 warps x 2 ring stages (the default,
  * measured fastest), 4 x 3 or 2 x 2; other values give the default.
- * PKV_DECODE_L2_AHEAD (0..16, read at each call, also by the shared-prefix
- * calls) makes every decode warp ask L2 for that many of its blocks beyond
- * its ring (bulk L2 prefetches), so that short work units put all their
- * reads to DRAM at once.
  */
 PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,

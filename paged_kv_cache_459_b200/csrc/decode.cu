@@ -112,10 +112,11 @@ __global__ void __launch_bounds__(kOrderThreads)
 template <int D>
 __global__ void __launch_bounds__(D) splitk_merge_kernel(const DecodeParams p) {
     constexpr int kMaxParts = 256;  // per pass; longer rows loop
+    constexpr int kFewParts = 16;   // rows with at most this many partials: all loads at once
     __shared__ float s_w[kMaxParts];
     __shared__ float s_red[D / 32][2];
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
-    pdl_wait_primary();  // the decode grid's partials
+    // the partition count comes from the decode's inputs, read before the wait
     int len = __ldg(p.seq_lens + b);
     len = len < 0 ? 0 : min(len, p.W * kBlockTokens);
     int start = 0;
@@ -125,6 +126,36 @@ __global__ void __launch_bounds__(D) splitk_merge_kernel(const DecodeParams p) {
     const size_t row = static_cast<size_t>(b) * p.Hq + h;
     const float *ml = p.ws_ml + 2 * (row * p.ws_parts + p.ws_part0);
     const float *o = p.ws_o + (row * p.ws_parts + p.ws_part0) * D;
+    pdl_wait_primary();  // the decode grid's partials
+    if (np <= kFewParts) {
+        float mv[kFewParts], lv[kFewParts], ov[kFewParts];
+#pragma unroll
+        for (int q = 0; q < kFewParts; ++q) {
+            mv[q] = -INFINITY;
+            lv[q] = 0.f;
+            ov[q] = 0.f;
+            if (q < np) {
+                const float2 v = *reinterpret_cast<const float2 *>(ml + 2 * q);
+                mv[q] = v.x;
+                lv[q] = v.y;
+                ov[q] = o[static_cast<size_t>(q) * D + e];
+            }
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kFewParts; ++q) M = fmaxf(M, mv[q]);
+        float L = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int q = 0; q < kFewParts; ++q) {
+                const float w = mv[q] == -INFINITY ? 0.f : exp2f(mv[q] - M);
+                L = fmaf(lv[q], w, L);
+                O = fmaf(ov[q], w, O);
+            }
+        }
+        p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
+        return;
+    }
     // M over all partitions
     float mx = -INFINITY;
     for (int q = e; q < np; q += D) mx = fmaxf(mx, ml[2 * q]);
@@ -170,7 +201,7 @@ template <int D, int NW, int S, bool MMA, int MODE>
 cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                        cudaStream_t stream) {
     using G = Geometry<D, NW, S>;
-    constexpr int kSmem = MODE == kModeCluster ? G::kClusterSmemBytes : G::kSmemBytes;
+    constexpr int kSmem = MODE == kModeSingle ? G::kSmemBytes : G::kStagedSmemBytes;
     auto kern = paged_decode_kernel<D, NW, S, MMA, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;

@@ -48,8 +48,9 @@ __device__ __forceinline__ void flag(unsigned int *err, unsigned int bit) {
     if (err != nullptr) atomicOr(err, bit);
 }
 
-// Cluster mode copies a table row of up to this many entries into shared
-// memory (behind the barriers), wider rows are read from global memory.
+// Cluster-mode units and split-K units past a skipped prefix copy a table row
+// of up to this many entries into shared memory (behind the barriers); wider
+// rows are read from global memory.
 constexpr int kStagedTable = 1024;
 
 template <int D, int NW, int S>
@@ -59,7 +60,7 @@ struct Geometry {
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = NW * S * kStageBytes;
     static constexpr int kSmemBytes = kRingBytes + NW * S * 8 + 1024;  // + barriers + alignment
-    static constexpr int kClusterSmemBytes = kSmemBytes + 4 * kStagedTable;  // + the table row
+    static constexpr int kStagedSmemBytes = kSmemBytes + 4 * kStagedTable;  // + a table row
 };
 
 // Block-table entries of one warp's blocks, 32 per register load.

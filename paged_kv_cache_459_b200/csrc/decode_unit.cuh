@@ -40,9 +40,10 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     // cluster mode), they are loaded now, beside the length, for every block
     // the table row holds in this unit's range; entries past the sequence are
     // read but never used.  Otherwise after the length, below.
-    // Cluster mode with a table row of at most kStagedTable entries: the whole
-    // row is read into shared memory beside the length (the part's range needs
-    // the length), and the window reads it there.
+    // Cluster mode, and split-K past a skipped prefix, with a table row of at
+    // most kStagedTable entries: the whole row is read into shared memory
+    // beside the length (the unit's range needs the length, or the prefix
+    // length), and the window reads it there.
     const bool early_table = !CLUSTER && p.start_blocks == nullptr;
     TableWindow tw;
     tw.row = p.block_tables + static_cast<size_t>(b) * p.W;
@@ -58,10 +59,11 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     extern __shared__ uint8_t smem_raw[];
     // Stage buffers must sit on 1024-byte boundaries for the 128-byte swizzle.
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    constexpr int kTabPer = CLUSTER ? kStagedTable / (NW * 32) : 1;
-    const bool staged = CLUSTER && p.W <= kStagedTable;
+    constexpr bool kMayStage = CLUSTER || SPLIT;
+    constexpr int kTabPer = kMayStage ? kStagedTable / (NW * 32) : 1;
+    const bool staged = kMayStage && (CLUSTER || p.start_blocks != nullptr) && p.W <= kStagedTable;
     int32_t tab[kTabPer];
-    if constexpr (CLUSTER) {
+    if constexpr (kMayStage) {
         if (staged) {
 #pragma unroll
             for (int k = 0; k < kTabPer; ++k) {
@@ -102,7 +104,7 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
 
     uint8_t *ring = smem + warp * S * G::kStageBytes;
     const uint32_t bars = smem_u32(smem + G::kRingBytes) + warp * S * 8;
-    if constexpr (CLUSTER) {
+    if constexpr (kMayStage) {
         if (staged) {
             int32_t *tab_s = reinterpret_cast<int32_t *>(smem + G::kRingBytes + NW * S * 8);
 #pragma unroll
@@ -153,24 +155,6 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
             }
         }
     };
-
-    // L2 read-ahead: block i + S + ahead is asked for when block i + S is
-    // loaded, and blocks S .. S + ahead - 1 at the start (lane j takes block
-    // S + j, its table entry fetched from the window by shuffle).
-    const int ahead = p.l2_ahead;
-    auto prefetch_l2 = [&](int32_t phys) {  // one lane
-        if (phys >= 0 && phys < p.num_blocks) {
-            const size_t off = (static_cast<size_t>(phys) * p.Hkv + kvh) * kBlockTokens * D;
-            bulk_prefetch_l2(p.k_cache + off, kBlockTokens * D * 2);
-            bulk_prefetch_l2(p.v_cache + off, kBlockTokens * D * 2);
-        }
-    };
-    if (ahead > 0) {
-        const int i = S + lane;  // < 64: in the window's first two chunks
-        const int32_t a = __shfl_sync(0xffffffffu, tw.cur, i & 31);
-        const int32_t c = __shfl_sync(0xffffffffu, tw.nxt, i & 31);
-        if (lane < ahead && i < n_mine) prefetch_l2(i < 32 ? a : c);
-    }
 
     using Head = typename std::conditional<MMA, GroupHeads<D>, ScalarHead<D>>::type;
     Head st;
@@ -238,10 +222,6 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         if (i + S < n_mine) {
             if (writer && i + S == i_write) store_new();
             issue(i + S);
-            if (ahead > 0 && i + S + ahead < n_mine) {
-                const int32_t ph = tw.get(i + S + ahead);
-                if (lane == 1) prefetch_l2(ph);
-            }
         }
     }
     if (i < n_mine) {

@@ -48,11 +48,7 @@ struct DecodeParams {
     // into the slot of position len - 1 before that unit reads the block.
     const __nv_bfloat16 *k_new, *v_new;
     __nv_bfloat16 *k_cache, *v_cache;  // [num_blocks][Hkv][16][D], for those stores
-    // Blocks each warp asks L2 for beyond its TMA ring (0: none, at most
-    // kMaxL2Ahead): short units then put all their reads to DRAM at once.
-    int l2_ahead;
 };
-constexpr int kMaxL2Ahead = 16;
 
 // Longest-first order of the sequences (by block count) into order[B], for
 // the single-pass decode grid; one CTA, counting sort.

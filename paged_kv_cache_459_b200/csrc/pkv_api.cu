@@ -213,15 +213,15 @@ int cluster_parts_for(int max_blocks_per_seq, int partition_tokens) {
 // few CTAs for a long context: split-K with the merge kernel balances better.
 constexpr int kClusterMaxPartBlocks = 64;
 
-// L2 read-ahead of the decode units (blocks per warp beyond the TMA ring).
-int l2_ahead_for(int fallback) {
-    return std::clamp(env_int("PKV_DECODE_L2_AHEAD", fallback), 0, pkv::kMaxL2Ahead);
-}
-
 struct DecodePlan {
     int variant;  // PKV_DECODE_SINGLE, _SPLIT or _CLUSTER
     int parts;    // cluster parts per sequence (cluster variant)
 };
+
+// Split-K partials, then (256-byte aligned) the longest-first order.
+size_t split_order_bytes(size_t split_bytes, int num_seqs) {
+    return (split_bytes + 255) / 256 * 256 + order_bytes(num_seqs);
+}
 
 // The automatic choice.  Single pass, its units run longest first when the
 // workspace holds the order (measured best when the units fill the GPU);
@@ -229,7 +229,8 @@ struct DecodePlan {
 // units at 3 CTAs per SM (4 waves without the order, whose tail is longer) --
 // each sequence is cut into parts: one cluster of up to 8 CTAs per unit,
 // merged on chip, while a part stays short (kClusterMaxPartBlocks), else
-// 512-token split-K partitions and the merge kernel (long contexts).
+// 512-token split-K partitions and the merge kernel (long contexts), their
+// sequences longest first when the workspace holds the order too.
 DecodePlan plan_auto(int num_seqs, int num_heads, int num_kv_heads, int max_blocks_per_seq,
                      int partition_tokens, size_t workspace_bytes, size_t split_bytes) {
     const int64_t units = decode_units(num_seqs, num_heads, num_kv_heads);
@@ -252,6 +253,7 @@ size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads, 
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads ||
         head_dim <= 0 || max_blocks_per_seq <= 0)
         return 0;
+    if (partition_tokens <= 0) partition_tokens = kDefaultPartitionTokens;
     const size_t split = pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
                                                     max_blocks_per_seq, partition_tokens);
     const size_t order = order_bytes(num_seqs);
@@ -259,7 +261,7 @@ size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads, 
         case PKV_DECODE_SINGLE:   // optional: longest-first scheduling
         case PKV_DECODE_CLUSTER: return order;
         case PKV_DECODE_SPLIT: return split;
-        case PKV_DECODE_AUTO: return std::max(split, order);
+        case PKV_DECODE_AUTO: return std::max(split_order_bytes(split, num_seqs), order);
         default: return 0;
     }
 }
@@ -359,14 +361,19 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
     p.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
     int mode = 0;  // single pass
     bool use_order = false;
+    size_t order_at = 0;  // byte offset of the order in the workspace
     if (plan.variant == PKV_DECODE_SPLIT) {
         mode = 1;
         p.part_blocks = part_blocks;
         p.num_parts = num_parts_for(max_blocks_per_seq, partition_tokens);
-        const size_t rows_ws = static_cast<size_t>(num_seqs) * num_heads * p.num_parts;
+        p.ws_parts = p.num_parts;
+        const size_t rows_ws = static_cast<size_t>(num_seqs) * num_heads * p.ws_parts;
         p.ws_o = static_cast<float *>(workspace);
         p.ws_ml = p.ws_o + rows_ws * head_dim;
-        p.ws_parts = p.num_parts;
+        // the longest sequences' units first (the last units of the grid are
+        // then short), when the order fits behind the partials
+        order_at = (split_bytes + 255) / 256 * 256;
+        use_order = num_seqs >= 2 && have >= split_order_bytes(split_bytes, num_seqs);
     } else if (plan.variant == PKV_DECODE_CLUSTER) {
         mode = 2;
         p.part_blocks = 0;  // per sequence: its blocks / num_parts
@@ -380,14 +387,13 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
         use_order = have >= static_cast<size_t>(num_seqs) * sizeof(int32_t);
     }
     if (use_order) {
-        int32_t *order = static_cast<int32_t *>(workspace);
+        int32_t *order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + order_at);
         cudaError_t e = pkv::launch_order(seq_lens, num_seqs, max_blocks_per_seq, order,
                                           static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_status(e);
         p.order = order;
     }
     pkv::DecodeTuning t{env_int("PKV_DECODE_WARPS", 4), env_int("PKV_DECODE_STAGES", 2)};
-    p.l2_ahead = l2_ahead_for(0);
     cudaError_t e = pkv::launch_decode(tmk, tmv, p, head_dim, mode, t,
                                        static_cast<cudaStream_t>(stream));
     return cuda_status(e);
@@ -531,7 +537,6 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
     dp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
     dp.k_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_cache));
     dp.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
-    dp.l2_ahead = l2_ahead_for(0);
 
     cudaError_t e = pkv::launch_cascade(tmk, tmv, pp, dp, head_dim, num_groups,
                                         static_cast<cudaStream_t>(stream));

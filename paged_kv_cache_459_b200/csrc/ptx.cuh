@@ -62,12 +62,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     }
 }
 
-// Asks L2 for `bytes` (a multiple of 16) of global memory at p (16-byte
-// aligned); nothing is waited for and nothing lands in shared memory.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // Orders this thread's earlier generic-proxy global-memory writes before later
 // async-proxy (TMA) reads of the same bytes.
 __device__ __forceinline__ void fence_proxy_async_global() {
