@@ -454,12 +454,8 @@ class Resident:
         """Whether the decode runs its sequences longest first (an order kernel)."""
         if self.cascade:
             return False
-        order = (4 * self.B + 255) // 256 * 256
         if self.chosen == self.pkv.DECODE_CLUSTER:
-            return self.B >= 16 and self.ws.numel() >= order
-        if self.chosen == self.pkv.DECODE_SPLIT:
-            split = self.pkv.decode_workspace_bytes(self.B, self.hq, self.d, self.W, self.partition)
-            return self.B >= 2 and self.ws.numel() >= (split + 255) // 256 * 256 + order
+            return self.B >= 16 and self.ws.numel() >= (4 * self.B + 255) // 256 * 256
         return self.chosen == self.pkv.DECODE_SINGLE and self.ws.numel() >= 4 * self.B
 
     def launches_per_step(self) -> int:
@@ -475,8 +471,7 @@ class Resident:
             return "shared-prefix cascade (prefix once per group x KV head, split-K suffixes, merge)"
         return {pkv.DECODE_SINGLE: "single pass (one CTA per sequence x KV head, longest first)"
                 if self.ordered() else "single pass (one CTA per sequence x KV head)",
-                pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % self.partition +
-                (", longest first" if self.ordered() else ""),
+                pkv.DECODE_SPLIT: "split-K %d-token partitions + merge" % self.partition,
                 pkv.DECODE_CLUSTER: f"cluster split ({self.parts} equal parts per sequence, one "
                                     f"CTA each, merged in distributed shared memory" +
                                     (", longest first)" if self.ordered() else ")"),

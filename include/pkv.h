@@ -125,14 +125,11 @@ PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_
 
 /*
  * Workspace (device bytes) that `variant` can use for these sizes
- * (PKV_DECODE_AUTO: enough for any variant it may pick -- the split-K
- * partials rounded up to 256 bytes, then the order; PKV_DECODE_SPLIT: what
- * it needs, pkv_decode_workspace_bytes(...); PKV_DECODE_SINGLE and
- * PKV_DECODE_CLUSTER: room for the optional longest-first order of the
- * sequences, 4 bytes per sequence rounded up to 256 -- they also run without
- * any workspace); 0 if a size is invalid.  partition_tokens <= 0 means 512.
- * Split-K runs its sequences longest first when the workspace holds the
- * partials and the order behind them (the PKV_DECODE_AUTO size).
+ * (PKV_DECODE_AUTO: enough for any variant it may pick; PKV_DECODE_SPLIT:
+ * what it needs; PKV_DECODE_SINGLE and PKV_DECODE_CLUSTER: room for the
+ * optional longest-first order of the sequences, 4 bytes per sequence
+ * rounded up to 256 -- they also run without any workspace); 0 if a size is
+ * invalid.  partition_tokens <= 0 means 512.
  */
 PKV_API size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads,
                                               int num_kv_heads, int head_dim,

@@ -201,7 +201,7 @@ template <int D, int NW, int S, bool MMA, int MODE>
 cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                        cudaStream_t stream) {
     using G = Geometry<D, NW, S>;
-    constexpr int kSmem = MODE == kModeSingle ? G::kSmemBytes : G::kStagedSmemBytes;
+    constexpr int kSmem = G::kSmemBytes;
     auto kern = paged_decode_kernel<D, NW, S, MMA, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;

@@ -48,11 +48,6 @@ __device__ __forceinline__ void flag(unsigned int *err, unsigned int bit) {
     if (err != nullptr) atomicOr(err, bit);
 }
 
-// Cluster-mode units and split-K units past a skipped prefix copy a table row
-// of up to this many entries into shared memory (behind the barriers); wider
-// rows are read from global memory.
-constexpr int kStagedTable = 1024;
-
 template <int D, int NW, int S>
 struct Geometry {
     static constexpr int kHalves = D / 64;
@@ -60,20 +55,17 @@ struct Geometry {
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kRingBytes = NW * S * kStageBytes;
     static constexpr int kSmemBytes = kRingBytes + NW * S * 8 + 1024;  // + barriers + alignment
-    static constexpr int kStagedSmemBytes = kSmemBytes + 4 * kStagedTable;  // + a table row
 };
 
 // Block-table entries of one warp's blocks, 32 per register load.
 struct TableWindow {
-    const int32_t *row;  // this sequence's table row (global memory, or a copy in shared memory)
-    bool shared_row;
+    const int32_t *row;  // this sequence's table row
     int first, stride, count;
     int cur_chunk;
     int32_t cur, nxt;
 
     __device__ __forceinline__ int32_t load(int i) const {
-        if (i >= count) return -1;
-        return shared_row ? row[first + stride * i] : __ldg(row + first + stride * i);
+        return i < count ? __ldg(row + first + stride * i) : -1;
     }
     __device__ __forceinline__ void init(int lane) {
         cur_chunk = 0;

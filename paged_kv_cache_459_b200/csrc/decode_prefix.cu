@@ -425,7 +425,7 @@ template <int D, bool MMA>
 cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
                              const DecodeParams &dp, int num_groups, cudaStream_t stream) {
     constexpr int kPre = PrefixTcGeometry<D, kPrefixChunkBlocks>::kSmemBytes;
-    constexpr int kSmem = std::max(kPre, Geometry<D, kPrefixWarps, 2>::kStagedSmemBytes);
+    constexpr int kSmem = std::max(kPre, Geometry<D, kPrefixWarps, 2>::kSmemBytes);
     auto kern = cascade_kernel<D, MMA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;

@@ -40,15 +40,10 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     // cluster mode), they are loaded now, beside the length, for every block
     // the table row holds in this unit's range; entries past the sequence are
     // read but never used.  Otherwise after the length, below.
-    // Cluster mode, and split-K past a skipped prefix, with a table row of at
-    // most kStagedTable entries: the whole row is read into shared memory
-    // beside the length (the unit's range needs the length, or the prefix
-    // length), and the window reads it there.
     const bool early_table = !CLUSTER && p.start_blocks == nullptr;
     TableWindow tw;
     tw.row = p.block_tables + static_cast<size_t>(b) * p.W;
     tw.stride = kStride;
-    tw.shared_row = false;
     if (early_table) {
         const int first_blk = part * p.part_blocks;
         const int last_blk = min(p.W, first_blk + p.part_blocks);  // exclusive, within the row
@@ -59,19 +54,6 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     extern __shared__ uint8_t smem_raw[];
     // Stage buffers must sit on 1024-byte boundaries for the 128-byte swizzle.
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    constexpr bool kMayStage = CLUSTER || SPLIT;
-    constexpr int kTabPer = kMayStage ? kStagedTable / (NW * 32) : 1;
-    const bool staged = kMayStage && (CLUSTER || p.start_blocks != nullptr) && p.W <= kStagedTable;
-    int32_t tab[kTabPer];
-    if constexpr (kMayStage) {
-        if (staged) {
-#pragma unroll
-            for (int k = 0; k < kTabPer; ++k) {
-                const int j = threadIdx.x + k * NW * 32;
-                tab[k] = j < p.W ? __ldg(tw.row + j) : -1;
-            }
-        }
-    }
 
     int len = __ldg(p.seq_lens + b);
     if (len < 0 || len > p.W * kBlockTokens) {
@@ -104,18 +86,6 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
 
     uint8_t *ring = smem + warp * S * G::kStageBytes;
     const uint32_t bars = smem_u32(smem + G::kRingBytes) + warp * S * 8;
-    if constexpr (kMayStage) {
-        if (staged) {
-            int32_t *tab_s = reinterpret_cast<int32_t *>(smem + G::kRingBytes + NW * S * 8);
-#pragma unroll
-            for (int k = 0; k < kTabPer; ++k) {
-                const int j = threadIdx.x + k * NW * 32;
-                if (j < p.W) tab_s[j] = tab[k];
-            }
-            tw.row = tab_s;
-            tw.shared_row = true;
-        }
-    }
 
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(bars + 8 * s, 1);

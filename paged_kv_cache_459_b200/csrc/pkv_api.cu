@@ -218,10 +218,6 @@ struct DecodePlan {
     int parts;    // cluster parts per sequence (cluster variant)
 };
 
-// Split-K partials, then (256-byte aligned) the longest-first order.
-size_t split_order_bytes(size_t split_bytes, int num_seqs) {
-    return (split_bytes + 255) / 256 * 256 + order_bytes(num_seqs);
-}
 
 // The automatic choice.  Single pass, its units run longest first when the
 // workspace holds the order (measured best when the units fill the GPU);
@@ -229,8 +225,7 @@ size_t split_order_bytes(size_t split_bytes, int num_seqs) {
 // units at 3 CTAs per SM (4 waves without the order, whose tail is longer) --
 // each sequence is cut into parts: one cluster of up to 8 CTAs per unit,
 // merged on chip, while a part stays short (kClusterMaxPartBlocks), else
-// 512-token split-K partitions and the merge kernel (long contexts), their
-// sequences longest first when the workspace holds the order too.
+// 512-token split-K partitions and the merge kernel (long contexts).
 DecodePlan plan_auto(int num_seqs, int num_heads, int num_kv_heads, int max_blocks_per_seq,
                      int partition_tokens, size_t workspace_bytes, size_t split_bytes) {
     const int64_t units = decode_units(num_seqs, num_heads, num_kv_heads);
@@ -261,7 +256,7 @@ size_t pkv_decode_workspace_bytes_for(int variant, int num_seqs, int num_heads, 
         case PKV_DECODE_SINGLE:   // optional: longest-first scheduling
         case PKV_DECODE_CLUSTER: return order;
         case PKV_DECODE_SPLIT: return split;
-        case PKV_DECODE_AUTO: return std::max(split_order_bytes(split, num_seqs), order);
+        case PKV_DECODE_AUTO: return std::max(split, order);
         default: return 0;
     }
 }
@@ -361,7 +356,6 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
     p.v_cache = static_cast<__nv_bfloat16 *>(const_cast<void *>(v_cache));
     int mode = 0;  // single pass
     bool use_order = false;
-    size_t order_at = 0;  // byte offset of the order in the workspace
     if (plan.variant == PKV_DECODE_SPLIT) {
         mode = 1;
         p.part_blocks = part_blocks;
@@ -370,10 +364,6 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
         const size_t rows_ws = static_cast<size_t>(num_seqs) * num_heads * p.ws_parts;
         p.ws_o = static_cast<float *>(workspace);
         p.ws_ml = p.ws_o + rows_ws * head_dim;
-        // the longest sequences' units first (the last units of the grid are
-        // then short), when the order fits behind the partials
-        order_at = (split_bytes + 255) / 256 * 256;
-        use_order = num_seqs >= 2 && have >= split_order_bytes(split_bytes, num_seqs);
     } else if (plan.variant == PKV_DECODE_CLUSTER) {
         mode = 2;
         p.part_blocks = 0;  // per sequence: its blocks / num_parts
@@ -387,7 +377,7 @@ static pkv_status decode_impl(void *out, const void *q, const void *k_cache, con
         use_order = have >= static_cast<size_t>(num_seqs) * sizeof(int32_t);
     }
     if (use_order) {
-        int32_t *order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + order_at);
+        int32_t *order = static_cast<int32_t *>(workspace);
         cudaError_t e = pkv::launch_order(seq_lens, num_seqs, max_blocks_per_seq, order,
                                           static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_status(e);

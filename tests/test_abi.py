@@ -137,9 +137,7 @@ def test_variant_choice_and_workspace_sizes():
     B, hq, hkv, d, W = 64, 32, 32, 128, 128
     split = pkv.decode_workspace_bytes_for(pkv.DECODE_SPLIT, B, hq, hkv, d, W)
     assert split == pkv.decode_workspace_bytes(B, hq, d, W)
-    # AUTO: the split partials (rounded up to 256 bytes), then the longest-first order
-    assert pkv.decode_workspace_bytes_for(pkv.DECODE_AUTO, B, hq, hkv, d, W) == \
-        (split + 255) // 256 * 256 + 256
+    assert pkv.decode_workspace_bytes_for(pkv.DECODE_AUTO, B, hq, hkv, d, W) == max(split, 256)
     assert pkv.decode_workspace_bytes_for(pkv.DECODE_SINGLE, B, hq, hkv, d, W) == 256  # the order
     assert pkv.decode_workspace_bytes_for(pkv.DECODE_CLUSTER, B, hq, hkv, d, W) == 256
     assert pkv.decode_workspace_bytes_for(pkv.DECODE_CLUSTER, B, 28, 5, d, W) == 0  # 28 % 5

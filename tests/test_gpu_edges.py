@@ -96,10 +96,9 @@ def test_python_binding_rejects_bad_tensors():
     assert e.value.code == pkv.ERR_UNSUPPORTED
 
 
-def test_ordered_split_edges():
-    """The automatic choice's split-K, sequences longest first: a zero-length
-    row, a bad table entry, lengths past the table or negative -- flagged,
-    skipped, zero rows."""
+def test_auto_split_edges():
+    """Split-K through the automatic choice: a zero-length row, a bad table
+    entry, lengths past the table or negative -- flagged, skipped, zero rows."""
     w = build("llama", 8, batch=9, len_lo=40, len_hi=700, head_dim=64)
     c = w.cfg
     assert pkv.decode_variant_for(c["batch"], c["num_heads"], c["num_kv_heads"], c["head_dim"],
@@ -112,7 +111,7 @@ def test_ordered_split_edges():
     ref = oracle.paged_decode(w.q, kc, vc, w.block_tables, lens, c["scale"])
     out = d.decode(pkv.DECODE_AUTO, 512, lens=torch.from_numpy(lens).cuda())
     assert (out[2] == 0).all()
-    check_close(out, ref, "ordered split, zero-length row")
+    check_close(out, ref, "automatic split, zero-length row")
     assert d.err_word() == 0
     t = w.block_tables.copy()
     t[1, 1] = w.num_blocks + 7
@@ -120,7 +119,7 @@ def test_ordered_split_edges():
     assert np.isfinite(bits_to_f64(out)).all()
     keep = [0] + list(range(2, c["batch"]))
     ref = oracle.paged_decode(w.q, kc, vc, w.block_tables, w.lens, c["scale"])
-    check_close(out[keep], ref[keep], "ordered split, rows beside a bad table entry")
+    check_close(out[keep], ref[keep], "automatic split, rows beside a bad table entry")
     assert d.err_word() & pkv.DEV_ERR_BAD_BLOCK
     d.err.zero_()
     lens = w.lens.copy()
