@@ -319,15 +319,22 @@ __device__ __forceinline__ void prefix_unit_tc(const CUtensorMap &tmk, const CUt
 
 // Merge of one (sequence, query head): prefix chunks [0, ceil(pb / CB)) and
 // the suffix split-K partitions that hold tokens past the prefix (counted
-// from the prefix end), in slot order, by log-sum-exp.  As in the split-K
-// merge: all (m, l) read at once, weights computed once, output loads batched.
+// from the prefix end), in slot order, by log-sum-exp.  One warp per row,
+// kMergeRows rows per CTA, so that the whole merge grid is resident at once
+// (a CTA of D threads per row made two waves of short CTAs at batch 128,
+// 32 heads); lane l holds columns [l V, l V + V).  A lane reads the (m, l)
+// of one slot, the warp reduces them, then every slot's o is loaded 8 slots
+// at a time and accumulated in slot order.
+constexpr int kMergeRows = 4;
+
 template <int D, int CB>
-__global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) {
-    constexpr int kMaxSlots = 256;
-    __shared__ float s_w[kMaxSlots];
-    __shared__ float s_red[D / 32][2];
-    const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
-    pdl_wait_primary();  // the cascade grid's partials
+__global__ void __launch_bounds__(kMergeRows * 32) cascade_merge_kernel(const PrefixParams p) {
+    constexpr int V = D / 32;  // columns per lane
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x * kMergeRows + warp;  // row = b * Hq + h
+    const bool live = r < p.B * p.Hq;
+    const int b = live ? r / p.Hq : 0;
+    // the slot count comes from the step's inputs, read before the wait
     int len = __ldg(p.seq_lens + b);
     len = len < 0 ? 0 : min(len, p.W * kBlockTokens);
     const int nblk = (len + kBlockTokens - 1) / kBlockTokens;
@@ -338,46 +345,66 @@ __global__ void __launch_bounds__(D) cascade_merge_kernel(const PrefixParams p) 
     const int ntot = nchunks + min((nblk - pb + p.part_blocks - 1) / p.part_blocks,
                                    p.ws_parts - p.prefix_parts);
     const auto slot = [&](int q) { return q < nchunks ? q : p.prefix_parts + (q - nchunks); };
-    const size_t row = static_cast<size_t>(b) * p.Hq + h;
+    const size_t row = static_cast<size_t>(live ? r : 0);
     const float *ml = p.ws_ml + 2 * row * p.ws_parts;
-    const float *o = p.ws_o + row * p.ws_parts * D;
-    float mx = -INFINITY;
-    for (int q = e; q < ntot; q += D) mx = fmaxf(mx, ml[2 * slot(q)]);
-#pragma unroll
-    for (int m = 16; m > 0; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-    if ((e & 31) == 0) s_red[e >> 5][0] = mx;
-    __syncthreads();
+    const float *o = p.ws_o + row * p.ws_parts * D + lane * V;
+    pdl_wait_primary();  // the cascade grid's partials
+    if (!live) return;
     float M = -INFINITY;
+    for (int q = lane; q < ntot; q += 32) M = fmaxf(M, ml[2 * slot(q)]);
 #pragma unroll
-    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, s_red[w][0]);
-    float L = 0.f, O = 0.f;
-    for (int base = 0; base < ntot; base += kMaxSlots) {
-        const int n = min(kMaxSlots, ntot - base);
-        __syncthreads();  // s_w and s_red reuse
-        float lsum = 0.f;
-        for (int q = e; q < n; q += D) {
-            const float2 v = *reinterpret_cast<const float2 *>(ml + 2 * slot(base + q));
-            const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-            s_w[q] = w;
-            lsum = fmaf(v.y, w, lsum);
+    for (int m = 16; m > 0; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    float L = 0.f, O[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) O[v] = 0.f;
+    if (M != -INFINITY) {
+        for (int q0 = 0; q0 < ntot; q0 += 32) {
+            // weight of slot q0 + lane, then the slots' o in order
+            float w = 0.f, lq = 0.f;
+            if (q0 + lane < ntot) {
+                const float2 v = *reinterpret_cast<const float2 *>(ml + 2 * slot(q0 + lane));
+                w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+                lq = v.y * w;
+            }
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) lq += __shfl_xor_sync(0xffffffffu, lq, m);
+            L += lq;
+            const int n = min(32, ntot - q0);
+            for (int k0 = 0; k0 < n; k0 += 8) {
+                float x[8][V];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (k0 + k < n) {
+                        const float *src = o + static_cast<size_t>(slot(q0 + k0 + k)) * D;
+                        if constexpr (V == 4) {
+                            const float4 t = *reinterpret_cast<const float4 *>(src);
+                            x[k][0] = t.x;
+                            x[k][1] = t.y;
+                            x[k][2] = t.z;
+                            x[k][3] = t.w;
+                        } else {
+                            const float2 t = *reinterpret_cast<const float2 *>(src);
+                            x[k][0] = t.x;
+                            x[k][1] = t.y;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float wk = __shfl_sync(0xffffffffu, w, (k0 + k) & 31);
+                    if (k0 + k < n) {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) O[v] = fmaf(x[k][v], wk, O[v]);
+                    }
+                }
+            }
         }
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
-        if ((e & 31) == 0) s_red[e >> 5][1] = lsum;
-        __syncthreads();
-#pragma unroll
-        for (int w = 0; w < D / 32; ++w) L += s_red[w][1];
-        int q = 0;
-        for (; q + 8 <= n; q += 8) {
-            float x[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = o[static_cast<size_t>(slot(base + q + i)) * D + e];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) O = fmaf(x[i], s_w[q + i], O);
-        }
-        for (; q < n; ++q) O = fmaf(o[static_cast<size_t>(slot(base + q)) * D + e], s_w[q], O);
     }
-    p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __nv_bfloat16 *dst = p.out + row * D + lane * V;
+#pragma unroll
+    for (int v = 0; v < V; v += 2)
+        *reinterpret_cast<__nv_bfloat162 *>(dst + v) = __floats2bfloat162_rn(O[v] * inv, O[v + 1] * inv);
 }
 
 // One launch for the prefix chunks and the suffix split-K units.  Prefix
@@ -436,9 +463,10 @@ cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, con
     kern<<<static_cast<unsigned>(n_pre + n_suf), kPrefixWarps * 32, kSmem, stream>>>(
         tmk, tmv, pp, dp, static_cast<int>(n_pre));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long rows = static_cast<long long>(pp.B) * pp.Hq;
     return launch_dependent(cascade_merge_kernel<D, kPrefixChunkBlocks>,
-                            dim3(static_cast<unsigned>(pp.Hq), static_cast<unsigned>(pp.B)), dim3(D),
-                            stream, pp);
+                            dim3(static_cast<unsigned>((rows + kMergeRows - 1) / kMergeRows)),
+                            dim3(kMergeRows * 32), stream, pp);
 }
 
 template <int D>
