@@ -45,11 +45,8 @@ template <int D, int NW, int S, bool MMA, int MODE>
 __global__ void __launch_bounds__(NW * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-    int b = blockIdx.z;
-    if (p.order != nullptr) {
-        pdl_wait_primary();  // the order kernel's output
-        b = __ldg(p.order + b);
-    }
+    pdl_wait_primary();  // the preceding grid (the order kernel, or the previous call)
+    const int b = p.order != nullptr ? __ldg(p.order + blockIdx.z) : static_cast<int>(blockIdx.z);
     decode_unit<D, NW, S, MMA, MODE>(tmk, tmv, p, blockIdx.x, blockIdx.y, b);
 }
 
@@ -61,6 +58,7 @@ constexpr int kOrderBuckets = 4096;
 __global__ void __launch_bounds__(kOrderThreads)
     order_kernel(const int32_t *__restrict__ seq_lens, int B, int W, int shift, int32_t *order) {
     pdl_launch_dependents();
+    pdl_wait_primary();  // the previous call's grid
     __shared__ int count[kOrderBuckets];
     __shared__ int warp_tot[kOrderThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -115,6 +113,7 @@ __global__ void __launch_bounds__(D) splitk_merge_kernel(const DecodeParams p) {
     constexpr int kFewParts = 16;   // rows with at most this many partials: all loads at once
     __shared__ float s_w[kMaxParts];
     __shared__ float s_red[D / 32][2];
+    pdl_launch_dependents();  // the next call's first grid may be scheduled
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
     // the partition count comes from the decode's inputs, read before the wait
     int len = __ldg(p.seq_lens + b);
@@ -208,7 +207,7 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
     const dim3 grid(static_cast<unsigned>(p.num_parts),
                     static_cast<unsigned>(MMA ? p.Hkv * p.chunks : p.Hq),
                     static_cast<unsigned>(p.B));
-    if (p.order != nullptr || MODE == kModeCluster) {
+    {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = grid;
         cfg.blockDim = dim3(NW * 32);
@@ -216,10 +215,10 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
         cfg.stream = stream;
         cudaLaunchAttribute attr[2];
         unsigned n = 0;
-        if (p.order != nullptr) {  // waits (griddepcontrol.wait) for the order kernel
-            attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[n++].val.programmaticStreamSerializationAllowed = 1;
-        }
+        // a programmatic dependent of the preceding grid (the order kernel, or
+        // the previous call's last grid): it waits at its start
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n++].val.programmaticStreamSerializationAllowed = 1;
         if (MODE == kModeCluster) {  // the parts of one (sequence, head) form a cluster
             attr[n].id = cudaLaunchAttributeClusterDimension;
             attr[n].val.clusterDim.x = static_cast<unsigned>(p.num_parts);
@@ -229,9 +228,6 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
         cfg.attrs = attr;
         cfg.numAttrs = n;
         e = cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p);
-    } else {
-        kern<<<grid, NW * 32, kSmem, stream>>>(tmk, tmv, p);
-        e = cudaGetLastError();
     }
     if (e != cudaSuccess || MODE != kModeSplit || p.skip_merge) return e;
     return launch_dependent(splitk_merge_kernel<D>, dim3(static_cast<unsigned>(p.Hq), static_cast<unsigned>(p.B)),
@@ -269,8 +265,8 @@ cudaError_t launch_d(const CUtensorMap &tmk, const CUtensorMap &tmv, const Decod
 cudaError_t launch_order(const int32_t *seq_lens, int B, int W, int32_t *order, cudaStream_t stream) {
     int shift = 0;
     while ((W >> shift) >= kOrderBuckets) ++shift;
-    order_kernel<<<1, kOrderThreads, 0, stream>>>(seq_lens, B, W, shift, order);
-    return cudaGetLastError();
+    return launch_dependent(order_kernel, dim3(1), dim3(kOrderThreads), stream, seq_lens, B, W, shift,
+                            order);
 }
 
 cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,

@@ -15,14 +15,17 @@ namespace pkv {
 
 // Launches `kern` so that it may be scheduled before the preceding kernel in
 // the stream finishes (programmatic dependent launch); the kernel must call
-// pdl_wait_primary() before it reads that kernel's output.
+// pdl_wait_primary() before it touches memory that kernel may use.  Every
+// kernel of the decode path is launched this way and waits at its start, so
+// that a call's grid is scheduled while the previous call's last grid drains
+// (that grid lets its dependents launch once all its CTAs have started).
 template <typename... Args>
-cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, cudaStream_t stream,
-                             Args... args) {
+cudaError_t launch_dependent_smem(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, Args... args) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = block;
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -30,6 +33,12 @@ cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, cudaS
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <typename... Args>
+cudaError_t launch_dependent(void (*kern)(Args...), dim3 grid, dim3 block, cudaStream_t stream,
+                             Args... args) {
+    return launch_dependent_smem(kern, grid, block, 0, stream, args...);
 }
 
 namespace dev {

@@ -330,6 +330,7 @@ constexpr int kMergeRows = 4;
 template <int D, int CB>
 __global__ void __launch_bounds__(kMergeRows * 32) cascade_merge_kernel(const PrefixParams p) {
     constexpr int V = D / 32;  // columns per lane
+    pdl_launch_dependents();  // the next call's first grid may be scheduled
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x * kMergeRows + warp;  // row = b * Hq + h
     const bool live = r < p.B * p.Hq;
@@ -418,6 +419,7 @@ __global__ void __launch_bounds__(kPrefixWarps * 32)
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const PrefixParams pp, const DecodeParams dp, int n_pre) {
     pdl_launch_dependents();
+    pdl_wait_primary();  // the previous call's grid
     int id = blockIdx.x;
     const int stride = n_pre > 0 ? static_cast<int>(gridDim.x) / n_pre : 1;
     if (n_pre > 0 && id % stride == 0 && id / stride < n_pre) {
@@ -460,9 +462,9 @@ cudaError_t launch_cascade_d(const CUtensorMap &tmk, const CUtensorMap &tmv, con
     const long long ny = MMA ? dp.Hkv * dp.chunks : dp.Hq;
     const long long n_suf = static_cast<long long>(dp.num_parts) * ny * dp.B;
     if (n_pre + n_suf >= (1ll << 31)) return cudaErrorInvalidValue;
-    kern<<<static_cast<unsigned>(n_pre + n_suf), kPrefixWarps * 32, kSmem, stream>>>(
-        tmk, tmv, pp, dp, static_cast<int>(n_pre));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_dependent_smem(kern, dim3(static_cast<unsigned>(n_pre + n_suf)), dim3(kPrefixWarps * 32),
+                              kSmem, stream, tmk, tmv, pp, dp, static_cast<int>(n_pre));
+    if (e != cudaSuccess) return e;
     const long long rows = static_cast<long long>(pp.B) * pp.Hq;
     return launch_dependent(cascade_merge_kernel<D, kPrefixChunkBlocks>,
                             dim3(static_cast<unsigned>((rows + kMergeRows - 1) / kMergeRows)),

@@ -23,9 +23,9 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     using G = Geometry<D, NW, S>;
     constexpr bool SPLIT = MODE == kModeSplit;
     constexpr bool CLUSTER = MODE == kModeCluster;
-    // The merge kernel may be scheduled as soon as every unit has started; it
-    // waits for this grid to finish before reading the partials.
-    if constexpr (SPLIT) pdl_launch_dependents();
+    // The next grid (the merge kernel, or the next call's) may be scheduled
+    // as soon as every unit has started; it waits for this grid to finish.
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kvh = MMA ? by / p.chunks : by;
     const int chunk = MMA ? by % p.chunks : 0;
