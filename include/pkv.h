@@ -203,7 +203,8 @@ PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *q, const vo
  * For tuning sweeps, the environment variables PKV_DECODE_WARPS and
  * PKV_DECODE_STAGES (read at each call) pick the decode CTA shape of the
  * single-pass and split-K kernels: 4 warps x 2 ring stages (the default,
- * measured fastest), 4 x 3 or 2 x 2; other values give the default.
+ * measured fastest), 4 x 3 or 2 x 2; other values give the default.  The
+ * cluster variant always runs 4 x 2.
  */
 PKV_API pkv_status pkv_paged_attention_decode_ex(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,

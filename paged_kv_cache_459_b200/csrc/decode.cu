@@ -200,7 +200,7 @@ template <int D, int NW, int S, bool MMA, int MODE>
 cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                        cudaStream_t stream) {
     using G = Geometry<D, NW, S>;
-    constexpr int kSmem = G::kSmemBytes;
+    constexpr int kSmem = G::kSmemBytes + (MODE == kModeCluster ? cluster_land_bytes<D, MMA>() : 0);
     auto kern = paged_decode_kernel<D, NW, S, MMA, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
@@ -249,7 +249,8 @@ template <int D, bool MMA>
 cudaError_t launch_m(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeParams &p,
                      int mode, DecodeTuning t, cudaStream_t stream) {
     if (mode == kModeSplit) return launch_tuned<D, MMA, kModeSplit>(tmk, tmv, p, t, stream);
-    if (mode == kModeCluster) return launch_tuned<D, MMA, kModeCluster>(tmk, tmv, p, t, stream);
+    // cluster mode: 4 x 2 only (part 0's ring holds the other parts' rows of a head group)
+    if (mode == kModeCluster) return launch_one<D, 4, 2, MMA, kModeCluster>(tmk, tmv, p, stream);
     return launch_tuned<D, MMA, kModeSingle>(tmk, tmv, p, t, stream);
 }
 

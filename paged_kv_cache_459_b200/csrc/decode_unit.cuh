@@ -14,6 +14,26 @@ constexpr int kModeSplit = 1;    // one token partition: (m, l, o) partial to th
 constexpr int kModeCluster = 2;  // one of p.num_parts equal parts of the sequence, the parts
                                  // a thread-block cluster, merged through its shared memory
 
+// Cluster mode: the shared memory of part 0 past its ring and barriers takes
+// an mbarrier (16 bytes with padding) and, with one query head per CTA, the
+// combined rows of parts 1 .. P - 1, each [m of <= H heads][l of <= H
+// heads][o: H x D] floats, so that they can arrive while part 0 still reads
+// its own blocks.  With a group of heads (8 x the rows) they go into part 0's
+// ring instead, behind its own rows, once part 0 has passed a cluster barrier
+// after its blocks (three CTAs per SM either way).
+template <int D, bool MMA>
+constexpr int cluster_slot_floats() {
+    return (MMA ? 8 : 1) * (D + 2);
+}
+template <bool MMA>
+constexpr bool cluster_land_in_ring() {
+    return MMA;
+}
+template <int D, bool MMA>
+constexpr int cluster_land_bytes() {
+    return 16 + (cluster_land_in_ring<MMA>() ? 0 : (kMaxClusterParts - 1) * cluster_slot_floats<D, MMA>() * 4);
+}
+
 // One work unit (partition `part` of sequence b, KV head / head chunk `by`)
 // of the per-unit decode kernel, run by a CTA of NW warps.  The warps take
 // the unit's blocks round-robin and are combined in shared memory at the end.
@@ -95,7 +115,25 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
+    // Cluster mode: parts 1 .. P - 1 store their combined rows into part 0's
+    // shared memory and arrive on its mbarrier `land`; part 0 merges.  A
+    // cluster barrier whose wait comes before the first store makes the
+    // mbarrier's initialisation visible to the other parts; it starts here
+    // when the rows land outside part 0's ring, else after each part's blocks.
+    const int P = CLUSTER ? p.num_parts : 1;
+    const uint32_t land = smem_u32(smem + G::kRingBytes + NW * S * 8);
+    uint32_t rank = 0;
+    if constexpr (CLUSTER) {
+        rank = cluster_ctarank();
+        if (P > 1 && rank == 0 && threadIdx.x == 0) {
+            mbar_init(land, P - 1);
+            fence_mbar_init();
+        }
+    }
     __syncthreads();
+    if constexpr (CLUSTER) {
+        if (P > 1 && !cluster_land_in_ring<MMA>()) cluster_arrive_release();
+    }
 
     const int n_mine = blk_end - blk_begin > lead ? (blk_end - blk_begin - lead + kStride - 1) / kStride : 0;
     if (!early_table) {
@@ -202,18 +240,34 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     }
 
     constexpr int kRed = MMA ? 16 + 8 * D : D + 2;
+    constexpr int kHeadsMax = MMA ? 8 : 1;
+    constexpr int kSlot = cluster_slot_floats<D, MMA>();
     // ---- combine the warps of this CTA (all rings are drained) ----
     __syncthreads();
     float *red = reinterpret_cast<float *>(smem);
-    // cluster mode: this CTA's combined rows for the other CTAs of the
-    // cluster -- m of head n at [n], l at [8 + n], o at [16 + n * D + e]
+    // cluster mode, part 0: its own combined rows -- m of head n at [n], l at
+    // [8 + n], o at [16 + n * D + e]
     float *xch = red + NW * kRed;
     st.finish(red + warp * kRed, lane);
     __syncthreads();
+    uint32_t my_slot = 0;  // cluster mode, parts 1 .. P - 1: this part's rows in part 0
+    // where the other parts' rows land in part 0: behind xch in the ring, or
+    // behind the mbarrier
+    const uint32_t land_rows = cluster_land_in_ring<MMA>()
+                                   ? (smem_u32(xch + 16 + 8 * D) + 15u) & ~15u
+                                   : land + 16;
+    static_assert(!CLUSTER || !cluster_land_in_ring<MMA>() ||
+                      (NW * kRed + 16 + 8 * D + 4) * 4 + (kMaxClusterParts - 1) * kSlot * 4 <= G::kRingBytes,
+                  "the other parts' rows must fit in part 0's ring");
     if constexpr (CLUSTER) {
         if (blk_begin >= blk_end && p.k_new != nullptr && len > 0 && start >= nblk && part == 0 &&
             threadIdx.x == 0 && (!MMA || by % p.chunks == 0))
             flag(p.err, PKV_DEV_ERR_BAD_LEN);  // the fused write's token lies inside the skipped prefix
+        if (P > 1) {
+            if (cluster_land_in_ring<MMA>()) cluster_arrive_release();  // this part's blocks are read
+            cluster_wait_acquire();  // part 0's mbarrier is initialised (and its ring free)
+            if (rank != 0) my_slot = dsmem_addr(land_rows + (rank - 1) * kSlot * 4, 0);
+        }
     }
     for (int idx = threadIdx.x; idx < heads * D; idx += NW * 32) {
         const int n = idx / D, e = idx % D;
@@ -242,35 +296,56 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
                 p.ws_ml[2 * pr + 1] = L;
             }
         } else if constexpr (CLUSTER) {
-            xch[16 + n * D + e] = O;
-            if (e == 0) {
-                xch[n] = M;
-                xch[8 + n] = L;
+            if (rank == 0) {
+                xch[16 + n * D + e] = O;
+                if (e == 0) {
+                    xch[n] = M;
+                    xch[8 + n] = L;
+                }
+            } else {
+                st_dsmem_f32(my_slot + 4 * (2 * kHeadsMax + n * D + e), O);
+                if (e == 0) {
+                    st_dsmem_f32(my_slot + 4 * n, M);
+                    st_dsmem_f32(my_slot + 4 * (kHeadsMax + n), L);
+                }
             }
         } else {
             p.out[row * D + e] = __float2bfloat16(L > 0.f ? O / L : 0.f);
         }
     }
     if constexpr (CLUSTER) {
-        // Log-sum-exp merge of the cluster's parts, in part order (the same
-        // arithmetic as the split-K merge kernel): each CTA merges an equal
-        // slice of the (head, column) elements, reading every part's m, l and
-        // o from the owning CTA's shared memory.
-        cluster_sync();
-        const int P = p.num_parts;
-        const int total = heads * D;
-        const int per = (total + P - 1) / P;
-        const int lo = static_cast<int>(cluster_ctarank()) * per, hi = min(total, lo + per);
-        for (int idx = lo + threadIdx.x; idx < hi; idx += NW * 32) {
+        if (rank != 0) {
+            // every thread's stores are issued; one release at cluster scope
+            // covers them, and the part may leave (nothing reads its memory)
+            fence_acq_rel_cluster();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                fence_acq_rel_cluster();
+                mbar_arrive_remote(dsmem_addr(land, 0));
+            }
+            return;
+        }
+        // Part 0: log-sum-exp merge of the cluster's parts, in part order
+        // (the same arithmetic as the split-K merge kernel), its own rows from
+        // xch and the others' from its landing area.  The wait outlasts every
+        // part's own bounded waits, so no part stores here after part 0 left.
+        if (P > 1 && !mbar_wait_cluster(land, 0, kWaitLimitNs * static_cast<uint64_t>(pblk + 4)) &&
+            threadIdx.x == 0)
+            flag(p.err, PKV_DEV_ERR_TIMEOUT);
+        __syncthreads();  // xch complete
+        const float *lz = reinterpret_cast<const float *>(smem + (land_rows - smem_u32(smem)));
+        for (int idx = threadIdx.x; idx < heads * D; idx += NW * 32) {
             const int n = idx / D, e = idx % D;
-            // every part's m, l and o requested at once (one round trip through
-            // the cluster), then combined in part order
             float mc[kMaxClusterParts], lc[kMaxClusterParts], oc[kMaxClusterParts];
+            mc[0] = xch[n];
+            lc[0] = xch[8 + n];
+            oc[0] = xch[16 + n * D + e];
 #pragma unroll
-            for (int c = 0; c < kMaxClusterParts; ++c) {
-                mc[c] = c < P ? ld_dsmem_f32(xch + n, c) : -INFINITY;
-                lc[c] = c < P ? ld_dsmem_f32(xch + 8 + n, c) : 0.f;
-                oc[c] = c < P ? ld_dsmem_f32(xch + 16 + n * D + e, c) : 0.f;
+            for (int c = 1; c < kMaxClusterParts; ++c) {
+                const float *sl = lz + (c - 1) * kSlot;
+                mc[c] = c < P ? sl[n] : -INFINITY;
+                lc[c] = c < P ? sl[kHeadsMax + n] : 0.f;
+                oc[c] = c < P ? sl[2 * kHeadsMax + n * D + e] : 0.f;
             }
             float M = -INFINITY;
 #pragma unroll
@@ -288,7 +363,6 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
             p.out[(static_cast<size_t>(b) * p.Hq + h0 + n) * D + e] =
                 __float2bfloat16(L > 0.f ? O / L : 0.f);
         }
-        cluster_sync();  // no CTA leaves while the others still read its shared memory
     }
 }
 

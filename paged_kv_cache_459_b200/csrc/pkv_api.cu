@@ -190,11 +190,10 @@ int64_t decode_units(int num_seqs, int num_heads, int num_kv_heads) {
 }
 
 // Cluster variant, automatic: as many parts per sequence as keep the whole
-// grid resident at once (three CTAs per SM) -- a CTA that waits at the
-// cluster barrier for a peer still queued would hold its slot idle; measured:
-// 8 parts at batch 32 ran 2x slower than the single pass -- at most
-// kMaxClusterParts, and at least one block per consumer warp (4) in a part of
-// the longest sequence.
+// grid resident at once (three CTAs per SM) -- a part that waits for a peer
+// still queued would hold its slot idle; measured: 8 parts at batch 32 ran 2x
+// slower than the single pass -- at most kMaxClusterParts, and at least one
+// block per consumer warp (4) in a part of the longest sequence.
 int cluster_parts_auto(int64_t units, int max_blocks_per_seq) {
     const int64_t slots = 3 * static_cast<int64_t>(sm_count());
     int64_t parts = slots / std::max<int64_t>(units, 1);

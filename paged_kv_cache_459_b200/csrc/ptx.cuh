@@ -87,28 +87,70 @@ __device__ __forceinline__ void pdl_wait_primary() {
 }
 
 // ------------------------------------------------------- thread-block clusters
-// Barrier over every thread of every CTA of the cluster (all threads must
-// reach it, like __syncthreads): this CTA's earlier shared-memory writes are
-// visible to the cluster's CTAs after it.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
     return r;
 }
 
-// The float at this CTA's shared-memory address `p`, read from the same
-// address in the shared memory of cluster CTA `rank` (distributed shared memory).
-__device__ __forceinline__ float ld_dsmem_f32(const float *p, uint32_t rank) {
+// A barrier over every thread of every CTA of the cluster, in two halves so
+// that the wait can come later (all threads must execute both, like
+// __syncthreads): this CTA's writes before the arrive are visible to the
+// cluster's CTAs after their wait.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The shared::cluster address of this CTA's shared-memory address `a` in the
+// shared memory of cluster CTA `rank` (distributed shared memory).
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t a, uint32_t rank) {
     uint32_t remote;
-    float v;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-    return v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(a), "r"(rank));
+    return remote;
+}
+
+__device__ __forceinline__ void st_dsmem_f32(uint32_t remote, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
+// Orders this thread's earlier memory accesses (and, after a CTA barrier,
+// its CTA's) before its later ones at cluster scope.
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
+// Arrives (release, cluster scope) on an mbarrier in another CTA's shared
+// memory, `remote` from dsmem_addr.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote)
+                 : "memory");
+}
+
+// As mbar_wait, acquiring at cluster scope (arrivals from other CTAs).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // ---------------------------------------------------------------- TMA

@@ -42,24 +42,26 @@ def test_sources_found():
 
 
 def test_mbarrier_polls_go_through_the_bounded_wait():
-    """Only ptx.cuh polls an mbarrier, and its one loop gives up after a
-    globaltimer limit; every other file waits through mbar_wait(bar, parity,
-    limit)."""
+    """Only ptx.cuh polls an mbarrier (one poll at CTA scope, one acquiring at
+    cluster scope), and each of its two loops gives up after a globaltimer
+    limit; every other file waits through mbar_wait(bar, parity, limit) or
+    mbar_wait_cluster(bar, parity, limit)."""
     for path in SOURCES:
         code = _code(path)
         if path.name == "ptx.cuh":
-            assert code.count("mbarrier.try_wait") == 1
+            assert code.count("mbarrier.try_wait") == 2
             loops = re.findall(r"while\s*\(\s*true\s*\)|for\s*\(\s*;\s*;\s*\)", code)
-            assert len(loops) == 1
-            body = code[code.index("bool mbar_wait("):]
-            body = body[:body.index("\n}\n")]
-            assert "globaltimer_ns() - t0 > limit_ns" in body and "return false" in body
+            assert len(loops) == 2
+            for name in ("bool mbar_wait(", "bool mbar_wait_cluster("):
+                body = code[code.index(name):]
+                body = body[:body.index("\n}\n")]
+                assert "globaltimer_ns() - t0 > limit_ns" in body and "return false" in body, name
             continue
         assert "mbarrier.try_wait" not in code and "mbarrier.wait" not in code, path.name
-        assert "mbar_try_wait(" not in code, path.name
-        for m in re.finditer(r"\bmbar_wait\(", code):
+        assert "mbar_try_wait(" not in code and "mbar_try_wait_cluster(" not in code, path.name
+        for m in re.finditer(r"\bmbar_wait(_cluster)?\(", code):
             args = _call_args(code, m.end())
-            assert len(args) == 3 and args[2], f"{path.name}: mbar_wait without a limit: {args}"
+            assert len(args) == 3 and args[2], f"{path.name}: mbarrier wait without a limit: {args}"
 
 
 def test_no_unbounded_spin_loops_in_kernels():
