@@ -38,7 +38,8 @@ constexpr int kKeys = 128;                 // keys per tile (MMA N of S, K of P.
 constexpr int kWarpsPerTile = 4;           // one softmax warpgroup per Q tile
 constexpr int kSoftmaxWarps = kTiles * kWarpsPerTile;
 constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr int kQWarp = kSoftmaxWarps + 2;  // + x: the Q rows of tile x
+constexpr int kThreads = (kSoftmaxWarps + 2 + kTiles) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // ------------------------------------------------ packed f32x2 arithmetic
@@ -81,7 +82,7 @@ struct TcGeometry {
     static constexpr int kTmemSlot = kBars + 32 * 8;
     static constexpr int kSmemBytes = kTmemSlot + 16 + 1024;
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-    static_assert(2 * (kKStages + kVStages) + 10 <= 32, "barrier slots");
+    static_assert(2 * (kKStages + kVStages) + 12 <= 32, "barrier slots");
     // TMEM columns: S of tile x at kKeys x (P, bf16, over its first half),
     // O of tile x at kO + D x.
     static constexpr int kO = kTiles * kKeys;
@@ -144,8 +145,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 }
 
 // Persistent: one CTA per SM walks its items; TMEM is allocated once, every
-// barrier's phase runs on across items, and the next item's Q rows are
-// fetched (cp.async) as soon as the current item's last S product is done.
+// barrier's phase runs on across items, and a dedicated warp fetches the next
+// item's Q rows (cp.async) as soon as the current item's last S product of
+// that Q tile is done.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk,
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t bar0 = smem_u32(smem + Geo::kBars);
     // barriers: k_full[KS] k_empty[KS] v_full[VS] v_empty[VS], then per Q tile
-    // s_full p_full o_done q_full o_free
+    // s_full p_full o_done q_full o_free q_free
     const auto k_full = [&](int s) { return bar0 + 8 * s; };
     const auto k_empty = [&](int s) { return bar0 + 8 * (KS + s); };
     const auto v_full = [&](int s) { return bar0 + 8 * (2 * KS + s); };
@@ -170,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const auto o_done = [&](int x) { return tile_bars + 8 * (4 + x); };
     const auto q_full = [&](int x) { return tile_bars + 8 * (6 + x); };
     const auto o_free = [&](int x) { return tile_bars + 8 * (8 + x); };
+    const auto q_free = [&](int x) { return tile_bars + 8 * (10 + x); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Geo::kTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Geo::kTmemSlot + 4);
 
@@ -186,8 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(s_full(x), 1);
             mbar_init(p_full(x), kWarpsPerTile);
             mbar_init(o_done(x), 1);
-            mbar_init(q_full(x), kWarpsPerTile);
+            mbar_init(q_full(x), 1);
             mbar_init(o_free(x), kWarpsPerTile);
+            mbar_init(q_free(x), 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -333,7 +337,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (nk_t[x] == 0) continue;
                 wait(q_full(x), static_cast<uint32_t>(n_it & 1));
                 tc::fence_after();
-                if (ok && lane == 0) issue_s(x, gk % KS);
+                if (ok && lane == 0) {
+                    issue_s(x, gk % KS);
+                    if (nk_t[x] == 1) tc::commit(q_free(x));  // the item's last S_x has read Q_x
+                }
                 __syncwarp();
             }
             if (ok && lane == 0) tc::commit(k_empty(gk % KS));
@@ -380,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (ok && lane == 0) {
                             issue_s(x, gk % KS);
                             if (x == last_k) tc::commit(k_empty(gk % KS));
+                            if (j + 2 == nk_t[x]) tc::commit(q_free(x));  // the item's last S_x
                         }
                     }
                     __syncwarp();
@@ -391,11 +399,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (nk_t[x] > 0) continue;
                 wait(q_full(x), static_cast<uint32_t>(n_it & 1));
                 if (n_it > 0) wait(o_free(x), static_cast<uint32_t>((n_it - 1) & 1));
-                if (ok && lane == 0) tc::commit(o_done(x));
+                if (ok && lane == 0) {
+                    tc::commit(o_done(x));
+                    tc::commit(q_free(x));
+                }
                 __syncwarp();
             }
             k = kn;
         }
+    } else if (warp >= kQWarp) {
+        // ---------------- Q rows of each item into shared memory (K-major,
+        // 128-byte swizzle; rows past the item's rows zero-filled), one warp
+        // per Q tile: tile x's rows of item n once the last S_x product of
+        // item n - 1 has read Q_x (q_free), then q_full.  Off the softmax
+        // warps, whose last step of an item this 32 KB of cp.async per tile
+        // used to lengthen.
+        const int x = warp - kQWarp;
+        bool ok = true;
+        int n_it = 0;
+        TcItem it, nx;
+        for (int k = tc_next_item(p, 0, it); k >= 0 && ok; it = nx, ++n_it) {
+            const int kn = tc_next_item(p, k + 1, nx);
+            {
+                if (n_it > 0 && (!mbar_wait(q_free(x), static_cast<uint32_t>((n_it - 1) & 1), kWaitLimitNs) ||
+                                 *abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *qtile = smem + Geo::kQ + x * Geo::kQBytes;
+#pragma unroll 1
+                for (int rr = lane; rr < kRows; rr += 32) {
+                    const int r = it.r_begin + x * kRows + rr;
+                    const __nv_bfloat16 *src = p.q;
+                    uint32_t bytes = 0;
+                    if (r < it.rows) {
+                        src = p.q + (static_cast<size_t>(it.q0 + r / G) * p.Hq + it.kvh * G + r % G) * D;
+                        bytes = 16;
+                    }
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c)
+                        cp_async16(smem_u32(qtile + (c >> 3) * (kRows * 128) + rr * 128 + (((c & 7) ^ (rr & 7)) << 4)),
+                                   src + (bytes ? c * 8 : 0), bytes);
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                asm volatile("cp.async.wait_all;" ::: "memory");
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_full(x));
+            }
+            k = kn;
+        }
+        if (!ok && lane == 0) {
+            flag(p.err, PKV_DEV_ERR_TIMEOUT);
+            *abort_flag = 1;
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
         // ---------------- softmax warps: thread t of tile x = TMEM lane t = row r_begin + 128 x + t
         const int tile = warp / kWarpsPerTile;
@@ -403,38 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = static_cast<uint32_t>((warp % kWarpsPerTile) * 32) << 16;
         const uint32_t t_s = tmem + lane_addr + kKeys * tile;
         const uint32_t t_o = tmem + lane_addr + Geo::kO + D * tile;
-        uint8_t *qrow = smem + Geo::kQ + tile * Geo::kQBytes + t * 128;
-        // this thread's Q row of an item into shared memory (K-major, 128-byte
-        // swizzle; rows past the item's rows are zero-filled)
-        const auto fetch_q = [&](const TcItem &nx) {
-            const int r = nx.r_begin + tile * kRows + t;
-            const __nv_bfloat16 *src = p.q;
-            uint32_t bytes = 0;
-            if (r < nx.rows) {
-                src = p.q + (static_cast<size_t>(nx.q0 + r / G) * p.Hq + nx.kvh * G + r % G) * D;
-                bytes = 16;
-            }
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c)
-                cp_async16(smem_u32(qrow + (c >> 3) * (kRows * 128) + (((c & 7) ^ (t & 7)) << 4)),
-                           src + (bytes ? c * 8 : 0), bytes);
-            asm volatile("cp.async.commit_group;" ::: "memory");
-        };
-        const auto publish_q = [&]() {  // the fetched rows, to the tensor core
-            asm volatile("cp.async.wait_all;" ::: "memory");
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(q_full(tile));
-        };
         bool ok = true;
         int ns = 0;    // S products seen (s_full / p_full phases)
         int n_it = 0;  // items done (o_done phases)
         TcItem it, nx;  // the current and the next item
         int k = tc_next_item(p, 0, it);
-        if (k >= 0) {
-            fetch_q(it);
-            publish_q();
-        }
         while (k >= 0 && ok) {
             const int kn = tc_next_item(p, k + 1, nx);
             const int r = it.r_begin + tile * kRows + t;
@@ -443,7 +474,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __nv_bfloat16 *out_row =
                 p.out + (static_cast<size_t>(it.q0 + r / G) * p.Hq + it.kvh * G + r % G) * D;
             float m_run = -INFINITY, l_run = 0.f;
-            if (my_nk == 0 && kn >= 0) fetch_q(nx);
             for (int j = 0; j < my_nk; ++j, ++ns) {
                 // S_x(j) done; it was issued after PV_x(j - 1), so O_x is free too
                 if (!mbar_wait(s_full(tile), static_cast<uint32_t>(ns & 1), kWaitLimitNs) || *abort_flag) {
@@ -451,25 +481,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc::fence_after();
-                // the last S product of this item has read Q_x: fetch the next item's rows
-                if (j + 1 == my_nk && kn >= 0) fetch_q(nx);
                 // Two passes over S in TMEM, 64 columns at a time, so that a row
-                // never sits in registers whole (ten warps leave 168 registers
+                // never sits in registers whole (twelve warps leave 170 registers
                 // a thread): the row max first, then exp2 and P.
                 const int k0 = j * kKeys;
                 const bool masked = __any_sync(0xffffffffu, k0 + kKeys - 1 > row_pos);
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1  // one half's 64 registers live at a time
                 for (int h = 0; h < kKeys / 64; ++h) {
+                    // causal mask by position (only tiles that reach past some row
+                    // need it), decided per 64-key half and warp: a half past
+                    // every row of the warp is skipped, one before every row
+                    // needs no mask
+                    const int lim = row_pos - (k0 + 64 * h);  // keys c > lim are masked
+                    if (masked && __all_sync(0xffffffffu, lim < 0)) continue;
                     uint32_t sr[64];
                     tc::ld32(t_s + 64 * h, sr);
                     tc::ld32(t_s + 64 * h + 32, sr + 32);
                     tc::wait_ld();
-                    // causal mask by position (only tiles that reach past some row need it)
-                    if (masked) {
+                    if (masked && !__all_sync(0xffffffffu, lim >= 63)) {
 #pragma unroll
                         for (int c = 0; c < 64; ++c)
-                            if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;  // -inf
+                            if (c > lim) sr[c] = 0xFF800000u;  // -inf
                     }
 #pragma unroll
                     for (int c = 0; c < 64; c += 2)
@@ -489,15 +522,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
 #pragma unroll 1  // one half's 64 registers live at a time
                 for (int h = 0; h < kKeys / 64; ++h) {
+                    const int lim = row_pos - (k0 + 64 * h);
+                    uint32_t pk[32];
+                    if (masked && __all_sync(0xffffffffu, lim < 0)) {  // P = 0 over the whole half
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+                        tc::st32(t_s + 32 * h, pk);
+                        continue;
+                    }
                     uint32_t sr[64];
                     tc::ld32(t_s + 64 * h, sr);
                     tc::ld32(t_s + 64 * h + 32, sr + 32);
                     tc::wait_ld();
-                    uint32_t pk[32];
-                    if (masked) {  // diagonal tiles: -inf scores (2^-inf = 0)
+                    if (masked && !__all_sync(0xffffffffu, lim >= 63)) {  // -inf scores (2^-inf = 0)
 #pragma unroll
                         for (int c = 0; c < 64; ++c)
-                            if (k0 + 64 * h + c > row_pos) sr[c] = 0xFF800000u;
+                            if (c > lim) sr[c] = 0xFF800000u;
                     }
 #pragma unroll
                     for (int c = 0; c < 64; c += 2) {  // scale and shift two at a time, 2^x on the SFU
@@ -536,9 +576,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full(tile));
-                // This tile's S products of the item are all done, so the tensor
-                // core has taken this item's Q phase: the next one may be posted.
-                if (j + 1 == my_nk && kn >= 0) publish_q();
             }
             if (!ok) break;
             // O_x of this item complete (a tile without rows gets a bare commit)
@@ -547,7 +584,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc::fence_after();
-            if (my_nk == 0 && kn >= 0) publish_q();  // after o_done: at most one phase ahead
             ++n_it;
             if (my_nk == 0) {
                 __syncwarp();
@@ -590,7 +626,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             flag(p.err, PKV_DEV_ERR_TIMEOUT);
             *abort_flag = 1;
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     // everyone (the producer's copies included) is done with TMEM and shared memory
     tc::fence_before();
