@@ -511,14 +511,15 @@ class L2Flush:
 
 
 def device_steps(step, K: int, dev, flush_buf=None):
-    """Device time of K calls of step(): per-step CUDA events (ms each) and the
-    whole loop (ms).  With flush_buf (an L2Flush), L2 is emptied before every
-    step, outside its events."""
+    """Device time of K calls of step(): per-step times (ms each) and the
+    whole loop (ms).  Without flush_buf the K steps run back to back between
+    two events and each step is the loop's mean; with flush_buf (an L2Flush),
+    L2 is emptied before every step, outside that step's own two events."""
     import torch
 
     stream = torch.cuda.current_stream(dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+          for _ in range(K)] if flush_buf is not None else []
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
     torch.cuda._sleep(SPIN_CYCLES_LEAD)
@@ -528,12 +529,16 @@ def device_steps(step, K: int, dev, flush_buf=None):
             if i and i % FLUSH_CHUNK == 0:
                 torch.cuda._sleep(SPIN_CYCLES_CHUNK)
             flush_buf()  # L2 holds none of this step's inputs and no dirty lines
-        ev[i][0].record(stream)
+            ev[i][0].record(stream)
         step()
-        ev[i][1].record(stream)
+        if flush_buf is not None:
+            ev[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
-    return [a.elapsed_time(b) for a, b in ev], t0.elapsed_time(t1)
+    loop = t0.elapsed_time(t1)
+    if flush_buf is None:
+        return [loop / K] * K, loop
+    return [a.elapsed_time(b) for a, b in ev], loop
 
 
 def rotating_steps(r: Resident, K: int, dev, fn=None) -> float:
@@ -894,8 +899,8 @@ def run_gpu(args):
                    f"as a model's layers each read their own cache), K steps back to back; the "
                    f"'flushed' key times each step alone after an L2 flush") if m["flush"] else
                   f"inputs larger than L2 (KV {ab['kv'] / 1e9:.2f} GB per step vs 126 MB L2), no flush",
-            "timing": "CUDA events on the launching stream; a spin kernel lets the host enqueue "
-                      "ahead of the device, outside the steps' events",
+            "timing": "K steps back to back between two CUDA events on the launching stream; a "
+                      "spin kernel before the first lets the host enqueue ahead of the device",
             "parallelism": f"{world} independent replicas (batch per GPU fixed)",
             "seed": args.seed,
         },

@@ -288,9 +288,10 @@ PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, c
  * prefix_blocks[b] = 0.  The group's shared block ids are read from its first
  * member's table row.  pkv_alloc_prefix_groups builds all three arrays from
  * the allocator's state.  All five arrays are device int32.
- * Work: one launch computes each group's prefix attention in chunks of 8
- * blocks on the 5th-generation tensor cores (tcgen05.mma, queries of all
- * members x heads as the MMA rows, products in tensor memory) beside split-K
+ * Work: one launch computes each group's prefix attention in spans of 32
+ * blocks (one CTA and one partial per span, its keys in steps of 64) on the
+ * 5th-generation tensor cores (tcgen05.mma, queries of all members x heads
+ * as the MMA rows, products in tensor memory) beside split-K
  * units (partition_tokens, <= 0: 512) that cover each sequence past its
  * prefix; a merge kernel combines the partials.  Workspace:
  * pkv_decode_prefix_workspace_bytes(...), else PKV_ERR_WORKSPACE.

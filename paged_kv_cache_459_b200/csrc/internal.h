@@ -72,7 +72,7 @@ cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const 
 
 // Shared-prefix (cascade) decode: prefix blocks read once per (group, KV
 // head) by a dense tensor-core kernel; suffixes by split-K; LSE merge.
-constexpr int kPrefixChunkBlocks = 8;  // prefix blocks per CTA
+constexpr int kPrefixSpanBlocks = 32;  // prefix blocks per CTA (a span: one partial per row)
 
 struct PrefixParams {
     __nv_bfloat16 *out;
@@ -88,7 +88,7 @@ struct PrefixParams {
     long long num_blocks;
     int W, B, Hq, Hkv, group;
     int ws_parts;      // prefix_parts + suffix partitions
-    int prefix_parts;  // ceil(W / kPrefixChunkBlocks): slots 0.. hold prefix chunks
+    int prefix_parts;  // ceil(W / kPrefixSpanBlocks): slots 0.. hold prefix spans
     int part_blocks;   // suffix split-K partition (blocks)
     float scale_log2;
 };

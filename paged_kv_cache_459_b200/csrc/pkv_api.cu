@@ -424,7 +424,7 @@ size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_heads, int head_d
     if (partition_tokens % PKV_BLOCK_TOKENS) return 0;
     const size_t parts =
         static_cast<size_t>(num_parts_for(max_blocks_per_seq, partition_tokens)) +
-        (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+        (max_blocks_per_seq + pkv::kPrefixSpanBlocks - 1) / pkv::kPrefixSpanBlocks;
     return static_cast<size_t>(num_seqs) * num_heads * parts * (static_cast<size_t>(head_dim) + 2) *
            sizeof(float);
 }
@@ -473,7 +473,7 @@ static pkv_status prefix_impl(void *out, const void *q, const void *k_cache,
                                   ? max_suffix_blocks
                                   : max_blocks_per_seq;
     const int suffix_parts = num_parts_for(suffix_blocks, partition_tokens);
-    const int prefix_parts = (max_blocks_per_seq + pkv::kPrefixChunkBlocks - 1) / pkv::kPrefixChunkBlocks;
+    const int prefix_parts = (max_blocks_per_seq + pkv::kPrefixSpanBlocks - 1) / pkv::kPrefixSpanBlocks;
     const size_t ws_rows = static_cast<size_t>(num_seqs) * num_heads * (prefix_parts + suffix_parts);
     float *ws_o = static_cast<float *>(workspace);
     float *ws_ml = ws_o + ws_rows * head_dim;

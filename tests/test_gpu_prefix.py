@@ -40,6 +40,10 @@ CASES = [
     ("prefix", dict(batch=7, prefix_len=144, suffix_lo=1, suffix_hi=90, head_dim=64,
                     num_heads=16, num_kv_heads=2)),
     ("prefix", dict(batch=40, prefix_len=16, suffix_lo=1, suffix_hi=20)),   # one shared block
+    ("prefix", dict(batch=5, prefix_len=1008, suffix_lo=1, suffix_hi=60)),  # two spans, 32 + 31 blocks
+    # 280 rows (three row tiles) over two spans, grouped heads
+    ("prefix", dict(batch=40, prefix_len=704, suffix_lo=1, suffix_hi=30, num_heads=28,
+                    num_kv_heads=4)),
     ("prefix", dict(batch=5, prefix_len=48, suffix_lo=1, suffix_hi=1)),     # suffix = new token
     # more than 128 rows per (group, KV head): several row tiles, the last one ragged
     ("prefix", dict(batch=40, prefix_len=272, suffix_lo=1, suffix_hi=40, num_heads=28,
