@@ -257,7 +257,6 @@ PKV_API pkv_status pkv_paged_decode_step(void *out, const void *q, const void *k
  *    pkv_decode_workspace_bytes) are rejected with PKV_ERR_WORKSPACE.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, once per device, with that device current).
- *    Make that first call before any stream capture begins.
  *  - All calls share the one array and it keeps the last call's contents
  *    (nothing in it needs clearing).  Calls that overlap on the GPU -- on
  *    unordered streams, or from several host threads -- race on it and give

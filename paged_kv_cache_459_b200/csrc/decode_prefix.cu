@@ -40,7 +40,7 @@ struct PrefixTcGeometry {
     static constexpr int kSmemBytes = kRing + kMeta + 1024;
     static constexpr int kTmemCols = 256;                     // S (P over its first half) | O | Q
     static constexpr int kColS = 0, kColO = kSubKeys, kColQ = kSubKeys + D;
-    static_assert(SB % kSubBlocks == 0 && SB <= 32, "span layout");
+    static_assert(SB % kSubBlocks == 0 && SB <= 64, "span layout");
     static_assert(kColQ + D / 2 <= kTmemCols, "tensor memory columns");
     static_assert(kRing >= 128 * D * 4, "a row tile's partials staged through the ring");
 };
@@ -93,29 +93,33 @@ __device__ __forceinline__ void prefix_unit_tc(const CUtensorMap &tmk, const CUt
     const auto kv_full = [&](int st) { return bars + 8 * st; };  // a stage's K and V landed
     const uint32_t m_bar = bars + 16;                             // the MMAs issued so far are done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Geo::kRing + 24);
-    uint32_t *keep_slot = reinterpret_cast<uint32_t *>(smem + Geo::kRing + 28);
+    uint32_t *keep_slot = reinterpret_cast<uint32_t *>(smem + Geo::kRing + 32);  // [2]: blocks 0-31, 32-63
     int *rows = reinterpret_cast<int *>(smem + Geo::kRing + 64);  // [SB] tensor-map row of each block
 
-    if (warp == 0) {  // lane i: block j0 + i of the span
+    if (warp == 0) {  // lane i: blocks j0 + i and j0 + 32 + i of the span
         const int32_t *trow = p.block_tables + static_cast<size_t>(b0) * p.W;
         const int y_none = static_cast<int>(p.num_blocks * p.Hkv * kBlockTokens);  // past the tensor: zeros
-        bool ok_blk = false;
-        if (lane < SB) {
-            int y = y_none;
-            if (j0 + lane < j1) {
-                const int32_t phys = __ldg(trow + j0 + lane);
-                if (phys >= 0 && phys < p.num_blocks) {
-                    y = (phys * p.Hkv + kvh) * kBlockTokens;
-                    ok_blk = true;
-                } else {
-                    flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
+#pragma unroll
+        for (int hw = 0; hw < 2; ++hw) {
+            const int blk = 32 * hw + lane;
+            bool ok_blk = false;
+            if (blk < SB) {
+                int y = y_none;
+                if (j0 + blk < j1) {
+                    const int32_t phys = __ldg(trow + j0 + blk);
+                    if (phys >= 0 && phys < p.num_blocks) {
+                        y = (phys * p.Hkv + kvh) * kBlockTokens;
+                        ok_blk = true;
+                    } else {
+                        flag(p.err, PKV_DEV_ERR_BAD_BLOCK);
+                    }
                 }
+                rows[blk] = y;
             }
-            rows[lane] = y;
+            const uint32_t bits = __ballot_sync(0xffffffffu, ok_blk);
+            if (lane == 0) keep_slot[hw] = bits;
         }
-        const uint32_t bits = __ballot_sync(0xffffffffu, ok_blk);
         if (lane == 0) {
-            *keep_slot = bits;
             mbar_init(kv_full(0), 1);
             mbar_init(kv_full(1), 1);
             mbar_init(m_bar, 1);
@@ -129,7 +133,7 @@ __device__ __forceinline__ void prefix_unit_tc(const CUtensorMap &tmk, const CUt
     __syncthreads();  // barriers, rows[], keep bits and the TMEM base
     tc::fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t keep = *keep_slot;
+    const uint64_t keep = static_cast<uint64_t>(keep_slot[0]) | (static_cast<uint64_t>(keep_slot[1]) << 32);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // this thread's lane
     const uint64_t policy = l2_policy_evict_first();
 
@@ -215,7 +219,7 @@ __device__ __forceinline__ void prefix_unit_tc(const CUtensorMap &tmk, const CUt
             tc::fence_after();
 
             // softmax of the row over the step's 64 keys (4 blocks)
-            const uint32_t kbits = keep >> (i * kSubBlocks);
+            const uint32_t kbits = static_cast<uint32_t>(keep >> (i * kSubBlocks));
             uint32_t sv[64];
             tc::ld32(lane_base + kColS, sv);
             tc::ld32(lane_base + kColS + 32, sv + 32);
