@@ -287,7 +287,7 @@ PKV_API pkv_status pkv_paged_attention_decode_static(void *out, const void *q, c
  * prefix_blocks[b] = 0.  The group's shared block ids are read from its first
  * member's table row.  pkv_alloc_prefix_groups builds all three arrays from
  * the allocator's state.  All five arrays are device int32.
- * Work: one launch computes each group's prefix attention in spans of 32
+ * Work: one launch computes each group's prefix attention in spans of 64
  * blocks (one CTA and one partial per span, its keys in steps of 64) on the
  * 5th-generation tensor cores (tcgen05.mma, queries of all members x heads
  * as the MMA rows, products in tensor memory) beside split-K

@@ -443,12 +443,13 @@ __global__ void __launch_bounds__(kMergeRows * 32) cascade_merge_kernel(const Pr
 
 // One launch for the prefix spans and the suffix split-K units.  Prefix
 // span k (span fastest, then KV head, then group) is CTA k * stride, spread
-// evenly through the first quarter of the grid, so that the latency-bound
+// evenly through the first eighth of the grid, so that the latency-bound
 // prefix work runs beside the bandwidth-bound suffix stream and its long
-// CTAs (a span of 512 keys) are done well before the stream is (spread over
-// the whole grid, the last spans started late and ended after it: 119.5
-// against 109.8 us per step); the other CTAs take suffix units in order
-// (partition fastest, then head segment, then sequence).
+// CTAs (a span of up to 1024 keys) are done well before the stream is
+// (spread over the whole grid, the last spans started late and ended after
+// it: 119.5 against 109.8 us per step with 32-block spans); the other CTAs
+// take suffix units in order (partition fastest, then head segment, then
+// sequence).
 template <int D, bool MMA>
 __global__ void __launch_bounds__(kPrefixWarps * 32, 3)  // three CTAs per SM, as the suffix units need
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(kPrefixWarps * 32, 3)  // three CTAs per SM, a
     pdl_launch_dependents();
     pdl_wait_primary();  // the previous call's grid
     int id = blockIdx.x;
-    const int stride = n_pre > 0 ? max(1, static_cast<int>(gridDim.x) / 4 / n_pre) : 1;
+    const int stride = n_pre > 0 ? max(1, static_cast<int>(gridDim.x) / 8 / n_pre) : 1;
     if (n_pre > 0 && id % stride == 0 && id / stride < n_pre) {
         id /= stride;
         const int c = id % pp.prefix_parts;

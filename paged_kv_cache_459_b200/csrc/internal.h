@@ -72,7 +72,7 @@ cudaError_t launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const 
 
 // Shared-prefix (cascade) decode: prefix blocks read once per (group, KV
 // head) by a dense tensor-core kernel; suffixes by split-K; LSE merge.
-constexpr int kPrefixSpanBlocks = 32;  // prefix blocks per CTA (a span: one partial per row)
+constexpr int kPrefixSpanBlocks = 64;  // prefix blocks per CTA (a span: one partial per row)
 
 struct PrefixParams {
     __nv_bfloat16 *out;
