@@ -6,6 +6,16 @@
  * and every call is asynchronous on the caller's CUDA stream (`stream` is a
  * cudaStream_t passed as void*; NULL = the legacy default stream).
  *
+ * Stream order: the decode kernels are programmatic dependent launches, so a
+ * call's grid can be resident while the kernel before it on the stream still
+ * runs.  Every read of q, the new tokens, the caches and the workspace, and
+ * every write, waits for that kernel to finish.  The decode calls without a
+ * longest-first order may read seq_lens and block_tables before that wait,
+ * so the kernel right before such a call must not write those arrays after
+ * it lets dependents launch early (griddepcontrol.launch_dependents).
+ * Kernels that never do that are fine, as are copies and memsets; none of
+ * this library's kernels writes them.
+ *
  * The method (page titles and sections of the pages this library follows):
  *  - "vLLM 與 PagedAttention：高吞吐推理的關鍵", section 二: the KV cache is cut
  *    into fixed blocks of 16 tokens; a per-sequence block table maps logical

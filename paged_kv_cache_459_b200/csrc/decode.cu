@@ -45,9 +45,18 @@ template <int D, int NW, int S, bool MMA, int MODE>
 __global__ void __launch_bounds__(NW * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
-    pdl_wait_primary();  // the preceding grid (the order kernel, or the previous call)
-    const int b = p.order != nullptr ? __ldg(p.order + blockIdx.z) : static_cast<int>(blockIdx.z);
-    decode_unit<D, NW, S, MMA, MODE>(tmk, tmv, p, blockIdx.x, blockIdx.y, b);
+    // The preceding grid (the order kernel, or the previous call's last grid):
+    // with an order it is read first; otherwise the unit reads the sequence's
+    // length and table row before waiting for that grid, so that a step's
+    // grid, resident while the previous one drains, starts its K/V loads as
+    // soon as it is released.
+    if (p.order != nullptr) {
+        pdl_wait_primary();
+        decode_unit<D, NW, S, MMA, MODE>(tmk, tmv, p, blockIdx.x, blockIdx.y, __ldg(p.order + blockIdx.z));
+    } else {
+        decode_unit<D, NW, S, MMA, MODE>(tmk, tmv, p, blockIdx.x, blockIdx.y, static_cast<int>(blockIdx.z),
+                                         true);
+    }
 }
 
 // Longest-first order of the sequences by block count (counting sort; ties in

@@ -39,7 +39,8 @@ constexpr int cluster_land_bytes() {
 // the unit's blocks round-robin and are combined in shared memory at the end.
 template <int D, int NW, int S, bool MMA, int MODE>
 __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtensorMap &tmv,
-                                            const DecodeParams &p, int part, int by, int b) {
+                                            const DecodeParams &p, int part, int by, int b,
+                                            bool wait_pending = false) {
     using G = Geometry<D, NW, S>;
     constexpr bool SPLIT = MODE == kModeSplit;
     constexpr bool CLUSTER = MODE == kModeCluster;
@@ -91,6 +92,7 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
     // Cluster mode: an empty part still takes part in the merge (every CTA of
     // the cluster must reach its barriers); it contributes nothing.
     if (blk_begin >= blk_end && !CLUSTER) {
+        if (wait_pending) pdl_wait_primary();
         // Nothing to read.  Single pass: the (empty) sequence's rows are zero.
         // Split-K: the merge kernel only reads partitions that hold tokens.
         // A fused write whose token lies before the start block (inside a
@@ -164,6 +166,10 @@ __device__ __forceinline__ void decode_unit(const CUtensorMap &tmk, const CUtens
         }
     };
 
+    // The lengths and the table row (host-written metadata) were read above;
+    // everything from here on -- q, the new token, K/V, the outputs -- may be
+    // the preceding grid's, so the wait for it comes first.
+    if (wait_pending) pdl_wait_primary();
     using Head = typename std::conditional<MMA, GroupHeads<D>, ScalarHead<D>>::type;
     Head st;
     if constexpr (MMA)
