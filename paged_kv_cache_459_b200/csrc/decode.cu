@@ -225,7 +225,8 @@ cudaError_t launch_one(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
         cudaLaunchAttribute attr[2];
         unsigned n = 0;
         // a programmatic dependent of the preceding grid (the order kernel, or
-        // the previous call's last grid): it waits at its start
+        // the previous call's last grid): it waits before it reads anything
+        // that grid may write
         attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[n++].val.programmaticStreamSerializationAllowed = 1;
         if (MODE == kModeCluster) {  // the parts of one (sequence, head) form a cluster
