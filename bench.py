@@ -827,8 +827,8 @@ def run_gpu(args):
         else:
             r.step(sets[i % 2], outs[i % 2])
 
-    def pipelined(run_step) -> float:
-        """K steps: upload of step i+1 and download of step i (two copy streams,
+    def pipelined(run_step, n=K) -> float:
+        """n steps: upload of step i+1 and download of step i (two copy streams,
         one per direction) overlap step i's kernels; returns the device time of
         the whole loop (ms)."""
         if world > 1:
@@ -840,14 +840,14 @@ def run_gpu(args):
         with torch.cuda.stream(copy_stream):
             stage_d[0].copy_(stage_h, non_blocking=True)
             h2d_done[0].record(copy_stream)
-        for i in range(K):
+        for i in range(n):
             cur, nxt = i % 2, (i + 1) % 2
             stream.wait_event(h2d_done[cur])
             if i >= 2:
                 stream.wait_event(d2h_done[cur])  # the output buffer's previous read is done
             run_step(i)
             comp_done[cur].record(stream)
-            if i + 1 < K:
+            if i + 1 < n:
                 with torch.cuda.stream(copy_stream):
                     if i >= 1:
                         copy_stream.wait_event(comp_done[nxt])  # its inputs were consumed
@@ -864,11 +864,14 @@ def run_gpu(args):
         r.check_err("after the end-to-end steps")
         # the end-to-end steps ran the same inputs through staged copies: the
         # kernels are deterministic, so the output read back must match bit for bit
-        if K > 0 and not torch.equal(outs_h[(K - 1) % 2].view(torch.int16),
+        if n > 0 and not torch.equal(outs_h[(n - 1) % 2].view(torch.int16),
                                      r.out.cpu().view(torch.int16)):
             raise SystemExit("end-to-end output differs from the device-timed output")
         return e2e_ev[0].elapsed_time(e2e_ev[1])
 
+    # an untimed pass of the same loop first (its first steps pay for the first use of
+    # the copy streams, events and staging buffers), then the K timed steps
+    pipelined(step_on, max(3, Wm))
     e2e_ms = pipelined(step_on)
     # The same loop with each step's write + decode replayed from a CUDA graph
     # (one per input/output buffer set), as serving engines run decode: the
@@ -879,6 +882,7 @@ def run_gpu(args):
         with torch.cuda.graph(g):
             step_on(bset)
         graphs.append(g)
+    pipelined(lambda i: graphs[i % 2].replay(), max(3, Wm))
     e2e_graph_ms = pipelined(lambda i: graphs[i % 2].replay())
     del graphs
     e2e_ms, e2e_graph_ms = max_over_ranks([e2e_ms, e2e_graph_ms], device=dev)
@@ -919,11 +923,10 @@ def run_gpu(args):
         "e2e": {"value": job_throughput(B, K, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                 "how": "one pinned staging buffer per step in, output out; double-buffered, "
-                       "uploads and downloads on their own streams, overlapping the kernels; the "
-                       "step through pkv.prepare_decode_step (argument checks once per buffer set)"
-                       if prepared is not None else
-                       "one pinned staging buffer per step in, output out; double-buffered, "
-                       "uploads and downloads on their own streams, overlapping the kernels"},
+                       "uploads and downloads on their own streams, overlapping the kernels; K "
+                       "steps timed after an untimed pass of max(3, W) steps of the same loop" +
+                       ("; the step through pkv.prepare_decode_step (argument checks once per "
+                        "buffer set)" if prepared is not None else "")},
         "e2e_graph": {"value": job_throughput(B, K, world, e2e_graph_ms), "unit": UNIT,
                       "ms_per_step": e2e_graph_ms / K,
                       "how": "the same loop, each step replayed from a CUDA graph"},
