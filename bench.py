@@ -700,10 +700,13 @@ def batch_sweep_key(args, dev) -> dict:
 
     rows = []
     sampler = ClockSampler(device_pci_id(dev))
+    # at least 200 timed steps per row: a batch-1 step is ~11 us, so that K = 20 would
+    # time ~0.2 ms in all
+    steps = max(args.steps, 200)
     for B in (1, 8, 32, 64, 128):
         r = Resident(args, "llama", args.seed, dev, batch=B)
-        m = timed_decode(r, args.steps, max(3, args.warmup), world=1)
-        row = {"batch": B, "variant": r.variant_text(), "decode_us": m["step_us"],
+        m = timed_decode(r, steps, max(3, args.warmup), world=1)
+        row = {"batch": B, "steps": steps, "variant": r.variant_text(), "decode_us": m["step_us"],
                "kv_hbm_gbs": m["kv_hbm_gbs"],
                "kv_frac_of_measured_copy": m["kv_frac_of_measured_copy"],
                "value": m["value"],
