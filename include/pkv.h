@@ -10,9 +10,10 @@
  * call's grid can be resident while the kernel before it on the stream still
  * runs.  Every read of q, the new tokens, the caches and the workspace, and
  * every write, waits for that kernel to finish.  The decode calls without a
- * longest-first order may read seq_lens and block_tables before that wait,
- * so the kernel right before such a call must not write those arrays after
- * it lets dependents launch early (griddepcontrol.launch_dependents).
+ * longest-first order, and the shared-prefix calls, may read seq_lens,
+ * block_tables and prefix_blocks before that wait, so the kernel right
+ * before such a call must not write those arrays after it lets dependents
+ * launch early (griddepcontrol.launch_dependents).
  * Kernels that never do that are fine, as are copies and memsets; none of
  * this library's kernels writes them.
  *

@@ -455,10 +455,10 @@ __global__ void __launch_bounds__(kPrefixWarps * 32, 3)  // three CTAs per SM, a
     cascade_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const PrefixParams pp, const DecodeParams dp, int n_pre) {
     pdl_launch_dependents();
-    pdl_wait_primary();  // the previous call's grid
     int id = blockIdx.x;
     const int stride = n_pre > 0 ? max(1, static_cast<int>(gridDim.x) / 8 / n_pre) : 1;
     if (n_pre > 0 && id % stride == 0 && id / stride < n_pre) {
+        pdl_wait_primary();  // the previous call's grid
         id /= stride;
         const int c = id % pp.prefix_parts;
         id /= pp.prefix_parts;
@@ -483,7 +483,9 @@ __global__ void __launch_bounds__(kPrefixWarps * 32, 3)  // three CTAs per SM, a
         if (start + dp.num_parts * dp.part_blocks < (len + kBlockTokens - 1) / kBlockTokens)
             flag(dp.err, PKV_DEV_ERR_BAD_LEN);
     }
-    decode_unit<D, kPrefixWarps, 2, MMA, kModeSplit>(tmk, tmv, dp, part, id % ny, b);
+    // the unit reads the length, start block and table row, then waits for the
+    // previous call's grid before anything that grid may write
+    decode_unit<D, kPrefixWarps, 2, MMA, kModeSplit>(tmk, tmv, dp, part, id % ny, b, true);
 }
 
 template <int D, bool MMA>
