@@ -128,3 +128,35 @@ def test_auto_split_edges():
     out = d.decode(pkv.DECODE_AUTO, 512, lens=torch.from_numpy(lens).cuda())
     assert d.err_word() & pkv.DEV_ERR_BAD_LEN
     assert (out[1] == 0).all()
+
+
+@pytest.mark.parametrize("variant,part", [(pkv.DECODE_AUTO, 512), (pkv.DECODE_SINGLE, 512),
+                                          (pkv.DECODE_SPLIT, 64), (pkv.DECODE_CLUSTER, 128)])
+def test_lengths_and_tables_written_by_the_kernel_just_before_the_call(variant, part):
+    """The decode grids without a longest-first order read each sequence's
+    length and table row before they wait for the kernel ahead of them on the
+    stream.  A kernel that never lets dependents launch early (every torch
+    kernel) may still write them right before the call.  Here torch kernels
+    relabel two physical blocks (pool and tables) and then shorten the
+    lengths, the last one immediately before the decode; the result is the
+    oracle's for the shortened lengths (relabelling changes nothing)."""
+    w = build("llama", 26, batch=6, len_lo=40, len_hi=700)
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    cut = np.array([0, 5, 17, 1, 33, 2])
+    lens2 = (np.asarray(w.lens) - cut).astype(np.int64)
+    ref = oracle.paged_decode(w.q, kc, vc, w.block_tables, lens2, w.cfg["scale"])
+    d = DeviceStep(w)
+    d.write()
+    a, b = int(w.block_tables[0, 0]), int(w.block_tables[1, 0])
+    torch.cuda.synchronize()
+    for cache in (d.kc, d.vc):
+        tmp = cache[a].clone()
+        cache[a] = cache[b]
+        cache[b] = tmp
+    ma, mb = d.tables == a, d.tables == b
+    d.tables.masked_fill_(ma, b)
+    d.tables.masked_fill_(mb, a)
+    d.lens.sub_(torch.from_numpy(cut.astype(np.int32)).cuda())
+    out = d.decode(variant, part)
+    check_close(out, ref, f"metadata written just before the call, variant {variant}/{part}")
+    assert d.err_word() == 0
