@@ -9,11 +9,10 @@
  * Stream order: the decode kernels are programmatic dependent launches, so a
  * call's grid can be resident while the kernel before it on the stream still
  * runs.  Every read of q, the new tokens, the caches and the workspace, and
- * every write, waits for that kernel to finish.  The decode calls without a
- * longest-first order, and the shared-prefix calls, may read seq_lens,
- * block_tables and prefix_blocks before that wait, so the kernel right
- * before such a call must not write those arrays after it lets dependents
- * launch early (griddepcontrol.launch_dependents).
+ * every write, waits for that kernel to finish.  The decode and shared-
+ * prefix calls may read seq_lens, block_tables and prefix_blocks before that
+ * wait, so the kernel right before such a call must not write those arrays
+ * after it lets dependents launch early (griddepcontrol.launch_dependents).
  * Kernels that never do that are fine, as are copies and memsets; none of
  * this library's kernels writes them.
  *

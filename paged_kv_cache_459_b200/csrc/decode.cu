@@ -67,7 +67,8 @@ constexpr int kOrderBuckets = 4096;
 __global__ void __launch_bounds__(kOrderThreads)
     order_kernel(const int32_t *__restrict__ seq_lens, int B, int W, int shift, int32_t *order) {
     pdl_launch_dependents();
-    pdl_wait_primary();  // the previous call's grid
+    // the counting and the scan read only the lengths: they run before the
+    // wait for the previous call's grid, which still reads the old order
     __shared__ int count[kOrderBuckets];
     __shared__ int warp_tot[kOrderThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -107,6 +108,7 @@ __global__ void __launch_bounds__(kOrderThreads)
         run += local[i];
     }
     __syncthreads();
+    pdl_wait_primary();
     for (int b = tid; b < B; b += kOrderThreads) order[atomicAdd(&count[bucket(b)], 1)] = b;
 }
 
