@@ -16,9 +16,11 @@ namespace pkv {
 // Launches `kern` so that it may be scheduled before the preceding kernel in
 // the stream finishes (programmatic dependent launch); the kernel must call
 // pdl_wait_primary() before it touches memory that kernel may use.  Every
-// kernel of the decode path is launched this way and waits at its start, so
-// that a call's grid is scheduled while the previous call's last grid drains
-// (that grid lets its dependents launch once all its CTAs have started).
+// kernel of the decode path is launched this way and waits before its first
+// access to such memory (the host-written lengths and tables may be read
+// earlier), so that a call's grid is scheduled while the previous call's
+// last grid drains (that grid lets its dependents launch once all its CTAs
+// have started).
 template <typename... Args>
 cudaError_t launch_dependent_smem(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
                                   cudaStream_t stream, Args... args) {
