@@ -460,7 +460,7 @@ class Resident:
 
     def launches_per_step(self) -> int:
         pkv = self.pkv
-        if self.cascade:  # (write;) prefix chunks + suffix split-K in one launch, merge
+        if self.cascade:  # (write;) prefix spans + suffix split-K in one launch, merge
             return 2 if self.fused else 3
         return (1 if self.fused else 2) + (1 if self.chosen == pkv.DECODE_SPLIT else 0) + \
             (1 if self.ordered() else 0)
@@ -480,7 +480,7 @@ class Resident:
     def kernel_text(self) -> str:
         pkv = self.pkv
         if self.cascade:
-            return ("cascade_kernel (prefix chunks + suffix units" +
+            return ("cascade_kernel (prefix spans + suffix units" +
                     (", fused write" if self.fused else "") + ") + cascade_merge_kernel")
         return (("paged_decode_kernel with the fused write" if self.fused else "paged_decode_kernel")
                 + (" (cluster mode)" if self.chosen == pkv.DECODE_CLUSTER else "")

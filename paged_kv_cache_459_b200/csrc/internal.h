@@ -93,7 +93,7 @@ struct PrefixParams {
     float scale_log2;
 };
 
-// One launch running prefix chunks (tcgen05/TMEM) and suffix split-K units
+// One launch running prefix spans (tcgen05/TMEM) and suffix split-K units
 // side by side, then the merge.  dp must describe split-K with start_blocks
 // = prefix_blocks.
 cudaError_t launch_cascade(const CUtensorMap &tmk, const CUtensorMap &tmv, const PrefixParams &pp,
